@@ -1,0 +1,132 @@
+"""CPU oracle for the 3D convolution -- TEST INFRASTRUCTURE ONLY.
+
+This package is the plain, slow, obviously-correct fp64 definition that the
+CUDA library is checked against.  Only ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py`` may import it; the library package
+never does, and the two share no code.
+
+The arithmetic lives in ``conv3d_oracle.c`` (compiled with gcc and OpenMP by
+:func:`build`); this module only marshals numpy arrays through ctypes.
+
+Citations (page title, section):
+  * engineering.drawthings.ai, "Metal conv3d" post -- conv3d computed as an
+    implicit GEMM "similar to 2D convolution": the result is the plain
+    convolution sum, which is what the oracle evaluates directly.
+  * engineering.drawthings.ai, Qwen Image post, "Video VAE" -- causal 3D
+    convolution whose frames before the first are padding (zero for Wan);
+    a first-frame 3D conv reduces to a 2D conv with adjusted weights.
+
+Parity status: every function here is pinned by tests/test_oracle_pins.py
+(brute force, closed forms, invariants and a library cross-check); the pages
+print no worked numeric example, so no pin comes from printed page values.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "conv3d_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_conv3d.so")
+
+F16 = 0
+BF16 = 1
+TPAD_ZERO = 0
+TPAD_CAUSAL_REPLICATE = 1
+TPAD_CAUSAL_ZERO = 2
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile conv3d_oracle.c into liboracle_conv3d.so (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        u16p = ctypes.c_void_p
+        lib.oracle_conv3d_f64.restype = ctypes.c_int
+        lib.oracle_conv3d_f64.argtypes = (
+            [u16p, u16p, u16p, u16p, ctypes.c_int]
+            + [ctypes.c_int] * 16
+            + [i64p, ctypes.c_int64, ctypes.c_void_p]
+        )
+        lib.oracle_output_shape.restype = ctypes.c_int
+        lib.oracle_output_shape.argtypes = [ctypes.c_int] * 13 + [ctypes.POINTER(ctypes.c_int)]
+        lib.oracle_decode16.restype = None
+        lib.oracle_decode16.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle uses (OMP_NUM_THREADS or all cores)."""
+    return int(_load().oracle_num_threads())
+
+
+def decode16(bits: np.ndarray, dtype: int) -> np.ndarray:
+    """Exact decode of 16-bit patterns (bf16 or fp16) to float64."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    out = np.empty(bits.shape, dtype=np.float64)
+    _load().oracle_decode16(bits.ctypes.data, out.ctypes.data, bits.size, dtype)
+    return out
+
+
+def output_shape(D, H, W, kernel, stride, pad, tpad):
+    """(Do, Ho, Wo) for the padding rule of ``tpad`` (see conv3d_oracle.c)."""
+    out = (ctypes.c_int * 3)()
+    rc = _load().oracle_output_shape(D, H, W, *kernel, *stride, *pad, tpad, out)
+    if rc != 0:
+        raise ValueError("ill-formed convolution shape")
+    return tuple(out)
+
+
+def conv3d(x_bits, w_bits, bias_bits, res_bits, dtype, kernel, stride, pad, tpad, rows=None):
+    """fp64 oracle convolution.
+
+    x_bits: uint16 [N,D,H,W,Cin]; w_bits: uint16 [Cout,kt,kh,kw,Cin];
+    bias_bits: uint16 [Cout] or None; res_bits: uint16 [N,Do,Ho,Wo,Cout] or None.
+    rows: optional int64 array of flat output-pixel indices m; when given the
+    result is [len(rows), Cout], else [N,Do,Ho,Wo,Cout].  Unrounded float64.
+    """
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    w_bits = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    N, D, H, W, Cin = x_bits.shape
+    Cout, kt, kh, kw, Cin_w = w_bits.shape
+    if Cin_w != Cin or tuple(kernel) != (kt, kh, kw):
+        raise ValueError("weight shape does not match x / kernel")
+    Do, Ho, Wo = output_shape(D, H, W, kernel, stride, pad, tpad)
+    b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+    r = None if res_bits is None else np.ascontiguousarray(res_bits, dtype=np.uint16)
+    if b is not None and b.shape != (Cout,):
+        raise ValueError("bias shape")
+    if r is not None and r.shape != (N, Do, Ho, Wo, Cout):
+        raise ValueError("residual shape")
+    if rows is None:
+        out = np.empty((N, Do, Ho, Wo, Cout), dtype=np.float64)
+        rows_p, n_rows = None, 0
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        out = np.empty((rows.size, Cout), dtype=np.float64)
+        rows_p, n_rows = rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), rows.size
+    rc = _load().oracle_conv3d_f64(
+        x_bits.ctypes.data, w_bits.ctypes.data,
+        None if b is None else b.ctypes.data,
+        None if r is None else r.ctypes.data,
+        dtype, N, Cin, D, H, W, Cout, kt, kh, kw, *stride, *pad, tpad,
+        rows_p, n_rows, out.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle rejected the problem")
+    return out

@@ -1,0 +1,162 @@
+/*
+ * conv3d_oracle.c -- plain fp64 direct 3D convolution (cross-correlation).
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the oracle that the CUDA path is
+ * checked against.  Only tests/, __graft_entry__.smoke() and the CPU-baseline
+ * leg of bench.py may load it.  It shares no code, header, table or helper
+ * with the CUDA library, and it is deliberately slow and literal.
+ *
+ * What it computes (engineering.drawthings.ai, "Metal conv3d" post: the
+ * implicit-GEMM conv3d reaches the result of a plain 3D convolution, only
+ * faster; "Video VAE" section of the Qwen Image post: causal 3D convolution in
+ * which the frames before the first one are padding):
+ *
+ *   y[n,to,ho,wo,co] = bias[co] + residual[n,to,ho,wo,co]
+ *     + sum_{it<kt} sum_{ih<kh} sum_{iw<kw} sum_{ci<Cin}
+ *         w[co,it,ih,iw,ci] * Xpad[n, to*st+it-pf, ho*sh+ih-ph, wo*sw+iw-pw, ci]
+ *
+ * Layouts: x is NDHWC [N,D,H,W,Cin]; w is [Cout,kt,kh,kw,Cin]; y and residual
+ * are [N,Do,Ho,Wo,Cout].  Xpad is x extended by padding:
+ *   - spatially: 0 outside [0,H) x [0,W);
+ *   - temporally, mode 0 (zero):            pf = pb = pt, 0 outside [0,D);
+ *   - temporally, mode 1 (causal replicate): pf = kt-1, pb = 0, frames f<0
+ *                                            read frame 0;
+ *   - temporally, mode 2 (causal zero):      pf = kt-1, pb = 0, frames f<0
+ *                                            are 0 (the Wan first-frame rule).
+ * Do = (D + pf + pb - kt)/st + 1, Ho = (H + 2ph - kh)/sh + 1,
+ * Wo = (W + 2pw - kw)/sw + 1.
+ *
+ * Inputs are the raw 16-bit patterns (bf16 or fp16) that the GPU is given;
+ * they are decoded exactly to double.  The sum is accumulated in double and
+ * NOT rounded to the 16-bit output type.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORACLE_F16 0
+#define ORACLE_BF16 1
+
+/* bf16 is the top half of an IEEE binary32: widen and reinterpret. */
+static double oracle_bf16_to_double(uint16_t h) {
+  uint32_t u = ((uint32_t)h) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+static double oracle_f16_to_double(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1f;
+  int m = h & 0x3ff;
+  double v;
+  if (e == 0) {
+    v = ldexp((double)m, -24); /* subnormal: m * 2^-14 * 2^-10 */
+  } else if (e == 31) {
+    v = (m == 0) ? INFINITY : NAN;
+  } else {
+    v = ldexp((double)(1024 + m), e - 25); /* (1 + m/1024) * 2^(e-15) */
+  }
+  return sign ? -v : v;
+}
+
+static double oracle_decode(uint16_t h, int dtype) {
+  return dtype == ORACLE_BF16 ? oracle_bf16_to_double(h) : oracle_f16_to_double(h);
+}
+
+/* Exposed so the tests can pin the decoders against numpy for all 65536 codes. */
+void oracle_decode16(const uint16_t* in, double* out, int64_t n, int dtype) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_decode(in[i], dtype);
+}
+
+/* Output extents.  Returns 0 on success, -1 when the problem is empty or
+ * ill-formed.  out[0..2] = Do, Ho, Wo. */
+int oracle_output_shape(int D, int H, int W, int kt, int kh, int kw, int st, int sh, int sw,
+                        int pt, int ph, int pw, int tpad_mode, int* out) {
+  int pf, pb;
+  if (tpad_mode == 0) {
+    pf = pt;
+    pb = pt;
+  } else {
+    pf = kt - 1;
+    pb = 0;
+  }
+  if (st <= 0 || sh <= 0 || sw <= 0) return -1;
+  int nd = D + pf + pb - kt, nh = H + 2 * ph - kh, nw = W + 2 * pw - kw;
+  if (nd < 0 || nh < 0 || nw < 0) return -1;
+  out[0] = nd / st + 1;
+  out[1] = nh / sh + 1;
+  out[2] = nw / sw + 1;
+  return 0;
+}
+
+/*
+ * Evaluate the definition above at the output pixels listed in rows[] (each a
+ * flat index m = ((n*Do + to)*Ho + ho)*Wo + wo), all Cout channels each, and
+ * write y_out[r*Cout + co].  rows == NULL means every output pixel in order.
+ * bias and residual may be NULL (treated as 0).  The residual, when given, is
+ * indexed by the same m.  OpenMP splits the list of pixels; each output value
+ * is one sequential sum in the fixed order (it, ih, iw, ci).
+ * Returns 0, or -1 on an ill-formed problem.
+ */
+int oracle_conv3d_f64(const uint16_t* x, const uint16_t* w, const uint16_t* bias,
+                      const uint16_t* residual, int dtype, int N, int Cin, int D, int H, int W,
+                      int Cout, int kt, int kh, int kw, int st, int sh, int sw, int pt, int ph,
+                      int pw, int tpad_mode, const int64_t* rows, int64_t n_rows, double* y_out) {
+  int od[3];
+  if (oracle_output_shape(D, H, W, kt, kh, kw, st, sh, sw, pt, ph, pw, tpad_mode, od) != 0)
+    return -1;
+  if (tpad_mode < 0 || tpad_mode > 2) return -1;
+  const int Do = od[0], Ho = od[1], Wo = od[2];
+  const int pf = (tpad_mode == 0) ? pt : kt - 1;
+  const int64_t M = (int64_t)N * Do * Ho * Wo;
+  const int64_t count = rows ? n_rows : M;
+
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t r = 0; r < count; ++r) {
+    const int64_t m = rows ? rows[r] : r;
+    if (m < 0 || m >= M) continue;
+    int64_t q = m;
+    const int wo = (int)(q % Wo); q /= Wo;
+    const int ho = (int)(q % Ho); q /= Ho;
+    const int to = (int)(q % Do); q /= Do;
+    const int n = (int)q;
+    for (int co = 0; co < Cout; ++co) {
+      double acc = 0.0;
+      for (int it = 0; it < kt; ++it) {
+        int f = to * st + it - pf;
+        if (f < 0) {
+          if (tpad_mode == 1) f = 0;      /* causal replicate: frame 0 */
+          else continue;                  /* zero / causal zero        */
+        }
+        if (f >= D) continue;             /* back padding is zero      */
+        for (int ih = 0; ih < kh; ++ih) {
+          const int hi = ho * sh + ih - ph;
+          if (hi < 0 || hi >= H) continue;
+          for (int iw = 0; iw < kw; ++iw) {
+            const int wi = wo * sw + iw - pw;
+            if (wi < 0 || wi >= W) continue;
+            const uint16_t* xp = x + ((((int64_t)n * D + f) * H + hi) * W + wi) * Cin;
+            const uint16_t* wp = w + ((((int64_t)co * kt + it) * kh + ih) * kw + iw) * Cin;
+            for (int ci = 0; ci < Cin; ++ci)
+              acc += oracle_decode(wp[ci], dtype) * oracle_decode(xp[ci], dtype);
+          }
+        }
+      }
+      if (bias) acc += oracle_decode(bias[co], dtype);
+      if (residual) acc += oracle_decode(residual[m * Cout + co], dtype);
+      y_out[r * Cout + co] = acc;
+    }
+  }
+  return 0;
+}
+
+/* Number of threads OpenMP will use for the next parallel region. */
+#ifdef _OPENMP
+#include <omp.h>
+int oracle_num_threads(void) { return omp_get_max_threads(); }
+#else
+int oracle_num_threads(void) { return 1; }
+#endif

@@ -1,0 +1,385 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+The pages (engineering.drawthings.ai "Metal conv3d" post; Qwen Image post,
+"Video VAE" section) print no numeric worked example, so the oracle is pinned
+by a hand-worked fixture (tests/golden/), closed forms, invariants, a second
+independent formulation on tiny inputs (brute force) and a library routine
+(torch.nn.functional.conv3d in float64).  Each pin is chosen so that a
+plausible slip in the oracle -- a dropped tap, a flipped kernel, a wrong pad
+frame, an off-by-one in the output size, a transposed weight -- fails it.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import seeded_inputs as si
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+BF16, F16 = oracle.BF16, oracle.F16
+ZERO, CREP, CZERO = oracle.TPAD_ZERO, oracle.TPAD_CAUSAL_REPLICATE, oracle.TPAD_CAUSAL_ZERO
+
+
+def bf16_bits(a):
+    """float64 array -> bf16 bit patterns (values chosen exactly representable)."""
+    t = torch.from_numpy(np.asarray(a, dtype=np.float64)).to(torch.float32).to(torch.bfloat16)
+    return si.bits(t)
+
+
+def rand_problem(N, Cin, D, H, W, Cout, kernel, seed, dtype=torch.bfloat16):
+    fan = Cin * kernel[0] * kernel[1] * kernel[2]
+    x = si.tensor((N, D, H, W, Cin), seed, 0, 1.0, dtype)
+    w = si.tensor((Cout, *kernel, Cin), seed, 1, fan ** -0.5, dtype)
+    b = si.tensor((Cout,), seed, 2, 0.1, dtype)
+    return si.bits(x), si.bits(w), si.bits(b)
+
+
+def dec(bits, dtype=BF16):
+    return oracle.decode16(bits, dtype)
+
+
+# ---------------------------------------------------------------- decoders
+
+def test_decode_bf16_all_codes():
+    codes = np.arange(65536, dtype=np.uint16)
+    with np.errstate(invalid="ignore"):
+        ref = (codes.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    got = oracle.decode16(codes, BF16)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_decode_f16_all_codes():
+    codes = np.arange(65536, dtype=np.uint16)
+    ref = codes.view(np.float16).astype(np.float64)
+    got = oracle.decode16(codes, F16)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+# ---------------------------------------------------------------- hand-worked fixture
+
+def test_golden_box_sum():
+    rows = []
+    with open(os.path.join(HERE, "golden", "box_sum_3x3x3.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                mode, to, ho, wo, y = line.split()
+                rows.append((int(mode), int(to), int(ho), int(wo), float(y)))
+    assert len(rows) == 54
+    frame0 = np.arange(1, 10, dtype=np.float64).reshape(3, 3)
+    x = np.stack([frame0, 10 * frame0]).reshape(1, 2, 3, 3, 1)
+    w = np.ones((1, 3, 3, 3, 1))
+    b = np.array([0.5])
+    for mode in (ZERO, CREP, CZERO):
+        pad = (1, 1, 1) if mode == ZERO else (0, 1, 1)
+        y = oracle.conv3d(bf16_bits(x), bf16_bits(w), bf16_bits(b), None, BF16,
+                          (3, 3, 3), (1, 1, 1), pad, mode)
+        assert y.shape == (1, 2, 3, 3, 1)
+        for m, to, ho, wo, expect in rows:
+            if m == mode:
+                assert y[0, to, ho, wo, 0] == expect, (mode, to, ho, wo)
+
+
+# ---------------------------------------------------------------- output size
+
+@pytest.mark.parametrize("D,H,W", [(1, 1, 1), (5, 7, 4), (9, 16, 12)])
+@pytest.mark.parametrize("kernel,stride,pad", [
+    ((3, 3, 3), (1, 1, 1), (1, 1, 1)), ((1, 1, 1), (1, 1, 1), (0, 0, 0)),
+    ((3, 3, 3), (2, 2, 2), (1, 1, 1)), ((2, 3, 1), (1, 2, 1), (0, 2, 0))])
+@pytest.mark.parametrize("tpad", [ZERO, CREP, CZERO])
+def test_output_shape_by_counting(D, H, W, kernel, stride, pad, tpad):
+    """Count the output positions whose window starts inside the padded extent."""
+    kt, kh, kw = kernel
+    pf, pb = (pad[0], pad[0]) if tpad == ZERO else (kt - 1, 0)
+
+    def count(n, p_lo, p_hi, k, s):
+        return len([o for o in range(0, n + p_lo + p_hi) if o % s == 0 and o + k <= n + p_lo + p_hi])
+
+    expect = (count(D, pf, pb, kt, stride[0]), count(H, pad[1], pad[1], kh, stride[1]),
+              count(W, pad[2], pad[2], kw, stride[2]))
+    if min(expect) <= 0:
+        with pytest.raises(ValueError):
+            oracle.output_shape(D, H, W, kernel, stride, pad, tpad)
+    else:
+        assert oracle.output_shape(D, H, W, kernel, stride, pad, tpad) == expect
+
+
+# ---------------------------------------------------------------- P1 brute force
+
+def brute_force(xd, wd, bd, kernel, stride, pad, tpad):
+    """Independent formulation: explicit padded tensor, dense im2col, one matmul."""
+    N, D, H, W, Cin = xd.shape
+    Cout = wd.shape[0]
+    kt, kh, kw = kernel
+    st, sh, sw = stride
+    pt, ph, pw = pad
+    pf, pb = (pt, pt) if tpad == ZERO else (kt - 1, 0)
+    xp = np.zeros((N, D + pf + pb, H + 2 * ph, W + 2 * pw, Cin))
+    xp[:, pf:pf + D, ph:ph + H, pw:pw + W] = xd
+    if tpad == CREP:
+        xp[:, :pf, ph:ph + H, pw:pw + W] = xd[:, :1]
+    Do = (D + pf + pb - kt) // st + 1
+    Ho = (H + 2 * ph - kh) // sh + 1
+    Wo = (W + 2 * pw - kw) // sw + 1
+    cols = np.zeros((N, Do, Ho, Wo, kt, kh, kw, Cin))
+    for a in range(kt):
+        for b_ in range(kh):
+            for c in range(kw):
+                cols[:, :, :, :, a, b_, c] = xp[:, a:a + st * (Do - 1) + 1:st,
+                                                b_:b_ + sh * (Ho - 1) + 1:sh,
+                                                c:c + sw * (Wo - 1) + 1:sw]
+    A = cols.reshape(-1, kt * kh * kw * Cin)
+    B = wd.reshape(Cout, -1)
+    return (A @ B.T + bd).reshape(N, Do, Ho, Wo, Cout)
+
+
+@pytest.mark.parametrize("tpad", [ZERO, CREP, CZERO])
+@pytest.mark.parametrize("kernel,stride,pad", [
+    ((3, 3, 3), (1, 1, 1), (1, 1, 1)), ((1, 1, 1), (1, 1, 1), (0, 0, 0)),
+    ((2, 3, 1), (1, 1, 1), (0, 1, 0)), ((3, 3, 3), (2, 1, 2), (1, 1, 1)),
+    ((3, 2, 3), (1, 2, 1), (2, 0, 1))])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_p1_brute_force(tpad, kernel, stride, pad, dtype):
+    code = BF16 if dtype == torch.bfloat16 else F16
+    N, Cin, D, H, W, Cout = 2, 3, 4, 5, 5, 4
+    xb, wb, bb = rand_problem(N, Cin, D, H, W, Cout, kernel, seed=11, dtype=dtype)
+    y = oracle.conv3d(xb, wb, bb, None, code, kernel, stride, pad, tpad)
+    ref = brute_force(dec(xb, code), dec(wb, code), dec(bb, code), kernel, stride, pad, tpad)
+    assert y.shape == ref.shape
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- P2 delta kernels
+
+@pytest.mark.parametrize("tpad", [ZERO, CREP, CZERO])
+def test_p2_centre_delta_reproduces_input(tpad):
+    N, C, D, H, W = 1, 4, 3, 5, 6
+    xb, _, bb = rand_problem(N, C, D, H, W, C, (3, 3, 3), seed=3)
+    w = np.zeros((C, 3, 3, 3, C))
+    it = 1 if tpad == ZERO else 2           # the tap that reads frame `to`
+    for c in range(C):
+        w[c, it, 1, 1, c] = 1.0
+    pad = (1, 1, 1) if tpad == ZERO else (0, 1, 1)
+    y = oracle.conv3d(xb, bf16_bits(w), bb, None, BF16, (3, 3, 3), (1, 1, 1), pad, tpad)
+    assert np.array_equal(y, dec(xb) + dec(bb))
+
+
+@pytest.mark.parametrize("tpad", [ZERO, CREP, CZERO])
+@pytest.mark.parametrize("tap", [(0, 0, 0), (0, 2, 1), (2, 0, 2), (1, 1, 0)])
+def test_p2_offcentre_delta_is_a_shift(tpad, tap):
+    """A single off-centre tap (it,ih,iw) gives y[to,ho,wo] = Xpad[to+it-pf, ho+ih-1, wo+iw-1].
+
+    Pins the orientation (cross-correlation, not a flipped convolution) and
+    every padding rule, element by element, with a hand-written index map.
+    """
+    N, C, D, H, W = 1, 2, 4, 4, 5
+    xb, _, _ = rand_problem(N, C, D, H, W, C, (3, 3, 3), seed=5)
+    xd = dec(xb)
+    w = np.zeros((C, 3, 3, 3, C))
+    for c in range(C):
+        w[c, tap[0], tap[1], tap[2], c] = 1.0
+    pad = (1, 1, 1) if tpad == ZERO else (0, 1, 1)
+    pf = 1 if tpad == ZERO else 2
+    y = oracle.conv3d(xb, bf16_bits(w), None, None, BF16, (3, 3, 3), (1, 1, 1), pad, tpad)
+    for to in range(y.shape[1]):
+        for ho in range(H):
+            for wo in range(W):
+                f, h, ww = to + tap[0] - pf, ho + tap[1] - 1, wo + tap[2] - 1
+                if f < 0 and tpad == CREP:
+                    f = 0
+                inside = 0 <= f < D and 0 <= h < H and 0 <= ww < W
+                expect = xd[0, f, h, ww] if inside else np.zeros(C)
+                assert np.array_equal(y[0, to, ho, wo], expect), (to, ho, wo)
+
+
+# ---------------------------------------------------------------- P3 linearity
+
+def test_p3_linearity_in_x_and_w():
+    N, Cin, D, H, W, Cout = 1, 3, 3, 4, 4, 2
+    k = (3, 3, 3)
+    # small-integer tensors so that the combinations are exact in bf16
+    rng = np.random.default_rng(0)
+    x1, x2 = rng.integers(-4, 5, (2, N, D, H, W, Cin)).astype(np.float64)
+    w1, w2 = rng.integers(-4, 5, (2, Cout, *k, Cin)).astype(np.float64)
+    a, b = 3.0, -2.0
+    for tpad, pad in ((ZERO, (1, 1, 1)), (CREP, (0, 1, 1)), (CZERO, (0, 1, 1))):
+        def conv(x, w):
+            return oracle.conv3d(bf16_bits(x), bf16_bits(w), None, None, BF16, k, (1, 1, 1), pad, tpad)
+        np.testing.assert_allclose(conv(a * x1 + b * x2, w1), a * conv(x1, w1) + b * conv(x2, w1),
+                                   rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(conv(x1, a * w1 + b * w2), a * conv(x1, w1) + b * conv(x1, w2),
+                                   rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- P4 1x1x1 = matmul
+
+def test_p4_pointwise_is_matmul():
+    N, Cin, D, H, W, Cout = 2, 16, 3, 4, 5, 8
+    xb, wb, bb = rand_problem(N, Cin, D, H, W, Cout, (1, 1, 1), seed=7)
+    rb = si.bits(si.tensor((N, D, H, W, Cout), 7, 3))
+    y = oracle.conv3d(xb, wb, bb, rb, BF16, (1, 1, 1), (1, 1, 1), (0, 0, 0), ZERO)
+    ref = dec(xb).reshape(-1, Cin) @ dec(wb).reshape(Cout, Cin).T + dec(bb) + dec(rb).reshape(-1, Cout)
+    np.testing.assert_allclose(y.reshape(-1, Cout), ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- P5 causal = explicit frames
+
+@pytest.mark.parametrize("kt", [2, 3])
+def test_p5_causal_modes_equal_explicit_front_frames(kt):
+    N, Cin, D, H, W, Cout = 2, 3, 4, 4, 3, 2
+    k = (kt, 3, 3)
+    xb, wb, bb = rand_problem(N, Cin, D, H, W, Cout, k, seed=13)
+    rep = np.concatenate([xb[:, :1]] * (kt - 1) + [xb], axis=1)
+    zer = np.concatenate([np.zeros_like(xb[:, :1])] * (kt - 1) + [xb], axis=1)
+    y_rep = oracle.conv3d(xb, wb, bb, None, BF16, k, (1, 1, 1), (0, 1, 1), CREP)
+    y_zer = oracle.conv3d(xb, wb, bb, None, BF16, k, (1, 1, 1), (0, 1, 1), CZERO)
+    ref_rep = oracle.conv3d(rep, wb, bb, None, BF16, k, (1, 1, 1), (0, 1, 1), ZERO)
+    ref_zer = oracle.conv3d(zer, wb, bb, None, BF16, k, (1, 1, 1), (0, 1, 1), ZERO)
+    assert y_rep.shape == (N, D, H, W, Cout)
+    assert np.array_equal(y_rep, ref_rep)
+    assert np.array_equal(y_zer, ref_zer)
+
+
+# ---------------------------------------------------------------- P6 outer taps zero = 2D conv
+
+def conv2d_frames(xd, w2, bd):
+    """Own per-frame 2D cross-correlation, 3x3, zero pad 1 (plain loops)."""
+    N, D, H, W, Cin = xd.shape
+    Cout = w2.shape[0]
+    xp = np.zeros((N, D, H + 2, W + 2, Cin))
+    xp[:, :, 1:-1, 1:-1] = xd
+    y = np.zeros((N, D, H, W, Cout)) + bd
+    for ih in range(3):
+        for iw in range(3):
+            y += np.einsum("ndhwc,oc->ndhwo", xp[:, :, ih:ih + H, iw:iw + W], w2[:, ih, iw])
+    return y
+
+
+@pytest.mark.parametrize("tpad", [ZERO, CREP, CZERO])
+def test_p6_zero_outer_taps_equal_2d_conv(tpad):
+    N, Cin, D, H, W, Cout = 1, 4, 3, 5, 4, 3
+    xb, wb, bb = rand_problem(N, Cin, D, H, W, Cout, (3, 3, 3), seed=17)
+    it = 1 if tpad == ZERO else 2
+    wz = np.zeros_like(wb)
+    wz[:, it] = wb[:, it]
+    pad = (1, 1, 1) if tpad == ZERO else (0, 1, 1)
+    y = oracle.conv3d(xb, wz, bb, None, BF16, (3, 3, 3), (1, 1, 1), pad, tpad)
+    ref = conv2d_frames(dec(xb), dec(wb)[:, it], dec(bb))
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- P7 first frame = folded 2D conv
+
+def test_p7_first_frame_fold():
+    """At D=1 the causal 3D conv equals a 2D conv: replicate -> sum of the kt
+    taps, zero -> the last tap only (Qwen Image post, "Video VAE")."""
+    N, Cin, H, W, Cout = 2, 5, 6, 5, 4
+    xb, wb, bb = rand_problem(N, Cin, 1, H, W, Cout, (3, 3, 3), seed=19)
+    y_rep = oracle.conv3d(xb, wb, bb, None, BF16, (3, 3, 3), (1, 1, 1), (0, 1, 1), CREP)
+    y_zer = oracle.conv3d(xb, wb, bb, None, BF16, (3, 3, 3), (1, 1, 1), (0, 1, 1), CZERO)
+    wd = dec(wb)
+    np.testing.assert_allclose(y_rep, conv2d_frames(dec(xb), wd.sum(axis=1), dec(bb)),
+                               rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(y_zer, conv2d_frames(dec(xb), wd[:, 2], dec(bb)),
+                               rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- P8 closed form
+
+@pytest.mark.parametrize("tpad", [ZERO, CREP, CZERO])
+def test_p8_constant_input_closed_form(tpad):
+    N, Cin, D, H, W, Cout = 1, 3, 4, 5, 6, 2
+    c = 0.75
+    _, wb, bb = rand_problem(N, Cin, D, H, W, Cout, (3, 3, 3), seed=23)
+    xb = bf16_bits(np.full((N, D, H, W, Cin), c))
+    pad = (1, 1, 1) if tpad == ZERO else (0, 1, 1)
+    y = oracle.conv3d(xb, wb, bb, None, BF16, (3, 3, 3), (1, 1, 1), pad, tpad)
+    wd, bd = dec(wb), dec(bb)
+    pf = 1 if tpad == ZERO else 2
+    for to in range(D):
+        for ho in range(H):
+            for wo in range(W):
+                # taps whose source position is inside the (replicate-extended) clip
+                mask = np.zeros((3, 3, 3))
+                for it in range(3):
+                    f = to + it - pf
+                    tin = (0 <= f < D) or (f < 0 and tpad == CREP)
+                    for ih in range(3):
+                        for iw in range(3):
+                            if tin and 0 <= ho + ih - 1 < H and 0 <= wo + iw - 1 < W:
+                                mask[it, ih, iw] = 1
+                expect = c * np.einsum("otijc,tij->o", wd, mask) + bd
+                np.testing.assert_allclose(y[0, to, ho, wo], expect, rtol=1e-12, atol=1e-12)
+    # interior outputs are c * sum(w) + b, and with causal replicate the first frames equal the interior
+    interior = c * wd.reshape(Cout, -1).sum(axis=1) + bd
+    np.testing.assert_allclose(y[0, D - 2, 2, 2], interior, rtol=1e-12)
+    if tpad == CREP:
+        np.testing.assert_allclose(y[0, 0, 2, 2], interior, rtol=1e-12)
+
+
+# ---------------------------------------------------------------- P9 translation equivariance
+
+def test_p9_translation_equivariance():
+    N, Cin, D, H, W, Cout = 1, 2, 7, 8, 8, 2
+    rng = np.random.default_rng(1)
+    core = rng.integers(-3, 4, (N, 3, 3, 3, Cin)).astype(np.float64)
+    x1 = np.zeros((N, D, H, W, Cin))
+    x2 = np.zeros((N, D, H, W, Cin))
+    x1[:, 2:5, 2:5, 2:5] = core
+    x2[:, 3:6, 3:6, 3:6] = core
+    _, wb, _ = rand_problem(N, Cin, D, H, W, Cout, (3, 3, 3), seed=29)
+    y1 = oracle.conv3d(bf16_bits(x1), wb, None, None, BF16, (3, 3, 3), (1, 1, 1), (1, 1, 1), ZERO)
+    y2 = oracle.conv3d(bf16_bits(x2), wb, None, None, BF16, (3, 3, 3), (1, 1, 1), (1, 1, 1), ZERO)
+    assert np.array_equal(y1[:, 1:6, 1:7, 1:7], y2[:, 2:7, 2:8, 2:8])
+
+
+# ---------------------------------------------------------------- P10 library cross-check
+
+@pytest.mark.parametrize("tpad", [ZERO, CREP, CZERO])
+@pytest.mark.parametrize("kernel,stride,pad", [
+    ((3, 3, 3), (1, 1, 1), (1, 1, 1)), ((1, 1, 1), (1, 1, 1), (0, 0, 0)),
+    ((3, 3, 3), (2, 2, 1), (1, 1, 1))])
+def test_p10_torch_conv3d_float64(tpad, kernel, stride, pad):
+    N, Cin, D, H, W, Cout = 2, 8, 5, 9, 7, 6
+    xb, wb, bb = rand_problem(N, Cin, D, H, W, Cout, kernel, seed=31)
+    rb_shape = (N, *oracle.output_shape(D, H, W, kernel, stride, pad, tpad), Cout)
+    rb = si.bits(si.tensor(rb_shape, 31, 3))
+    y = oracle.conv3d(xb, wb, bb, rb, BF16, kernel, stride, pad, tpad)
+    x = torch.from_numpy(dec(xb)).permute(0, 4, 1, 2, 3)
+    w = torch.from_numpy(dec(wb)).permute(0, 4, 1, 2, 3)
+    kt = kernel[0]
+    if tpad == ZERO:
+        x = F.pad(x, (0, 0, 0, 0, pad[0], pad[0]))
+    elif tpad == CREP:
+        x = torch.cat([x[:, :, :1]] * (kt - 1) + [x], dim=2)
+    else:
+        x = F.pad(x, (0, 0, 0, 0, kt - 1, 0))
+    ref = F.conv3d(x, w, torch.from_numpy(dec(bb)), stride=stride, padding=(0, pad[1], pad[2]))
+    ref = ref.permute(0, 2, 3, 4, 1).numpy() + dec(rb)
+    np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-10)
+
+
+# ---------------------------------------------------------------- sampled rows
+
+def test_sampled_rows_match_full_output():
+    N, Cin, D, H, W, Cout = 2, 8, 4, 6, 5, 4
+    xb, wb, bb = rand_problem(N, Cin, D, H, W, Cout, (3, 3, 3), seed=37)
+    full = oracle.conv3d(xb, wb, bb, None, BF16, (3, 3, 3), (1, 1, 1), (0, 1, 1), CREP)
+    rows = np.array([0, 1, 29, 30, 59, 60, 119, 239], dtype=np.int64)
+    part = oracle.conv3d(xb, wb, bb, None, BF16, (3, 3, 3), (1, 1, 1), (0, 1, 1), CREP, rows=rows)
+    assert np.array_equal(part, full.reshape(-1, Cout)[rows])
+
+
+def test_rejects_mismatched_shapes():
+    xb, wb, bb = rand_problem(1, 4, 2, 3, 3, 2, (3, 3, 3), seed=1)
+    with pytest.raises(ValueError):
+        oracle.conv3d(xb, wb[:, :, :, :, :3], bb, None, BF16, (3, 3, 3), (1, 1, 1), (1, 1, 1), ZERO)
+    with pytest.raises(ValueError):
+        oracle.output_shape(2, 3, 3, (3, 3, 3), (1, 1, 1), (0, 0, 0), ZERO)
