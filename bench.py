@@ -1,0 +1,494 @@
+"""Benchmark: device-timed conv3d TFLOP/s on the video-VAE decoder workloads.
+
+Default workload: bf16 256->256, 9x128x128 frames, 3x3x3 kernel, causal
+replicate temporal padding, fused residual add (the 256-channel decoder block).
+One step = one conv3d_fwd call over one synthetic batch (every stage of the
+path: for this workload one kernel launch).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (launched with torch.distributed.run): every rank convolves its own
+seeded sample (data parallel over the batch, no data-path collective), so the
+scaling is weak; value = FLOPs of all ranks / the slowest rank's time.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import seeded_inputs as si  # noqa: E402
+from seeded_inputs.workloads import WORKLOADS  # noqa: E402
+
+METRIC = "conv3d TFLOPS (bf16, video-VAE decoder shapes) and % of B200 dense peak"
+TORCH_DTYPE = {"bf16": torch.bfloat16, "f16": torch.float16}
+KERNEL_NAME = "conv3d_implicit_gemm_kernel"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- workload arithmetic
+
+def out_shape(wl):
+    kt, kh, kw = wl.kernel
+    pt, ph, pw = wl.pad
+    pf, pb = (pt, pt) if wl.tpad == 0 else (kt - 1, 0)
+    return (wl.D + pf + pb - kt + 1, wl.H + 2 * ph - kh + 1, wl.W + 2 * pw - kw + 1)
+
+
+def algorithmic_flops(wl):
+    """2 * Cout * Cin * kh * kw * sum over output pixels of the temporal taps that
+    read a real frame (taps reading zero padding are not work).  A single causal
+    replicate frame counts one folded temporal tap (the first-frame 2D conv)."""
+    Do, Ho, Wo = out_shape(wl)
+    kt, kh, kw = wl.kernel
+    if wl.tpad == 1 and wl.D == 1:
+        taps_t = Do * 1
+    else:
+        pf = wl.pad[0] if wl.tpad == 0 else kt - 1
+        taps_t = 0
+        for to in range(Do):
+            for it in range(kt):
+                f = to + it - pf
+                if f < 0 and wl.tpad == 1:
+                    f = 0
+                taps_t += 0 <= f < wl.D
+    return 2.0 * wl.N * Ho * Wo * wl.Cout * wl.Cin * kh * kw * taps_t
+
+
+def algorithmic_bytes(wl):
+    """x, w, bias, residual read once; y written once (16-bit elements)."""
+    Do, Ho, Wo = out_shape(wl)
+    x = wl.N * wl.D * wl.H * wl.W * wl.Cin
+    w = wl.Cout * wl.kernel[0] * wl.kernel[1] * wl.kernel[2] * wl.Cin
+    y = wl.N * Do * Ho * Wo * wl.Cout
+    return 2.0 * (x + w + wl.Cout + y + (y if wl.residual else 0))
+
+
+def describe(wl, world):
+    Do, Ho, Wo = out_shape(wl)
+    return {
+        "workload": f"conv3d {wl.name}: {wl.note}",
+        "dtype": wl.dtype, "N_per_gpu": wl.N, "global_batch": wl.N * world,
+        "Cin": wl.Cin, "Cout": wl.Cout, "D": wl.D, "H": wl.H, "W": wl.W,
+        "kernel": list(wl.kernel), "stride": [1, 1, 1], "pad": list(wl.pad),
+        "temporal_pad": ["zero", "causal_replicate", "causal_zero"][wl.tpad],
+        "residual": wl.residual, "out": [Do, Ho, Wo],
+        "gemm": {"M": wl.N * Do * Ho * Wo, "N": wl.Cout,
+                 "K": wl.Cin * wl.kernel[0] * wl.kernel[1] * wl.kernel[2]},
+        "seed": wl.seed, "parallelism": f"dp{world}" if world > 1 else "single",
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash():
+    """Fingerprint of the device code the ncu counters were taken on."""
+    h = hashlib.sha256()
+    for rel in ("csrc/conv3d_kernel.cuh", "csrc/ptx.cuh"):
+        with open(os.path.join(ROOT, "video_vae_convolution_implicit_b200", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(wl_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(wl_name)
+    if not e or e.get("kernel_sha") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks (NVML, read only)
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons every ~20 ms while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = None
+            try:  # CUDA and NVML number devices differently under CUDA_VISIBLE_DEVICES
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # no NVML: report null clocks
+            self._err = str(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(0.02)
+
+    def _sample(self):
+        try:
+            self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+            mask = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            for bit, name in self.REASONS.items():
+                if mask & bit and name != "gpu_idle":
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        if self._ok:
+            self._sample()
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return None
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- oracle (CPU) timing
+
+def host_bits(p):
+    """16-bit patterns of the problem's tensors on the host (converted once)."""
+    return {k: (None if p[k] is None else si.bits(p[k])) for k in ("x", "w", "bias", "residual")}
+
+
+def oracle_rows_timed(hb, wl, rows):
+    """The oracle on the given output pixels; returns (values, seconds of oracle work)."""
+    import oracle
+    t0 = time.perf_counter()
+    ref = oracle.conv3d(hb["x"], hb["w"], hb["bias"], hb["residual"],
+                        oracle.BF16 if wl.dtype == "bf16" else oracle.F16, wl.kernel, (1, 1, 1),
+                        wl.pad, wl.tpad, rows=rows)
+    return ref, time.perf_counter() - t0
+
+
+def flops_per_row(wl):
+    Do, Ho, Wo = out_shape(wl)
+    return algorithmic_flops(wl) / (wl.N * Do * Ho * Wo)
+
+
+def calibrated_rows(hb, wl, seconds, rng):
+    """Number of output pixels the oracle finishes in about `seconds`."""
+    Do, Ho, Wo = out_shape(wl)
+    M = wl.N * Do * Ho * Wo
+    n = 64
+    while True:
+        probe = np.sort(rng.choice(M, size=min(n, M), replace=False)).astype(np.int64)
+        _, dt = oracle_rows_timed(hb, wl, probe)
+        if dt > 0.5 or n >= M:
+            break
+        n *= 4
+    per_row = max(dt / min(n, M), 1e-7)
+    return int(max(16, min(M, seconds / per_row)))
+
+
+def host_problem(wl, seed):
+    out = out_shape(wl)
+    return si.conv3d_problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, out, seed,
+                             TORCH_DTYPE[wl.dtype], True, wl.residual, "cpu")
+
+
+def run_reference(args, wl, rank, world):
+    """The reference arm: the fp64 CPU oracle as it stands, on a bounded sample."""
+    if rank != 0:
+        return 0
+    import oracle
+    hb = host_bits(host_problem(wl, wl.seed))
+    Do, Ho, Wo = out_shape(wl)
+    M = wl.N * Do * Ho * Wo
+    rng = np.random.default_rng(wl.seed)
+    budget = float(os.environ.get("CONV3D_REFERENCE_SECONDS", "90"))
+    per_step_rows = calibrated_rows(hb, wl, budget / max(1, args.steps + args.warmup), rng)
+    for _ in range(args.warmup):
+        oracle_rows_timed(hb, wl, np.sort(rng.choice(M, per_step_rows, replace=False)))
+    times = []
+    for _ in range(args.steps):
+        rows = np.sort(rng.choice(M, per_step_rows, replace=False)).astype(np.int64)
+        _, dt = oracle_rows_timed(hb, wl, rows)
+        times.append(dt)
+    flops = flops_per_row(wl) * per_step_rows
+    value = flops * len(times) / sum(times) / 1e12
+    sample = (f"{per_step_rows} random output pixels (all {wl.Cout} channels) of {M} per step, "
+              f"{args.steps} timed steps")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": describe(wl, 1),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- multi-rank plumbing
+
+def rank_seed(wl, rank):
+    """Each rank convolves its own independent sample (data parallel over the batch)."""
+    return wl.seed + 1000 * rank
+
+
+def max_over_ranks(value, device):
+    """The slowest rank's time: MAX all-reduce (a timing collective, not a data path)."""
+    if not torch.distributed.is_initialized() or torch.distributed.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step, world, steps, max_ms):
+    """Units processed by all ranks divided by the slowest rank's time."""
+    return flops_per_rank_step * world * steps / (max_ms * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, wl, rank, world, local_rank):
+    import video_vae_convolution_implicit_b200 as c3
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dt = TORCH_DTYPE[wl.dtype]
+    Do, Ho, Wo = out_shape(wl)
+    seed = rank_seed(wl, rank)
+    p = si.conv3d_problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, (Do, Ho, Wo), seed,
+                          dt, True, wl.residual, dev)
+    y = torch.empty((wl.N, Do, Ho, Wo, wl.Cout), dtype=dt, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        c3.conv3d_fwd(p["x"], p["w"], p["bias"], p["residual"], y, (1, 1, 1), wl.pad, wl.tpad,
+                      stream=stream)
+
+    launches_per_step = 1 + (1 if (wl.tpad == 1 and wl.D == 1 and wl.kernel[0] > 1) else 0)
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if c3.poll_status(stream) != c3.Status.OK:
+        raise RuntimeError("device status after warm-up is not OK")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clocks:
+        region0 = torch.cuda.Event(enable_timing=True)
+        region1 = torch.cuda.Event(enable_timing=True)
+        region0.record(stream)
+        for i in range(args.steps):
+            flush.zero_()                       # L2 flushed between timed steps
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        region1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    my_ms = sum(step_ms)
+    max_ms = max_over_ranks(my_ms, dev)
+    status = c3.poll_status(stream)
+
+    flops = algorithmic_flops(wl)
+    ms_per_step = max_ms / args.steps
+    value = whole_job_tflops(flops, world, args.steps, max_ms)
+    peaks, peak_kind = load_peaks()
+    kernel_ms = statistics.mean(step_ms)  # one conv kernel launch per step for T > 1
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic (seeded SplitMix64 normals; no model weights)",
+        "config": dict(describe(wl, world), l2="flushed (2x L2 write) between timed steps"),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(wl.name),
+                     "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                     "kernel": KERNEL_NAME, "algorithmic_flops_per_launch": flops,
+                     "algorithmic_bytes_per_launch": algorithmic_bytes(wl)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+        "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms),
+                    "max": max(step_ms)},
+        "region_ms": region0.elapsed_time(region1),
+        "device_status": c3.status_string(status),
+    }
+
+    # end to end through the public API from pinned host buffers
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, wl, p, y, stream, dev, c3, flops)
+
+    # parity gate on sampled rows (a timing is reported only with a passing check)
+    if rank == 0:
+        line["parity"] = parity_sample(wl, p, y)
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, p)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    ok = status == c3.Status.OK and (rank != 0 or line["parity"]["ok"])
+    return 0 if ok else 1
+
+
+def run_e2e(args, wl, p, y, stream, dev, c3, flops):
+    host = {k: (None if p[k] is None else p[k].cpu().pin_memory()) for k in ("x", "w", "bias", "residual")}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    dbuf = {k: (None if p[k] is None else torch.empty_like(p[k])) for k in host}
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = y_host.numel() * y_host.element_size()
+    steps = max(1, min(args.steps, 20))
+
+    def e2e_step():
+        for k, v in host.items():
+            if v is not None:
+                dbuf[k].copy_(v, non_blocking=True)
+        c3.conv3d_fwd(dbuf["x"], dbuf["w"], dbuf["bias"], dbuf["residual"], y, (1, 1, 1), wl.pad,
+                      wl.tpad, stream=stream)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = s.elapsed_time(e) / steps
+    return {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
+            "path": "pinned host -> device copies, conv3d_fwd (C ABI), device -> pinned host"}
+
+
+def _rows_for_parity(wl, n_random=48):
+    Do, Ho, Wo = out_shape(wl)
+    HoWo = Ho * Wo
+    rows = set()
+    for to in sorted({0, 1, Do - 1} & set(range(Do))):
+        base = to * HoWo
+        rows.update([base, base + Wo - 1, base + HoWo - 1, base + HoWo // 2])
+    rng = np.random.default_rng(12345)
+    rows.update(int(v) for v in rng.integers(0, wl.N * Do * HoWo, n_random))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def parity_sample(wl, p, y):
+    rows = _rows_for_parity(wl)
+    ref, _ = oracle_rows_timed(host_bits(p), wl, rows)
+    got = y.view(-1, wl.Cout)[torch.from_numpy(rows).to(y.device)].double().cpu().numpy()
+    err = np.abs(got - ref)
+    max_ratio = float(err.max() / np.abs(ref).max())
+    rel_l1 = float(err.sum() / np.abs(ref).sum())
+    return {"rows": int(rows.size), "max_err_over_max_ref": max_ratio, "rel_l1": rel_l1,
+            "ok": bool(np.isfinite(got).all() and max_ratio <= 1e-2 and rel_l1 <= 2e-3)}
+
+
+def cpu_baseline(wl, p):
+    import oracle
+    hb = host_bits(p)
+    Do, Ho, Wo = out_shape(wl)
+    M = wl.N * Do * Ho * Wo
+    rng = np.random.default_rng(7)
+    seconds = float(os.environ.get("CONV3D_CPU_BASELINE_SECONDS", "15"))
+    n = calibrated_rows(hb, wl, seconds, rng)
+    rows = np.sort(rng.choice(M, n, replace=False)).astype(np.int64)
+    _, dt = oracle_rows_timed(hb, wl, rows)
+    value = flops_per_row(wl) * n / dt / 1e12
+    return {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} random output pixels (all {wl.Cout} channels) of {M}, {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="cfg2", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    wl = WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        return run_reference(args, wl, rank, world)
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        rc = run_ours(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,142 @@
+/*
+ * conv3d.h -- C ABI of libconv3d: implicit-GEMM 3D convolution on B200 (sm_100a).
+ *
+ * The operation (engineering.drawthings.ai, "Metal conv3d" post: 3D
+ * convolution implemented as an implicit GEMM, the way 2D convolution is;
+ * Qwen Image post, "Video VAE" section: causal 3D convolution in video-VAE
+ * decoders, whose frames before the first are padding, and whose first-frame
+ * case reduces to a 2D convolution with adjusted weights):
+ *
+ *   y[n,to,ho,wo,co] = round( bias[co] + residual[n,to,ho,wo,co]
+ *       + sum_{it,ih,iw,ci} w[co,it,ih,iw,ci] * Xpad[n, to+it-pf, ho+ih-ph, wo+iw-pw, ci] )
+ *
+ * computed as the GEMM  M = N*Do*Ho*Wo,  N_gemm = Cout,  K = Cin*kt*kh*kw,
+ * with fp16/bf16 operands, fp32 accumulation and one round-to-nearest-even to
+ * the output type.  Xpad is x extended by zeros spatially and, temporally,
+ * by the rule of conv3d_tpad_t.
+ *
+ * Layouts (row-major, innermost last):
+ *   x        [N, D, H, W, Cin]            (NDHWC)
+ *   w        [Cout, kt, kh, kw, Cin]      (K-major: row co is the K vector)
+ *   bias     [Cout]                        (optional)
+ *   residual [N, Do, Ho, Wo, Cout]         (optional, same type as y)
+ *   y        [N, Do, Ho, Wo, Cout]
+ *   Do = (D + pf + pb - kt) + 1, Ho = H + 2*ph - kh + 1, Wo = W + 2*pw - kw + 1
+ *   (stride 1; pf/pb are the front/back temporal pads of the mode).
+ *
+ * All tensor pointers are DEVICE pointers to caller-owned memory on the
+ * current CUDA device; the library never frees them and keeps none after a
+ * call returns.  Every call enqueues on `stream` and returns without
+ * synchronising.
+ */
+#ifndef LIBCONV3D_CONV3D_H
+#define LIBCONV3D_CONV3D_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define CONV3D_API __attribute__((visibility("default")))
+#else
+#define CONV3D_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t is `struct CUstream_st *`; NULL = legacy default stream */
+
+typedef enum { CONV3D_F16 = 0, CONV3D_BF16 = 1 } conv3d_dtype_t;
+
+/* Temporal padding rule (the spatial rule is always zero padding ph, pw). */
+typedef enum {
+  CONV3D_TPAD_ZERO = 0,             /* pad[0] zero frames in front and behind          */
+  CONV3D_TPAD_CAUSAL_REPLICATE = 1, /* kt-1 copies of frame 0 in front, none behind    */
+  CONV3D_TPAD_CAUSAL_ZERO = 2       /* kt-1 zero frames in front, none behind (Wan)    */
+} conv3d_tpad_t;
+
+typedef enum {
+  CONV3D_OK = 0,
+  CONV3D_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad enum, overlap  */
+  CONV3D_ERR_UNSUPPORTED = 2,  /* valid convolution outside the supported set         */
+  CONV3D_ERR_ALIGNMENT = 3,    /* a tensor pointer is not 16-byte aligned             */
+  CONV3D_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (conv3d_last_error) */
+  CONV3D_ERR_TIMEOUT = 5,      /* a device-side wait ran out of time                  */
+  CONV3D_ERR_DEVICE_CHECK = 6, /* a device-side consistency check failed              */
+  CONV3D_ERR_WORKSPACE = 7     /* workspace missing or smaller than required          */
+} conv3d_status_t;
+
+/*
+ * conv3d_fwd -- y = conv3d(x, w) + bias + residual (see the top of this file).
+ *
+ * kernel = {kt, kh, kw}, each in [1, 8].  stride = {1, 1, 1} (other strides
+ * return CONV3D_ERR_UNSUPPORTED).  pad = {pt, ph, pw}: pt is used by
+ * CONV3D_TPAD_ZERO only and must be 0 for the causal modes; pt, ph, pw in
+ * [0, 127], and the output extents Do, Ho, Wo must be >= 1.
+ * Supported set: Cin % 8 == 0, Cout % 8 == 0, 16-byte aligned pointers, y not
+ * overlapping x, w or bias; residual may be exactly y (in-place add) but not
+ * partially overlap it.  bias and residual may be NULL.
+ *
+ * First-frame path: with CONV3D_TPAD_CAUSAL_REPLICATE and D == 1 every
+ * temporal tap reads frame 0, so the kt taps are summed (fp32) into one 2D
+ * weight, kept as a high and a low 16-bit part, and a 2D convolution over
+ * the two parts runs instead of kt taps (2/kt of the tensor-core work); the
+ * bias is unchanged.  That fold needs conv3d_workspace_bytes() of device
+ * scratch: conv3d_fwd takes it from a per-device buffer that the library
+ * allocates on the first such call and keeps until conv3d_release() (calls
+ * that need it and overlap on different streams race on it -- use
+ * conv3d_fwd_ws for those).
+ *
+ * Errors: argument, alignment and support errors return before anything is
+ * enqueued, with y untouched.  A failed launch returns CONV3D_ERR_CUDA.
+ * Device-side timeouts are reported by conv3d_poll_status().
+ */
+CONV3D_API conv3d_status_t conv3d_fwd(const void* x, const void* w, const void* bias,
+                                      const void* residual, void* y, int N, int Cin, int D, int H,
+                                      int W, int Cout, const int kernel[3], const int stride[3],
+                                      const int pad[3], conv3d_tpad_t tpad, conv3d_dtype_t dtype,
+                                      struct CUstream_st* stream);
+
+/* conv3d_fwd with caller-provided device scratch (never allocates).
+ * `workspace` must be 256-byte aligned and hold conv3d_workspace_bytes();
+ * it may be NULL when that is 0.  Too small -> CONV3D_ERR_WORKSPACE. */
+CONV3D_API conv3d_status_t conv3d_fwd_ws(const void* x, const void* w, const void* bias,
+                                         const void* residual, void* y, int N, int Cin, int D,
+                                         int H, int W, int Cout, const int kernel[3],
+                                         const int stride[3], const int pad[3], conv3d_tpad_t tpad,
+                                         conv3d_dtype_t dtype, void* workspace, size_t ws_bytes,
+                                         struct CUstream_st* stream);
+
+/* Device scratch bytes conv3d_fwd_ws needs for this problem (0 if none). */
+CONV3D_API size_t conv3d_workspace_bytes(int Cin, int Cout, int D, const int kernel[3], conv3d_tpad_t tpad);
+
+/* Output extents {Do, Ho, Wo} for the problem; CONV3D_ERR_INVALID_ARG if any is < 1. */
+CONV3D_API conv3d_status_t conv3d_output_shape(int D, int H, int W, const int kernel[3], const int stride[3],
+                                    const int pad[3], conv3d_tpad_t tpad, int out_dhw[3]);
+
+/* Synchronises `stream`, then returns and clears the device status word of the
+ * current device (CONV3D_OK, CONV3D_ERR_TIMEOUT or CONV3D_ERR_DEVICE_CHECK). */
+CONV3D_API conv3d_status_t conv3d_poll_status(struct CUstream_st* stream);
+
+/* Static English text for a status code. */
+CONV3D_API const char* conv3d_status_string(conv3d_status_t status);
+
+/* Text of the last CONV3D_ERR_CUDA / CONV3D_ERR_UNSUPPORTED detail on this thread. */
+CONV3D_API const char* conv3d_last_error(void);
+
+/* Frees the cached per-device workspace.  Not to be called while work that
+ * uses it is in flight. */
+CONV3D_API void conv3d_release(void);
+
+/* Failure-detection self test: launches one CTA that waits, with the same
+ * bounded wait the convolution uses, on an mbarrier that nothing completes,
+ * limited to `timeout_ms` (1..10000).  Synchronises and returns the status
+ * the device recorded: CONV3D_ERR_TIMEOUT when the mechanism works.  The
+ * status word is cleared before returning. */
+CONV3D_API conv3d_status_t conv3d_selftest_wait_timeout(int timeout_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBCONV3D_CONV3D_H */

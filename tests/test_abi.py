@@ -1,0 +1,136 @@
+"""The C ABI: exports, host-side validation and error codes (no GPU needed).
+
+Validation runs before any CUDA call, so these tests pass fake, never
+dereferenced device addresses and check that the library answers with the
+documented status code.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import video_vae_convolution_implicit_b200 as c3
+from video_vae_convolution_implicit_b200 import Status
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+# fake, 256-byte aligned, widely separated "device" addresses (never touched)
+X, Wt, B, R, Y = 0x100000000, 0x200000000, 0x300000000, 0x400000000, 0x500000000
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"CONV3D_API\s+[\w\s\*]*?\b(conv3d_\w+)\s*\(", text)
+    return names
+
+
+def test_library_exports_every_declared_function():
+    names = declared_functions()
+    assert "conv3d_fwd" in names and "conv3d_fwd_ws" in names
+    lib = ctypes.CDLL(c3.lib_path)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for s in range(8):
+        assert c3.status_string(s) and c3.status_string(s) != "unknown status"
+    assert c3.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("D,H,W,k,pad,tpad,expect", [
+    (9, 128, 128, (3, 3, 3), (0, 1, 1), c3.TPAD_CAUSAL_REPLICATE, (9, 128, 128)),
+    (5, 32, 32, (3, 3, 3), (1, 1, 1), c3.TPAD_ZERO, (5, 32, 32)),
+    (5, 32, 32, (3, 3, 3), (0, 1, 1), c3.TPAD_ZERO, (3, 32, 32)),
+    (1, 256, 256, (3, 3, 3), (0, 1, 1), c3.TPAD_CAUSAL_ZERO, (1, 256, 256)),
+    (33, 128, 128, (1, 1, 1), (0, 0, 0), c3.TPAD_ZERO, (33, 128, 128)),
+    (4, 7, 9, (2, 3, 1), (0, 0, 2), c3.TPAD_CAUSAL_REPLICATE, (4, 5, 13)),
+])
+def test_output_shape(D, H, W, k, pad, tpad, expect):
+    assert c3.output_shape(D, H, W, k, (1, 1, 1), pad, tpad) == expect
+
+
+def test_output_shape_rejects_empty():
+    with pytest.raises(c3.Conv3dError):
+        c3.output_shape(1, 2, 2, (3, 3, 3), (1, 1, 1), (0, 0, 0), c3.TPAD_ZERO)
+
+
+def test_workspace_bytes():
+    # first-frame fold: (hi, lo) x Cout*kh*kw*Cin 16-bit values, rounded up to 256 bytes
+    assert c3.workspace_bytes(256, 256, 1, (3, 3, 3), c3.TPAD_CAUSAL_REPLICATE) == 2 * 256 * 9 * 256 * 2
+    assert c3.workspace_bytes(8, 8, 1, (3, 3, 3), c3.TPAD_CAUSAL_REPLICATE) == 2304
+    assert c3.workspace_bytes(256, 256, 2, (3, 3, 3), c3.TPAD_CAUSAL_REPLICATE) == 0
+    assert c3.workspace_bytes(256, 256, 1, (3, 3, 3), c3.TPAD_CAUSAL_ZERO) == 0
+    assert c3.workspace_bytes(256, 256, 1, (1, 3, 3), c3.TPAD_CAUSAL_REPLICATE) == 0
+
+
+def call(**kw):
+    a = dict(x=X, w=Wt, bias=B, residual=None, y=Y, N=1, Cin=64, D=4, H=16, W=16, Cout=64,
+             kernel=(3, 3, 3), stride=(1, 1, 1), pad=(0, 1, 1), tpad=c3.TPAD_CAUSAL_REPLICATE,
+             dtype=c3.BF16, stream=None)
+    a.update(kw)
+    return c3.conv3d_fwd_ptr(**a)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(x=None), Status.INVALID_ARG),
+    (dict(w=None), Status.INVALID_ARG),
+    (dict(y=None), Status.INVALID_ARG),
+    (dict(N=0), Status.INVALID_ARG),
+    (dict(Cin=-8), Status.INVALID_ARG),
+    (dict(dtype=7), Status.INVALID_ARG),
+    (dict(tpad=9), Status.INVALID_ARG),
+    (dict(kernel=(3, 0, 3)), Status.INVALID_ARG),
+    (dict(pad=(1, 1, 1)), Status.INVALID_ARG),            # pt must be 0 in causal modes
+    (dict(pad=(0, -1, 1), tpad=c3.TPAD_ZERO), Status.INVALID_ARG),
+    (dict(H=1, pad=(0, 0, 1)), Status.INVALID_ARG),        # padded input smaller than kernel
+    (dict(stride=(1, 2, 2)), Status.UNSUPPORTED),
+    (dict(Cin=12), Status.UNSUPPORTED),
+    (dict(Cout=20), Status.UNSUPPORTED),
+    (dict(kernel=(3, 9, 3)), Status.UNSUPPORTED),
+    (dict(x=X + 8), Status.ALIGNMENT),
+    (dict(y=Y + 2), Status.ALIGNMENT),
+    (dict(bias=B + 4), Status.ALIGNMENT),
+    (dict(residual=R + 8), Status.ALIGNMENT),
+    (dict(y=X + 256), Status.INVALID_ARG),                 # y overlaps x
+    (dict(residual=Y + 4096), Status.INVALID_ARG),         # residual partially overlaps y
+])
+def test_validation_errors(kw, expect):
+    assert call(**kw) == expect
+    assert c3.last_error()
+
+
+def test_ws_entry_point_requires_workspace_for_first_frame():
+    a = dict(x=X, w=Wt, bias=B, residual=None, y=Y, N=1, Cin=64, D=1, H=16, W=16, Cout=64,
+             kernel=(3, 3, 3), stride=(1, 1, 1), pad=(0, 1, 1), tpad=c3.TPAD_CAUSAL_REPLICATE,
+             dtype=c3.BF16, stream=None)
+    assert c3.conv3d_fwd_ws_ptr(**a, workspace=None, ws_bytes=0) == Status.WORKSPACE
+    need = c3.workspace_bytes(64, 64, 1, (3, 3, 3), c3.TPAD_CAUSAL_REPLICATE)
+    assert c3.conv3d_fwd_ws_ptr(**a, workspace=0x600000000, ws_bytes=need - 1) == Status.WORKSPACE
+    assert c3.conv3d_fwd_ws_ptr(**a, workspace=0x600000010, ws_bytes=need) == Status.ALIGNMENT
+    assert c3.conv3d_fwd_ws_ptr(**a, workspace=Wt, ws_bytes=need) == Status.INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_valid_call_without_gpu_reports_cuda_error():
+    # a well-formed problem gets past validation and fails at the first CUDA call
+    assert call() == Status.CUDA
+    assert c3.last_error()
+
+
+def test_selftest_rejects_bad_limits():
+    assert c3.selftest_wait_timeout(0) == Status.INVALID_ARG
+    assert c3.selftest_wait_timeout(20000) == Status.INVALID_ARG
+
+
+def test_torch_wrapper_rejects_host_tensors():
+    x = torch.zeros(1, 2, 4, 4, 8, dtype=torch.bfloat16)
+    w = torch.zeros(8, 3, 3, 3, 8, dtype=torch.bfloat16)
+    y = torch.zeros(1, 2, 4, 4, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        c3.conv3d_fwd(x, w, None, None, y)

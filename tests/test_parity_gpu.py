@@ -1,0 +1,157 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Small problems are compared on every output element; the full-size workloads
+are compared on sampled rows (borders, first/last frames, first/last tiles,
+random interior points) that the oracle evaluates one by one, in the same
+launch configuration the bench times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import seeded_inputs as si
+import video_vae_convolution_implicit_b200 as c3
+from seeded_inputs.workloads import WORKLOADS
+from parity import assert_close, oracle_ref, problem, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+ZERO, CREP, CZERO = c3.TPAD_ZERO, c3.TPAD_CAUSAL_REPLICATE, c3.TPAD_CAUSAL_ZERO
+
+
+def run(p, residual_into_y=False, workspace=None):
+    Do, Ho, Wo = p["out"]
+    y = torch.empty((p["N"], Do, Ho, Wo, p["Cout"]), dtype=p["x"].dtype, device="cuda")
+    res = p["residual"]
+    if residual_into_y:
+        y.copy_(res)
+        res = y
+    c3.conv3d_fwd(p["x"], p["w"], p["bias"], res, y, (1, 1, 1), p["pad"], p["tpad"],
+                  workspace=workspace)
+    assert c3.poll_status() == c3.Status.OK
+    return y
+
+
+def full_check(p, **kw):
+    ref = oracle_ref(p)
+    y = run(p, **kw)
+    return assert_close(y.double().cpu().numpy(), ref, str({k: p[k] for k in ("N", "Cin", "Cout", "D", "H", "W", "kernel", "pad", "tpad")}))
+
+
+# ------------------------------------------------------------------ small, every element
+
+SMALL = [
+    # N, Cin, D, H, W, Cout, kernel, pad, tpad, dtype, residual
+    (1, 32, 5, 32, 32, 32, (3, 3, 3), (1, 1, 1), ZERO, "f16", False),      # workload cfg1 shape
+    (2, 64, 3, 9, 13, 64, (3, 3, 3), (0, 1, 1), CREP, "bf16", True),      # ragged frame < 1 tile
+    (1, 128, 4, 20, 19, 96, (3, 3, 3), (0, 1, 1), CZERO, "bf16", False),  # 3 tiles/frame, ragged
+    (1, 40, 3, 12, 12, 264, (3, 3, 3), (1, 1, 1), ZERO, "bf16", True),    # partial chunk, 2 N tiles
+    (1, 8, 3, 6, 7, 8, (3, 3, 3), (0, 1, 1), CREP, "bf16", False),        # minimal channels
+    (1, 256, 2, 16, 16, 128, (1, 1, 1), (0, 0, 0), ZERO, "bf16", False),  # pointwise
+    (1, 64, 4, 10, 14, 64, (1, 3, 3), (0, 1, 1), CREP, "bf16", False),
+    (1, 64, 5, 10, 10, 32, (3, 1, 1), (0, 0, 0), CREP, "f16", False),
+    (2, 64, 4, 9, 9, 48, (2, 3, 3), (0, 1, 1), CZERO, "bf16", True),
+    (1, 64, 6, 8, 8, 64, (3, 3, 3), (0, 1, 1), ZERO, "bf16", False),      # zero pt=0: Do = D-2
+    (1, 64, 3, 8, 8, 64, (3, 3, 3), (2, 1, 1), ZERO, "bf16", False),      # pt=2: edge frames 1 tap
+    (1, 64, 2, 8, 8, 64, (3, 3, 3), (3, 1, 1), ZERO, "bf16", True),       # windows fully in padding
+    (1, 192, 2, 11, 23, 200, (3, 3, 3), (0, 2, 0), CREP, "f16", True),    # asymmetric pads
+    (3, 16, 2, 5, 5, 24, (3, 3, 3), (0, 1, 1), CREP, "bf16", False),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "x".join(map(str, c[:6])) + f"-k{''.join(map(str, c[6]))}-t{c[8]}-{c[9]}")
+def test_small_every_element(case):
+    N, Cin, D, H, W, Cout, k, pad, tpad, dt, res = case
+    p = problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=100 + Cin + Cout, dtype=dt, residual=res)
+    full_check(p)
+
+
+def test_no_bias_no_residual():
+    p = problem(1, 64, 3, 10, 12, 64, (3, 3, 3), (0, 1, 1), CREP, seed=3, bias=False)
+    full_check(p)
+
+
+def test_residual_in_place():
+    p = problem(1, 64, 3, 10, 12, 64, (3, 3, 3), (0, 1, 1), CREP, seed=4, residual=True)
+    full_check(p, residual_into_y=True)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+def test_first_frame_fold(dt):
+    """D=1 with causal replicate padding runs the folded 2D path."""
+    p = problem(2, 64, 1, 24, 24, 64, (3, 3, 3), (0, 1, 1), CREP, seed=5, dtype=dt, residual=True)
+    full_check(p)
+
+
+def test_first_frame_fold_explicit_workspace():
+    p = problem(1, 128, 1, 16, 20, 64, (3, 3, 3), (0, 1, 1), CREP, seed=6)
+    need = c3.workspace_bytes(128, 64, 1, (3, 3, 3), CREP)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    ref = oracle_ref(p)
+    y = run(p, workspace=ws)
+    assert_close(y.double().cpu().numpy(), ref)
+
+
+def test_first_frame_causal_zero_uses_last_tap_only():
+    p = problem(1, 64, 1, 16, 16, 64, (3, 3, 3), (0, 1, 1), CZERO, seed=7)
+    full_check(p)
+
+
+# ------------------------------------------------------------------ robustness
+
+def test_every_output_written_and_no_overrun():
+    """Poison y with NaN, put a canary after it: all of y is written, the canary is not."""
+    p = problem(1, 64, 3, 11, 13, 40, (3, 3, 3), (0, 1, 1), CREP, seed=8, residual=True)
+    Do, Ho, Wo = p["out"]
+    n = p["N"] * Do * Ho * Wo * p["Cout"]
+    buf = torch.full((n + 4096,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    buf[n:] = 1234.0
+    y = buf[:n].view(p["N"], Do, Ho, Wo, p["Cout"])
+    c3.conv3d_fwd(p["x"], p["w"], p["bias"], p["residual"], y, (1, 1, 1), p["pad"], p["tpad"])
+    assert c3.poll_status() == c3.Status.OK
+    assert torch.isfinite(y).all()
+    assert (buf[n:] == 1234.0).all()
+    assert_close(y.double().cpu().numpy(), oracle_ref(p))
+
+
+def test_deterministic_bitwise():
+    p = problem(1, 256, 3, 32, 32, 256, (3, 3, 3), (0, 1, 1), CREP, seed=9, residual=True)
+    y1 = run(p)
+    y2 = run(p)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_rejected_call_leaves_y_untouched():
+    p = problem(1, 64, 2, 8, 8, 64, (3, 3, 3), (0, 1, 1), CREP, seed=10)
+    y = torch.full((1, 2, 8, 8, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    st = c3.conv3d_fwd_ptr(p["x"].data_ptr(), p["w"].data_ptr(), None, None, y.data_ptr(),
+                           1, 64, 2, 8, 8, 64, (3, 3, 3), (1, 2, 2), (0, 1, 1), CREP, c3.BF16, 0)
+    assert st == c3.Status.UNSUPPORTED
+    torch.cuda.synchronize()
+    assert (y == 7.0).all()
+
+
+def test_bounded_wait_reports_timeout():
+    """The device wait gives up after its limit and reports it; the context stays usable."""
+    import time
+    t0 = time.time()
+    assert c3.selftest_wait_timeout(50) == c3.Status.TIMEOUT
+    assert time.time() - t0 < 5.0
+    assert c3.poll_status() == c3.Status.OK       # the word was cleared
+    test_no_bias_no_residual()                    # and the GPU still computes
+
+
+# ------------------------------------------------------------------ full-size workloads, sampled
+
+@pytest.mark.parametrize("name", ["cfg1", "cfg2", "cfg3", "cfg4", "cfg5a", "cfg5b", "cfg5c", "cfg5d"])
+def test_workload_sampled(name):
+    wl = WORKLOADS[name]
+    p = problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, wl.pad, wl.tpad, wl.seed,
+                wl.dtype, True, wl.residual)
+    y = run(p)
+    Do, Ho, Wo = p["out"]
+    rows = sample_rows(wl.N, Do, Ho, Wo, n_random=256, seed=wl.seed)
+    ref = oracle_ref(p, rows=rows)
+    got = y.view(-1, wl.Cout)[torch.from_numpy(rows).cuda()].double().cpu().numpy()
+    assert_close(got, ref, name)
+    assert torch.isfinite(y).all()

@@ -1,0 +1,210 @@
+"""Python binding of libconv3d: implicit-GEMM 3D convolution on B200 (sm_100a).
+
+Argument marshalling only.  Every step of the convolution runs in the CUDA
+library ``libconv3d.so`` (built from ``csrc/`` by ``build.py``); torch is used
+here for device memory and streams.  There is no fallback: if the library is
+missing or fails to load, importing this package raises.
+
+Operation (engineering.drawthings.ai, "Metal conv3d" post; Qwen Image post,
+"Video VAE" section): y = conv3d(x, w) + bias + residual with NDHWC
+activations, [Cout, kt, kh, kw, Cin] weights, spatial zero padding and a
+temporal padding mode (zero, causal replicate-first-frame, causal zero).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "TPAD_ZERO", "TPAD_CAUSAL_REPLICATE", "TPAD_CAUSAL_ZERO", "F16", "BF16", "Status",
+    "Conv3dError", "lib_path", "conv3d", "conv3d_fwd", "conv3d_fwd_ptr", "conv3d_fwd_ws_ptr",
+    "output_shape", "workspace_bytes", "poll_status", "selftest_wait_timeout", "release",
+]
+
+F16 = 0
+BF16 = 1
+TPAD_ZERO = 0
+TPAD_CAUSAL_REPLICATE = 1
+TPAD_CAUSAL_ZERO = 2
+
+
+class Status:
+    OK = 0
+    INVALID_ARG = 1
+    UNSUPPORTED = 2
+    ALIGNMENT = 3
+    CUDA = 4
+    TIMEOUT = 5
+    DEVICE_CHECK = 6
+    WORKSPACE = 7
+
+
+class Conv3dError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"libconv3d status {status}: {message}")
+        self.status = status
+
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_PKG, "libconv3d.so")
+
+if not os.path.exists(lib_path):
+    raise ImportError(f"{lib_path} is missing: build it with "
+                      "`python video_vae_convolution_implicit_b200/build.py` (nvcc, sm_100a)")
+_lib = ctypes.CDLL(lib_path)
+
+_i3 = ctypes.c_int * 3
+_vp = ctypes.c_void_p
+_c = ctypes.c_int
+
+_lib.conv3d_fwd.restype = _c
+_lib.conv3d_fwd.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp]
+_lib.conv3d_fwd_ws.restype = _c
+_lib.conv3d_fwd_ws.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp, ctypes.c_size_t, _vp]
+_lib.conv3d_workspace_bytes.restype = ctypes.c_size_t
+_lib.conv3d_workspace_bytes.argtypes = [_c, _c, _c, _i3, _c]
+_lib.conv3d_output_shape.restype = _c
+_lib.conv3d_output_shape.argtypes = [_c, _c, _c, _i3, _i3, _i3, _c, _i3]
+_lib.conv3d_poll_status.restype = _c
+_lib.conv3d_poll_status.argtypes = [_vp]
+_lib.conv3d_status_string.restype = ctypes.c_char_p
+_lib.conv3d_status_string.argtypes = [_c]
+_lib.conv3d_last_error.restype = ctypes.c_char_p
+_lib.conv3d_last_error.argtypes = []
+_lib.conv3d_release.restype = None
+_lib.conv3d_release.argtypes = []
+_lib.conv3d_selftest_wait_timeout.restype = _c
+_lib.conv3d_selftest_wait_timeout.argtypes = [_c]
+
+
+def raw_library() -> ctypes.CDLL:
+    """The loaded ctypes handle of libconv3d.so."""
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.conv3d_status_string(status).decode()
+
+
+def last_error() -> str:
+    return _lib.conv3d_last_error().decode()
+
+
+def _check(status: int) -> None:
+    if status != Status.OK:
+        raise Conv3dError(status, f"{status_string(status)}: {last_error()}")
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return BF16
+    if t == torch.float16:
+        return F16
+    raise TypeError(f"libconv3d computes in bf16 or fp16, got {t}")
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def output_shape(D, H, W, kernel, stride=(1, 1, 1), pad=(0, 1, 1), tpad=TPAD_CAUSAL_REPLICATE):
+    out = _i3()
+    _check(_lib.conv3d_output_shape(D, H, W, _i3(*kernel), _i3(*stride), _i3(*pad), tpad, out))
+    return tuple(out)
+
+
+def workspace_bytes(Cin, Cout, D, kernel, tpad) -> int:
+    return int(_lib.conv3d_workspace_bytes(Cin, Cout, D, _i3(*kernel), tpad))
+
+
+def conv3d_fwd_ptr(x, w, bias, residual, y, N, Cin, D, H, W, Cout, kernel, stride, pad, tpad,
+                   dtype, stream) -> int:
+    """Raw-pointer call of conv3d_fwd; returns the status code (no raise)."""
+    return _lib.conv3d_fwd(x, w, bias, residual, y, N, Cin, D, H, W, Cout, _i3(*kernel),
+                           _i3(*stride), _i3(*pad), tpad, dtype, stream)
+
+
+def conv3d_fwd_ws_ptr(x, w, bias, residual, y, N, Cin, D, H, W, Cout, kernel, stride, pad, tpad,
+                      dtype, workspace, ws_bytes, stream) -> int:
+    """Raw-pointer call of conv3d_fwd_ws; returns the status code (no raise)."""
+    return _lib.conv3d_fwd_ws(x, w, bias, residual, y, N, Cin, D, H, W, Cout, _i3(*kernel),
+                              _i3(*stride), _i3(*pad), tpad, dtype, workspace, ws_bytes, stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def conv3d_fwd(x: torch.Tensor, w: torch.Tensor, bias, residual, y: torch.Tensor,
+               stride=(1, 1, 1), pad=(0, 1, 1), tpad=TPAD_CAUSAL_REPLICATE, stream=None,
+               workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Enqueue y = conv3d(x, w) + bias + residual on ``stream`` (default: current stream).
+
+    x: [N, D, H, W, Cin]; w: [Cout, kt, kh, kw, Cin]; bias: [Cout] or None;
+    residual: y's shape or None; y: [N, Do, Ho, Wo, Cout].  All contiguous CUDA
+    tensors of one dtype (bf16 or fp16).  With ``workspace`` (a uint8 CUDA
+    tensor) the call goes through conv3d_fwd_ws and never allocates.
+    """
+    for name, t in (("x", x), ("w", w), ("y", y), ("bias", bias), ("residual", residual)):
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.dtype != x.dtype:
+            raise TypeError(f"{name} has dtype {t.dtype}, x has {x.dtype}")
+    if x.dim() != 5 or w.dim() != 5:
+        raise ValueError("x must be [N,D,H,W,Cin] and w [Cout,kt,kh,kw,Cin]")
+    N, D, H, W, Cin = x.shape
+    Cout, kt, kh, kw, Cin_w = w.shape
+    if Cin_w != Cin:
+        raise ValueError("w's last extent must equal Cin")
+    out = output_shape(D, H, W, (kt, kh, kw), stride, pad, tpad)
+    if tuple(y.shape) != (N, *out, Cout):
+        raise ValueError(f"y must be {(N, *out, Cout)}, got {tuple(y.shape)}")
+    if residual is not None and tuple(residual.shape) != tuple(y.shape):
+        raise ValueError("residual must have y's shape")
+    if bias is not None and tuple(bias.shape) != (Cout,):
+        raise ValueError("bias must be [Cout]")
+    code = _dtype_code(x.dtype)
+    s = _stream_handle(stream)
+    if workspace is None:
+        st = conv3d_fwd_ptr(_ptr(x), _ptr(w), _ptr(bias), _ptr(residual), _ptr(y), N, Cin, D, H,
+                            W, Cout, (kt, kh, kw), stride, pad, tpad, code, s)
+    else:
+        st = conv3d_fwd_ws_ptr(_ptr(x), _ptr(w), _ptr(bias), _ptr(residual), _ptr(y), N, Cin, D,
+                               H, W, Cout, (kt, kh, kw), stride, pad, tpad, code,
+                               _ptr(workspace), workspace.numel() * workspace.element_size(), s)
+    _check(st)
+    return y
+
+
+def conv3d(x: torch.Tensor, w: torch.Tensor, bias=None, residual=None, stride=(1, 1, 1),
+           pad=(0, 1, 1), tpad=TPAD_CAUSAL_REPLICATE, stream=None) -> torch.Tensor:
+    """Allocate y (torch) and run :func:`conv3d_fwd`."""
+    N, D, H, W, _ = x.shape
+    Cout, kt, kh, kw, _ = w.shape
+    out = output_shape(D, H, W, (kt, kh, kw), stride, pad, tpad)
+    y = torch.empty((N, *out, Cout), dtype=x.dtype, device=x.device)
+    return conv3d_fwd(x, w, bias, residual, y, stride, pad, tpad, stream)
+
+
+def poll_status(stream=None) -> int:
+    """Synchronise ``stream`` and return (and clear) the device status word."""
+    return int(_lib.conv3d_poll_status(_stream_handle(stream)))
+
+
+def selftest_wait_timeout(timeout_ms: int) -> int:
+    """Run the bounded-wait self test; returns Status.TIMEOUT when it works."""
+    return int(_lib.conv3d_selftest_wait_timeout(timeout_ms))
+
+
+def release() -> None:
+    _lib.conv3d_release()

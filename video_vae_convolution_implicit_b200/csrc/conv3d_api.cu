@@ -1,0 +1,597 @@
+// conv3d_api.cu -- the C ABI of libconv3d (declared in include/conv3d.h):
+// argument validation, problem -> GEMM mapping, tensor-map encoding, the
+// first-frame weight fold and the kernel launch.  No call synchronises except
+// conv3d_poll_status and the self test; nothing allocates except the cached
+// first-frame workspace of conv3d_fwd.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "conv3d.h"
+#include "conv3d_kernel.cuh"
+
+namespace {
+
+using namespace conv3d;
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+
+thread_local char g_last_error[512] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+}
+
+conv3d_status_t cuda_fail(cudaError_t e, const char* what) {
+  set_error("%s: %s", what, cudaGetErrorString(e));
+  return CONV3D_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ problem
+
+struct Problem {
+  int N, Cin, D, H, W, Cout;
+  int kt, kh, kw;
+  int pt, ph, pw;
+  int pf, pb;
+  int Do, Ho, Wo;
+  conv3d_tpad_t tpad;
+  conv3d_dtype_t dtype;
+  bool fold;  // first-frame path: fold the temporal taps into a (hi, lo) pair
+};
+
+bool output_extents(int D, int H, int W, const int k[3], const int pad[3], conv3d_tpad_t tpad,
+                    int& pf, int& pb, int out[3]) {
+  if (tpad == CONV3D_TPAD_ZERO) {
+    pf = pad[0];
+    pb = pad[0];
+  } else {
+    pf = k[0] - 1;
+    pb = 0;
+  }
+  long long nd = static_cast<long long>(D) + pf + pb - k[0];
+  long long nh = static_cast<long long>(H) + 2LL * pad[1] - k[1];
+  long long nw = static_cast<long long>(W) + 2LL * pad[2] - k[2];
+  if (nd < 0 || nh < 0 || nw < 0) return false;
+  out[0] = static_cast<int>(nd + 1);
+  out[1] = static_cast<int>(nh + 1);
+  out[2] = static_cast<int>(nw + 1);
+  return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+conv3d_status_t validate(const void* x, const void* w, const void* bias, const void* residual,
+                         const void* y, int N, int Cin, int D, int H, int W, int Cout,
+                         const int kernel[3], const int stride[3], const int pad[3],
+                         conv3d_tpad_t tpad, conv3d_dtype_t dtype, Problem& P) {
+  if (!x || !w || !y || !kernel || !stride || !pad) {
+    set_error("x, w, y, kernel, stride and pad must be non-null");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if (N < 1 || Cin < 1 || D < 1 || H < 1 || W < 1 || Cout < 1) {
+    set_error("sizes must be >= 1");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if (dtype != CONV3D_F16 && dtype != CONV3D_BF16) {
+    set_error("unknown dtype %d", static_cast<int>(dtype));
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if (tpad != CONV3D_TPAD_ZERO && tpad != CONV3D_TPAD_CAUSAL_REPLICATE &&
+      tpad != CONV3D_TPAD_CAUSAL_ZERO) {
+    set_error("unknown temporal padding mode %d", static_cast<int>(tpad));
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  for (int i = 0; i < 3; ++i) {
+    if (kernel[i] < 1 || stride[i] < 1 || pad[i] < 0) {
+      set_error("kernel and stride must be >= 1 and pad >= 0");
+      return CONV3D_ERR_INVALID_ARG;
+    }
+  }
+  if (tpad != CONV3D_TPAD_ZERO && pad[0] != 0) {
+    set_error("pad[0] must be 0 for the causal temporal modes");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  int out[3];
+  int pf = 0, pb = 0;
+  if (!output_extents(D, H, W, kernel, pad, tpad, pf, pb, out)) {
+    set_error("the padded input is smaller than the kernel");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if (stride[0] != 1 || stride[1] != 1 || stride[2] != 1) {
+    set_error("only stride (1,1,1) is supported");
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  for (int i = 0; i < 3; ++i) {
+    if (kernel[i] > 8 || pad[i] > 127) {
+      set_error("kernel extents must be <= 8 and pads <= 127");
+      return CONV3D_ERR_UNSUPPORTED;
+    }
+  }
+  if (Cin % 8 != 0 || Cout % 8 != 0) {
+    set_error("Cin and Cout must be multiples of 8 (got %d, %d)", Cin, Cout);
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  const long long frames = static_cast<long long>(N) * D;
+  const long long M = static_cast<long long>(N) * out[0] * out[1] * out[2];
+  const long long HoWo = static_cast<long long>(out[1]) * out[2];
+  const long long tiles = static_cast<long long>(N) * out[0] * ((HoWo + BM - 1) / BM) *
+                          ((Cout + 255) / 256);
+  if (frames > 0x7FFFFFFFLL || HoWo > 0x7FFFFFFFLL || tiles > 0x7FFFFFFFLL ||
+      static_cast<long long>(H) * W > 0x7FFFFFFFLL) {
+    set_error("problem too large for 32-bit tile indexing");
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y) || (bias && !aligned16(bias)) ||
+      (residual && !aligned16(residual))) {
+    set_error("tensor pointers must be 16-byte aligned");
+    return CONV3D_ERR_ALIGNMENT;
+  }
+  const size_t xb = static_cast<size_t>(frames) * H * W * Cin * 2;
+  const size_t wb = static_cast<size_t>(Cout) * kernel[0] * kernel[1] * kernel[2] * Cin * 2;
+  const size_t yb = static_cast<size_t>(M) * Cout * 2;
+  if (overlaps(y, yb, x, xb) || overlaps(y, yb, w, wb) || overlaps(y, yb, bias, Cout * 2ull)) {
+    set_error("y must not overlap x, w or bias");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if (residual && residual != y && overlaps(y, yb, residual, yb)) {
+    set_error("residual must be exactly y or not overlap it");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  P.N = N; P.Cin = Cin; P.D = D; P.H = H; P.W = W; P.Cout = Cout;
+  P.kt = kernel[0]; P.kh = kernel[1]; P.kw = kernel[2];
+  P.pt = pad[0]; P.ph = pad[1]; P.pw = pad[2];
+  P.pf = pf; P.pb = pb;
+  P.Do = out[0]; P.Ho = out[1]; P.Wo = out[2];
+  P.tpad = tpad;
+  P.dtype = dtype;
+  P.fold = (tpad == CONV3D_TPAD_CAUSAL_REPLICATE && D == 1 && kernel[0] > 1);
+  return CONV3D_OK;
+}
+
+// The folded weight holds a high and a low 16-bit part per element.
+size_t fold_bytes(int Cin, int Cout, const int k[3]) {
+  const size_t b = 2 * static_cast<size_t>(Cout) * k[1] * k[2] * Cin * 2;
+  return (b + 255) & ~static_cast<size_t>(255);
+}
+
+// ------------------------------------------------------------------ driver entry points
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+PFN_cuTensorMapEncodeIm2col_v12000 g_encode_im2col = nullptr;
+std::once_flag g_entry_once;
+cudaError_t g_entry_err = cudaSuccess;
+
+conv3d_status_t load_entry_points() {
+  std::call_once(g_entry_once, [] {
+    cudaDriverEntryPointQueryResult q1, q2;
+    void* p1 = nullptr;
+    void* p2 = nullptr;
+    cudaError_t e1 = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p1, cudaEnableDefault, &q1);
+    cudaError_t e2 = cudaGetDriverEntryPoint("cuTensorMapEncodeIm2col", &p2, cudaEnableDefault, &q2);
+    if (e1 != cudaSuccess || q1 != cudaDriverEntryPointSuccess || !p1) {
+      g_entry_err = e1 != cudaSuccess ? e1 : cudaErrorNotSupported;
+    } else if (e2 != cudaSuccess || q2 != cudaDriverEntryPointSuccess || !p2) {
+      g_entry_err = e2 != cudaSuccess ? e2 : cudaErrorNotSupported;
+    } else {
+      g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p1);
+      g_encode_im2col = reinterpret_cast<PFN_cuTensorMapEncodeIm2col_v12000>(p2);
+    }
+  });
+  if (!g_encode_tiled || !g_encode_im2col) return cuda_fail(g_entry_err, "driver entry points");
+  return CONV3D_OK;
+}
+
+// ------------------------------------------------------------------ per-device state
+
+struct DeviceState {
+  bool init = false;
+  int num_sms = 0;
+  int max_smem_optin = 0;
+  int* status = nullptr;         // address of g_status on this device
+  void* workspace = nullptr;     // cached first-frame fold buffer (conv3d_fwd)
+  size_t workspace_bytes = 0;
+  bool attr_set[2] = {false, false};
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+__device__ int g_status;
+
+conv3d_status_t device_state(DeviceState*& out, int& dev) {
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) {
+    set_error("device ordinal %d out of range", dev);
+    return CONV3D_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.init) {
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&s.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                    dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    if (major != 10 || minor != 0) {
+      set_error("libconv3d is built for sm_100a; device %d is sm_%d%d", dev, major, minor);
+      return CONV3D_ERR_UNSUPPORTED;
+    }
+    void* sp = nullptr;
+    if ((e = cudaGetSymbolAddress(&sp, g_status)) != cudaSuccess)
+      return cuda_fail(e, "cudaGetSymbolAddress(status)");
+    s.status = static_cast<int*>(sp);
+    s.init = true;
+  }
+  out = &s;
+  return CONV3D_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+conv3d_status_t encode_maps(const Problem& P, const void* x, const void* wmat, int kt_eff,
+                            int BN, CUtensorMap& map_a, CUtensorMap& map_b) {
+  const CUtensorMapDataType dt =
+      P.dtype == CONV3D_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  // A: the input viewed as N*D images of H x W pixels with Cin channels;
+  // each load gathers BM output pixels' windows shifted by one tap.
+  {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(P.Cin), static_cast<cuuint64_t>(P.W),
+                                static_cast<cuuint64_t>(P.H),
+                                static_cast<cuuint64_t>(P.N) * static_cast<cuuint64_t>(P.D)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(P.Cin) * 2,
+                                   static_cast<cuuint64_t>(P.W) * P.Cin * 2,
+                                   static_cast<cuuint64_t>(P.H) * P.W * P.Cin * 2};
+    // Window-origin box: first origin at -pad, last at dim-1+pad-(k-1).
+    const int lower[2] = {-P.pw, -P.ph};
+    const int upper[2] = {P.pw - (P.kw - 1), P.ph - (P.kh - 1)};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode_im2col(&map_a, dt, 4, const_cast<void*>(x), dims, strides, lower, upper,
+                                 BK, BM, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+      set_error("cuTensorMapEncodeIm2col failed (%d)", static_cast<int>(r));
+      return CONV3D_ERR_CUDA;
+    }
+  }
+  // B: w viewed as [Cout][taps][Cin]; a box is 64 channels of one tap for BN
+  // output channels.  Channels past Cin and rows past Cout read as zero.
+  {
+    const int taps = kt_eff * P.kh * P.kw;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(P.Cin), static_cast<cuuint64_t>(taps),
+                                static_cast<cuuint64_t>(P.Cout)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(P.Cin) * 2,
+                                   static_cast<cuuint64_t>(taps) * P.Cin * 2};
+    const cuuint32_t box[3] = {BK, 1, static_cast<cuuint32_t>(BN)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode_tiled(&map_b, dt, 3, const_cast<void*>(wmat), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+      set_error("cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+      return CONV3D_ERR_CUDA;
+    }
+  }
+  return CONV3D_OK;
+}
+
+// ------------------------------------------------------------------ launch
+
+uint32_t pow2_at_least(uint32_t v) {
+  uint32_t p = 32;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+template <bool kBF16>
+conv3d_status_t launch_main(DeviceState& S, int dev, const Problem& P, const void* x,
+                            const void* wmat, const void* bias, const void* residual, void* y,
+                            cudaStream_t stream) {
+  // The folded weight is a kt = 2 (hi, lo) kernel over the single frame; with
+  // causal replicate padding both of its taps read frame 0.
+  const int kt_eff = P.fold ? 2 : P.kt;
+  KernelParams kp{};
+  kp.n_tiles_n = (P.Cout + 255) / 256;
+  const int per_tile = (P.Cout + kp.n_tiles_n - 1) / kp.n_tiles_n;
+  kp.BN = ((per_tile + 31) / 32) * 32;
+  kp.D = P.fold ? 1 : P.D;
+  kp.Do = P.Do;
+  kp.Ho = P.Ho;
+  kp.Wo = P.Wo;
+  kp.HoWo = P.Ho * P.Wo;
+  kp.Cin = P.Cin;
+  kp.Cout = P.Cout;
+  kp.kt = kt_eff;
+  kp.kh = P.kh;
+  kp.kw = P.kw;
+  kp.pf = P.fold ? 1 : P.pf;
+  kp.ph = P.ph;
+  kp.pw = P.pw;
+  kp.tpad = P.fold ? 1 : static_cast<int>(P.tpad);
+  kp.n_chunks = (P.Cin + BK - 1) / BK;
+  kp.tiles_per_frame = (kp.HoWo + BM - 1) / BM;
+  kp.num_tiles = P.N * P.Do * kp.tiles_per_frame * kp.n_tiles_n;
+  const int b_stage = kp.BN * BK * 2;
+  const int stage_bytes = A_STAGE_BYTES + b_stage;
+  const int reserve = 1024 /*alignment slack*/ + 8 * (2 * MAX_STAGES + 5);
+  int stages = (S.max_smem_optin - reserve - 64 /*static smem*/) / stage_bytes;
+  if (stages > MAX_STAGES) stages = MAX_STAGES;
+  if (stages < 2) {
+    set_error("not enough shared memory for two pipeline stages");
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  kp.stages = stages;
+  kp.tmem_cols = pow2_at_least(2u * kp.BN);
+  kp.idesc = idesc_f16(kBF16, BM, kp.BN);
+  kp.bias = bias;
+  kp.residual = residual;
+  kp.y = y;
+  kp.status = S.status;
+  kp.timeout_ns = kDefaultTimeoutNs;
+  const size_t smem = static_cast<size_t>(stages) * stage_bytes + reserve;
+
+  CUtensorMap map_a, map_b;
+  conv3d_status_t st = encode_maps(P, x, wmat, kt_eff, kp.BN, map_a, map_b);
+  if (st != CONV3D_OK) return st;
+
+  auto kern = conv3d_implicit_gemm_kernel<kBF16>;
+  cudaError_t e;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!S.attr_set[kBF16 ? 1 : 0]) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               S.max_smem_optin - 64);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      S.attr_set[kBF16 ? 1 : 0] = true;
+    }
+  }
+  const int grid = kp.num_tiles < S.num_sms ? kp.num_tiles : S.num_sms;
+  kern<<<grid, NUM_THREADS, smem, stream>>>(map_a, map_b, kp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "conv3d kernel launch");
+  (void)dev;
+  return CONV3D_OK;
+}
+
+conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* bias,
+                    const void* residual, void* y, void* ws, size_t ws_bytes, bool cached_ws,
+                    cudaStream_t stream) {
+  conv3d_status_t st = load_entry_points();
+  if (st != CONV3D_OK) return st;
+  DeviceState* S = nullptr;
+  int dev = 0;
+  if ((st = device_state(S, dev)) != CONV3D_OK) return st;
+  const bool bf16 = P.dtype == CONV3D_BF16;
+  const void* wmat = w;
+  if (P.fold) {
+    const int k[3] = {P.kt, P.kh, P.kw};
+    const size_t need = fold_bytes(P.Cin, P.Cout, k);
+    if (cached_ws) {
+      std::lock_guard<std::mutex> lock(g_mu);
+      if (S->workspace_bytes < need) {
+        if (S->workspace) {
+          cudaError_t e = cudaFree(S->workspace);
+          S->workspace = nullptr;
+          S->workspace_bytes = 0;
+          if (e != cudaSuccess) return cuda_fail(e, "cudaFree(workspace)");
+        }
+        cudaError_t e = cudaMalloc(&S->workspace, need);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(workspace)");
+        S->workspace_bytes = need;
+      }
+      ws = S->workspace;
+    } else {
+      if (ws == nullptr || ws_bytes < need) {
+        set_error("workspace of %zu bytes required", need);
+        return CONV3D_ERR_WORKSPACE;
+      }
+      if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) {
+        set_error("workspace must be 256-byte aligned");
+        return CONV3D_ERR_ALIGNMENT;
+      }
+    }
+    const int spatial_cin = P.kh * P.kw * P.Cin;
+    const long long total = static_cast<long long>(P.Cout) * spatial_cin;
+    int blocks = static_cast<int>((total + 255) / 256);
+    if (blocks > 4 * S->num_sms) blocks = 4 * S->num_sms;
+    if (bf16)
+      fold_temporal_taps_kernel<true><<<blocks, 256, 0, stream>>>(
+          static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), P.Cout, P.kt, spatial_cin);
+    else
+      fold_temporal_taps_kernel<false><<<blocks, 256, 0, stream>>>(
+          static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), P.Cout, P.kt, spatial_cin);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "fold kernel launch");
+    wmat = ws;
+  }
+  return bf16 ? launch_main<true>(*S, dev, P, x, wmat, bias, residual, y, stream)
+              : launch_main<false>(*S, dev, P, x, wmat, bias, residual, y, stream);
+}
+
+__global__ void selftest_wait_kernel(int* status, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_abort;
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    mbar_init(smem_addr(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    SharedCtl ctl{&s_abort, status, timeout_ns};
+    // Nothing ever arrives on `bar`: the bounded wait must give up.
+    wait_bounded(smem_addr(&bar), 0, ctl, false);
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+conv3d_status_t conv3d_fwd(const void* x, const void* w, const void* bias, const void* residual,
+                           void* y, int N, int Cin, int D, int H, int W, int Cout,
+                           const int kernel[3], const int stride[3], const int pad[3],
+                           conv3d_tpad_t tpad, conv3d_dtype_t dtype, struct CUstream_st* stream) {
+  Problem P;
+  conv3d_status_t st = validate(x, w, bias, residual, y, N, Cin, D, H, W, Cout, kernel, stride,
+                                pad, tpad, dtype, P);
+  if (st != CONV3D_OK) return st;
+  return run(P, x, w, bias, residual, y, nullptr, 0, true, stream);
+}
+
+conv3d_status_t conv3d_fwd_ws(const void* x, const void* w, const void* bias, const void* residual,
+                              void* y, int N, int Cin, int D, int H, int W, int Cout,
+                              const int kernel[3], const int stride[3], const int pad[3],
+                              conv3d_tpad_t tpad, conv3d_dtype_t dtype, void* workspace,
+                              size_t ws_bytes, struct CUstream_st* stream) {
+  Problem P;
+  conv3d_status_t st = validate(x, w, bias, residual, y, N, Cin, D, H, W, Cout, kernel, stride,
+                                pad, tpad, dtype, P);
+  if (st != CONV3D_OK) return st;
+  if (P.fold) {
+    const size_t need = fold_bytes(Cin, Cout, kernel);
+    if (workspace == nullptr || ws_bytes < need) {
+      set_error("workspace of %zu bytes required", need);
+      return CONV3D_ERR_WORKSPACE;
+    }
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) {
+      set_error("workspace must be 256-byte aligned");
+      return CONV3D_ERR_ALIGNMENT;
+    }
+    const size_t wsz = static_cast<size_t>(Cout) * kernel[0] * kernel[1] * kernel[2] * Cin * 2;
+    const size_t ysz = static_cast<size_t>(N) * P.Do * P.Ho * P.Wo * Cout * 2;
+    if (overlaps(workspace, need, w, wsz) || overlaps(workspace, need, y, ysz) ||
+        overlaps(workspace, need, x, static_cast<size_t>(N) * D * H * W * Cin * 2)) {
+      set_error("workspace must not overlap x, w or y");
+      return CONV3D_ERR_INVALID_ARG;
+    }
+  }
+  return run(P, x, w, bias, residual, y, workspace, ws_bytes, false, stream);
+}
+
+size_t conv3d_workspace_bytes(int Cin, int Cout, int D, const int kernel[3], conv3d_tpad_t tpad) {
+  if (!kernel || Cin < 1 || Cout < 1 || D < 1) return 0;
+  if (tpad == CONV3D_TPAD_CAUSAL_REPLICATE && D == 1 && kernel[0] > 1)
+    return fold_bytes(Cin, Cout, kernel);
+  return 0;
+}
+
+conv3d_status_t conv3d_output_shape(int D, int H, int W, const int kernel[3], const int stride[3],
+                                    const int pad[3], conv3d_tpad_t tpad, int out_dhw[3]) {
+  if (!kernel || !stride || !pad || !out_dhw || D < 1 || H < 1 || W < 1)
+    return CONV3D_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (kernel[i] < 1 || stride[i] < 1 || pad[i] < 0) return CONV3D_ERR_INVALID_ARG;
+  int pf, pb;
+  int out[3];
+  if (tpad == CONV3D_TPAD_ZERO) {
+    pf = pb = pad[0];
+  } else if (tpad == CONV3D_TPAD_CAUSAL_REPLICATE || tpad == CONV3D_TPAD_CAUSAL_ZERO) {
+    pf = kernel[0] - 1;
+    pb = 0;
+  } else {
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  const long long ext[3] = {static_cast<long long>(D) + pf + pb, static_cast<long long>(H) + 2LL * pad[1],
+                            static_cast<long long>(W) + 2LL * pad[2]};
+  for (int i = 0; i < 3; ++i) {
+    if (ext[i] < kernel[i]) return CONV3D_ERR_INVALID_ARG;
+    out[i] = static_cast<int>((ext[i] - kernel[i]) / stride[i] + 1);
+  }
+  for (int i = 0; i < 3; ++i) out_dhw[i] = out[i];
+  return CONV3D_OK;
+}
+
+conv3d_status_t conv3d_poll_status(struct CUstream_st* stream) {
+  DeviceState* S = nullptr;
+  int dev = 0;
+  conv3d_status_t st = device_state(S, dev);
+  if (st != CONV3D_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  if ((e = cudaMemcpy(&v, S->status, sizeof v, cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "read status");
+  const int zero = 0;
+  if ((e = cudaMemcpy(S->status, &zero, sizeof zero, cudaMemcpyHostToDevice)) != cudaSuccess)
+    return cuda_fail(e, "clear status");
+  return static_cast<conv3d_status_t>(v);
+}
+
+const char* conv3d_status_string(conv3d_status_t s) {
+  switch (s) {
+    case CONV3D_OK: return "ok";
+    case CONV3D_ERR_INVALID_ARG: return "invalid argument";
+    case CONV3D_ERR_UNSUPPORTED: return "unsupported problem";
+    case CONV3D_ERR_ALIGNMENT: return "misaligned pointer";
+    case CONV3D_ERR_CUDA: return "CUDA error";
+    case CONV3D_ERR_TIMEOUT: return "device wait timed out";
+    case CONV3D_ERR_DEVICE_CHECK: return "device check failed";
+    case CONV3D_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+const char* conv3d_last_error(void) { return g_last_error; }
+
+void conv3d_release(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return;
+  for (int d = 0; d < kMaxDevices; ++d) {
+    if (g_dev[d].workspace) {
+      cudaSetDevice(d);
+      cudaFree(g_dev[d].workspace);
+      g_dev[d].workspace = nullptr;
+      g_dev[d].workspace_bytes = 0;
+    }
+  }
+  cudaSetDevice(cur);
+}
+
+conv3d_status_t conv3d_selftest_wait_timeout(int timeout_ms) {
+  if (timeout_ms < 1 || timeout_ms > 10000) {
+    set_error("timeout_ms must be in [1, 10000]");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  DeviceState* S = nullptr;
+  int dev = 0;
+  conv3d_status_t st = device_state(S, dev);
+  if (st != CONV3D_OK) return st;
+  cudaStream_t s;
+  cudaError_t e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreate");
+  selftest_wait_kernel<<<1, 32, 0, s>>>(S->status, static_cast<unsigned long long>(timeout_ms) * 1000000ull);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    cudaStreamDestroy(s);
+    return cuda_fail(e, "self-test launch");
+  }
+  st = conv3d_poll_status(s);
+  cudaStreamDestroy(s);
+  return st;
+}
+
+}  // extern "C"
