@@ -107,6 +107,41 @@ CONV3D_API conv3d_status_t conv3d_fwd_ws(const void* x, const void* w, const voi
                                          conv3d_dtype_t dtype, void* workspace, size_t ws_bytes,
                                          struct CUstream_st* stream);
 
+/*
+ * conv3d_fwd_noalloc -- conv3d_fwd for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it is an interface
+ * addition of this library.
+ *
+ * Some callers must not call cudaMalloc: a host framework or plug-in host
+ * that owns all device memory through its own allocator and forbids any
+ * other allocation, a latency-critical path where an allocation may block or
+ * fail in the middle of a frame, or a deployment whose device-memory budget
+ * is fixed at start-up.  This call allocates nothing.  The caller passes x, w,
+ * bias, residual and y exactly as for conv3d_fwd; the only scratch the path
+ * needs -- the folded first-frame weight -- lives in a fixed 16 MiB array
+ * inside the library's device memory, which every GPU that loads the library
+ * holds until the process exits.
+ *
+ * Limit: a first-frame problem (CONV3D_TPAD_CAUSAL_REPLICATE, D == 1, kt > 1)
+ * must have Cout*kh*kw*Cin <= 4,194,304 (conv3d_workspace_bytes() <= 16 MiB);
+ * a larger one returns CONV3D_ERR_WORKSPACE before anything is enqueued.
+ * Problems that need no scratch run exactly as with conv3d_fwd.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array and it keeps the
+ * last call's contents; every element a call's kernels read is first written
+ * by the same call, so nothing has to start at zero.  Calls whose work
+ * overlaps on the GPU (several streams, or several host threads) race on the
+ * array: serialise them.
+ */
+CONV3D_API conv3d_status_t conv3d_fwd_noalloc(const void* x, const void* w, const void* bias,
+                                              const void* residual, void* y, int N, int Cin,
+                                              int D, int H, int W, int Cout, const int kernel[3],
+                                              const int stride[3], const int pad[3],
+                                              conv3d_tpad_t tpad, conv3d_dtype_t dtype,
+                                              struct CUstream_st* stream);
+
 /* Device scratch bytes conv3d_fwd_ws needs for this problem (0 if none). */
 CONV3D_API size_t conv3d_workspace_bytes(int Cin, int Cout, int D, const int kernel[3], conv3d_tpad_t tpad);
 

@@ -20,6 +20,7 @@ import torch
 __all__ = [
     "TPAD_ZERO", "TPAD_CAUSAL_REPLICATE", "TPAD_CAUSAL_ZERO", "F16", "BF16", "Status",
     "Conv3dError", "lib_path", "conv3d", "conv3d_fwd", "conv3d_fwd_ptr", "conv3d_fwd_ws_ptr",
+    "conv3d_fwd_noalloc_ptr",
     "output_shape", "workspace_bytes", "poll_status", "selftest_wait_timeout", "release",
 ]
 
@@ -63,6 +64,8 @@ _lib.conv3d_fwd.restype = _c
 _lib.conv3d_fwd.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp]
 _lib.conv3d_fwd_ws.restype = _c
 _lib.conv3d_fwd_ws.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp, ctypes.c_size_t, _vp]
+_lib.conv3d_fwd_noalloc.restype = _c
+_lib.conv3d_fwd_noalloc.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp]
 _lib.conv3d_workspace_bytes.restype = ctypes.c_size_t
 _lib.conv3d_workspace_bytes.argtypes = [_c, _c, _c, _i3, _c]
 _lib.conv3d_output_shape.restype = _c
@@ -135,6 +138,15 @@ def conv3d_fwd_ws_ptr(x, w, bias, residual, y, N, Cin, D, H, W, Cout, kernel, st
     """Raw-pointer call of conv3d_fwd_ws; returns the status code (no raise)."""
     return _lib.conv3d_fwd_ws(x, w, bias, residual, y, N, Cin, D, H, W, Cout, _i3(*kernel),
                               _i3(*stride), _i3(*pad), tpad, dtype, workspace, ws_bytes, stream)
+
+
+def conv3d_fwd_noalloc_ptr(x, w, bias, residual, y, N, Cin, D, H, W, Cout, kernel, stride, pad,
+                           tpad, dtype, stream) -> int:
+    """Raw-pointer call of conv3d_fwd_noalloc (for callers that cannot allocate
+    device memory; its first-frame scratch is a fixed 16 MiB array inside the
+    library).  Returns the status code (no raise)."""
+    return _lib.conv3d_fwd_noalloc(x, w, bias, residual, y, N, Cin, D, H, W, Cout, _i3(*kernel),
+                                   _i3(*stride), _i3(*pad), tpad, dtype, stream)
 
 
 def _ptr(t):

@@ -429,6 +429,40 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
               : launch_main<false>(*S, dev, P, x, wmat, bias, residual, y, stream);
 }
 
+// ------------------------------------------------------------------ allocation-free entry
+
+// Fixed scratch for conv3d_fwd_noalloc: the folded first-frame weight (hi/lo
+// parts) of any problem with Cout*kh*kw*Cin <= 4,194,304.  It lives in the
+// library's own device memory, so every GPU that loads the library holds these
+// 16 MiB until the process exits.  In host code `g_noalloc_scratch` names a
+// host-side stand-in, not a device address: the device address is looked up
+// once per device with cudaGetSymbolAddress and handed to the kernels.
+constexpr size_t kNoallocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) uint16_t g_noalloc_scratch[kNoallocScratchBytes / 2];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (set-up on first use).
+conv3d_status_t noalloc_scratch(void*& out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) {
+    set_error("device ordinal %d out of range", dev);
+    return CONV3D_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(noalloc scratch)");
+    g_noalloc_ptr[dev] = ptr;
+  }
+  out = g_noalloc_ptr[dev];
+  return CONV3D_OK;
+}
+
 __global__ void selftest_wait_kernel(int* status, unsigned long long timeout_ns) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int s_abort;
@@ -489,6 +523,28 @@ conv3d_status_t conv3d_fwd_ws(const void* x, const void* w, const void* bias, co
     }
   }
   return run(P, x, w, bias, residual, y, workspace, ws_bytes, false, stream);
+}
+
+conv3d_status_t conv3d_fwd_noalloc(const void* x, const void* w, const void* bias,
+                                   const void* residual, void* y, int N, int Cin, int D, int H,
+                                   int W, int Cout, const int kernel[3], const int stride[3],
+                                   const int pad[3], conv3d_tpad_t tpad, conv3d_dtype_t dtype,
+                                   struct CUstream_st* stream) {
+  Problem P;
+  conv3d_status_t st = validate(x, w, bias, residual, y, N, Cin, D, H, W, Cout, kernel, stride,
+                                pad, tpad, dtype, P);
+  if (st != CONV3D_OK) return st;
+  if (!P.fold) return run(P, x, w, bias, residual, y, nullptr, 0, false, stream);
+  const size_t need = fold_bytes(Cin, Cout, kernel);
+  if (need > kNoallocScratchBytes) {
+    set_error("the first-frame fold needs %zu bytes of scratch; conv3d_fwd_noalloc holds %zu "
+              "(Cout*kh*kw*Cin must be <= %zu); use conv3d_fwd_ws",
+              need, kNoallocScratchBytes, kNoallocScratchBytes / 4);
+    return CONV3D_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(scratch)) != CONV3D_OK) return st;
+  return run(P, x, w, bias, residual, y, scratch, kNoallocScratchBytes, false, stream);
 }
 
 size_t conv3d_workspace_bytes(int Cin, int Cout, int D, const int kernel[3], conv3d_tpad_t tpad) {
