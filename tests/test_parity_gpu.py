@@ -59,25 +59,35 @@ SMALL = [
 ]
 
 
+@pytest.fixture(params=["single", "pair", "swap"])
+def cta_mode(request, monkeypatch):
+    """Run a test with each kernel variant: one CTA per 128-pixel tile (M = pixels),
+    a CTA pair per 256-pixel tile (cta_group::2), or the transposed product
+    (M = 128 channels, N = 256 pixels)."""
+    monkeypatch.setenv("CONV3D_CTA_PAIR", "1" if request.param == "pair" else "0")
+    monkeypatch.setenv("CONV3D_SWAP", "1" if request.param == "swap" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: "x".join(map(str, c[:6])) + f"-k{''.join(map(str, c[6]))}-t{c[8]}-{c[9]}")
-def test_small_every_element(case):
+def test_small_every_element(case, cta_mode):
     N, Cin, D, H, W, Cout, k, pad, tpad, dt, res = case
     p = problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=100 + Cin + Cout, dtype=dt, residual=res)
     full_check(p)
 
 
-def test_no_bias_no_residual():
+def test_no_bias_no_residual(cta_mode):
     p = problem(1, 64, 3, 10, 12, 64, (3, 3, 3), (0, 1, 1), CREP, seed=3, bias=False)
     full_check(p)
 
 
-def test_residual_in_place():
+def test_residual_in_place(cta_mode):
     p = problem(1, 64, 3, 10, 12, 64, (3, 3, 3), (0, 1, 1), CREP, seed=4, residual=True)
     full_check(p, residual_into_y=True)
 
 
 @pytest.mark.parametrize("dt", ["bf16", "f16"])
-def test_first_frame_fold(dt):
+def test_first_frame_fold(dt, cta_mode):
     """D=1 with causal replicate padding runs the folded 2D path."""
     p = problem(2, 64, 1, 24, 24, 64, (3, 3, 3), (0, 1, 1), CREP, seed=5, dtype=dt, residual=True)
     full_check(p)
@@ -99,7 +109,7 @@ def test_first_frame_causal_zero_uses_last_tap_only():
 
 # ------------------------------------------------------------------ robustness
 
-def test_every_output_written_and_no_overrun():
+def test_every_output_written_and_no_overrun(cta_mode):
     """Poison y with NaN, put a canary after it: all of y is written, the canary is not."""
     p = problem(1, 64, 3, 11, 13, 40, (3, 3, 3), (0, 1, 1), CREP, seed=8, residual=True)
     Do, Ho, Wo = p["out"]
@@ -114,7 +124,7 @@ def test_every_output_written_and_no_overrun():
     assert_close(y.double().cpu().numpy(), oracle_ref(p))
 
 
-def test_deterministic_bitwise():
+def test_deterministic_bitwise(cta_mode):
     p = problem(1, 256, 3, 32, 32, 256, (3, 3, 3), (0, 1, 1), CREP, seed=9, residual=True)
     y1 = run(p)
     y2 = run(p)
@@ -138,13 +148,17 @@ def test_bounded_wait_reports_timeout():
     assert c3.selftest_wait_timeout(50) == c3.Status.TIMEOUT
     assert time.time() - t0 < 5.0
     assert c3.poll_status() == c3.Status.OK       # the word was cleared
-    test_no_bias_no_residual()                    # and the GPU still computes
+    p = problem(1, 64, 3, 10, 12, 64, (3, 3, 3), (0, 1, 1), CREP, seed=3, bias=False)
+    full_check(p)                                 # and the GPU still computes
 
 
 # ------------------------------------------------------------------ full-size workloads, sampled
 
 @pytest.mark.parametrize("name", ["cfg1", "cfg2", "cfg3", "cfg4", "cfg5a", "cfg5b", "cfg5c", "cfg5d"])
-def test_workload_sampled(name):
+def test_workload_sampled(name, monkeypatch):
+    """Full-size workloads in the launch configuration the bench times (automatic choice)."""
+    monkeypatch.delenv("CONV3D_CTA_PAIR", raising=False)
+    monkeypatch.delenv("CONV3D_SWAP", raising=False)
     wl = WORKLOADS[name]
     p = problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, wl.pad, wl.tpad, wl.seed,
                 wl.dtype, True, wl.residual)

@@ -10,6 +10,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -47,6 +48,7 @@ struct Problem {
   int Do, Ho, Wo;
   conv3d_tpad_t tpad;
   conv3d_dtype_t dtype;
+  bool has_residual;
   bool fold;  // first-frame path: fold the temporal taps into a (hi, lo) pair
 };
 
@@ -161,6 +163,7 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
   P.Do = out[0]; P.Ho = out[1]; P.Wo = out[2];
   P.tpad = tpad;
   P.dtype = dtype;
+  P.has_residual = residual != nullptr;
   P.fold = (tpad == CONV3D_TPAD_CAUSAL_REPLICATE && D == 1 && kernel[0] > 1);
   return CONV3D_OK;
 }
@@ -207,7 +210,8 @@ struct DeviceState {
   int* status = nullptr;         // address of g_status on this device
   void* workspace = nullptr;     // cached first-frame fold buffer (conv3d_fwd)
   size_t workspace_bytes = 0;
-  bool attr_set[2] = {false, false};
+  bool attr_set[8] = {};         // per kernel variant
+  int pair_clusters = 0;         // co-resident CTA pairs (occupancy query)
 };
 
 std::mutex g_mu;
@@ -249,7 +253,8 @@ conv3d_status_t device_state(DeviceState*& out, int& dev) {
 // ------------------------------------------------------------------ tensor maps
 
 conv3d_status_t encode_maps(const Problem& P, const void* x, const void* wmat, int kt_eff,
-                            int BN, CUtensorMap& map_a, CUtensorMap& map_b) {
+                            int b_box_rows, int pixels_per_load, CUtensorMap& map_a,
+                            CUtensorMap& map_b) {
   const CUtensorMapDataType dt =
       P.dtype == CONV3D_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   // A: the input viewed as N*D images of H x W pixels with Cin channels;
@@ -266,7 +271,8 @@ conv3d_status_t encode_maps(const Problem& P, const void* x, const void* wmat, i
     const int upper[2] = {P.pw - (P.kw - 1), P.ph - (P.kh - 1)};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = g_encode_im2col(&map_a, dt, 4, const_cast<void*>(x), dims, strides, lower, upper,
-                                 BK, BM, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 BK, static_cast<cuuint32_t>(pixels_per_load), estr,
+                                 CU_TENSOR_MAP_INTERLEAVE_NONE,
                                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -274,15 +280,17 @@ conv3d_status_t encode_maps(const Problem& P, const void* x, const void* wmat, i
       return CONV3D_ERR_CUDA;
     }
   }
-  // B: w viewed as [Cout][taps][Cin]; a box is 64 channels of one tap for BN
-  // output channels.  Channels past Cin and rows past Cout read as zero.
+  // w viewed as [Cout][taps][Cin]; a box is 64 channels of one tap for
+  // b_box_rows output channels (the tile's channels, or half of them for a
+  // CTA pair).
+  // Channels past Cin and rows past Cout read as zero.
   {
     const int taps = kt_eff * P.kh * P.kw;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(P.Cin), static_cast<cuuint64_t>(taps),
                                 static_cast<cuuint64_t>(P.Cout)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(P.Cin) * 2,
                                    static_cast<cuuint64_t>(taps) * P.Cin * 2};
-    const cuuint32_t box[3] = {BK, 1, static_cast<cuuint32_t>(BN)};
+    const cuuint32_t box[3] = {BK, 1, static_cast<cuuint32_t>(b_box_rows)};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode_tiled(&map_b, dt, 3, const_cast<void*>(wmat), dims, strides, box, estr,
                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -296,6 +304,29 @@ conv3d_status_t encode_maps(const Problem& P, const void* x, const void* wmat, i
   return CONV3D_OK;
 }
 
+// y (or the residual) viewed as [N*Do frames][Ho*Wo pixels][Cout]; a box is 32
+// channels x 32 pixels of one frame, 64-byte swizzled.  Stores clip pixels
+// past the frame and channels past Cout; loads read them as zero.
+conv3d_status_t encode_out_map(const Problem& P, const void* base, CUtensorMap& map) {
+  const CUtensorMapDataType dt =
+      P.dtype == CONV3D_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t howo = static_cast<cuuint64_t>(P.Ho) * P.Wo;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(P.Cout), howo,
+                              static_cast<cuuint64_t>(P.N) * static_cast<cuuint64_t>(P.Do)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(P.Cout) * 2, howo * P.Cout * 2};
+  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode_tiled(&map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled (output) failed (%d)", static_cast<int>(r));
+    return CONV3D_ERR_CUDA;
+  }
+  return CONV3D_OK;
+}
+
 // ------------------------------------------------------------------ launch
 
 uint32_t pow2_at_least(uint32_t v) {
@@ -304,17 +335,24 @@ uint32_t pow2_at_least(uint32_t v) {
   return p;
 }
 
-template <bool kBF16>
-conv3d_status_t launch_main(DeviceState& S, int dev, const Problem& P, const void* x,
-                            const void* wmat, const void* bias, const void* residual, void* y,
-                            cudaStream_t stream) {
+// Tile shape and pipeline depth for one problem.
+struct LaunchPlan {
+  bool pair;          // cta_group::2 over 256-row tiles (cluster of two CTAs)
+  bool swap;          // transposed product: M = 128 channels, N = 256 pixels
+  KernelParams kp;
+  size_t smem;
+};
+
+conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, LaunchPlan& L) {
   // The folded weight is a kt = 2 (hi, lo) kernel over the single frame; with
   // causal replicate padding both of its taps read frame 0.
   const int kt_eff = P.fold ? 2 : P.kt;
-  KernelParams kp{};
+  KernelParams& kp = L.kp;
+  kp = KernelParams{};
   kp.n_tiles_n = (P.Cout + 255) / 256;
   const int per_tile = (P.Cout + kp.n_tiles_n - 1) / kp.n_tiles_n;
   kp.BN = ((per_tile + 31) / 32) * 32;
+  kp.co_tile = kp.BN;
   kp.D = P.fold ? 1 : P.D;
   kp.Do = P.Do;
   kp.Ho = P.Ho;
@@ -330,11 +368,43 @@ conv3d_status_t launch_main(DeviceState& S, int dev, const Problem& P, const voi
   kp.pw = P.pw;
   kp.tpad = P.fold ? 1 : static_cast<int>(P.tpad);
   kp.n_chunks = (P.Cin + BK - 1) / BK;
-  kp.tiles_per_frame = (kp.HoWo + BM - 1) / BM;
+
+  // A tcgen05.mma step with N < 256 takes as long as one with N = 256, so
+  // layers whose channel count leaves the N side short run transposed
+  // (M = 128 channels, N = 256 pixels) when that needs fewer MMA steps and
+  // still gives every SM pair a tile.  CONV3D_SWAP=0/1 forces the choice.
+  const long long frames_out = static_cast<long long>(P.N) * P.Do;
+  const long long normal_steps = frames_out * ((kp.HoWo + BM - 1) / BM) * kp.n_tiles_n;
+  const long long swap_tiles = frames_out * ((kp.HoWo + 255) / 256) * ((P.Cout + 127) / 128);
+  L.swap = swap_tiles < normal_steps && swap_tiles >= S.num_sms / 2;
+  if (const char* env = getenv("CONV3D_SWAP")) {
+    if (env[0] == '0') L.swap = false;
+    if (env[0] == '1') L.swap = true;
+  }
+  // CTA pairs when there is at least one wave of 256-row tiles for them (they
+  // measure on par with single CTAs, so they are off unless forced);
+  // CONV3D_CTA_PAIR=0/1 forces the choice (tuning and tests).
+  L.pair = false;
+  if (const char* env = getenv("CONV3D_CTA_PAIR")) {
+    if (env[0] == '1') L.pair = true;
+  }
+  if (L.swap) L.pair = false;
+  const int ctas = L.pair ? 2 : 1;
+  if (L.swap) {
+    kp.co_tile = 128;
+    kp.BN = 256;                       // N = pixels
+    kp.pix_tile = 256;
+    kp.n_tiles_n = (P.Cout + 127) / 128;
+  } else {
+    kp.pix_tile = ctas * BM;
+  }
+  kp.tiles_per_frame = (kp.HoWo + kp.pix_tile - 1) / kp.pix_tile;
   kp.num_tiles = P.N * P.Do * kp.tiles_per_frame * kp.n_tiles_n;
-  const int b_stage = kp.BN * BK * 2;
+  const int b_stage = kp.BN / ctas * BK * 2;
   const int stage_bytes = A_STAGE_BYTES + b_stage;
-  const int reserve = 1024 /*alignment slack*/ + 8 * (2 * MAX_STAGES + 5);
+  kp.has_residual = P.has_residual ? 1 : 0;
+  const int reserve = 1024 /*alignment slack*/ + EPI_Y_BYTES * (kp.has_residual ? 2 : 1) +
+                      8 * (2 * MAX_STAGES + 5 + 2 * EPI_WARPS);
   int stages = (S.max_smem_optin - reserve - 64 /*static smem*/) / stage_bytes;
   if (stages > MAX_STAGES) stages = MAX_STAGES;
   if (stages < 2) {
@@ -343,35 +413,95 @@ conv3d_status_t launch_main(DeviceState& S, int dev, const Problem& P, const voi
   }
   kp.stages = stages;
   kp.tmem_cols = pow2_at_least(2u * kp.BN);
-  kp.idesc = idesc_f16(kBF16, BM, kp.BN);
-  kp.bias = bias;
-  kp.residual = residual;
-  kp.y = y;
-  kp.status = S.status;
+  kp.idesc = idesc_f16(bf16, ctas * BM, kp.BN);  // swapped: M = 128 channels, N = 256 pixels
   kp.timeout_ns = kDefaultTimeoutNs;
-  const size_t smem = static_cast<size_t>(stages) * stage_bytes + reserve;
+  L.smem = static_cast<size_t>(stages) * stage_bytes + reserve;
+  return CONV3D_OK;
+}
 
-  CUtensorMap map_a, map_b;
-  conv3d_status_t st = encode_maps(P, x, wmat, kt_eff, kp.BN, map_a, map_b);
-  if (st != CONV3D_OK) return st;
-
-  auto kern = conv3d_implicit_gemm_kernel<kBF16>;
+template <bool kBF16, bool kPair, bool kSwap>
+conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtensorMap& map_a,
+                              const CUtensorMap& map_b, const CUtensorMap& map_y,
+                              const CUtensorMap& map_r, cudaStream_t stream) {
+  auto kern = conv3d_implicit_gemm_kernel<kBF16, kPair, kSwap>;
+  const int variant = (kBF16 ? 1 : 0) + (kPair ? 2 : 0) + (kSwap ? 4 : 0);
   cudaError_t e;
+  int units = S.num_sms;  // co-resident CTAs (or CTA pairs)
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!S.attr_set[kBF16 ? 1 : 0]) {
+    if (!S.attr_set[variant]) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                S.max_smem_optin - 64);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-      S.attr_set[kBF16 ? 1 : 0] = true;
+      S.attr_set[variant] = true;
+    }
+    if (kPair) {
+      if (S.pair_clusters <= 0) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (S.num_sms / 2), 1, 1);
+        cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = S.max_smem_optin - 64;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+        if (e != cudaSuccess || clusters < 1) clusters = S.num_sms / 2;
+        S.pair_clusters = clusters;
+      }
+      units = S.pair_clusters;
     }
   }
-  const int grid = kp.num_tiles < S.num_sms ? kp.num_tiles : S.num_sms;
-  kern<<<grid, NUM_THREADS, smem, stream>>>(map_a, map_b, kp);
+  const int unit_count = L.kp.num_tiles < units ? L.kp.num_tiles : units;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kPair ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((kPair ? 2 : 1) * unit_count, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = L.smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = kPair ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, kern, map_a, map_b, map_y, map_r, L.kp);
+  if (e != cudaSuccess) return cuda_fail(e, "conv3d kernel launch");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "conv3d kernel launch");
-  (void)dev;
   return CONV3D_OK;
+}
+
+conv3d_status_t launch_main(DeviceState& S, const Problem& P, const void* x, const void* wmat,
+                            const void* bias, const void* residual, void* y, cudaStream_t stream) {
+  const bool bf16 = P.dtype == CONV3D_BF16;
+  LaunchPlan L;
+  conv3d_status_t st = plan_launch(S, P, bf16, L);
+  if (st != CONV3D_OK) return st;
+  L.kp.bias = bias;
+  L.kp.status = S.status;
+  CUtensorMap map_a, map_b, map_y, map_r;
+  st = L.swap ? encode_maps(P, x, wmat, L.kp.kt, L.kp.co_tile, L.kp.pix_tile, map_a, map_b)
+              : encode_maps(P, x, wmat, L.kp.kt, L.kp.BN / (L.pair ? 2 : 1), BM, map_a, map_b);
+  if (st != CONV3D_OK) return st;
+  if ((st = encode_out_map(P, y, map_y)) != CONV3D_OK) return st;
+  if (residual) {
+    if ((st = encode_out_map(P, residual, map_r)) != CONV3D_OK) return st;
+  } else {
+    map_r = map_y;  // never read: has_residual == 0
+  }
+  if (L.swap)
+    return bf16 ? launch_kernel<true, false, true>(S, L, map_a, map_b, map_y, map_r, stream)
+                : launch_kernel<false, false, true>(S, L, map_a, map_b, map_y, map_r, stream);
+  if (bf16)
+    return L.pair ? launch_kernel<true, true, false>(S, L, map_a, map_b, map_y, map_r, stream)
+                  : launch_kernel<true, false, false>(S, L, map_a, map_b, map_y, map_r, stream);
+  return L.pair ? launch_kernel<false, true, false>(S, L, map_a, map_b, map_y, map_r, stream)
+                : launch_kernel<false, false, false>(S, L, map_a, map_b, map_y, map_r, stream);
 }
 
 conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* bias,
@@ -425,8 +555,8 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
     if (e != cudaSuccess) return cuda_fail(e, "fold kernel launch");
     wmat = ws;
   }
-  return bf16 ? launch_main<true>(*S, dev, P, x, wmat, bias, residual, y, stream)
-              : launch_main<false>(*S, dev, P, x, wmat, bias, residual, y, stream);
+  (void)dev;
+  return launch_main(*S, P, x, wmat, bias, residual, y, stream);
 }
 
 // ------------------------------------------------------------------ allocation-free entry

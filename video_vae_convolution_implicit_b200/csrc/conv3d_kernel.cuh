@@ -12,8 +12,9 @@
 // replicate padding; the tap is skipped when it reads zero padding), so no
 // padded copy of the input is ever written.
 //
-// One CTA per SM, persistent over output tiles of BM = 128 pixels x BN output
-// channels.  Warp roles (192 threads):
+// One CTA per SM, persistent over output tiles of 128 pixels x BN output
+// channels (or a CTA pair over 256-pixel tiles, see below).  Warp roles
+// (192 threads):
 //   warp 0     TMA producer: per k-block one im2col load of A (128 pixels x 64
 //              channels of one tap) and one tiled load of B (BN x 64), both
 //              128-byte swizzled, into a ring of `stages` shared-memory slots
@@ -51,19 +52,33 @@ struct KernelParams {
   int pf, ph, pw;                    // front temporal pad, spatial pads
   int tpad;                          // 0 zero, 1 causal replicate, 2 causal zero
   int n_chunks;                      // ceil(Cin / BK)
-  int BN;                            // output channels per tile (multiple of 32, <= 256)
-  int n_tiles_n;                     // ceil(Cout / BN)
-  int tiles_per_frame;               // ceil(HoWo / BM)
+  int BN;                            // MMA N: channels per tile, or 256 pixels (swapped)
+  int co_tile;                       // output channels per tile
+  int pix_tile;                      // output pixels per tile (128, or 256 for a CTA pair / swapped)
+  int n_tiles_n;                     // ceil(Cout / co_tile)
+  int tiles_per_frame;               // ceil(HoWo / pix_tile)
   int num_tiles;
   int stages;
   uint32_t tmem_cols;                // power of two >= 2*BN
   uint32_t idesc;
   const void* bias;                  // [Cout] or null
-  const void* residual;              // [M, Cout] or null
-  void* y;                           // [M, Cout]
+  int has_residual;                  // residual is read through map_r
   int* status;                       // device status word
   unsigned long long timeout_ns;
 };
+
+// Epilogue staging: each epilogue warp owns two 32-row x 32-channel buffers
+// (64-byte rows, 64-byte swizzle) for y and, with a residual, two more.
+constexpr int EPI_WARPS = 4;
+constexpr int EPI_BUF_BYTES = 32 * 32 * 2;
+constexpr int EPI_Y_BYTES = EPI_WARPS * 2 * EPI_BUF_BYTES;
+
+// Byte offset of 16-byte chunk c of row r in a 32 x 64-byte buffer written or
+// read by TMA with the 64-byte swizzle (chunk index XOR bits 7-8 of the row
+// offset).
+__device__ __forceinline__ uint32_t swz64(uint32_t r, uint32_t c) {
+  return r * 64u + ((c ^ ((r >> 1) & 3u)) << 4);
+}
 
 struct Tile {
   int frame_out;  // n*Do + to
@@ -77,10 +92,10 @@ __device__ __forceinline__ Tile decode_tile(const KernelParams& p, int t) {
   const int nt = t % p.n_tiles_n;
   const int mt = t / p.n_tiles_n;
   r.frame_out = mt / p.tiles_per_frame;
-  r.p0 = (mt - r.frame_out * p.tiles_per_frame) * BM;
+  r.p0 = (mt - r.frame_out * p.tiles_per_frame) * p.pix_tile;
   r.n = r.frame_out / p.Do;
   r.to = r.frame_out - r.n * p.Do;
-  r.co0 = nt * p.BN;
+  r.co0 = nt * p.co_tile;
   return r;
 }
 
@@ -155,31 +170,55 @@ struct Cvt<false> {
   }
 };
 
-template <bool kBF16>
+// kPair = false: one CTA per tile of 128 pixels x BN channels (cta_group::1).
+// kPair = true:  a cluster of two CTAs per tile of 256 pixels x BN channels
+//   (cta_group::2, M = 256): CTA r loads the A rows [128r, 128r+128) of the
+//   tile and the B rows [BN/2 r, BN/2 (r+1)) into its own shared memory, both
+//   loads signalling the even CTA's full barrier; the even CTA issues the MMAs
+//   and commits them to the stage and accumulator barriers of both CTAs; each
+//   CTA's epilogue drains its own TMEM (its 128 rows) and releases the
+//   accumulator on the even CTA's barrier.  No load is shared between the CTAs.
+// kSwap = true (one CTA): the transposed product Y^T = W * A^T, so that layers
+//   with few output channels still issue full-width MMAs: M = 128 output
+//   channels (the weight tile is the A operand), N = 256 output pixels (the
+//   im2col tile is the B operand).  TMEM lane = channel, column = pixel; the
+//   epilogue transposes through shared memory before the TMA store.
+template <bool kBF16, bool kPair, bool kSwap>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     conv3d_implicit_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                                 const __grid_constant__ CUtensorMap map_b,
+                                const __grid_constant__ CUtensorMap map_y,
+                                const __grid_constant__ CUtensorMap map_r,
                                 const KernelParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
   __shared__ int s_abort;
 
+  constexpr int kCtas = kPair ? 2 : 1;
   const uint32_t warp = threadIdx.x / 32;
   const uint32_t lane = threadIdx.x % 32;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0;
+  const bool leader = rank == 0;
+  const int unit = blockIdx.x / kCtas;        // this CTA's cluster (or CTA) index
+  const int num_units = gridDim.x / kCtas;
 
   // Carve shared memory: A ring, B ring (both 1024-byte aligned for the
   // 128-byte swizzle), then the mbarriers.
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t b_stage_bytes = static_cast<uint32_t>(p.BN) * BK * 2;
+  const uint32_t b_rows = static_cast<uint32_t>(p.BN) / kCtas;
+  const uint32_t b_stage_bytes = b_rows * BK * 2;
   const uint32_t a_ring = base;
   const uint32_t b_ring = a_ring + p.stages * A_STAGE_BYTES;
-  const uint32_t bars = b_ring + p.stages * b_stage_bytes;
+  const uint32_t y_stage = b_ring + p.stages * b_stage_bytes;        // [EPI_WARPS][2] buffers
+  const uint32_t r_stage = y_stage + EPI_Y_BYTES;                     // same, with a residual
+  const uint32_t bars = r_stage + (p.has_residual ? EPI_Y_BYTES : 0);
   const uint32_t full_bar = bars;                         // [stages]
   const uint32_t empty_bar = bars + 8 * p.stages;         // [stages]
   const uint32_t tfull_bar = bars + 16 * p.stages;        // [2]
   const uint32_t tempty_bar = tfull_bar + 16;             // [2]
   const uint32_t drain_bar = tempty_bar + 16;             // [1]
+  const uint32_t rfull_bar = drain_bar + 8;               // [EPI_WARPS][2]
 
   SharedCtl ctl{&s_abort, p.status, p.timeout_ns};
 
@@ -191,35 +230,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar + 8 * a, 1);
-      mbar_init(tempty_bar + 8 * a, 4);
+      mbar_init(tempty_bar + 8 * a, 4 * kCtas);
     }
     mbar_init(drain_bar, 1);
+    for (int e = 0; e < 2 * EPI_WARPS; ++e) mbar_init(rfull_bar + 8 * e, 1);
     fence_mbar_init();
     prefetch_tensormap(&map_a);
     prefetch_tensormap(&map_b);
+    prefetch_tensormap(&map_y);
+    if (p.has_residual) prefetch_tensormap(&map_r);
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(&s_tmem_base), p.tmem_cols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_addr(&s_tmem_base), p.tmem_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_addr(&s_tmem_base), p.tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();   // the peer's barriers are initialised
   tc_fence_after();
   const uint32_t tmem_base = s_tmem_base;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint32_t tx_bytes = A_STAGE_BYTES + b_stage_bytes;
+      const uint32_t tx_bytes = kCtas * (A_STAGE_BYTES + b_stage_bytes);
       uint32_t stage = 0, phase = 0;
       long long issued = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+      for (int t = unit; ok && t < p.num_tiles; t += num_units) {
         const Tile tl = decode_tile(p, t);
-        const int ho0 = tl.p0 / p.Wo;
-        const int wo0 = tl.p0 - ho0 * p.Wo;
-        const int w_org = wo0 - p.pw;   // window origin of the tile's first pixel
+        // first output pixel of this CTA's rows; rows past the frame are
+        // computed from any valid window origin and masked by the epilogue
+        int row0 = tl.p0 + static_cast<int>(rank) * BM;
+        if (row0 >= p.HoWo) row0 = 0;
+        const int ho0 = row0 / p.Wo;
+        const int wo0 = row0 - ho0 * p.Wo;
+        const int w_org = wo0 - p.pw;   // window origin of the first pixel
         const int h_org = ho0 - p.ph;
+        const int co_b = tl.co0 + static_cast<int>(rank * b_rows);
         for (int it = 0; ok && it < p.kt; ++it) {
           const int f = source_frame(p, tl.to, it);
           if (f < 0) continue;
@@ -232,12 +285,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   ok = false;
                   break;
                 }
-                mbar_arrive_expect_tx(full_bar + 8 * stage, tx_bytes);
-                tma_load_im2col_4d(a_ring + stage * A_STAGE_BYTES, &map_a, full_bar + 8 * stage,
-                                   cc * BK, w_org, h_org, img, static_cast<uint16_t>(iw),
-                                   static_cast<uint16_t>(ih));
-                tma_load_3d(b_ring + stage * b_stage_bytes, &map_b, full_bar + 8 * stage,
-                            cc * BK, tap, tl.co0);
+                const uint32_t fb = full_bar + 8 * stage;
+                if (leader) mbar_arrive_expect_tx(fb, tx_bytes);
+                if constexpr (kSwap) {
+                  // A operand = 128 output channels of w, B operand = 256 pixels
+                  tma_load_3d(a_ring + stage * A_STAGE_BYTES, &map_b, fb, cc * BK, tap, tl.co0);
+                  tma_load_im2col_4d(b_ring + stage * b_stage_bytes, &map_a, fb, cc * BK, w_org,
+                                     h_org, img, static_cast<uint16_t>(iw),
+                                     static_cast<uint16_t>(ih));
+                } else if constexpr (kPair) {
+                  const uint32_t fb_leader = mapa_shared(fb, 0);
+                  tma_load_im2col_4d_pair(a_ring + stage * A_STAGE_BYTES, &map_a, fb_leader,
+                                          cc * BK, w_org, h_org, img, static_cast<uint16_t>(iw),
+                                          static_cast<uint16_t>(ih));
+                  tma_load_3d_pair(b_ring + stage * b_stage_bytes, &map_b, fb_leader, cc * BK,
+                                   tap, co_b);
+                } else {
+                  tma_load_im2col_4d(a_ring + stage * A_STAGE_BYTES, &map_a, fb, cc * BK, w_org,
+                                     h_org, img, static_cast<uint16_t>(iw),
+                                     static_cast<uint16_t>(ih));
+                  tma_load_3d(b_ring + stage * b_stage_bytes, &map_b, fb, cc * BK, tap, co_b);
+                }
                 ++issued;
                 if (++stage == static_cast<uint32_t>(p.stages)) {
                   stage = 0;
@@ -250,21 +318,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok) {
         // Let the copies already in flight land before the CTA may exit.
-        const long long first = issued > p.stages ? issued - p.stages : 0;
-        for (long long i = first; i < issued; ++i) {
-          const uint32_t s = static_cast<uint32_t>(i % p.stages);
-          const uint32_t par = static_cast<uint32_t>((i / p.stages) & 1);
-          wait_bounded(full_bar + 8 * s, par, ctl, false);
+        if (leader) {
+          const long long first = issued > p.stages ? issued - p.stages : 0;
+          for (long long i = first; i < issued; ++i) {
+            const uint32_t s = static_cast<uint32_t>(i % p.stages);
+            const uint32_t par = static_cast<uint32_t>((i / p.stages) & 1);
+            wait_bounded(full_bar + 8 * s, par, ctl, false);
+          }
+        } else {
+          // the odd CTA's copies complete on the even CTA's barriers: give them
+          // time to land (both CTAs stay resident until the final cluster barrier)
+          const uint64_t t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 200000ull) {
+          }
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       int local = 0;
-      for (int t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++local) {
+      for (int t = unit; ok && t < p.num_tiles; t += num_units, ++local) {
         const Tile tl = decode_tile(p, t);
         const int nkb = kblocks_of_tile(p, tl.to);
         const uint32_t acc = local & 1;
@@ -284,87 +360,274 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int k = 0; k < BK / 16; ++k) {
             // +32 bytes along K inside the swizzled 128-byte row = +2 in the
             // descriptor's address field.
-            mma_f16_ss(d_tmem, da + 2 * k, db + 2 * k, p.idesc, (kb | k) != 0);
+            if constexpr (kPair)
+              mma_f16_ss_pair(d_tmem, da + 2 * k, db + 2 * k, p.idesc, (kb | k) != 0);
+            else
+              mma_f16_ss(d_tmem, da + 2 * k, db + 2 * k, p.idesc, (kb | k) != 0);
           }
-          mma_commit(empty_bar + 8 * stage);
+          if constexpr (kPair) {
+            mma_commit_pair(empty_bar + 8 * stage);
+            mma_commit_pair(mapa_shared(empty_bar + 8 * stage, 1));
+          } else {
+            mma_commit(empty_bar + 8 * stage);
+          }
           if (++stage == static_cast<uint32_t>(p.stages)) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        mma_commit(tfull_bar + 8 * acc);
+        if constexpr (kPair) {
+          mma_commit_pair(tfull_bar + 8 * acc);
+          mma_commit_pair(mapa_shared(tfull_bar + 8 * acc, 1));
+        } else {
+          mma_commit(tfull_bar + 8 * acc);
+        }
       }
-      // All tensor-core work of this CTA has finished once the drain fires.
-      mma_commit(drain_bar);
+      // All tensor-core work of this CTA (pair) has finished once the drain fires.
+      if constexpr (kPair)
+        mma_commit_pair(drain_bar);
+      else
+        mma_commit(drain_bar);
       wait_bounded(drain_bar, 0, ctl, false);
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Warp q drains TMEM lanes [32q, 32q+32) = 32 output pixels of the tile,
+    // 32 channels at a time: tcgen05.ld -> + bias + residual (fp32) -> one
+    // rounding -> swizzled shared-memory buffer -> TMA store into y viewed as
+    // [frames][Ho*Wo][Cout], which clips rows past the frame and channels past
+    // Cout.  The residual chunk is fetched by TMA two chunks ahead (the first
+    // two before the accumulator is ready).
     using C = Cvt<kBF16>;
     const uint32_t quarter = warp & 3;            // TMEM lanes [32q, 32q+32)
-    const int row = static_cast<int>(quarter * 32 + lane);
+    const uint32_t ew = warp - 2;                 // epilogue warp index, 0..3
+    const uint32_t ybuf = y_stage + ew * 2 * EPI_BUF_BYTES;
+    const uint32_t rbuf = r_stage + ew * 2 * EPI_BUF_BYTES;
+    const uint32_t rbar = rfull_bar + ew * 16;
+    uint32_t rphase[2] = {0, 0};
+    bool rpending[2] = {false, false};   // a residual copy into buffer b is in flight
     int local = 0;
     const uint4* bias4 = reinterpret_cast<const uint4*>(p.bias);
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
-      const uint32_t acc = local & 1;
-      const uint32_t acc_phase = (local >> 1) & 1;
-      if (!wait_bounded(tfull_bar + 8 * acc, acc_phase, ctl, true)) break;
-      tc_fence_after();
-      const Tile tl = decode_tile(p, t);
-      const bool has_acc = kblocks_of_tile(p, tl.to) > 0;
-      const int pix = tl.p0 + row;
-      const bool row_ok = pix < p.HoWo;
-      const long long m = static_cast<long long>(tl.frame_out) * p.HoWo + pix;
-      const uint32_t t_row = tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.BN);
-      for (int j = 0; j < p.BN / 32; ++j) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + j * 32, r);
-        tmem_ld_wait();
-        const int cb = tl.co0 + j * 32;
-        if (row_ok) {
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int co = cb + g * 8;
-            if (co < p.Cout) {
-              float v[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) v[e] = has_acc ? __uint_as_float(r[g * 8 + e]) : 0.0f;
-              if (bias4 != nullptr) {
-                const uint4 b = __ldg(bias4 + co / 8);
-                v[0] += C::lo(b.x); v[1] += C::hi(b.x); v[2] += C::lo(b.y); v[3] += C::hi(b.y);
-                v[4] += C::lo(b.z); v[5] += C::hi(b.z); v[6] += C::lo(b.w); v[7] += C::hi(b.w);
-              }
-              const long long off = m * p.Cout + co;  // element offset, multiple of 8
-              if (p.residual != nullptr) {
-                const uint4 q = *reinterpret_cast<const uint4*>(
-                    static_cast<const uint16_t*>(p.residual) + off);
-                v[0] += C::lo(q.x); v[1] += C::hi(q.x); v[2] += C::lo(q.y); v[3] += C::hi(q.y);
-                v[4] += C::lo(q.z); v[5] += C::hi(q.z); v[6] += C::lo(q.w); v[7] += C::hi(q.w);
-              }
-              uint4 o;
-              o.x = C::pack(v[0], v[1]);
-              o.y = C::pack(v[2], v[3]);
-              o.z = C::pack(v[4], v[5]);
-              o.w = C::pack(v[6], v[7]);
-              *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.y) + off) = o;
+    const int chunks = p.BN / 32;
+    bool ok = true;
+    if constexpr (kSwap) {
+      // Thread = one output channel (TMEM lane), 32 pixels (columns) per chunk.
+      for (int t = unit; ok && t < p.num_tiles; t += num_units, ++local) {
+        const uint32_t acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        const Tile tl = decode_tile(p, t);
+        const int ch0 = tl.co0 + static_cast<int>(quarter) * 32;   // this warp's channels
+        const bool warp_live = ch0 < p.Cout;
+        int live_chunks = (p.HoWo - tl.p0 + 31) / 32;   // pixel chunks inside the frame
+        if (live_chunks > chunks) live_chunks = chunks;
+        if (!warp_live) live_chunks = 0;
+        const int ch = ch0 + static_cast<int>(lane);
+        float bv = 0.0f;
+        if (p.bias != nullptr && ch < p.Cout)
+          bv = C::lo(static_cast<const uint16_t*>(p.bias)[ch]);
+        const bool use_res = p.has_residual != 0;
+        if (use_res) {
+          for (int j = 0; j < 2 && j < live_chunks; ++j) {
+            if (lane == 0) {
+              mbar_arrive_expect_tx(rbar + 8 * j, EPI_BUF_BYTES);
+              tma_load_3d(rbuf + j * EPI_BUF_BYTES, &map_r, rbar + 8 * j, ch0, tl.p0 + 32 * j,
+                          tl.frame_out);
             }
+            rpending[j] = true;
           }
         }
+        if (!wait_bounded(tfull_bar + 8 * acc, acc_phase, ctl, true)) {
+          ok = false;
+        } else {
+          tc_fence_after();
+          const bool has_acc = kblocks_of_tile(p, tl.to) > 0;
+          const uint32_t t_row =
+              tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.BN);
+          // byte offset of (pixel e, this thread's channel) in a 32 x 32 buffer
+          const uint32_t col_byte = (lane & 7u) * 2u;
+          for (int j = 0; j < live_chunks; ++j) {
+            const uint32_t b = j & 1;
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + j * 32, r);
+            tmem_ld_wait();
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = (has_acc ? __uint_as_float(r[e]) : 0.0f) + bv;
+            if (use_res) {
+              if (!wait_bounded(rbar + 8 * b, rphase[b], ctl, true)) {
+                ok = false;
+                break;
+              }
+              rphase[b] ^= 1;
+              rpending[b] = false;
+              const uint32_t rb = rbuf + b * EPI_BUF_BYTES;
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                uint16_t q;
+                asm volatile("ld.shared.u16 %0, [%1];"
+                             : "=h"(q)
+                             : "r"(rb + swz64(e, lane >> 3) + col_byte)
+                             : "memory");
+                v[e] += C::lo(q);
+              }
+            }
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+            const uint32_t yb = ybuf + b * EPI_BUF_BYTES;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const uint16_t q = static_cast<uint16_t>(C::pack(v[e], 0.0f) & 0xFFFFu);
+              asm volatile("st.shared.u16 [%0], %1;" ::"r"(yb + swz64(e, lane >> 3) + col_byte),
+                           "h"(q)
+                           : "memory");
+            }
+            fence_proxy_async_shared();
+            __syncwarp();
+            const int pix0 = tl.p0 + 32 * j;
+            const bool refill = use_res && j + 2 < live_chunks;
+            if (lane == 0) {
+              tma_store_3d(&map_y, yb, ch0, pix0, tl.frame_out);
+              bulk_commit_group();
+              if (refill) {
+                mbar_arrive_expect_tx(rbar + 8 * b, EPI_BUF_BYTES);
+                tma_load_3d(rbuf + b * EPI_BUF_BYTES, &map_r, rbar + 8 * b, ch0, pix0 + 64,
+                            tl.frame_out);
+              }
+            }
+            if (refill) rpending[b] = true;
+          }
+        }
+        if (!ok && lane == 0) {
+          for (int j = 0; j < 2; ++j)
+            if (rpending[j]) wait_bounded(rbar + 8 * j, rphase[j], ctl, false);
+        }
+        if (!ok) break;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar + 8 * acc);
       }
+    } else
+    for (int t = unit; ok && t < p.num_tiles; t += num_units, ++local) {
+      const uint32_t acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      const Tile tl = decode_tile(p, t);
+      const int row_base = tl.p0 + static_cast<int>(rank) * BM + static_cast<int>(quarter) * 32;
+      const bool rows_live = row_base < p.HoWo;   // some of this warp's rows are in the frame
+      // channel chunks that hold at least one real output channel
+      int live_chunks = (p.Cout - tl.co0 + 31) / 32;
+      if (live_chunks > chunks) live_chunks = chunks;
+      const bool use_res = p.has_residual && rows_live;
+      if (use_res) {
+        for (int j = 0; j < 2 && j < live_chunks; ++j) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(rbar + 8 * j, EPI_BUF_BYTES);
+            tma_load_3d(rbuf + j * EPI_BUF_BYTES, &map_r, rbar + 8 * j, tl.co0 + 32 * j,
+                        row_base, tl.frame_out);
+          }
+          rpending[j] = true;
+        }
+      }
+      if (!wait_bounded(tfull_bar + 8 * acc, acc_phase, ctl, true)) {
+        ok = false;
+      } else {
+        tc_fence_after();
+        const bool has_acc = kblocks_of_tile(p, tl.to) > 0;
+        const uint32_t t_row =
+            tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.BN);
+        for (int j = 0; rows_live && j < live_chunks; ++j) {
+          const uint32_t b = j & 1;
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + j * 32, r);
+          tmem_ld_wait();
+          float v[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = has_acc ? __uint_as_float(r[e]) : 0.0f;
+          const int cb = tl.co0 + j * 32;
+          if (bias4 != nullptr) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              if (cb + 8 * g < p.Cout) {
+                const uint4 q = __ldg(bias4 + cb / 8 + g);
+                v[8 * g + 0] += C::lo(q.x); v[8 * g + 1] += C::hi(q.x);
+                v[8 * g + 2] += C::lo(q.y); v[8 * g + 3] += C::hi(q.y);
+                v[8 * g + 4] += C::lo(q.z); v[8 * g + 5] += C::hi(q.z);
+                v[8 * g + 6] += C::lo(q.w); v[8 * g + 7] += C::hi(q.w);
+              }
+            }
+          }
+          if (use_res) {
+            if (!wait_bounded(rbar + 8 * b, rphase[b], ctl, true)) {
+              ok = false;
+              break;
+            }
+            rphase[b] ^= 1;
+            rpending[b] = false;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const uint4 q = ld_shared_v4(rbuf + b * EPI_BUF_BYTES + swz64(lane, g));
+              v[8 * g + 0] += C::lo(q.x); v[8 * g + 1] += C::hi(q.x);
+              v[8 * g + 2] += C::lo(q.y); v[8 * g + 3] += C::hi(q.y);
+              v[8 * g + 4] += C::lo(q.z); v[8 * g + 5] += C::hi(q.z);
+              v[8 * g + 6] += C::lo(q.w); v[8 * g + 7] += C::hi(q.w);
+            }
+          }
+          // the store issued from this buffer two chunks ago must have read it
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            st_shared_v4(ybuf + b * EPI_BUF_BYTES + swz64(lane, g),
+                         C::pack(v[8 * g + 0], v[8 * g + 1]), C::pack(v[8 * g + 2], v[8 * g + 3]),
+                         C::pack(v[8 * g + 4], v[8 * g + 5]), C::pack(v[8 * g + 6], v[8 * g + 7]));
+          }
+          fence_proxy_async_shared();
+          __syncwarp();
+          // every lane has read residual buffer b: refill it with chunk j+2
+          const bool refill = use_res && j + 2 < live_chunks;
+          if (lane == 0) {
+            tma_store_3d(&map_y, ybuf + b * EPI_BUF_BYTES, cb, row_base, tl.frame_out);
+            bulk_commit_group();
+            if (refill) {
+              mbar_arrive_expect_tx(rbar + 8 * b, EPI_BUF_BYTES);
+              tma_load_3d(rbuf + b * EPI_BUF_BYTES, &map_r, rbar + 8 * b, cb + 64, row_base,
+                          tl.frame_out);
+            }
+          }
+          if (refill) rpending[b] = true;
+        }
+      }
+      if (!ok && lane == 0) {
+        // residual copies of this tile still in flight must land before exit
+        for (int j = 0; j < 2; ++j)
+          if (rpending[j]) wait_bounded(rbar + 8 * j, rphase[j], ctl, false);
+      }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar + 8 * acc);
+      if (lane == 0) {
+        if constexpr (kPair)
+          mbar_arrive_cluster(mapa_shared(tempty_bar + 8 * acc, 0));
+        else
+          mbar_arrive(tempty_bar + 8 * acc);
+      }
     }
+    // y stores must be complete (and their shared-memory sources read) before exit
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
 
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();   // no CTA leaves while its peer may touch it
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, p.tmem_cols);
+    if constexpr (kPair)
+      tmem_dealloc_pair(tmem_base, p.tmem_cols);
+    else
+      tmem_dealloc(tmem_base, p.tmem_cols);
   }
 }
 
