@@ -43,6 +43,9 @@ WORKLOADS = {
                       "bf16 512->256, 33x128x128, causal replicate pad"),
     "cfg5c": Workload("cfg5c", "bf16", 1, 512, 256, 33, 128, 128, (1, 1, 1), (0, 0, 0), 0, 7, False,
                       "bf16 1x1x1 shortcut 512->256, 33x128x128"),
+    "cfg4s": Workload("cfg4s", "bf16", 1, 128, 128, 9, 256, 256, (3, 3, 3), (0, 1, 1), 1, 9, False,
+                      "bf16 128->128, 9x256x256, causal replicate pad (a 9-frame slice of the late "
+                      "decoder stage, small enough for ncu replays)"),
     "cfg5d": Workload("cfg5d", "bf16", 1, 256, 256, 1, 256, 256, (3, 3, 3), (0, 1, 1), 1, 8, False,
                       "bf16 first frame T=1 256->256, 256x256, causal replicate pad (a 2D conv)"),
 }
