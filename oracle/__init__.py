@@ -37,6 +37,7 @@ BF16 = 1
 TPAD_ZERO = 0
 TPAD_CAUSAL_REPLICATE = 1
 TPAD_CAUSAL_ZERO = 2
+TPAD_CAUSAL_CACHED = 3
 
 _lib = None
 
@@ -58,7 +59,7 @@ def _load():
         u16p = ctypes.c_void_p
         lib.oracle_conv3d_f64.restype = ctypes.c_int
         lib.oracle_conv3d_f64.argtypes = (
-            [u16p, u16p, u16p, u16p, ctypes.c_int]
+            [u16p, u16p, u16p, u16p, u16p, ctypes.c_int]
             + [ctypes.c_int] * 16
             + [i64p, ctypes.c_int64, ctypes.c_void_p]
         )
@@ -93,11 +94,13 @@ def output_shape(D, H, W, kernel, stride, pad, tpad):
     return tuple(out)
 
 
-def conv3d(x_bits, w_bits, bias_bits, res_bits, dtype, kernel, stride, pad, tpad, rows=None):
+def conv3d(x_bits, w_bits, bias_bits, res_bits, dtype, kernel, stride, pad, tpad, rows=None,
+           prev_bits=None):
     """fp64 oracle convolution.
 
     x_bits: uint16 [N,D,H,W,Cin]; w_bits: uint16 [Cout,kt,kh,kw,Cin];
-    bias_bits: uint16 [Cout] or None; res_bits: uint16 [N,Do,Ho,Wo,Cout] or None.
+    bias_bits: uint16 [Cout] or None; res_bits: uint16 [N,Do,Ho,Wo,Cout] or None;
+    prev_bits: uint16 [N,kt-1,H,W,Cin], the cached frames before x (mode 3 only).
     rows: optional int64 array of flat output-pixel indices m; when given the
     result is [len(rows), Cout], else [N,Do,Ho,Wo,Cout].  Unrounded float64.
     """
@@ -114,6 +117,13 @@ def conv3d(x_bits, w_bits, bias_bits, res_bits, dtype, kernel, stride, pad, tpad
         raise ValueError("bias shape")
     if r is not None and r.shape != (N, Do, Ho, Wo, Cout):
         raise ValueError("residual shape")
+    pv = None
+    if tpad == TPAD_CAUSAL_CACHED and kt > 1:
+        if prev_bits is None:
+            raise ValueError("the cached mode needs prev")
+        pv = np.ascontiguousarray(prev_bits, dtype=np.uint16)
+        if pv.shape != (N, kt - 1, H, W, Cin):
+            raise ValueError("prev shape")
     if rows is None:
         out = np.empty((N, Do, Ho, Wo, Cout), dtype=np.float64)
         rows_p, n_rows = None, 0
@@ -122,7 +132,7 @@ def conv3d(x_bits, w_bits, bias_bits, res_bits, dtype, kernel, stride, pad, tpad
         out = np.empty((rows.size, Cout), dtype=np.float64)
         rows_p, n_rows = rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), rows.size
     rc = _load().oracle_conv3d_f64(
-        x_bits.ctypes.data, w_bits.ctypes.data,
+        x_bits.ctypes.data, None if pv is None else pv.ctypes.data, w_bits.ctypes.data,
         None if b is None else b.ctypes.data,
         None if r is None else r.ctypes.data,
         dtype, N, Cin, D, H, W, Cout, kt, kh, kw, *stride, *pad, tpad,

@@ -22,7 +22,11 @@
  *   - temporally, mode 1 (causal replicate): pf = kt-1, pb = 0, frames f<0
  *                                            read frame 0;
  *   - temporally, mode 2 (causal zero):      pf = kt-1, pb = 0, frames f<0
- *                                            are 0 (the Wan first-frame rule).
+ *                                            are 0 (the Wan first-frame rule);
+ *   - temporally, mode 3 (causal, cached):   pf = kt-1, pb = 0, frames f<0
+ *                                            are the cached frames of the
+ *                                            previous chunk, prev[n, kt-1+f]
+ *                                            (prev is [N, kt-1, H, W, Cin]).
  * Do = (D + pf + pb - kt)/st + 1, Ho = (H + 2ph - kh)/sh + 1,
  * Wo = (W + 2pw - kw)/sw + 1.
  *
@@ -101,14 +105,16 @@ int oracle_output_shape(int D, int H, int W, int kt, int kh, int kw, int st, int
  * is one sequential sum in the fixed order (it, ih, iw, ci).
  * Returns 0, or -1 on an ill-formed problem.
  */
-int oracle_conv3d_f64(const uint16_t* x, const uint16_t* w, const uint16_t* bias,
-                      const uint16_t* residual, int dtype, int N, int Cin, int D, int H, int W,
-                      int Cout, int kt, int kh, int kw, int st, int sh, int sw, int pt, int ph,
-                      int pw, int tpad_mode, const int64_t* rows, int64_t n_rows, double* y_out) {
+int oracle_conv3d_f64(const uint16_t* x, const uint16_t* prev, const uint16_t* w,
+                      const uint16_t* bias, const uint16_t* residual, int dtype, int N, int Cin,
+                      int D, int H, int W, int Cout, int kt, int kh, int kw, int st, int sh, int sw,
+                      int pt, int ph, int pw, int tpad_mode, const int64_t* rows, int64_t n_rows,
+                      double* y_out) {
   int od[3];
   if (oracle_output_shape(D, H, W, kt, kh, kw, st, sh, sw, pt, ph, pw, tpad_mode, od) != 0)
     return -1;
-  if (tpad_mode < 0 || tpad_mode > 2) return -1;
+  if (tpad_mode < 0 || tpad_mode > 3) return -1;
+  if (tpad_mode == 3 && prev == NULL && kt > 1) return -1;
   const int Do = od[0], Ho = od[1], Wo = od[2];
   const int pf = (tpad_mode == 0) ? pt : kt - 1;
   const int64_t M = (int64_t)N * Do * Ho * Wo;
@@ -127,18 +133,28 @@ int oracle_conv3d_f64(const uint16_t* x, const uint16_t* w, const uint16_t* bias
       double acc = 0.0;
       for (int it = 0; it < kt; ++it) {
         int f = to * st + it - pf;
+        const uint16_t* src = x;          /* frames of x, or of prev   */
+        int64_t src_frames = D;
         if (f < 0) {
-          if (tpad_mode == 1) f = 0;      /* causal replicate: frame 0 */
-          else continue;                  /* zero / causal zero        */
+          if (tpad_mode == 1) {
+            f = 0;                        /* causal replicate: frame 0 */
+          } else if (tpad_mode == 3) {
+            src = prev;                   /* cached previous frames    */
+            src_frames = kt - 1;
+            f = kt - 1 + f;
+          } else {
+            continue;                     /* zero / causal zero        */
+          }
+        } else if (f >= D) {
+          continue;                       /* back padding is zero      */
         }
-        if (f >= D) continue;             /* back padding is zero      */
         for (int ih = 0; ih < kh; ++ih) {
           const int hi = ho * sh + ih - ph;
           if (hi < 0 || hi >= H) continue;
           for (int iw = 0; iw < kw; ++iw) {
             const int wi = wo * sw + iw - pw;
             if (wi < 0 || wi >= W) continue;
-            const uint16_t* xp = x + ((((int64_t)n * D + f) * H + hi) * W + wi) * Cin;
+            const uint16_t* xp = src + ((((int64_t)n * src_frames + f) * H + hi) * W + wi) * Cin;
             const uint16_t* wp = w + ((((int64_t)co * kt + it) * kh + ih) * kw + iw) * Cin;
             for (int ci = 0; ci < Cin; ++ci)
               acc += oracle_decode(wp[ci], dtype) * oracle_decode(xp[ci], dtype);

@@ -383,3 +383,69 @@ def test_rejects_mismatched_shapes():
         oracle.conv3d(xb, wb[:, :, :, :, :3], bb, None, BF16, (3, 3, 3), (1, 1, 1), (1, 1, 1), ZERO)
     with pytest.raises(ValueError):
         oracle.output_shape(2, 3, 3, (3, 3, 3), (1, 1, 1), (0, 0, 0), ZERO)
+
+
+# ---------------------------------------------------------------- cached previous frames (chunked decoding)
+
+CACHED = oracle.TPAD_CAUSAL_CACHED
+
+
+@pytest.mark.parametrize("kt", [2, 3])
+def test_cached_mode_equals_conv_over_explicit_concatenation(kt):
+    """Mode 3 reads prev[n, kt-1+f] for f < 0: the same as a zero-pad-free conv
+    over the clip with the cached frames put in front (checked with torch too)."""
+    N, Cin, D, H, W, Cout = 2, 4, 3, 5, 6, 3
+    k = (kt, 3, 3)
+    xb, wb, bb = rand_problem(N, Cin, D, H, W, Cout, k, seed=41)
+    pb = si.bits(si.tensor((N, kt - 1, H, W, Cin), 41, 4))
+    y = oracle.conv3d(xb, wb, bb, None, BF16, k, (1, 1, 1), (0, 1, 1), CACHED, prev_bits=pb)
+    cat = np.concatenate([pb, xb], axis=1)
+    ref = oracle.conv3d(cat, wb, bb, None, BF16, k, (1, 1, 1), (0, 1, 1), ZERO)
+    assert y.shape == (N, D, H, W, Cout)
+    assert np.array_equal(y, ref)
+    xt = torch.from_numpy(dec(cat)).permute(0, 4, 1, 2, 3)
+    wt = torch.from_numpy(dec(wb)).permute(0, 4, 1, 2, 3)
+    lib = F.conv3d(xt, wt, torch.from_numpy(dec(bb)), padding=(0, 1, 1)).permute(0, 2, 3, 4, 1)
+    np.testing.assert_allclose(y, lib.numpy(), rtol=1e-10, atol=1e-10)
+
+
+@pytest.mark.parametrize("first_mode", [CREP, CZERO])
+def test_chunked_decoding_equals_whole_clip(first_mode):
+    """A clip convolved causally in one piece equals the same clip cut into
+    chunks, the first with the causal rule and each later one with the last
+    kt-1 input frames of its predecessor as cached frames (bitwise: the same
+    terms are summed in the same order)."""
+    N, Cin, D, H, W, Cout = 1, 3, 8, 4, 5, 2
+    k = (3, 3, 3)
+    xb, wb, bb = rand_problem(N, Cin, D, H, W, Cout, k, seed=43)
+    whole = oracle.conv3d(xb, wb, bb, None, BF16, k, (1, 1, 1), (0, 1, 1), first_mode)
+    parts, t0 = [], 0
+    for size in (3, 1, 4):
+        chunk = xb[:, t0:t0 + size]
+        if t0 == 0:
+            parts.append(oracle.conv3d(chunk, wb, bb, None, BF16, k, (1, 1, 1), (0, 1, 1), first_mode))
+        else:
+            prev = xb[:, t0 - 2:t0] if t0 >= 2 else None
+            if prev is None:   # fewer than kt-1 earlier frames: not a case this test builds
+                raise AssertionError
+            parts.append(oracle.conv3d(chunk, wb, bb, None, BF16, k, (1, 1, 1), (0, 1, 1), CACHED,
+                                       prev_bits=prev))
+        t0 += size
+    assert np.array_equal(np.concatenate(parts, axis=1), whole)
+
+
+def test_cached_mode_brute_force():
+    N, Cin, D, H, W, Cout = 2, 3, 4, 5, 5, 4
+    k = (3, 2, 3)
+    xb, wb, bb = rand_problem(N, Cin, D, H, W, Cout, k, seed=47)
+    pb = si.bits(si.tensor((N, 2, H, W, Cin), 47, 4))
+    y = oracle.conv3d(xb, wb, bb, None, BF16, k, (1, 1, 1), (0, 1, 2), CACHED, prev_bits=pb)
+    ref = brute_force(dec(np.concatenate([pb, xb], axis=1)), dec(wb), dec(bb), k, (1, 1, 1),
+                      (0, 1, 2), ZERO)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_cached_mode_requires_prev():
+    xb, wb, bb = rand_problem(1, 4, 2, 3, 3, 2, (3, 3, 3), seed=1)
+    with pytest.raises(ValueError):
+        oracle.conv3d(xb, wb, bb, None, BF16, (3, 3, 3), (1, 1, 1), (0, 1, 1), CACHED)
