@@ -56,6 +56,8 @@ def algorithmic_flops(wl):
     kt, kh, kw = wl.kernel
     if wl.tpad == 1 and wl.D == 1:
         taps_t = Do * 1
+    elif wl.tpad == 3:
+        taps_t = Do * kt          # every tap reads a real (current or cached) frame
     else:
         pf = wl.pad[0] if wl.tpad == 0 else kt - 1
         taps_t = 0
@@ -71,7 +73,7 @@ def algorithmic_flops(wl):
 def algorithmic_bytes(wl):
     """x, w, bias, residual read once; y written once (16-bit elements)."""
     Do, Ho, Wo = out_shape(wl)
-    x = wl.N * wl.D * wl.H * wl.W * wl.Cin
+    x = wl.N * (wl.D + (wl.kernel[0] - 1 if wl.tpad == 3 else 0)) * wl.H * wl.W * wl.Cin
     w = wl.Cout * wl.kernel[0] * wl.kernel[1] * wl.kernel[2] * wl.Cin
     y = wl.N * Do * Ho * Wo * wl.Cout
     return 2.0 * (x + w + wl.Cout + y + (y if wl.residual else 0))
@@ -84,7 +86,7 @@ def describe(wl, world):
         "dtype": wl.dtype, "N_per_gpu": wl.N, "global_batch": wl.N * world,
         "Cin": wl.Cin, "Cout": wl.Cout, "D": wl.D, "H": wl.H, "W": wl.W,
         "kernel": list(wl.kernel), "stride": [1, 1, 1], "pad": list(wl.pad),
-        "temporal_pad": ["zero", "causal_replicate", "causal_zero"][wl.tpad],
+        "temporal_pad": ["zero", "causal_replicate", "causal_zero", "causal_cached"][wl.tpad],
         "residual": wl.residual, "out": [Do, Ho, Wo],
         "gemm": {"M": wl.N * Do * Ho * Wo, "N": wl.Cout,
                  "K": wl.Cin * wl.kernel[0] * wl.kernel[1] * wl.kernel[2]},
@@ -194,7 +196,8 @@ class ClockSampler:
 
 def host_bits(p):
     """16-bit patterns of the problem's tensors on the host (converted once)."""
-    return {k: (None if p[k] is None else si.bits(p[k])) for k in ("x", "w", "bias", "residual")}
+    return {k: (None if p.get(k) is None else si.bits(p[k]))
+            for k in ("x", "w", "bias", "residual", "prev")}
 
 
 def oracle_rows_timed(hb, wl, rows):
@@ -203,7 +206,7 @@ def oracle_rows_timed(hb, wl, rows):
     t0 = time.perf_counter()
     ref = oracle.conv3d(hb["x"], hb["w"], hb["bias"], hb["residual"],
                         oracle.BF16 if wl.dtype == "bf16" else oracle.F16, wl.kernel, (1, 1, 1),
-                        wl.pad, wl.tpad, rows=rows)
+                        wl.pad, wl.tpad, rows=rows, prev_bits=hb["prev"])
     return ref, time.perf_counter() - t0
 
 
@@ -227,10 +230,14 @@ def calibrated_rows(hb, wl, seconds, rng):
     return int(max(16, min(M, seconds / per_row)))
 
 
+def prev_frames(wl):
+    return wl.kernel[0] - 1 if wl.tpad == 3 else 0
+
+
 def host_problem(wl, seed):
     out = out_shape(wl)
     return si.conv3d_problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, out, seed,
-                             TORCH_DTYPE[wl.dtype], True, wl.residual, "cpu")
+                             TORCH_DTYPE[wl.dtype], True, wl.residual, "cpu", prev_frames(wl))
 
 
 def run_reference(args, wl, rank, world):
@@ -300,7 +307,7 @@ def run_ours(args, wl, rank, world, local_rank):
     Do, Ho, Wo = out_shape(wl)
     seed = rank_seed(wl, rank)
     p = si.conv3d_problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, (Do, Ho, Wo), seed,
-                          dt, True, wl.residual, dev)
+                          dt, True, wl.residual, dev, prev_frames(wl))
     y = torch.empty((wl.N, Do, Ho, Wo, wl.Cout), dtype=dt, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
@@ -308,7 +315,7 @@ def run_ours(args, wl, rank, world, local_rank):
 
     def step():
         c3.conv3d_fwd(p["x"], p["w"], p["bias"], p["residual"], y, (1, 1, 1), wl.pad, wl.tpad,
-                      stream=stream)
+                      stream=stream, prev=p["prev"])
 
     launches_per_step = 1 + (1 if (wl.tpad == 1 and wl.D == 1 and wl.kernel[0] > 1) else 0)
     for _ in range(max(3, args.warmup)):
@@ -363,7 +370,10 @@ def run_ours(args, wl, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
         "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms),
-                    "max": max(step_ms)},
+                    "max": max(step_ms),
+                    "quarter_means": [statistics.mean(q) for q in
+                                      (step_ms[i * len(step_ms) // 4:(i + 1) * len(step_ms) // 4]
+                                       for i in range(4)) if q]},
         "region_ms": region0.elapsed_time(region1),
         "device_status": c3.status_string(status),
     }
@@ -384,7 +394,8 @@ def run_ours(args, wl, rank, world, local_rank):
 
 
 def run_e2e(args, wl, p, y, stream, dev, c3, flops):
-    host = {k: (None if p[k] is None else p[k].cpu().pin_memory()) for k in ("x", "w", "bias", "residual")}
+    host = {k: (None if p[k] is None else p[k].cpu().pin_memory())
+            for k in ("x", "w", "bias", "residual", "prev")}
     y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     dbuf = {k: (None if p[k] is None else torch.empty_like(p[k])) for k in host}
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
@@ -396,7 +407,7 @@ def run_e2e(args, wl, p, y, stream, dev, c3, flops):
             if v is not None:
                 dbuf[k].copy_(v, non_blocking=True)
         c3.conv3d_fwd(dbuf["x"], dbuf["w"], dbuf["bias"], dbuf["residual"], y, (1, 1, 1), wl.pad,
-                      wl.tpad, stream=stream)
+                      wl.tpad, stream=stream, prev=dbuf["prev"])
         y_host.copy_(y, non_blocking=True)
 
     for _ in range(2):

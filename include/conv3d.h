@@ -52,7 +52,9 @@ typedef enum { CONV3D_F16 = 0, CONV3D_BF16 = 1 } conv3d_dtype_t;
 typedef enum {
   CONV3D_TPAD_ZERO = 0,             /* pad[0] zero frames in front and behind          */
   CONV3D_TPAD_CAUSAL_REPLICATE = 1, /* kt-1 copies of frame 0 in front, none behind    */
-  CONV3D_TPAD_CAUSAL_ZERO = 2       /* kt-1 zero frames in front, none behind (Wan)    */
+  CONV3D_TPAD_CAUSAL_ZERO = 2,      /* kt-1 zero frames in front, none behind (Wan)    */
+  CONV3D_TPAD_CAUSAL_CACHED = 3     /* kt-1 cached frames of the previous chunk in front
+                                       (conv3d_fwd_cached only), none behind          */
 } conv3d_tpad_t;
 
 typedef enum {
@@ -141,6 +143,31 @@ CONV3D_API conv3d_status_t conv3d_fwd_noalloc(const void* x, const void* w, cons
                                               const int stride[3], const int pad[3],
                                               conv3d_tpad_t tpad, conv3d_dtype_t dtype,
                                               struct CUstream_st* stream);
+
+/*
+ * conv3d_fwd_cached -- one chunk of a causal convolution over a long clip.
+ *
+ * A video-VAE decoder that decodes a long clip chunk by chunk must give each
+ * chunk the frames that precede it as its temporal front padding (Qwen Image
+ * post, "Video VAE": Wan's causal convolutions pad the frames before the first
+ * with zeros; after the first chunk those frames are real).  This entry point
+ * computes conv3d_fwd with temporal rule CONV3D_TPAD_CAUSAL_CACHED: output
+ * frame to reads input frame to + it - (kt-1), and a negative index f reads
+ * prev[n, kt-1+f].  Convolving a clip in chunks -- the first with the causal
+ * replicate or zero rule, each later one with prev = the last kt-1 input
+ * frames of the chunk before it -- gives exactly the whole-clip result.
+ *
+ * prev: device pointer to [N, kt-1, H, W, Cin] of the same dtype (may be NULL
+ * when kt == 1), 16-byte aligned, not overlapping y.  pad[0] must be 0;
+ * Do = D.  Every other argument, the layouts and the error behaviour are
+ * those of conv3d_fwd.  Needs no workspace.
+ */
+CONV3D_API conv3d_status_t conv3d_fwd_cached(const void* x, const void* prev, const void* w,
+                                             const void* bias, const void* residual, void* y,
+                                             int N, int Cin, int D, int H, int W, int Cout,
+                                             const int kernel[3], const int stride[3],
+                                             const int pad[3], conv3d_dtype_t dtype,
+                                             struct CUstream_st* stream);
 
 /* Device scratch bytes conv3d_fwd_ws needs for this problem (0 if none). */
 CONV3D_API size_t conv3d_workspace_bytes(int Cin, int Cout, int D, const int kernel[3], conv3d_tpad_t tpad);

@@ -19,7 +19,7 @@ result does not depend on torch's RNG or its version):
   * value = mean + std * z in float64 -> float32 (round to nearest even) ->
     bf16 / fp16 (round to nearest even).
 
-Tensor streams: x = 0, w = 1, bias = 2, residual = 3.
+Tensor streams: x = 0, w = 1, bias = 2, residual = 3, cached previous frames = 4.
 Distributions (the workloads' recipe): x, residual ~ N(0, 1);
 w ~ N(0, std = 1/sqrt(Cin*kt*kh*kw)); bias ~ N(0, std = 0.1).
 """
@@ -37,6 +37,7 @@ STREAM_X = 0
 STREAM_W = 1
 STREAM_BIAS = 2
 STREAM_RESIDUAL = 3
+STREAM_PREV = 4
 
 
 def _s64(v: int) -> int:
@@ -115,11 +116,13 @@ def _normal_range(seed, stream, start, count, device):
 
 
 def conv3d_problem(N, Cin, D, H, W, Cout, kernel, out_dhw, seed, dtype=torch.bfloat16,
-                   bias=True, residual=False, device="cpu"):
-    """x, w, bias, residual for one convolution, following the workload recipe.
+                   bias=True, residual=False, device="cpu", prev_frames=0):
+    """x, w, bias, residual (and cached previous frames) for one convolution,
+    following the workload recipe.
 
     Returns a dict of torch tensors (NDHWC x, [Cout,kt,kh,kw,Cin] w, [Cout] bias,
-    [N,Do,Ho,Wo,Cout] residual); absent ones are None.
+    [N,Do,Ho,Wo,Cout] residual, [N,prev_frames,H,W,Cin] prev ~ N(0,1)); absent
+    ones are None.
     """
     kt, kh, kw = kernel
     fan_in = Cin * kt * kh * kw
@@ -130,7 +133,10 @@ def conv3d_problem(N, Cin, D, H, W, Cout, kernel, out_dhw, seed, dtype=torch.bfl
     if residual:
         Do, Ho, Wo = out_dhw
         r = tensor((N, Do, Ho, Wo, Cout), seed, STREAM_RESIDUAL, 1.0, dtype, device)
-    return {"x": x, "w": w, "bias": b, "residual": r}
+    pv = None
+    if prev_frames > 0:
+        pv = tensor((N, prev_frames, H, W, Cin), seed, STREAM_PREV, 1.0, dtype, device)
+    return {"x": x, "w": w, "bias": b, "residual": r, "prev": pv}
 
 
 def bits(t: torch.Tensor):

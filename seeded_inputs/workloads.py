@@ -3,7 +3,8 @@
 Data only.  These stand in for the video-VAE decoder layers the pages discuss
 (LTX-2.x and Wan 2.x decoder convolutions); no weights or real latents exist
 here, so every tensor is drawn by ``seeded_inputs.conv3d_problem``.
-Temporal modes: 0 zero, 1 causal replicate-first-frame, 2 causal zero.
+Temporal modes: 0 zero, 1 causal replicate-first-frame, 2 causal zero,
+3 causal with the previous chunk's last kt-1 frames cached in front.
 """
 from __future__ import annotations
 
@@ -33,6 +34,9 @@ WORKLOADS = {
                      "fp16 32->32, 5x32x32, zero pad 1 on all dims (small correctness case)"),
     "cfg2": Workload("cfg2", "bf16", 1, 256, 256, 9, 128, 128, (3, 3, 3), (0, 1, 1), 1, 1, True,
                      "bf16 256->256, 9x128x128, causal replicate pad, fused residual"),
+    "cfg2c": Workload("cfg2c", "bf16", 1, 256, 256, 9, 128, 128, (3, 3, 3), (0, 1, 1), 3, 10, True,
+                      "bf16 256->256, a 9-frame chunk of 128x128 with 2 cached previous frames, "
+                      "fused residual (chunked decoding)"),
     "cfg3": Workload("cfg3", "bf16", 1, 512, 512, 17, 64, 96, (3, 3, 3), (0, 1, 1), 1, 2, False,
                      "bf16 512->512, 17x64x96, causal replicate pad (deep mid-block)"),
     "cfg4": Workload("cfg4", "bf16", 1, 128, 128, 121, 256, 256, (3, 3, 3), (0, 1, 1), 1, 3, False,

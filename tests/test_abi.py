@@ -50,6 +50,7 @@ def test_status_strings():
     (1, 256, 256, (3, 3, 3), (0, 1, 1), c3.TPAD_CAUSAL_ZERO, (1, 256, 256)),
     (33, 128, 128, (1, 1, 1), (0, 0, 0), c3.TPAD_ZERO, (33, 128, 128)),
     (4, 7, 9, (2, 3, 1), (0, 0, 2), c3.TPAD_CAUSAL_REPLICATE, (4, 5, 13)),
+    (3, 16, 16, (3, 3, 3), (0, 1, 1), c3.TPAD_CAUSAL_CACHED, (3, 16, 16)),
 ])
 def test_output_shape(D, H, W, k, pad, tpad, expect):
     assert c3.output_shape(D, H, W, k, (1, 1, 1), pad, tpad) == expect
@@ -99,6 +100,7 @@ def call(**kw):
     (dict(residual=R + 8), Status.ALIGNMENT),
     (dict(y=X + 256), Status.INVALID_ARG),                 # y overlaps x
     (dict(residual=Y + 4096), Status.INVALID_ARG),         # residual partially overlaps y
+    (dict(tpad=c3.TPAD_CAUSAL_CACHED), Status.INVALID_ARG),  # needs conv3d_fwd_cached's prev
 ])
 def test_validation_errors(kw, expect):
     assert call(**kw) == expect
@@ -134,3 +136,30 @@ def test_torch_wrapper_rejects_host_tensors():
     y = torch.zeros(1, 2, 4, 4, 8, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         c3.conv3d_fwd(x, w, None, None, y)
+
+
+P = 0x700000000   # fake cached-frames address
+
+
+def call_cached(**kw):
+    a = dict(x=X, prev=P, w=Wt, bias=B, residual=None, y=Y, N=1, Cin=64, D=4, H=16, W=16, Cout=64,
+             kernel=(3, 3, 3), stride=(1, 1, 1), pad=(0, 1, 1), dtype=c3.BF16, stream=None)
+    a.update(kw)
+    return c3.conv3d_fwd_cached_ptr(**a)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(prev=None), Status.INVALID_ARG),                 # kt > 1 needs the cached frames
+    (dict(prev=P + 8), Status.ALIGNMENT),
+    (dict(prev=Y + 512), Status.INVALID_ARG),              # prev overlaps y
+    (dict(pad=(1, 1, 1)), Status.INVALID_ARG),
+    (dict(stride=(2, 1, 1)), Status.UNSUPPORTED),
+])
+def test_cached_entry_validation(kw, expect):
+    assert call_cached(**kw) == expect
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_cached_entry_without_gpu_reports_cuda_error():
+    assert call_cached() == Status.CUDA
+    assert call_cached(prev=None, kernel=(1, 3, 3)) == Status.CUDA   # kt = 1 needs no prev

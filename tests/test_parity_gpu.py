@@ -17,6 +17,7 @@ from parity import assert_close, oracle_ref, problem, sample_rows
 pytestmark = pytest.mark.gpu
 
 ZERO, CREP, CZERO = c3.TPAD_ZERO, c3.TPAD_CAUSAL_REPLICATE, c3.TPAD_CAUSAL_ZERO
+CACHED = c3.TPAD_CAUSAL_CACHED
 
 
 def run(p, residual_into_y=False, workspace=None):
@@ -27,7 +28,7 @@ def run(p, residual_into_y=False, workspace=None):
         y.copy_(res)
         res = y
     c3.conv3d_fwd(p["x"], p["w"], p["bias"], res, y, (1, 1, 1), p["pad"], p["tpad"],
-                  workspace=workspace)
+                  workspace=workspace, prev=p["prev"])
     assert c3.poll_status() == c3.Status.OK
     return y
 
@@ -56,6 +57,9 @@ SMALL = [
     (1, 64, 2, 8, 8, 64, (3, 3, 3), (3, 1, 1), ZERO, "bf16", True),       # windows fully in padding
     (1, 192, 2, 11, 23, 200, (3, 3, 3), (0, 2, 0), CREP, "f16", True),    # asymmetric pads
     (3, 16, 2, 5, 5, 24, (3, 3, 3), (0, 1, 1), CREP, "bf16", False),
+    (2, 64, 3, 9, 13, 64, (3, 3, 3), (0, 1, 1), CACHED, "bf16", True),    # cached previous frames
+    (1, 128, 1, 20, 19, 128, (3, 3, 3), (0, 1, 1), CACHED, "f16", False), # one-frame chunk
+    (1, 40, 4, 12, 12, 72, (2, 3, 3), (0, 1, 1), CACHED, "bf16", False),
 ]
 
 
@@ -169,3 +173,29 @@ def test_workload_sampled(name, monkeypatch):
     got = y.view(-1, wl.Cout)[torch.from_numpy(rows).cuda()].double().cpu().numpy()
     assert_close(got, ref, name)
     assert torch.isfinite(y).all()
+
+
+@pytest.mark.parametrize("first", [CREP, CZERO])
+def test_chunked_decoding_equals_whole_clip(first, cta_mode):
+    """A clip convolved in one call equals the same clip convolved chunk by
+    chunk (first chunk: the causal rule; later chunks: conv3d_fwd_cached with
+    the previous chunk's last kt-1 input frames), bit for bit: every tile sums
+    the same products in the same order."""
+    N, Cin, D, H, W, Cout = 1, 64, 9, 16, 20, 128
+    p = problem(N, Cin, D, H, W, Cout, (3, 3, 3), (0, 1, 1), first, seed=51, residual=True)
+    whole = run(p)
+    parts, t0 = [], 0
+    for size in (4, 1, 4):
+        sl = slice(t0, t0 + size)
+        x = p["x"][:, sl].contiguous()
+        res = p["residual"][:, sl].contiguous()
+        y = torch.empty((N, size, H, W, Cout), dtype=x.dtype, device="cuda")
+        if t0 == 0:
+            c3.conv3d_fwd(x, p["w"], p["bias"], res, y, (1, 1, 1), (0, 1, 1), first)
+        else:
+            prev = p["x"][:, t0 - 2:t0].contiguous()
+            c3.conv3d_fwd(x, p["w"], p["bias"], res, y, (1, 1, 1), (0, 1, 1), CACHED, prev=prev)
+        assert c3.poll_status() == c3.Status.OK
+        parts.append(y)
+        t0 += size
+    assert torch.equal(torch.cat(parts, dim=1).view(torch.int16), whole.view(torch.int16))

@@ -18,7 +18,8 @@ import os
 import torch
 
 __all__ = [
-    "TPAD_ZERO", "TPAD_CAUSAL_REPLICATE", "TPAD_CAUSAL_ZERO", "F16", "BF16", "Status",
+    "TPAD_ZERO", "TPAD_CAUSAL_REPLICATE", "TPAD_CAUSAL_ZERO", "TPAD_CAUSAL_CACHED", "F16", "BF16",
+    "Status", "conv3d_fwd_cached_ptr",
     "Conv3dError", "lib_path", "conv3d", "conv3d_fwd", "conv3d_fwd_ptr", "conv3d_fwd_ws_ptr",
     "conv3d_fwd_noalloc_ptr",
     "output_shape", "workspace_bytes", "poll_status", "selftest_wait_timeout", "release",
@@ -29,6 +30,7 @@ BF16 = 1
 TPAD_ZERO = 0
 TPAD_CAUSAL_REPLICATE = 1
 TPAD_CAUSAL_ZERO = 2
+TPAD_CAUSAL_CACHED = 3
 
 
 class Status:
@@ -64,6 +66,8 @@ _lib.conv3d_fwd.restype = _c
 _lib.conv3d_fwd.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp]
 _lib.conv3d_fwd_ws.restype = _c
 _lib.conv3d_fwd_ws.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp, ctypes.c_size_t, _vp]
+_lib.conv3d_fwd_cached.restype = _c
+_lib.conv3d_fwd_cached.argtypes = [_vp] * 6 + [_c] * 6 + [_i3] * 3 + [_c, _vp]
 _lib.conv3d_fwd_noalloc.restype = _c
 _lib.conv3d_fwd_noalloc.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp]
 _lib.conv3d_workspace_bytes.restype = ctypes.c_size_t
@@ -149,21 +153,33 @@ def conv3d_fwd_noalloc_ptr(x, w, bias, residual, y, N, Cin, D, H, W, Cout, kerne
                                    _i3(*stride), _i3(*pad), tpad, dtype, stream)
 
 
+def conv3d_fwd_cached_ptr(x, prev, w, bias, residual, y, N, Cin, D, H, W, Cout, kernel, stride,
+                          pad, dtype, stream) -> int:
+    """Raw-pointer call of conv3d_fwd_cached (one chunk of a causal conv whose
+    front padding is the previous chunk's last kt-1 frames).  Returns the status."""
+    return _lib.conv3d_fwd_cached(x, prev, w, bias, residual, y, N, Cin, D, H, W, Cout,
+                                  _i3(*kernel), _i3(*stride), _i3(*pad), dtype, stream)
+
+
 def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
 def conv3d_fwd(x: torch.Tensor, w: torch.Tensor, bias, residual, y: torch.Tensor,
                stride=(1, 1, 1), pad=(0, 1, 1), tpad=TPAD_CAUSAL_REPLICATE, stream=None,
-               workspace: torch.Tensor | None = None) -> torch.Tensor:
+               workspace: torch.Tensor | None = None, prev: torch.Tensor | None = None
+               ) -> torch.Tensor:
     """Enqueue y = conv3d(x, w) + bias + residual on ``stream`` (default: current stream).
 
     x: [N, D, H, W, Cin]; w: [Cout, kt, kh, kw, Cin]; bias: [Cout] or None;
     residual: y's shape or None; y: [N, Do, Ho, Wo, Cout].  All contiguous CUDA
     tensors of one dtype (bf16 or fp16).  With ``workspace`` (a uint8 CUDA
-    tensor) the call goes through conv3d_fwd_ws and never allocates.
+    tensor) the call goes through conv3d_fwd_ws and never allocates.  With
+    tpad=TPAD_CAUSAL_CACHED, ``prev`` ([N, kt-1, H, W, Cin]) holds the frames
+    before x and the call goes through conv3d_fwd_cached.
     """
-    for name, t in (("x", x), ("w", w), ("y", y), ("bias", bias), ("residual", residual)):
+    for name, t in (("x", x), ("w", w), ("y", y), ("bias", bias), ("residual", residual),
+                    ("prev", prev)):
         if t is None:
             continue
         if not t.is_cuda:
@@ -187,7 +203,13 @@ def conv3d_fwd(x: torch.Tensor, w: torch.Tensor, bias, residual, y: torch.Tensor
         raise ValueError("bias must be [Cout]")
     code = _dtype_code(x.dtype)
     s = _stream_handle(stream)
-    if workspace is None:
+    if tpad == TPAD_CAUSAL_CACHED:
+        if prev is not None and tuple(prev.shape) != (N, kt - 1, H, W, Cin):
+            raise ValueError(f"prev must be {(N, kt - 1, H, W, Cin)}")
+        st = conv3d_fwd_cached_ptr(_ptr(x), _ptr(prev), _ptr(w), _ptr(bias), _ptr(residual),
+                                   _ptr(y), N, Cin, D, H, W, Cout, (kt, kh, kw), stride, pad, code,
+                                   s)
+    elif workspace is None:
         st = conv3d_fwd_ptr(_ptr(x), _ptr(w), _ptr(bias), _ptr(residual), _ptr(y), N, Cin, D, H,
                             W, Cout, (kt, kh, kw), stride, pad, tpad, code, s)
     else:
@@ -199,13 +221,13 @@ def conv3d_fwd(x: torch.Tensor, w: torch.Tensor, bias, residual, y: torch.Tensor
 
 
 def conv3d(x: torch.Tensor, w: torch.Tensor, bias=None, residual=None, stride=(1, 1, 1),
-           pad=(0, 1, 1), tpad=TPAD_CAUSAL_REPLICATE, stream=None) -> torch.Tensor:
+           pad=(0, 1, 1), tpad=TPAD_CAUSAL_REPLICATE, stream=None, prev=None) -> torch.Tensor:
     """Allocate y (torch) and run :func:`conv3d_fwd`."""
     N, D, H, W, _ = x.shape
     Cout, kt, kh, kw, _ = w.shape
     out = output_shape(D, H, W, (kt, kh, kw), stride, pad, tpad)
     y = torch.empty((N, *out, Cout), dtype=x.dtype, device=x.device)
-    return conv3d_fwd(x, w, bias, residual, y, stride, pad, tpad, stream)
+    return conv3d_fwd(x, w, bias, residual, y, stride, pad, tpad, stream, prev=prev)
 
 
 def poll_status(stream=None) -> int:

@@ -49,6 +49,7 @@ struct Problem {
   conv3d_tpad_t tpad;
   conv3d_dtype_t dtype;
   bool has_residual;
+  const void* prev;  // cached frames before the chunk (CONV3D_TPAD_CAUSAL_CACHED) or null
   bool fold;  // first-frame path: fold the temporal taps into a (hi, lo) pair
 };
 
@@ -82,7 +83,8 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 conv3d_status_t validate(const void* x, const void* w, const void* bias, const void* residual,
                          const void* y, int N, int Cin, int D, int H, int W, int Cout,
                          const int kernel[3], const int stride[3], const int pad[3],
-                         conv3d_tpad_t tpad, conv3d_dtype_t dtype, Problem& P) {
+                         conv3d_tpad_t tpad, conv3d_dtype_t dtype, Problem& P,
+                         const void* prev = nullptr) {
   if (!x || !w || !y || !kernel || !stride || !pad) {
     set_error("x, w, y, kernel, stride and pad must be non-null");
     return CONV3D_ERR_INVALID_ARG;
@@ -96,8 +98,12 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
     return CONV3D_ERR_INVALID_ARG;
   }
   if (tpad != CONV3D_TPAD_ZERO && tpad != CONV3D_TPAD_CAUSAL_REPLICATE &&
-      tpad != CONV3D_TPAD_CAUSAL_ZERO) {
+      tpad != CONV3D_TPAD_CAUSAL_ZERO && tpad != CONV3D_TPAD_CAUSAL_CACHED) {
     set_error("unknown temporal padding mode %d", static_cast<int>(tpad));
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if (tpad == CONV3D_TPAD_CAUSAL_CACHED && kernel && kernel[0] > 1 && !prev) {
+    set_error("the cached-frames mode needs the previous frames (conv3d_fwd_cached)");
     return CONV3D_ERR_INVALID_ARG;
   }
   for (int i = 0; i < 3; ++i) {
@@ -141,7 +147,7 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
     return CONV3D_ERR_UNSUPPORTED;
   }
   if (!aligned16(x) || !aligned16(w) || !aligned16(y) || (bias && !aligned16(bias)) ||
-      (residual && !aligned16(residual))) {
+      (residual && !aligned16(residual)) || (prev && !aligned16(prev))) {
     set_error("tensor pointers must be 16-byte aligned");
     return CONV3D_ERR_ALIGNMENT;
   }
@@ -156,6 +162,11 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
     set_error("residual must be exactly y or not overlap it");
     return CONV3D_ERR_INVALID_ARG;
   }
+  const size_t pb_bytes = static_cast<size_t>(N) * (kernel[0] - 1) * H * W * Cin * 2;
+  if (prev && overlaps(y, yb, prev, pb_bytes)) {
+    set_error("y must not overlap prev");
+    return CONV3D_ERR_INVALID_ARG;
+  }
   P.N = N; P.Cin = Cin; P.D = D; P.H = H; P.W = W; P.Cout = Cout;
   P.kt = kernel[0]; P.kh = kernel[1]; P.kw = kernel[2];
   P.pt = pad[0]; P.ph = pad[1]; P.pw = pad[2];
@@ -164,6 +175,7 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
   P.tpad = tpad;
   P.dtype = dtype;
   P.has_residual = residual != nullptr;
+  P.prev = tpad == CONV3D_TPAD_CAUSAL_CACHED ? prev : nullptr;
   P.fold = (tpad == CONV3D_TPAD_CAUSAL_REPLICATE && D == 1 && kernel[0] > 1);
   return CONV3D_OK;
 }
@@ -252,34 +264,42 @@ conv3d_status_t device_state(DeviceState*& out, int& dev) {
 
 // ------------------------------------------------------------------ tensor maps
 
+// An activation tensor viewed as `images` images of H x W pixels with Cin
+// channels; each load gathers `pixels_per_load` output pixels' windows shifted
+// by one tap (the tap is the load's im2col offset).
+conv3d_status_t encode_im2col(const Problem& P, const void* base, long long images,
+                              int pixels_per_load, CUtensorMap& map) {
+  const CUtensorMapDataType dt =
+      P.dtype == CONV3D_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(P.Cin), static_cast<cuuint64_t>(P.W),
+                              static_cast<cuuint64_t>(P.H), static_cast<cuuint64_t>(images)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(P.Cin) * 2,
+                                 static_cast<cuuint64_t>(P.W) * P.Cin * 2,
+                                 static_cast<cuuint64_t>(P.H) * P.W * P.Cin * 2};
+  // Window-origin box: first origin at -pad, last at dim-1+pad-(k-1).
+  const int lower[2] = {-P.pw, -P.ph};
+  const int upper[2] = {P.pw - (P.kw - 1), P.ph - (P.kh - 1)};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode_im2col(&map, dt, 4, const_cast<void*>(base), dims, strides, lower, upper,
+                               BK, static_cast<cuuint32_t>(pixels_per_load), estr,
+                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeIm2col failed (%d)", static_cast<int>(r));
+    return CONV3D_ERR_CUDA;
+  }
+  return CONV3D_OK;
+}
+
 conv3d_status_t encode_maps(const Problem& P, const void* x, const void* wmat, int kt_eff,
                             int b_box_rows, int pixels_per_load, CUtensorMap& map_a,
                             CUtensorMap& map_b) {
   const CUtensorMapDataType dt =
       P.dtype == CONV3D_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  // A: the input viewed as N*D images of H x W pixels with Cin channels;
-  // each load gathers BM output pixels' windows shifted by one tap.
-  {
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(P.Cin), static_cast<cuuint64_t>(P.W),
-                                static_cast<cuuint64_t>(P.H),
-                                static_cast<cuuint64_t>(P.N) * static_cast<cuuint64_t>(P.D)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(P.Cin) * 2,
-                                   static_cast<cuuint64_t>(P.W) * P.Cin * 2,
-                                   static_cast<cuuint64_t>(P.H) * P.W * P.Cin * 2};
-    // Window-origin box: first origin at -pad, last at dim-1+pad-(k-1).
-    const int lower[2] = {-P.pw, -P.ph};
-    const int upper[2] = {P.pw - (P.kw - 1), P.ph - (P.kh - 1)};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = g_encode_im2col(&map_a, dt, 4, const_cast<void*>(x), dims, strides, lower, upper,
-                                 BK, static_cast<cuuint32_t>(pixels_per_load), estr,
-                                 CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
-      set_error("cuTensorMapEncodeIm2col failed (%d)", static_cast<int>(r));
-      return CONV3D_ERR_CUDA;
-    }
-  }
+  conv3d_status_t st =
+      encode_im2col(P, x, static_cast<long long>(P.N) * P.D, pixels_per_load, map_a);
+  if (st != CONV3D_OK) return st;
   // w viewed as [Cout][taps][Cin]; a box is 64 channels of one tap for
   // b_box_rows output channels (the tile's channels, or half of them for a
   // CTA pair).
@@ -422,7 +442,8 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, L
 template <bool kBF16, bool kPair, bool kSwap>
 conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtensorMap& map_a,
                               const CUtensorMap& map_b, const CUtensorMap& map_y,
-                              const CUtensorMap& map_r, cudaStream_t stream) {
+                              const CUtensorMap& map_r, const CUtensorMap& map_p,
+                              cudaStream_t stream) {
   auto kern = conv3d_implicit_gemm_kernel<kBF16, kPair, kSwap>;
   const int variant = (kBF16 ? 1 : 0) + (kPair ? 2 : 0) + (kSwap ? 4 : 0);
   cudaError_t e;
@@ -469,22 +490,23 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = kPair ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, kern, map_a, map_b, map_y, map_r, L.kp);
+  e = cudaLaunchKernelEx(&cfg, kern, map_a, map_b, map_y, map_r, map_p, L.kp);
   if (e != cudaSuccess) return cuda_fail(e, "conv3d kernel launch");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "conv3d kernel launch");
   return CONV3D_OK;
 }
 
-conv3d_status_t launch_main(DeviceState& S, const Problem& P, const void* x, const void* wmat,
-                            const void* bias, const void* residual, void* y, cudaStream_t stream) {
+conv3d_status_t launch_main(DeviceState& S, const Problem& P, const void* x, const void* prev,
+                            const void* wmat, const void* bias, const void* residual, void* y,
+                            cudaStream_t stream) {
   const bool bf16 = P.dtype == CONV3D_BF16;
   LaunchPlan L;
   conv3d_status_t st = plan_launch(S, P, bf16, L);
   if (st != CONV3D_OK) return st;
   L.kp.bias = bias;
   L.kp.status = S.status;
-  CUtensorMap map_a, map_b, map_y, map_r;
+  CUtensorMap map_a, map_b, map_y, map_r, map_p;
   st = L.swap ? encode_maps(P, x, wmat, L.kp.kt, L.kp.co_tile, L.kp.pix_tile, map_a, map_b)
               : encode_maps(P, x, wmat, L.kp.kt, L.kp.BN / (L.pair ? 2 : 1), BM, map_a, map_b);
   if (st != CONV3D_OK) return st;
@@ -494,14 +516,22 @@ conv3d_status_t launch_main(DeviceState& S, const Problem& P, const void* x, con
   } else {
     map_r = map_y;  // never read: has_residual == 0
   }
+  if (P.tpad == CONV3D_TPAD_CAUSAL_CACHED && P.kt > 1) {
+    // the kt-1 cached frames before the chunk, read for temporal taps before frame 0
+    st = encode_im2col(P, prev, static_cast<long long>(P.N) * (P.kt - 1),
+                       L.swap ? L.kp.pix_tile : BM, map_p);
+    if (st != CONV3D_OK) return st;
+  } else {
+    map_p = map_a;  // never read: no tap reads before frame 0 in this mode
+  }
   if (L.swap)
-    return bf16 ? launch_kernel<true, false, true>(S, L, map_a, map_b, map_y, map_r, stream)
-                : launch_kernel<false, false, true>(S, L, map_a, map_b, map_y, map_r, stream);
+    return bf16 ? launch_kernel<true, false, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream)
+                : launch_kernel<false, false, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
   if (bf16)
-    return L.pair ? launch_kernel<true, true, false>(S, L, map_a, map_b, map_y, map_r, stream)
-                  : launch_kernel<true, false, false>(S, L, map_a, map_b, map_y, map_r, stream);
-  return L.pair ? launch_kernel<false, true, false>(S, L, map_a, map_b, map_y, map_r, stream)
-                : launch_kernel<false, false, false>(S, L, map_a, map_b, map_y, map_r, stream);
+    return L.pair ? launch_kernel<true, true, false>(S, L, map_a, map_b, map_y, map_r, map_p, stream)
+                  : launch_kernel<true, false, false>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+  return L.pair ? launch_kernel<false, true, false>(S, L, map_a, map_b, map_y, map_r, map_p, stream)
+                : launch_kernel<false, false, false>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
 }
 
 conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* bias,
@@ -556,7 +586,7 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
     wmat = ws;
   }
   (void)dev;
-  return launch_main(*S, P, x, wmat, bias, residual, y, stream);
+  return launch_main(*S, P, x, P.prev, wmat, bias, residual, y, stream);
 }
 
 // ------------------------------------------------------------------ allocation-free entry
@@ -677,6 +707,18 @@ conv3d_status_t conv3d_fwd_noalloc(const void* x, const void* w, const void* bia
   return run(P, x, w, bias, residual, y, scratch, kNoallocScratchBytes, false, stream);
 }
 
+conv3d_status_t conv3d_fwd_cached(const void* x, const void* prev, const void* w,
+                                  const void* bias, const void* residual, void* y, int N,
+                                  int Cin, int D, int H, int W, int Cout, const int kernel[3],
+                                  const int stride[3], const int pad[3], conv3d_dtype_t dtype,
+                                  struct CUstream_st* stream) {
+  Problem P;
+  conv3d_status_t st = validate(x, w, bias, residual, y, N, Cin, D, H, W, Cout, kernel, stride,
+                                pad, CONV3D_TPAD_CAUSAL_CACHED, dtype, P, prev);
+  if (st != CONV3D_OK) return st;
+  return run(P, x, w, bias, residual, y, nullptr, 0, false, stream);
+}
+
 size_t conv3d_workspace_bytes(int Cin, int Cout, int D, const int kernel[3], conv3d_tpad_t tpad) {
   if (!kernel || Cin < 1 || Cout < 1 || D < 1) return 0;
   if (tpad == CONV3D_TPAD_CAUSAL_REPLICATE && D == 1 && kernel[0] > 1)
@@ -694,7 +736,8 @@ conv3d_status_t conv3d_output_shape(int D, int H, int W, const int kernel[3], co
   int out[3];
   if (tpad == CONV3D_TPAD_ZERO) {
     pf = pb = pad[0];
-  } else if (tpad == CONV3D_TPAD_CAUSAL_REPLICATE || tpad == CONV3D_TPAD_CAUSAL_ZERO) {
+  } else if (tpad == CONV3D_TPAD_CAUSAL_REPLICATE || tpad == CONV3D_TPAD_CAUSAL_ZERO ||
+             tpad == CONV3D_TPAD_CAUSAL_CACHED) {
     pf = kernel[0] - 1;
     pb = 0;
   } else {

@@ -50,7 +50,7 @@ struct KernelParams {
   int Cin, Cout;
   int kt, kh, kw;
   int pf, ph, pw;                    // front temporal pad, spatial pads
-  int tpad;                          // 0 zero, 1 causal replicate, 2 causal zero
+  int tpad;                          // 0 zero, 1 causal replicate, 2 causal zero, 3 cached
   int n_chunks;                      // ceil(Cin / BK)
   int BN;                            // MMA N: channels per tile, or 256 pixels (swapped)
   int co_tile;                       // output channels per tile
@@ -99,17 +99,24 @@ __device__ __forceinline__ Tile decode_tile(const KernelParams& p, int t) {
   return r;
 }
 
-// Source frame read by temporal tap `it` of output frame `to`, or -1 when the
-// tap reads zero padding (and contributes nothing).
+constexpr int kNoFrame = -0x40000000;
+
+// Source frame read by temporal tap `it` of output frame `to`: a frame of x
+// (>= 0), a cached frame of the previous chunk (-(kt-1) .. -1, cached mode), or
+// kNoFrame when the tap reads zero padding (and contributes nothing).
 __device__ __forceinline__ int source_frame(const KernelParams& p, int to, int it) {
-  int f = to + it - p.pf;
-  if (f < 0) return p.tpad == 1 ? 0 : -1;
-  return f < p.D ? f : -1;
+  const int f = to + it - p.pf;
+  if (f < 0) {
+    if (p.tpad == 1) return 0;      // causal replicate: frame 0
+    if (p.tpad == 3) return f;      // cached frame kt-1+f of the previous chunk
+    return kNoFrame;                // zero padding
+  }
+  return f < p.D ? f : kNoFrame;
 }
 
 __device__ __forceinline__ int kblocks_of_tile(const KernelParams& p, int to) {
   int valid = 0;
-  for (int it = 0; it < p.kt; ++it) valid += source_frame(p, to, it) >= 0;
+  for (int it = 0; it < p.kt; ++it) valid += source_frame(p, to, it) != kNoFrame;
   return valid * p.kh * p.kw * p.n_chunks;
 }
 
@@ -189,6 +196,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                 const __grid_constant__ CUtensorMap map_b,
                                 const __grid_constant__ CUtensorMap map_y,
                                 const __grid_constant__ CUtensorMap map_r,
+                                const __grid_constant__ CUtensorMap map_p,
                                 const KernelParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
@@ -239,6 +247,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefetch_tensormap(&map_b);
     prefetch_tensormap(&map_y);
     if (p.has_residual) prefetch_tensormap(&map_r);
+    if (p.tpad == 3) prefetch_tensormap(&map_p);
   }
   if (warp == 1) {
     if constexpr (kPair) {
@@ -275,8 +284,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int co_b = tl.co0 + static_cast<int>(rank * b_rows);
         for (int it = 0; ok && it < p.kt; ++it) {
           const int f = source_frame(p, tl.to, it);
-          if (f < 0) continue;
-          const int img = tl.n * p.D + f;
+          if (f == kNoFrame) continue;
+          // frames before the chunk come from the cached-frames tensor
+          const CUtensorMap* xmap = f < 0 ? &map_p : &map_a;
+          const int img = f < 0 ? tl.n * (p.kt - 1) + (p.kt - 1) + f : tl.n * p.D + f;
           for (int ih = 0; ok && ih < p.kh; ++ih) {
             for (int iw = 0; ok && iw < p.kw; ++iw) {
               const int tap = (it * p.kh + ih) * p.kw + iw;
@@ -290,18 +301,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if constexpr (kSwap) {
                   // A operand = 128 output channels of w, B operand = 256 pixels
                   tma_load_3d(a_ring + stage * A_STAGE_BYTES, &map_b, fb, cc * BK, tap, tl.co0);
-                  tma_load_im2col_4d(b_ring + stage * b_stage_bytes, &map_a, fb, cc * BK, w_org,
+                  tma_load_im2col_4d(b_ring + stage * b_stage_bytes, xmap, fb, cc * BK, w_org,
                                      h_org, img, static_cast<uint16_t>(iw),
                                      static_cast<uint16_t>(ih));
                 } else if constexpr (kPair) {
                   const uint32_t fb_leader = mapa_shared(fb, 0);
-                  tma_load_im2col_4d_pair(a_ring + stage * A_STAGE_BYTES, &map_a, fb_leader,
+                  tma_load_im2col_4d_pair(a_ring + stage * A_STAGE_BYTES, xmap, fb_leader,
                                           cc * BK, w_org, h_org, img, static_cast<uint16_t>(iw),
                                           static_cast<uint16_t>(ih));
                   tma_load_3d_pair(b_ring + stage * b_stage_bytes, &map_b, fb_leader, cc * BK,
                                    tap, co_b);
                 } else {
-                  tma_load_im2col_4d(a_ring + stage * A_STAGE_BYTES, &map_a, fb, cc * BK, w_org,
+                  tma_load_im2col_4d(a_ring + stage * A_STAGE_BYTES, xmap, fb, cc * BK, w_org,
                                      h_org, img, static_cast<uint16_t>(iw),
                                      static_cast<uint16_t>(ih));
                   tma_load_3d(b_ring + stage * b_stage_bytes, &map_b, fb, cc * BK, tap, co_b);
