@@ -44,8 +44,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def out_shape(wl):
     kt, kh, kw = wl.kernel
     pt, ph, pw = wl.pad
+    st, sh, sw = wl.stride
     pf, pb = (pt, pt) if wl.tpad == 0 else (kt - 1, 0)
-    return (wl.D + pf + pb - kt + 1, wl.H + 2 * ph - kh + 1, wl.W + 2 * pw - kw + 1)
+    return ((wl.D + pf + pb - kt) // st + 1, (wl.H + 2 * ph - kh) // sh + 1,
+            (wl.W + 2 * pw - kw) // sw + 1)
 
 
 def algorithmic_flops(wl):
@@ -63,7 +65,7 @@ def algorithmic_flops(wl):
         taps_t = 0
         for to in range(Do):
             for it in range(kt):
-                f = to + it - pf
+                f = to * wl.stride[0] + it - pf
                 if f < 0 and wl.tpad == 1:
                     f = 0
                 taps_t += 0 <= f < wl.D
@@ -85,7 +87,7 @@ def describe(wl, world):
         "workload": f"conv3d {wl.name}: {wl.note}",
         "dtype": wl.dtype, "N_per_gpu": wl.N, "global_batch": wl.N * world,
         "Cin": wl.Cin, "Cout": wl.Cout, "D": wl.D, "H": wl.H, "W": wl.W,
-        "kernel": list(wl.kernel), "stride": [1, 1, 1], "pad": list(wl.pad),
+        "kernel": list(wl.kernel), "stride": list(wl.stride), "pad": list(wl.pad),
         "temporal_pad": ["zero", "causal_replicate", "causal_zero", "causal_cached"][wl.tpad],
         "residual": wl.residual, "out": [Do, Ho, Wo],
         "gemm": {"M": wl.N * Do * Ho * Wo, "N": wl.Cout,
@@ -205,7 +207,7 @@ def oracle_rows_timed(hb, wl, rows):
     import oracle
     t0 = time.perf_counter()
     ref = oracle.conv3d(hb["x"], hb["w"], hb["bias"], hb["residual"],
-                        oracle.BF16 if wl.dtype == "bf16" else oracle.F16, wl.kernel, (1, 1, 1),
+                        oracle.BF16 if wl.dtype == "bf16" else oracle.F16, wl.kernel, wl.stride,
                         wl.pad, wl.tpad, rows=rows, prev_bits=hb["prev"])
     return ref, time.perf_counter() - t0
 
@@ -314,7 +316,7 @@ def run_ours(args, wl, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        c3.conv3d_fwd(p["x"], p["w"], p["bias"], p["residual"], y, (1, 1, 1), wl.pad, wl.tpad,
+        c3.conv3d_fwd(p["x"], p["w"], p["bias"], p["residual"], y, wl.stride, wl.pad, wl.tpad,
                       stream=stream, prev=p["prev"])
 
     launches_per_step = 1 + (1 if (wl.tpad == 1 and wl.D == 1 and wl.kernel[0] > 1) else 0)
@@ -406,7 +408,7 @@ def run_e2e(args, wl, p, y, stream, dev, c3, flops):
         for k, v in host.items():
             if v is not None:
                 dbuf[k].copy_(v, non_blocking=True)
-        c3.conv3d_fwd(dbuf["x"], dbuf["w"], dbuf["bias"], dbuf["residual"], y, (1, 1, 1), wl.pad,
+        c3.conv3d_fwd(dbuf["x"], dbuf["w"], dbuf["bias"], dbuf["residual"], y, wl.stride, wl.pad,
                       wl.tpad, stream=stream, prev=dbuf["prev"])
         y_host.copy_(y, non_blocking=True)
 

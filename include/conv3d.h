@@ -8,7 +8,8 @@
  * case reduces to a 2D convolution with adjusted weights):
  *
  *   y[n,to,ho,wo,co] = round( bias[co] + residual[n,to,ho,wo,co]
- *       + sum_{it,ih,iw,ci} w[co,it,ih,iw,ci] * Xpad[n, to+it-pf, ho+ih-ph, wo+iw-pw, ci] )
+ *       + sum_{it,ih,iw,ci} w[co,it,ih,iw,ci]
+ *                           * Xpad[n, to*st+it-pf, ho*sh+ih-ph, wo*sw+iw-pw, ci] )
  *
  * computed as the GEMM  M = N*Do*Ho*Wo,  N_gemm = Cout,  K = Cin*kt*kh*kw,
  * with fp16/bf16 operands, fp32 accumulation and one round-to-nearest-even to
@@ -21,8 +22,9 @@
  *   bias     [Cout]                        (optional)
  *   residual [N, Do, Ho, Wo, Cout]         (optional, same type as y)
  *   y        [N, Do, Ho, Wo, Cout]
- *   Do = (D + pf + pb - kt) + 1, Ho = H + 2*ph - kh + 1, Wo = W + 2*pw - kw + 1
- *   (stride 1; pf/pb are the front/back temporal pads of the mode).
+ *   Do = (D + pf + pb - kt)/st + 1, Ho = (H + 2*ph - kh)/sh + 1, Wo = (W + 2*pw - kw)/sw + 1
+ *   (pf/pb are the front/back temporal pads of the mode); output pixel (to, ho, wo)
+ *   reads input frame to*st + it - pf, row ho*sh + ih - ph, column wo*sw + iw - pw.
  *
  * All tensor pointers are DEVICE pointers to caller-owned memory on the
  * current CUDA device; the library never frees them and keeps none after a
@@ -71,8 +73,8 @@ typedef enum {
 /*
  * conv3d_fwd -- y = conv3d(x, w) + bias + residual (see the top of this file).
  *
- * kernel = {kt, kh, kw}, each in [1, 8].  stride = {1, 1, 1} (other strides
- * return CONV3D_ERR_UNSUPPORTED).  pad = {pt, ph, pw}: pt is used by
+ * kernel = {kt, kh, kw}, each in [1, 8].  stride = {st, sh, sw}, each in
+ * [1, 8] (larger returns CONV3D_ERR_UNSUPPORTED).  pad = {pt, ph, pw}: pt is used by
  * CONV3D_TPAD_ZERO only and must be 0 for the causal modes; pt, ph, pw in
  * [0, 127], and the output extents Do, Ho, Wo must be >= 1.
  * Supported set: Cin % 8 == 0, Cout % 8 == 0, 16-byte aligned pointers, y not

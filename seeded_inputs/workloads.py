@@ -27,6 +27,7 @@ class Workload:
     seed: int
     residual: bool
     note: str
+    stride: tuple = (1, 1, 1)
 
 
 WORKLOADS = {
@@ -37,6 +38,9 @@ WORKLOADS = {
     "cfg2c": Workload("cfg2c", "bf16", 1, 256, 256, 9, 128, 128, (3, 3, 3), (0, 1, 1), 3, 10, True,
                       "bf16 256->256, a 9-frame chunk of 128x128 with 2 cached previous frames, "
                       "fused residual (chunked decoding)"),
+    "cfg2s": Workload("cfg2s", "bf16", 1, 256, 256, 9, 256, 256, (3, 3, 3), (0, 1, 1), 1, 11, False,
+                      "bf16 256->256, 9x256x256 -> 9x128x128, stride (1,2,2), causal replicate pad "
+                      "(spatial downsampling, as in video-VAE encoders)", (1, 2, 2)),
     "cfg3": Workload("cfg3", "bf16", 1, 512, 512, 17, 64, 96, (3, 3, 3), (0, 1, 1), 1, 2, False,
                      "bf16 512->512, 17x64x96, causal replicate pad (deep mid-block)"),
     "cfg4": Workload("cfg4", "bf16", 1, 128, 128, 121, 256, 256, (3, 3, 3), (0, 1, 1), 1, 3, False,

@@ -21,13 +21,13 @@ ORACLE_DTYPE = {"bf16": oracle.BF16, "f16": oracle.F16}
 
 
 def problem(N, Cin, D, H, W, Cout, kernel, pad, tpad, seed, dtype="bf16", bias=True,
-            residual=False, device="cuda"):
-    out = oracle.output_shape(D, H, W, kernel, (1, 1, 1), pad, tpad)
+            residual=False, device="cuda", stride=(1, 1, 1)):
+    out = oracle.output_shape(D, H, W, kernel, stride, pad, tpad)
     cached = tpad == oracle.TPAD_CAUSAL_CACHED
     p = si.conv3d_problem(N, Cin, D, H, W, Cout, kernel, out, seed, TORCH_DTYPE[dtype], bias,
                           residual, device, prev_frames=kernel[0] - 1 if cached else 0)
     p.update(dict(N=N, Cin=Cin, D=D, H=H, W=W, Cout=Cout, kernel=tuple(kernel), pad=tuple(pad),
-                  tpad=tpad, dtype=dtype, out=out))
+                  tpad=tpad, dtype=dtype, out=out, stride=tuple(stride)))
     return p
 
 
@@ -36,7 +36,7 @@ def oracle_ref(p, rows=None):
     return oracle.conv3d(si.bits(p["x"]), si.bits(p["w"]),
                          None if p["bias"] is None else si.bits(p["bias"]),
                          None if p["residual"] is None else si.bits(p["residual"]),
-                         ORACLE_DTYPE[p["dtype"]], p["kernel"], (1, 1, 1), p["pad"], p["tpad"],
+                         ORACLE_DTYPE[p["dtype"]], p["kernel"], p["stride"], p["pad"], p["tpad"],
                          rows=rows, prev_bits=None if p["prev"] is None else si.bits(p["prev"]))
 
 

@@ -56,6 +56,20 @@ def test_output_shape(D, H, W, k, pad, tpad, expect):
     assert c3.output_shape(D, H, W, k, (1, 1, 1), pad, tpad) == expect
 
 
+@pytest.mark.parametrize("stride", [(1, 2, 2), (2, 2, 2), (2, 1, 3)])
+def test_output_shape_strided_matches_oracle(stride):
+    import oracle
+    for tpad in (c3.TPAD_ZERO, c3.TPAD_CAUSAL_REPLICATE, c3.TPAD_CAUSAL_ZERO):
+        pad = (1, 1, 1) if tpad == c3.TPAD_ZERO else (0, 1, 1)
+        assert c3.output_shape(9, 17, 20, (3, 3, 3), stride, pad, tpad) == \
+            oracle.output_shape(9, 17, 20, (3, 3, 3), stride, pad, tpad)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_strided_call_passes_validation_without_gpu():
+    assert call(stride=(2, 2, 2)) == Status.CUDA
+
+
 def test_output_shape_rejects_empty():
     with pytest.raises(c3.Conv3dError):
         c3.output_shape(1, 2, 2, (3, 3, 3), (1, 1, 1), (0, 0, 0), c3.TPAD_ZERO)
@@ -90,7 +104,7 @@ def call(**kw):
     (dict(pad=(1, 1, 1)), Status.INVALID_ARG),            # pt must be 0 in causal modes
     (dict(pad=(0, -1, 1), tpad=c3.TPAD_ZERO), Status.INVALID_ARG),
     (dict(H=1, pad=(0, 0, 1)), Status.INVALID_ARG),        # padded input smaller than kernel
-    (dict(stride=(1, 2, 2)), Status.UNSUPPORTED),
+    (dict(stride=(1, 9, 9)), Status.UNSUPPORTED),          # TMA traversal strides are <= 8
     (dict(Cin=12), Status.UNSUPPORTED),
     (dict(Cout=20), Status.UNSUPPORTED),
     (dict(kernel=(3, 9, 3)), Status.UNSUPPORTED),
@@ -153,7 +167,7 @@ def call_cached(**kw):
     (dict(prev=P + 8), Status.ALIGNMENT),
     (dict(prev=Y + 512), Status.INVALID_ARG),              # prev overlaps y
     (dict(pad=(1, 1, 1)), Status.INVALID_ARG),
-    (dict(stride=(2, 1, 1)), Status.UNSUPPORTED),
+    (dict(stride=(9, 1, 1)), Status.UNSUPPORTED),
 ])
 def test_cached_entry_validation(kw, expect):
     assert call_cached(**kw) == expect

@@ -27,7 +27,7 @@ def run(p, residual_into_y=False, workspace=None):
     if residual_into_y:
         y.copy_(res)
         res = y
-    c3.conv3d_fwd(p["x"], p["w"], p["bias"], res, y, (1, 1, 1), p["pad"], p["tpad"],
+    c3.conv3d_fwd(p["x"], p["w"], p["bias"], res, y, p["stride"], p["pad"], p["tpad"],
                   workspace=workspace, prev=p["prev"])
     assert c3.poll_status() == c3.Status.OK
     return y
@@ -36,7 +36,7 @@ def run(p, residual_into_y=False, workspace=None):
 def full_check(p, **kw):
     ref = oracle_ref(p)
     y = run(p, **kw)
-    return assert_close(y.double().cpu().numpy(), ref, str({k: p[k] for k in ("N", "Cin", "Cout", "D", "H", "W", "kernel", "pad", "tpad")}))
+    return assert_close(y.double().cpu().numpy(), ref, str({k: p[k] for k in ("N", "Cin", "Cout", "D", "H", "W", "kernel", "stride", "pad", "tpad")}))
 
 
 # ------------------------------------------------------------------ small, every element
@@ -139,7 +139,7 @@ def test_rejected_call_leaves_y_untouched():
     p = problem(1, 64, 2, 8, 8, 64, (3, 3, 3), (0, 1, 1), CREP, seed=10)
     y = torch.full((1, 2, 8, 8, 64), 7.0, dtype=torch.bfloat16, device="cuda")
     st = c3.conv3d_fwd_ptr(p["x"].data_ptr(), p["w"].data_ptr(), None, None, y.data_ptr(),
-                           1, 64, 2, 8, 8, 64, (3, 3, 3), (1, 2, 2), (0, 1, 1), CREP, c3.BF16, 0)
+                           1, 64, 2, 8, 8, 64, (3, 3, 3), (1, 9, 9), (0, 1, 1), CREP, c3.BF16, 0)
     assert st == c3.Status.UNSUPPORTED
     torch.cuda.synchronize()
     assert (y == 7.0).all()
@@ -158,14 +158,14 @@ def test_bounded_wait_reports_timeout():
 
 # ------------------------------------------------------------------ full-size workloads, sampled
 
-@pytest.mark.parametrize("name", ["cfg1", "cfg2", "cfg3", "cfg4", "cfg5a", "cfg5b", "cfg5c", "cfg5d"])
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
 def test_workload_sampled(name, monkeypatch):
     """Full-size workloads in the launch configuration the bench times (automatic choice)."""
     monkeypatch.delenv("CONV3D_CTA_PAIR", raising=False)
     monkeypatch.delenv("CONV3D_SWAP", raising=False)
     wl = WORKLOADS[name]
     p = problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, wl.pad, wl.tpad, wl.seed,
-                wl.dtype, True, wl.residual)
+                wl.dtype, True, wl.residual, stride=wl.stride)
     y = run(p)
     Do, Ho, Wo = p["out"]
     rows = sample_rows(wl.N, Do, Ho, Wo, n_random=256, seed=wl.seed)
@@ -199,3 +199,28 @@ def test_chunked_decoding_equals_whole_clip(first, cta_mode):
         parts.append(y)
         t0 += size
     assert torch.equal(torch.cat(parts, dim=1).view(torch.int16), whole.view(torch.int16))
+
+
+STRIDED = [
+    # N, Cin, D, H, W, Cout, kernel, stride, pad, tpad, dtype, residual
+    (1, 64, 5, 16, 20, 64, (3, 3, 3), (1, 2, 2), (0, 1, 1), CREP, "bf16", False),   # spatial downsample
+    (1, 128, 9, 18, 17, 128, (3, 3, 3), (2, 2, 2), (0, 1, 1), CREP, "bf16", True),  # causal 2x2x2
+    (2, 64, 6, 12, 12, 96, (3, 3, 3), (2, 1, 1), (1, 1, 1), ZERO, "f16", False),    # temporal only
+    (1, 32, 4, 10, 23, 40, (3, 3, 3), (1, 1, 2), (0, 0, 1), CZERO, "bf16", False),  # width only
+    (1, 64, 3, 15, 15, 64, (1, 3, 3), (1, 3, 3), (0, 1, 1), CREP, "bf16", False),   # stride 3
+    (1, 64, 5, 12, 12, 64, (3, 3, 3), (2, 2, 2), (0, 1, 1), CACHED, "bf16", False), # cached + stride
+    (1, 256, 2, 16, 16, 128, (1, 1, 1), (1, 2, 2), (0, 0, 0), ZERO, "bf16", False), # strided 1x1x1
+]
+
+
+@pytest.mark.parametrize("case", STRIDED, ids=lambda c: f"s{''.join(map(str, c[7]))}-k{''.join(map(str, c[6]))}-t{c[9]}-{c[10]}")
+def test_strided_every_element(case, cta_mode):
+    N, Cin, D, H, W, Cout, k, stride, pad, tpad, dt, res = case
+    p = problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=200 + Cin + Cout, dtype=dt,
+                residual=res, stride=stride)
+    full_check(p)
+
+
+def test_strided_first_frame_fold(cta_mode):
+    p = problem(1, 64, 1, 24, 24, 64, (3, 3, 3), (0, 1, 1), CREP, seed=61, stride=(2, 2, 2))
+    full_check(p)

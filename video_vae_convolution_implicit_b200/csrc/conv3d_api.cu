@@ -44,6 +44,7 @@ struct Problem {
   int N, Cin, D, H, W, Cout;
   int kt, kh, kw;
   int pt, ph, pw;
+  int st, sh, sw;
   int pf, pb;
   int Do, Ho, Wo;
   conv3d_tpad_t tpad;
@@ -53,8 +54,8 @@ struct Problem {
   bool fold;  // first-frame path: fold the temporal taps into a (hi, lo) pair
 };
 
-bool output_extents(int D, int H, int W, const int k[3], const int pad[3], conv3d_tpad_t tpad,
-                    int& pf, int& pb, int out[3]) {
+bool output_extents(int D, int H, int W, const int k[3], const int stride[3], const int pad[3],
+                    conv3d_tpad_t tpad, int& pf, int& pb, int out[3]) {
   if (tpad == CONV3D_TPAD_ZERO) {
     pf = pad[0];
     pb = pad[0];
@@ -66,9 +67,9 @@ bool output_extents(int D, int H, int W, const int k[3], const int pad[3], conv3
   long long nh = static_cast<long long>(H) + 2LL * pad[1] - k[1];
   long long nw = static_cast<long long>(W) + 2LL * pad[2] - k[2];
   if (nd < 0 || nh < 0 || nw < 0) return false;
-  out[0] = static_cast<int>(nd + 1);
-  out[1] = static_cast<int>(nh + 1);
-  out[2] = static_cast<int>(nw + 1);
+  out[0] = static_cast<int>(nd / stride[0] + 1);
+  out[1] = static_cast<int>(nh / stride[1] + 1);
+  out[2] = static_cast<int>(nw / stride[2] + 1);
   return true;
 }
 
@@ -118,12 +119,12 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
   }
   int out[3];
   int pf = 0, pb = 0;
-  if (!output_extents(D, H, W, kernel, pad, tpad, pf, pb, out)) {
+  if (!output_extents(D, H, W, kernel, stride, pad, tpad, pf, pb, out)) {
     set_error("the padded input is smaller than the kernel");
     return CONV3D_ERR_INVALID_ARG;
   }
-  if (stride[0] != 1 || stride[1] != 1 || stride[2] != 1) {
-    set_error("only stride (1,1,1) is supported");
+  if (stride[0] > 8 || stride[1] > 8 || stride[2] > 8) {
+    set_error("strides must be <= 8 (the TMA traversal-stride limit)");
     return CONV3D_ERR_UNSUPPORTED;
   }
   for (int i = 0; i < 3; ++i) {
@@ -170,12 +171,15 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
   P.N = N; P.Cin = Cin; P.D = D; P.H = H; P.W = W; P.Cout = Cout;
   P.kt = kernel[0]; P.kh = kernel[1]; P.kw = kernel[2];
   P.pt = pad[0]; P.ph = pad[1]; P.pw = pad[2];
+  P.st = stride[0]; P.sh = stride[1]; P.sw = stride[2];
   P.pf = pf; P.pb = pb;
   P.Do = out[0]; P.Ho = out[1]; P.Wo = out[2];
   P.tpad = tpad;
   P.dtype = dtype;
   P.has_residual = residual != nullptr;
   P.prev = tpad == CONV3D_TPAD_CAUSAL_CACHED ? prev : nullptr;
+  // a single causal-replicate frame: every temporal tap of the one output
+  // frame reads frame 0 (whatever the temporal stride)
   P.fold = (tpad == CONV3D_TPAD_CAUSAL_REPLICATE && D == 1 && kernel[0] > 1);
   return CONV3D_OK;
 }
@@ -279,7 +283,9 @@ conv3d_status_t encode_im2col(const Problem& P, const void* base, long long imag
   // Window-origin box: first origin at -pad, last at dim-1+pad-(k-1).
   const int lower[2] = {-P.pw, -P.ph};
   const int upper[2] = {P.pw - (P.kw - 1), P.ph - (P.kh - 1)};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  // traversal strides: consecutive output pixels' window origins are sw
+  // columns (sh rows at a row wrap) apart
+  const cuuint32_t estr[4] = {1, static_cast<cuuint32_t>(P.sw), static_cast<cuuint32_t>(P.sh), 1};
   CUresult r = g_encode_im2col(&map, dt, 4, const_cast<void*>(base), dims, strides, lower, upper,
                                BK, static_cast<cuuint32_t>(pixels_per_load), estr,
                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -384,6 +390,9 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, L
   kp.kh = P.kh;
   kp.kw = P.kw;
   kp.pf = P.fold ? 1 : P.pf;
+  kp.st = P.fold ? 1 : P.st;
+  kp.sh = P.sh;
+  kp.sw = P.sw;
   kp.ph = P.ph;
   kp.pw = P.pw;
   kp.tpad = P.fold ? 1 : static_cast<int>(P.tpad);

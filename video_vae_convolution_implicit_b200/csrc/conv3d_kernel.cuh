@@ -50,6 +50,7 @@ struct KernelParams {
   int Cin, Cout;
   int kt, kh, kw;
   int pf, ph, pw;                    // front temporal pad, spatial pads
+  int st, sh, sw;                    // strides
   int tpad;                          // 0 zero, 1 causal replicate, 2 causal zero, 3 cached
   int n_chunks;                      // ceil(Cin / BK)
   int BN;                            // MMA N: channels per tile, or 256 pixels (swapped)
@@ -105,7 +106,7 @@ constexpr int kNoFrame = -0x40000000;
 // (>= 0), a cached frame of the previous chunk (-(kt-1) .. -1, cached mode), or
 // kNoFrame when the tap reads zero padding (and contributes nothing).
 __device__ __forceinline__ int source_frame(const KernelParams& p, int to, int it) {
-  const int f = to + it - p.pf;
+  const int f = to * p.st + it - p.pf;
   if (f < 0) {
     if (p.tpad == 1) return 0;      // causal replicate: frame 0
     if (p.tpad == 3) return f;      // cached frame kt-1+f of the previous chunk
@@ -279,8 +280,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (row0 >= p.HoWo) row0 = 0;
         const int ho0 = row0 / p.Wo;
         const int wo0 = row0 - ho0 * p.Wo;
-        const int w_org = wo0 - p.pw;   // window origin of the first pixel
-        const int h_org = ho0 - p.ph;
+        const int w_org = wo0 * p.sw - p.pw;   // window origin of the first pixel
+        const int h_org = ho0 * p.sh - p.ph;
         const int co_b = tl.co0 + static_cast<int>(rank * b_rows);
         for (int it = 0; ok && it < p.kt; ++it) {
           const int f = source_frame(p, tl.to, it);
