@@ -68,6 +68,9 @@ def _load():
         lib.oracle_decode16.restype = None
         lib.oracle_decode16.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_groupnorm_silu_f64.restype = ctypes.c_int
+        lib.oracle_groupnorm_silu_f64.argtypes = (
+            [u16p, u16p, u16p] + [ctypes.c_int] * 8 + [ctypes.c_double, ctypes.c_int, ctypes.c_void_p])
         _lib = lib
     return _lib
 
@@ -139,4 +142,25 @@ def conv3d(x_bits, w_bits, bias_bits, res_bits, dtype, kernel, stride, pad, tpad
         rows_p, n_rows, out.ctypes.data)
     if rc != 0:
         raise ValueError("oracle rejected the problem")
+    return out
+
+
+def groupnorm_silu(x_bits, gamma_bits, beta_bits, dtype, groups, eps=1e-6, per_frame=False,
+                   silu=True):
+    """fp64 GroupNorm (+ SiLU) of a [N,D,H,W,C] tensor of 16-bit patterns.
+
+    Statistics per (sample, group), or per (sample, frame, group) with
+    per_frame.  gamma/beta: [C] patterns or None.  Returns unrounded float64.
+    """
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    N, D, H, W, C = x_bits.shape
+    g = None if gamma_bits is None else np.ascontiguousarray(gamma_bits, dtype=np.uint16)
+    b = None if beta_bits is None else np.ascontiguousarray(beta_bits, dtype=np.uint16)
+    out = np.empty(x_bits.shape, dtype=np.float64)
+    rc = _load().oracle_groupnorm_silu_f64(
+        x_bits.ctypes.data, None if g is None else g.ctypes.data,
+        None if b is None else b.ctypes.data, dtype, N, D, H, W, C, groups, int(per_frame),
+        float(eps), int(silu), out.ctypes.data)
+    if rc != 0:
+        raise ValueError("channels must be a multiple of groups")
     return out

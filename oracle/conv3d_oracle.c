@@ -176,3 +176,53 @@ int oracle_num_threads(void) { return omp_get_max_threads(); }
 #else
 int oracle_num_threads(void) { return 1; }
 #endif
+
+/*
+ * GroupNorm followed by SiLU, the normalisation and activation in front of
+ * every decoder convolution (stable-diffusion.cpp discussion "Exe Heavy
+ * Metal": a GROUP_NORM kernel; news.bugfactory.tech: a fused GroupNorm + SiLU
+ * kernel).  Standard GroupNorm: for sample n (and, with per_frame, frame d)
+ * and group g (channels [g*C/G, (g+1)*C/G)), over every element of the group:
+ *   mu = mean(x), var = mean((x - mu)^2)       (biased variance, two passes)
+ *   z  = (x - mu) / sqrt(var + eps) * gamma[c] + beta[c]
+ *   y  = z / (1 + exp(-z))                      (SiLU; silu == 0 returns z)
+ * x is [N, D, H, W, C] (16-bit patterns); gamma, beta are [C] (16-bit, may be
+ * NULL for 1 and 0); y is fp64, unrounded.  Returns 0, or -1 if C % G != 0.
+ */
+int oracle_groupnorm_silu_f64(const uint16_t* x, const uint16_t* gamma, const uint16_t* beta,
+                              int dtype, int N, int D, int H, int W, int C, int G,
+                              int per_frame, double eps, int silu, double* y) {
+  if (G <= 0 || C % G != 0) return -1;
+  const int cg = C / G;
+  const int64_t pixels = (int64_t)D * H * W;
+  const int sets = per_frame ? N * D : N;             /* statistic sets per group */
+  const int64_t set_pixels = per_frame ? (int64_t)H * W : pixels;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+  for (int s = 0; s < sets; ++s) {
+    for (int g = 0; g < G; ++g) {
+      const int64_t p0 = (int64_t)s * set_pixels;      /* first pixel of the set */
+      double sum = 0.0;
+      for (int64_t p = 0; p < set_pixels; ++p)
+        for (int j = 0; j < cg; ++j) sum += oracle_decode(x[(p0 + p) * C + g * cg + j], dtype);
+      const double count = (double)set_pixels * cg;
+      const double mu = sum / count;
+      double ss = 0.0;
+      for (int64_t p = 0; p < set_pixels; ++p)
+        for (int j = 0; j < cg; ++j) {
+          const double d = oracle_decode(x[(p0 + p) * C + g * cg + j], dtype) - mu;
+          ss += d * d;
+        }
+      const double rstd = 1.0 / sqrt(ss / count + eps);
+      for (int64_t p = 0; p < set_pixels; ++p)
+        for (int j = 0; j < cg; ++j) {
+          const int c = g * cg + j;
+          const double ga = gamma ? oracle_decode(gamma[c], dtype) : 1.0;
+          const double be = beta ? oracle_decode(beta[c], dtype) : 0.0;
+          const int64_t i = (p0 + p) * C + c;
+          const double z = (oracle_decode(x[i], dtype) - mu) * rstd * ga + be;
+          y[i] = silu ? z / (1.0 + exp(-z)) : z;
+        }
+    }
+  }
+  return 0;
+}
