@@ -31,7 +31,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import seeded_inputs as si  # noqa: E402
-from seeded_inputs.workloads import WORKLOADS  # noqa: E402
+from seeded_inputs.workloads import NORM_WORKLOADS, WORKLOADS  # noqa: E402
 
 METRIC = "conv3d TFLOPS (bf16, video-VAE decoder shapes) and % of B200 dense peak"
 TORCH_DTYPE = {"bf16": torch.bfloat16, "f16": torch.float16}
@@ -465,6 +465,102 @@ def cpu_baseline(wl, p):
             "sample": f"{n} random output pixels (all {wl.Cout} channels) of {M}, {dt:.1f} s"}
 
 
+# ---------------------------------------------------------------- GroupNorm + SiLU workloads
+
+def run_norm(args, wl, rank, world, local_rank):
+    """GroupNorm statistics + fused normalise/SiLU over one activation tensor per
+    step: HBM-bound (x read twice, y written once)."""
+    import oracle
+    import video_vae_convolution_implicit_b200 as c3
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    td = TORCH_DTYPE[wl.dtype]
+    N, D, H, W, C = wl.shape
+    seed = wl.seed + 1000 * rank
+    x = si.tensor(wl.shape, seed, 0, 1.0, td, dev)
+    gamma = (si.tensor((C,), seed, 1, 0.2, torch.float32, dev) + 1.0).to(td)
+    beta = si.tensor((C,), seed, 2, 0.2, td, dev)
+    y = torch.empty_like(x)
+    sets = N * D if wl.per_frame else N
+    stats = torch.empty((sets, wl.groups, 2), dtype=torch.float64, device=dev)
+    flush = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size // 4 + 1024,
+                        dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        c3.groupnorm_stats(x, wl.groups, 1e-6, wl.per_frame, stats, stream)
+        if ev:
+            ev[1].record(stream)
+        c3.groupnorm_silu(x, stats, gamma, beta, y, wl.groups, wl.per_frame, True, stream)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    stats_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    apply_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    my_ms = sum(a + b for a, b in zip(stats_ms, apply_ms))
+    max_ms = max_over_ranks(my_ms, dev)
+    tensor_bytes = x.numel() * x.element_size()
+    step_bytes = 3 * tensor_bytes
+    value = step_bytes * world * args.steps / (max_ms * 1e-3) / 1e9
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["hbm_gbs"])
+    apply_gbs = 2 * tensor_bytes / (statistics.mean(apply_ms) * 1e-3) / 1e9
+    stats_gbs = tensor_bytes / (statistics.mean(stats_ms) * 1e-3) / 1e9
+    line = {
+        "metric": "GroupNorm+SiLU HBM GB/s (x read twice, y written once)", "value": value,
+        "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded SplitMix64 normals)",
+        "config": {"workload": f"{wl.name}: {wl.note}", "shape_ndhwc": list(wl.shape),
+                   "groups": wl.groups, "per_frame": wl.per_frame, "global_batch": N * world,
+                   "l2": "flushed (2x L2 write) between timed steps"},
+        "roofline": {"bound": "hbm", "achieved": apply_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": apply_gbs / peak, "traffic": None,
+                     "peak_source": f"{peak_kind} hbm_gbs", "kernel": "gn_apply_kernel",
+                     "algorithmic_bytes_per_launch": 2 * tensor_bytes,
+                     "stats_kernel_gbs": stats_gbs, "stats_kernel_frac": stats_gbs / peak},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        # parity gate: the oracle on the whole tensor (or on whole frames when the
+        # statistics are per frame)
+        if wl.per_frame:
+            frames = sorted({0, D - 1})
+            xs = x[:, frames].contiguous()
+            got = y[:, frames].double().cpu().numpy()
+        else:
+            xs = x
+            got = y.double().cpu().numpy()
+        ref = oracle.groupnorm_silu(si.bits(xs), si.bits(gamma), si.bits(beta),
+                                    oracle.BF16 if wl.dtype == "bf16" else oracle.F16, wl.groups,
+                                    eps=1e-6, per_frame=wl.per_frame)
+        err = np.abs(got - ref)
+        mr = float(err.max() / np.abs(ref).max())
+        rl = float(err.sum() / np.abs(ref).sum())
+        line["parity"] = {"elements": int(ref.size), "max_err_over_max_ref": mr, "rel_l1": rl,
+                          "ok": bool(np.isfinite(got).all() and mr <= 1e-2 and rl <= 2e-3)}
+        print(json.dumps(line), flush=True)
+    return 0 if rank != 0 or line["parity"]["ok"] else 1
+
+
 # ---------------------------------------------------------------- main
 
 def main():
@@ -472,14 +568,15 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="cfg2", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="cfg2", choices=sorted(WORKLOADS) + sorted(NORM_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    wl = WORKLOADS[args.workload]
+    is_norm = args.workload in NORM_WORKLOADS
+    wl = NORM_WORKLOADS[args.workload] if is_norm else WORKLOADS[args.workload]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -488,6 +585,10 @@ def main():
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
 
     if args.impl == "reference":
+        if is_norm:
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the reference arm times the convolution oracle only"}))
+            return 0
         return run_reference(args, wl, rank, world)
 
     if world > 1:
@@ -496,7 +597,7 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        rc = run_ours(args, wl, rank, world, local_rank)
+        rc = (run_norm if is_norm else run_ours)(args, wl, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

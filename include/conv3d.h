@@ -171,6 +171,35 @@ CONV3D_API conv3d_status_t conv3d_fwd_cached(const void* x, const void* prev, co
                                              const int pad[3], conv3d_dtype_t dtype,
                                              struct CUstream_st* stream);
 
+/*
+ * GroupNorm (+ SiLU): the normalisation and activation in front of each
+ * decoder convolution (stable-diffusion.cpp discussion "Exe Heavy Metal":
+ * GROUP_NORM on the GPU; news.bugfactory.tech: a fused GroupNorm + SiLU
+ * kernel).  x and y are [N, D, H, W, C] (NDHWC), C % 8 == 0, C % groups == 0,
+ * C <= 2048.  A statistic set is one sample (per_frame = 0: all D*H*W pixels)
+ * or one frame of one sample (per_frame = 1: H*W pixels, for causal decoders
+ * whose statistics may not look ahead in time).  stats is a caller-owned
+ * device buffer of sets * groups * 2 doubles (sets = N, or N*D), 8-byte
+ * aligned; tensors are 16-byte aligned.
+ *
+ * conv3d_groupnorm_stats: stats[s][g] = {mean, 1/sqrt(var + eps)} of set s,
+ *   group g (biased variance), from one read of x.  Overwrites stats.
+ * conv3d_groupnorm_silu: y = silu((x - mean) * rstd * gamma[c] + beta[c])
+ *   (apply_silu = 0: without the silu), one read of x and one write of y,
+ *   rounded once to the dtype.  gamma/beta ([C], dtype) may be NULL (1 / 0).
+ *   y may be x (in place) but must not partially overlap it.
+ * Both enqueue on `stream` and return before completion.
+ */
+CONV3D_API conv3d_status_t conv3d_groupnorm_stats(const void* x, int N, int D, int H, int W,
+                                                  int C, int groups, int per_frame, float eps,
+                                                  conv3d_dtype_t dtype, double* stats,
+                                                  struct CUstream_st* stream);
+CONV3D_API conv3d_status_t conv3d_groupnorm_silu(const void* x, const double* stats,
+                                                 const void* gamma, const void* beta, void* y,
+                                                 int N, int D, int H, int W, int C, int groups,
+                                                 int per_frame, int apply_silu,
+                                                 conv3d_dtype_t dtype, struct CUstream_st* stream);
+
 /* Device scratch bytes conv3d_fwd_ws needs for this problem (0 if none). */
 CONV3D_API size_t conv3d_workspace_bytes(int Cin, int Cout, int D, const int kernel[3], conv3d_tpad_t tpad);
 

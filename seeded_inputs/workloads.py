@@ -57,3 +57,23 @@ WORKLOADS = {
     "cfg5d": Workload("cfg5d", "bf16", 1, 256, 256, 1, 256, 256, (3, 3, 3), (0, 1, 1), 1, 8, False,
                       "bf16 first frame T=1 256->256, 256x256, causal replicate pad (a 2D conv)"),
 }
+
+
+@dataclass(frozen=True)
+class NormWorkload:
+    name: str
+    dtype: str
+    shape: tuple        # [N, D, H, W, C]
+    groups: int
+    per_frame: bool
+    seed: int
+    note: str
+
+
+NORM_WORKLOADS = {
+    "gn_cfg2": NormWorkload("gn_cfg2", "bf16", (1, 9, 128, 128, 256), 32, False, 12,
+                            "GroupNorm(32) + SiLU of the 256-channel 9x128x128 activation"),
+    "gn_cfg4": NormWorkload("gn_cfg4", "bf16", (1, 121, 256, 256, 128), 32, True, 13,
+                            "per-frame GroupNorm(32) + SiLU of the 128-channel 121x256x256 "
+                            "activation"),
+}

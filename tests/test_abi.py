@@ -177,3 +177,38 @@ def test_cached_entry_validation(kw, expect):
 def test_cached_entry_without_gpu_reports_cuda_error():
     assert call_cached() == Status.CUDA
     assert call_cached(prev=None, kernel=(1, 3, 3)) == Status.CUDA   # kt = 1 needs no prev
+
+
+# ---------------------------------------------------------------- GroupNorm entry points
+
+ST = 0x800000000   # fake stats address
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(x=None), Status.INVALID_ARG),
+    (dict(C=96, groups=7), Status.INVALID_ARG),            # C % groups
+    (dict(C=12, groups=3), Status.UNSUPPORTED),            # C % 8
+    (dict(x=X + 8), Status.ALIGNMENT),
+    (dict(stats=ST + 4), Status.ALIGNMENT),
+    (dict(stats=None), Status.INVALID_ARG),
+    (dict(eps=-1.0), Status.INVALID_ARG),
+    (dict(dtype=5), Status.INVALID_ARG),
+])
+def test_groupnorm_stats_validation(kw, expect):
+    a = dict(x=X, N=1, D=2, H=4, W=4, C=64, groups=8, per_frame=0, eps=1e-6, dtype=c3.BF16,
+             stats=ST, stream=None)
+    a.update(kw)
+    assert c3.groupnorm_stats_ptr(**a) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(y=None), Status.INVALID_ARG),
+    (dict(y=Y + 2), Status.ALIGNMENT),
+    (dict(gamma=B + 8), Status.ALIGNMENT),
+    (dict(C=64, groups=6), Status.INVALID_ARG),
+])
+def test_groupnorm_silu_validation(kw, expect):
+    a = dict(x=X, stats=ST, gamma=B, beta=None, y=Y, N=1, D=2, H=4, W=4, C=64, groups=8,
+             per_frame=0, apply_silu=1, dtype=c3.BF16, stream=None)
+    a.update(kw)
+    assert c3.groupnorm_silu_ptr(**a) == expect

@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "TPAD_ZERO", "TPAD_CAUSAL_REPLICATE", "TPAD_CAUSAL_ZERO", "TPAD_CAUSAL_CACHED", "F16", "BF16",
-    "Status", "conv3d_fwd_cached_ptr",
+    "Status", "conv3d_fwd_cached_ptr", "groupnorm_stats", "groupnorm_silu",
     "Conv3dError", "lib_path", "conv3d", "conv3d_fwd", "conv3d_fwd_ptr", "conv3d_fwd_ws_ptr",
     "conv3d_fwd_noalloc_ptr",
     "output_shape", "workspace_bytes", "poll_status", "selftest_wait_timeout", "release",
@@ -68,6 +68,10 @@ _lib.conv3d_fwd_ws.restype = _c
 _lib.conv3d_fwd_ws.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp, ctypes.c_size_t, _vp]
 _lib.conv3d_fwd_cached.restype = _c
 _lib.conv3d_fwd_cached.argtypes = [_vp] * 6 + [_c] * 6 + [_i3] * 3 + [_c, _vp]
+_lib.conv3d_groupnorm_stats.restype = _c
+_lib.conv3d_groupnorm_stats.argtypes = [_vp] + [_c] * 7 + [ctypes.c_float, _c, _vp, _vp]
+_lib.conv3d_groupnorm_silu.restype = _c
+_lib.conv3d_groupnorm_silu.argtypes = [_vp] * 5 + [_c] * 8 + [_c, _vp]
 _lib.conv3d_fwd_noalloc.restype = _c
 _lib.conv3d_fwd_noalloc.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp]
 _lib.conv3d_workspace_bytes.restype = ctypes.c_size_t
@@ -242,3 +246,53 @@ def selftest_wait_timeout(timeout_ms: int) -> int:
 
 def release() -> None:
     _lib.conv3d_release()
+
+
+def groupnorm_stats_ptr(x, N, D, H, W, C, groups, per_frame, eps, dtype, stats, stream) -> int:
+    """Raw-pointer call of conv3d_groupnorm_stats; returns the status code."""
+    return _lib.conv3d_groupnorm_stats(x, N, D, H, W, C, groups, int(per_frame), eps, dtype, stats,
+                                       stream)
+
+
+def groupnorm_silu_ptr(x, stats, gamma, beta, y, N, D, H, W, C, groups, per_frame, apply_silu,
+                       dtype, stream) -> int:
+    """Raw-pointer call of conv3d_groupnorm_silu; returns the status code."""
+    return _lib.conv3d_groupnorm_silu(x, stats, gamma, beta, y, N, D, H, W, C, groups,
+                                      int(per_frame), int(apply_silu), dtype, stream)
+
+
+def groupnorm_stats(x: torch.Tensor, groups: int, eps: float = 1e-6, per_frame: bool = False,
+                    stats: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """{mean, 1/sqrt(var+eps)} per (sample [, frame], group) of an NDHWC tensor, as a
+    float64 CUDA tensor [sets, groups, 2] (``stats`` is reused when given)."""
+    if not x.is_cuda or not x.is_contiguous() or x.dim() != 5:
+        raise ValueError("x must be a contiguous CUDA tensor [N, D, H, W, C]")
+    N, D, H, W, C = x.shape
+    sets = N * D if per_frame else N
+    if stats is None:
+        stats = torch.empty((sets, groups, 2), dtype=torch.float64, device=x.device)
+    elif tuple(stats.shape) != (sets, groups, 2) or stats.dtype != torch.float64:
+        raise ValueError(f"stats must be float64 {(sets, groups, 2)}")
+    _check(groupnorm_stats_ptr(x.data_ptr(), N, D, H, W, C, groups, per_frame, eps,
+                               _dtype_code(x.dtype), stats.data_ptr(), _stream_handle(stream)))
+    return stats
+
+
+def groupnorm_silu(x: torch.Tensor, stats: torch.Tensor, gamma=None, beta=None, y=None,
+                   groups: int | None = None, per_frame: bool = False, apply_silu: bool = True,
+                   stream=None) -> torch.Tensor:
+    """y = silu((x - mean) * rstd * gamma + beta) with ``stats`` from groupnorm_stats.
+    ``y`` may be ``x`` (in place); it is allocated when None."""
+    if not x.is_cuda or not x.is_contiguous() or x.dim() != 5:
+        raise ValueError("x must be a contiguous CUDA tensor [N, D, H, W, C]")
+    N, D, H, W, C = x.shape
+    groups = stats.shape[1] if groups is None else groups
+    if y is None:
+        y = torch.empty_like(x)
+    for name, t in (("gamma", gamma), ("beta", beta)):
+        if t is not None and (tuple(t.shape) != (C,) or t.dtype != x.dtype or not t.is_cuda):
+            raise ValueError(f"{name} must be a CUDA [C] tensor of x's dtype")
+    _check(groupnorm_silu_ptr(x.data_ptr(), stats.data_ptr(), _ptr(gamma), _ptr(beta),
+                              y.data_ptr(), N, D, H, W, C, groups, per_frame, apply_silu,
+                              _dtype_code(x.dtype), _stream_handle(stream)))
+    return y
