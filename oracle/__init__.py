@@ -68,6 +68,10 @@ def _load():
         lib.oracle_decode16.restype = None
         lib.oracle_decode16.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_conv3d_backward_f64.restype = ctypes.c_int
+        lib.oracle_conv3d_backward_f64.argtypes = (
+            [u16p, u16p, u16p, ctypes.c_int] + [ctypes.c_int] * 16
+            + [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p])
         lib.oracle_groupnorm_silu_f64.restype = ctypes.c_int
         lib.oracle_groupnorm_silu_f64.argtypes = (
             [u16p, u16p, u16p] + [ctypes.c_int] * 8 + [ctypes.c_double, ctypes.c_int, ctypes.c_void_p])
@@ -164,3 +168,25 @@ def groupnorm_silu(x_bits, gamma_bits, beta_bits, dtype, groups, eps=1e-6, per_f
     if rc != 0:
         raise ValueError("channels must be a multiple of groups")
     return out
+
+
+def conv3d_backward(x_bits, w_bits, dy_bits, dtype, kernel, stride, pad, tpad):
+    """fp64 adjoints of :func:`conv3d` for the upstream gradient ``dy_bits``
+    (y's shape): returns (dx [N,D,H,W,Cin], dw [Cout,kt,kh,kw,Cin], dbias [Cout])."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    w_bits = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    dy_bits = np.ascontiguousarray(dy_bits, dtype=np.uint16)
+    N, D, H, W, Cin = x_bits.shape
+    Cout = w_bits.shape[0]
+    Do, Ho, Wo = output_shape(D, H, W, kernel, stride, pad, tpad)
+    if dy_bits.shape != (N, Do, Ho, Wo, Cout):
+        raise ValueError("dy shape")
+    dx = np.empty(x_bits.shape, dtype=np.float64)
+    dw = np.empty(w_bits.shape, dtype=np.float64)
+    db = np.empty((Cout,), dtype=np.float64)
+    rc = _load().oracle_conv3d_backward_f64(
+        x_bits.ctypes.data, w_bits.ctypes.data, dy_bits.ctypes.data, dtype, N, Cin, D, H, W, Cout,
+        *kernel, *stride, *pad, tpad, dx.ctypes.data, dw.ctypes.data, db.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle rejected the problem")
+    return dx, dw, db

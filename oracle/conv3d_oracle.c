@@ -226,3 +226,65 @@ int oracle_groupnorm_silu_f64(const uint16_t* x, const uint16_t* gamma, const ui
   }
   return 0;
 }
+
+/*
+ * Backward pass of the convolution above (the pages' on-device LoRA/LoCon
+ * fine-tuning trains convolution layers: engineering.drawthings.ai, LoRA
+ * post).  Both are the adjoints of the forward definition, written as the
+ * same loop with the accumulation reversed: every forward product
+ *     w[co,it,ih,iw,ci] * Xpad[n, f, hi, wi, ci]   (f after the padding rule)
+ * that lands in y[n,to,ho,wo,co] sends dy[n,to,ho,wo,co] * w[...] to
+ * dx[n, f, hi, wi, ci] and dy * Xpad[...] to dw[co,it,ih,iw,ci].  Taps that
+ * read zero padding contribute nothing; with causal replicate padding the
+ * frames before the first are frame 0, so their gradient lands on frame 0.
+ *   dx [N,D,H,W,Cin], dw [Cout,kt,kh,kw,Cin], dbias [Cout] = sum of dy.
+ * dy holds 16-bit patterns of y's shape; outputs are fp64 and unrounded.
+ * Serial loops (the scatter into dx would race under threads).
+ */
+int oracle_conv3d_backward_f64(const uint16_t* x, const uint16_t* w, const uint16_t* dy,
+                               int dtype, int N, int Cin, int D, int H, int W, int Cout, int kt,
+                               int kh, int kw, int st, int sh, int sw, int pt, int ph, int pw,
+                               int tpad_mode, double* dx, double* dw, double* dbias) {
+  int od[3];
+  if (tpad_mode < 0 || tpad_mode > 2) return -1;
+  if (oracle_output_shape(D, H, W, kt, kh, kw, st, sh, sw, pt, ph, pw, tpad_mode, od) != 0)
+    return -1;
+  const int Do = od[0], Ho = od[1], Wo = od[2];
+  const int pf = (tpad_mode == 0) ? pt : kt - 1;
+  if (dx) memset(dx, 0, sizeof(double) * (size_t)N * D * H * W * Cin);
+  if (dw) memset(dw, 0, sizeof(double) * (size_t)Cout * kt * kh * kw * Cin);
+  if (dbias) memset(dbias, 0, sizeof(double) * (size_t)Cout);
+  for (int n = 0; n < N; ++n)
+    for (int to = 0; to < Do; ++to)
+      for (int ho = 0; ho < Ho; ++ho)
+        for (int wo = 0; wo < Wo; ++wo) {
+          const int64_t m = (((int64_t)n * Do + to) * Ho + ho) * Wo + wo;
+          for (int co = 0; co < Cout; ++co) {
+            const double g = oracle_decode(dy[m * Cout + co], dtype);
+            if (dbias) dbias[co] += g;
+            for (int it = 0; it < kt; ++it) {
+              int f = to * st + it - pf;
+              if (f < 0) {
+                if (tpad_mode == 1) f = 0;
+                else continue;
+              }
+              if (f >= D) continue;
+              for (int ih = 0; ih < kh; ++ih) {
+                const int hi = ho * sh + ih - ph;
+                if (hi < 0 || hi >= H) continue;
+                for (int iw = 0; iw < kw; ++iw) {
+                  const int wi = wo * sw + iw - pw;
+                  if (wi < 0 || wi >= W) continue;
+                  const int64_t xo = ((((int64_t)n * D + f) * H + hi) * W + wi) * Cin;
+                  const int64_t wo_ = ((((int64_t)co * kt + it) * kh + ih) * kw + iw) * Cin;
+                  for (int ci = 0; ci < Cin; ++ci) {
+                    if (dx) dx[xo + ci] += g * oracle_decode(w[wo_ + ci], dtype);
+                    if (dw) dw[wo_ + ci] += g * oracle_decode(x[xo + ci], dtype);
+                  }
+                }
+              }
+            }
+          }
+        }
+  return 0;
+}

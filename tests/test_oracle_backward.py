@@ -1,0 +1,95 @@
+"""Pins for the oracle's backward pass (dx, dw, dbias of the convolution).
+
+The adjoint identities tie the backward loops to the forward oracle, which is
+pinned separately: for any upstream gradient g,
+    <conv(x, w), g> = <x, dx(g)>,   <conv(x, w), g> = <w, dw(x, g)>,
+    dbias = sum of g over pixels,
+and torch.autograd in float64 (with the padding written as explicit ops)
+checks the same gradients with a library routine.
+"""
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import seeded_inputs as si
+
+BF16 = oracle.BF16
+ZERO, CREP, CZERO = oracle.TPAD_ZERO, oracle.TPAD_CAUSAL_REPLICATE, oracle.TPAD_CAUSAL_ZERO
+
+
+def dec(b):
+    return oracle.decode16(b, BF16)
+
+
+def problem(N, Cin, D, H, W, Cout, k, stride, pad, tpad, seed):
+    fan = Cin * k[0] * k[1] * k[2]
+    xb = si.bits(si.tensor((N, D, H, W, Cin), seed, 0))
+    wb = si.bits(si.tensor((Cout, *k, Cin), seed, 1, fan ** -0.5))
+    out = oracle.output_shape(D, H, W, k, stride, pad, tpad)
+    gb = si.bits(si.tensor((N, *out, Cout), seed, 5))
+    return xb, wb, gb
+
+
+CASES = [
+    ((2, 3, 4, 5, 6, 4), (3, 3, 3), (1, 1, 1), (1, 1, 1), ZERO),
+    ((1, 4, 5, 4, 4, 3), (3, 3, 3), (1, 1, 1), (0, 1, 1), CREP),
+    ((1, 4, 5, 4, 4, 3), (3, 3, 3), (1, 1, 1), (0, 1, 1), CZERO),
+    ((2, 2, 6, 5, 7, 3), (3, 3, 3), (2, 2, 2), (0, 1, 1), CREP),
+    ((1, 3, 3, 6, 6, 2), (2, 3, 1), (1, 2, 1), (0, 0, 2), CZERO),
+    ((1, 5, 2, 3, 3, 4), (1, 1, 1), (1, 1, 1), (0, 0, 0), ZERO),
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_adjoint_identities(case):
+    (N, Cin, D, H, W, Cout), k, stride, pad, tpad = case
+    xb, wb, gb = problem(N, Cin, D, H, W, Cout, k, stride, pad, tpad, seed=3)
+    y = oracle.conv3d(xb, wb, None, None, BF16, k, stride, pad, tpad)
+    dx, dw, db = oracle.conv3d_backward(xb, wb, gb, BF16, k, stride, pad, tpad)
+    g = dec(gb)
+    lhs = float(np.sum(y * g))
+    assert np.isclose(lhs, float(np.sum(dec(xb) * dx)), rtol=1e-12, atol=1e-12)
+    assert np.isclose(lhs, float(np.sum(dec(wb) * dw)), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(db, g.reshape(-1, Cout).sum(axis=0), rtol=1e-12, atol=1e-12)
+
+
+def torch_grads(xd, wd, gd, k, stride, pad, tpad):
+    x = torch.from_numpy(xd).permute(0, 4, 1, 2, 3).requires_grad_(True)
+    w = torch.from_numpy(wd).permute(0, 4, 1, 2, 3).requires_grad_(True)
+    kt = k[0]
+    if tpad == ZERO:
+        xp = F.pad(x, (0, 0, 0, 0, pad[0], pad[0]))
+    elif tpad == CREP:
+        xp = torch.cat([x[:, :, :1]] * (kt - 1) + [x], dim=2)
+    else:
+        xp = F.pad(x, (0, 0, 0, 0, kt - 1, 0))
+    y = F.conv3d(xp, w, stride=stride, padding=(0, pad[1], pad[2]))
+    y.backward(torch.from_numpy(gd).permute(0, 4, 1, 2, 3))
+    return (x.grad.permute(0, 2, 3, 4, 1).numpy(), w.grad.permute(0, 2, 3, 4, 1).numpy())
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_matches_torch_autograd_float64(case):
+    (N, Cin, D, H, W, Cout), k, stride, pad, tpad = case
+    xb, wb, gb = problem(N, Cin, D, H, W, Cout, k, stride, pad, tpad, seed=5)
+    dx, dw, _ = oracle.conv3d_backward(xb, wb, gb, BF16, k, stride, pad, tpad)
+    tdx, tdw = torch_grads(dec(xb), dec(wb), dec(gb), k, stride, pad, tpad)
+    np.testing.assert_allclose(dx, tdx, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(dw, tdw, rtol=1e-10, atol=1e-10)
+
+
+def test_causal_replicate_sends_front_gradients_to_frame_zero():
+    """With causal replicate padding, dx of frame 0 = dx of the explicitly
+    extended clip summed over frame 0 and its kt-1 copies (the adjoint of
+    copying frame 0)."""
+    N, Cin, D, H, W, Cout, k = 1, 3, 4, 4, 5, 2, (3, 3, 3)
+    xb, wb, gb = problem(N, Cin, D, H, W, Cout, k, (1, 1, 1), (0, 1, 1), CREP, seed=7)
+    dx, _, _ = oracle.conv3d_backward(xb, wb, gb, BF16, k, (1, 1, 1), (0, 1, 1), CREP)
+    ext = np.concatenate([xb[:, :1]] * 2 + [xb], axis=1)
+    # the extended clip under zero padding with pt = 0 has the same D output frames
+    assert oracle.output_shape(D + 2, H, W, k, (1, 1, 1), (0, 1, 1), ZERO)[0] == D
+    dxe, _, _ = oracle.conv3d_backward(ext, wb, gb, BF16, k, (1, 1, 1), (0, 1, 1), ZERO)
+    np.testing.assert_allclose(dx[:, 0], dxe[:, :3].sum(axis=1), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dx[:, 1:], dxe[:, 3:], rtol=1e-12, atol=1e-12)
