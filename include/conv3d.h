@@ -200,6 +200,61 @@ CONV3D_API conv3d_status_t conv3d_groupnorm_silu(const void* x, const double* st
                                                  int per_frame, int apply_silu,
                                                  conv3d_dtype_t dtype, struct CUstream_st* stream);
 
+/*
+ * conv3d_bwd_data -- dx, the gradient of the convolution's input (the pages'
+ * on-device fine-tuning trains convolution layers: engineering.drawthings.ai,
+ * LoRA post).  For stride 1 it is itself a convolution, of dy with every tap
+ * of w mirrored and the channel roles exchanged, under the complementary
+ * padding (kh-1-ph, kw-1-pw spatially; kt-1-pf in front temporally); with
+ * causal replicate padding the gradient of the kt-1 virtual frames in front
+ * is added to frame 0.  Runs the forward kernel on dy, after a weight
+ * transform into the workspace.
+ *
+ * Arguments describe the FORWARD problem: dy is [N, Do, Ho, Wo, Cout] (y's
+ * shape), w [Cout, kt, kh, kw, Cin], dx [N, D, H, W, Cin] (written).  Supported:
+ * stride (1,1,1), pads <= kernel extent - 1, temporal rules zero, causal
+ * replicate and causal zero, plus the forward call's channel and alignment
+ * rules.  workspace: device, 256-byte aligned, conv3d_bwd_data_workspace_bytes()
+ * bytes, not overlapping the tensors.  dx must not overlap dy or w.
+ * Errors: CONV3D_ERR_UNSUPPORTED for a stride other than 1, the cached-frames
+ * rule or pads beyond kernel extent - 1; CONV3D_ERR_WORKSPACE for a missing or
+ * short workspace; otherwise as conv3d_fwd.
+ */
+CONV3D_API conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, int Cin,
+                                           int D, int H, int W, int Cout, const int kernel[3],
+                                           const int stride[3], const int pad[3],
+                                           conv3d_tpad_t tpad, conv3d_dtype_t dtype,
+                                           void* workspace, size_t ws_bytes,
+                                           struct CUstream_st* stream);
+CONV3D_API size_t conv3d_bwd_data_workspace_bytes(int N, int Cin, int D, int H, int W, int Cout,
+                                                  const int kernel[3], const int pad[3],
+                                                  conv3d_tpad_t tpad);
+
+/*
+ * conv3d_bwd_weight -- dw (and optionally dbias), the gradients of the
+ * convolution's weight and bias: dw[co, tap, ci] = sum over output pixels of
+ * dy[.., co] * Xpad[.., tap-shifted, ci] (the same implicit im2col matrix the
+ * forward pass reads, with the same padding rules), dbias[co] = sum of dy.
+ * Accumulated in fp32 in the workspace (split over pixel ranges, fp32
+ * atomics: the summation order varies from run to run), rounded once.
+ *
+ * Arguments describe the FORWARD problem: x [N, D, H, W, Cin], dy [N, Do, Ho,
+ * Wo, Cout], dw [Cout, kt, kh, kw, Cin] (written), dbias [Cout] or NULL.
+ * Strides up to 8, temporal rules zero, causal replicate and causal zero.
+ * workspace: device, 256-byte aligned, conv3d_bwd_weight_workspace_bytes()
+ * bytes (cleared by the call).  Errors: CONV3D_ERR_UNSUPPORTED for the
+ * cached-frames rule, CONV3D_ERR_INVALID_ARG for a null dw or overlapping
+ * buffers, CONV3D_ERR_ALIGNMENT for a dbias not 16-byte aligned,
+ * CONV3D_ERR_WORKSPACE for a missing or short workspace; otherwise as conv3d_fwd.
+ */
+CONV3D_API conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void* dbias,
+                                             int N, int Cin, int D, int H, int W, int Cout,
+                                             const int kernel[3], const int stride[3],
+                                             const int pad[3], conv3d_tpad_t tpad,
+                                             conv3d_dtype_t dtype, void* workspace,
+                                             size_t ws_bytes, struct CUstream_st* stream);
+CONV3D_API size_t conv3d_bwd_weight_workspace_bytes(int Cin, int Cout, const int kernel[3]);
+
 /* Device scratch bytes conv3d_fwd_ws needs for this problem (0 if none). */
 CONV3D_API size_t conv3d_workspace_bytes(int Cin, int Cout, int D, const int kernel[3], conv3d_tpad_t tpad);
 

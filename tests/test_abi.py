@@ -212,3 +212,67 @@ def test_groupnorm_silu_validation(kw, expect):
              per_frame=0, apply_silu=1, dtype=c3.BF16, stream=None)
     a.update(kw)
     assert c3.groupnorm_silu_ptr(**a) == expect
+
+
+# ---------------------------------------------------------------- backward entry points
+
+WS = 0x900000000   # fake workspace address
+
+
+def call_bwd_data(**kw):
+    a = dict(dy=Y, w=Wt, dx=X, N=1, Cin=64, D=4, H=16, W=16, Cout=64, kernel=(3, 3, 3),
+             stride=(1, 1, 1), pad=(0, 1, 1), tpad=c3.TPAD_CAUSAL_REPLICATE, dtype=c3.BF16,
+             workspace=WS, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return c3.conv3d_bwd_data_ptr(**a)
+
+
+def call_bwd_weight(**kw):
+    a = dict(x=X, dy=Y, dw=Wt, dbias=B, N=1, Cin=64, D=4, H=16, W=16, Cout=64, kernel=(3, 3, 3),
+             stride=(1, 1, 1), pad=(0, 1, 1), tpad=c3.TPAD_CAUSAL_REPLICATE, dtype=c3.BF16,
+             workspace=WS, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return c3.conv3d_bwd_weight_ptr(**a)
+
+
+def test_bwd_workspace_bytes():
+    # replicate padding keeps the kt-1 padded frames' gradient in fp32
+    assert c3.bwd_data_workspace_bytes(1, 64, 4, 16, 16, 64, (3, 3, 3), (0, 1, 1),
+                                       c3.TPAD_CAUSAL_REPLICATE) >= 1 * 6 * 16 * 16 * 64 * 4
+    dw = 64 * 27 * 32 * 4
+    assert c3.bwd_weight_workspace_bytes(32, 64, (3, 3, 3)) >= dw + 64 * 4
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(stride=(1, 2, 2)), Status.UNSUPPORTED),
+    (dict(tpad=c3.TPAD_CAUSAL_CACHED), Status.UNSUPPORTED),
+    (dict(pad=(0, 3, 1)), Status.UNSUPPORTED),             # pad > kernel extent - 1
+    (dict(workspace=None), Status.WORKSPACE),
+    (dict(ws_bytes=64), Status.WORKSPACE),
+    (dict(workspace=WS + 16), Status.ALIGNMENT),
+    (dict(dx=X + 2), Status.ALIGNMENT),
+    (dict(Cin=12), Status.UNSUPPORTED),
+])
+def test_bwd_data_validation(kw, expect):
+    assert call_bwd_data(**kw) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dw=None), Status.INVALID_ARG),
+    (dict(tpad=c3.TPAD_CAUSAL_CACHED), Status.UNSUPPORTED),
+    (dict(dbias=B + 4), Status.ALIGNMENT),
+    (dict(workspace=None), Status.WORKSPACE),
+    (dict(ws_bytes=1024), Status.WORKSPACE),
+    (dict(workspace=WS + 128), Status.ALIGNMENT),
+    (dict(workspace=X + 4096), Status.INVALID_ARG),        # workspace overlaps x
+    (dict(Cout=20), Status.UNSUPPORTED),
+])
+def test_bwd_weight_validation(kw, expect):
+    assert call_bwd_weight(**kw) == expect
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_bwd_entries_without_gpu_report_cuda_error():
+    assert call_bwd_data() == Status.CUDA
+    assert call_bwd_weight() == Status.CUDA
+    assert call_bwd_weight(stride=(2, 2, 2), dbias=None) == Status.CUDA   # strided wgrad is valid

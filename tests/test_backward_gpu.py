@@ -1,0 +1,89 @@
+"""GPU backward pass against the fp64 oracle's adjoints (parity tolerance:
+max|err| <= 1e-2 max|ref|, relative L1 <= 2e-3)."""
+import pytest
+import torch
+
+import oracle
+import seeded_inputs as si
+import video_vae_convolution_implicit_b200 as c3
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+ZERO, CREP, CZERO = c3.TPAD_ZERO, c3.TPAD_CAUSAL_REPLICATE, c3.TPAD_CAUSAL_ZERO
+TD = {"bf16": (torch.bfloat16, oracle.BF16), "f16": (torch.float16, oracle.F16)}
+
+
+def grads_problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed, dt, stride=(1, 1, 1)):
+    td, od = TD[dt]
+    fan = Cin * k[0] * k[1] * k[2]
+    x = si.tensor((N, D, H, W, Cin), seed, 0, 1.0, td, "cuda")
+    w = si.tensor((Cout, *k, Cin), seed, 1, fan ** -0.5, td, "cuda")
+    out = oracle.output_shape(D, H, W, k, stride, pad, tpad)
+    dy = si.tensor((N, *out, Cout), seed, 5, 1.0, td, "cuda")
+    return x, w, dy, od
+
+
+@pytest.fixture(params=["single", "swap"])
+def variant(request, monkeypatch):
+    monkeypatch.setenv("CONV3D_CTA_PAIR", "0")
+    monkeypatch.setenv("CONV3D_SWAP", "1" if request.param == "swap" else "0")
+    return request.param
+
+
+DATA_CASES = [
+    # N, Cin, D, H, W, Cout, kernel, pad, tpad, dtype
+    (1, 64, 4, 10, 12, 64, (3, 3, 3), (0, 1, 1), CREP, "bf16"),
+    (2, 64, 3, 9, 13, 128, (3, 3, 3), (0, 1, 1), CZERO, "bf16"),
+    (1, 32, 5, 8, 8, 48, (3, 3, 3), (1, 1, 1), ZERO, "f16"),
+    (1, 64, 6, 7, 9, 64, (3, 3, 3), (0, 1, 1), ZERO, "bf16"),        # pt = 0: Do = D - 2
+    (1, 128, 2, 16, 16, 64, (1, 1, 1), (0, 0, 0), ZERO, "bf16"),
+    (1, 48, 3, 11, 10, 40, (2, 3, 3), (0, 0, 1), CREP, "bf16"),
+    (1, 64, 1, 12, 12, 64, (3, 3, 3), (0, 1, 1), CREP, "bf16"),       # single frame
+]
+
+
+@pytest.mark.parametrize("case", DATA_CASES, ids=lambda c: "x".join(map(str, c[:6])) + f"-k{''.join(map(str, c[6]))}-t{c[8]}-{c[9]}")
+def test_bwd_data_every_element(case, variant):
+    N, Cin, D, H, W, Cout, k, pad, tpad, dt = case
+    x, w, dy, od = grads_problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=300 + Cin, dt=dt)
+    dx = c3.conv3d_bwd_data(dy, w, x.shape, pad, tpad)
+    assert c3.poll_status() == c3.Status.OK
+    ref, _, _ = oracle.conv3d_backward(si.bits(x), si.bits(w), si.bits(dy), od, k, (1, 1, 1),
+                                       pad, tpad)
+    assert_close(dx.double().cpu().numpy(), ref, str(case))
+
+
+def test_bwd_data_rejects_strides_and_cached_mode():
+    x, w, dy, _ = grads_problem(1, 64, 4, 8, 8, 64, (3, 3, 3), (0, 1, 1), CREP, 1, "bf16",
+                                stride=(1, 2, 2))
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    st = c3.conv3d_bwd_data_ptr(dy.data_ptr(), w.data_ptr(), x.data_ptr(), 1, 64, 4, 8, 8, 64,
+                                (3, 3, 3), (1, 2, 2), (0, 1, 1), CREP, c3.BF16, ws.data_ptr(),
+                                ws.numel(), 0)
+    assert st == c3.Status.UNSUPPORTED
+
+
+WEIGHT_CASES = [
+    # N, Cin, D, H, W, Cout, kernel, stride, pad, tpad, dtype
+    (1, 64, 4, 10, 12, 64, (3, 3, 3), (1, 1, 1), (0, 1, 1), CREP, "bf16"),
+    (2, 128, 3, 9, 13, 256, (3, 3, 3), (1, 1, 1), (0, 1, 1), CZERO, "bf16"),
+    (1, 32, 5, 8, 8, 48, (3, 3, 3), (1, 1, 1), (1, 1, 1), ZERO, "f16"),
+    (1, 64, 5, 12, 12, 64, (3, 3, 3), (2, 2, 2), (0, 1, 1), CREP, "bf16"),   # strided
+    (1, 256, 2, 16, 16, 320, (1, 1, 1), (1, 1, 1), (0, 0, 0), ZERO, "bf16"), # 2 co tiles, 1x1x1
+    (1, 192, 3, 7, 9, 40, (2, 3, 3), (1, 1, 1), (0, 1, 1), CREP, "bf16"),    # partial blocks
+    (1, 64, 6, 8, 8, 64, (3, 3, 3), (1, 1, 1), (3, 1, 1), ZERO, "bf16"),     # taps fully in padding
+]
+
+
+@pytest.mark.parametrize("case", WEIGHT_CASES, ids=lambda c: "x".join(map(str, c[:6])) + f"-k{''.join(map(str, c[6]))}-s{''.join(map(str, c[7]))}-t{c[9]}-{c[10]}")
+def test_bwd_weight_every_element(case):
+    N, Cin, D, H, W, Cout, k, stride, pad, tpad, dt = case
+    x, w, dy, od = grads_problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=400 + Cin, dt=dt,
+                                 stride=stride)
+    dw, db = c3.conv3d_bwd_weight(x, dy, k, stride, pad, tpad)
+    assert c3.poll_status() == c3.Status.OK
+    _, ref_dw, ref_db = oracle.conv3d_backward(si.bits(x), si.bits(w), si.bits(dy), od, k, stride,
+                                               pad, tpad)
+    assert_close(dw.double().cpu().numpy(), ref_dw, "dw " + str(case))
+    assert_close(db.double().cpu().numpy(), ref_db, "dbias " + str(case))

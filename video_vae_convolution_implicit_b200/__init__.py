@@ -19,7 +19,8 @@ import torch
 
 __all__ = [
     "TPAD_ZERO", "TPAD_CAUSAL_REPLICATE", "TPAD_CAUSAL_ZERO", "TPAD_CAUSAL_CACHED", "F16", "BF16",
-    "Status", "conv3d_fwd_cached_ptr", "groupnorm_stats", "groupnorm_silu",
+    "Status", "conv3d_fwd_cached_ptr", "groupnorm_stats", "groupnorm_silu", "conv3d_bwd_data",
+    "conv3d_bwd_weight",
     "Conv3dError", "lib_path", "conv3d", "conv3d_fwd", "conv3d_fwd_ptr", "conv3d_fwd_ws_ptr",
     "conv3d_fwd_noalloc_ptr",
     "output_shape", "workspace_bytes", "poll_status", "selftest_wait_timeout", "release",
@@ -72,6 +73,16 @@ _lib.conv3d_groupnorm_stats.restype = _c
 _lib.conv3d_groupnorm_stats.argtypes = [_vp] + [_c] * 7 + [ctypes.c_float, _c, _vp, _vp]
 _lib.conv3d_groupnorm_silu.restype = _c
 _lib.conv3d_groupnorm_silu.argtypes = [_vp] * 5 + [_c] * 8 + [_c, _vp]
+_lib.conv3d_bwd_data.restype = _c
+_lib.conv3d_bwd_data.argtypes = [_vp] * 3 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp, ctypes.c_size_t,
+                                                                   _vp]
+_lib.conv3d_bwd_data_workspace_bytes.restype = ctypes.c_size_t
+_lib.conv3d_bwd_data_workspace_bytes.argtypes = [_c] * 6 + [_i3, _i3, _c]
+_lib.conv3d_bwd_weight.restype = _c
+_lib.conv3d_bwd_weight.argtypes = [_vp] * 4 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp,
+                                                                     ctypes.c_size_t, _vp]
+_lib.conv3d_bwd_weight_workspace_bytes.restype = ctypes.c_size_t
+_lib.conv3d_bwd_weight_workspace_bytes.argtypes = [_c, _c, _i3]
 _lib.conv3d_fwd_noalloc.restype = _c
 _lib.conv3d_fwd_noalloc.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp]
 _lib.conv3d_workspace_bytes.restype = ctypes.c_size_t
@@ -296,3 +307,68 @@ def groupnorm_silu(x: torch.Tensor, stats: torch.Tensor, gamma=None, beta=None, 
                               y.data_ptr(), N, D, H, W, C, groups, per_frame, apply_silu,
                               _dtype_code(x.dtype), _stream_handle(stream)))
     return y
+
+
+def conv3d_bwd_data_ptr(dy, w, dx, N, Cin, D, H, W, Cout, kernel, stride, pad, tpad, dtype,
+                        workspace, ws_bytes, stream) -> int:
+    """Raw-pointer call of conv3d_bwd_data; returns the status code."""
+    return _lib.conv3d_bwd_data(dy, w, dx, N, Cin, D, H, W, Cout, _i3(*kernel), _i3(*stride),
+                                _i3(*pad), tpad, dtype, workspace, ws_bytes, stream)
+
+
+def bwd_data_workspace_bytes(N, Cin, D, H, W, Cout, kernel, pad, tpad) -> int:
+    return int(_lib.conv3d_bwd_data_workspace_bytes(N, Cin, D, H, W, Cout, _i3(*kernel), _i3(*pad),
+                                                    tpad))
+
+
+def conv3d_bwd_data(dy: torch.Tensor, w: torch.Tensor, x_shape, pad=(0, 1, 1),
+                    tpad=TPAD_CAUSAL_REPLICATE, dx: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """dx for the forward problem x [x_shape] -> y (dy has y's shape), stride 1."""
+    N, D, H, W, Cin = x_shape
+    Cout, kt, kh, kw, _ = w.shape
+    if dx is None:
+        dx = torch.empty(tuple(x_shape), dtype=dy.dtype, device=dy.device)
+    need = bwd_data_workspace_bytes(N, Cin, D, H, W, Cout, (kt, kh, kw), pad, tpad)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dy.device)
+    for name, t in (("dy", dy), ("w", w), ("dx", dx)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != dy.dtype:
+            raise ValueError(f"{name} must be a contiguous CUDA tensor of dy's dtype")
+    _check(conv3d_bwd_data_ptr(dy.data_ptr(), w.data_ptr(), dx.data_ptr(), N, Cin, D, H, W, Cout,
+                               (kt, kh, kw), (1, 1, 1), pad, tpad, _dtype_code(dy.dtype),
+                               workspace.data_ptr(), workspace.numel(), _stream_handle(stream)))
+    return dx
+
+
+def conv3d_bwd_weight_ptr(x, dy, dw, dbias, N, Cin, D, H, W, Cout, kernel, stride, pad, tpad,
+                          dtype, workspace, ws_bytes, stream) -> int:
+    """Raw-pointer call of conv3d_bwd_weight; returns the status code."""
+    return _lib.conv3d_bwd_weight(x, dy, dw, dbias, N, Cin, D, H, W, Cout, _i3(*kernel),
+                                  _i3(*stride), _i3(*pad), tpad, dtype, workspace, ws_bytes,
+                                  stream)
+
+
+def bwd_weight_workspace_bytes(Cin, Cout, kernel) -> int:
+    return int(_lib.conv3d_bwd_weight_workspace_bytes(Cin, Cout, _i3(*kernel)))
+
+
+def conv3d_bwd_weight(x: torch.Tensor, dy: torch.Tensor, kernel, stride=(1, 1, 1), pad=(0, 1, 1),
+                      tpad=TPAD_CAUSAL_REPLICATE, with_bias: bool = True,
+                      workspace: torch.Tensor | None = None, stream=None):
+    """(dw, dbias) for the forward problem x -> y with upstream gradient dy."""
+    N, D, H, W, Cin = x.shape
+    Cout = dy.shape[-1]
+    dw = torch.empty((Cout, *kernel, Cin), dtype=x.dtype, device=x.device)
+    db = torch.empty((Cout,), dtype=x.dtype, device=x.device) if with_bias else None
+    need = bwd_weight_workspace_bytes(Cin, Cout, kernel)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    for name, t in (("x", x), ("dy", dy)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype:
+            raise ValueError(f"{name} must be a contiguous CUDA tensor of x's dtype")
+    _check(conv3d_bwd_weight_ptr(x.data_ptr(), dy.data_ptr(), dw.data_ptr(), _ptr(db), N, Cin, D,
+                                 H, W, Cout, tuple(kernel), stride, pad, tpad,
+                                 _dtype_code(x.dtype), workspace.data_ptr(), workspace.numel(),
+                                 _stream_handle(stream)))
+    return dw, db

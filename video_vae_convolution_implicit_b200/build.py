@@ -10,7 +10,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libconv3d.so")
 SOURCES = [os.path.join(CSRC, "conv3d_api.cu"), os.path.join(CSRC, "groupnorm.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("conv3d_kernel.cuh", "ptx.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("conv3d_kernel.cuh", "wgrad_kernel.cuh", "ptx.cuh")] + [
     os.path.join(ROOT, "include", "conv3d.h")]
 
 

@@ -16,6 +16,7 @@
 
 #include "conv3d.h"
 #include "conv3d_kernel.cuh"
+#include "wgrad_kernel.cuh"
 
 namespace {
 
@@ -50,6 +51,7 @@ struct Problem {
   conv3d_tpad_t tpad;
   conv3d_dtype_t dtype;
   bool has_residual;
+  bool out_f32;      // write y in fp32 (internal: the backward pass's padded-frame gradient)
   const void* prev;  // cached frames before the chunk (CONV3D_TPAD_CAUSAL_CACHED) or null
   bool fold;  // first-frame path: fold the temporal taps into a (hi, lo) pair
 };
@@ -177,6 +179,7 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
   P.tpad = tpad;
   P.dtype = dtype;
   P.has_residual = residual != nullptr;
+  P.out_f32 = false;
   P.prev = tpad == CONV3D_TPAD_CAUSAL_CACHED ? prev : nullptr;
   // a single causal-replicate frame: every temporal tap of the one output
   // frame reads frame 0 (whatever the temporal stride)
@@ -333,17 +336,22 @@ conv3d_status_t encode_maps(const Problem& P, const void* x, const void* wmat, i
 // y (or the residual) viewed as [N*Do frames][Ho*Wo pixels][Cout]; a box is 32
 // channels x 32 pixels of one frame, 64-byte swizzled.  Stores clip pixels
 // past the frame and channels past Cout; loads read them as zero.
-conv3d_status_t encode_out_map(const Problem& P, const void* base, CUtensorMap& map) {
+conv3d_status_t encode_out_map(const Problem& P, const void* base, CUtensorMap& map,
+                               bool f32 = false) {
   const CUtensorMapDataType dt =
-      P.dtype == CONV3D_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+      f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+          : (P.dtype == CONV3D_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  const cuuint64_t esize = f32 ? 4 : 2;
   const cuuint64_t howo = static_cast<cuuint64_t>(P.Ho) * P.Wo;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(P.Cout), howo,
                               static_cast<cuuint64_t>(P.N) * static_cast<cuuint64_t>(P.Do)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(P.Cout) * 2, howo * P.Cout * 2};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(P.Cout) * esize, howo * P.Cout * esize};
   const cuuint32_t box[3] = {32, 32, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode_tiled(&map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -418,6 +426,7 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, L
     if (env[0] == '1') L.pair = true;
   }
   if (L.swap) L.pair = false;
+  if (P.out_f32) L.swap = L.pair = false;   // the fp32 epilogue exists in the single variant
   const int ctas = L.pair ? 2 : 1;
   if (L.swap) {
     kp.co_tile = 128;
@@ -432,7 +441,9 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, L
   const int b_stage = kp.BN / ctas * BK * 2;
   const int stage_bytes = A_STAGE_BYTES + b_stage;
   kp.has_residual = P.has_residual ? 1 : 0;
-  const int reserve = 1024 /*alignment slack*/ + EPI_Y_BYTES * (kp.has_residual ? 2 : 1) +
+  kp.out_f32 = P.out_f32 ? 1 : 0;
+  const int reserve = 1024 /*alignment slack*/ + EPI_Y_BYTES * (kp.out_f32 ? 2 : 1) +
+                      EPI_Y_BYTES * (kp.has_residual ? 1 : 0) +
                       8 * (2 * MAX_STAGES + 5 + 2 * EPI_WARPS);
   int stages = (S.max_smem_optin - reserve - 64 /*static smem*/) / stage_bytes;
   if (stages > MAX_STAGES) stages = MAX_STAGES;
@@ -519,7 +530,7 @@ conv3d_status_t launch_main(DeviceState& S, const Problem& P, const void* x, con
   st = L.swap ? encode_maps(P, x, wmat, L.kp.kt, L.kp.co_tile, L.kp.pix_tile, map_a, map_b)
               : encode_maps(P, x, wmat, L.kp.kt, L.kp.BN / (L.pair ? 2 : 1), BM, map_a, map_b);
   if (st != CONV3D_OK) return st;
-  if ((st = encode_out_map(P, y, map_y)) != CONV3D_OK) return st;
+  if ((st = encode_out_map(P, y, map_y, P.out_f32)) != CONV3D_OK) return st;
   if (residual) {
     if ((st = encode_out_map(P, residual, map_r)) != CONV3D_OK) return st;
   } else {
@@ -632,6 +643,67 @@ conv3d_status_t noalloc_scratch(void*& out) {
   return CONV3D_OK;
 }
 
+// ------------------------------------------------------------------ backward data pass
+
+struct BwdDataPlan {
+  Problem fwd;      // the forward problem being differentiated
+  Problem tr;       // the transposed convolution that produces dx (or its extension)
+  size_t wt_bytes;  // flipped weight
+  size_t ext_bytes; // gradient of the padded frames (causal replicate only)
+};
+
+conv3d_status_t plan_bwd_data(const void* dy, const void* w, const void* dx, int N, int Cin, int D,
+                              int H, int W, int Cout, const int kernel[3], const int stride[3],
+                              const int pad[3], conv3d_tpad_t tpad, conv3d_dtype_t dtype,
+                              BwdDataPlan& B) {
+  if (tpad == CONV3D_TPAD_CAUSAL_CACHED) {
+    set_error("the backward pass of the cached-frames mode is not supported");
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  // validate as the forward problem x -> y (x = dx, y = dy)
+  conv3d_status_t st = validate(dx, w, nullptr, nullptr, dy, N, Cin, D, H, W, Cout, kernel,
+                                stride, pad, tpad, dtype, B.fwd);
+  if (st != CONV3D_OK) return st;
+  if (stride[0] != 1 || stride[1] != 1 || stride[2] != 1) {
+    set_error("the backward data pass supports stride (1,1,1) only");
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  const Problem& F = B.fwd;
+  if (F.ph > F.kh - 1 || F.pw > F.kw - 1 || F.pf > F.kt - 1 || F.pb > F.kt - 1) {
+    set_error("the backward data pass needs pads <= kernel extent - 1");
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  const bool rep = tpad == CONV3D_TPAD_CAUSAL_REPLICATE && F.kt > 1;
+  Problem& T = B.tr;
+  T = Problem{};
+  T.N = N;
+  T.Cin = Cout;              // dy's channels
+  T.D = F.Do;
+  T.H = F.Ho;
+  T.W = F.Wo;
+  T.Cout = Cin;              // dx's channels
+  T.kt = F.kt; T.kh = F.kh; T.kw = F.kw;
+  T.st = T.sh = T.sw = 1;
+  T.ph = F.kh - 1 - F.ph;
+  T.pw = F.kw - 1 - F.pw;
+  // dx[f] gathers dy[f + it' - (kt-1-pf)]; with replicate padding the output is
+  // extended to the kt-1 virtual frames in front (folded onto frame 0 afterwards)
+  T.pf = F.kt - 1 - F.pf + (rep ? F.kt - 1 : 0);
+  T.pb = F.kt - 1 - F.pb;
+  T.Do = D + (rep ? F.kt - 1 : 0);
+  T.Ho = H;
+  T.Wo = W;
+  T.tpad = CONV3D_TPAD_ZERO;  // dy frames outside [0, Do) contribute nothing
+  T.dtype = dtype;
+  T.has_residual = false;
+  T.out_f32 = rep;            // the padded-frame gradient stays fp32 until the fold
+  T.prev = nullptr;
+  T.fold = false;
+  B.wt_bytes = (static_cast<size_t>(Cout) * F.kt * F.kh * F.kw * Cin * 2 + 255) & ~size_t(255);
+  B.ext_bytes = rep ? (static_cast<size_t>(N) * T.Do * H * W * Cin * 4 + 255) & ~size_t(255) : 0;
+  return CONV3D_OK;
+}
+
 __global__ void selftest_wait_kernel(int* status, unsigned long long timeout_ns) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int s_abort;
@@ -726,6 +798,238 @@ conv3d_status_t conv3d_fwd_cached(const void* x, const void* prev, const void* w
                                 pad, CONV3D_TPAD_CAUSAL_CACHED, dtype, P, prev);
   if (st != CONV3D_OK) return st;
   return run(P, x, w, bias, residual, y, nullptr, 0, false, stream);
+}
+
+size_t conv3d_bwd_data_workspace_bytes(int N, int Cin, int D, int H, int W, int Cout,
+                                       const int kernel[3], const int pad[3], conv3d_tpad_t tpad) {
+  if (!kernel || !pad || N < 1 || Cin < 1 || D < 1 || H < 1 || W < 1 || Cout < 1) return 0;
+  const size_t wt = (static_cast<size_t>(Cout) * kernel[0] * kernel[1] * kernel[2] * Cin * 2 + 255) &
+                    ~size_t(255);
+  size_t ext = 0;
+  if (tpad == CONV3D_TPAD_CAUSAL_REPLICATE && kernel[0] > 1)
+    ext = (static_cast<size_t>(N) * (D + kernel[0] - 1) * H * W * Cin * 4 + 255) & ~size_t(255);
+  return wt + ext;
+}
+
+conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, int Cin, int D,
+                                int H, int W, int Cout, const int kernel[3], const int stride[3],
+                                const int pad[3], conv3d_tpad_t tpad, conv3d_dtype_t dtype,
+                                void* workspace, size_t ws_bytes, struct CUstream_st* stream) {
+  BwdDataPlan B;
+  conv3d_status_t st = plan_bwd_data(dy, w, dx, N, Cin, D, H, W, Cout, kernel, stride, pad, tpad,
+                                     dtype, B);
+  if (st != CONV3D_OK) return st;
+  const size_t need = B.wt_bytes + B.ext_bytes;
+  if (workspace == nullptr || ws_bytes < need) {
+    set_error("workspace of %zu bytes required", need);
+    return CONV3D_ERR_WORKSPACE;
+  }
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) {
+    set_error("workspace must be 256-byte aligned");
+    return CONV3D_ERR_ALIGNMENT;
+  }
+  const size_t dx_bytes = static_cast<size_t>(N) * D * H * W * Cin * 2;
+  const size_t dy_bytes = static_cast<size_t>(N) * B.fwd.Do * B.fwd.Ho * B.fwd.Wo * Cout * 2;
+  const size_t w_bytes = static_cast<size_t>(Cout) * kernel[0] * kernel[1] * kernel[2] * Cin * 2;
+  if (overlaps(workspace, need, dx, dx_bytes) || overlaps(workspace, need, dy, dy_bytes) ||
+      overlaps(workspace, need, w, w_bytes) || overlaps(dx, dx_bytes, dy, dy_bytes)) {
+    set_error("dx, dy, w and the workspace must not overlap");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if ((st = load_entry_points()) != CONV3D_OK) return st;
+  DeviceState* S = nullptr;
+  int dev = 0;
+  if ((st = device_state(S, dev)) != CONV3D_OK) return st;
+  uint16_t* wt = static_cast<uint16_t*>(workspace);
+  {
+    const long long total = static_cast<long long>(Cout) * kernel[0] * kernel[1] * kernel[2] * Cin;
+    int blocks = static_cast<int>((total + 255) / 256);
+    if (blocks > 8 * S->num_sms) blocks = 8 * S->num_sms;
+    flip_transpose_weight_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(w), wt,
+                                                            Cout, kernel[0], kernel[1], kernel[2],
+                                                            Cin);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
+  }
+  void* out = B.ext_bytes ? static_cast<void*>(static_cast<char*>(workspace) + B.wt_bytes) : dx;
+  if ((st = launch_main(*S, B.tr, dy, nullptr, wt, nullptr, nullptr, out, stream)) != CONV3D_OK)
+    return st;
+  if (B.ext_bytes) {
+    const long long frame_elems = static_cast<long long>(H) * W * Cin;
+    const long long total = static_cast<long long>(N) * D * (frame_elems / 8);
+    int blocks = static_cast<int>((total + 255) / 256);
+    if (blocks > 8 * S->num_sms) blocks = 8 * S->num_sms;
+    if (dtype == CONV3D_BF16)
+      fold_front_gradient_kernel<true><<<blocks, 256, 0, stream>>>(
+          static_cast<const float*>(out), static_cast<uint16_t*>(dx), N, D, kernel[0],
+          frame_elems);
+    else
+      fold_front_gradient_kernel<false><<<blocks, 256, 0, stream>>>(
+          static_cast<const float*>(out), static_cast<uint16_t*>(dx), N, D, kernel[0],
+          frame_elems);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "gradient fold launch");
+  }
+  return CONV3D_OK;
+}
+
+size_t conv3d_bwd_weight_workspace_bytes(int Cin, int Cout, const int kernel[3]) {
+  if (!kernel || Cin < 1 || Cout < 1) return 0;
+  const size_t dw = static_cast<size_t>(Cout) * kernel[0] * kernel[1] * kernel[2] * Cin * 4;
+  return ((dw + 255) & ~size_t(255)) + ((static_cast<size_t>(Cout) * 4 + 255) & ~size_t(255));
+}
+
+conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void* dbias, int N,
+                                  int Cin, int D, int H, int W, int Cout, const int kernel[3],
+                                  const int stride[3], const int pad[3], conv3d_tpad_t tpad,
+                                  conv3d_dtype_t dtype, void* workspace, size_t ws_bytes,
+                                  struct CUstream_st* stream) {
+  if (tpad == CONV3D_TPAD_CAUSAL_CACHED) {
+    set_error("the backward pass of the cached-frames mode is not supported");
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  Problem F;
+  conv3d_status_t st = validate(x, dw ? dw : workspace, nullptr, nullptr, dy, N, Cin, D, H, W,
+                                Cout, kernel, stride, pad, tpad, dtype, F);
+  if (st != CONV3D_OK) return st;
+  if (!dw) {
+    set_error("dw must be non-null");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if (dbias && (reinterpret_cast<uintptr_t>(dbias) & 15u)) {
+    set_error("dbias must be 16-byte aligned");
+    return CONV3D_ERR_ALIGNMENT;
+  }
+  const size_t need = conv3d_bwd_weight_workspace_bytes(Cin, Cout, kernel);
+  if (workspace == nullptr || ws_bytes < need) {
+    set_error("workspace of %zu bytes required", need);
+    return CONV3D_ERR_WORKSPACE;
+  }
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) {
+    set_error("workspace must be 256-byte aligned");
+    return CONV3D_ERR_ALIGNMENT;
+  }
+  const long long taps = static_cast<long long>(kernel[0]) * kernel[1] * kernel[2];
+  const size_t dw_elems = static_cast<size_t>(Cout) * taps * Cin;
+  const size_t x_bytes = static_cast<size_t>(N) * D * H * W * Cin * 2;
+  const size_t dy_bytes = static_cast<size_t>(N) * F.Do * F.Ho * F.Wo * Cout * 2;
+  if (overlaps(workspace, need, x, x_bytes) || overlaps(workspace, need, dy, dy_bytes) ||
+      overlaps(workspace, need, dw, dw_elems * 2) || overlaps(dw, dw_elems * 2, x, x_bytes) ||
+      overlaps(dw, dw_elems * 2, dy, dy_bytes)) {
+    set_error("x, dy, dw and the workspace must not overlap");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if ((st = load_entry_points()) != CONV3D_OK) return st;
+  DeviceState* S = nullptr;
+  int dev = 0;
+  if ((st = device_state(S, dev)) != CONV3D_OK) return st;
+  const bool bf16 = dtype == CONV3D_BF16;
+  float* dw32 = static_cast<float*>(workspace);
+  float* db32 = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                         ((dw_elems * 4 + 255) & ~size_t(255)));
+
+  WgradParams wp{};
+  wp.D = F.D; wp.Do = F.Do; wp.Ho = F.Ho; wp.Wo = F.Wo; wp.HoWo = F.Ho * F.Wo;
+  wp.Cin = Cin; wp.Cout = Cout;
+  wp.kt = F.kt; wp.kh = F.kh; wp.kw = F.kw;
+  wp.st = F.st; wp.sh = F.sh; wp.sw = F.sw;
+  wp.pf = F.pf; wp.ph = F.ph; wp.pw = F.pw;
+  wp.tpad = static_cast<int>(tpad);
+  wp.taps = static_cast<int>(taps);
+  wp.cblocks = (Cin + 127) / 128;
+  wp.BN = Cout >= 256 ? 256 : ((Cout + 63) / 64) * 64;
+  wp.co_tiles = (Cout + wp.BN - 1) / wp.BN;
+  wp.chunks_per_frame = (wp.HoWo + WG_PIX - 1) / WG_PIX;
+  wp.total_chunks = static_cast<long long>(N) * F.Do * wp.chunks_per_frame;
+  const long long base_units = static_cast<long long>(wp.taps) * wp.cblocks * wp.co_tiles;
+  long long splits = (2LL * S->num_sms + base_units - 1) / base_units;
+  if (splits > wp.total_chunks / 4) splits = wp.total_chunks / 4;
+  if (splits < 1) splits = 1;
+  if (base_units * splits > 0x7FFFFFFFLL) {
+    set_error("problem too large");
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  wp.splits = static_cast<int>(splits);
+  wp.num_units = static_cast<int>(base_units * splits);
+  const int stage_bytes = WG_A_BYTES + wp.BN * WG_PIX * 2;
+  const int reserve = 1024 + 8 * (2 * MAX_STAGES + 5);
+  int stages = (S->max_smem_optin - reserve - 64) / stage_bytes;
+  if (stages > MAX_STAGES) stages = MAX_STAGES;
+  wp.stages = stages;
+  wp.tmem_cols = pow2_at_least(2u * wp.BN);
+  wp.idesc = idesc_f16(bf16, BM, wp.BN) | (1u << 15) | (1u << 16);  // both operands MN-major
+  wp.dw = dw32;
+  wp.status = S->status;
+  wp.timeout_ns = kDefaultTimeoutNs;
+  const size_t smem = static_cast<size_t>(stages) * stage_bytes + reserve;
+
+  // x through the forward im2col map (64 pixels per load); dy as [frames][pixels][Cout]
+  CUtensorMap map_x, map_dy;
+  if ((st = encode_im2col(F, x, static_cast<long long>(N) * D, WG_PIX, map_x)) != CONV3D_OK)
+    return st;
+  {
+    const CUtensorMapDataType dt =
+        bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const cuuint64_t howo = static_cast<cuuint64_t>(F.Ho) * F.Wo;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(Cout), howo,
+                                static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(F.Do)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(Cout) * 2, howo * Cout * 2};
+    const cuuint32_t box[3] = {64, WG_PIX, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode_tiled(&map_dy, dt, 3, const_cast<void*>(dy), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+      set_error("cuTensorMapEncodeTiled (dy) failed (%d)", static_cast<int>(r));
+      return CONV3D_ERR_CUDA;
+    }
+  }
+  cudaError_t e = cudaMemsetAsync(workspace, 0, need, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
+  auto kern = bf16 ? conv3d_wgrad_kernel<true> : conv3d_wgrad_kernel<false>;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             S->max_smem_optin - 64);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  }
+  const int grid = wp.num_units < S->num_sms ? wp.num_units : S->num_sms;
+  kern<<<grid, NUM_THREADS, smem, stream>>>(map_x, map_dy, wp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "wgrad kernel launch");
+  {
+    int blocks = static_cast<int>((dw_elems + 255) / 256);
+    if (blocks > 8 * S->num_sms) blocks = 8 * S->num_sms;
+    if (bf16)
+      f32_to_16_kernel<true><<<blocks, 256, 0, stream>>>(dw32, static_cast<uint16_t*>(dw),
+                                                         static_cast<long long>(dw_elems));
+    else
+      f32_to_16_kernel<false><<<blocks, 256, 0, stream>>>(dw32, static_cast<uint16_t*>(dw),
+                                                          static_cast<long long>(dw_elems));
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dw conversion launch");
+  }
+  if (dbias) {
+    const long long pixels = static_cast<long long>(N) * F.Do * F.Ho * F.Wo;
+    const int vecs = Cout / 8;
+    int rows = 256 / vecs;
+    if (rows < 1) rows = 1;
+    const int threads = vecs * rows > 1024 ? 1024 : vecs * rows;
+    const long long per = 1024;
+    const long long blocks = (pixels + per - 1) / per;
+    if (bf16)
+      bias_grad_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+          static_cast<const uint16_t*>(dy), db32, pixels, Cout, per);
+    else
+      bias_grad_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+          static_cast<const uint16_t*>(dy), db32, pixels, Cout, per);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dbias launch");
+    if (bf16)
+      f32_to_16_kernel<true><<<1, 256, 0, stream>>>(db32, static_cast<uint16_t*>(dbias), Cout);
+    else
+      f32_to_16_kernel<false><<<1, 256, 0, stream>>>(db32, static_cast<uint16_t*>(dbias), Cout);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dbias conversion launch");
+  }
+  return CONV3D_OK;
 }
 
 size_t conv3d_workspace_bytes(int Cin, int Cout, int D, const int kernel[3], conv3d_tpad_t tpad) {

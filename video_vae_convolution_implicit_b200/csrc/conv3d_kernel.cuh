@@ -64,6 +64,7 @@ struct KernelParams {
   uint32_t idesc;
   const void* bias;                  // [Cout] or null
   int has_residual;                  // residual is read through map_r
+  int out_f32;                       // y is fp32 (single-CTA, non-transposed variant only)
   int* status;                       // device status word
   unsigned long long timeout_ns;
 };
@@ -79,6 +80,11 @@ constexpr int EPI_Y_BYTES = EPI_WARPS * 2 * EPI_BUF_BYTES;
 // offset).
 __device__ __forceinline__ uint32_t swz64(uint32_t r, uint32_t c) {
   return r * 64u + ((c ^ ((r >> 1) & 3u)) << 4);
+}
+
+// The same for 32 x 128-byte rows (fp32 output) with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t c) {
+  return r * 128u + ((c ^ (r & 7u)) << 4);
 }
 
 struct Tile {
@@ -219,8 +225,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t b_stage_bytes = b_rows * BK * 2;
   const uint32_t a_ring = base;
   const uint32_t b_ring = a_ring + p.stages * A_STAGE_BYTES;
+  const uint32_t ybytes = p.out_f32 ? 2 * EPI_BUF_BYTES : EPI_BUF_BYTES;   // one y buffer
   const uint32_t y_stage = b_ring + p.stages * b_stage_bytes;        // [EPI_WARPS][2] buffers
-  const uint32_t r_stage = y_stage + EPI_Y_BYTES;                     // same, with a residual
+  const uint32_t r_stage = y_stage + EPI_WARPS * 2 * ybytes;          // same, with a residual
   const uint32_t bars = r_stage + (p.has_residual ? EPI_Y_BYTES : 0);
   const uint32_t full_bar = bars;                         // [stages]
   const uint32_t empty_bar = bars + 8 * p.stages;         // [stages]
@@ -414,7 +421,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     using C = Cvt<kBF16>;
     const uint32_t quarter = warp & 3;            // TMEM lanes [32q, 32q+32)
     const uint32_t ew = warp - 2;                 // epilogue warp index, 0..3
-    const uint32_t ybuf = y_stage + ew * 2 * EPI_BUF_BYTES;
+    const uint32_t ybuf = y_stage + ew * 2 * ybytes;
     const uint32_t rbuf = r_stage + ew * 2 * EPI_BUF_BYTES;
     const uint32_t rbar = rfull_bar + ew * 16;
     uint32_t rphase[2] = {0, 0};
@@ -486,7 +493,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             if (lane == 0) bulk_wait_group_read<1>();
             __syncwarp();
-            const uint32_t yb = ybuf + b * EPI_BUF_BYTES;
+            const uint32_t yb = ybuf + b * ybytes;
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const uint16_t q = static_cast<uint16_t>(C::pack(v[e], 0.0f) & 0xFFFFu);
@@ -587,18 +594,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // the store issued from this buffer two chunks ago must have read it
           if (lane == 0) bulk_wait_group_read<1>();
           __syncwarp();
+          if (p.out_f32) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            st_shared_v4(ybuf + b * EPI_BUF_BYTES + swz64(lane, g),
-                         C::pack(v[8 * g + 0], v[8 * g + 1]), C::pack(v[8 * g + 2], v[8 * g + 3]),
-                         C::pack(v[8 * g + 4], v[8 * g + 5]), C::pack(v[8 * g + 6], v[8 * g + 7]));
+            for (int c = 0; c < 8; ++c)
+              st_shared_v4(ybuf + b * ybytes + swz128(lane, c), __float_as_uint(v[4 * c + 0]),
+                           __float_as_uint(v[4 * c + 1]), __float_as_uint(v[4 * c + 2]),
+                           __float_as_uint(v[4 * c + 3]));
+          } else {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              st_shared_v4(ybuf + b * ybytes + swz64(lane, g),
+                           C::pack(v[8 * g + 0], v[8 * g + 1]), C::pack(v[8 * g + 2], v[8 * g + 3]),
+                           C::pack(v[8 * g + 4], v[8 * g + 5]), C::pack(v[8 * g + 6], v[8 * g + 7]));
+            }
           }
           fence_proxy_async_shared();
           __syncwarp();
           // every lane has read residual buffer b: refill it with chunk j+2
           const bool refill = use_res && j + 2 < live_chunks;
           if (lane == 0) {
-            tma_store_3d(&map_y, ybuf + b * EPI_BUF_BYTES, cb, row_base, tl.frame_out);
+            tma_store_3d(&map_y, ybuf + b * ybytes, cb, row_base, tl.frame_out);
             bulk_commit_group();
             if (refill) {
               mbar_arrive_expect_tx(rbar + 8 * b, EPI_BUF_BYTES);
@@ -670,6 +685,67 @@ __global__ void fold_temporal_taps_kernel(const uint16_t* __restrict__ w, uint16
     const uint32_t lo = C::pack(s - C::lo(hi), 0.0f) & 0xFFFFu;
     w2[co * 2 * spatial_cin + rest] = static_cast<uint16_t>(hi);
     w2[co * 2 * spatial_cin + spatial_cin + rest] = static_cast<uint16_t>(lo);
+  }
+}
+
+// Backward data pass: the weight the transposed convolution runs with,
+// wt[ci, it, ih, iw, co] = w[co, kt-1-it, kh-1-ih, kw-1-iw, ci] (every tap
+// mirrored, the channel roles exchanged).
+__global__ void flip_transpose_weight_kernel(const uint16_t* __restrict__ w,
+                                             uint16_t* __restrict__ wt, int Cout, int kt, int kh,
+                                             int kw, int Cin) {
+  const long long taps = static_cast<long long>(kt) * kh * kw;
+  const long long total = taps * Cout * Cin;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    // i indexes wt = [Cin][kt][kh][kw][Cout]
+    const long long co = i % Cout;
+    long long q = i / Cout;
+    const int iw = static_cast<int>(q % kw); q /= kw;
+    const int ih = static_cast<int>(q % kh); q /= kh;
+    const int it = static_cast<int>(q % kt); q /= kt;
+    const long long ci = q;
+    const long long src =
+        (((co * kt + (kt - 1 - it)) * kh + (kh - 1 - ih)) * kw + (kw - 1 - iw)) * Cin + ci;
+    wt[i] = w[src];
+  }
+}
+
+// Causal replicate padding reads frame 0 for the kt-1 frames in front, so the
+// gradient of those virtual frames belongs to frame 0: dx[n, 0] = sum of
+// ext[n, 0 .. kt-1], dx[n, f] = ext[n, f + kt - 1] for f >= 1, where ext holds
+// the gradient of the D + kt - 1 padded frames.  8 values per thread.
+template <bool kBF16>
+__global__ void fold_front_gradient_kernel(const float* __restrict__ ext,
+                                           uint16_t* __restrict__ dx, int N, int D, int kt,
+                                           long long frame_elems) {
+  using C = Cvt<kBF16>;
+  // ext is fp32 so that frame 0's sum is rounded once
+  const long long vecs_per_frame = frame_elems / 8;
+  const long long total = static_cast<long long>(N) * D * vecs_per_frame;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long v = i % vecs_per_frame;
+    const long long nf = i / vecs_per_frame;
+    const int f = static_cast<int>(nf % D);
+    const long long n = nf / D;
+    const long long ext_frames = static_cast<long long>(D) + kt - 1;
+    const float4* e4 = reinterpret_cast<const float4*>(ext);
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const int e_begin = f > 0 ? f + kt - 1 : 0;
+    const int e_end = f > 0 ? f + kt : kt;
+    for (int e = e_begin; e < e_end; ++e) {
+      const long long at = ((n * ext_frames + e) * vecs_per_frame + v) * 2;
+      const float4 a = e4[at], b = e4[at + 1];
+      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+    }
+    uint4 out;
+    out.x = C::pack(acc[0], acc[1]);
+    out.y = C::pack(acc[2], acc[3]);
+    out.z = C::pack(acc[4], acc[5]);
+    out.w = C::pack(acc[6], acc[7]);
+    reinterpret_cast<uint4*>(dx)[nf * vecs_per_frame + v] = out;
   }
 }
 

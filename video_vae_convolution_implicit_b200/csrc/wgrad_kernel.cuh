@@ -1,0 +1,332 @@
+// wgrad_kernel.cuh -- the weight gradient of the implicit-GEMM convolution,
+// dw[co, tap, ci] = sum over output pixels m of dy[m, co] * A[m, (tap, ci)],
+// A being the same implicit im2col matrix the forward pass reads (the pages'
+// on-device fine-tuning trains convolution layers: engineering.drawthings.ai,
+// LoRA post).
+//
+// As a GEMM the reduction runs over output pixels, which neither x nor dy
+// stores innermost, so both tcgen05 operands are MN-major: M = 128 rows of
+// (tap, ci) -- one tap, two 64-channel chunks -- and N = up to 256 output
+// channels, K = 64 output pixels per pipeline stage (four K = 16 MMAs).  A
+// stage holds two im2col loads (64 pixels x 64 channels) and BN/64 tiled loads
+// of dy (64 pixels x 64 channels), each 64 rows of 128 swizzled bytes: exactly
+// the MN-major 128-byte-swizzle layout (64-element blocks 8 KB apart along
+// M/N, 8-row groups 1 KB apart along K).
+//
+// Work unit = (tap and 128-channel block, output-channel block, range of
+// 64-pixel chunks); persistent CTAs walk the units.  Chunks whose temporal tap
+// reads zero padding are skipped by producer and MMA alike; chunk rows past
+// the frame read dy as zero.  Each finished unit adds its 128 x BN fp32 block
+// to a zeroed fp32 gradient with coalesced atomics (one warp: 32 consecutive
+// (tap, ci) entries of one output channel per instruction).
+#pragma once
+
+#include "conv3d_kernel.cuh"
+
+namespace conv3d {
+
+struct WgradParams {
+  int D, Do, Ho, Wo, HoWo;
+  int Cin, Cout;
+  int kt, kh, kw;
+  int st, sh, sw;
+  int pf, ph, pw;
+  int tpad;                 // 0 zero, 1 causal replicate, 2 causal zero
+  int taps;
+  int cblocks;              // ceil(Cin / 128)
+  int BN;                   // output channels per unit (multiple of 64, <= 256)
+  int co_tiles;             // ceil(Cout / BN)
+  int chunks_per_frame;     // ceil(HoWo / 64)
+  long long total_chunks;   // N * Do * chunks_per_frame
+  int splits;               // chunk ranges per (tap block, co tile)
+  int num_units;
+  int stages;
+  uint32_t tmem_cols;
+  uint32_t idesc;
+  float* dw;                // [Cout][taps][Cin] fp32, accumulated
+  int* status;
+  unsigned long long timeout_ns;
+};
+
+constexpr int WG_PIX = 64;                          // pixels (K) per stage
+constexpr int WG_A_BYTES = 2 * WG_PIX * 64 * 2;     // two 64-channel im2col boxes
+
+// Shared-memory matrix descriptor for an MN-major operand in 64-element x
+// 8-row atoms with the 128-byte swizzle: leading byte offset = distance of
+// consecutive 64-element blocks along M/N, stride byte offset = distance of
+// consecutive 8-row groups along K, version 1, layout type 2.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t mn_block_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>((mn_block_bytes >> 4) & 0x3FFF) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+__device__ __forceinline__ int wg_source_frame(const WgradParams& p, int to, int it) {
+  const int f = to * p.st + it - p.pf;
+  if (f < 0) return p.tpad == 1 ? 0 : -1;
+  return f < p.D ? f : -1;
+}
+
+struct WgUnit {
+  int tap, cb, co0;
+  long long c_begin, c_end;
+};
+
+__device__ __forceinline__ WgUnit wg_decode(const WgradParams& p, int u) {
+  WgUnit r;
+  const int split = u % p.splits;
+  const int rest = u / p.splits;
+  const int cot = rest % p.co_tiles;
+  const int mb = rest / p.co_tiles;
+  r.tap = mb / p.cblocks;
+  r.cb = mb - r.tap * p.cblocks;
+  r.co0 = cot * p.BN;
+  const long long per = (p.total_chunks + p.splits - 1) / p.splits;
+  r.c_begin = static_cast<long long>(split) * per;
+  r.c_end = r.c_begin + per < p.total_chunks ? r.c_begin + per : p.total_chunks;
+  return r;
+}
+
+template <bool kBF16>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    conv3d_wgrad_kernel(const __grid_constant__ CUtensorMap map_x,
+                        const __grid_constant__ CUtensorMap map_dy, const WgradParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t s_tmem_base;
+  __shared__ int s_abort;
+  const uint32_t warp = threadIdx.x / 32;
+  const uint32_t lane = threadIdx.x % 32;
+
+  const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  const uint32_t b_stage_bytes = static_cast<uint32_t>(p.BN) * WG_PIX * 2;
+  const uint32_t a_ring = base;
+  const uint32_t b_ring = a_ring + p.stages * WG_A_BYTES;
+  const uint32_t bars = b_ring + p.stages * b_stage_bytes;
+  const uint32_t full_bar = bars;
+  const uint32_t empty_bar = bars + 8 * p.stages;
+  const uint32_t tfull_bar = bars + 16 * p.stages;
+  const uint32_t tempty_bar = tfull_bar + 16;
+  const uint32_t drain_bar = tempty_bar + 16;
+  SharedCtl ctl{&s_abort, p.status, p.timeout_ns};
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(full_bar + 8 * s, 1);
+      mbar_init(empty_bar + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar + 8 * a, 1);
+      mbar_init(tempty_bar + 8 * a, 4);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+    prefetch_tensormap(&map_x);
+    prefetch_tensormap(&map_dy);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&s_tmem_base), p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = s_tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint32_t tx_bytes = WG_A_BYTES + b_stage_bytes;
+      uint32_t stage = 0, phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        const WgUnit wu = wg_decode(p, u);
+        const int it = wu.tap / (p.kh * p.kw);
+        const int ih = (wu.tap / p.kw) % p.kh;
+        const int iw = wu.tap % p.kw;
+        for (long long c = wu.c_begin; ok && c < wu.c_end; ++c) {
+          const long long fo = c / p.chunks_per_frame;
+          const int p0 = static_cast<int>(c - fo * p.chunks_per_frame) * WG_PIX;
+          const int n = static_cast<int>(fo / p.Do);
+          const int to = static_cast<int>(fo - static_cast<long long>(n) * p.Do);
+          const int f = wg_source_frame(p, to, it);
+          if (f < 0) continue;
+          if (!wait_bounded(empty_bar + 8 * stage, phase ^ 1, ctl, true)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full_bar + 8 * stage;
+          mbar_arrive_expect_tx(fb, tx_bytes);
+          const int ho0 = p0 / p.Wo;
+          const int wo0 = p0 - ho0 * p.Wo;
+          const int img = n * p.D + f;
+          // A box whose channels all lie past Cin (or past Cout for dy) is loaded
+          // from the block's first chunk instead: those rows/columns of the
+          // product are never written out, and every copy starts in bounds.
+          for (int j = 0; j < 2; ++j) {
+            int c0 = (2 * wu.cb + j) * 64;
+            if (c0 >= p.Cin) c0 = 2 * wu.cb * 64;
+            tma_load_im2col_4d(a_ring + stage * WG_A_BYTES + j * (WG_PIX * 128), &map_x, fb, c0,
+                               wo0 * p.sw - p.pw, ho0 * p.sh - p.ph, img,
+                               static_cast<uint16_t>(iw), static_cast<uint16_t>(ih));
+          }
+          for (int j = 0; j < p.BN / 64; ++j) {
+            int c0 = wu.co0 + 64 * j;
+            if (c0 >= p.Cout) c0 = wu.co0;
+            tma_load_3d(b_ring + stage * b_stage_bytes + j * (WG_PIX * 128), &map_dy, fb, c0, p0,
+                        static_cast<int>(fo));
+          }
+          ++issued;
+          if (++stage == static_cast<uint32_t>(p.stages)) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        const long long first = issued > p.stages ? issued - p.stages : 0;
+        for (long long i = first; i < issued; ++i)
+          wait_bounded(full_bar + 8 * static_cast<uint32_t>(i % p.stages),
+                       static_cast<uint32_t>((i / p.stages) & 1), ctl, false);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      int local = 0;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++local) {
+        const WgUnit wu = wg_decode(p, u);
+        const int it = wu.tap / (p.kh * p.kw);
+        const uint32_t acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!wait_bounded(tempty_bar + 8 * acc, acc_phase ^ 1, ctl, true)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * static_cast<uint32_t>(p.BN);
+        bool first = true;
+        for (long long c = wu.c_begin; c < wu.c_end; ++c) {
+          const long long fo = c / p.chunks_per_frame;
+          const int n = static_cast<int>(fo / p.Do);
+          const int to = static_cast<int>(fo - static_cast<long long>(n) * p.Do);
+          if (wg_source_frame(p, to, it) < 0) continue;
+          if (!wait_bounded(full_bar + 8 * stage, phase, ctl, true)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = a_ring + stage * WG_A_BYTES;
+          const uint32_t b0 = b_ring + stage * b_stage_bytes;
+#pragma unroll
+          for (int k = 0; k < WG_PIX / 16; ++k) {
+            // 16 pixels = two 8-row groups further along K
+            const uint64_t da = smem_desc_mn_sw128(a0 + k * 2048, WG_PIX * 128);
+            const uint64_t db = smem_desc_mn_sw128(b0 + k * 2048, WG_PIX * 128);
+            mma_f16_ss(d_tmem, da, db, p.idesc, first ? 0u : 1u);
+            first = false;
+          }
+          mma_commit(empty_bar + 8 * stage);
+          if (++stage == static_cast<uint32_t>(p.stages)) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit(tfull_bar + 8 * acc);
+      }
+      mma_commit(drain_bar);
+      wait_bounded(drain_bar, 0, ctl, false);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // Thread = one (tap, ci) row of the unit (TMEM lane); 32 output channels
+    // per TMEM load; fp32 atomic adds into dw[co][tap][ci].
+    const uint32_t quarter = warp & 3;
+    int local = 0;
+    const long long K = static_cast<long long>(p.taps) * p.Cin;
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++local) {
+      const uint32_t acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!wait_bounded(tfull_bar + 8 * acc, acc_phase, ctl, true)) break;
+      tc_fence_after();
+      const WgUnit wu = wg_decode(p, u);
+      const int it = wu.tap / (p.kh * p.kw);
+      // a unit whose chunks all read zero padding issued no MMA: nothing to add
+      bool any = false;
+      for (long long c = wu.c_begin; c < wu.c_end && !any; ++c) {
+        const long long fo = c / p.chunks_per_frame;
+        const int n = static_cast<int>(fo / p.Do);
+        any = wg_source_frame(p, static_cast<int>(fo - static_cast<long long>(n) * p.Do), it) >= 0;
+      }
+      const int ci = wu.cb * 128 + static_cast<int>(quarter * 32 + lane);
+      const bool row_ok = any && ci < p.Cin;
+      const uint32_t t_row =
+          tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.BN);
+      for (int j = 0; j < p.BN / 32; ++j) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + j * 32, r);
+        tmem_ld_wait();
+        if (row_ok) {
+          for (int e = 0; e < 32; ++e) {
+            const int co = wu.co0 + j * 32 + e;
+            if (co < p.Cout)
+              atomicAdd(p.dw + static_cast<long long>(co) * K + static_cast<long long>(wu.tap) * p.Cin + ci,
+                        __uint_as_float(r[e]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar + 8 * acc);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+// fp32 accumulation -> the 16-bit weight gradient (one rounding).
+template <bool kBF16>
+__global__ void f32_to_16_kernel(const float* __restrict__ src, uint16_t* __restrict__ dst,
+                                 long long n) {
+  using C = Cvt<kBF16>;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    dst[i] = static_cast<uint16_t>(C::pack(src[i], 0.0f) & 0xFFFFu);
+}
+
+// dbias[co] += sum over pixels of dy[m, co]: 8 channels per thread, fp32
+// partial sums over a slab of pixels, one atomic per channel and thread.
+template <bool kBF16>
+__global__ void bias_grad_kernel(const uint16_t* __restrict__ dy, float* __restrict__ db,
+                                 long long pixels, int Cout, long long pixels_per_block) {
+  using C = Cvt<kBF16>;
+  const int vecs = Cout / 8;
+  const int rows = blockDim.x / vecs;
+  const int v = threadIdx.x % vecs;
+  const int r = threadIdx.x / vecs;
+  if (r >= rows) return;
+  const long long p_begin = blockIdx.x * pixels_per_block;
+  long long p_end = p_begin + pixels_per_block;
+  if (p_end > pixels) p_end = pixels;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (long long p = p_begin + r; p < p_end; p += rows) {
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(dy + p * Cout + 8 * v));
+    acc[0] += C::lo(q.x); acc[1] += C::hi(q.x); acc[2] += C::lo(q.y); acc[3] += C::hi(q.y);
+    acc[4] += C::lo(q.z); acc[5] += C::hi(q.z); acc[6] += C::lo(q.w); acc[7] += C::hi(q.w);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) atomicAdd(db + 8 * v + j, acc[j]);
+}
+
+}  // namespace conv3d
