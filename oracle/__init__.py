@@ -72,6 +72,10 @@ def _load():
         lib.oracle_conv3d_backward_f64.argtypes = (
             [u16p, u16p, u16p, ctypes.c_int] + [ctypes.c_int] * 16
             + [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p])
+        for fn in (lib.oracle_conv3d_dx_at_f64, lib.oracle_conv3d_dw_at_f64):
+            fn.restype = ctypes.c_int
+            fn.argtypes = ([u16p, u16p, ctypes.c_int] + [ctypes.c_int] * 16
+                           + [i64p, ctypes.c_int64, ctypes.c_void_p])
         lib.oracle_groupnorm_silu_f64.restype = ctypes.c_int
         lib.oracle_groupnorm_silu_f64.argtypes = (
             [u16p, u16p, u16p] + [ctypes.c_int] * 8 + [ctypes.c_double, ctypes.c_int, ctypes.c_void_p])
@@ -190,3 +194,40 @@ def conv3d_backward(x_bits, w_bits, dy_bits, dtype, kernel, stride, pad, tpad):
     if rc != 0:
         raise ValueError("oracle rejected the problem")
     return dx, dw, db
+
+
+def conv3d_dx_at(w_bits, dy_bits, dtype, x_shape, kernel, stride, pad, tpad, pixels):
+    """fp64 dx at the given flat input pixels ((n*D + f)*H + h)*W + w: [len, Cin]."""
+    w_bits = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    dy_bits = np.ascontiguousarray(dy_bits, dtype=np.uint16)
+    N, D, H, W, Cin = x_shape
+    Cout = w_bits.shape[0]
+    if dy_bits.shape != (N, *output_shape(D, H, W, kernel, stride, pad, tpad), Cout):
+        raise ValueError("dy shape")
+    pixels = np.ascontiguousarray(pixels, dtype=np.int64)
+    out = np.empty((pixels.size, Cin), dtype=np.float64)
+    rc = _load().oracle_conv3d_dx_at_f64(
+        w_bits.ctypes.data, dy_bits.ctypes.data, dtype, N, Cin, D, H, W, Cout, *kernel, *stride,
+        *pad, tpad, pixels.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), pixels.size,
+        out.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle rejected the problem")
+    return out
+
+
+def conv3d_dw_at(x_bits, dy_bits, dtype, Cout, kernel, stride, pad, tpad, entries):
+    """fp64 dw at the given flat indices into [Cout, kt, kh, kw, Cin]: [len]."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    dy_bits = np.ascontiguousarray(dy_bits, dtype=np.uint16)
+    N, D, H, W, Cin = x_bits.shape
+    if dy_bits.shape != (N, *output_shape(D, H, W, kernel, stride, pad, tpad), Cout):
+        raise ValueError("dy shape")
+    entries = np.ascontiguousarray(entries, dtype=np.int64)
+    out = np.empty(entries.size, dtype=np.float64)
+    rc = _load().oracle_conv3d_dw_at_f64(
+        x_bits.ctypes.data, dy_bits.ctypes.data, dtype, N, Cin, D, H, W, Cout, *kernel, *stride,
+        *pad, tpad, entries.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), entries.size,
+        out.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle rejected the problem")
+    return out

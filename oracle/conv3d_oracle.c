@@ -288,3 +288,113 @@ int oracle_conv3d_backward_f64(const uint16_t* x, const uint16_t* w, const uint1
         }
   return 0;
 }
+
+/*
+ * The same two adjoints, evaluated one element at a time for large problems
+ * whose full backward the serial loop above cannot finish quickly.  Each
+ * element is the plain sum that defines it, over every forward product it
+ * receives:
+ *   dx[n,f,hi,wi,ci] = sum over (to, it, ih, iw, co) with src(to,it) == f,
+ *                      to*st+it-pf mapped by the padding rule, ho*sh+ih-ph == hi
+ *                      and wo*sw+iw-pw == wi, of dy[n,to,ho,wo,co] * w[co,it,ih,iw,ci];
+ *   dw[co,it,ih,iw,ci] = sum over (n, to, ho, wo) whose tap reads a real pixel
+ *                      of dy[n,to,ho,wo,co] * x[n, src(to,it), ho*sh+ih-ph, wo*sw+iw-pw, ci].
+ * pixels: flat input-pixel indices ((n*D + f)*H + hi)*W + wi; dx_out [n_pix][Cin].
+ * entries: flat indices into dw [Cout,kt,kh,kw,Cin]; dw_out [n_entries].
+ * Elements are independent, so the loops over them run in parallel threads.
+ */
+static int oracle_source_frame(int to, int it, int st, int pf, int D, int tpad_mode) {
+  int f = to * st + it - pf;
+  if (f < 0) {
+    if (tpad_mode != 1) return -1;
+    f = 0;
+  }
+  return f < D ? f : -1;
+}
+
+int oracle_conv3d_dx_at_f64(const uint16_t* w, const uint16_t* dy, int dtype, int N, int Cin,
+                            int D, int H, int W, int Cout, int kt, int kh, int kw, int st, int sh,
+                            int sw, int pt, int ph, int pw, int tpad_mode, const int64_t* pixels,
+                            int64_t n_pix, double* dx_out) {
+  int od[3];
+  if (tpad_mode < 0 || tpad_mode > 2) return -1;
+  if (oracle_output_shape(D, H, W, kt, kh, kw, st, sh, sw, pt, ph, pw, tpad_mode, od) != 0)
+    return -1;
+  const int Do = od[0], Ho = od[1], Wo = od[2];
+  const int pf = (tpad_mode == 0) ? pt : kt - 1;
+  for (int64_t q = 0; q < n_pix; ++q)
+    if (pixels[q] < 0 || pixels[q] >= (int64_t)N * D * H * W) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t q = 0; q < n_pix; ++q) {
+    const int64_t pix = pixels[q];
+    const int wi = (int)(pix % W);
+    const int hi = (int)((pix / W) % H);
+    const int f = (int)((pix / ((int64_t)W * H)) % D);
+    const int n = (int)(pix / ((int64_t)W * H * D));
+    double* acc = dx_out + q * Cin;
+    for (int ci = 0; ci < Cin; ++ci) acc[ci] = 0.0;
+    for (int to = 0; to < Do; ++to)
+      for (int it = 0; it < kt; ++it) {
+        if (oracle_source_frame(to, it, st, pf, D, tpad_mode) != f) continue;
+        for (int ih = 0; ih < kh; ++ih) {
+          const int hs = hi + ph - ih;           /* = ho * sh */
+          if (hs < 0 || hs % sh != 0 || hs / sh >= Ho) continue;
+          const int ho = hs / sh;
+          for (int iw = 0; iw < kw; ++iw) {
+            const int ws = wi + pw - iw;         /* = wo * sw */
+            if (ws < 0 || ws % sw != 0 || ws / sw >= Wo) continue;
+            const int wo = ws / sw;
+            const int64_t m = (((int64_t)n * Do + to) * Ho + ho) * Wo + wo;
+            for (int co = 0; co < Cout; ++co) {
+              const double g = oracle_decode(dy[m * Cout + co], dtype);
+              const int64_t wo_ = ((((int64_t)co * kt + it) * kh + ih) * kw + iw) * Cin;
+              for (int ci = 0; ci < Cin; ++ci) acc[ci] += g * oracle_decode(w[wo_ + ci], dtype);
+            }
+          }
+        }
+      }
+  }
+  return 0;
+}
+
+int oracle_conv3d_dw_at_f64(const uint16_t* x, const uint16_t* dy, int dtype, int N, int Cin,
+                            int D, int H, int W, int Cout, int kt, int kh, int kw, int st, int sh,
+                            int sw, int pt, int ph, int pw, int tpad_mode, const int64_t* entries,
+                            int64_t n_entries, double* dw_out) {
+  int od[3];
+  if (tpad_mode < 0 || tpad_mode > 2) return -1;
+  if (oracle_output_shape(D, H, W, kt, kh, kw, st, sh, sw, pt, ph, pw, tpad_mode, od) != 0)
+    return -1;
+  const int Do = od[0], Ho = od[1], Wo = od[2];
+  const int pf = (tpad_mode == 0) ? pt : kt - 1;
+  for (int64_t q = 0; q < n_entries; ++q)
+    if (entries[q] < 0 || entries[q] >= (int64_t)Cout * kt * kh * kw * Cin) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t q = 0; q < n_entries; ++q) {
+    int64_t e = entries[q];
+    const int ci = (int)(e % Cin); e /= Cin;
+    const int iw = (int)(e % kw); e /= kw;
+    const int ih = (int)(e % kh); e /= kh;
+    const int it = (int)(e % kt);
+    const int co = (int)(e / kt);
+    double acc = 0.0;
+    for (int n = 0; n < N; ++n)
+      for (int to = 0; to < Do; ++to) {
+        const int f = oracle_source_frame(to, it, st, pf, D, tpad_mode);
+        if (f < 0) continue;
+        for (int ho = 0; ho < Ho; ++ho) {
+          const int hi = ho * sh + ih - ph;
+          if (hi < 0 || hi >= H) continue;
+          for (int wo = 0; wo < Wo; ++wo) {
+            const int wi = wo * sw + iw - pw;
+            if (wi < 0 || wi >= W) continue;
+            const int64_t m = (((int64_t)n * Do + to) * Ho + ho) * Wo + wo;
+            const int64_t xo = ((((int64_t)n * D + f) * H + hi) * W + wi) * Cin + ci;
+            acc += oracle_decode(dy[m * Cout + co], dtype) * oracle_decode(x[xo], dtype);
+          }
+        }
+      }
+    dw_out[q] = acc;
+  }
+  return 0;
+}

@@ -93,3 +93,31 @@ def test_causal_replicate_sends_front_gradients_to_frame_zero():
     dxe, _, _ = oracle.conv3d_backward(ext, wb, gb, BF16, k, (1, 1, 1), (0, 1, 1), ZERO)
     np.testing.assert_allclose(dx[:, 0], dxe[:, :3].sum(axis=1), rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(dx[:, 1:], dxe[:, 3:], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_elementwise_adjoints_match_torch_autograd(case):
+    """The per-element gather forms (used at sizes the serial scatter cannot
+    finish) against float64 autograd, on every element, and against the
+    scatter form."""
+    (N, Cin, D, H, W, Cout), k, stride, pad, tpad = case
+    xb, wb, gb = problem(N, Cin, D, H, W, Cout, k, stride, pad, tpad, seed=11)
+    tdx, tdw = torch_grads(dec(xb), dec(wb), dec(gb), k, stride, pad, tpad)
+    pixels = np.arange(N * D * H * W)
+    dx = oracle.conv3d_dx_at(wb, gb, BF16, xb.shape, k, stride, pad, tpad, pixels)
+    np.testing.assert_allclose(dx, tdx.reshape(-1, Cin), rtol=1e-10, atol=1e-10)
+    entries = np.arange(wb.size)[::-1].copy()          # any order
+    dw = oracle.conv3d_dw_at(xb, gb, BF16, Cout, k, stride, pad, tpad, entries)
+    np.testing.assert_allclose(dw, tdw.reshape(-1)[entries], rtol=1e-10, atol=1e-10)
+    sdx, sdw, _ = oracle.conv3d_backward(xb, wb, gb, BF16, k, stride, pad, tpad)
+    np.testing.assert_allclose(dx, sdx.reshape(-1, Cin), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dw, sdw.reshape(-1)[entries], rtol=1e-12, atol=1e-12)
+
+
+def test_elementwise_adjoints_reject_bad_indices():
+    xb, wb, gb = problem(1, 2, 3, 4, 4, 2, (3, 3, 3), (1, 1, 1), (1, 1, 1), ZERO, seed=1)
+    with pytest.raises(ValueError):
+        oracle.conv3d_dx_at(wb, gb, BF16, xb.shape, (3, 3, 3), (1, 1, 1), (1, 1, 1), ZERO,
+                            [1 * 3 * 4 * 4])
+    with pytest.raises(ValueError):
+        oracle.conv3d_dw_at(xb, gb, BF16, 2, (3, 3, 3), (1, 1, 1), (1, 1, 1), ZERO, [-1])
