@@ -494,6 +494,191 @@ def cpu_baseline(wl, p):
             "sample": f"{n} random output pixels (all {wl.Cout} channels) of {M}, {dt:.1f} s"}
 
 
+# ---------------------------------------------------------------- backward passes
+
+def run_backward(args, wl, rank, world, local_rank):
+    """dx (``--pass dgrad``) or dw + dbias (``--pass wgrad``) of one workload per
+    step, through the C ABI.  Algorithmic FLOPs are the forward's: the backward
+    passes form the same products.  One call launches several kernels (weight
+    transform / clear, the tcgen05 GEMM, fold / conversion), so the roofline
+    figure divides by the whole call's time and is a lower bound for the GEMM."""
+    import video_vae_convolution_implicit_b200 as c3
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dt = TORCH_DTYPE[wl.dtype]
+    Do, Ho, Wo = out_shape(wl)
+    seed = rank_seed(wl, rank)
+    p = si.conv3d_problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, (Do, Ho, Wo), seed,
+                          dt, True, False, dev)
+    dy = si.tensor((wl.N, Do, Ho, Wo, wl.Cout), seed, 5, 1.0, dt, dev)
+    x_shape = (wl.N, wl.D, wl.H, wl.W, wl.Cin)
+    dtc = c3.BF16 if wl.dtype == "bf16" else c3.F16
+    if args.pass_ == "dgrad":
+        ws_bytes = c3.bwd_data_workspace_bytes(*x_shape[:1], wl.Cin, wl.D, wl.H, wl.W, wl.Cout,
+                                               wl.kernel, wl.pad, wl.tpad)
+        out = torch.empty(x_shape, dtype=dt, device=dev)
+        db = None
+    else:
+        ws_bytes = c3.bwd_weight_workspace_bytes(wl.Cin, wl.Cout, wl.kernel)
+        out = torch.empty((wl.Cout, *wl.kernel, wl.Cin), dtype=dt, device=dev)
+        db = torch.empty((wl.Cout,), dtype=dt, device=dev)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+
+    def step():
+        if args.pass_ == "dgrad":
+            st = c3.conv3d_bwd_data_ptr(dy.data_ptr(), p["w"].data_ptr(), out.data_ptr(),
+                                        *x_shape[:1], wl.Cin, wl.D, wl.H, wl.W, wl.Cout,
+                                        wl.kernel, wl.stride, wl.pad, wl.tpad, dtc,
+                                        ws.data_ptr(), ws.numel(), sh)
+        else:
+            st = c3.conv3d_bwd_weight_ptr(p["x"].data_ptr(), dy.data_ptr(), out.data_ptr(),
+                                          db.data_ptr(), wl.N, wl.Cin, wl.D, wl.H, wl.W,
+                                          wl.Cout, wl.kernel, wl.stride, wl.pad, wl.tpad, dtc,
+                                          ws.data_ptr(), ws.numel(), sh)
+        if st != c3.Status.OK:
+            raise RuntimeError(f"backward call failed: {c3.status_string(st)}")
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if c3.poll_status(stream) != c3.Status.OK:
+        raise RuntimeError("device status after warm-up is not OK")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    max_ms = max_over_ranks(sum(step_ms), dev)
+    status = c3.poll_status(stream)
+    flops = algorithmic_flops(wl)
+    value = whole_job_tflops(flops, world, args.steps, max_ms)
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (statistics.mean(step_ms) * 1e-3) / 1e12
+    rep = wl.tpad == 1 and wl.kernel[0] > 1
+    if args.pass_ == "dgrad":
+        launches = 2 + (1 if rep else 0)       # weight transform, GEMM, front-frame fold
+        kernel = "conv3d_implicit_gemm_kernel (dgrad: transposed convolution of dy)"
+    else:
+        launches = 3 + 1                       # clear, GEMM, dw rounding, bias column sums
+        kernel = "conv3d_wgrad_kernel"
+    line = {
+        "metric": f"conv3d backward {args.pass_} TFLOPS (forward-equivalent FLOPs)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded SplitMix64 normals; dy stream 5)",
+        "config": dict(describe(wl, world), direction=args.pass_, residual=False,
+                       l2="flushed (2x L2 write) between timed steps"),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_kind} bf16_tflops (burst)", "kernel": kernel,
+                     "timed": "whole call (all its launches): a lower bound for the GEMM",
+                     "algorithmic_flops_per_launch": flops},
+        "gpu_launches": launches * args.steps,
+        "clocks": clocks.summary(),
+        "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms),
+                    "max": max(step_ms)},
+        "device_status": c3.status_string(status),
+    }
+    if rank == 0:
+        line["parity"] = backward_parity(args.pass_, wl, p, dy, out, db)
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = backward_cpu_baseline(args.pass_, wl, p, dy, flops)
+        print(json.dumps(line), flush=True)
+    ok = status == c3.Status.OK and (rank != 0 or line["parity"]["ok"])
+    return 0 if ok else 1
+
+
+def _backward_samples(which, wl, n, seed):
+    rng = np.random.default_rng(seed)
+    if which == "dgrad":
+        total = wl.N * wl.D * wl.H * wl.W
+        fixed = [0, wl.W - 1, wl.H * wl.W - 1, total - 1]      # corners, first / last frame
+    else:
+        total = wl.Cout * wl.kernel[0] * wl.kernel[1] * wl.kernel[2] * wl.Cin
+        fixed = [0, total - 1]
+    idx = set(fixed) | {int(v) for v in rng.integers(0, total, n)}
+    return np.array(sorted(idx), dtype=np.int64), total
+
+
+def _oracle_backward_at(which, wl, hb, dy_bits, idx):
+    import oracle
+    dt = oracle.BF16 if wl.dtype == "bf16" else oracle.F16
+    if which == "dgrad":
+        return oracle.conv3d_dx_at(hb["w"], dy_bits, dt, (wl.N, wl.D, wl.H, wl.W, wl.Cin),
+                                   wl.kernel, wl.stride, wl.pad, wl.tpad, idx)
+    return oracle.conv3d_dw_at(hb["x"], dy_bits, dt, wl.Cout, wl.kernel, wl.stride, wl.pad,
+                               wl.tpad, idx)
+
+
+def backward_parity(which, wl, p, dy, out, db):
+    """Sampled elements of dx (whole pixels, all channels) or dw (single
+    entries) and the whole dbias against the oracle's per-element sums."""
+    hb = host_bits(p)
+    dyb = si.bits(dy)
+    idx, _ = _backward_samples(which, wl, 48 if which == "dgrad" else 256, 4321)
+    ref = _oracle_backward_at(which, wl, hb, dyb, idx)
+    flat = out.view(-1, wl.Cin) if which == "dgrad" else out.view(-1)
+    got = flat[torch.from_numpy(idx).to(out.device)].double().cpu().numpy()
+    errs = [np.abs(got - ref)]
+    refs = [ref]
+    if db is not None:
+        import oracle
+        ref_db = oracle.decode16(dyb, oracle.BF16 if wl.dtype == "bf16" else oracle.F16)
+        ref_db = ref_db.reshape(-1, wl.Cout).sum(axis=0)
+        errs.append(np.abs(db.double().cpu().numpy() - ref_db))
+        refs.append(ref_db)
+    res = {"samples": int(idx.size), "what": "dx pixels" if which == "dgrad" else "dw entries"}
+    ok = bool(np.isfinite(got).all())
+    for name, e, r in zip(("", "dbias_"), errs, refs):
+        mr = float(e.max() / np.abs(r).max())
+        rl = float(e.sum() / np.abs(r).sum())
+        res[name + "max_err_over_max_ref"] = mr
+        res[name + "rel_l1"] = rl
+        ok = ok and mr <= 1e-2 and rl <= 2e-3
+    res["ok"] = ok
+    return res
+
+
+def backward_cpu_baseline(which, wl, p, dy, flops):
+    """The oracle's per-element sums on a bounded random sample, scaled to FLOPs
+    by the sampled fraction of the elements (every element of dw, or every
+    pixel of dx, carries on average total/elements of the work)."""
+    import oracle
+    hb = host_bits(p)
+    dyb = si.bits(dy)
+    seconds = float(os.environ.get("CONV3D_CPU_BASELINE_SECONDS", "15"))
+    n = 16
+    while True:
+        idx, total = _backward_samples(which, wl, n, 99)
+        t0 = time.perf_counter()
+        _oracle_backward_at(which, wl, hb, dyb, idx)
+        dt = time.perf_counter() - t0
+        if dt > seconds / 4 or idx.size >= total:
+            break
+        n = int(n * min(16.0, max(2.0, seconds / max(dt, 1e-3) / 2)))
+    value = flops * idx.size / total / dt / 1e12
+    what = "input pixels (all channels) of dx" if which == "dgrad" else "entries of dw"
+    return {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{idx.size} random {what} of {total}, {dt:.1f} s"}
+
+
 # ---------------------------------------------------------------- GroupNorm + SiLU workloads
 
 def run_norm(args, wl, rank, world, local_rank):
@@ -599,6 +784,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="cfg2", choices=sorted(WORKLOADS) + sorted(NORM_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "dgrad", "wgrad"],
+                    help="forward convolution (default) or one of its backward passes")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -626,7 +813,11 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        rc = (run_norm if is_norm else run_ours)(args, wl, rank, world, local_rank)
+        if is_norm:
+            fn = run_norm
+        else:
+            fn = run_ours if args.pass_ == "fwd" else run_backward
+        rc = fn(args, wl, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -87,3 +87,54 @@ def test_bwd_weight_every_element(case):
                                                pad, tpad)
     assert_close(dw.double().cpu().numpy(), ref_dw, "dw " + str(case))
     assert_close(db.double().cpu().numpy(), ref_db, "dbias " + str(case))
+
+
+# ------------------------------------------------------ full-size workloads, sampled
+
+from seeded_inputs.workloads import WORKLOADS  # noqa: E402
+
+FULL = ["cfg2", "cfg3", "cfg4s", "cfg5c", "cfg5d", "cfg2s"]
+
+
+def _full_problem(name):
+    wl = WORKLOADS[name]
+    x, w, dy, od = grads_problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, wl.pad,
+                                 wl.tpad, wl.seed, wl.dtype, wl.stride)
+    return wl, x, w, dy, od
+
+
+@pytest.mark.parametrize("name", [n for n in FULL if WORKLOADS[n].stride == (1, 1, 1)])
+def test_bwd_data_full_size_sampled(name):
+    import numpy as np
+    wl, x, w, dy, od = _full_problem(name)
+    dx = c3.conv3d_bwd_data(dy, w, x.shape, wl.pad, wl.tpad)
+    assert c3.poll_status() == c3.Status.OK
+    total = wl.N * wl.D * wl.H * wl.W
+    HW = wl.H * wl.W
+    rng = np.random.default_rng(5)
+    pix = {0, wl.W - 1, HW - 1, HW // 2 + wl.W // 2, total - 1, (wl.D - 1) * HW}
+    pix |= {int(v) for v in rng.integers(0, total, 40)}
+    pix = np.array(sorted(pix), dtype=np.int64)
+    ref = oracle.conv3d_dx_at(si.bits(w), si.bits(dy), od, x.shape, wl.kernel, wl.stride, wl.pad,
+                              wl.tpad, pix)
+    got = dx.view(-1, wl.Cin)[torch.from_numpy(pix).cuda()].double().cpu().numpy()
+    assert_close(got, ref, name)
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_bwd_weight_full_size_sampled(name):
+    import numpy as np
+    wl, x, w, dy, od = _full_problem(name)
+    dw, db = c3.conv3d_bwd_weight(x, dy, wl.kernel, wl.stride, wl.pad, wl.tpad)
+    assert c3.poll_status() == c3.Status.OK
+    total = dw.numel()
+    rng = np.random.default_rng(6)
+    ent = {0, total - 1, wl.Cin - 1, total - wl.Cin}
+    ent |= {int(v) for v in rng.integers(0, total, 200)}
+    ent = np.array(sorted(ent), dtype=np.int64)
+    ref = oracle.conv3d_dw_at(si.bits(x), si.bits(dy), od, wl.Cout, wl.kernel, wl.stride, wl.pad,
+                              wl.tpad, ent)
+    got = dw.view(-1)[torch.from_numpy(ent).cuda()].double().cpu().numpy()
+    assert_close(got, ref, name + " dw")
+    ref_db = oracle.decode16(si.bits(dy), od).reshape(-1, wl.Cout).sum(axis=0)
+    assert_close(db.double().cpu().numpy(), ref_db, name + " dbias")
