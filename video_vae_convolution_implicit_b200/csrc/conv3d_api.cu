@@ -873,6 +873,30 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
   return CONV3D_OK;
 }
 
+// Number of pixel ranges each (tap block, output-channel tile) is split into.
+// The persistent grid runs units in rounds of `sms`; the cost of a choice is
+// the chunks one CTA walks (rounds x chunks per unit) plus a fixed cost per
+// unit for its epilogue (fp32 atomics of a 128 x BN block, about the time of
+// eight chunks).  The cheapest split wins; ties go to fewer splits.
+long long choose_wgrad_splits(long long base_units, long long total_chunks, int sms) {
+  constexpr long long kEpilogueChunks = 8;
+  long long best = 1;
+  long long best_cost = -1;
+  const long long max_splits = total_chunks < 1024 ? total_chunks : 1024;
+  for (long long s = 1; s <= max_splits; ++s) {
+    const long long units = base_units * s;
+    const long long rounds = (units + sms - 1) / sms;
+    const long long per = (total_chunks + s - 1) / s;
+    const long long cost = rounds * (per + kEpilogueChunks);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+    if (rounds > 64) break;
+  }
+  return best;
+}
+
 size_t conv3d_bwd_weight_workspace_bytes(int Cin, int Cout, const int kernel[3]) {
   if (!kernel || Cin < 1 || Cout < 1) return 0;
   const size_t dw = static_cast<size_t>(Cout) * kernel[0] * kernel[1] * kernel[2] * Cin * 4;
@@ -942,9 +966,7 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   wp.chunks_per_frame = (wp.HoWo + WG_PIX - 1) / WG_PIX;
   wp.total_chunks = static_cast<long long>(N) * F.Do * wp.chunks_per_frame;
   const long long base_units = static_cast<long long>(wp.taps) * wp.cblocks * wp.co_tiles;
-  long long splits = (2LL * S->num_sms + base_units - 1) / base_units;
-  if (splits > wp.total_chunks / 4) splits = wp.total_chunks / 4;
-  if (splits < 1) splits = 1;
+  const long long splits = choose_wgrad_splits(base_units, wp.total_chunks, S->num_sms);
   if (base_units * splits > 0x7FFFFFFFLL) {
     set_error("problem too large");
     return CONV3D_ERR_UNSUPPORTED;
@@ -1009,18 +1031,21 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dw conversion launch");
   }
   if (dbias) {
+    // channel groups of up to 2048 along y; about four blocks per SM in all,
+    // the pixels split evenly between the blocks of a group
     const long long pixels = static_cast<long long>(N) * F.Do * F.Ho * F.Wo;
-    const int vecs = Cout / 8;
-    int rows = 256 / vecs;
-    if (rows < 1) rows = 1;
-    const int threads = vecs * rows > 1024 ? 1024 : vecs * rows;
-    const long long per = 1024;
-    const long long blocks = (pixels + per - 1) / per;
+    const int groups = (Cout + BIAS_CHANNELS - 1) / BIAS_CHANNELS;
+    long long blocks = (4LL * S->num_sms + groups - 1) / groups;
+    long long per = (pixels + blocks - 1) / blocks;
+    if (per < 64) per = 64;
+    blocks = (pixels + per - 1) / per;
+    const dim3 grid(static_cast<unsigned>(blocks), static_cast<unsigned>(groups));
+    const size_t part_bytes = BIAS_THREADS * 8 * sizeof(float);
     if (bf16)
-      bias_grad_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+      bias_grad_kernel<true><<<grid, BIAS_THREADS, part_bytes, stream>>>(
           static_cast<const uint16_t*>(dy), db32, pixels, Cout, per);
     else
-      bias_grad_kernel<false><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+      bias_grad_kernel<false><<<grid, BIAS_THREADS, part_bytes, stream>>>(
           static_cast<const uint16_t*>(dy), db32, pixels, Cout, per);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dbias launch");
     if (bf16)

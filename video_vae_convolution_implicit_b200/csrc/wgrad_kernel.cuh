@@ -87,9 +87,45 @@ __device__ __forceinline__ WgUnit wg_decode(const WgradParams& p, int u) {
   r.co0 = cot * p.BN;
   const long long per = (p.total_chunks + p.splits - 1) / p.splits;
   r.c_begin = static_cast<long long>(split) * per;
+  if (r.c_begin > p.total_chunks) r.c_begin = p.total_chunks;
   r.c_end = r.c_begin + per < p.total_chunks ? r.c_begin + per : p.total_chunks;
   return r;
 }
+
+// Walks a unit's chunk range one output frame at a time: each step yields the
+// frame (fo = n*Do + to), the first chunk in it and how many chunks of the
+// range it holds.  One division per unit; none per chunk (the issuing threads
+// are single threads whose per-chunk cost must stay well under one stage's
+// MMA time).
+struct FrameWalk {
+  long long fo, left;
+  int n, to, pc, count;
+
+  __device__ __forceinline__ FrameWalk(const WgradParams& p, const WgUnit& u) {
+    fo = u.c_begin / p.chunks_per_frame;
+    pc = static_cast<int>(u.c_begin - fo * p.chunks_per_frame);
+    n = static_cast<int>(fo / p.Do);
+    to = static_cast<int>(fo - static_cast<long long>(n) * p.Do);
+    left = u.c_end - u.c_begin;
+    count = 0;
+  }
+  // Advances to the next frame segment; false once the range is exhausted.
+  __device__ __forceinline__ bool next(const WgradParams& p) {
+    if (count > 0) {
+      left -= count;
+      pc = 0;
+      ++fo;
+      if (++to == p.Do) {
+        to = 0;
+        ++n;
+      }
+    }
+    if (left <= 0) return false;
+    const long long room = p.chunks_per_frame - pc;
+    count = static_cast<int>(left < room ? left : room);
+    return true;
+  }
+};
 
 template <bool kBF16>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -149,42 +185,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int it = wu.tap / (p.kh * p.kw);
         const int ih = (wu.tap / p.kw) % p.kh;
         const int iw = wu.tap % p.kw;
-        for (long long c = wu.c_begin; ok && c < wu.c_end; ++c) {
-          const long long fo = c / p.chunks_per_frame;
-          const int p0 = static_cast<int>(c - fo * p.chunks_per_frame) * WG_PIX;
-          const int n = static_cast<int>(fo / p.Do);
-          const int to = static_cast<int>(fo - static_cast<long long>(n) * p.Do);
-          const int f = wg_source_frame(p, to, it);
-          if (f < 0) continue;
-          if (!wait_bounded(empty_bar + 8 * stage, phase ^ 1, ctl, true)) {
-            ok = false;
-            break;
-          }
-          const uint32_t fb = full_bar + 8 * stage;
-          mbar_arrive_expect_tx(fb, tx_bytes);
-          const int ho0 = p0 / p.Wo;
-          const int wo0 = p0 - ho0 * p.Wo;
-          const int img = n * p.D + f;
-          // A box whose channels all lie past Cin (or past Cout for dy) is loaded
-          // from the block's first chunk instead: those rows/columns of the
-          // product are never written out, and every copy starts in bounds.
-          for (int j = 0; j < 2; ++j) {
-            int c0 = (2 * wu.cb + j) * 64;
-            if (c0 >= p.Cin) c0 = 2 * wu.cb * 64;
-            tma_load_im2col_4d(a_ring + stage * WG_A_BYTES + j * (WG_PIX * 128), &map_x, fb, c0,
-                               wo0 * p.sw - p.pw, ho0 * p.sh - p.ph, img,
+        // A box whose channels all lie past Cin (or past Cout for dy) is loaded
+        // from the block's first chunk instead: those rows/columns of the
+        // product are never written out, and every copy starts in bounds.
+        const int xc0 = 2 * wu.cb * 64;
+        const int xc1 = xc0 + 64 < p.Cin ? xc0 + 64 : xc0;
+        FrameWalk fw(p, wu);
+        while (ok && fw.next(p)) {
+          const int f = wg_source_frame(p, fw.to, it);
+          if (f < 0) continue;                  // this tap reads zero padding here
+          const int img = fw.n * p.D + f;
+          int p0 = fw.pc * WG_PIX;
+          int ho0 = p0 / p.Wo;
+          int wo0 = p0 - ho0 * p.Wo;
+          for (int j = 0; j < fw.count; ++j) {
+            if (!wait_bounded(empty_bar + 8 * stage, phase ^ 1, ctl, true)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = full_bar + 8 * stage;
+            mbar_arrive_expect_tx(fb, tx_bytes);
+            const uint32_t a_dst = a_ring + stage * WG_A_BYTES;
+            const int wx = wo0 * p.sw - p.pw, hx = ho0 * p.sh - p.ph;
+            tma_load_im2col_4d(a_dst, &map_x, fb, xc0, wx, hx, img,
                                static_cast<uint16_t>(iw), static_cast<uint16_t>(ih));
-          }
-          for (int j = 0; j < p.BN / 64; ++j) {
-            int c0 = wu.co0 + 64 * j;
-            if (c0 >= p.Cout) c0 = wu.co0;
-            tma_load_3d(b_ring + stage * b_stage_bytes + j * (WG_PIX * 128), &map_dy, fb, c0, p0,
-                        static_cast<int>(fo));
-          }
-          ++issued;
-          if (++stage == static_cast<uint32_t>(p.stages)) {
-            stage = 0;
-            phase ^= 1;
+            tma_load_im2col_4d(a_dst + WG_PIX * 128, &map_x, fb, xc1, wx, hx, img,
+                               static_cast<uint16_t>(iw), static_cast<uint16_t>(ih));
+            const uint32_t b_dst = b_ring + stage * b_stage_bytes;
+            for (int q = 0; q < p.BN / 64; ++q) {
+              const int dc = wu.co0 + 64 * q < p.Cout ? wu.co0 + 64 * q : wu.co0;
+              tma_load_3d(b_dst + q * (WG_PIX * 128), &map_dy, fb, dc, p0,
+                          static_cast<int>(fw.fo));
+            }
+            ++issued;
+            if (++stage == static_cast<uint32_t>(p.stages)) {
+              stage = 0;
+              phase ^= 1;
+            }
+            p0 += WG_PIX;
+            wo0 += WG_PIX;
+            while (wo0 >= p.Wo) {
+              wo0 -= p.Wo;
+              ++ho0;
+            }
           }
         }
       }
@@ -201,6 +244,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       int local = 0;
+      // descriptors of stage 0; a stage or a K step moves the start address
+      // (bits 0-13, in 16-byte units) only
+      const uint64_t da0 = smem_desc_mn_sw128(a_ring, WG_PIX * 128);
+      const uint64_t db0 = smem_desc_mn_sw128(b_ring, WG_PIX * 128);
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++local) {
         const WgUnit wu = wg_decode(p, u);
         const int it = wu.tap / (p.kh * p.kw);
@@ -209,31 +256,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!wait_bounded(tempty_bar + 8 * acc, acc_phase ^ 1, ctl, true)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * static_cast<uint32_t>(p.BN);
-        bool first = true;
-        for (long long c = wu.c_begin; c < wu.c_end; ++c) {
-          const long long fo = c / p.chunks_per_frame;
-          const int n = static_cast<int>(fo / p.Do);
-          const int to = static_cast<int>(fo - static_cast<long long>(n) * p.Do);
-          if (wg_source_frame(p, to, it) < 0) continue;
-          if (!wait_bounded(full_bar + 8 * stage, phase, ctl, true)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a0 = a_ring + stage * WG_A_BYTES;
-          const uint32_t b0 = b_ring + stage * b_stage_bytes;
+        uint32_t accumulate = 0;
+        FrameWalk fw(p, wu);
+        while (ok && fw.next(p)) {
+          if (wg_source_frame(p, fw.to, it) < 0) continue;
+          for (int j = 0; j < fw.count; ++j) {
+            if (!wait_bounded(full_bar + 8 * stage, phase, ctl, true)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t da = da0 + ((stage * WG_A_BYTES) >> 4);
+            const uint64_t db = db0 + ((stage * b_stage_bytes) >> 4);
 #pragma unroll
-          for (int k = 0; k < WG_PIX / 16; ++k) {
-            // 16 pixels = two 8-row groups further along K
-            const uint64_t da = smem_desc_mn_sw128(a0 + k * 2048, WG_PIX * 128);
-            const uint64_t db = smem_desc_mn_sw128(b0 + k * 2048, WG_PIX * 128);
-            mma_f16_ss(d_tmem, da, db, p.idesc, first ? 0u : 1u);
-            first = false;
-          }
-          mma_commit(empty_bar + 8 * stage);
-          if (++stage == static_cast<uint32_t>(p.stages)) {
-            stage = 0;
-            phase ^= 1;
+            for (int k = 0; k < WG_PIX / 16; ++k) {
+              // 16 pixels = two 8-row groups (2 KB) further along K
+              mma_f16_ss(d_tmem, da + k * (2048 >> 4), db + k * (2048 >> 4), p.idesc,
+                         accumulate);
+              accumulate = 1;
+            }
+            mma_commit(empty_bar + 8 * stage);
+            if (++stage == static_cast<uint32_t>(p.stages)) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
         }
         if (!ok) break;
@@ -245,7 +291,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     // Thread = one (tap, ci) row of the unit (TMEM lane); 32 output channels
-    // per TMEM load; fp32 atomic adds into dw[co][tap][ci].
+    // per TMEM load; fp32 atomic adds into dw[co][tap][ci], one warp-wide
+    // instruction covering 32 consecutive ci of one co (128 bytes).
     const uint32_t quarter = warp & 3;
     int local = 0;
     const long long K = static_cast<long long>(p.taps) * p.Cin;
@@ -258,26 +305,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int it = wu.tap / (p.kh * p.kw);
       // a unit whose chunks all read zero padding issued no MMA: nothing to add
       bool any = false;
-      for (long long c = wu.c_begin; c < wu.c_end && !any; ++c) {
-        const long long fo = c / p.chunks_per_frame;
-        const int n = static_cast<int>(fo / p.Do);
-        any = wg_source_frame(p, static_cast<int>(fo - static_cast<long long>(n) * p.Do), it) >= 0;
-      }
+      FrameWalk fw(p, wu);
+      while (!any && fw.next(p)) any = wg_source_frame(p, fw.to, it) >= 0;
       const int ci = wu.cb * 128 + static_cast<int>(quarter * 32 + lane);
       const bool row_ok = any && ci < p.Cin;
       const uint32_t t_row =
           tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.BN);
+      float* dst = p.dw + static_cast<long long>(wu.co0) * K +
+                   static_cast<long long>(wu.tap) * p.Cin + ci;
       for (int j = 0; j < p.BN / 32; ++j) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + j * 32, r);
         tmem_ld_wait();
         if (row_ok) {
-          for (int e = 0; e < 32; ++e) {
-            const int co = wu.co0 + j * 32 + e;
-            if (co < p.Cout)
-              atomicAdd(p.dw + static_cast<long long>(co) * K + static_cast<long long>(wu.tap) * p.Cin + ci,
-                        __uint_as_float(r[e]));
-          }
+          const int co_left = p.Cout - (wu.co0 + j * 32);
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (e < co_left) atomicAdd(dst + static_cast<long long>(j * 32 + e) * K,
+                                       __uint_as_float(r[e]));
         }
       }
       tc_fence_before();
@@ -305,28 +350,60 @@ __global__ void f32_to_16_kernel(const float* __restrict__ src, uint16_t* __rest
     dst[i] = static_cast<uint16_t>(C::pack(src[i], 0.0f) & 0xFFFFu);
 }
 
-// dbias[co] += sum over pixels of dy[m, co]: 8 channels per thread, fp32
-// partial sums over a slab of pixels, one atomic per channel and thread.
+// dbias[co] += sum over pixels of dy[m, co].  Block = a slab of pixels and
+// up to 2048 channels (blockIdx.y picks the group); thread = 8 channels (one
+// 16-byte load) of every rows-th pixel of the slab, four loads in flight.  The
+// block's rows are then reduced in shared memory and each channel takes one
+// atomic per block.  256 threads, 8 KB of dynamic shared memory.
+constexpr int BIAS_THREADS = 256;
+constexpr int BIAS_CHANNELS = 2048;
+
 template <bool kBF16>
-__global__ void bias_grad_kernel(const uint16_t* __restrict__ dy, float* __restrict__ db,
-                                 long long pixels, int Cout, long long pixels_per_block) {
+__global__ void __launch_bounds__(BIAS_THREADS) bias_grad_kernel(
+    const uint16_t* __restrict__ dy, float* __restrict__ db, long long pixels, int Cout,
+    long long pixels_per_block) {
   using C = Cvt<kBF16>;
-  const int vecs = Cout / 8;
-  const int rows = blockDim.x / vecs;
+  extern __shared__ float s_part[];                 // [rows][channels of the group]
+  const int c0 = blockIdx.y * BIAS_CHANNELS;
+  const int cb = Cout - c0 < BIAS_CHANNELS ? Cout - c0 : BIAS_CHANNELS;
+  const int vecs = cb / 8;
+  const int rows = BIAS_THREADS / vecs;
   const int v = threadIdx.x % vecs;
   const int r = threadIdx.x / vecs;
-  if (r >= rows) return;
   const long long p_begin = blockIdx.x * pixels_per_block;
   long long p_end = p_begin + pixels_per_block;
   if (p_end > pixels) p_end = pixels;
-  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (long long p = p_begin + r; p < p_end; p += rows) {
-    const uint4 q = __ldg(reinterpret_cast<const uint4*>(dy + p * Cout + 8 * v));
-    acc[0] += C::lo(q.x); acc[1] += C::hi(q.x); acc[2] += C::lo(q.y); acc[3] += C::hi(q.y);
-    acc[4] += C::lo(q.z); acc[5] += C::hi(q.z); acc[6] += C::lo(q.w); acc[7] += C::hi(q.w);
-  }
+  if (r < rows) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const long long stride = Cout / 8;              // 16-byte vectors per pixel
+    const uint4* src = reinterpret_cast<const uint4*>(dy) + c0 / 8 + v;
+    long long p = p_begin + r;
+    for (; p + 3 * rows < p_end; p += 4 * rows) {
+      uint4 q[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) atomicAdd(db + 8 * v + j, acc[j]);
+      for (int u = 0; u < 4; ++u) q[u] = __ldg(src + (p + u * rows) * stride);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc[0] += C::lo(q[u].x); acc[1] += C::hi(q[u].x);
+        acc[2] += C::lo(q[u].y); acc[3] += C::hi(q[u].y);
+        acc[4] += C::lo(q[u].z); acc[5] += C::hi(q[u].z);
+        acc[6] += C::lo(q[u].w); acc[7] += C::hi(q[u].w);
+      }
+    }
+    for (; p < p_end; p += rows) {
+      const uint4 q = __ldg(src + p * stride);
+      acc[0] += C::lo(q.x); acc[1] += C::hi(q.x); acc[2] += C::lo(q.y); acc[3] += C::hi(q.y);
+      acc[4] += C::lo(q.z); acc[5] += C::hi(q.z); acc[6] += C::lo(q.w); acc[7] += C::hi(q.w);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s_part[r * cb + 8 * v + j] = acc[j];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < cb; c += BIAS_THREADS) {
+    float t = 0.0f;
+    for (int q = 0; q < rows; ++q) t += s_part[q * cb + c];
+    atomicAdd(db + c0 + c, t);
+  }
 }
 
 }  // namespace conv3d
