@@ -208,7 +208,10 @@ CONV3D_API conv3d_status_t conv3d_groupnorm_silu(const void* x, const double* st
  * padding (kh-1-ph, kw-1-pw spatially; kt-1-pf in front temporally); with
  * causal replicate padding the gradient of the kt-1 virtual frames in front
  * is added to frame 0.  Runs the forward kernel on dy, after a weight
- * transform into the workspace.
+ * transform into the workspace; with causal replicate padding it runs twice
+ * (frames 1.. straight into dx, one launch per sample; the kt frames
+ * -(kt-1)..0 in fp32 into the workspace, summed into frame 0 with one
+ * rounding).
  *
  * Arguments describe the FORWARD problem: dy is [N, Do, Ho, Wo, Cout] (y's
  * shape), w [Cout, kt, kh, kw, Cin], dx [N, D, H, W, Cin] (written).  Supported:

@@ -236,9 +236,12 @@ def call_bwd_weight(**kw):
 
 
 def test_bwd_workspace_bytes():
-    # replicate padding keeps the kt-1 padded frames' gradient in fp32
+    # flipped weight + (replicate padding) the fp32 gradient of frames -2..0
+    wt = 64 * 27 * 64 * 2
     assert c3.bwd_data_workspace_bytes(1, 64, 4, 16, 16, 64, (3, 3, 3), (0, 1, 1),
-                                       c3.TPAD_CAUSAL_REPLICATE) >= 1 * 6 * 16 * 16 * 64 * 4
+                                       c3.TPAD_CAUSAL_REPLICATE) == wt + 3 * 16 * 16 * 64 * 4
+    assert c3.bwd_data_workspace_bytes(2, 64, 4, 16, 16, 64, (3, 3, 3), (1, 1, 1),
+                                       c3.TPAD_ZERO) == wt
     dw = 64 * 27 * 32 * 4
     assert c3.bwd_weight_workspace_bytes(32, 64, (3, 3, 3)) >= dw + 64 * 4
 

@@ -73,11 +73,21 @@ WEIGHT_CASES = [
     (1, 256, 2, 16, 16, 320, (1, 1, 1), (1, 1, 1), (0, 0, 0), ZERO, "bf16"), # 2 co tiles, 1x1x1
     (1, 192, 3, 7, 9, 40, (2, 3, 3), (1, 1, 1), (0, 1, 1), CREP, "bf16"),    # partial blocks
     (1, 64, 6, 8, 8, 64, (3, 3, 3), (1, 1, 1), (3, 1, 1), ZERO, "bf16"),     # taps fully in padding
+    (1, 128, 4, 9, 11, 96, (3, 3, 3), (1, 1, 1), (0, 1, 1), CZERO, "f16"),   # 18 entries per tap
+    (1, 64, 3, 8, 8, 320, (1, 3, 3), (1, 1, 1), (0, 1, 1), ZERO, "bf16"),    # 3 co tiles of 128
 ]
 
 
+@pytest.fixture(params=["plain", "swap"])
+def wgrad_variant(request, monkeypatch):
+    """The weight-gradient kernel's two operand assignments (swap needs Cin % 64 == 0;
+    otherwise the plain one runs either way)."""
+    monkeypatch.setenv("CONV3D_WGRAD_SWAP", "1" if request.param == "swap" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("case", WEIGHT_CASES, ids=lambda c: "x".join(map(str, c[:6])) + f"-k{''.join(map(str, c[6]))}-s{''.join(map(str, c[7]))}-t{c[9]}-{c[10]}")
-def test_bwd_weight_every_element(case):
+def test_bwd_weight_every_element(case, wgrad_variant):
     N, Cin, D, H, W, Cout, k, stride, pad, tpad, dt = case
     x, w, dy, od = grads_problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=400 + Cin, dt=dt,
                                  stride=stride)

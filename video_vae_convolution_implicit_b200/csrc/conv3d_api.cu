@@ -645,11 +645,28 @@ conv3d_status_t noalloc_scratch(void*& out) {
 
 // ------------------------------------------------------------------ backward data pass
 
+// dx of a stride-1 convolution is the convolution of dy with the mirrored,
+// channel-transposed weight under the complementary padding ("tr").  With
+// causal replicate padding frame 0 also collects the gradient of the kt-1
+// copies of itself in front.  That case runs in two parts so that only frame
+// 0 needs an fp32 intermediate:
+//   front -- the kt frames -(kt-1)..0 of the extended gradient, in fp32 (frame
+//            0's own taps included); a fold kernel sums them into dx[:, 0];
+//   body  -- frames 1..D-1, straight to dx, one launch per sample (dy and dx
+//            offset by one frame, so the body is the plain transposed
+//            convolution of dy[n, 1:]).
+// A single frame (D = 1) needs neither: dx[n, 0] = sum over taps of the 2D
+// transposed convolution of dy[n, 0], i.e. the forward first-frame problem on
+// dy with the transformed weight, which folds the taps into a (hi, lo) pair.
 struct BwdDataPlan {
   Problem fwd;      // the forward problem being differentiated
-  Problem tr;       // the transposed convolution that produces dx (or its extension)
+  Problem tr;       // the whole transposed convolution (no replicate padding), or
+                    // the first-frame problem (replicate padding, D = 1)
+  Problem front;    // replicate padding, D > 1: extended frames, fp32
+  Problem body;     // replicate padding, D > 1: frames 1.., one sample
+  bool rep;         // front + body + fold
   size_t wt_bytes;  // flipped weight
-  size_t ext_bytes; // gradient of the padded frames (causal replicate only)
+  size_t ext_bytes; // fp32 gradient of the front frames, or the folded weight (D = 1)
 };
 
 conv3d_status_t plan_bwd_data(const void* dy, const void* w, const void* dx, int N, int Cin, int D,
@@ -686,21 +703,44 @@ conv3d_status_t plan_bwd_data(const void* dy, const void* w, const void* dx, int
   T.st = T.sh = T.sw = 1;
   T.ph = F.kh - 1 - F.ph;
   T.pw = F.kw - 1 - F.pw;
-  // dx[f] gathers dy[f + it' - (kt-1-pf)]; with replicate padding the output is
-  // extended to the kt-1 virtual frames in front (folded onto frame 0 afterwards)
-  T.pf = F.kt - 1 - F.pf + (rep ? F.kt - 1 : 0);
+  // dx[f] gathers dy[f + it' - (kt-1-pf)]
+  T.pf = F.kt - 1 - F.pf;
   T.pb = F.kt - 1 - F.pb;
-  T.Do = D + (rep ? F.kt - 1 : 0);
+  T.Do = D;
   T.Ho = H;
   T.Wo = W;
   T.tpad = CONV3D_TPAD_ZERO;  // dy frames outside [0, Do) contribute nothing
   T.dtype = dtype;
   T.has_residual = false;
-  T.out_f32 = rep;            // the padded-frame gradient stays fp32 until the fold
+  T.out_f32 = false;
   T.prev = nullptr;
   T.fold = false;
+  B.rep = rep && D > 1;
+  if (rep && D == 1) {
+    T.tpad = CONV3D_TPAD_CAUSAL_REPLICATE;
+    T.pf = F.kt - 1;
+    T.pb = 0;
+    T.fold = true;
+  }
+  if (B.rep) {
+    // causal: pf = kt-1, so T.pf = 0 and output frame f reads dy[f .. f+kt-1]
+    Problem& Fr = B.front;
+    Fr = T;
+    Fr.pf = T.pf + F.kt - 1;    // output frames -(kt-1)..0
+    Fr.Do = F.kt;
+    Fr.out_f32 = true;
+    Problem& Bo = B.body;
+    Bo = T;
+    Bo.N = 1;
+    Bo.D = F.Do - 1;            // dy[n, 1:]
+    Bo.Do = D - 1;              // dx[n, 1:]
+  }
   B.wt_bytes = (static_cast<size_t>(Cout) * F.kt * F.kh * F.kw * Cin * 2 + 255) & ~size_t(255);
-  B.ext_bytes = rep ? (static_cast<size_t>(N) * T.Do * H * W * Cin * 4 + 255) & ~size_t(255) : 0;
+  B.ext_bytes = 0;
+  if (B.rep)
+    B.ext_bytes = (static_cast<size_t>(N) * F.kt * H * W * Cin * 4 + 255) & ~size_t(255);
+  else if (T.fold)
+    B.ext_bytes = (fold_bytes(Cout, Cin, kernel) + 255) & ~size_t(255);
   return CONV3D_OK;
 }
 
@@ -806,8 +846,12 @@ size_t conv3d_bwd_data_workspace_bytes(int N, int Cin, int D, int H, int W, int 
   const size_t wt = (static_cast<size_t>(Cout) * kernel[0] * kernel[1] * kernel[2] * Cin * 2 + 255) &
                     ~size_t(255);
   size_t ext = 0;
-  if (tpad == CONV3D_TPAD_CAUSAL_REPLICATE && kernel[0] > 1)
-    ext = (static_cast<size_t>(N) * (D + kernel[0] - 1) * H * W * Cin * 4 + 255) & ~size_t(255);
+  if (tpad == CONV3D_TPAD_CAUSAL_REPLICATE && kernel[0] > 1) {
+    if (D > 1)
+      ext = (static_cast<size_t>(N) * kernel[0] * H * W * Cin * 4 + 255) & ~size_t(255);
+    else
+      ext = (fold_bytes(Cout, Cin, kernel) + 255) & ~size_t(255);
+  }
   return wt + ext;
 }
 
@@ -851,22 +895,36 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
   }
-  void* out = B.ext_bytes ? static_cast<void*>(static_cast<char*>(workspace) + B.wt_bytes) : dx;
-  if ((st = launch_main(*S, B.tr, dy, nullptr, wt, nullptr, nullptr, out, stream)) != CONV3D_OK)
+  if (B.tr.fold)
+    return run(B.tr, dy, wt, nullptr, nullptr, dx, static_cast<char*>(workspace) + B.wt_bytes,
+               B.ext_bytes, false, stream);
+  if (!B.rep)
+    return launch_main(*S, B.tr, dy, nullptr, wt, nullptr, nullptr, dx, stream);
+
+  float* ext = reinterpret_cast<float*>(static_cast<char*>(workspace) + B.wt_bytes);
+  if ((st = launch_main(*S, B.front, dy, nullptr, wt, nullptr, nullptr, ext, stream)) != CONV3D_OK)
     return st;
-  if (B.ext_bytes) {
-    const long long frame_elems = static_cast<long long>(H) * W * Cin;
-    const long long total = static_cast<long long>(N) * D * (frame_elems / 8);
+  const long long frame_elems = static_cast<long long>(H) * W * Cin;
+  if (B.body.Do > 0) {
+    const long long dy_frame = static_cast<long long>(B.fwd.Ho) * B.fwd.Wo * Cout;
+    for (int n = 0; n < N; ++n) {
+      const uint16_t* dy_n = static_cast<const uint16_t*>(dy) + (n * static_cast<long long>(B.fwd.Do) + 1) * dy_frame;
+      uint16_t* dx_n = static_cast<uint16_t*>(dx) + (n * static_cast<long long>(D) + 1) * frame_elems;
+      if ((st = launch_main(*S, B.body, dy_n, nullptr, wt, nullptr, nullptr, dx_n, stream)) !=
+          CONV3D_OK)
+        return st;
+    }
+  }
+  {
+    const long long total = static_cast<long long>(N) * (frame_elems / 8);
     int blocks = static_cast<int>((total + 255) / 256);
     if (blocks > 8 * S->num_sms) blocks = 8 * S->num_sms;
     if (dtype == CONV3D_BF16)
       fold_front_gradient_kernel<true><<<blocks, 256, 0, stream>>>(
-          static_cast<const float*>(out), static_cast<uint16_t*>(dx), N, D, kernel[0],
-          frame_elems);
+          ext, static_cast<uint16_t*>(dx), N, D, kernel[0], frame_elems);
     else
       fold_front_gradient_kernel<false><<<blocks, 256, 0, stream>>>(
-          static_cast<const float*>(out), static_cast<uint16_t*>(dx), N, D, kernel[0],
-          frame_elems);
+          ext, static_cast<uint16_t*>(dx), N, D, kernel[0], frame_elems);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "gradient fold launch");
   }
@@ -963,9 +1021,27 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   wp.cblocks = (Cin + 127) / 128;
   wp.BN = Cout >= 256 ? 256 : ((Cout + 63) / 64) * 64;
   wp.co_tiles = (Cout + wp.BN - 1) / wp.BN;
+  wp.c64s = Cin / 64;
+  wp.ents = F.kh * F.kw * wp.c64s;
+  wp.eblocks = (wp.ents + 3) / 4;
+  // The swapped variant needs whole 64-channel input boxes; it wins when it
+  // issues fewer MMA steps (an N = 128 step costs about as much as N = 256).
+  bool swap = false;
+  if (Cin % 64 == 0) {
+    const long long plain_steps = taps * wp.cblocks * wp.co_tiles;
+    const long long swap_steps = static_cast<long long>(F.kt) * wp.eblocks * ((Cout + 127) / 128);
+    swap = swap_steps < plain_steps;
+    if (const char* env = getenv("CONV3D_WGRAD_SWAP")) swap = env[0] == '1';
+  }
+  if (swap) {
+    wp.BN = 128;
+    wp.co_tiles = (Cout + 127) / 128;
+  }
   wp.chunks_per_frame = (wp.HoWo + WG_PIX - 1) / WG_PIX;
   wp.total_chunks = static_cast<long long>(N) * F.Do * wp.chunks_per_frame;
-  const long long base_units = static_cast<long long>(wp.taps) * wp.cblocks * wp.co_tiles;
+  const long long base_units =
+      swap ? static_cast<long long>(F.kt) * wp.eblocks * wp.co_tiles
+           : static_cast<long long>(wp.taps) * wp.cblocks * wp.co_tiles;
   const long long splits = choose_wgrad_splits(base_units, wp.total_chunks, S->num_sms);
   if (base_units * splits > 0x7FFFFFFFLL) {
     set_error("problem too large");
@@ -973,13 +1049,15 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   }
   wp.splits = static_cast<int>(splits);
   wp.num_units = static_cast<int>(base_units * splits);
-  const int stage_bytes = WG_A_BYTES + wp.BN * WG_PIX * 2;
+  const int stage_bytes = WG_A_BYTES + (swap ? 4 * WG_PIX * 128 : wp.BN * WG_PIX * 2);
   const int reserve = 1024 + 8 * (2 * MAX_STAGES + 5);
   int stages = (S->max_smem_optin - reserve - 64) / stage_bytes;
   if (stages > MAX_STAGES) stages = MAX_STAGES;
   wp.stages = stages;
-  wp.tmem_cols = pow2_at_least(2u * wp.BN);
-  wp.idesc = idesc_f16(bf16, BM, wp.BN) | (1u << 15) | (1u << 16);  // both operands MN-major
+  wp.acc_cols = swap ? 256u : static_cast<uint32_t>(wp.BN);
+  wp.tmem_cols = pow2_at_least(2u * wp.acc_cols);
+  // both operands MN-major; the swapped variant sets N per unit
+  wp.idesc = idesc_f16(bf16, BM, swap ? 256 : wp.BN) | (1u << 15) | (1u << 16);
   wp.dw = dw32;
   wp.status = S->status;
   wp.timeout_ns = kDefaultTimeoutNs;
@@ -1009,7 +1087,8 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   }
   cudaError_t e = cudaMemsetAsync(workspace, 0, need, stream);
   if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
-  auto kern = bf16 ? conv3d_wgrad_kernel<true> : conv3d_wgrad_kernel<false>;
+  auto kern = bf16 ? (swap ? conv3d_wgrad_kernel<true, true> : conv3d_wgrad_kernel<true, false>)
+                   : (swap ? conv3d_wgrad_kernel<false, true> : conv3d_wgrad_kernel<false, false>);
   {
     std::lock_guard<std::mutex> lock(g_mu);
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

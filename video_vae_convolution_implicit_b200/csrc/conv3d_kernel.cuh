@@ -713,29 +713,24 @@ __global__ void flip_transpose_weight_kernel(const uint16_t* __restrict__ w,
 
 // Causal replicate padding reads frame 0 for the kt-1 frames in front, so the
 // gradient of those virtual frames belongs to frame 0: dx[n, 0] = sum of
-// ext[n, 0 .. kt-1], dx[n, f] = ext[n, f + kt - 1] for f >= 1, where ext holds
-// the gradient of the D + kt - 1 padded frames.  8 values per thread.
+// ext[n, 0 .. kt-1], ext holding the fp32 gradient of the kt frames
+// -(kt-1)..0 (frame 0's own taps in ext[n, kt-1]); one rounding.  Frames >= 1
+// are written by the convolution itself.  8 values per thread.
 template <bool kBF16>
 __global__ void fold_front_gradient_kernel(const float* __restrict__ ext,
                                            uint16_t* __restrict__ dx, int N, int D, int kt,
                                            long long frame_elems) {
   using C = Cvt<kBF16>;
-  // ext is fp32 so that frame 0's sum is rounded once
   const long long vecs_per_frame = frame_elems / 8;
-  const long long total = static_cast<long long>(N) * D * vecs_per_frame;
+  const long long total = static_cast<long long>(N) * vecs_per_frame;
+  const float4* e4 = reinterpret_cast<const float4*>(ext);
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long v = i % vecs_per_frame;
-    const long long nf = i / vecs_per_frame;
-    const int f = static_cast<int>(nf % D);
-    const long long n = nf / D;
-    const long long ext_frames = static_cast<long long>(D) + kt - 1;
-    const float4* e4 = reinterpret_cast<const float4*>(ext);
+    const long long n = i / vecs_per_frame;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    const int e_begin = f > 0 ? f + kt - 1 : 0;
-    const int e_end = f > 0 ? f + kt : kt;
-    for (int e = e_begin; e < e_end; ++e) {
-      const long long at = ((n * ext_frames + e) * vecs_per_frame + v) * 2;
+    for (int e = 0; e < kt; ++e) {
+      const long long at = ((n * kt + e) * vecs_per_frame + v) * 2;
       const float4 a = e4[at], b = e4[at + 1];
       acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
       acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
@@ -745,7 +740,7 @@ __global__ void fold_front_gradient_kernel(const float* __restrict__ ext,
     out.y = C::pack(acc[2], acc[3]);
     out.z = C::pack(acc[4], acc[5]);
     out.w = C::pack(acc[6], acc[7]);
-    reinterpret_cast<uint4*>(dx)[nf * vecs_per_frame + v] = out;
+    reinterpret_cast<uint4*>(dx)[n * D * vecs_per_frame + v] = out;
   }
 }
 

@@ -13,8 +13,15 @@
 // the MN-major 128-byte-swizzle layout (64-element blocks 8 KB apart along
 // M/N, 8-row groups 1 KB apart along K).
 //
+// A swapped variant serves layers with at most 128 output channels, where an
+// N = 128 product would take as long as an N = 256 one: M = 128 output
+// channels (dy, two 64-channel boxes) and N = up to 256 (tap, ci) entries --
+// four 64-channel im2col boxes of taps that share the temporal offset, so
+// every chunk is skipped or used by the whole unit.
+//
 // Work unit = (tap and 128-channel block, output-channel block, range of
-// 64-pixel chunks); persistent CTAs walk the units.  Chunks whose temporal tap
+// 64-pixel chunks), or (temporal tap and block of four entries, ...) when
+// swapped; persistent CTAs walk the units.  Chunks whose temporal tap
 // reads zero padding are skipped by producer and MMA alike; chunk rows past
 // the frame read dy as zero.  Each finished unit adds its 128 x BN fp32 block
 // to a zeroed fp32 gradient with coalesced atomics (one warp: 32 consecutive
@@ -33,15 +40,19 @@ struct WgradParams {
   int pf, ph, pw;
   int tpad;                 // 0 zero, 1 causal replicate, 2 causal zero
   int taps;
-  int cblocks;              // ceil(Cin / 128)
-  int BN;                   // output channels per unit (multiple of 64, <= 256)
+  int cblocks;              // ceil(Cin / 128)                  (plain variant)
+  int BN;                   // output channels per unit: multiple of 64, <= 256 (plain), 128 (swap)
   int co_tiles;             // ceil(Cout / BN)
+  int c64s;                 // Cin / 64                          (swap variant)
+  int ents;                 // kh * kw * Cin / 64 entries per temporal tap (swap)
+  int eblocks;              // ceil(ents / 4)                    (swap)
   int chunks_per_frame;     // ceil(HoWo / 64)
   long long total_chunks;   // N * Do * chunks_per_frame
   int splits;               // chunk ranges per (tap block, co tile)
   int num_units;
   int stages;
   uint32_t tmem_cols;
+  uint32_t acc_cols;        // TMEM columns per accumulator (BN plain, 256 swapped)
   uint32_t idesc;
   float* dw;                // [Cout][taps][Cin] fp32, accumulated
   int* status;
@@ -72,18 +83,31 @@ __device__ __forceinline__ int wg_source_frame(const WgradParams& p, int to, int
 }
 
 struct WgUnit {
-  int tap, cb, co0;
+  int it;            // temporal tap
+  int tap, cb;       // plain: tap and 128-channel block
+  int e0, nent;      // swap: first entry of the block and entries in it (1..4)
+  int co0;
   long long c_begin, c_end;
 };
 
+template <bool kSwap>
 __device__ __forceinline__ WgUnit wg_decode(const WgradParams& p, int u) {
   WgUnit r;
   const int split = u % p.splits;
   const int rest = u / p.splits;
   const int cot = rest % p.co_tiles;
   const int mb = rest / p.co_tiles;
-  r.tap = mb / p.cblocks;
-  r.cb = mb - r.tap * p.cblocks;
+  if (kSwap) {
+    r.it = mb / p.eblocks;
+    r.e0 = (mb - r.it * p.eblocks) * 4;
+    r.nent = p.ents - r.e0 < 4 ? p.ents - r.e0 : 4;
+    r.tap = r.cb = 0;
+  } else {
+    r.tap = mb / p.cblocks;
+    r.cb = mb - r.tap * p.cblocks;
+    r.it = r.tap / (p.kh * p.kw);
+    r.e0 = r.nent = 0;
+  }
   r.co0 = cot * p.BN;
   const long long per = (p.total_chunks + p.splits - 1) / p.splits;
   r.c_begin = static_cast<long long>(split) * per;
@@ -127,7 +151,14 @@ struct FrameWalk {
   }
 };
 
-template <bool kBF16>
+// 128-bit fp32 reduction into global memory (four consecutive floats).
+__device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+template <bool kBF16, bool kSwap>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     conv3d_wgrad_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_dy, const WgradParams p) {
@@ -138,7 +169,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t lane = threadIdx.x % 32;
 
   const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
-  const uint32_t b_stage_bytes = static_cast<uint32_t>(p.BN) * WG_PIX * 2;
+  // B operand: dy boxes (plain, BN/64 of them) or up to four x boxes (swapped)
+  const uint32_t b_stage_bytes = kSwap ? 4u * WG_PIX * 128 : static_cast<uint32_t>(p.BN) * WG_PIX * 2;
   const uint32_t a_ring = base;
   const uint32_t b_ring = a_ring + p.stages * WG_A_BYTES;
   const uint32_t bars = b_ring + p.stages * b_stage_bytes;
@@ -176,23 +208,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint32_t tx_bytes = WG_A_BYTES + b_stage_bytes;
       uint32_t stage = 0, phase = 0;
       long long issued = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-        const WgUnit wu = wg_decode(p, u);
-        const int it = wu.tap / (p.kh * p.kw);
-        const int ih = (wu.tap / p.kw) % p.kh;
-        const int iw = wu.tap % p.kw;
+        const WgUnit wu = wg_decode<kSwap>(p, u);
+        // The im2col boxes of the unit: (kw offset, kh offset, first channel).
         // A box whose channels all lie past Cin (or past Cout for dy) is loaded
-        // from the block's first chunk instead: those rows/columns of the
-        // product are never written out, and every copy starts in bounds.
-        const int xc0 = 2 * wu.cb * 64;
-        const int xc1 = xc0 + 64 < p.Cin ? xc0 + 64 : xc0;
+        // from the unit's first box instead: those rows/columns of the product
+        // are never written out, and every copy starts in bounds.
+        int bw[4], bh[4], bc[4];
+        int nx;
+        if (kSwap) {
+          nx = wu.nent;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int e = wu.e0 + (j < nx ? j : 0);
+            const int sp = e / p.c64s;
+            bc[j] = (e - sp * p.c64s) * 64;
+            bh[j] = sp / p.kw;
+            bw[j] = sp - bh[j] * p.kw;
+          }
+        } else {
+          nx = 2;
+          const int sp = wu.tap - wu.it * p.kh * p.kw;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            bh[j] = sp / p.kw;
+            bw[j] = sp - bh[j] * p.kw;
+            bc[j] = 2 * wu.cb * 64 + (j == 1 && 2 * wu.cb * 64 + 64 < p.Cin ? 64 : 0);
+          }
+        }
+        // dy boxes: the unit's output channels in 64-channel steps
+        const int ndy = kSwap ? 2 : p.BN / 64;
+        const uint32_t x_ring = kSwap ? b_ring : a_ring;
+        const uint32_t x_stage = kSwap ? b_stage_bytes : WG_A_BYTES;
+        const uint32_t dy_ring = kSwap ? a_ring : b_ring;
+        const uint32_t dy_stage = kSwap ? WG_A_BYTES : b_stage_bytes;
+        const uint32_t tx_bytes = static_cast<uint32_t>(nx + ndy) * (WG_PIX * 128);
         FrameWalk fw(p, wu);
         while (ok && fw.next(p)) {
-          const int f = wg_source_frame(p, fw.to, it);
+          const int f = wg_source_frame(p, fw.to, wu.it);
           if (f < 0) continue;                  // this tap reads zero padding here
           const int img = fw.n * p.D + f;
           int p0 = fw.pc * WG_PIX;
@@ -205,16 +261,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             const uint32_t fb = full_bar + 8 * stage;
             mbar_arrive_expect_tx(fb, tx_bytes);
-            const uint32_t a_dst = a_ring + stage * WG_A_BYTES;
+            const uint32_t x_dst = x_ring + stage * x_stage;
             const int wx = wo0 * p.sw - p.pw, hx = ho0 * p.sh - p.ph;
-            tma_load_im2col_4d(a_dst, &map_x, fb, xc0, wx, hx, img,
-                               static_cast<uint16_t>(iw), static_cast<uint16_t>(ih));
-            tma_load_im2col_4d(a_dst + WG_PIX * 128, &map_x, fb, xc1, wx, hx, img,
-                               static_cast<uint16_t>(iw), static_cast<uint16_t>(ih));
-            const uint32_t b_dst = b_ring + stage * b_stage_bytes;
-            for (int q = 0; q < p.BN / 64; ++q) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (q < nx)
+                tma_load_im2col_4d(x_dst + q * (WG_PIX * 128), &map_x, fb, bc[q], wx, hx, img,
+                                   static_cast<uint16_t>(bw[q]), static_cast<uint16_t>(bh[q]));
+            const uint32_t dy_dst = dy_ring + stage * dy_stage;
+            for (int q = 0; q < ndy; ++q) {
               const int dc = wu.co0 + 64 * q < p.Cout ? wu.co0 + 64 * q : wu.co0;
-              tma_load_3d(b_dst + q * (WG_PIX * 128), &map_dy, fb, dc, p0,
+              tma_load_3d(dy_dst + q * (WG_PIX * 128), &map_dy, fb, dc, p0,
                           static_cast<int>(fw.fo));
             }
             ++issued;
@@ -249,17 +306,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t da0 = smem_desc_mn_sw128(a_ring, WG_PIX * 128);
       const uint64_t db0 = smem_desc_mn_sw128(b_ring, WG_PIX * 128);
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++local) {
-        const WgUnit wu = wg_decode(p, u);
-        const int it = wu.tap / (p.kh * p.kw);
+        const WgUnit wu = wg_decode<kSwap>(p, u);
+        // swapped: N = 64 per entry of the block
+        const uint32_t idesc =
+            kSwap ? (p.idesc & ~(0x3Fu << 17)) | (static_cast<uint32_t>(wu.nent * 64 >> 3) << 17)
+                  : p.idesc;
         const uint32_t acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!wait_bounded(tempty_bar + 8 * acc, acc_phase ^ 1, ctl, true)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * static_cast<uint32_t>(p.BN);
+        const uint32_t d_tmem = tmem_base + acc * static_cast<uint32_t>(p.acc_cols);
         uint32_t accumulate = 0;
         FrameWalk fw(p, wu);
         while (ok && fw.next(p)) {
-          if (wg_source_frame(p, fw.to, it) < 0) continue;
+          if (wg_source_frame(p, fw.to, wu.it) < 0) continue;
           for (int j = 0; j < fw.count; ++j) {
             if (!wait_bounded(full_bar + 8 * stage, phase, ctl, true)) {
               ok = false;
@@ -271,8 +331,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int k = 0; k < WG_PIX / 16; ++k) {
               // 16 pixels = two 8-row groups (2 KB) further along K
-              mma_f16_ss(d_tmem, da + k * (2048 >> 4), db + k * (2048 >> 4), p.idesc,
-                         accumulate);
+              mma_f16_ss(d_tmem, da + k * (2048 >> 4), db + k * (2048 >> 4), idesc, accumulate);
               accumulate = 1;
             }
             mma_commit(empty_bar + 8 * stage);
@@ -290,9 +349,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // Thread = one (tap, ci) row of the unit (TMEM lane); 32 output channels
-    // per TMEM load; fp32 atomic adds into dw[co][tap][ci], one warp-wide
-    // instruction covering 32 consecutive ci of one co (128 bytes).
+    // Plain: thread = one (tap, ci) row of the unit (TMEM lane), 32 output
+    // channels per TMEM load; fp32 atomic adds into dw[co][tap][ci], one
+    // warp-wide instruction covering 32 consecutive ci of one co (128 bytes).
+    // Swapped: thread = one output channel, 32 consecutive ci of one entry per
+    // TMEM load, added with eight 16-byte reductions.
     const uint32_t quarter = warp & 3;
     int local = 0;
     const long long K = static_cast<long long>(p.taps) * p.Cin;
@@ -301,28 +362,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!wait_bounded(tfull_bar + 8 * acc, acc_phase, ctl, true)) break;
       tc_fence_after();
-      const WgUnit wu = wg_decode(p, u);
-      const int it = wu.tap / (p.kh * p.kw);
+      const WgUnit wu = wg_decode<kSwap>(p, u);
       // a unit whose chunks all read zero padding issued no MMA: nothing to add
       bool any = false;
       FrameWalk fw(p, wu);
-      while (!any && fw.next(p)) any = wg_source_frame(p, fw.to, it) >= 0;
-      const int ci = wu.cb * 128 + static_cast<int>(quarter * 32 + lane);
-      const bool row_ok = any && ci < p.Cin;
+      while (!any && fw.next(p)) any = wg_source_frame(p, fw.to, wu.it) >= 0;
       const uint32_t t_row =
-          tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.BN);
-      float* dst = p.dw + static_cast<long long>(wu.co0) * K +
-                   static_cast<long long>(wu.tap) * p.Cin + ci;
-      for (int j = 0; j < p.BN / 32; ++j) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + j * 32, r);
-        tmem_ld_wait();
-        if (row_ok) {
-          const int co_left = p.Cout - (wu.co0 + j * 32);
+          tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.acc_cols);
+      if (kSwap) {
+        const int co = wu.co0 + static_cast<int>(quarter * 32 + lane);
+        const bool row_ok = any && co < p.Cout;
+        for (int j = 0; j < 2 * wu.nent; ++j) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + j * 32, r);
+          tmem_ld_wait();
+          if (row_ok) {
+            const int e = wu.e0 + j / 2;
+            const int sp = e / p.c64s;
+            const int tap = wu.it * p.kh * p.kw + sp;
+            const int ci0 = (e - sp * p.c64s) * 64 + (j & 1) * 32;
+            float* dst = p.dw + static_cast<long long>(co) * K +
+                         static_cast<long long>(tap) * p.Cin + ci0;
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (e < co_left) atomicAdd(dst + static_cast<long long>(j * 32 + e) * K,
-                                       __uint_as_float(r[e]));
+            for (int q = 0; q < 8; ++q)
+              red_add_v4(dst + 4 * q, __uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                         __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+          }
+        }
+      } else {
+        const int ci = wu.cb * 128 + static_cast<int>(quarter * 32 + lane);
+        const bool row_ok = any && ci < p.Cin;
+        float* dst = p.dw + static_cast<long long>(wu.co0) * K +
+                     static_cast<long long>(wu.tap) * p.Cin + ci;
+        for (int j = 0; j < p.BN / 32; ++j) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + j * 32, r);
+          tmem_ld_wait();
+          if (row_ok) {
+            const int co_left = p.Cout - (wu.co0 + j * 32);
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (e < co_left) atomicAdd(dst + static_cast<long long>(j * 32 + e) * K,
+                                         __uint_as_float(r[e]));
+          }
         }
       }
       tc_fence_before();
