@@ -632,7 +632,12 @@ def backward_parity(which, wl, p, dy, out, db):
     entries) and the whole dbias against the oracle's per-element sums."""
     hb = host_bits(p)
     dyb = si.bits(dy)
-    idx, _ = _backward_samples(which, wl, 48 if which == "dgrad" else 256, 4321)
+    if which == "dgrad":
+        n = 48
+    else:   # each dw entry sums over every output pixel: keep the oracle to ~5e8 products
+        Do, Ho, Wo = out_shape(wl)
+        n = int(min(256, max(32, 5e8 / (wl.N * Do * Ho * Wo))))
+    idx, _ = _backward_samples(which, wl, n, 4321)
     ref = _oracle_backward_at(which, wl, hb, dyb, idx)
     flat = out.view(-1, wl.Cin) if which == "dgrad" else out.view(-1)
     got = flat[torch.from_numpy(idx).to(out.device)].double().cpu().numpy()

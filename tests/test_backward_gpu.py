@@ -75,6 +75,8 @@ WEIGHT_CASES = [
     (1, 64, 6, 8, 8, 64, (3, 3, 3), (1, 1, 1), (3, 1, 1), ZERO, "bf16"),     # taps fully in padding
     (1, 128, 4, 9, 11, 96, (3, 3, 3), (1, 1, 1), (0, 1, 1), CZERO, "f16"),   # 18 entries per tap
     (1, 64, 3, 8, 8, 320, (1, 3, 3), (1, 1, 1), (0, 1, 1), ZERO, "bf16"),    # 3 co tiles of 128
+    (2, 64, 1, 10, 12, 64, (3, 3, 3), (1, 1, 1), (0, 1, 1), CREP, "bf16"),   # single frame: taps equal
+    (1, 128, 1, 9, 9, 96, (2, 3, 3), (1, 1, 1), (0, 1, 1), CREP, "f16"),     # single frame, kt = 2
 ]
 
 

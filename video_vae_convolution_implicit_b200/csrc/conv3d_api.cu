@@ -886,12 +886,10 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
   if ((st = device_state(S, dev)) != CONV3D_OK) return st;
   uint16_t* wt = static_cast<uint16_t*>(workspace);
   {
-    const long long total = static_cast<long long>(Cout) * kernel[0] * kernel[1] * kernel[2] * Cin;
-    int blocks = static_cast<int>((total + 255) / 256);
-    if (blocks > 8 * S->num_sms) blocks = 8 * S->num_sms;
-    flip_transpose_weight_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint16_t*>(w), wt,
-                                                            Cout, kernel[0], kernel[1], kernel[2],
-                                                            Cin);
+    const int taps = kernel[0] * kernel[1] * kernel[2];
+    const dim3 grid((Cin + 31) / 32, (Cout + 31) / 32, taps);
+    flip_transpose_weight_kernel<<<grid, dim3(32, 8), 0, stream>>>(
+        static_cast<const uint16_t*>(w), wt, Cout, taps, Cin);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
   }
@@ -1006,6 +1004,12 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   int dev = 0;
   if ((st = device_state(S, dev)) != CONV3D_OK) return st;
   const bool bf16 = dtype == CONV3D_BF16;
+  // A single causal-replicate frame: every temporal tap reads frame 0, so the
+  // kt tap gradients are equal; the kernel computes the kt = 1 problem over
+  // frame 0 and the rounding pass writes it to all kt taps.
+  const bool frame0 = tpad == CONV3D_TPAD_CAUSAL_REPLICATE && D == 1 && F.kt > 1;
+  const int kt_run = frame0 ? 1 : F.kt;
+  const long long taps_run = static_cast<long long>(kt_run) * F.kh * F.kw;
   float* dw32 = static_cast<float*>(workspace);
   float* db32 = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                          ((dw_elems * 4 + 255) & ~size_t(255)));
@@ -1013,11 +1017,11 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   WgradParams wp{};
   wp.D = F.D; wp.Do = F.Do; wp.Ho = F.Ho; wp.Wo = F.Wo; wp.HoWo = F.Ho * F.Wo;
   wp.Cin = Cin; wp.Cout = Cout;
-  wp.kt = F.kt; wp.kh = F.kh; wp.kw = F.kw;
+  wp.kt = kt_run; wp.kh = F.kh; wp.kw = F.kw;
   wp.st = F.st; wp.sh = F.sh; wp.sw = F.sw;
-  wp.pf = F.pf; wp.ph = F.ph; wp.pw = F.pw;
-  wp.tpad = static_cast<int>(tpad);
-  wp.taps = static_cast<int>(taps);
+  wp.pf = frame0 ? 0 : F.pf; wp.ph = F.ph; wp.pw = F.pw;
+  wp.tpad = frame0 ? 0 : static_cast<int>(tpad);
+  wp.taps = static_cast<int>(taps_run);
   wp.cblocks = (Cin + 127) / 128;
   wp.BN = Cout >= 256 ? 256 : ((Cout + 63) / 64) * 64;
   wp.co_tiles = (Cout + wp.BN - 1) / wp.BN;
@@ -1028,8 +1032,8 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   // issues fewer MMA steps (an N = 128 step costs about as much as N = 256).
   bool swap = false;
   if (Cin % 64 == 0) {
-    const long long plain_steps = taps * wp.cblocks * wp.co_tiles;
-    const long long swap_steps = static_cast<long long>(F.kt) * wp.eblocks * ((Cout + 127) / 128);
+    const long long plain_steps = taps_run * wp.cblocks * wp.co_tiles;
+    const long long swap_steps = static_cast<long long>(kt_run) * wp.eblocks * ((Cout + 127) / 128);
     swap = swap_steps < plain_steps;
     if (const char* env = getenv("CONV3D_WGRAD_SWAP")) swap = env[0] == '1';
   }
@@ -1040,7 +1044,7 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   wp.chunks_per_frame = (wp.HoWo + WG_PIX - 1) / WG_PIX;
   wp.total_chunks = static_cast<long long>(N) * F.Do * wp.chunks_per_frame;
   const long long base_units =
-      swap ? static_cast<long long>(F.kt) * wp.eblocks * wp.co_tiles
+      swap ? static_cast<long long>(kt_run) * wp.eblocks * wp.co_tiles
            : static_cast<long long>(wp.taps) * wp.cblocks * wp.co_tiles;
   const long long splits = choose_wgrad_splits(base_units, wp.total_chunks, S->num_sms);
   if (base_units * splits > 0x7FFFFFFFLL) {
@@ -1101,12 +1105,16 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   {
     int blocks = static_cast<int>((dw_elems + 255) / 256);
     if (blocks > 8 * S->num_sms) blocks = 8 * S->num_sms;
-    if (bf16)
-      f32_to_16_kernel<true><<<blocks, 256, 0, stream>>>(dw32, static_cast<uint16_t*>(dw),
-                                                         static_cast<long long>(dw_elems));
+    uint16_t* d16 = static_cast<uint16_t*>(dw);
+    const long long run_per_co = taps_run * Cin;
+    if (frame0 && bf16)
+      f32_to_16_bcast_kernel<true><<<blocks, 256, 0, stream>>>(dw32, d16, Cout, F.kt, run_per_co);
+    else if (frame0)
+      f32_to_16_bcast_kernel<false><<<blocks, 256, 0, stream>>>(dw32, d16, Cout, F.kt, run_per_co);
+    else if (bf16)
+      f32_to_16_kernel<true><<<blocks, 256, 0, stream>>>(dw32, d16, static_cast<long long>(dw_elems));
     else
-      f32_to_16_kernel<false><<<blocks, 256, 0, stream>>>(dw32, static_cast<uint16_t*>(dw),
-                                                          static_cast<long long>(dw_elems));
+      f32_to_16_kernel<false><<<blocks, 256, 0, stream>>>(dw32, d16, static_cast<long long>(dw_elems));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dw conversion launch");
   }
   if (dbias) {

@@ -690,24 +690,28 @@ __global__ void fold_temporal_taps_kernel(const uint16_t* __restrict__ w, uint16
 
 // Backward data pass: the weight the transposed convolution runs with,
 // wt[ci, it, ih, iw, co] = w[co, kt-1-it, kh-1-ih, kw-1-iw, ci] (every tap
-// mirrored, the channel roles exchanged).
+// mirrored, the channel roles exchanged).  Mirroring all three tap indices
+// reverses the linear tap order, so each tap is a [Cout x Cin] -> [Cin x Cout]
+// transpose: block = one tap and a 32 x 32 tile, staged in shared memory so
+// that both the reads and the writes run along contiguous channels.
+// Launch: grid (ceil(Cin/32), ceil(Cout/32), taps), block (32, 8).
 __global__ void flip_transpose_weight_kernel(const uint16_t* __restrict__ w,
-                                             uint16_t* __restrict__ wt, int Cout, int kt, int kh,
-                                             int kw, int Cin) {
-  const long long taps = static_cast<long long>(kt) * kh * kw;
-  const long long total = taps * Cout * Cin;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    // i indexes wt = [Cin][kt][kh][kw][Cout]
-    const long long co = i % Cout;
-    long long q = i / Cout;
-    const int iw = static_cast<int>(q % kw); q /= kw;
-    const int ih = static_cast<int>(q % kh); q /= kh;
-    const int it = static_cast<int>(q % kt); q /= kt;
-    const long long ci = q;
-    const long long src =
-        (((co * kt + (kt - 1 - it)) * kh + (kh - 1 - ih)) * kw + (kw - 1 - iw)) * Cin + ci;
-    wt[i] = w[src];
+                                             uint16_t* __restrict__ wt, int Cout, int taps,
+                                             int Cin) {
+  __shared__ uint16_t tile[32][33];
+  const int ci0 = blockIdx.x * 32, co0 = blockIdx.y * 32;
+  const int tap = blockIdx.z;                  // tap of wt
+  const int tap_src = taps - 1 - tap;          // mirrored tap of w
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    const int co = co0 + r, ci = ci0 + threadIdx.x;
+    if (co < Cout && ci < Cin)
+      tile[r][threadIdx.x] = w[(static_cast<long long>(co) * taps + tap_src) * Cin + ci];
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += 8) {
+    const int ci = ci0 + r, co = co0 + threadIdx.x;
+    if (co < Cout && ci < Cin)
+      wt[(static_cast<long long>(ci) * taps + tap) * Cout + co] = tile[threadIdx.x][r];
   }
 }
 

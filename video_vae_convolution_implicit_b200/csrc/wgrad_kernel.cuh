@@ -432,6 +432,21 @@ __global__ void f32_to_16_kernel(const float* __restrict__ src, uint16_t* __rest
     dst[i] = static_cast<uint16_t>(C::pack(src[i], 0.0f) & 0xFFFFu);
 }
 
+// The same rounding, written to each of kt equal temporal taps:
+// dst[co][it][s] = src[co][s] for s < per_co (kh * kw * Cin entries).
+template <bool kBF16>
+__global__ void f32_to_16_bcast_kernel(const float* __restrict__ src, uint16_t* __restrict__ dst,
+                                       int Cout, int kt, long long per_co) {
+  using C = Cvt<kBF16>;
+  const long long n = static_cast<long long>(Cout) * kt * per_co;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long co = i / (kt * per_co);
+    const long long s = i % per_co;
+    dst[i] = static_cast<uint16_t>(C::pack(src[co * per_co + s], 0.0f) & 0xFFFFu);
+  }
+}
+
 // dbias[co] += sum over pixels of dy[m, co].  Block = a slab of pixels and
 // up to 2048 channels (blockIdx.y picks the group); thread = 8 channels (one
 // 16-byte load) of every rows-th pixel of the slab, four loads in flight.  The
