@@ -80,11 +80,13 @@ WEIGHT_CASES = [
 ]
 
 
-@pytest.fixture(params=["plain", "swap"])
+@pytest.fixture(params=["plain", "pair", "swap"])
 def wgrad_variant(request, monkeypatch):
-    """The weight-gradient kernel's two operand assignments (swap needs Cin % 64 == 0;
-    otherwise the plain one runs either way)."""
+    """The weight-gradient kernel's variants: one CTA, a CTA pair (256-channel output
+    tiles only) and the swapped operand assignment (Cin % 64 == 0 only); where a
+    variant does not apply the call falls back to the plain one."""
     monkeypatch.setenv("CONV3D_WGRAD_SWAP", "1" if request.param == "swap" else "0")
+    monkeypatch.setenv("CONV3D_WGRAD_PAIR", "1" if request.param == "pair" else "0")
     return request.param
 
 

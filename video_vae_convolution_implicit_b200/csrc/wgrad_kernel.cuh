@@ -19,9 +19,15 @@
 // four 64-channel im2col boxes of taps that share the temporal offset, so
 // every chunk is skipped or used by the whole unit.
 //
+// A pair variant (cta_group::2, a cluster of two CTAs) computes M = 256:
+// CTA r holds the 128 rows of its own (tap, channel block) -- the two blocks
+// share the temporal tap -- and half of the 256 output channels of dy, so
+// each CTA moves 32 KB per chunk instead of 48 KB for the same products.
+//
 // Work unit = (tap and 128-channel block, output-channel block, range of
 // 64-pixel chunks), or (temporal tap and block of four entries, ...) when
-// swapped; persistent CTAs walk the units.  Chunks whose temporal tap
+// swapped, or (temporal tap and pair of blocks, ...) for CTA pairs;
+// persistent CTAs (or clusters) walk the units.  Chunks whose temporal tap
 // reads zero padding are skipped by producer and MMA alike; chunk rows past
 // the frame read dy as zero.  Each finished unit adds its 128 x BN fp32 block
 // to a zeroed fp32 gradient with coalesced atomics (one warp: 32 consecutive
@@ -46,6 +52,7 @@ struct WgradParams {
   int c64s;                 // Cin / 64                          (swap variant)
   int ents;                 // kh * kw * Cin / 64 entries per temporal tap (swap)
   int eblocks;              // ceil(ents / 4)                    (swap)
+  int pairs_per_it;         // ceil(kh * kw * cblocks / 2)       (pair)
   int chunks_per_frame;     // ceil(HoWo / 64)
   long long total_chunks;   // N * Do * chunks_per_frame
   int splits;               // chunk ranges per (tap block, co tile)
@@ -84,20 +91,35 @@ __device__ __forceinline__ int wg_source_frame(const WgradParams& p, int to, int
 
 struct WgUnit {
   int it;            // temporal tap
-  int tap, cb;       // plain: tap and 128-channel block
+  int tap, cb;       // plain / pair: tap and 128-channel block of this CTA
   int e0, nent;      // swap: first entry of the block and entries in it (1..4)
+  bool dup;          // pair: this CTA's block repeats its peer's (odd count): not written
   int co0;
   long long c_begin, c_end;
 };
 
-template <bool kSwap>
-__device__ __forceinline__ WgUnit wg_decode(const WgradParams& p, int u) {
+template <bool kSwap, bool kPair>
+__device__ __forceinline__ WgUnit wg_decode(const WgradParams& p, int u, uint32_t rank = 0) {
   WgUnit r;
+  r.dup = false;
   const int split = u % p.splits;
   const int rest = u / p.splits;
   const int cot = rest % p.co_tiles;
   const int mb = rest / p.co_tiles;
-  if (kSwap) {
+  if (kPair) {
+    // blocks of one temporal tap, (spatial tap, channel block) in order, taken two at a time
+    r.it = mb / p.pairs_per_it;
+    const int per_it = p.kh * p.kw * p.cblocks;
+    int e = 2 * (mb - r.it * p.pairs_per_it) + static_cast<int>(rank);
+    if (e >= per_it) {
+      e = per_it - 1;
+      r.dup = true;
+    }
+    const int sp = e / p.cblocks;
+    r.cb = e - sp * p.cblocks;
+    r.tap = r.it * p.kh * p.kw + sp;
+    r.e0 = r.nent = 0;
+  } else if (kSwap) {
     r.it = mb / p.eblocks;
     r.e0 = (mb - r.it * p.eblocks) * 4;
     r.nent = p.ents - r.e0 < 4 ? p.ents - r.e0 : 4;
@@ -158,19 +180,27 @@ __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c
                : "memory");
 }
 
-template <bool kBF16, bool kSwap>
+template <bool kBF16, bool kSwap, bool kPair>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     conv3d_wgrad_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_dy, const WgradParams p) {
+  static_assert(!(kSwap && kPair), "the pair variant is the plain operand assignment");
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
   __shared__ int s_abort;
+  constexpr int kCtas = kPair ? 2 : 1;
   const uint32_t warp = threadIdx.x / 32;
   const uint32_t lane = threadIdx.x % 32;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0;
+  const bool leader = rank == 0;
+  const int first_unit = blockIdx.x / kCtas;   // this CTA's cluster (or CTA) index
+  const int unit_step = gridDim.x / kCtas;
 
   const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
-  // B operand: dy boxes (plain, BN/64 of them) or up to four x boxes (swapped)
-  const uint32_t b_stage_bytes = kSwap ? 4u * WG_PIX * 128 : static_cast<uint32_t>(p.BN) * WG_PIX * 2;
+  // B operand: dy boxes (plain: BN/64 of them; pair: this CTA's half) or up to
+  // four x boxes (swapped)
+  const uint32_t b_stage_bytes =
+      kSwap ? 4u * WG_PIX * 128 : static_cast<uint32_t>(p.BN / kCtas) * WG_PIX * 2;
   const uint32_t a_ring = base;
   const uint32_t b_ring = a_ring + p.stages * WG_A_BYTES;
   const uint32_t bars = b_ring + p.stages * b_stage_bytes;
@@ -189,7 +219,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar + 8 * a, 1);
-      mbar_init(tempty_bar + 8 * a, 4);
+      mbar_init(tempty_bar + 8 * a, 4 * kCtas);
     }
     mbar_init(drain_bar, 1);
     fence_mbar_init();
@@ -197,11 +227,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefetch_tensormap(&map_dy);
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(&s_tmem_base), p.tmem_cols);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_addr(&s_tmem_base), p.tmem_cols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_addr(&s_tmem_base), p.tmem_cols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();   // the peer's barriers are initialised
   tc_fence_after();
   const uint32_t tmem_base = s_tmem_base;
 
@@ -211,8 +247,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t stage = 0, phase = 0;
       long long issued = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-        const WgUnit wu = wg_decode<kSwap>(p, u);
+      for (int u = first_unit; ok && u < p.num_units; u += unit_step) {
+        const WgUnit wu = wg_decode<kSwap, kPair>(p, u, rank);
         // The im2col boxes of the unit: (kw offset, kh offset, first channel).
         // A box whose channels all lie past Cin (or past Cout for dy) is loaded
         // from the unit's first box instead: those rows/columns of the product
@@ -239,13 +275,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             bc[j] = 2 * wu.cb * 64 + (j == 1 && 2 * wu.cb * 64 + 64 < p.Cin ? 64 : 0);
           }
         }
-        // dy boxes: the unit's output channels in 64-channel steps
-        const int ndy = kSwap ? 2 : p.BN / 64;
+        // dy boxes: the unit's output channels (this CTA's half for a pair) in
+        // 64-channel steps
+        const int ndy = kSwap ? 2 : p.BN / 64 / kCtas;
+        const int dy_c0 = wu.co0 + static_cast<int>(rank) * (p.BN / kCtas);
         const uint32_t x_ring = kSwap ? b_ring : a_ring;
         const uint32_t x_stage = kSwap ? b_stage_bytes : WG_A_BYTES;
         const uint32_t dy_ring = kSwap ? a_ring : b_ring;
         const uint32_t dy_stage = kSwap ? WG_A_BYTES : b_stage_bytes;
-        const uint32_t tx_bytes = static_cast<uint32_t>(nx + ndy) * (WG_PIX * 128);
+        const uint32_t tx_bytes = static_cast<uint32_t>(kCtas * (nx + ndy)) * (WG_PIX * 128);
         FrameWalk fw(p, wu);
         while (ok && fw.next(p)) {
           const int f = wg_source_frame(p, fw.to, wu.it);
@@ -260,19 +298,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               break;
             }
             const uint32_t fb = full_bar + 8 * stage;
-            mbar_arrive_expect_tx(fb, tx_bytes);
+            if (leader) mbar_arrive_expect_tx(fb, tx_bytes);
             const uint32_t x_dst = x_ring + stage * x_stage;
-            const int wx = wo0 * p.sw - p.pw, hx = ho0 * p.sh - p.ph;
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (q < nx)
-                tma_load_im2col_4d(x_dst + q * (WG_PIX * 128), &map_x, fb, bc[q], wx, hx, img,
-                                   static_cast<uint16_t>(bw[q]), static_cast<uint16_t>(bh[q]));
             const uint32_t dy_dst = dy_ring + stage * dy_stage;
-            for (int q = 0; q < ndy; ++q) {
-              const int dc = wu.co0 + 64 * q < p.Cout ? wu.co0 + 64 * q : wu.co0;
-              tma_load_3d(dy_dst + q * (WG_PIX * 128), &map_dy, fb, dc, p0,
-                          static_cast<int>(fw.fo));
+            const int wx = wo0 * p.sw - p.pw, hx = ho0 * p.sh - p.ph;
+            if constexpr (kPair) {
+              // both CTAs' copies complete on the even CTA's barrier
+              const uint32_t fb0 = mapa_shared(fb, 0);
+#pragma unroll
+              for (int q = 0; q < 2; ++q)
+                tma_load_im2col_4d_pair(x_dst + q * (WG_PIX * 128), &map_x, fb0, bc[q], wx, hx,
+                                        img, static_cast<uint16_t>(bw[q]),
+                                        static_cast<uint16_t>(bh[q]));
+              for (int q = 0; q < ndy; ++q) {
+                const int dc = dy_c0 + 64 * q < p.Cout ? dy_c0 + 64 * q : wu.co0;
+                tma_load_3d_pair(dy_dst + q * (WG_PIX * 128), &map_dy, fb0, dc, p0,
+                                 static_cast<int>(fw.fo));
+              }
+            } else {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                if (q < nx)
+                  tma_load_im2col_4d(x_dst + q * (WG_PIX * 128), &map_x, fb, bc[q], wx, hx, img,
+                                     static_cast<uint16_t>(bw[q]), static_cast<uint16_t>(bh[q]));
+              for (int q = 0; q < ndy; ++q) {
+                const int dc = dy_c0 + 64 * q < p.Cout ? dy_c0 + 64 * q : wu.co0;
+                tma_load_3d(dy_dst + q * (WG_PIX * 128), &map_dy, fb, dc, p0,
+                            static_cast<int>(fw.fo));
+              }
             }
             ++issued;
             if (++stage == static_cast<uint32_t>(p.stages)) {
@@ -289,15 +342,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       if (!ok) {
-        const long long first = issued > p.stages ? issued - p.stages : 0;
-        for (long long i = first; i < issued; ++i)
-          wait_bounded(full_bar + 8 * static_cast<uint32_t>(i % p.stages),
-                       static_cast<uint32_t>((i / p.stages) & 1), ctl, false);
+        if (leader) {
+          // let the copies already in flight land before the CTA may exit
+          const long long first = issued > p.stages ? issued - p.stages : 0;
+          for (long long i = first; i < issued; ++i)
+            wait_bounded(full_bar + 8 * static_cast<uint32_t>(i % p.stages),
+                         static_cast<uint32_t>((i / p.stages) & 1), ctl, false);
+        } else {
+          // the odd CTA's copies complete on the even CTA's barriers: give them
+          // time to land (both CTAs stay resident until the final cluster barrier)
+          const uint64_t t0 = globaltimer_ns();
+          while (globaltimer_ns() - t0 < 200000ull) {
+          }
+        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       int local = 0;
@@ -305,8 +367,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // (bits 0-13, in 16-byte units) only
       const uint64_t da0 = smem_desc_mn_sw128(a_ring, WG_PIX * 128);
       const uint64_t db0 = smem_desc_mn_sw128(b_ring, WG_PIX * 128);
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x, ++local) {
-        const WgUnit wu = wg_decode<kSwap>(p, u);
+      for (int u = first_unit; ok && u < p.num_units; u += unit_step, ++local) {
+        const WgUnit wu = wg_decode<kSwap, kPair>(p, u);
         // swapped: N = 64 per entry of the block
         const uint32_t idesc =
             kSwap ? (p.idesc & ~(0x3Fu << 17)) | (static_cast<uint32_t>(wu.nent * 64 >> 3) << 17)
@@ -331,10 +393,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int k = 0; k < WG_PIX / 16; ++k) {
               // 16 pixels = two 8-row groups (2 KB) further along K
-              mma_f16_ss(d_tmem, da + k * (2048 >> 4), db + k * (2048 >> 4), idesc, accumulate);
+              if constexpr (kPair)
+                mma_f16_ss_pair(d_tmem, da + k * (2048 >> 4), db + k * (2048 >> 4), idesc,
+                                accumulate);
+              else
+                mma_f16_ss(d_tmem, da + k * (2048 >> 4), db + k * (2048 >> 4), idesc, accumulate);
               accumulate = 1;
             }
-            mma_commit(empty_bar + 8 * stage);
+            if constexpr (kPair) {
+              mma_commit_pair(empty_bar + 8 * stage);
+              mma_commit_pair(mapa_shared(empty_bar + 8 * stage, 1));
+            } else {
+              mma_commit(empty_bar + 8 * stage);
+            }
             if (++stage == static_cast<uint32_t>(p.stages)) {
               stage = 0;
               phase ^= 1;
@@ -342,9 +413,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         if (!ok) break;
-        mma_commit(tfull_bar + 8 * acc);
+        if constexpr (kPair) {
+          mma_commit_pair(tfull_bar + 8 * acc);
+          mma_commit_pair(mapa_shared(tfull_bar + 8 * acc, 1));
+        } else {
+          mma_commit(tfull_bar + 8 * acc);
+        }
       }
-      mma_commit(drain_bar);
+      if constexpr (kPair)
+        mma_commit_pair(drain_bar);
+      else
+        mma_commit(drain_bar);
       wait_bounded(drain_bar, 0, ctl, false);
     }
   } else {
@@ -357,12 +436,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t quarter = warp & 3;
     int local = 0;
     const long long K = static_cast<long long>(p.taps) * p.Cin;
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++local) {
+    for (int u = first_unit; u < p.num_units; u += unit_step, ++local) {
       const uint32_t acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!wait_bounded(tfull_bar + 8 * acc, acc_phase, ctl, true)) break;
       tc_fence_after();
-      const WgUnit wu = wg_decode<kSwap>(p, u);
+      const WgUnit wu = wg_decode<kSwap, kPair>(p, u, rank);
       // a unit whose chunks all read zero padding issued no MMA: nothing to add
       bool any = false;
       FrameWalk fw(p, wu);
@@ -391,7 +470,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       } else {
         const int ci = wu.cb * 128 + static_cast<int>(quarter * 32 + lane);
-        const bool row_ok = any && ci < p.Cin;
+        const bool row_ok = any && !wu.dup && ci < p.Cin;
         float* dst = p.dw + static_cast<long long>(wu.co0) * K +
                      static_cast<long long>(wu.tap) * p.Cin + ci;
         for (int j = 0; j < p.BN / 32; ++j) {
@@ -409,16 +488,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar + 8 * acc);
+      if (lane == 0) {
+        if constexpr (kPair)
+          mbar_arrive_cluster(mapa_shared(tempty_bar + 8 * acc, 0));
+        else
+          mbar_arrive(tempty_bar + 8 * acc);
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (kPair) cluster_sync();   // no CTA leaves while its peer may touch it
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, p.tmem_cols);
+    if constexpr (kPair)
+      tmem_dealloc_pair(tmem_base, p.tmem_cols);
+    else
+      tmem_dealloc(tmem_base, p.tmem_cols);
   }
 }
 
