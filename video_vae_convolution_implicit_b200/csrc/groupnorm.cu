@@ -53,7 +53,7 @@ __device__ __forceinline__ void unpack8(const uint4 q, uint32_t (&e)[8]) {
 // channels of each group in shared memory and issues one pair of fp64 atomics
 // per group.
 template <bool kBF16>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
     gn_stats_kernel(const uint16_t* __restrict__ x,
                                                        double* __restrict__ stats, int C,
                                                        int groups, long long set_pixels,
@@ -82,24 +82,20 @@ __global__ void __launch_bounds__(256)
       s2[j] = 0.0f;
     }
   }
-  // software-pipelined: the next four rows are in flight while these four are summed
+  // four rows' loads in flight per thread; with four 8-warp blocks per SM that
+  // keeps ~64 KB of reads outstanding on every SM
   constexpr int U = 4;
-  uint4 cur[U], nxt[U];
-  long long p = p_begin + r;
-#pragma unroll
-  for (int u = 0; u < U; ++u)
-    if (p + u * rows < p_end) cur[u] = __ldg(reinterpret_cast<const uint4*>(xs + (p + u * rows) * C + 8 * v));
-  for (; p < p_end; p += U * rows) {
-    const long long pn = p + U * rows;
+  for (long long p = p_begin + r; p < p_end; p += U * rows) {
+    uint4 q[U];
 #pragma unroll
     for (int u = 0; u < U; ++u)
-      if (pn + u * rows < p_end)
-        nxt[u] = __ldg(reinterpret_cast<const uint4*>(xs + (pn + u * rows) * C + 8 * v));
+      if (p + u * rows < p_end)
+        q[u] = __ldg(reinterpret_cast<const uint4*>(xs + (p + u * rows) * C + 8 * v));
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (p + u * rows < p_end) {
         uint32_t e[8];
-        unpack8(cur[u], e);
+        unpack8(q[u], e);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const float d = to_f<kBF16>(e[j]) - K[j];
@@ -108,8 +104,6 @@ __global__ void __launch_bounds__(256)
         }
       }
     }
-#pragma unroll
-    for (int u = 0; u < U; ++u) cur[u] = nxt[u];
   }
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -264,7 +258,9 @@ conv3d_status_t conv3d_groupnorm_stats(const void* x, int N, int D, int H, int W
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // about eight blocks per SM over the whole tensor, at least 16 pixels per row of threads
+  // about two resident waves (four blocks per SM) over the whole tensor: one
+  // wave would leave a second, nearly empty wave whenever the per-set chunk
+  // count rounds up; at least 16 pixels per row of threads
   long long chunk_pixels = (sets * set_pixels + 8LL * sms - 1) / (8LL * sms);
   if (chunk_pixels < 16LL * rows) chunk_pixels = 16LL * rows;
   if (const char* env = getenv("CONV3D_GN_CHUNK")) {   // tuning knob: pixels per block

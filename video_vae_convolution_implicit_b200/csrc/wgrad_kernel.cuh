@@ -102,8 +102,11 @@ template <bool kSwap, bool kPair>
 __device__ __forceinline__ WgUnit wg_decode(const WgradParams& p, int u, uint32_t rank = 0) {
   WgUnit r;
   r.dup = false;
-  const int split = u % p.splits;
-  const int rest = u / p.splits;
+  // split-major: the units that run at the same time share a pixel range, so
+  // x and dy come from DRAM about once and serve every tap block from L2
+  const int per_split = p.num_units / p.splits;
+  const int split = u / per_split;
+  const int rest = u - split * per_split;
   const int cot = rest % p.co_tiles;
   const int mb = rest / p.co_tiles;
   if (kPair) {
