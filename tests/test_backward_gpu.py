@@ -40,6 +40,9 @@ DATA_CASES = [
     (1, 128, 2, 16, 16, 64, (1, 1, 1), (0, 0, 0), ZERO, "bf16"),
     (1, 48, 3, 11, 10, 40, (2, 3, 3), (0, 0, 1), CREP, "bf16"),
     (1, 64, 1, 12, 12, 64, (3, 3, 3), (0, 1, 1), CREP, "bf16"),       # single frame
+    (3, 64, 4, 8, 10, 64, (3, 3, 3), (0, 1, 1), CREP, "bf16"),        # body launch per sample
+    (2, 128, 2, 9, 7, 64, (2, 3, 3), (0, 1, 1), CREP, "f16"),         # kt = 2, two samples
+    (2, 64, 1, 8, 8, 128, (3, 3, 3), (0, 1, 1), CREP, "bf16"),        # single frame, two samples
 ]
 
 
