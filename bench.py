@@ -81,6 +81,12 @@ def algorithmic_bytes(wl):
     return 2.0 * (x + w + wl.Cout + y + (y if wl.residual else 0))
 
 
+def nominal_flops(wl):
+    """2 * M * N * K of the GEMM view (every tap counted, padding included)."""
+    Do, Ho, Wo = out_shape(wl)
+    return 2.0 * wl.N * Do * Ho * Wo * wl.Cout * wl.Cin * wl.kernel[0] * wl.kernel[1] * wl.kernel[2]
+
+
 def describe(wl, world):
     Do, Ho, Wo = out_shape(wl)
     return {
@@ -355,8 +361,17 @@ def run_ours(args, wl, rank, world, local_rank):
     value = whole_job_tflops(flops, world, args.steps, max_ms)
     peaks, peak_kind = load_peaks()
     kernel_ms = statistics.mean(step_ms)  # one conv kernel launch per step for T > 1
-    achieved = flops / (kernel_ms * 1e-3) / 1e12
-    peak = float(peaks["bf16_tflops"])
+    abytes = algorithmic_bytes(wl)
+    # the roofline that bounds this workload: tensor above the ridge point, HBM below
+    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    if flops / abytes >= ridge:
+        roof = {"bound": "tensor", "achieved": flops / (kernel_ms * 1e-3) / 1e12,
+                "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                "peak_source": f"{peak_kind} bf16_tflops (burst)"}
+    else:
+        roof = {"bound": "hbm", "achieved": abytes / (kernel_ms * 1e-3) / 1e9,
+                "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "peak_source": f"{peak_kind} hbm_gbs"}
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -364,11 +379,13 @@ def run_ours(args, wl, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic (seeded SplitMix64 normals; no model weights)",
         "config": dict(describe(wl, world), l2="flushed (2x L2 write) between timed steps"),
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(wl.name),
-                     "peak_source": f"{peak_kind} bf16_tflops (burst)",
-                     "kernel": KERNEL_NAME, "algorithmic_flops_per_launch": flops,
-                     "algorithmic_bytes_per_launch": algorithmic_bytes(wl)},
+        "roofline": dict(roof, frac=roof["achieved"] / roof["peak"],
+                         traffic=profiled_traffic(wl.name), kernel=KERNEL_NAME,
+                         algorithmic_flops_per_launch=flops,
+                         algorithmic_bytes_per_launch=abytes,
+                         flop_per_byte=flops / abytes, ridge_flop_per_byte=ridge),
+        "nominal_tflops": whole_job_tflops(nominal_flops(wl), world, args.steps, max_ms),
+        "algorithmic_gbs": abytes * world * args.steps / (max_ms * 1e-3) / 1e9,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
         "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms),
@@ -568,14 +585,36 @@ def run_backward(args, wl, rank, world, local_rank):
     flops = algorithmic_flops(wl)
     value = whole_job_tflops(flops, world, args.steps, max_ms)
     peaks, peak_kind = load_peaks()
-    peak = float(peaks["bf16_tflops"])
-    achieved = flops / (statistics.mean(step_ms) * 1e-3) / 1e12
+    call_ms = statistics.mean(step_ms)
+    # algorithmic bytes: dgrad reads dy and w and writes dx; wgrad reads x and dy
+    # and writes dw (+ dbias), all 16-bit
+    x_el = wl.N * wl.D * wl.H * wl.W * wl.Cin
+    y_el = wl.N * Do * Ho * Wo * wl.Cout
+    w_el = wl.Cout * wl.kernel[0] * wl.kernel[1] * wl.kernel[2] * wl.Cin
+    abytes = 2.0 * (y_el + w_el + x_el + (wl.Cout if args.pass_ == "wgrad" else 0))
+    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    if flops / abytes >= ridge:
+        roof = {"bound": "tensor", "achieved": flops / (call_ms * 1e-3) / 1e12,
+                "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                "peak_source": f"{peak_kind} bf16_tflops (burst)"}
+    else:
+        roof = {"bound": "hbm", "achieved": abytes / (call_ms * 1e-3) / 1e9,
+                "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "peak_source": f"{peak_kind} hbm_gbs"}
     rep = wl.tpad == 1 and wl.kernel[0] > 1
     if args.pass_ == "dgrad":
-        launches = 2 + (1 if rep else 0)       # weight transform, GEMM, front-frame fold
+        # weight transform + the GEMM; with replicate padding and D > 1 the front
+        # GEMM, one body GEMM per sample and the front-frame fold; a single
+        # replicate frame folds the weight taps (one more launch) instead
+        if rep and wl.D > 1:
+            launches = 1 + 1 + wl.N + 1
+        elif rep:
+            launches = 3
+        else:
+            launches = 2
         kernel = "conv3d_implicit_gemm_kernel (dgrad: transposed convolution of dy)"
     else:
-        launches = 3 + 1                       # clear, GEMM, dw rounding, bias column sums
+        launches = 4          # GEMM, dw rounding, bias column sums, dbias rounding
         kernel = "conv3d_wgrad_kernel"
     line = {
         "metric": f"conv3d backward {args.pass_} TFLOPS (forward-equivalent FLOPs)",
@@ -585,11 +624,12 @@ def run_backward(args, wl, rank, world, local_rank):
         "data": "synthetic (seeded SplitMix64 normals; dy stream 5)",
         "config": dict(describe(wl, world), direction=args.pass_, residual=False,
                        l2="flushed (2x L2 write) between timed steps"),
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
-                     "peak_source": f"{peak_kind} bf16_tflops (burst)", "kernel": kernel,
-                     "timed": "whole call (all its launches): a lower bound for the GEMM",
-                     "algorithmic_flops_per_launch": flops},
+        "roofline": dict(roof, frac=roof["achieved"] / roof["peak"], traffic=None,
+                         kernel=kernel,
+                         timed="whole call (all its launches): a lower bound for the GEMM",
+                         algorithmic_flops_per_launch=flops, algorithmic_bytes_per_launch=abytes,
+                         flop_per_byte=flops / abytes, ridge_flop_per_byte=ridge),
+        "nominal_tflops": whole_job_tflops(nominal_flops(wl), world, args.steps, max_ms),
         "gpu_launches": launches * args.steps,
         "clocks": clocks.summary(),
         "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms),
