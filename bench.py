@@ -469,8 +469,13 @@ def run_e2e(args, wl, p, y, stream, dev, c3, flops):
     end.record(s_in)
     torch.cuda.synchronize(dev)
     ms = start.elapsed_time(end) / steps
-    return {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
+    # whole job: every rank's steps over the slowest rank's time (each rank ran
+    # this leg, so the MAX reduction is a matching collective on all of them)
+    world = torch.distributed.get_world_size() if torch.distributed.is_initialized() else 1
+    max_ms = max_over_ranks(ms, dev)
+    return {"value": whole_job_tflops(flops, world, 1, max_ms), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world,
+            "ms_per_step": max_ms, "steps": steps, "ranks": world,
             "path": "pinned host -> device copies, conv3d_fwd (C ABI), device -> pinned host; "
                     "3 streams, 2 buffer sets (upload, compute and download of consecutive steps "
                     "overlap)"}
