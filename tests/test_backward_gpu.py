@@ -43,6 +43,8 @@ DATA_CASES = [
     (3, 64, 4, 8, 10, 64, (3, 3, 3), (0, 1, 1), CREP, "bf16"),        # body launch per sample
     (2, 128, 2, 9, 7, 64, (2, 3, 3), (0, 1, 1), CREP, "f16"),         # kt = 2, two samples
     (2, 64, 1, 8, 8, 128, (3, 3, 3), (0, 1, 1), CREP, "bf16"),        # single frame, two samples
+    (1, 64, 3, 1, 1, 64, (3, 3, 3), (0, 1, 1), CREP, "bf16"),         # 1x1 frames
+    (1, 32, 2, 2, 300, 64, (3, 3, 3), (1, 1, 1), ZERO, "bf16"),       # rows longer than a tile
 ]
 
 
@@ -80,6 +82,8 @@ WEIGHT_CASES = [
     (1, 64, 3, 8, 8, 320, (1, 3, 3), (1, 1, 1), (0, 1, 1), ZERO, "bf16"),    # 3 co tiles of 128
     (2, 64, 1, 10, 12, 64, (3, 3, 3), (1, 1, 1), (0, 1, 1), CREP, "bf16"),   # single frame: taps equal
     (1, 128, 1, 9, 9, 96, (2, 3, 3), (1, 1, 1), (0, 1, 1), CREP, "f16"),     # single frame, kt = 2
+    (1, 64, 3, 1, 1, 256, (3, 3, 3), (1, 1, 1), (0, 1, 1), CREP, "bf16"),    # 1x1 frames
+    (1, 256, 2, 2, 300, 256, (3, 3, 3), (1, 1, 1), (1, 1, 1), ZERO, "bf16"), # rows longer than a chunk
 ]
 
 

@@ -60,6 +60,9 @@ SMALL = [
     (2, 64, 3, 9, 13, 64, (3, 3, 3), (0, 1, 1), CACHED, "bf16", True),    # cached previous frames
     (1, 128, 1, 20, 19, 128, (3, 3, 3), (0, 1, 1), CACHED, "f16", False), # one-frame chunk
     (1, 40, 4, 12, 12, 72, (2, 3, 3), (0, 1, 1), CACHED, "bf16", False),
+    (1, 64, 3, 1, 1, 64, (3, 3, 3), (0, 1, 1), CREP, "bf16", False),      # 1x1 frames
+    (2, 32, 2, 1, 7, 48, (3, 3, 3), (1, 1, 1), ZERO, "f16", True),        # one-row frames
+    (1, 64, 2, 3, 300, 64, (3, 3, 3), (0, 1, 1), CZERO, "bf16", False),   # rows longer than a tile
 ]
 
 
