@@ -258,10 +258,14 @@ conv3d_status_t conv3d_groupnorm_stats(const void* x, int N, int D, int H, int W
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // about two resident waves (four blocks per SM) over the whole tensor: one
-  // wave would leave a second, nearly empty wave whenever the per-set chunk
-  // count rounds up; at least 16 pixels per row of threads
-  long long chunk_pixels = (sets * set_pixels + 8LL * sms - 1) / (8LL * sms);
+  // Pixels per block: one resident wave (four blocks per SM) for small
+  // tensors, so that few blocks end in a reduction and same-address atomics;
+  // at most 1024 for large ones, so that the many waves leave a short tail
+  // (measured on B200: 75 MB single set 41 -> 37 us; 2 GB per-frame sets,
+  // where 8 blocks per SM rounded up to 2.04 waves, 384 -> 336 us); at
+  // least 16 pixels per row of threads.
+  long long chunk_pixels = (sets * set_pixels + 4LL * sms - 1) / (4LL * sms);
+  if (chunk_pixels > 1024) chunk_pixels = 1024;
   if (chunk_pixels < 16LL * rows) chunk_pixels = 16LL * rows;
   if (const char* env = getenv("CONV3D_GN_CHUNK")) {   // tuning knob: pixels per block
     const long long v = atoll(env);
