@@ -159,3 +159,12 @@ def test_bwd_weight_full_size_sampled(name):
     assert_close(got, ref, name + " dw")
     ref_db = oracle.decode16(si.bits(dy), od).reshape(-1, wl.Cout).sum(axis=0)
     assert_close(db.double().cpu().numpy(), ref_db, name + " dbias")
+
+
+def test_bwd_data_deterministic_bitwise():
+    """dx runs the forward kernel and a fixed-order fold: repeated calls agree bit for bit."""
+    x, w, dy, od = grads_problem(2, 64, 4, 10, 12, 64, (3, 3, 3), (0, 1, 1), CREP, 17, "bf16")
+    a = c3.conv3d_bwd_data(dy, w, x.shape, (0, 1, 1), CREP)
+    b = c3.conv3d_bwd_data(dy, w, x.shape, (0, 1, 1), CREP)
+    assert c3.poll_status() == c3.Status.OK
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
