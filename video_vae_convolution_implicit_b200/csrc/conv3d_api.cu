@@ -1110,7 +1110,7 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   wp.timeout_ns = kDefaultTimeoutNs;
   const size_t smem = static_cast<size_t>(stages) * stage_bytes + reserve;
 
-  // x through the forward im2col map (64 pixels per load); dy as [frames][pixels][Cout]
+  // x through the forward im2col map (WG_PIX pixels per load); dy as [frames][pixels][Cout]
   CUtensorMap map_x, map_dy;
   if ((st = encode_im2col(F, x, static_cast<long long>(N) * D, WG_PIX, map_x)) != CONV3D_OK)
     return st;
