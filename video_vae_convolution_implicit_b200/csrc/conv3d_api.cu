@@ -410,11 +410,19 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, L
   // A tcgen05.mma step with N < 256 takes as long as one with N = 256, so
   // layers whose channel count leaves the N side short run transposed
   // (M = 128 channels, N = 256 pixels) when that needs fewer MMA steps and
-  // still gives every SM pair a tile.  CONV3D_SWAP=0/1 forces the choice.
+  // still gives every SM pair a tile.  A single-tap (1x1x1) layer is bound by
+  // streaming x from HBM: transposed, x fills the larger operand slot (32 KB
+  // of each stage instead of 16 KB), so more of it is in flight per SM; with
+  // at least 8 k-blocks per tile it runs transposed whenever that needs no
+  // more steps (measured on B200: 512->256 33x128x128, 5.06 -> 5.27 TB/s; with
+  // 4 k-blocks, 256->512, the transposing epilogue dominates and it lost 9%).
+  // CONV3D_SWAP=0/1 forces the choice.
   const long long frames_out = static_cast<long long>(P.N) * P.Do;
   const long long normal_steps = frames_out * ((kp.HoWo + BM - 1) / BM) * kp.n_tiles_n;
   const long long swap_tiles = frames_out * ((kp.HoWo + 255) / 256) * ((P.Cout + 127) / 128);
-  L.swap = swap_tiles < normal_steps && swap_tiles >= S.num_sms / 2;
+  const bool single_tap = kt_eff * P.kh * P.kw == 1 && kp.n_chunks >= 8;
+  L.swap = (swap_tiles < normal_steps || (single_tap && swap_tiles <= normal_steps)) &&
+           swap_tiles >= S.num_sms / 2;
   if (const char* env = getenv("CONV3D_SWAP")) {
     if (env[0] == '0') L.swap = false;
     if (env[0] == '1') L.swap = true;
