@@ -59,6 +59,33 @@ static int cpu_checks(void) {
   CHECK(conv3d_fwd_cached(x, NULL, w, NULL, NULL, y, 1, 64, 4, 8, 8, 64, k3, s1, p_causal,
                           CONV3D_BF16, NULL) == CONV3D_ERR_INVALID_ARG);
   CHECK(strlen(conv3d_last_error()) > 0);
+
+  /* backward entry points: workspace sizes and argument errors */
+  void* ws = (void*)0x400000000ull;
+  void* dx = (void*)0x500000000ull;
+  CHECK(conv3d_bwd_weight_workspace_bytes(64, 64, k3) >=
+        (size_t)64 * 27 * 64 * 4 + (size_t)64 * 4);
+  CHECK(conv3d_bwd_data_workspace_bytes(1, 64, 4, 8, 8, 64, k3, p_zero, CONV3D_TPAD_ZERO) ==
+        (size_t)64 * 27 * 64 * 2);
+  CHECK(conv3d_bwd_data(y, w, dx, 1, 64, 4, 8, 8, 64, k3, s2, p_causal,
+                        CONV3D_TPAD_CAUSAL_REPLICATE, CONV3D_BF16, ws, (size_t)1 << 30,
+                        NULL) == CONV3D_ERR_UNSUPPORTED);          /* stride 2 */
+  CHECK(conv3d_bwd_data(y, w, dx, 1, 64, 4, 8, 8, 64, k3, s1, p_causal,
+                        CONV3D_TPAD_CAUSAL_REPLICATE, CONV3D_BF16, NULL, 0, NULL) ==
+        CONV3D_ERR_WORKSPACE);
+  CHECK(conv3d_bwd_weight(x, y, NULL, NULL, 1, 64, 4, 8, 8, 64, k3, s1, p_causal,
+                          CONV3D_TPAD_CAUSAL_REPLICATE, CONV3D_BF16, ws, (size_t)1 << 30,
+                          NULL) == CONV3D_ERR_INVALID_ARG);        /* dw missing */
+  CHECK(conv3d_bwd_weight(x, y, dx, NULL, 1, 64, 4, 8, 8, 64, k3, s1, p_causal,
+                          CONV3D_TPAD_CAUSAL_CACHED, CONV3D_BF16, ws, (size_t)1 << 30,
+                          NULL) == CONV3D_ERR_UNSUPPORTED);
+
+  /* GroupNorm entry points: argument errors */
+  double* stats = (double*)0x600000000ull;
+  CHECK(conv3d_groupnorm_stats(x, 1, 2, 4, 4, 64, 7, 0, 1e-6f, CONV3D_BF16, stats, NULL) ==
+        CONV3D_ERR_INVALID_ARG);                                   /* C % groups */
+  CHECK(conv3d_groupnorm_silu(x, stats, NULL, NULL, (char*)y + 2, 1, 2, 4, 4, 64, 8, 0, 1,
+                              CONV3D_BF16, NULL) == CONV3D_ERR_ALIGNMENT);
   return failures;
 }
 
