@@ -435,7 +435,7 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, L
     if (env[0] == '1') L.pair = true;
   }
   if (L.swap) L.pair = false;
-  if (P.out_f32) L.swap = L.pair = false;   // the fp32 epilogue exists in the single variant
+  if (P.out_f32) L.pair = false;   // the fp32 epilogue exists in the single and transposed variants
   const int ctas = L.pair ? 2 : 1;
   if (L.swap) {
     kp.co_tile = 128;

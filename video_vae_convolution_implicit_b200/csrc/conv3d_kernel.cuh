@@ -494,12 +494,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (lane == 0) bulk_wait_group_read<1>();
             __syncwarp();
             const uint32_t yb = ybuf + b * ybytes;
+            if (p.out_f32) {
+              // fp32 rows of 32 channels (128 bytes, 128-byte swizzle): this
+              // thread's channel is 4-byte word (lane & 3) of 16-byte chunk lane >> 2
+              const uint32_t word = (lane & 3u) * 4u;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const uint16_t q = static_cast<uint16_t>(C::pack(v[e], 0.0f) & 0xFFFFu);
-              asm volatile("st.shared.u16 [%0], %1;" ::"r"(yb + swz64(e, lane >> 3) + col_byte),
-                           "h"(q)
-                           : "memory");
+              for (int e = 0; e < 32; ++e)
+                asm volatile("st.shared.f32 [%0], %1;" ::"r"(yb + swz128(e, lane >> 2) + word),
+                             "f"(v[e])
+                             : "memory");
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const uint16_t q = static_cast<uint16_t>(C::pack(v[e], 0.0f) & 0xFFFFu);
+                asm volatile("st.shared.u16 [%0], %1;" ::"r"(yb + swz64(e, lane >> 3) + col_byte),
+                             "h"(q)
+                             : "memory");
+              }
             }
             fence_proxy_async_shared();
             __syncwarp();
