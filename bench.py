@@ -6,6 +6,12 @@ One step = one conv3d_fwd call over one synthetic batch (every stage of the
 path: for this workload one kernel launch).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                  [--pass fwd|dgrad|wgrad] [--no-e2e] [--no-cpu-baseline]
+
+Workloads: the convolutions cfg1..cfg5d, cfg2c (cached frames), cfg2s (stride), cfg4s, and the
+GroupNorm + SiLU passes gn_cfg2, gn_cfg4.  --pass dgrad|wgrad times the backward passes of a
+convolution workload (forward-equivalent FLOPs).  The roofline is tensor or HBM by the workload's
+flop/B against the measured ridge point.
 
 Multi-GPU (launched with torch.distributed.run): every rank convolves its own
 seeded sample (data parallel over the batch, no data-path collective), so the
