@@ -291,6 +291,55 @@ def run_reference(args, wl, rank, world):
     return 0
 
 
+def run_reference_backward(args, wl, rank, world):
+    """The reference arm of --pass dgrad|wgrad: the oracle's per-element adjoint sums as
+    they stand, on a bounded random sample per step, scaled to forward-equivalent FLOPs
+    by the sampled fraction of the elements."""
+    if rank != 0:
+        return 0
+    import oracle
+    Do, Ho, Wo = out_shape(wl)
+    p = host_problem(wl, wl.seed)
+    dy = si.tensor((wl.N, Do, Ho, Wo, wl.Cout), wl.seed, 5, 1.0, TORCH_DTYPE[wl.dtype], "cpu")
+    hb, dyb = host_bits(p), si.bits(dy)
+    flops = algorithmic_flops(wl)
+    budget = float(os.environ.get("CONV3D_REFERENCE_SECONDS", "90")) / max(1, args.steps + args.warmup)
+    n = 8
+    while True:                                  # calibrate the sample to the per-step budget
+        idx, total = _backward_samples(args.pass_, wl, n, 5)
+        t0 = time.perf_counter()
+        _oracle_backward_at(args.pass_, wl, hb, dyb, idx)
+        dt = time.perf_counter() - t0
+        if dt > budget / 4 or idx.size >= total:
+            break
+        n = int(n * min(16.0, max(2.0, budget / max(dt, 1e-3) / 2)))
+    n = max(1, int(n * budget / max(dt, 1e-6))) if idx.size < total else n
+    times, sizes = [], []
+    for i in range(args.warmup + args.steps):
+        idx, total = _backward_samples(args.pass_, wl, n, 100 + i)
+        t0 = time.perf_counter()
+        _oracle_backward_at(args.pass_, wl, hb, dyb, idx)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+            sizes.append(idx.size)
+    value = flops * sum(sizes) / total / sum(times) / 1e12
+    what = "input pixels (all channels) of dx" if args.pass_ == "dgrad" else "entries of dw"
+    sample = (f"about {int(statistics.mean(sizes))} random {what} of {total} per step, "
+              f"{args.steps} timed steps")
+    line = {
+        "impl": "reference", "metric": f"conv3d backward {args.pass_} TFLOPS (forward-equivalent FLOPs)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": dict(describe(wl, 1), direction=args.pass_),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------- multi-rank plumbing
 
 def rank_seed(wl, rank):
@@ -866,6 +915,8 @@ def main():
             print(json.dumps({"impl": "reference", "unavailable":
                               "the reference arm times the convolution oracle only"}))
             return 0
+        if args.pass_ != "fwd":
+            return run_reference_backward(args, wl, rank, world)
         return run_reference(args, wl, rank, world)
 
     if world > 1:
