@@ -235,7 +235,9 @@ CONV3D_API size_t conv3d_bwd_data_workspace_bytes(int N, int Cin, int D, int H, 
 
 /*
  * conv3d_bwd_weight -- dw (and optionally dbias), the gradients of the
- * convolution's weight and bias: dw[co, tap, ci] = sum over output pixels of
+ * convolution's weight and bias (the trainable parameters of the pages'
+ * on-device conv-layer fine-tuning: engineering.drawthings.ai, LoRA post):
+ * dw[co, tap, ci] = sum over output pixels of
  * dy[.., co] * Xpad[.., tap-shifted, ci] (the same implicit im2col matrix the
  * forward pass reads, with the same padding rules), dbias[co] = sum of dy.
  * Accumulated in fp32 in the workspace (split over pixel ranges, fp32
