@@ -279,3 +279,8 @@ def test_bwd_entries_without_gpu_report_cuda_error():
     assert call_bwd_data() == Status.CUDA
     assert call_bwd_weight() == Status.CUDA
     assert call_bwd_weight(stride=(2, 2, 2), dbias=None) == Status.CUDA   # strided wgrad is valid
+
+
+def test_autograd_function_is_exported():
+    assert issubclass(c3.Conv3dFunction, torch.autograd.Function)
+    assert callable(c3.conv3d_autograd)

@@ -168,3 +168,23 @@ def test_bwd_data_deterministic_bitwise():
     b = c3.conv3d_bwd_data(dy, w, x.shape, (0, 1, 1), CREP)
     assert c3.poll_status() == c3.Status.OK
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.parametrize("tpad", [CREP, CZERO])
+def test_autograd_function_matches_the_oracle(tpad):
+    """Conv3dFunction: one backward through the library gives the oracle's adjoints
+    for x, w and bias, and dy itself for the residual."""
+    N, Cin, D, H, W, Cout, k, pad = 1, 64, 4, 9, 11, 96, (3, 3, 3), (0, 1, 1)
+    x, w, dy, od = grads_problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=31, dt="bf16")
+    bias = si.tensor((Cout,), 31, 2, 0.1, torch.bfloat16, "cuda")
+    res = si.tensor(dy.shape, 31, 3, 1.0, torch.bfloat16, "cuda")
+    leaves = [t.clone().requires_grad_(True) for t in (x, w, bias, res)]
+    y = c3.conv3d_autograd(*leaves, pad=pad, tpad=tpad)
+    y.backward(dy)
+    assert c3.poll_status() == c3.Status.OK
+    rdx, rdw, rdb = oracle.conv3d_backward(si.bits(x), si.bits(w), si.bits(dy), od, k, (1, 1, 1),
+                                           pad, tpad)
+    assert_close(leaves[0].grad.double().cpu().numpy(), rdx, "dx")
+    assert_close(leaves[1].grad.double().cpu().numpy(), rdw, "dw")
+    assert_close(leaves[2].grad.double().cpu().numpy(), rdb, "dbias")
+    assert torch.equal(leaves[3].grad, dy)

@@ -20,7 +20,7 @@ import torch
 __all__ = [
     "TPAD_ZERO", "TPAD_CAUSAL_REPLICATE", "TPAD_CAUSAL_ZERO", "TPAD_CAUSAL_CACHED", "F16", "BF16",
     "Status", "conv3d_fwd_cached_ptr", "groupnorm_stats", "groupnorm_silu", "conv3d_bwd_data",
-    "conv3d_bwd_weight",
+    "conv3d_bwd_weight", "Conv3dFunction", "conv3d_autograd",
     "Conv3dError", "lib_path", "conv3d", "conv3d_fwd", "conv3d_fwd_ptr", "conv3d_fwd_ws_ptr",
     "conv3d_fwd_noalloc_ptr",
     "output_shape", "workspace_bytes", "poll_status", "selftest_wait_timeout", "release",
@@ -372,3 +372,42 @@ def conv3d_bwd_weight(x: torch.Tensor, dy: torch.Tensor, kernel, stride=(1, 1, 1
                                  _dtype_code(x.dtype), workspace.data_ptr(), workspace.numel(),
                                  _stream_handle(stream)))
     return dw, db
+
+
+class Conv3dFunction(torch.autograd.Function):
+    """torch.autograd wrapper: forward through conv3d_fwd, backward through
+    conv3d_bwd_data (dx; stride 1 only) and conv3d_bwd_weight (dw, dbias).
+    The residual's gradient is dy itself.  Marshalling only: every product runs
+    in the library's kernels, none in torch."""
+
+    @staticmethod
+    def forward(ctx, x, w, bias, residual, stride, pad, tpad):
+        y = conv3d(x, w, bias, residual, stride, pad, tpad)
+        ctx.save_for_backward(x, w)
+        ctx.conf = (tuple(stride), tuple(pad), tpad, bias is not None, residual is not None)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, w = ctx.saved_tensors
+        stride, pad, tpad, has_bias, has_res = ctx.conf
+        dy = dy.contiguous()
+        dx = dw = db = dres = None
+        if ctx.needs_input_grad[0]:
+            if stride != (1, 1, 1):
+                raise NotImplementedError("the input gradient supports stride (1, 1, 1) only")
+            dx = conv3d_bwd_data(dy, w, x.shape, pad, tpad)
+        if ctx.needs_input_grad[1] or (has_bias and ctx.needs_input_grad[2]):
+            dw, db = conv3d_bwd_weight(x, dy, tuple(w.shape[1:4]), stride, pad, tpad,
+                                       with_bias=has_bias)
+            if not ctx.needs_input_grad[1]:
+                dw = None
+        if has_res and ctx.needs_input_grad[3]:
+            dres = dy
+        return dx, dw, db, dres, None, None, None
+
+
+def conv3d_autograd(x, w, bias=None, residual=None, stride=(1, 1, 1), pad=(0, 1, 1),
+                    tpad=TPAD_CAUSAL_REPLICATE):
+    """y = conv3d(x, w) + bias + residual with gradients for x, w, bias and residual."""
+    return Conv3dFunction.apply(x, w, bias, residual, tuple(stride), tuple(pad), tpad)
