@@ -7,8 +7,13 @@ missing or fails to load, importing this package raises.
 
 Operation (engineering.drawthings.ai, "Metal conv3d" post; Qwen Image post,
 "Video VAE" section): y = conv3d(x, w) + bias + residual with NDHWC
-activations, [Cout, kt, kh, kw, Cin] weights, spatial zero padding and a
-temporal padding mode (zero, causal replicate-first-frame, causal zero).
+activations, [Cout, kt, kh, kw, Cin] weights, spatial zero padding, strides
+and a temporal padding mode (zero, causal replicate-first-frame, causal zero,
+or the cached frames of the previous chunk).  Also: the GroupNorm + SiLU pass
+in front of a decoder convolution (groupnorm_stats / groupnorm_silu), the
+backward pass (conv3d_bwd_data, conv3d_bwd_weight) and a torch.autograd
+wrapper over both directions (Conv3dFunction / conv3d_autograd).  Each call has
+a raw-pointer twin (``*_ptr``) that returns the library's status code.
 """
 from __future__ import annotations
 
@@ -19,11 +24,14 @@ import torch
 
 __all__ = [
     "TPAD_ZERO", "TPAD_CAUSAL_REPLICATE", "TPAD_CAUSAL_ZERO", "TPAD_CAUSAL_CACHED", "F16", "BF16",
-    "Status", "conv3d_fwd_cached_ptr", "groupnorm_stats", "groupnorm_silu", "conv3d_bwd_data",
-    "conv3d_bwd_weight", "Conv3dFunction", "conv3d_autograd",
-    "Conv3dError", "lib_path", "conv3d", "conv3d_fwd", "conv3d_fwd_ptr", "conv3d_fwd_ws_ptr",
-    "conv3d_fwd_noalloc_ptr",
-    "output_shape", "workspace_bytes", "poll_status", "selftest_wait_timeout", "release",
+    "Status", "Conv3dError", "lib_path", "status_string", "last_error",
+    "conv3d", "conv3d_fwd", "conv3d_fwd_ptr", "conv3d_fwd_ws_ptr", "conv3d_fwd_noalloc_ptr",
+    "conv3d_fwd_cached_ptr", "output_shape", "workspace_bytes",
+    "groupnorm_stats", "groupnorm_silu", "groupnorm_stats_ptr", "groupnorm_silu_ptr",
+    "conv3d_bwd_data", "conv3d_bwd_data_ptr", "bwd_data_workspace_bytes",
+    "conv3d_bwd_weight", "conv3d_bwd_weight_ptr", "bwd_weight_workspace_bytes",
+    "Conv3dFunction", "conv3d_autograd",
+    "poll_status", "selftest_wait_timeout", "release",
 ]
 
 F16 = 0
