@@ -232,6 +232,7 @@ struct DeviceState {
   bool attr_set[8] = {};         // per kernel variant
   int pair_clusters = 0;         // co-resident CTA pairs (occupancy query)
   int wg_pair_clusters = 0;      // the same for the weight-gradient kernel
+  bool wg_attr_set[8] = {};      // per weight-gradient kernel variant
 };
 
 std::mutex g_mu;
@@ -1067,9 +1068,14 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
                                   : conv3d_wgrad_kernel<false, false, false>);
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         S->max_smem_optin - 64);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    const int wg_variant = (bf16 ? 1 : 0) + (swap ? 2 : 0) + (pair ? 4 : 0);
+    cudaError_t e = cudaSuccess;
+    if (!S->wg_attr_set[wg_variant]) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               S->max_smem_optin - 64);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      S->wg_attr_set[wg_variant] = true;
+    }
     if (pair) {
       if (S->wg_pair_clusters <= 0) {
         cudaLaunchConfig_t cfg = {};
