@@ -144,7 +144,7 @@ def profiled_traffic(wl_name):
 # ---------------------------------------------------------------- clocks (NVML, read only)
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons every ~20 ms while running."""
+    """Samples SM clock and clock-event reasons every ~5 ms while running."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -176,7 +176,7 @@ class ClockSampler:
     def _run(self):
         while not self._stop.is_set():
             self._sample()
-            time.sleep(0.02)
+            time.sleep(0.005)
 
     def _sample(self):
         try:
@@ -204,7 +204,8 @@ class ClockSampler:
         if not self._ok or not self.samples:
             return None
         return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+                "sm_mhz_min": float(min(self.samples)), "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "sm_mhz_series": [int(v) for v in self.samples]}
 
 
 # ---------------------------------------------------------------- oracle (CPU) timing
