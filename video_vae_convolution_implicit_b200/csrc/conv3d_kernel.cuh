@@ -13,7 +13,8 @@
 // padded copy of the input is ever written.
 //
 // One CTA per SM, persistent over output tiles of 128 pixels x BN output
-// channels (or a CTA pair over 256-pixel tiles, see below).  Warp roles
+// channels (or a CTA pair over 256-pixel tiles, or the transposed product
+// for layers with at most 128 output channels: see the kernel).  Warp roles
 // (192 threads):
 //   warp 0     TMA producer: per k-block one im2col load of A (128 pixels x 64
 //              channels of one tap) and one tiled load of B (BN x 64), both
@@ -21,9 +22,11 @@
 //              guarded by full/empty mbarriers;
 //   warp 1     allocates tensor memory and issues tcgen05.mma (M=128, N=BN,
 //              K=16, four per k-block) into one of two fp32 TMEM accumulators;
-//   warps 2-5  epilogue: tcgen05.ld, + bias, + residual, one rounding to the
-//              output type, 16-byte stores; then frees the accumulator so the
-//              next tile's main loop overlaps this tile's epilogue.
+//   warps 2-5  epilogue: tcgen05.ld, + bias, + residual (fetched ahead by
+//              TMA), one rounding to the output type (or fp32 output for the
+//              backward pass's padded frames), staged through swizzled shared
+//              memory and written by TMA stores; then frees the accumulator so
+//              the next tile's main loop overlaps this tile's epilogue.
 // Every mbarrier wait is bounded in time; a wait that runs out records
 // CONV3D_ERR_TIMEOUT in the status word, and all roles leave their loops,
 // drain their asynchronous work and free tensor memory before exiting.
