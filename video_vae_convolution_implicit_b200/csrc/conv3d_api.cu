@@ -232,7 +232,7 @@ struct DeviceState {
   bool attr_set[8] = {};         // per kernel variant
   int pair_clusters = 0;         // co-resident CTA pairs (occupancy query)
   int wg_pair_clusters = 0;      // the same for the weight-gradient kernel
-  bool wg_attr_set[8] = {};      // per weight-gradient kernel variant
+  bool wg_attr_set[16] = {};     // per weight-gradient kernel variant
 };
 
 std::mutex g_mu;
@@ -771,6 +771,50 @@ __global__ void selftest_wait_kernel(int* status, unsigned long long timeout_ns)
   __syncthreads();
 }
 
+using WgradKernel = decltype(&conv3d_wgrad_kernel<true, false, false, WG_PIX>);
+
+// Pixels per stage: 128, or 96 where a 128-pixel stage leaves room for only
+// two stages (see the launch code).  CTA pairs always fit three 128-pixel
+// stages (96-pixel ones measured no faster), so they have one instance.
+template <bool kBF16>
+WgradKernel wgrad_kernel_of(bool swap, bool pair, int pix) {
+  if (pair) return conv3d_wgrad_kernel<kBF16, false, true, 128>;
+  if (swap)
+    return pix == 96 ? conv3d_wgrad_kernel<kBF16, true, false, 96>
+                     : conv3d_wgrad_kernel<kBF16, true, false, 128>;
+  return pix == 96 ? conv3d_wgrad_kernel<kBF16, false, false, 96>
+                   : conv3d_wgrad_kernel<kBF16, false, false, 128>;
+}
+
+WgradKernel wgrad_kernel_for(bool bf16, bool swap, bool pair, int pix) {
+  return bf16 ? wgrad_kernel_of<true>(swap, pair, pix) : wgrad_kernel_of<false>(swap, pair, pix);
+}
+
+// Number of pixel ranges each (tap block, output-channel tile) is split into.
+// The persistent grid runs units in rounds of `sms`; the cost of a choice is
+// the chunks one CTA walks (rounds x chunks per unit) plus a fixed cost per
+// unit for its epilogue (fp32 atomics of a 128 x BN block, about the time of
+// eight 128-pixel chunks).  The cheapest split wins; ties go to fewer splits.
+long long choose_wgrad_splits(long long base_units, long long total_chunks, int sms,
+                              int pix_per_chunk) {
+  const long long kEpilogueChunks = 8 * 128 / pix_per_chunk;
+  long long best = 1;
+  long long best_cost = -1;
+  const long long max_splits = total_chunks < 1024 ? total_chunks : 1024;
+  for (long long s = 1; s <= max_splits; ++s) {
+    const long long units = base_units * s;
+    const long long rounds = (units + sms - 1) / sms;
+    const long long per = (total_chunks + s - 1) / s;
+    const long long cost = rounds * (per + kEpilogueChunks);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+    if (rounds > 64) break;
+  }
+  return best;
+}
+
 }  // namespace
 
 extern "C" {
@@ -939,29 +983,6 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
   return CONV3D_OK;
 }
 
-// Number of pixel ranges each (tap block, output-channel tile) is split into.
-// The persistent grid runs units in rounds of `sms`; the cost of a choice is
-// the chunks one CTA walks (rounds x chunks per unit) plus a fixed cost per
-// unit for its epilogue (fp32 atomics of a 128 x BN block, about the time of
-// eight chunks).  The cheapest split wins; ties go to fewer splits.
-long long choose_wgrad_splits(long long base_units, long long total_chunks, int sms) {
-  constexpr long long kEpilogueChunks = 8;
-  long long best = 1;
-  long long best_cost = -1;
-  const long long max_splits = total_chunks < 1024 ? total_chunks : 1024;
-  for (long long s = 1; s <= max_splits; ++s) {
-    const long long units = base_units * s;
-    const long long rounds = (units + sms - 1) / sms;
-    const long long per = (total_chunks + s - 1) / s;
-    const long long cost = rounds * (per + kEpilogueChunks);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = s;
-    }
-    if (rounds > 64) break;
-  }
-  return best;
-}
 
 size_t conv3d_bwd_weight_workspace_bytes(int Cin, int Cout, const int kernel[3]) {
   if (!kernel || Cin < 1 || Cout < 1) return 0;
@@ -1060,15 +1081,26 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   wp.pairs_per_it = (F.kh * F.kw * wp.cblocks + 1) / 2;
   const int kCtas = pair ? 2 : 1;
   int lanes = S->num_sms;   // co-resident CTAs, or CTA pairs
-  auto kern = bf16 ? (swap ? conv3d_wgrad_kernel<true, true, false>
-                           : pair ? conv3d_wgrad_kernel<true, false, true>
-                                  : conv3d_wgrad_kernel<true, false, false>)
-                   : (swap ? conv3d_wgrad_kernel<false, true, false>
-                           : pair ? conv3d_wgrad_kernel<false, false, true>
-                                  : conv3d_wgrad_kernel<false, false, false>);
+  // Pixels per stage.  A stage holds two 64-channel x boxes and the dy boxes
+  // (plain, pair) or two dy boxes and four x boxes (swapped), 128 bytes per
+  // pixel each.  Three stages in flight keep the tensor cores fed; where
+  // 128-pixel stages leave room for only two (six boxes: the swapped variant,
+  // and one-CTA 256-channel tiles), 96-pixel stages fit three.  Measured on
+  // B200: swapped 128-channel workloads 2 x 128 px 921-1113, 4 x 64 px
+  // 987-1016, 3 x 96 px 1156-1260 TFLOP/s; 1x1x1 512->256 648 -> 677.
+  const int boxes = swap ? 6 : 2 + wp.BN / kCtas / 64;
+  const int reserve = 1024 + 8 * (2 * MAX_STAGES + 5);
+  const int smem_room = S->max_smem_optin - reserve - 64;
+  int pix = smem_room / (boxes * WG_PIX * 128) >= 3 ? WG_PIX : 96;
+  if (const char* env = getenv("CONV3D_WGRAD_PIX")) {
+    const int v = atoi(env);
+    if (!pair && (v == 96 || v == 128)) pix = v;
+  }
+  auto kern = wgrad_kernel_for(bf16, swap, pair, pix);
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    const int wg_variant = (bf16 ? 1 : 0) + (swap ? 2 : 0) + (pair ? 4 : 0);
+    const int kind = swap ? 2 : pair ? 1 : 0;
+    const int wg_variant = 4 * kind + 2 * (pix == 96 ? 1 : 0) + (bf16 ? 1 : 0);
     cudaError_t e = cudaSuccess;
     if (!S->wg_attr_set[wg_variant]) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1097,22 +1129,21 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
       lanes = S->wg_pair_clusters;
     }
   }
-  wp.chunks_per_frame = (wp.HoWo + WG_PIX - 1) / WG_PIX;
+  wp.chunks_per_frame = (wp.HoWo + pix - 1) / pix;
   wp.total_chunks = static_cast<long long>(N) * F.Do * wp.chunks_per_frame;
   const long long base_units =
       swap   ? static_cast<long long>(kt_run) * wp.eblocks * wp.co_tiles
       : pair ? static_cast<long long>(kt_run) * wp.pairs_per_it * wp.co_tiles
              : static_cast<long long>(wp.taps) * wp.cblocks * wp.co_tiles;
-  const long long splits = choose_wgrad_splits(base_units, wp.total_chunks, lanes);
+  const long long splits = choose_wgrad_splits(base_units, wp.total_chunks, lanes, pix);
   if (base_units * splits > 0x7FFFFFFFLL) {
     set_error("problem too large");
     return CONV3D_ERR_UNSUPPORTED;
   }
   wp.splits = static_cast<int>(splits);
   wp.num_units = static_cast<int>(base_units * splits);
-  const int stage_bytes = WG_A_BYTES + (swap ? 4 * WG_PIX * 128 : wp.BN / kCtas * WG_PIX * 2);
-  const int reserve = 1024 + 8 * (2 * MAX_STAGES + 5);
-  int stages = (S->max_smem_optin - reserve - 64) / stage_bytes;
+  const int stage_bytes = boxes * pix * 128;
+  int stages = smem_room / stage_bytes;
   if (stages > MAX_STAGES) stages = MAX_STAGES;
   wp.stages = stages;
   wp.acc_cols = swap ? 256u : static_cast<uint32_t>(wp.BN);
@@ -1124,9 +1155,9 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   wp.timeout_ns = kDefaultTimeoutNs;
   const size_t smem = static_cast<size_t>(stages) * stage_bytes + reserve;
 
-  // x through the forward im2col map (WG_PIX pixels per load); dy as [frames][pixels][Cout]
+  // x through the forward im2col map (pix pixels per load); dy as [frames][pixels][Cout]
   CUtensorMap map_x, map_dy;
-  if ((st = encode_im2col(F, x, static_cast<long long>(N) * D, WG_PIX, map_x)) != CONV3D_OK)
+  if ((st = encode_im2col(F, x, static_cast<long long>(N) * D, pix, map_x)) != CONV3D_OK)
     return st;
   {
     const CUtensorMapDataType dt =
@@ -1135,7 +1166,7 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(Cout), howo,
                                 static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(F.Do)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(Cout) * 2, howo * Cout * 2};
-    const cuuint32_t box[3] = {64, WG_PIX, 1};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(pix), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode_tiled(&map_dy, dt, 3, const_cast<void*>(dy), dims, strides, box, estr,
                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -14,7 +14,10 @@
 // along M/N, 8-row groups 1 KB apart along K).  128 pixels per stage rather
 // than 64 halves the copies and barrier round trips per byte (measured on
 // B200: 1290 -> 1608 TFLOP/s on a 256-channel 9x128x128 layer); 32 was far
-// slower.
+// slower.  A stage of six boxes (the swapped variant below, one-CTA
+// 256-channel tiles) is 96 KB at 128 pixels, so only two fit; those take
+// 96-pixel stages, three of them, so that two stages load while one feeds
+// the MMAs (kPix, chosen on the host).
 //
 // A swapped variant serves layers with at most 128 output channels, where an
 // N = 128 product would take as long as an N = 256 one: M = 128 output
@@ -28,7 +31,7 @@
 // each CTA moves 64 KB per chunk instead of 96 KB for the same products.
 //
 // Work unit = (tap and 128-channel block, output-channel block, range of
-// 128-pixel chunks), or (temporal tap and block of four entries, ...) when
+// kPix-pixel chunks), or (temporal tap and block of four entries, ...) when
 // swapped, or (temporal tap and pair of blocks, ...) for CTA pairs;
 // persistent CTAs (or clusters) walk the units.  Chunks whose temporal tap
 // reads zero padding are skipped by producer and MMA alike; chunk rows past
@@ -69,8 +72,7 @@ struct WgradParams {
   unsigned long long timeout_ns;
 };
 
-constexpr int WG_PIX = 128;                         // pixels (K) per stage
-constexpr int WG_A_BYTES = 2 * WG_PIX * 64 * 2;     // two 64-channel im2col boxes
+constexpr int WG_PIX = 128;                         // pixels (K) per stage, by default
 
 // Shared-memory matrix descriptor for an MN-major operand in 64-element x
 // 8-row atoms with the 128-byte swizzle: leading byte offset = distance of
@@ -186,11 +188,16 @@ __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c
                : "memory");
 }
 
-template <bool kBF16, bool kSwap, bool kPair>
+// kPix = pixels (K) per stage, a multiple of 16: every operand box is kPix
+// rows of 128 bytes (64 channels), and the A stage holds two of them.
+template <bool kBF16, bool kSwap, bool kPair, int kPix>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     conv3d_wgrad_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_dy, const WgradParams p) {
   static_assert(!(kSwap && kPair), "the pair variant is the plain operand assignment");
+  static_assert(kPix % 16 == 0 && kPix <= 256, "pixels per stage");
+  constexpr uint32_t kBox = kPix * 128;          // one 64-channel box
+  constexpr uint32_t kABytes = 2 * kBox;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
   __shared__ int s_abort;
@@ -206,9 +213,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // B operand: dy boxes (plain: BN/64 of them; pair: this CTA's half) or up to
   // four x boxes (swapped)
   const uint32_t b_stage_bytes =
-      kSwap ? 4u * WG_PIX * 128 : static_cast<uint32_t>(p.BN / kCtas) * WG_PIX * 2;
+      kSwap ? 4u * kBox : static_cast<uint32_t>(p.BN / kCtas) * kPix * 2;
   const uint32_t a_ring = base;
-  const uint32_t b_ring = a_ring + p.stages * WG_A_BYTES;
+  const uint32_t b_ring = a_ring + p.stages * kABytes;
   const uint32_t bars = b_ring + p.stages * b_stage_bytes;
   const uint32_t full_bar = bars;
   const uint32_t empty_bar = bars + 8 * p.stages;
@@ -286,16 +293,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int ndy = kSwap ? 2 : p.BN / 64 / kCtas;
         const int dy_c0 = wu.co0 + static_cast<int>(rank) * (p.BN / kCtas);
         const uint32_t x_ring = kSwap ? b_ring : a_ring;
-        const uint32_t x_stage = kSwap ? b_stage_bytes : WG_A_BYTES;
+        const uint32_t x_stage = kSwap ? b_stage_bytes : kABytes;
         const uint32_t dy_ring = kSwap ? a_ring : b_ring;
-        const uint32_t dy_stage = kSwap ? WG_A_BYTES : b_stage_bytes;
-        const uint32_t tx_bytes = static_cast<uint32_t>(kCtas * (nx + ndy)) * (WG_PIX * 128);
+        const uint32_t dy_stage = kSwap ? kABytes : b_stage_bytes;
+        const uint32_t tx_bytes = static_cast<uint32_t>(kCtas * (nx + ndy)) * kBox;
         FrameWalk fw(p, wu);
         while (ok && fw.next(p)) {
           const int f = wg_source_frame(p, fw.to, wu.it);
           if (f < 0) continue;                  // this tap reads zero padding here
           const int img = fw.n * p.D + f;
-          int p0 = fw.pc * WG_PIX;
+          int p0 = fw.pc * kPix;
           int ho0 = p0 / p.Wo;
           int wo0 = p0 - ho0 * p.Wo;
           for (int j = 0; j < fw.count; ++j) {
@@ -313,23 +320,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const uint32_t fb0 = mapa_shared(fb, 0);
 #pragma unroll
               for (int q = 0; q < 2; ++q)
-                tma_load_im2col_4d_pair(x_dst + q * (WG_PIX * 128), &map_x, fb0, bc[q], wx, hx,
+                tma_load_im2col_4d_pair(x_dst + q * kBox, &map_x, fb0, bc[q], wx, hx,
                                         img, static_cast<uint16_t>(bw[q]),
                                         static_cast<uint16_t>(bh[q]));
               for (int q = 0; q < ndy; ++q) {
                 const int dc = dy_c0 + 64 * q < p.Cout ? dy_c0 + 64 * q : wu.co0;
-                tma_load_3d_pair(dy_dst + q * (WG_PIX * 128), &map_dy, fb0, dc, p0,
+                tma_load_3d_pair(dy_dst + q * kBox, &map_dy, fb0, dc, p0,
                                  static_cast<int>(fw.fo));
               }
             } else {
 #pragma unroll
               for (int q = 0; q < 4; ++q)
                 if (q < nx)
-                  tma_load_im2col_4d(x_dst + q * (WG_PIX * 128), &map_x, fb, bc[q], wx, hx, img,
+                  tma_load_im2col_4d(x_dst + q * kBox, &map_x, fb, bc[q], wx, hx, img,
                                      static_cast<uint16_t>(bw[q]), static_cast<uint16_t>(bh[q]));
               for (int q = 0; q < ndy; ++q) {
                 const int dc = dy_c0 + 64 * q < p.Cout ? dy_c0 + 64 * q : wu.co0;
-                tma_load_3d(dy_dst + q * (WG_PIX * 128), &map_dy, fb, dc, p0,
+                tma_load_3d(dy_dst + q * kBox, &map_dy, fb, dc, p0,
                             static_cast<int>(fw.fo));
               }
             }
@@ -338,8 +345,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               stage = 0;
               phase ^= 1;
             }
-            p0 += WG_PIX;
-            wo0 += WG_PIX;
+            p0 += kPix;
+            wo0 += kPix;
             while (wo0 >= p.Wo) {
               wo0 -= p.Wo;
               ++ho0;
@@ -371,8 +378,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int local = 0;
       // descriptors of stage 0; a stage or a K step moves the start address
       // (bits 0-13, in 16-byte units) only
-      const uint64_t da0 = smem_desc_mn_sw128(a_ring, WG_PIX * 128);
-      const uint64_t db0 = smem_desc_mn_sw128(b_ring, WG_PIX * 128);
+      const uint64_t da0 = smem_desc_mn_sw128(a_ring, kBox);
+      const uint64_t db0 = smem_desc_mn_sw128(b_ring, kBox);
       for (int u = first_unit; ok && u < p.num_units; u += unit_step, ++local) {
         const WgUnit wu = wg_decode<kSwap, kPair>(p, u);
         // swapped: N = 64 per entry of the block
@@ -394,10 +401,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               break;
             }
             tc_fence_after();
-            const uint64_t da = da0 + ((stage * WG_A_BYTES) >> 4);
+            const uint64_t da = da0 + ((stage * kABytes) >> 4);
             const uint64_t db = db0 + ((stage * b_stage_bytes) >> 4);
 #pragma unroll
-            for (int k = 0; k < WG_PIX / 16; ++k) {
+            for (int k = 0; k < kPix / 16; ++k) {
               // 16 pixels = two 8-row groups (2 KB) further along K
               if constexpr (kPair)
                 mma_f16_ss_pair(d_tmem, da + k * (2048 >> 4), db + k * (2048 >> 4), idesc,
