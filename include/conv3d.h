@@ -211,7 +211,11 @@ CONV3D_API conv3d_status_t conv3d_groupnorm_silu(const void* x, const double* st
  * transform into the workspace; with causal replicate padding it runs twice
  * (frames 1.. straight into dx, one launch per sample; the kt frames
  * -(kt-1)..0 in fp32 into the workspace, summed into frame 0 with one
- * rounding).
+ * rounding).  For short clips (D - 1 <= 4 kt) the front frames run on a
+ * library-owned high-priority stream, forked from and joined back into
+ * `stream` with events (so the call still orders after and before the
+ * caller's work on `stream`, and can be captured in a CUDA graph), beside the
+ * body on `stream`.
  *
  * Arguments describe the FORWARD problem: dy is [N, Do, Ho, Wo, Cout] (y's
  * shape), w [Cout, kt, kh, kw, Cin], dx [N, D, H, W, Cin] (written).  Supported:
@@ -277,8 +281,8 @@ CONV3D_API const char* conv3d_status_string(conv3d_status_t status);
 /* Text of the last CONV3D_ERR_CUDA / CONV3D_ERR_UNSUPPORTED detail on this thread. */
 CONV3D_API const char* conv3d_last_error(void);
 
-/* Frees the cached per-device workspace.  Not to be called while work that
- * uses it is in flight. */
+/* Frees the cached per-device workspace and the backward pass's auxiliary
+ * stream.  Not to be called while work that uses them is being enqueued. */
 CONV3D_API void conv3d_release(void);
 
 /* Failure-detection self test: launches one CTA that waits, with the same

@@ -170,6 +170,25 @@ def test_bwd_data_deterministic_bitwise():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+@pytest.mark.parametrize("D", [4, 20])
+def test_bwd_data_front_beside_body_equals_sequential(D, monkeypatch):
+    """The causal front frames may run on the library's second stream beside the
+    body (short clips); the result is the same bits as running them one after
+    the other, and the caller's stream sees the finished dx."""
+    x, w, dy, od = grads_problem(2, 64, D, 8, 10, 64, (3, 3, 3), (0, 1, 1), CREP, 23, "bf16")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        a = c3.conv3d_bwd_data(dy, w, x.shape, (0, 1, 1), CREP)
+        a_copy = a.clone()             # ordered after the call on the same stream
+    monkeypatch.setenv("CONV3D_DGRAD_CONCURRENT", "0")
+    b = c3.conv3d_bwd_data(dy, w, x.shape, (0, 1, 1), CREP)
+    torch.cuda.synchronize()
+    assert c3.poll_status() == c3.Status.OK
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(a_copy.view(torch.int16), b.view(torch.int16))
+
+
 @pytest.mark.parametrize("tpad", [CREP, CZERO])
 def test_autograd_function_matches_the_oracle(tpad):
     """Conv3dFunction: one backward through the library gives the oracle's adjoints
