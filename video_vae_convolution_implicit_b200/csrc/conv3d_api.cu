@@ -278,11 +278,18 @@ conv3d_status_t device_state(DeviceState*& out, int& dev) {
 }
 
 // The device's aux stream and events, created on first use; false if they
-// cannot be had (the caller then runs everything on its own stream).
-bool aux_stream(DeviceState& s) {
+// cannot be had (the caller then runs everything on its own stream).  They
+// are not created while `caller` is being captured into a graph: that call
+// runs sequentially, and a later eager call creates them.
+bool aux_stream(DeviceState& s, cudaStream_t caller) {
   std::lock_guard<std::mutex> lock(g_mu);
   if (s.aux) return true;
   if (s.aux_failed) return false;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(caller, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+    cudaGetLastError();
+    return false;
+  }
   int least = 0, greatest = 0;
   cudaStream_t st = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
@@ -997,7 +1004,7 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
   // frames 1419 -> 1404 and 1447 -> 1403.
   bool concurrent = B.body.Do > 0 && D - 1 <= 4 * kernel[0];
   if (const char* env = getenv("CONV3D_DGRAD_CONCURRENT")) concurrent = concurrent && env[0] != '0';
-  if (concurrent) concurrent = aux_stream(*S);
+  if (concurrent) concurrent = aux_stream(*S, stream);
   std::unique_lock<std::mutex> aux_lock;
   cudaStream_t front_stream = stream;
   if (concurrent) {
