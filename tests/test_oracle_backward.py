@@ -7,6 +7,8 @@ pinned separately: for any upstream gradient g,
 and torch.autograd in float64 (with the padding written as explicit ops)
 checks the same gradients with a library routine.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -19,8 +21,47 @@ BF16 = oracle.BF16
 ZERO, CREP, CZERO = oracle.TPAD_ZERO, oracle.TPAD_CAUSAL_REPLICATE, oracle.TPAD_CAUSAL_ZERO
 
 
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
 def dec(b):
     return oracle.decode16(b, BF16)
+
+
+def bf16_bits(a):
+    """float64 array -> bf16 bit patterns (values chosen exactly representable)."""
+    t = torch.from_numpy(np.asarray(a, dtype=np.float64)).to(torch.float32).to(torch.bfloat16)
+    return si.bits(t)
+
+
+def test_golden_box_sum_backward():
+    """Hand-worked adjoints of the all-ones 3x3x3 kernel on a 2-frame 3x3 clip
+    (tests/golden/box_sum_backward.txt), in all three temporal padding modes."""
+    rows = []
+    with open(os.path.join(HERE, "golden", "box_sum_backward.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                mode, which, a, b, c, v = line.split()
+                rows.append((int(mode), which, int(a), int(b), int(c), float(v)))
+    assert len(rows) == 3 * (18 + 27 + 1)
+    frame0 = np.arange(1, 10, dtype=np.float64).reshape(3, 3)
+    x = np.stack([frame0, 10 * frame0]).reshape(1, 2, 3, 3, 1)
+    w = np.ones((1, 3, 3, 3, 1))
+    dy = np.stack([np.ones((3, 3)), 2 * np.ones((3, 3))]).reshape(1, 2, 3, 3, 1)
+    for mode in (ZERO, CREP, CZERO):
+        pad = (1, 1, 1) if mode == ZERO else (0, 1, 1)
+        dx, dw, db = oracle.conv3d_backward(bf16_bits(x), bf16_bits(w), bf16_bits(dy), BF16,
+                                            (3, 3, 3), (1, 1, 1), pad, mode)
+        seen = 0
+        for m, which, a, b, c, expect in rows:
+            if m != mode:
+                continue
+            got = {"dx": lambda: dx[0, a, b, c, 0], "dw": lambda: dw[0, a, b, c, 0],
+                   "db": lambda: db[0]}[which]()
+            assert got == expect, (mode, which, a, b, c, got, expect)
+            seen += 1
+        assert seen == 46
 
 
 def problem(N, Cin, D, H, W, Cout, k, stride, pad, tpad, seed):
