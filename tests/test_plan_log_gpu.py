@@ -1,0 +1,52 @@
+"""CONV3D_LOG=1: every kernel launch reports the plan chosen for it on stderr.
+
+The switch is read once per process, so each case runs in a fresh interpreter.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+SCRIPT = """
+import torch
+import seeded_inputs as si
+import video_vae_convolution_implicit_b200 as c3
+x = si.tensor((1, 3, 8, 8, 64), 7, 0, 1.0, torch.bfloat16, "cuda")
+w = si.tensor((64, 3, 3, 3, 64), 7, 1, (27 * 64) ** -0.5, torch.bfloat16, "cuda")
+y = c3.conv3d(x, w)
+dx = c3.conv3d_bwd_data(y, w, x.shape)
+dw, db = c3.conv3d_bwd_weight(x, y, (3, 3, 3))
+assert c3.poll_status() == c3.Status.OK
+"""
+
+
+def _run(log):
+    env = dict(os.environ)
+    env.pop("CONV3D_LOG", None)
+    if log:
+        env["CONV3D_LOG"] = "1"
+    return subprocess.run([sys.executable, "-c", SCRIPT], cwd=ROOT, env=env,
+                          capture_output=True, text=True, timeout=600)
+
+
+def test_plan_log_reports_each_launch():
+    r = _run(True)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stderr.splitlines() if l.startswith("libconv3d: ")]
+    # forward, then the data gradient (its plan line, front and body launches),
+    # then the weight gradient
+    assert any("implicit GEMM" in l and "16-bit output" in l for l in lines), lines
+    assert any("implicit GEMM" in l and "fp32 output" in l for l in lines), lines
+    assert any(l.startswith("libconv3d: data gradient: 3 front frames") for l in lines), lines
+    assert any(l.startswith("libconv3d: weight gradient") for l in lines), lines
+
+
+def test_plan_log_is_silent_by_default():
+    r = _run(False)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert "libconv3d: " not in r.stderr

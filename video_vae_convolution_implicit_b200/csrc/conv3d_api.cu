@@ -39,6 +39,16 @@ conv3d_status_t cuda_fail(cudaError_t e, const char* what) {
   return CONV3D_ERR_CUDA;
 }
 
+// CONV3D_LOG=1: one line per kernel launch on stderr with the plan chosen for
+// it (variant, tiles, grid, pipeline depth), read once per process.
+bool plan_log() {
+  static const bool on = [] {
+    const char* env = getenv("CONV3D_LOG");
+    return env != nullptr && env[0] == '1';
+  }();
+  return on;
+}
+
 // ------------------------------------------------------------------ problem
 
 struct Problem {
@@ -559,6 +569,14 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = kPair ? 1 : 0;
+  if (plan_log())
+    fprintf(stderr,
+            "libconv3d: implicit GEMM %s %s, %d tiles of %d pixels x %d channels, grid %d, "
+            "%d k-blocks x %d taps, %d stages, %zu B shared, %s output\n",
+            kSwap ? "transposed" : kPair ? "CTA pair" : "single", kBF16 ? "bf16" : "fp16",
+            L.kp.num_tiles, L.kp.pix_tile, L.kp.co_tile, static_cast<int>(cfg.gridDim.x),
+            L.kp.n_chunks, L.kp.kt * L.kp.kh * L.kp.kw, L.kp.stages, L.smem,
+            L.kp.out_f32 ? "fp32" : "16-bit");
   e = cudaLaunchKernelEx(&cfg, kern, map_a, map_b, map_y, map_r, map_p, L.kp);
   if (e != cudaSuccess) return cuda_fail(e, "conv3d kernel launch");
   e = cudaGetLastError();
@@ -1005,6 +1023,9 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
   bool concurrent = B.body.Do > 0 && D - 1 <= 4 * kernel[0];
   if (const char* env = getenv("CONV3D_DGRAD_CONCURRENT")) concurrent = concurrent && env[0] != '0';
   if (concurrent) concurrent = aux_stream(*S, stream);
+  if (plan_log())
+    fprintf(stderr, "libconv3d: data gradient: %d front frames %s %d body frames x %d samples\n",
+            kernel[0], concurrent ? "beside" : "before", B.body.Do, N);
   std::unique_lock<std::mutex> aux_lock;
   cudaStream_t front_stream = stream;
   if (concurrent) {
@@ -1258,6 +1279,13 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = pair ? 1 : 0;
+    if (plan_log())
+      fprintf(stderr,
+              "libconv3d: weight gradient %s %s, %d units (%d splits of %lld chunks of %d pixels), "
+              "grid %d, %d stages, %zu B shared\n",
+              swap ? "transposed" : pair ? "CTA pair" : "plain", bf16 ? "bf16" : "fp16",
+              wp.num_units, wp.splits, wp.total_chunks, pix, static_cast<int>(cfg.gridDim.x),
+              wp.stages, smem);
     e = cudaLaunchKernelEx(&cfg, kern, map_x, map_dy, wp);
     if (e != cudaSuccess) return cuda_fail(e, "wgrad kernel launch");
   }
