@@ -85,6 +85,15 @@ def test_golden_box_sum():
         for m, to, ho, wo, expect in rows:
             if m == mode:
                 assert y[0, to, ho, wo, 0] == expect, (mode, to, ho, wo)
+        # Stride 2 on every axis keeps the windows that start at even positions:
+        # Do = Ho = Wo = 1 + (padded extent - 3) / 2 = 1, 2, 2, and output
+        # (0, i, j) is the stride-1 output (0, 2i, 2j) of the same fixture.
+        ys = oracle.conv3d(bf16_bits(x), bf16_bits(w), bf16_bits(b), None, BF16,
+                           (3, 3, 3), (2, 2, 2), pad, mode)
+        assert ys.shape == (1, 1, 2, 2, 1)
+        for m, to, ho, wo, expect in rows:
+            if m == mode and to == 0 and ho % 2 == 0 and wo % 2 == 0:
+                assert ys[0, 0, ho // 2, wo // 2, 0] == expect, ("stride 2", mode, ho, wo)
 
 
 # ---------------------------------------------------------------- output size
