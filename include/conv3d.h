@@ -103,7 +103,9 @@ CONV3D_API conv3d_status_t conv3d_fwd(const void* x, const void* w, const void* 
 
 /* conv3d_fwd with caller-provided device scratch (never allocates).
  * `workspace` must be 256-byte aligned and hold conv3d_workspace_bytes();
- * it may be NULL when that is 0.  Too small -> CONV3D_ERR_WORKSPACE. */
+ * it may be NULL when that is 0.  Too small -> CONV3D_ERR_WORKSPACE.  When it
+ * is used, it must not overlap x, w, bias, residual or y
+ * (CONV3D_ERR_INVALID_ARG). */
 CONV3D_API conv3d_status_t conv3d_fwd_ws(const void* x, const void* w, const void* bias,
                                          const void* residual, void* y, int N, int Cin, int D,
                                          int H, int W, int Cout, const int kernel[3],
@@ -264,12 +266,30 @@ CONV3D_API conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void
                                              size_t ws_bytes, struct CUstream_st* stream);
 CONV3D_API size_t conv3d_bwd_weight_workspace_bytes(int Cin, int Cout, const int kernel[3]);
 
-/* Device scratch bytes conv3d_fwd_ws needs for this problem (0 if none). */
-CONV3D_API size_t conv3d_workspace_bytes(int Cin, int Cout, int D, const int kernel[3], conv3d_tpad_t tpad);
+/*
+ * Utilities.  The pages describe no API; these complete the convolution call
+ * above.  conv3d_workspace_bytes and conv3d_output_shape restate the
+ * problem's sizes (Qwen Image post, "Video VAE": the first-frame fold is the
+ * only step that needs scratch; the output extents follow from the padding
+ * rules at the top of this file).  conv3d_poll_status, conv3d_status_string,
+ * conv3d_last_error and conv3d_release exist because every call only enqueues
+ * work on the caller's stream and never synchronises (A1111 Metal discussion:
+ * a native op enqueues into the host framework's command stream rather than
+ * committing per call), so device-side errors must be collected separately.
+ */
 
-/* Output extents {Do, Ho, Wo} for the problem; CONV3D_ERR_INVALID_ARG if any is < 1. */
-CONV3D_API conv3d_status_t conv3d_output_shape(int D, int H, int W, const int kernel[3], const int stride[3],
-                                    const int pad[3], conv3d_tpad_t tpad, int out_dhw[3]);
+/* Device scratch bytes conv3d_fwd_ws needs for this problem: the folded
+ * first-frame weight for CONV3D_TPAD_CAUSAL_REPLICATE with D == 1 and kt > 1,
+ * 0 otherwise (also 0 for invalid sizes or a NULL kernel). */
+CONV3D_API size_t conv3d_workspace_bytes(int Cin, int Cout, const int kernel[3], int D,
+                                         conv3d_tpad_t tpad);
+
+/* Output extents {Do, Ho, Wo} for the problem (formula at the top of this
+ * file).  Returns CONV3D_ERR_INVALID_ARG, leaving out_dhw untouched, for a
+ * NULL array, a non-positive size, an unknown mode or an output extent < 1. */
+CONV3D_API conv3d_status_t conv3d_output_shape(int D, int H, int W, const int kernel[3],
+                                               const int stride[3], const int pad[3],
+                                               conv3d_tpad_t tpad, int out_dhw[3]);
 
 /* Synchronises `stream`, then returns and clears the device status word of the
  * current device (CONV3D_OK, CONV3D_ERR_TIMEOUT or CONV3D_ERR_DEVICE_CHECK). */
@@ -281,8 +301,9 @@ CONV3D_API const char* conv3d_status_string(conv3d_status_t status);
 /* Text of the last CONV3D_ERR_CUDA / CONV3D_ERR_UNSUPPORTED detail on this thread. */
 CONV3D_API const char* conv3d_last_error(void);
 
-/* Frees the cached per-device workspace and the backward pass's auxiliary
- * stream.  Not to be called while work that uses them is being enqueued. */
+/* Frees the cached per-device workspace, the cached tensor maps and the
+ * backward pass's auxiliary stream.  Not to be called while work that uses
+ * them is being enqueued. */
 CONV3D_API void conv3d_release(void);
 
 /* Failure-detection self test: launches one CTA that waits, with the same

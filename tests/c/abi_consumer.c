@@ -42,9 +42,9 @@ static int cpu_checks(void) {
   CHECK(out[0] == 9 && out[1] == 64 && out[2] == 64);
   CHECK(conv3d_output_shape(5, 32, 32, k3, s1, p_zero, CONV3D_TPAD_ZERO, out) == CONV3D_OK);
   CHECK(out[0] == 5);
-  CHECK(conv3d_workspace_bytes(256, 256, 1, k3, CONV3D_TPAD_CAUSAL_REPLICATE) ==
+  CHECK(conv3d_workspace_bytes(256, 256, k3, 1, CONV3D_TPAD_CAUSAL_REPLICATE) ==
         (size_t)2 * 256 * 9 * 256 * 2);
-  CHECK(conv3d_workspace_bytes(256, 256, 9, k3, CONV3D_TPAD_CAUSAL_REPLICATE) == 0);
+  CHECK(conv3d_workspace_bytes(256, 256, k3, 9, CONV3D_TPAD_CAUSAL_REPLICATE) == 0);
   CHECK(strcmp(conv3d_status_string(CONV3D_OK), "ok") == 0);
   /* fake, never dereferenced device addresses */
   const void* x = (const void*)0x100000000ull;

@@ -77,11 +77,11 @@ def test_output_shape_rejects_empty():
 
 def test_workspace_bytes():
     # first-frame fold: (hi, lo) x Cout*kh*kw*Cin 16-bit values, rounded up to 256 bytes
-    assert c3.workspace_bytes(256, 256, 1, (3, 3, 3), c3.TPAD_CAUSAL_REPLICATE) == 2 * 256 * 9 * 256 * 2
-    assert c3.workspace_bytes(8, 8, 1, (3, 3, 3), c3.TPAD_CAUSAL_REPLICATE) == 2304
-    assert c3.workspace_bytes(256, 256, 2, (3, 3, 3), c3.TPAD_CAUSAL_REPLICATE) == 0
-    assert c3.workspace_bytes(256, 256, 1, (3, 3, 3), c3.TPAD_CAUSAL_ZERO) == 0
-    assert c3.workspace_bytes(256, 256, 1, (1, 3, 3), c3.TPAD_CAUSAL_REPLICATE) == 0
+    assert c3.workspace_bytes(256, 256, (3, 3, 3), 1, c3.TPAD_CAUSAL_REPLICATE) == 2 * 256 * 9 * 256 * 2
+    assert c3.workspace_bytes(8, 8, (3, 3, 3), 1, c3.TPAD_CAUSAL_REPLICATE) == 2304
+    assert c3.workspace_bytes(256, 256, (3, 3, 3), 2, c3.TPAD_CAUSAL_REPLICATE) == 0
+    assert c3.workspace_bytes(256, 256, (3, 3, 3), 1, c3.TPAD_CAUSAL_ZERO) == 0
+    assert c3.workspace_bytes(256, 256, (1, 3, 3), 1, c3.TPAD_CAUSAL_REPLICATE) == 0
 
 
 def call(**kw):
@@ -126,10 +126,15 @@ def test_ws_entry_point_requires_workspace_for_first_frame():
              kernel=(3, 3, 3), stride=(1, 1, 1), pad=(0, 1, 1), tpad=c3.TPAD_CAUSAL_REPLICATE,
              dtype=c3.BF16, stream=None)
     assert c3.conv3d_fwd_ws_ptr(**a, workspace=None, ws_bytes=0) == Status.WORKSPACE
-    need = c3.workspace_bytes(64, 64, 1, (3, 3, 3), c3.TPAD_CAUSAL_REPLICATE)
+    need = c3.workspace_bytes(64, 64, (3, 3, 3), 1, c3.TPAD_CAUSAL_REPLICATE)
     assert c3.conv3d_fwd_ws_ptr(**a, workspace=0x600000000, ws_bytes=need - 1) == Status.WORKSPACE
     assert c3.conv3d_fwd_ws_ptr(**a, workspace=0x600000010, ws_bytes=need) == Status.ALIGNMENT
     assert c3.conv3d_fwd_ws_ptr(**a, workspace=Wt, ws_bytes=need) == Status.INVALID_ARG
+    # the main kernel reads bias and residual after the fold wrote the workspace
+    assert c3.conv3d_fwd_ws_ptr(**a, workspace=B, ws_bytes=need) == Status.INVALID_ARG
+    a["residual"] = R
+    assert c3.conv3d_fwd_ws_ptr(**a, workspace=R, ws_bytes=need) == Status.INVALID_ARG
+    assert "residual" in c3.last_error()
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")

@@ -102,7 +102,7 @@ def test_first_frame_fold(dt, cta_mode):
 
 def test_first_frame_fold_explicit_workspace():
     p = problem(1, 128, 1, 16, 20, 64, (3, 3, 3), (0, 1, 1), CREP, seed=6)
-    need = c3.workspace_bytes(128, 64, 1, (3, 3, 3), CREP)
+    need = c3.workspace_bytes(128, 64, (3, 3, 3), 1, CREP)
     ws = torch.empty(need, dtype=torch.uint8, device="cuda")
     ref = oracle_ref(p)
     y = run(p, workspace=ws)

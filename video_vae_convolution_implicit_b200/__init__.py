@@ -94,7 +94,7 @@ _lib.conv3d_bwd_weight_workspace_bytes.argtypes = [_c, _c, _i3]
 _lib.conv3d_fwd_noalloc.restype = _c
 _lib.conv3d_fwd_noalloc.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp]
 _lib.conv3d_workspace_bytes.restype = ctypes.c_size_t
-_lib.conv3d_workspace_bytes.argtypes = [_c, _c, _c, _i3, _c]
+_lib.conv3d_workspace_bytes.argtypes = [_c, _c, _i3, _c, _c]
 _lib.conv3d_output_shape.restype = _c
 _lib.conv3d_output_shape.argtypes = [_c, _c, _c, _i3, _i3, _i3, _c, _i3]
 _lib.conv3d_poll_status.restype = _c
@@ -149,8 +149,8 @@ def output_shape(D, H, W, kernel, stride=(1, 1, 1), pad=(0, 1, 1), tpad=TPAD_CAU
     return tuple(out)
 
 
-def workspace_bytes(Cin, Cout, D, kernel, tpad) -> int:
-    return int(_lib.conv3d_workspace_bytes(Cin, Cout, D, _i3(*kernel), tpad))
+def workspace_bytes(Cin, Cout, kernel, D, tpad) -> int:
+    return int(_lib.conv3d_workspace_bytes(Cin, Cout, _i3(*kernel), D, tpad))
 
 
 def conv3d_fwd_ptr(x, w, bias, residual, y, N, Cin, D, H, W, Cout, kernel, stride, pad, tpad,

@@ -908,9 +908,13 @@ conv3d_status_t conv3d_fwd_ws(const void* x, const void* w, const void* bias, co
     }
     const size_t wsz = static_cast<size_t>(Cout) * kernel[0] * kernel[1] * kernel[2] * Cin * 2;
     const size_t ysz = static_cast<size_t>(N) * P.Do * P.Ho * P.Wo * Cout * 2;
+    // the main kernel reads bias and residual after the fold has written the
+    // workspace, so the workspace may overlap no operand at all
     if (overlaps(workspace, need, w, wsz) || overlaps(workspace, need, y, ysz) ||
-        overlaps(workspace, need, x, static_cast<size_t>(N) * D * H * W * Cin * 2)) {
-      set_error("workspace must not overlap x, w or y");
+        overlaps(workspace, need, x, static_cast<size_t>(N) * D * H * W * Cin * 2) ||
+        overlaps(workspace, need, residual, ysz) ||
+        overlaps(workspace, need, bias, static_cast<size_t>(Cout) * 2)) {
+      set_error("workspace must not overlap x, w, bias, residual or y");
       return CONV3D_ERR_INVALID_ARG;
     }
   }
@@ -1331,7 +1335,7 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   return CONV3D_OK;
 }
 
-size_t conv3d_workspace_bytes(int Cin, int Cout, int D, const int kernel[3], conv3d_tpad_t tpad) {
+size_t conv3d_workspace_bytes(int Cin, int Cout, const int kernel[3], int D, conv3d_tpad_t tpad) {
   if (!kernel || Cin < 1 || Cout < 1 || D < 1) return 0;
   if (tpad == CONV3D_TPAD_CAUSAL_REPLICATE && D == 1 && kernel[0] > 1)
     return fold_bytes(Cin, Cout, kernel);
