@@ -6,7 +6,12 @@ One step = one conv3d_fwd call over one synthetic batch (every stage of the
 path: for this workload one kernel launch).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
-                  [--pass fwd|dgrad|wgrad] [--no-e2e] [--no-cpu-baseline]
+                  [--pass fwd|dgrad|wgrad] [--no-e2e] [--no-cpu-baseline] [--no-per-workload]
+
+With the default workload the line also carries ``per_workload``: every other
+decoder workload (cfg1, cfg3, cfg4, cfg5a-d) measured the same way in the same
+process -- its own TFLOP/s, roofline, sampled parity against the oracle and
+clocks.
 
 Workloads: the convolutions cfg1..cfg5d, cfg2c (cached frames), cfg2s (stride), cfg4s, and the
 GroupNorm + SiLU passes gn_cfg2, gn_cfg4.  --pass dgrad|wgrad times the backward passes of a
@@ -364,15 +369,47 @@ def whole_job_tflops(flops_per_rank_step, world, steps, max_ms):
 
 # ---------------------------------------------------------------- our arm
 
-def run_ours(args, wl, rank, world, local_rank):
-    import video_vae_convolution_implicit_b200 as c3
+PER_WORKLOAD = ("cfg1", "cfg3", "cfg4", "cfg5a", "cfg5b", "cfg5c", "cfg5d")
+
+
+def forward_launches(wl):
+    """Library kernel launches per conv3d_fwd call: the main kernel, plus the
+    first-frame fold for a single causal-replicate frame."""
+    return 1 + (1 if (wl.tpad == 1 and wl.D == 1 and wl.kernel[0] > 1) else 0)
+
+
+def roofline_for(flops, abytes, kernel_ms, peaks, peak_kind):
+    """The roofline that bounds a workload: tensor above the ridge point, HBM below."""
+    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    if flops / abytes >= ridge:
+        roof = {"bound": "tensor", "achieved": flops / (kernel_ms * 1e-3) / 1e12,
+                "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                "peak_source": f"{peak_kind} bf16_tflops (burst)"}
+    else:
+        roof = {"bound": "hbm", "achieved": abytes / (kernel_ms * 1e-3) / 1e9,
+                "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                "peak_source": f"{peak_kind} hbm_gbs"}
+    return dict(roof, frac=roof["achieved"] / roof["peak"],
+                frac_of_spec=roof["achieved"] / SPEC_PEAKS[roof["unit"]],
+                # long runs settle under the power cap: the measured sustained
+                # cuBLAS figure is the matching denominator there
+                frac_of_sustained=(roof["achieved"] / float(peaks["bf16_tflops_sustained"])
+                                   if roof["bound"] == "tensor" and
+                                   "bf16_tflops_sustained" in peaks else None),
+                algorithmic_flops_per_launch=flops, algorithmic_bytes_per_launch=abytes,
+                flop_per_byte=flops / abytes, ridge_flop_per_byte=ridge)
+
+
+def measure_forward(args, wl, rank, world, local_rank, c3, keep=False):
+    """One workload: seeded inputs on the device, warm-up, then args.steps
+    conv3d_fwd calls, each bracketed by CUDA events on the launching stream
+    with the L2 flushed in between; the slowest rank's total time.  Returns
+    the measurement and (when `keep`) the problem tensors for the e2e leg."""
     dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
     dt = TORCH_DTYPE[wl.dtype]
     Do, Ho, Wo = out_shape(wl)
-    seed = rank_seed(wl, rank)
-    p = si.conv3d_problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, (Do, Ho, Wo), seed,
-                          dt, True, wl.residual, dev, prev_frames(wl))
+    p = si.conv3d_problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, (Do, Ho, Wo),
+                          rank_seed(wl, rank), dt, True, wl.residual, dev, prev_frames(wl))
     y = torch.empty((wl.N, Do, Ho, Wo, wl.Cout), dtype=dt, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(2 * l2 // 4 + 1024, dtype=torch.float32, device=dev)
@@ -382,13 +419,12 @@ def run_ours(args, wl, rank, world, local_rank):
         c3.conv3d_fwd(p["x"], p["w"], p["bias"], p["residual"], y, wl.stride, wl.pad, wl.tpad,
                       stream=stream, prev=p["prev"])
 
-    launches_per_step = 1 + (1 if (wl.tpad == 1 and wl.D == 1 and wl.kernel[0] > 1) else 0)
     for _ in range(max(3, args.warmup)):
         flush.zero_()
         step()
     torch.cuda.synchronize(dev)
     if c3.poll_status(stream) != c3.Status.OK:
-        raise RuntimeError("device status after warm-up is not OK")
+        raise RuntimeError(f"{wl.name}: device status after warm-up is not OK")
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -408,48 +444,27 @@ def run_ours(args, wl, rank, world, local_rank):
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    my_ms = sum(step_ms)
-    max_ms = max_over_ranks(my_ms, dev)
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    max_ms = max_over_ranks(sum(step_ms), dev)
     status = c3.poll_status(stream)
 
     flops = algorithmic_flops(wl)
-    ms_per_step = max_ms / args.steps
-    value = whole_job_tflops(flops, world, args.steps, max_ms)
     peaks, peak_kind = load_peaks()
-    kernel_ms = statistics.mean(step_ms)  # one conv kernel launch per step for T > 1
+    # the dominant kernel's launch duration: the whole call's (for the first
+    # frame the call also runs the short weight fold, so this is a lower bound)
+    kernel_ms = statistics.mean(step_ms)
     abytes = algorithmic_bytes(wl)
-    # the roofline that bounds this workload: tensor above the ridge point, HBM below
-    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
-    if flops / abytes >= ridge:
-        roof = {"bound": "tensor", "achieved": flops / (kernel_ms * 1e-3) / 1e12,
-                "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
-                "peak_source": f"{peak_kind} bf16_tflops (burst)"}
-    else:
-        roof = {"bound": "hbm", "achieved": abytes / (kernel_ms * 1e-3) / 1e9,
-                "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
-                "peak_source": f"{peak_kind} hbm_gbs"}
-
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": wl.dtype, "data": "synthetic (seeded SplitMix64 normals; no model weights)",
-        "config": dict(describe(wl, world), l2="flushed (2x L2 write) between timed steps"),
-        "roofline": dict(roof, frac=roof["achieved"] / roof["peak"],
-                         frac_of_spec=roof["achieved"] / SPEC_PEAKS[roof["unit"]],
-                         # long runs settle under the power cap: the measured sustained
-                         # cuBLAS figure is the matching denominator there
-                         frac_of_sustained=(roof["achieved"] / float(peaks["bf16_tflops_sustained"])
-                                            if roof["bound"] == "tensor" and
-                                            "bf16_tflops_sustained" in peaks else None),
-                         traffic=profiled_traffic(wl.name), kernel=KERNEL_NAME,
-                         algorithmic_flops_per_launch=flops,
-                         algorithmic_bytes_per_launch=abytes,
-                         flop_per_byte=flops / abytes, ridge_flop_per_byte=ridge),
+    roof = roofline_for(flops, abytes, kernel_ms, peaks, peak_kind)
+    roof.update(traffic=profiled_traffic(wl.name), kernel=KERNEL_NAME,
+                timed=("whole call: the weight fold and the main kernel" if forward_launches(wl) > 1
+                       else "the one kernel launch of the call"))
+    res = {
+        "value": whole_job_tflops(flops, world, args.steps, max_ms), "unit": "TFLOP/s",
+        "ms_per_step": max_ms / args.steps,
+        "roofline": roof,
         "nominal_tflops": whole_job_tflops(nominal_flops(wl), world, args.steps, max_ms),
         "algorithmic_gbs": abytes * world * args.steps / (max_ms * 1e-3) / 1e9,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": forward_launches(wl) * args.steps,
         "clocks": clocks.summary(),
         "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms),
                     "p90": sorted(step_ms)[int(0.9 * (len(step_ms) - 1))], "max": max(step_ms),
@@ -458,21 +473,57 @@ def run_ours(args, wl, rank, world, local_rank):
                                        for i in range(4)) if q]},
         "region_ms": region0.elapsed_time(region1),
         "device_status": c3.status_string(status),
+        "status_ok": status == c3.Status.OK,
     }
+    if rank == 0:
+        res["parity"] = parity_sample(wl, p, y)
+    kept = (p, y, stream, dev, flops) if keep else None
+    del flush
+    return res, kept
+
+
+def run_ours(args, wl, rank, world, local_rank):
+    import video_vae_convolution_implicit_b200 as c3
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    res, (p, y, stream, dev, flops) = measure_forward(args, wl, rank, world, local_rank, c3,
+                                                      keep=True)
+    status_ok = res.pop("status_ok")
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic (seeded SplitMix64 normals; no model weights)",
+        "config": dict(describe(wl, world), l2="flushed (2x L2 write) between timed steps"),
+    }
+    line.update({k: v for k, v in res.items() if k not in ("value", "unit", "ms_per_step")})
 
     # end to end through the public API from pinned host buffers
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, wl, p, y, stream, dev, c3, flops)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, p)
+        line["speedup_over_oracle"] = line["value"] / line["cpu_baseline"]["value"]
+    del p, y
+    ok = status_ok and (rank != 0 or line["parity"]["ok"])
 
-    # parity gate on sampled rows (a timing is reported only with a passing check)
-    if rank == 0:
-        line["parity"] = parity_sample(wl, p, y)
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(wl, p)
-            line["speedup_over_oracle"] = value / line["cpu_baseline"]["value"]
+    # every other decoder workload, each measured the same way in this process
+    if not args.no_per_workload and wl.name == "cfg2":
+        per = {}
+        for name in PER_WORKLOAD:
+            other = WORKLOADS[name]
+            r, _ = measure_forward(args, other, rank, world, local_rank, c3)
+            r_ok = r.pop("status_ok")
+            if r.get("clocks"):
+                r["clocks"].pop("sm_mhz_series", None)
+            r["config"] = describe(other, world)
+            per[name] = r
+            ok = ok and r_ok and (rank != 0 or r["parity"]["ok"])
+            torch.cuda.empty_cache()
+        line["per_workload"] = per
+
     if rank == 0:
         print(json.dumps(line), flush=True)
-    ok = status == c3.Status.OK and (rank != 0 or line["parity"]["ok"])
     return 0 if ok else 1
 
 
@@ -570,6 +621,8 @@ def parity_sample(wl, p, y):
 
 
 def cpu_baseline(wl, p):
+    """The oracle as it stands on a bounded random sample of the workload's
+    output pixels (about CONV3D_CPU_BASELINE_SECONDS of CPU work)."""
     import oracle
     hb = host_bits(p)
     Do, Ho, Wo = out_shape(wl)
@@ -908,6 +961,8 @@ def main():
                     help="forward convolution (default) or one of its backward passes")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="with the default workload, skip the other decoder workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -313,6 +313,19 @@ CONV3D_API void conv3d_release(void);
  * status word is cleared before returning. */
 CONV3D_API conv3d_status_t conv3d_selftest_wait_timeout(int timeout_ms);
 
+/* Failure-detection test hook.  Arms the next `launches` launches of the
+ * convolution kernels (the forward kernel, which the data gradient also runs,
+ * and the weight-gradient kernel) so that their TMA producer skips the copies
+ * of its first pipeline stage: the tensor-core issuer's bounded wait on that
+ * stage then runs out after timeout_ms (1..10000).  launches = 0 disarms.  An
+ * armed launch aborts the way any timed-out wait does -- every role leaves its
+ * loop, the copies already in flight land, tensor memory is freed and the
+ * kernel returns -- so nothing faults and the context stays usable;
+ * conv3d_poll_status() then reports CONV3D_ERR_TIMEOUT and the call's output
+ * is unspecified.  Process-wide: arm it only while no other thread enqueues
+ * convolutions.  CONV3D_ERR_INVALID_ARG for arguments out of range. */
+CONV3D_API conv3d_status_t conv3d_test_arm_stall(int launches, int timeout_ms);
+
 #ifdef __cplusplus
 }
 #endif

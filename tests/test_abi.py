@@ -289,3 +289,11 @@ def test_bwd_entries_without_gpu_report_cuda_error():
 def test_autograd_function_is_exported():
     assert issubclass(c3.Conv3dFunction, torch.autograd.Function)
     assert callable(c3.conv3d_autograd)
+
+
+def test_arm_stall_rejects_bad_arguments():
+    # the failure-detection hook validates before touching anything
+    for launches, ms in ((-1, 50), (1, 0), (1, 20000)):
+        with pytest.raises(c3.Conv3dError):
+            c3.test_arm_stall(launches, ms)
+    c3.test_arm_stall(0, 50)

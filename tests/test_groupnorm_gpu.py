@@ -34,8 +34,11 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("silu_form", ["tanh", "exp"])
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"{'x'.join(map(str, c[0]))}-g{c[1]}-pf{int(c[2])}-{c[3]}")
-def test_groupnorm_silu_every_element(case):
+def test_groupnorm_silu_every_element(case, silu_form, monkeypatch):
+    # the default one-special-function SiLU (tanh) and the exp/division form
+    monkeypatch.setenv("CONV3D_GN_SILU", silu_form)
     shape, G, pf, dt, mean, std = case
     x, gamma, beta = make(shape, 7, dt, mean, std)
     stats = c3.groupnorm_stats(x, G, eps=1e-6, per_frame=pf)
@@ -66,3 +69,26 @@ def test_in_place_and_without_silu():
     ref = oracle.groupnorm_silu(xb, si.bits(gamma), si.bits(beta), oracle.BF16, 8, eps=1e-6,
                                 silu=False)
     assert_close(x.double().cpu().numpy(), ref)
+
+
+def test_silu_tanh_form_over_the_whole_bf16_range(monkeypatch):
+    # every bf16 value in [-40, 40] as a pre-activation (gamma 1, beta 0, and
+    # statistics that make the normalisation the identity), against the exact
+    # silu in fp64: the default tanh form must stay within the parity bounds
+    # element by element, including the far negative tail where sigmoid is tiny
+    monkeypatch.delenv("CONV3D_GN_SILU", raising=False)
+    codes = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = oracle.decode16(codes, oracle.BF16)
+    keep = np.isfinite(vals) & (np.abs(vals) <= 40.0)
+    v = vals[keep]
+    v = v[: (v.size // 8) * 8]
+    x = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).cuda().view(1, 1, 1, -1, 8)
+    stats = torch.tensor([[[0.0, 1.0]]], dtype=torch.float64, device="cuda")
+    y = c3.groupnorm_silu(x, stats, None, None, groups=1, per_frame=False)
+    torch.cuda.synchronize()
+    got = y.double().cpu().numpy().ravel()
+    ref = v / (1.0 + np.exp(-v))
+    err = np.abs(got - ref)
+    # each element: within bf16 rounding of the exact value plus 2^-10 of |z|/2
+    bound = np.abs(ref) * 2.0 ** -8 + np.abs(v) * 2.0 ** -11 + 1e-30
+    assert np.all(err <= bound), float((err / bound).max())

@@ -31,7 +31,7 @@ __all__ = [
     "conv3d_bwd_data", "conv3d_bwd_data_ptr", "bwd_data_workspace_bytes",
     "conv3d_bwd_weight", "conv3d_bwd_weight_ptr", "bwd_weight_workspace_bytes",
     "Conv3dFunction", "conv3d_autograd",
-    "poll_status", "selftest_wait_timeout", "release",
+    "poll_status", "selftest_wait_timeout", "release", "test_arm_stall",
 ]
 
 F16 = 0
@@ -107,6 +107,8 @@ _lib.conv3d_release.restype = None
 _lib.conv3d_release.argtypes = []
 _lib.conv3d_selftest_wait_timeout.restype = _c
 _lib.conv3d_selftest_wait_timeout.argtypes = [_c]
+_lib.conv3d_test_arm_stall.restype = _c
+_lib.conv3d_test_arm_stall.argtypes = [_c, _c]
 
 
 def raw_library() -> ctypes.CDLL:
@@ -265,6 +267,13 @@ def selftest_wait_timeout(timeout_ms: int) -> int:
 
 def release() -> None:
     _lib.conv3d_release()
+
+
+def test_arm_stall(launches: int, timeout_ms: int = 50) -> None:
+    """Failure-detection test hook: the next ``launches`` convolution-kernel
+    launches stall on their first pipeline stage and abort after ``timeout_ms``
+    (poll_status then returns Status.TIMEOUT).  0 disarms."""
+    _check(_lib.conv3d_test_arm_stall(int(launches), int(timeout_ms)))
 
 
 def groupnorm_stats_ptr(x, N, D, H, W, C, groups, per_frame, eps, dtype, stats, stream) -> int:

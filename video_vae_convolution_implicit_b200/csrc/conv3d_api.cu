@@ -2,7 +2,7 @@
 // argument validation, problem -> GEMM mapping, tensor-map encoding, the
 // first-frame weight fold and the kernel launch.  No call synchronises except
 // conv3d_poll_status and the self test; nothing allocates except the cached
-// first-frame workspace of conv3d_fwd.
+// per-stream workspace of conv3d_fwd (first-frame fold, tail-split partials).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -11,8 +11,11 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstdlib>
+#include <atomic>
 #include <cstring>
 #include <mutex>
+#include <string>
+#include <unordered_map>
 
 #include "conv3d.h"
 #include "conv3d_kernel.cuh"
@@ -47,6 +50,23 @@ bool plan_log() {
     return env != nullptr && env[0] == '1';
   }();
   return on;
+}
+
+// Failure-detection test hook (conv3d_test_arm_stall): the number of
+// convolution-kernel launches still armed and their wait limit.
+std::atomic<int> g_stall_launches{0};
+std::atomic<int> g_stall_timeout_ms{50};
+
+// True, consuming one armed launch, if this launch is to stall; sets its limit.
+bool take_stall(unsigned long long& timeout_ns) {
+  int n = g_stall_launches.load();
+  while (n > 0) {
+    if (g_stall_launches.compare_exchange_weak(n, n - 1)) {
+      timeout_ns = static_cast<unsigned long long>(g_stall_timeout_ms.load()) * 1000000ull;
+      return true;
+    }
+  }
+  return false;
 }
 
 // ------------------------------------------------------------------ problem
@@ -230,6 +250,95 @@ conv3d_status_t load_entry_points() {
   return CONV3D_OK;
 }
 
+// ------------------------------------------------------------------ tensor-map cache
+
+// A tensor map is a pure function of its encode arguments (address, sizes,
+// strides, box, traversal, swizzle), so a call that repeats an earlier call's
+// pointers and shape reuses the maps encoded then instead of asking the driver
+// again (3-5 encodes per launch).  Keyed by the raw argument bytes; at most
+// kMapCacheEntries maps are kept (the cache is emptied when full) and
+// conv3d_release empties it.
+constexpr size_t kMapCacheEntries = 1024;
+std::mutex g_map_mu;
+std::unordered_map<std::string, CUtensorMap> g_map_cache;
+
+// CONV3D_MAP_CACHE=0 encodes every map afresh (for measuring the cache).
+bool map_cache_on() {
+  static const bool on = [] {
+    const char* env = getenv("CONV3D_MAP_CACHE");
+    return env == nullptr || env[0] != '0';
+  }();
+  return on;
+}
+
+template <typename T>
+void key_add(std::string& k, const T* v, size_t n) {
+  k.append(reinterpret_cast<const char*>(v), sizeof(T) * n);
+}
+
+bool map_cache_get(const std::string& key, CUtensorMap& out) {
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  auto it = g_map_cache.find(key);
+  if (it == g_map_cache.end()) return false;
+  out = it->second;
+  return true;
+}
+
+void map_cache_put(const std::string& key, const CUtensorMap& m) {
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  if (g_map_cache.size() >= kMapCacheEntries) g_map_cache.clear();
+  g_map_cache.emplace(key, m);
+}
+
+CUresult encode_tiled_cached(CUtensorMap* map, CUtensorMapDataType dt, cuuint32_t rank, void* base,
+                             const cuuint64_t* dims, const cuuint64_t* strides,
+                             const cuuint32_t* box, const cuuint32_t* estr,
+                             CUtensorMapInterleave il, CUtensorMapSwizzle sw,
+                             CUtensorMapL2promotion l2, CUtensorMapFloatOOBfill oob) {
+  if (!map_cache_on())
+    return g_encode_tiled(map, dt, rank, base, dims, strides, box, estr, il, sw, l2, oob);
+  std::string key(1, 'T');
+  const int e[6] = {static_cast<int>(dt), static_cast<int>(rank), static_cast<int>(il),
+                    static_cast<int>(sw), static_cast<int>(l2), static_cast<int>(oob)};
+  key_add(key, e, 6);
+  key_add(key, &base, 1);
+  key_add(key, dims, rank);
+  key_add(key, strides, rank - 1);
+  key_add(key, box, rank);
+  key_add(key, estr, rank);
+  if (map_cache_get(key, *map)) return CUDA_SUCCESS;
+  CUresult r = g_encode_tiled(map, dt, rank, base, dims, strides, box, estr, il, sw, l2, oob);
+  if (r == CUDA_SUCCESS) map_cache_put(key, *map);
+  return r;
+}
+
+CUresult encode_im2col_cached(CUtensorMap* map, CUtensorMapDataType dt, cuuint32_t rank,
+                              void* base, const cuuint64_t* dims, const cuuint64_t* strides,
+                              const int* lower, const int* upper, cuuint32_t channels,
+                              cuuint32_t pixels, const cuuint32_t* estr, CUtensorMapInterleave il,
+                              CUtensorMapSwizzle sw, CUtensorMapL2promotion l2,
+                              CUtensorMapFloatOOBfill oob) {
+  if (!map_cache_on())
+    return g_encode_im2col(map, dt, rank, base, dims, strides, lower, upper, channels, pixels,
+                           estr, il, sw, l2, oob);
+  std::string key(1, 'I');
+  const int e[8] = {static_cast<int>(dt), static_cast<int>(rank), static_cast<int>(il),
+                    static_cast<int>(sw), static_cast<int>(l2), static_cast<int>(oob),
+                    static_cast<int>(channels), static_cast<int>(pixels)};
+  key_add(key, e, 8);
+  key_add(key, &base, 1);
+  key_add(key, dims, rank);
+  key_add(key, strides, rank - 1);
+  key_add(key, lower, rank - 2);
+  key_add(key, upper, rank - 2);
+  key_add(key, estr, rank);
+  if (map_cache_get(key, *map)) return CUDA_SUCCESS;
+  CUresult r = g_encode_im2col(map, dt, rank, base, dims, strides, lower, upper, channels, pixels,
+                               estr, il, sw, l2, oob);
+  if (r == CUDA_SUCCESS) map_cache_put(key, *map);
+  return r;
+}
+
 // ------------------------------------------------------------------ per-device state
 
 struct DeviceState {
@@ -237,8 +346,16 @@ struct DeviceState {
   int num_sms = 0;
   int max_smem_optin = 0;
   int* status = nullptr;         // address of g_status on this device
-  void* workspace = nullptr;     // cached first-frame fold buffer (conv3d_fwd)
-  size_t workspace_bytes = 0;
+  // conv3d_fwd's cached scratch, one buffer per stream it was called on: the
+  // first-frame folded weight and the tail split's partials and tickets
+  struct Scratch {
+    cudaStream_t stream;
+    void* ptr;
+    size_t bytes;
+    unsigned int gen;            // launch generation of the split tickets
+  };
+  Scratch scratch[16] = {};
+  int n_scratch = 0;
   bool attr_set[8] = {};         // per kernel variant
   int pair_clusters = 0;         // co-resident CTA pairs (occupancy query)
   int wg_pair_clusters = 0;      // the same for the weight-gradient kernel
@@ -340,7 +457,7 @@ conv3d_status_t encode_im2col(const Problem& P, const void* base, long long imag
   // traversal strides: consecutive output pixels' window origins are sw
   // columns (sh rows at a row wrap) apart
   const cuuint32_t estr[4] = {1, static_cast<cuuint32_t>(P.sw), static_cast<cuuint32_t>(P.sh), 1};
-  CUresult r = g_encode_im2col(&map, dt, 4, const_cast<void*>(base), dims, strides, lower, upper,
+  CUresult r = encode_im2col_cached(&map, dt, 4, const_cast<void*>(base), dims, strides, lower, upper,
                                BK, static_cast<cuuint32_t>(pixels_per_load), estr,
                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -372,7 +489,7 @@ conv3d_status_t encode_maps(const Problem& P, const void* x, const void* wmat, i
                                    static_cast<cuuint64_t>(taps) * P.Cin * 2};
     const cuuint32_t box[3] = {BK, 1, static_cast<cuuint32_t>(b_box_rows)};
     const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = g_encode_tiled(&map_b, dt, 3, const_cast<void*>(wmat), dims, strides, box, estr,
+    CUresult r = encode_tiled_cached(&map_b, dt, 3, const_cast<void*>(wmat), dims, strides, box, estr,
                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -400,7 +517,7 @@ conv3d_status_t encode_out_map(const Problem& P, const void* base, CUtensorMap& 
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(P.Cout) * esize, howo * P.Cout * esize};
   const cuuint32_t box[3] = {32, 32, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode_tiled(&map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = encode_tiled_cached(&map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
                               CU_TENSOR_MAP_INTERLEAVE_NONE,
                               f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -426,9 +543,22 @@ struct LaunchPlan {
   bool swap;          // transposed product: M = 128 channels, N = 256 pixels
   KernelParams kp;
   size_t smem;
+  size_t split_bytes; // scratch of the tail split (partials, then tickets); 0 if none
+  size_t split_part_bytes;
 };
 
-conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, LaunchPlan& L) {
+// CONV3D_SPLIT (tuning and tests): 0 turns the tail split off; n in 2..8
+// cuts every tile of the last round (of every round, when there is only one)
+// into n pieces whatever the shape; unset: the rule in plan_launch.
+int split_override() {
+  const char* env = getenv("CONV3D_SPLIT");
+  if (env == nullptr || env[0] == '\0') return -1;
+  const int v = atoi(env);
+  return v == 0 ? 0 : (v >= 2 && v <= 8 ? v : -1);
+}
+
+conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, bool allow_split,
+                            LaunchPlan& L) {
   // The folded weight is a kt = 2 (hi, lo) kernel over the single frame; with
   // causal replicate padding both of its taps read frame 0.
   const int kt_eff = P.fold ? 2 : P.kt;
@@ -497,6 +627,41 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, L
   }
   kp.tiles_per_frame = (kp.HoWo + kp.pix_tile - 1) / kp.pix_tile;
   kp.num_tiles = P.N * P.Do * kp.tiles_per_frame * kp.n_tiles_n;
+  // Tail split.  The persistent grid runs the tiles in rounds of one per SM;
+  // when the last round is at most half full (R tiles), the other SMs would
+  // idle through it.  Each of those R tiles is then cut into S pieces along K
+  // (S <= SMs / R, at most 8, at least 8 k-blocks a piece), the pieces run
+  // side by side on S*R SMs, and the piece that completes a tile adds up the
+  // S fp32 partials (in piece order) before the usual epilogue: the last
+  // round takes about 1/S of a tile's time.  Only with a library-owned
+  // workspace (conv3d_fwd), never for CTA pairs or fp32 outputs.
+  kp.num_items = kp.num_tiles;
+  kp.split_first = kp.num_tiles;
+  kp.split_s = 1;
+  L.split_bytes = 0;
+  L.split_part_bytes = 0;
+  const int forced = split_override();
+  if (allow_split && forced != 0 && !L.pair && !P.out_f32) {
+    const int U = S.num_sms;
+    const int T = kp.num_tiles;
+    int R = T % U;
+    const int kb_nominal = kt_eff * P.kh * P.kw * kp.n_chunks;
+    if (forced > 0 && R == 0) R = T < U ? T : U;
+    if (forced > 0 || (T >= U && R > 0 && 2 * R <= U)) {
+      int sp = forced > 0 ? forced : U / R;
+      if (forced < 0) {
+        if (sp > 8) sp = 8;
+        while (sp > 1 && kb_nominal / sp < 8) --sp;
+      }
+      if (sp >= 2) {
+        kp.split_first = T - R;
+        kp.split_s = sp;
+        kp.num_items = T - R + R * sp;
+        L.split_part_bytes = static_cast<size_t>(R) * sp * BM * kp.BN * sizeof(float);
+        L.split_bytes = L.split_part_bytes + static_cast<size_t>(R) * 4 * sizeof(unsigned long long);
+      }
+    }
+  }
   const int b_stage = kp.BN / ctas * BK * 2;
   const int stage_bytes = A_STAGE_BYTES + b_stage;
   kp.has_residual = P.has_residual ? 1 : 0;
@@ -556,7 +721,7 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
       units = S.pair_clusters;
     }
   }
-  const int unit_count = L.kp.num_tiles < units ? L.kp.num_tiles : units;
+  const int unit_count = L.kp.num_items < units ? L.kp.num_items : units;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -572,25 +737,28 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
   if (plan_log())
     fprintf(stderr,
             "libconv3d: implicit GEMM %s %s, %d tiles of %d pixels x %d channels, grid %d, "
-            "%d k-blocks x %d taps, %d stages, %zu B shared, %s output\n",
+            "%d k-blocks x %d taps, %d stages, %zu B shared, %s output, last %d tiles in %d "
+            "pieces\n",
             kSwap ? "transposed" : kPair ? "CTA pair" : "single", kBF16 ? "bf16" : "fp16",
             L.kp.num_tiles, L.kp.pix_tile, L.kp.co_tile, static_cast<int>(cfg.gridDim.x),
             L.kp.n_chunks, L.kp.kt * L.kp.kh * L.kp.kw, L.kp.stages, L.smem,
-            L.kp.out_f32 ? "fp32" : "16-bit");
-  e = cudaLaunchKernelEx(&cfg, kern, map_a, map_b, map_y, map_r, map_p, L.kp);
+            L.kp.out_f32 ? "fp32" : "16-bit", L.kp.num_tiles - L.kp.split_first, L.kp.split_s);
+  KernelParams kp = L.kp;
+  kp.test_stall = take_stall(kp.timeout_ns) ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, kern, map_a, map_b, map_y, map_r, map_p, kp);
   if (e != cudaSuccess) return cuda_fail(e, "conv3d kernel launch");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "conv3d kernel launch");
   return CONV3D_OK;
 }
 
-conv3d_status_t launch_main(DeviceState& S, const Problem& P, const void* x, const void* prev,
-                            const void* wmat, const void* bias, const void* residual, void* y,
-                            cudaStream_t stream) {
+// Launches the main kernel with a plan from plan_launch (whose split scratch,
+// if any, the caller has filled in).
+conv3d_status_t launch_planned(DeviceState& S, const Problem& P, LaunchPlan& L, const void* x,
+                               const void* prev, const void* wmat, const void* bias,
+                               const void* residual, void* y, cudaStream_t stream) {
   const bool bf16 = P.dtype == CONV3D_BF16;
-  LaunchPlan L;
-  conv3d_status_t st = plan_launch(S, P, bf16, L);
-  if (st != CONV3D_OK) return st;
+  conv3d_status_t st = CONV3D_OK;
   L.kp.bias = bias;
   L.kp.status = S.status;
   CUtensorMap map_a, map_b, map_y, map_r, map_p;
@@ -621,6 +789,50 @@ conv3d_status_t launch_main(DeviceState& S, const Problem& P, const void* x, con
                 : launch_kernel<false, false, false>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
 }
 
+// The main kernel without a tail split (no scratch needed).
+conv3d_status_t launch_main(DeviceState& S, const Problem& P, const void* x, const void* prev,
+                            const void* wmat, const void* bias, const void* residual, void* y,
+                            cudaStream_t stream) {
+  LaunchPlan L;
+  conv3d_status_t st = plan_launch(S, P, P.dtype == CONV3D_BF16, false, L);
+  if (st != CONV3D_OK) return st;
+  return launch_planned(S, P, L, x, prev, wmat, bias, residual, y, stream);
+}
+
+// conv3d_fwd's scratch for `stream` on this device, at least `need` bytes,
+// zeroed when (re)allocated; also returns the next launch generation.
+conv3d_status_t cached_scratch(DeviceState& S, cudaStream_t stream, size_t need, void*& ptr,
+                               unsigned int& gen) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState::Scratch* sc = nullptr;
+  for (int i = 0; i < S.n_scratch; ++i)
+    if (S.scratch[i].stream == stream) sc = &S.scratch[i];
+  if (sc == nullptr) {
+    if (S.n_scratch == 16) {
+      set_error("conv3d_fwd was called on more than 16 streams; use conv3d_fwd_ws");
+      return CONV3D_ERR_UNSUPPORTED;
+    }
+    sc = &S.scratch[S.n_scratch++];
+    *sc = DeviceState::Scratch{stream, nullptr, 0, 0};
+  }
+  if (sc->bytes < need) {
+    if (sc->ptr) {
+      cudaError_t e = cudaFree(sc->ptr);
+      sc->ptr = nullptr;
+      sc->bytes = 0;
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFree(workspace)");
+    }
+    cudaError_t e = cudaMalloc(&sc->ptr, need);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(workspace)");
+    if ((e = cudaMemset(sc->ptr, 0, need)) != cudaSuccess) return cuda_fail(e, "workspace clear");
+    sc->bytes = need;
+  }
+  if (++sc->gen == 0) ++sc->gen;
+  ptr = sc->ptr;
+  gen = sc->gen;
+  return CONV3D_OK;
+}
+
 conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* bias,
                     const void* residual, void* y, void* ws, size_t ws_bytes, bool cached_ws,
                     cudaStream_t stream) {
@@ -631,24 +843,25 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
   if ((st = device_state(S, dev)) != CONV3D_OK) return st;
   const bool bf16 = P.dtype == CONV3D_BF16;
   const void* wmat = w;
+  LaunchPlan L;
+  if ((st = plan_launch(*S, P, bf16, cached_ws, L)) != CONV3D_OK) return st;
+  const int kfold[3] = {P.kt, P.kh, P.kw};
+  const size_t fold_need = P.fold ? fold_bytes(P.Cin, P.Cout, kfold) : 0;   // 256-byte multiple
+  if (cached_ws && fold_need + L.split_bytes > 0) {
+    unsigned int gen = 0;
+    if ((st = cached_scratch(*S, stream, fold_need + L.split_bytes, ws, gen)) != CONV3D_OK)
+      return st;
+    ws_bytes = fold_need + L.split_bytes;
+    if (L.split_bytes > 0) {
+      char* base = static_cast<char*>(ws) + fold_need;
+      L.kp.part = reinterpret_cast<float*>(base);
+      L.kp.ticket = reinterpret_cast<unsigned long long*>(base + L.split_part_bytes);
+      L.kp.gen = gen;
+    }
+  }
   if (P.fold) {
-    const int k[3] = {P.kt, P.kh, P.kw};
-    const size_t need = fold_bytes(P.Cin, P.Cout, k);
-    if (cached_ws) {
-      std::lock_guard<std::mutex> lock(g_mu);
-      if (S->workspace_bytes < need) {
-        if (S->workspace) {
-          cudaError_t e = cudaFree(S->workspace);
-          S->workspace = nullptr;
-          S->workspace_bytes = 0;
-          if (e != cudaSuccess) return cuda_fail(e, "cudaFree(workspace)");
-        }
-        cudaError_t e = cudaMalloc(&S->workspace, need);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(workspace)");
-        S->workspace_bytes = need;
-      }
-      ws = S->workspace;
-    } else {
+    const size_t need = fold_need;
+    if (!cached_ws) {
       if (ws == nullptr || ws_bytes < need) {
         set_error("workspace of %zu bytes required", need);
         return CONV3D_ERR_WORKSPACE;
@@ -673,7 +886,7 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
     wmat = ws;
   }
   (void)dev;
-  return launch_main(*S, P, x, P.prev, wmat, bias, residual, y, stream);
+  return launch_planned(*S, P, L, x, P.prev, wmat, bias, residual, y, stream);
 }
 
 // ------------------------------------------------------------------ allocation-free entry
@@ -1243,6 +1456,7 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   wp.dw = dw32;
   wp.status = S->status;
   wp.timeout_ns = kDefaultTimeoutNs;
+  wp.test_stall = take_stall(wp.timeout_ns) ? 1 : 0;
   const size_t smem = static_cast<size_t>(stages) * stage_bytes + reserve;
 
   // x through the forward im2col map (pix pixels per load); dy as [frames][pixels][Cout]
@@ -1258,7 +1472,7 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(Cout) * 2, howo * Cout * 2};
     const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(pix), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = g_encode_tiled(&map_dy, dt, 3, const_cast<void*>(dy), dims, strides, box, estr,
+    CUresult r = encode_tiled_cached(&map_dy, dt, 3, const_cast<void*>(dy), dims, strides, box, estr,
                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -1402,18 +1616,20 @@ const char* conv3d_status_string(conv3d_status_t s) {
 const char* conv3d_last_error(void) { return g_last_error; }
 
 void conv3d_release(void) {
+  {
+    std::lock_guard<std::mutex> map_lock(g_map_mu);
+    g_map_cache.clear();
+  }
   std::lock_guard<std::mutex> aux_lock(g_aux_mu);
   std::lock_guard<std::mutex> lock(g_mu);
   int cur = -1;
   if (cudaGetDevice(&cur) != cudaSuccess) return;
   for (int d = 0; d < kMaxDevices; ++d) {
     DeviceState& s = g_dev[d];
-    if (s.workspace || s.aux) cudaSetDevice(d);
-    if (s.workspace) {
-      cudaFree(s.workspace);
-      s.workspace = nullptr;
-      s.workspace_bytes = 0;
-    }
+    if (s.n_scratch > 0 || s.aux) cudaSetDevice(d);
+    for (int i = 0; i < s.n_scratch; ++i)
+      if (s.scratch[i].ptr) cudaFree(s.scratch[i].ptr);
+    s.n_scratch = 0;
     if (s.aux) {
       // work still queued on the stream completes before its resources go
       cudaEventDestroy(s.aux_join);
@@ -1424,6 +1640,16 @@ void conv3d_release(void) {
     }
   }
   cudaSetDevice(cur);
+}
+
+conv3d_status_t conv3d_test_arm_stall(int launches, int timeout_ms) {
+  if (launches < 0 || timeout_ms < 1 || timeout_ms > 10000) {
+    set_error("launches must be >= 0 and timeout_ms in [1, 10000]");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  g_stall_timeout_ms.store(timeout_ms);
+  g_stall_launches.store(launches);
+  return CONV3D_OK;
 }
 
 conv3d_status_t conv3d_selftest_wait_timeout(int timeout_ms) {

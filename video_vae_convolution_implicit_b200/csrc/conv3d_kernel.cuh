@@ -62,6 +62,17 @@ struct KernelParams {
   int n_tiles_n;                     // ceil(Cout / co_tile)
   int tiles_per_frame;               // ceil(HoWo / pix_tile)
   int num_tiles;
+  // Tail split: tiles [split_first, num_tiles) are each cut into split_s
+  // pieces along K, so that the last, partly filled round of tiles spreads
+  // over the otherwise idle SMs.  Work items: tiles 0 .. split_first-1 whole,
+  // then split_s consecutive pieces per tail tile (num_items in all).
+  int num_items;
+  int split_first;
+  int split_s;                       // 1: no tail split
+  float* part;                       // [tail tiles][split_s][128 lanes][BN] fp32 partials
+  unsigned long long* ticket;        // [tail tiles][4 lane quarters]: (generation << 32) |
+                                     // pieces whose partial is stored
+  unsigned int gen;                  // this launch's generation (nonzero)
   int stages;
   uint32_t tmem_cols;                // power of two >= 2*BN
   uint32_t idesc;
@@ -70,6 +81,8 @@ struct KernelParams {
   int out_f32;                       // y is fp32 (single-CTA, non-transposed variant only)
   int* status;                       // device status word
   unsigned long long timeout_ns;
+  int test_stall;                    // failure-detection test: the producer skips the
+                                     // copies of its first stage (armed from the host)
 };
 
 // Epilogue staging: each epilogue warp owns two 32-row x 32-channel buffers
@@ -109,6 +122,38 @@ __device__ __forceinline__ Tile decode_tile(const KernelParams& p, int t) {
   return r;
 }
 
+// One work item: a whole tile, or one K-range piece of a tail tile.
+struct Work {
+  Tile tl;
+  int kb_lo, kb_hi;  // the item's k-blocks, in the tile's k-block order
+  int slot;          // partial slot (tail tile * split_s + piece), or -1 for a whole tile
+};
+
+__device__ __forceinline__ int kblocks_of_tile(const KernelParams& p, int to);
+
+__device__ __forceinline__ Work decode_work(const KernelParams& p, int i) {
+  Work w;
+  int t = i, piece = -1;
+  if (i >= p.split_first) {
+    const int j = i - p.split_first;
+    const int q = j / p.split_s;
+    t = p.split_first + q;
+    piece = j - q * p.split_s;
+  }
+  w.tl = decode_tile(p, t);
+  const int nkb = kblocks_of_tile(p, w.tl.to);
+  if (piece < 0) {
+    w.kb_lo = 0;
+    w.kb_hi = nkb;
+    w.slot = -1;
+  } else {
+    w.kb_lo = piece * nkb / p.split_s;
+    w.kb_hi = (piece + 1) * nkb / p.split_s;
+    w.slot = (t - p.split_first) * p.split_s + piece;
+  }
+  return w;
+}
+
 constexpr int kNoFrame = -0x40000000;
 
 // Source frame read by temporal tap `it` of output frame `to`: a frame of x
@@ -134,10 +179,13 @@ struct SharedCtl {
   volatile int* abort_flag;
   int* status;
   unsigned long long timeout_ns;
+  uint32_t peer_abort;   // shared::cluster address of the peer CTA's abort flag (pairs), or 0
 };
 
+// Every role of this CTA (and of its peer, for a pair) leaves its loop.
 __device__ __forceinline__ void raise_abort(const SharedCtl& c, int code) {
   *c.abort_flag = 1;
+  if (c.peer_abort != 0) st_cluster_u32(c.peer_abort, 1);
   atomicCAS(c.status, 0, code);
 }
 
@@ -156,6 +204,138 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const S
         raise_abort(c, STATUS_TIMEOUT);
         return false;
       }
+    }
+  }
+}
+
+// The same for a barrier that the peer CTA of a pair arrives on with release
+// semantics at cluster scope (what it stored before arriving is then visible).
+__device__ __noinline__ bool wait_bounded_cluster(uint32_t bar, uint32_t parity,
+                                                  const SharedCtl& c) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((i & 15) == 15 && globaltimer_ns() - t0 > c.timeout_ns) {
+      raise_abort(c, STATUS_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// End of a producer's loop.  After an abort no copy may still be writing into
+// shared memory when the CTA exits, so the producer waits until every stage
+// instance it (and, for a CTA pair, its peer) announced has landed:
+//   issued      stage instances this producer counted; with `skip_first`
+//               (the failure-detection test) instance 0 was counted but
+//               neither announced nor copied;
+//   half_bytes  one CTA's share of a stage's bytes (pairs).
+// The copies of both CTAs of a pair complete on the even CTA's barriers, so
+// the odd CTA publishes its own count in the even CTA (`peer_count`, a
+// release-arrive on `peer_bar`) at the end of every run, and the even CTA
+// settles each instance that only one of the two issued before waiting on it:
+// an instance it announced whose odd half will never come has that half
+// cancelled (complete_tx); one whose odd half is in flight but which it never
+// announced is announced now for that half alone.  Both producers are paced
+// by the same empty barriers and the MMAs need both halves, so the counts
+// differ by at most `stages` and every instance before max - stages has been
+// consumed.
+template <bool kPair>
+__device__ void producer_finish(bool aborted, long long issued, bool skip_first, int stages,
+                                uint32_t full_bar, uint32_t half_bytes, uint32_t peer_count,
+                                uint32_t peer_bar, const SharedCtl& c, bool leader) {
+  if constexpr (kPair) {
+    if (!leader) {
+      st_cluster_u64(mapa_shared(peer_count, 0), static_cast<unsigned long long>(issued));
+      mbar_arrive_cluster(mapa_shared(peer_bar, 0));
+      return;
+    }
+  }
+  if (!aborted) return;
+  long long peer = issued;
+  if constexpr (kPair) {
+    if (!wait_bounded_cluster(peer_bar, 0, c)) return;   // the peer never reported
+    unsigned long long v;
+    asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(peer_count) : "memory");
+    peer = static_cast<long long>(v);
+  }
+  const long long top = issued > peer ? issued : peer;
+  const long long first = top > stages ? top - stages : 0;
+  for (long long i = first; i < top; ++i) {
+    if (skip_first && i == 0) continue;
+    const uint32_t fb = full_bar + 8 * static_cast<uint32_t>(i % stages);
+    if constexpr (kPair) {
+      if (i < issued && i >= peer) mbar_complete_tx(fb, half_bytes);
+      else if (i >= issued && i < peer) mbar_arrive_expect_tx(fb, half_bytes);
+    }
+    wait_bounded(fb, static_cast<uint32_t>((i / stages) & 1), c, false);
+  }
+}
+
+// Ticket of one lane quarter of a split tail tile: counts, for this launch's
+// generation, the pieces whose partial is stored (an older generation counts
+// as none, so the tickets never need clearing).  True for the piece that
+// completes the quarter.  Each retry means another piece got in first, so at
+// most split_s attempts.
+__device__ __forceinline__ bool take_ticket(unsigned long long* t, unsigned int gen, int pieces) {
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(t);
+  for (;;) {
+    const unsigned long long done = (cur >> 32) == gen ? (cur & 0xFFFFFFFFull) : 0ull;
+    const unsigned long long next = (static_cast<unsigned long long>(gen) << 32) | (done + 1);
+    const unsigned long long seen = atomicCAS(t, cur, next);
+    if (seen == cur) return done + 1 == static_cast<unsigned long long>(pieces);
+    cur = seen;
+  }
+}
+
+// Tail piece, for the calling warp's 32 TMEM lanes (lane row = quarter*32 +
+// lane): store the raw fp32 accumulator (BN columns per lane) in the piece's
+// slot, then take the quarter's ticket.  Returns true in every lane of the
+// warp whose piece completed the quarter; every piece's partial of these
+// lanes is then visible to the warp.  Warp-level only (no other warp is
+// waited for), so an abort in another warp cannot hold this one.
+__device__ __forceinline__ bool store_piece(const KernelParams& p, int slot, uint32_t t_row,
+                                            bool has_acc, uint32_t quarter, uint32_t lane) {
+  float4* dst = reinterpret_cast<float4*>(
+      p.part + (static_cast<size_t>(slot) * BM + quarter * 32u + lane) * p.BN);
+  for (int j = 0; j < p.BN / 32; ++j) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(t_row + j * 32, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      dst[j * 8 + q] = has_acc ? make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                             __uint_as_float(r[4 * q + 2]),
+                                             __uint_as_float(r[4 * q + 3]))
+                               : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  }
+  __threadfence();
+  __syncwarp();
+  int last = 0;
+  if (lane == 0)
+    last = take_ticket(p.ticket + (slot / p.split_s) * 4 + quarter, p.gen, p.split_s) ? 1 : 0;
+  last = __shfl_sync(0xFFFFFFFFu, last, 0);
+  if (last) __threadfence();
+  return last != 0;
+}
+
+// Columns [32j, 32j+32) of the calling lane's row of a completed tail tile:
+// the sum of every piece's partial, in piece order (the result does not
+// depend on which piece finished last).  L2 loads: the partials were written
+// by other SMs.
+__device__ __forceinline__ void sum_pieces(const KernelParams& p, int slot0, uint32_t lane_row,
+                                           int j, float (&v)[32]) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+  for (int sp = 0; sp < p.split_s; ++sp) {
+    const float4* src = reinterpret_cast<const float4*>(
+        p.part + (static_cast<size_t>(slot0 + sp) * BM + lane_row) * p.BN + j * 32);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 a = __ldcg(src + q);
+      v[4 * q] += a.x;
+      v[4 * q + 1] += a.y;
+      v[4 * q + 2] += a.z;
+      v[4 * q + 3] += a.w;
     }
   }
 }
@@ -211,6 +391,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
   __shared__ int s_abort;
+  __shared__ __align__(8) uint64_t s_peer_bar;      // pairs: the odd CTA's end-of-run report
+  __shared__ unsigned long long s_peer_count;
 
   constexpr int kCtas = kPair ? 2 : 1;
   const uint32_t warp = threadIdx.x / 32;
@@ -239,7 +421,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t drain_bar = tempty_bar + 16;             // [1]
   const uint32_t rfull_bar = drain_bar + 8;               // [EPI_WARPS][2]
 
-  SharedCtl ctl{&s_abort, p.status, p.timeout_ns};
+  SharedCtl ctl{&s_abort, p.status, p.timeout_ns,
+                kPair ? mapa_shared(smem_addr(&s_abort), rank ^ 1u) : 0u};
+  const uint32_t peer_bar = smem_addr(&s_peer_bar);
+  const uint32_t peer_count = smem_addr(&s_peer_count);
 
   if (threadIdx.x == 0) {
     s_abort = 0;
@@ -252,6 +437,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(tempty_bar + 8 * a, 4 * kCtas);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(peer_bar, 1);
     for (int e = 0; e < 2 * EPI_WARPS; ++e) mbar_init(rfull_bar + 8 * e, 1);
     fence_mbar_init();
     prefetch_tensormap(&map_a);
@@ -279,11 +465,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint32_t tx_bytes = kCtas * (A_STAGE_BYTES + b_stage_bytes);
+      const bool stall = p.test_stall != 0;
       uint32_t stage = 0, phase = 0;
       long long issued = 0;
       bool ok = true;
-      for (int t = unit; ok && t < p.num_tiles; t += num_units) {
-        const Tile tl = decode_tile(p, t);
+      for (int i = unit; ok && i < p.num_items; i += num_units) {
+        const Work wk = decode_work(p, i);
+        const Tile& tl = wk.tl;
+        int kb = 0;          // k-block index within the tile; the item issues [kb_lo, kb_hi)
         // first output pixel of this CTA's rows; rows past the frame are
         // computed from any valid window origin and masked by the epilogue
         int row0 = tl.p0 + static_cast<int>(rank) * BM;
@@ -293,29 +482,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int w_org = wo0 * p.sw - p.pw;   // window origin of the first pixel
         const int h_org = ho0 * p.sh - p.ph;
         const int co_b = tl.co0 + static_cast<int>(rank * b_rows);
-        for (int it = 0; ok && it < p.kt; ++it) {
+        for (int it = 0; ok && kb < wk.kb_hi && it < p.kt; ++it) {
           const int f = source_frame(p, tl.to, it);
           if (f == kNoFrame) continue;
           // frames before the chunk come from the cached-frames tensor
           const CUtensorMap* xmap = f < 0 ? &map_p : &map_a;
           const int img = f < 0 ? tl.n * (p.kt - 1) + (p.kt - 1) + f : tl.n * p.D + f;
-          for (int ih = 0; ok && ih < p.kh; ++ih) {
-            for (int iw = 0; ok && iw < p.kw; ++iw) {
+          for (int ih = 0; ok && kb < wk.kb_hi && ih < p.kh; ++ih) {
+            for (int iw = 0; ok && kb < wk.kb_hi && iw < p.kw; ++iw) {
               const int tap = (it * p.kh + ih) * p.kw + iw;
-              for (int cc = 0; cc < p.n_chunks; ++cc) {
+              for (int cc = 0; cc < p.n_chunks && kb < wk.kb_hi; ++cc) {
+                if (kb++ < wk.kb_lo) continue;   // an earlier piece's k-block
                 if (!wait_bounded(empty_bar + 8 * stage, phase ^ 1, ctl, true)) {
                   ok = false;
                   break;
                 }
                 const uint32_t fb = full_bar + 8 * stage;
-                if (leader) mbar_arrive_expect_tx(fb, tx_bytes);
-                if constexpr (kSwap) {
+                if (stall && issued == 0) {
+                  // failure-detection test: this stage never fills, so the
+                  // tensor-core issuer's wait on it must run out
+                } else if constexpr (kSwap) {
                   // A operand = 128 output channels of w, B operand = 256 pixels
+                  mbar_arrive_expect_tx(fb, tx_bytes);
                   tma_load_3d(a_ring + stage * A_STAGE_BYTES, &map_b, fb, cc * BK, tap, tl.co0);
                   tma_load_im2col_4d(b_ring + stage * b_stage_bytes, xmap, fb, cc * BK, w_org,
                                      h_org, img, static_cast<uint16_t>(iw),
                                      static_cast<uint16_t>(ih));
                 } else if constexpr (kPair) {
+                  if (leader) mbar_arrive_expect_tx(fb, tx_bytes);
                   const uint32_t fb_leader = mapa_shared(fb, 0);
                   tma_load_im2col_4d_pair(a_ring + stage * A_STAGE_BYTES, xmap, fb_leader,
                                           cc * BK, w_org, h_org, img, static_cast<uint16_t>(iw),
@@ -323,6 +517,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   tma_load_3d_pair(b_ring + stage * b_stage_bytes, &map_b, fb_leader, cc * BK,
                                    tap, co_b);
                 } else {
+                  mbar_arrive_expect_tx(fb, tx_bytes);
                   tma_load_im2col_4d(a_ring + stage * A_STAGE_BYTES, xmap, fb, cc * BK, w_org,
                                      h_org, img, static_cast<uint16_t>(iw),
                                      static_cast<uint16_t>(ih));
@@ -338,23 +533,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      if (!ok) {
-        // Let the copies already in flight land before the CTA may exit.
-        if (leader) {
-          const long long first = issued > p.stages ? issued - p.stages : 0;
-          for (long long i = first; i < issued; ++i) {
-            const uint32_t s = static_cast<uint32_t>(i % p.stages);
-            const uint32_t par = static_cast<uint32_t>((i / p.stages) & 1);
-            wait_bounded(full_bar + 8 * s, par, ctl, false);
-          }
-        } else {
-          // the odd CTA's copies complete on the even CTA's barriers: give them
-          // time to land (both CTAs stay resident until the final cluster barrier)
-          const uint64_t t0 = globaltimer_ns();
-          while (globaltimer_ns() - t0 < 200000ull) {
-          }
-        }
-      }
+      producer_finish<kPair>(!ok, issued, stall, p.stages, full_bar, A_STAGE_BYTES + b_stage_bytes,
+                             peer_count, peer_bar, ctl, leader);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -362,9 +542,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t stage = 0, phase = 0;
       bool ok = true;
       int local = 0;
-      for (int t = unit; ok && t < p.num_tiles; t += num_units, ++local) {
-        const Tile tl = decode_tile(p, t);
-        const int nkb = kblocks_of_tile(p, tl.to);
+      for (int i = unit; ok && i < p.num_items; i += num_units, ++local) {
+        const Work wk = decode_work(p, i);
+        const int nkb = wk.kb_hi - wk.kb_lo;
         const uint32_t acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         if (!wait_bounded(tempty_bar + 8 * acc, acc_phase ^ 1, ctl, true)) break;
@@ -435,10 +615,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     if constexpr (kSwap) {
       // Thread = one output channel (TMEM lane), 32 pixels (columns) per chunk.
-      for (int t = unit; ok && t < p.num_tiles; t += num_units, ++local) {
+      for (int i = unit; ok && i < p.num_items; i += num_units, ++local) {
         const uint32_t acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
-        const Tile tl = decode_tile(p, t);
+        const Work wk = decode_work(p, i);
+        const Tile& tl = wk.tl;
+        const bool piece = wk.slot >= 0;
         const int ch0 = tl.co0 + static_cast<int>(quarter) * 32;   // this warp's channels
         const bool warp_live = ch0 < p.Cout;
         int live_chunks = (p.HoWo - tl.p0 + 31) / 32;   // pixel chunks inside the frame
@@ -449,7 +631,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (p.bias != nullptr && ch < p.Cout)
           bv = C::lo(static_cast<const uint16_t*>(p.bias)[ch]);
         const bool use_res = p.has_residual != 0;
-        if (use_res) {
+        // the first two residual chunks, fetched ahead of the accumulator (for a
+        // tail piece only once it is known to complete the tile)
+        auto prefetch_residual = [&]() {
           for (int j = 0; j < 2 && j < live_chunks; ++j) {
             if (lane == 0) {
               mbar_arrive_expect_tx(rbar + 8 * j, EPI_BUF_BYTES);
@@ -458,24 +642,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             rpending[j] = true;
           }
-        }
+        };
+        if (use_res && !piece) prefetch_residual();
+        bool write_out = true;
         if (!wait_bounded(tfull_bar + 8 * acc, acc_phase, ctl, true)) {
           ok = false;
         } else {
           tc_fence_after();
-          const bool has_acc = kblocks_of_tile(p, tl.to) > 0;
+          const bool has_acc = wk.kb_hi > wk.kb_lo;
           const uint32_t t_row =
               tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.BN);
+          bool from_parts = false;
+          if (piece) {
+            write_out = store_piece(p, wk.slot, t_row, has_acc, quarter, lane);
+            from_parts = write_out;
+            if (write_out && use_res) prefetch_residual();
+          }
           // byte offset of (pixel e, this thread's channel) in a 32 x 32 buffer
           const uint32_t col_byte = (lane & 7u) * 2u;
-          for (int j = 0; j < live_chunks; ++j) {
+          for (int j = 0; write_out && j < live_chunks; ++j) {
             const uint32_t b = j & 1;
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(t_row + j * 32, r);
-            tmem_ld_wait();
             float v[32];
+            if (from_parts) {
+              sum_pieces(p, wk.slot - wk.slot % p.split_s, quarter * 32u + lane, j, v);
+            } else {
+              uint32_t r[32];
+              tmem_ld_32x32b_x32(t_row + j * 32, r);
+              tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = (has_acc ? __uint_as_float(r[e]) : 0.0f) + bv;
+              for (int e = 0; e < 32; ++e) v[e] = has_acc ? __uint_as_float(r[e]) : 0.0f;
+            }
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] += bv;
             if (use_res) {
               if (!wait_bounded(rbar + 8 * b, rphase[b], ctl, true)) {
                 ok = false;
@@ -541,17 +739,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) mbar_arrive(tempty_bar + 8 * acc);
       }
     } else
-    for (int t = unit; ok && t < p.num_tiles; t += num_units, ++local) {
+    for (int i = unit; ok && i < p.num_items; i += num_units, ++local) {
       const uint32_t acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
-      const Tile tl = decode_tile(p, t);
+      const Work wk = decode_work(p, i);
+      const Tile& tl = wk.tl;
+      const bool piece = wk.slot >= 0;
       const int row_base = tl.p0 + static_cast<int>(rank) * BM + static_cast<int>(quarter) * 32;
       const bool rows_live = row_base < p.HoWo;   // some of this warp's rows are in the frame
       // channel chunks that hold at least one real output channel
       int live_chunks = (p.Cout - tl.co0 + 31) / 32;
       if (live_chunks > chunks) live_chunks = chunks;
       const bool use_res = p.has_residual && rows_live;
-      if (use_res) {
+      // the first two residual chunks, fetched ahead of the accumulator (for a
+      // tail piece only once it is known to complete the tile)
+      auto prefetch_residual = [&]() {
         for (int j = 0; j < 2 && j < live_chunks; ++j) {
           if (lane == 0) {
             mbar_arrive_expect_tx(rbar + 8 * j, EPI_BUF_BYTES);
@@ -560,22 +762,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           rpending[j] = true;
         }
-      }
+      };
+      if (use_res && !piece) prefetch_residual();
+      bool write_out = true;
       if (!wait_bounded(tfull_bar + 8 * acc, acc_phase, ctl, true)) {
         ok = false;
       } else {
         tc_fence_after();
-        const bool has_acc = kblocks_of_tile(p, tl.to) > 0;
+        const bool has_acc = wk.kb_hi > wk.kb_lo;
         const uint32_t t_row =
             tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.BN);
-        for (int j = 0; rows_live && j < live_chunks; ++j) {
+        bool from_parts = false;
+        if (piece) {
+          write_out = store_piece(p, wk.slot, t_row, has_acc, quarter, lane);
+          from_parts = write_out;
+          if (write_out && use_res) prefetch_residual();
+        }
+        for (int j = 0; write_out && rows_live && j < live_chunks; ++j) {
           const uint32_t b = j & 1;
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(t_row + j * 32, r);
-          tmem_ld_wait();
           float v[32];
+          if (from_parts) {
+            sum_pieces(p, wk.slot - wk.slot % p.split_s, quarter * 32u + lane, j, v);
+          } else {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + j * 32, r);
+            tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = has_acc ? __uint_as_float(r[e]) : 0.0f;
+            for (int e = 0; e < 32; ++e) v[e] = has_acc ? __uint_as_float(r[e]) : 0.0f;
+          }
           const int cb = tl.co0 + j * 32;
           if (bias4 != nullptr) {
 #pragma unroll

@@ -41,6 +41,21 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// SiLU with one special-function operation: silu(z) = z * sigmoid(z) and
+// sigmoid(z) = (1 + tanh(z/2)) / 2, so silu(z) = h + h * tanh(h) with h = z/2,
+// using the hardware tanh approximation (relative error about 2^-11, below the
+// 2^-9 of the bf16 rounding that follows).
+__device__ __forceinline__ float silu_tanh(float z) {
+  const float h = 0.5f * z;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+  return fmaf(h, t, h);
+}
+
+// The same as z / (1 + e^-z): two special-function operations (exp and the
+// reciprocal of the division).  Kept for comparison (CONV3D_GN_SILU=exp).
+__device__ __forceinline__ float silu_exp(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
 __device__ __forceinline__ void unpack8(const uint4 q, uint32_t (&e)[8]) {
   e[0] = q.x & 0xFFFFu; e[1] = q.x >> 16; e[2] = q.y & 0xFFFFu; e[3] = q.y >> 16;
   e[4] = q.z & 0xFFFFu; e[5] = q.z >> 16; e[6] = q.w & 0xFFFFu; e[7] = q.w >> 16;
@@ -212,7 +227,8 @@ __global__ void __launch_bounds__(256, 3) gn_apply_kernel(const uint16_t* x,
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         z[j] = fmaf(to_f<kBF16>(e[j]), scale[j], shift[j]);
-        if (apply_silu) z[j] = __fdividef(z[j], 1.0f + __expf(-z[j]));
+        if (apply_silu == 1) z[j] = silu_tanh(z[j]);
+        else if (apply_silu == 2) z[j] = silu_exp(z[j]);
       }
       // one two-lane conversion per pair (same round-to-nearest-even as one
       // conversion per value, fewer instructions: measured 929 -> 836 us on a
@@ -323,6 +339,12 @@ conv3d_status_t conv3d_groupnorm_silu(const void* x, const double* stats, const 
   const long long vecs = pixels * vpp;
   long long blocks = (vecs + 4LL * threads - 1) / (4LL * threads);
   if (blocks > static_cast<long long>(sms) * 3) blocks = static_cast<long long>(sms) * 3;
+  // SiLU form: 1 = tanh (one special-function op, the default), 2 = exp and
+  // division (CONV3D_GN_SILU=exp, for comparison)
+  if (apply_silu) {
+    const char* env = getenv("CONV3D_GN_SILU");
+    apply_silu = (env != nullptr && env[0] == 'e') ? 2 : 1;
+  }
   if (dtype == CONV3D_BF16)
     gn_apply_kernel<true><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
         static_cast<const uint16_t*>(x), stats, static_cast<const uint16_t*>(gamma),

@@ -70,6 +70,7 @@ struct WgradParams {
   float* dw;                // [Cout][taps][Cin] fp32, accumulated
   int* status;
   unsigned long long timeout_ns;
+  int test_stall;           // failure-detection test: the producer skips its first stage's copies
 };
 
 constexpr int WG_PIX = 128;                         // pixels (K) per stage, by default
@@ -201,6 +202,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
   __shared__ int s_abort;
+  __shared__ __align__(8) uint64_t s_peer_bar;      // pairs: the odd CTA's end-of-run report
+  __shared__ unsigned long long s_peer_count;
   constexpr int kCtas = kPair ? 2 : 1;
   const uint32_t warp = threadIdx.x / 32;
   const uint32_t lane = threadIdx.x % 32;
@@ -222,10 +225,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tfull_bar = bars + 16 * p.stages;
   const uint32_t tempty_bar = tfull_bar + 16;
   const uint32_t drain_bar = tempty_bar + 16;
-  SharedCtl ctl{&s_abort, p.status, p.timeout_ns};
+  SharedCtl ctl{&s_abort, p.status, p.timeout_ns,
+                kPair ? mapa_shared(smem_addr(&s_abort), rank ^ 1u) : 0u};
+  const uint32_t peer_bar = smem_addr(&s_peer_bar);
+  const uint32_t peer_count = smem_addr(&s_peer_count);
 
   if (threadIdx.x == 0) {
     s_abort = 0;
+    mbar_init(peer_bar, 1);
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(full_bar + 8 * s, 1);
       mbar_init(empty_bar + 8 * s, 1);
@@ -260,6 +267,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t stage = 0, phase = 0;
       long long issued = 0;
       bool ok = true;
+      const bool stall = p.test_stall != 0;
+      // one CTA's share of a stage (the same for every unit of a pair)
+      const uint32_t half_bytes = static_cast<uint32_t>(2 + p.BN / 64 / kCtas) * kBox;
       for (int u = first_unit; ok && u < p.num_units; u += unit_step) {
         const WgUnit wu = wg_decode<kSwap, kPair>(p, u, rank);
         // The im2col boxes of the unit: (kw offset, kh offset, first channel).
@@ -311,11 +321,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               break;
             }
             const uint32_t fb = full_bar + 8 * stage;
-            if (leader) mbar_arrive_expect_tx(fb, tx_bytes);
             const uint32_t x_dst = x_ring + stage * x_stage;
             const uint32_t dy_dst = dy_ring + stage * dy_stage;
             const int wx = wo0 * p.sw - p.pw, hx = ho0 * p.sh - p.ph;
-            if constexpr (kPair) {
+            if (stall && issued == 0) {
+              // failure-detection test: this stage never fills, so the
+              // tensor-core issuer's wait on it must run out
+            } else if constexpr (kPair) {
+              if (leader) mbar_arrive_expect_tx(fb, tx_bytes);
               // both CTAs' copies complete on the even CTA's barrier
               const uint32_t fb0 = mapa_shared(fb, 0);
 #pragma unroll
@@ -329,6 +342,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                  static_cast<int>(fw.fo));
               }
             } else {
+              mbar_arrive_expect_tx(fb, tx_bytes);
 #pragma unroll
               for (int q = 0; q < 4; ++q)
                 if (q < nx)
@@ -354,21 +368,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      if (!ok) {
-        if (leader) {
-          // let the copies already in flight land before the CTA may exit
-          const long long first = issued > p.stages ? issued - p.stages : 0;
-          for (long long i = first; i < issued; ++i)
-            wait_bounded(full_bar + 8 * static_cast<uint32_t>(i % p.stages),
-                         static_cast<uint32_t>((i / p.stages) & 1), ctl, false);
-        } else {
-          // the odd CTA's copies complete on the even CTA's barriers: give them
-          // time to land (both CTAs stay resident until the final cluster barrier)
-          const uint64_t t0 = globaltimer_ns();
-          while (globaltimer_ns() - t0 < 200000ull) {
-          }
-        }
-      }
+      producer_finish<kPair>(!ok, issued, stall, p.stages, full_bar, half_bytes, peer_count,
+                             peer_bar, ctl, leader);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
