@@ -948,6 +948,115 @@ def run_norm(args, wl, rank, world, local_rank):
     return 0 if rank != 0 or line["parity"]["ok"] else 1
 
 
+# ---------------------------------------------------------------- decoder block: GroupNorm + SiLU + conv
+
+def run_gnblock(args, wl, rank, world, local_rank):
+    """One decoder block (GroupNorm(32) + SiLU, then the workload's convolution)
+    timed three ways on the same inputs: `separate` = statistics pass, apply
+    pass (writes h) and conv3d_fwd(h); `fused` = statistics pass and
+    conv3d_fwd_gn (h never written); `chained` = conv3d_fwd_gn that also
+    gathers the GroupNorm statistics of its own output (what the next block
+    needs), with this block's statistics taken as given.  value = the chained
+    form's TFLOP/s; every form is parity-gated on sampled rows against the
+    oracle composition (GroupNorm + SiLU in fp64, one rounding, fp64 conv)."""
+    import oracle
+    import video_vae_convolution_implicit_b200 as c3
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    td = TORCH_DTYPE[wl.dtype]
+    Do, Ho, Wo = out_shape(wl)
+    G = 32
+    seed = rank_seed(wl, rank)
+    p = si.conv3d_problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, (Do, Ho, Wo), seed,
+                          td, True, wl.residual, dev)
+    x = p["x"]
+    gamma = (si.tensor((wl.Cin,), seed, 6, 0.2, torch.float32, dev) + 1.0).to(td)
+    beta = si.tensor((wl.Cin,), seed, 7, 0.2, td, dev)
+    h = torch.empty_like(x)
+    y = torch.empty((wl.N, Do, Ho, Wo, wl.Cout), dtype=td, device=dev)
+    stats = torch.empty((wl.N, G, 2), dtype=torch.float64, device=dev)
+    flush = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size // 4 + 1024,
+                        dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    kw = dict(stride=wl.stride, pad=wl.pad, tpad=wl.tpad, stream=stream)
+
+    def separate():
+        c3.groupnorm_stats(x, G, 1e-6, False, stats, stream)
+        c3.groupnorm_silu(x, stats, gamma, beta, h, G, False, True, stream)
+        c3.conv3d_fwd(h, p["w"], p["bias"], p["residual"], y, wl.stride, wl.pad, wl.tpad,
+                      stream=stream)
+
+    def fused():
+        c3.groupnorm_stats(x, G, 1e-6, False, stats, stream)
+        c3.conv3d_gn(x, stats, gamma, beta, p["w"], p["bias"], p["residual"], y, G, **kw)
+
+    def chained():
+        c3.conv3d_gn(x, stats, gamma, beta, p["w"], p["bias"], p["residual"], y, G,
+                     out_groups=G, **kw)
+
+    forms = {"separate": (separate, 3), "fused": (fused, 2), "chained": (chained, 3)}
+    flops = algorithmic_flops(wl)
+    res = {}
+    if rank == 0:
+        # the oracle's h: GroupNorm + SiLU in fp64, rounded once (as an unfused pipeline stores it)
+        hbits = si.bits(torch.from_numpy(oracle.groupnorm_silu(
+            si.bits(x), si.bits(gamma), si.bits(beta),
+            oracle.BF16 if wl.dtype == "bf16" else oracle.F16, G, eps=1e-6)).to(td))
+        hb = dict(host_bits(p), x=hbits)
+        rows = _rows_for_parity(wl)
+    for name, (fn, launches) in forms.items():
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        with ClockSampler(local_rank) as clocks:
+            for a, b in ev:
+                flush.zero_()
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize(dev)
+        ms = [a.elapsed_time(b) for a, b in ev]
+        max_ms = max_over_ranks(sum(ms), dev)
+        st = c3.poll_status(stream)
+        r = {"ms_per_step": max_ms / args.steps,
+             "tflops": whole_job_tflops(flops, world, args.steps, max_ms),
+             "gpu_launches": launches * args.steps, "device_status": c3.status_string(st),
+             "clocks": clocks.summary()}
+        if r["clocks"]:
+            r["clocks"].pop("sm_mhz_series", None)
+        if rank == 0:
+            ref, _ = oracle_rows_timed(hb, wl, rows)
+            got = y.view(-1, wl.Cout)[torch.from_numpy(rows).to(dev)].double().cpu().numpy()
+            err = np.abs(got - ref)
+            mr, rl = float(err.max() / np.abs(ref).max()), float(err.sum() / np.abs(ref).sum())
+            r["parity"] = {"rows": int(rows.size), "max_err_over_max_ref": mr, "rel_l1": rl,
+                           "ok": bool(np.isfinite(got).all() and mr <= 1e-2 and rl <= 2e-3)}
+        res[name] = r
+    peaks, peak_kind = load_peaks()
+    conv_roof = roofline_for(flops, algorithmic_bytes(wl), res["chained"]["ms_per_step"], peaks,
+                             peak_kind)
+    line = {
+        "metric": "decoder block (GroupNorm+SiLU -> conv3d) TFLOPS, conv FLOPs over the block's time",
+        "value": res["chained"]["tflops"], "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["chained"]["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded SplitMix64 normals)",
+        "config": dict(describe(wl, world), groupnorm_groups=G, l2="flushed between steps"),
+        "roofline": dict(conv_roof, kernel=KERNEL_NAME + " (GroupNorm variant)"),
+        "forms": res,
+        "gpu_launches": res["chained"]["gpu_launches"],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    ok = all(r["device_status"] == "ok" and (rank != 0 or r["parity"]["ok"]) for r in res.values())
+    return 0 if ok else 1
+
+
 # ---------------------------------------------------------------- main
 
 def main():
@@ -957,8 +1066,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="cfg2", choices=sorted(WORKLOADS) + sorted(NORM_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "dgrad", "wgrad"],
-                    help="forward convolution (default) or one of its backward passes")
+    ap.add_argument("--pass", dest="pass_", default="fwd",
+                    choices=["fwd", "dgrad", "wgrad", "gnblock"],
+                    help="forward convolution (default), one of its backward passes, or the "
+                         "decoder block GroupNorm+SiLU -> conv in its separate and fused forms")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true",
@@ -980,6 +1091,10 @@ def main():
             print(json.dumps({"impl": "reference", "unavailable":
                               "the reference arm times the convolution oracle only"}))
             return 0
+        if args.pass_ == "gnblock":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the reference arm times the convolution oracle only"}))
+            return 0
         if args.pass_ != "fwd":
             return run_reference_backward(args, wl, rank, world)
         return run_reference(args, wl, rank, world)
@@ -992,6 +1107,8 @@ def main():
     try:
         if is_norm:
             fn = run_norm
+        elif args.pass_ == "gnblock":
+            fn = run_gnblock
         else:
             fn = run_ours if args.pass_ == "fwd" else run_backward
         rc = fn(args, wl, rank, world, local_rank)

@@ -203,6 +203,44 @@ CONV3D_API conv3d_status_t conv3d_groupnorm_silu(const void* x, const double* st
                                                  conv3d_dtype_t dtype, struct CUstream_st* stream);
 
 /*
+ * conv3d_fwd_gn -- the convolution of a decoder block with the GroupNorm work
+ * around it fused in (news.bugfactory.tech: a fused GroupNorm + SiLU kernel;
+ * stable-diffusion.cpp discussion "Exe Heavy Metal": GROUP_NORM on the GPU;
+ * the decoder block runs normalise -> activate -> convolve, and the next
+ * block normalises the result again).
+ *
+ * In (stats non-NULL): y = conv3d(h, w) + bias + residual with
+ *   h[n,f,hh,ww,c] = silu((x - mean[s][g]) * rstd[s][g] * gamma[c] + beta[c]),
+ *   g = c / (Cin/groups), s = the statistic set of frame f (the sample, or the
+ *   frame of the sample with per_frame = 1), rounded once to the dtype -- the
+ *   value an unfused pipeline would store -- computed as the kernel reads x,
+ *   so h is never written to memory; the convolution's padding (spatial
+ *   zeros, the temporal rule) applies to h.  apply_silu = 0 leaves out the
+ *   SiLU.  stats: {mean, rstd} from conv3d_groupnorm_stats over x with the
+ *   same groups and per_frame ([sets][groups][2] doubles, 8-byte aligned);
+ *   gamma, beta: [Cin] of the dtype, 16-byte aligned, or NULL (1 and 0).
+ *   stats = NULL: plain x (groups, per_frame, apply_silu, gamma, beta unused).
+ * Out (out_stats non-NULL): also writes the GroupNorm statistics of y itself
+ *   -- what conv3d_groupnorm_stats(y, out_groups, per_frame = 0, out_eps)
+ *   would give, {mean, rstd} per sample and group of the rounded outputs,
+ *   [N][out_groups][2] doubles -- gathered by the kernel as it stores y, so
+ *   the next block's normalisation needs no statistics pass over y.
+ *   1 <= out_groups <= 64 dividing Cout; out_eps >= 0.
+ *
+ * Every other argument and rule is conv3d_fwd's (its workspace included);
+ * the cached-frames rule is not supported (CONV3D_ERR_UNSUPPORTED).
+ */
+CONV3D_API conv3d_status_t conv3d_fwd_gn(const void* x, const double* stats, const void* gamma,
+                                         const void* beta, int groups, int per_frame,
+                                         int apply_silu, const void* w, const void* bias,
+                                         const void* residual, void* y, int N, int Cin, int D,
+                                         int H, int W, int Cout, const int kernel[3],
+                                         const int stride[3], const int pad[3],
+                                         conv3d_tpad_t tpad, conv3d_dtype_t dtype,
+                                         double* out_stats, int out_groups, float out_eps,
+                                         struct CUstream_st* stream);
+
+/*
  * conv3d_bwd_data -- dx, the gradient of the convolution's input (the pages'
  * on-device fine-tuning trains convolution layers: engineering.drawthings.ai,
  * LoRA post).  For stride 1 it is itself a convolution, of dy with every tap

@@ -297,3 +297,18 @@ def test_arm_stall_rejects_bad_arguments():
         with pytest.raises(c3.Conv3dError):
             c3.test_arm_stall(launches, ms)
     c3.test_arm_stall(0, 50)
+
+
+def test_fused_groupnorm_entry_validates_before_any_launch():
+    S = 0x600000000      # fake stats, gamma, beta
+    args = (X, S, S + 0x10000, S + 0x20000)
+    rest = (Wt, B, None, Y, 1, 64, 3, 8, 8, 64, (3, 3, 3), (1, 1, 1), (0, 1, 1))
+    assert c3.conv3d_gn_ptr(*args, 8, 0, 1, *rest, c3.TPAD_CAUSAL_CACHED, c3.BF16, None) == \
+        Status.UNSUPPORTED
+    assert c3.conv3d_gn_ptr(*args, 7, 0, 1, *rest, c3.TPAD_CAUSAL_REPLICATE, c3.BF16, None) == \
+        Status.INVALID_ARG                                   # 7 groups do not divide 64
+    assert c3.conv3d_gn_ptr(*args, 8, 2, 1, *rest, c3.TPAD_CAUSAL_REPLICATE, c3.BF16, None) == \
+        Status.INVALID_ARG                                   # per_frame must be 0 or 1
+    bad = (X, S + 4, S + 0x10000, S + 0x20000)
+    assert c3.conv3d_gn_ptr(*bad, 8, 0, 1, *rest, c3.TPAD_CAUSAL_REPLICATE, c3.BF16, None) == \
+        Status.ALIGNMENT                                     # stats not 8-byte aligned

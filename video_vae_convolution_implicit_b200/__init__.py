@@ -26,7 +26,7 @@ __all__ = [
     "TPAD_ZERO", "TPAD_CAUSAL_REPLICATE", "TPAD_CAUSAL_ZERO", "TPAD_CAUSAL_CACHED", "F16", "BF16",
     "Status", "Conv3dError", "lib_path", "status_string", "last_error",
     "conv3d", "conv3d_fwd", "conv3d_fwd_ptr", "conv3d_fwd_ws_ptr", "conv3d_fwd_noalloc_ptr",
-    "conv3d_fwd_cached_ptr", "output_shape", "workspace_bytes",
+    "conv3d_fwd_cached_ptr", "conv3d_gn", "conv3d_gn_ptr", "output_shape", "workspace_bytes",
     "groupnorm_stats", "groupnorm_silu", "groupnorm_stats_ptr", "groupnorm_silu_ptr",
     "conv3d_bwd_data", "conv3d_bwd_data_ptr", "bwd_data_workspace_bytes",
     "conv3d_bwd_weight", "conv3d_bwd_weight_ptr", "bwd_weight_workspace_bytes",
@@ -107,6 +107,9 @@ _lib.conv3d_release.restype = None
 _lib.conv3d_release.argtypes = []
 _lib.conv3d_selftest_wait_timeout.restype = _c
 _lib.conv3d_selftest_wait_timeout.argtypes = [_c]
+_lib.conv3d_fwd_gn.restype = _c
+_lib.conv3d_fwd_gn.argtypes = ([_vp, _vp, _vp, _vp, _c, _c, _c] + [_vp] * 4 + [_c] * 6 + [_i3] * 3
+                                + [_c, _c, _vp, _c, ctypes.c_float, _vp])
 _lib.conv3d_test_arm_stall.restype = _c
 _lib.conv3d_test_arm_stall.argtypes = [_c, _c]
 
@@ -253,6 +256,46 @@ def conv3d(x: torch.Tensor, w: torch.Tensor, bias=None, residual=None, stride=(1
     out = output_shape(D, H, W, (kt, kh, kw), stride, pad, tpad)
     y = torch.empty((N, *out, Cout), dtype=x.dtype, device=x.device)
     return conv3d_fwd(x, w, bias, residual, y, stride, pad, tpad, stream, prev=prev)
+
+
+def conv3d_gn_ptr(x, stats, gamma, beta, groups, per_frame, apply_silu, w, bias, residual, y, N,
+                  Cin, D, H, W, Cout, kernel, stride, pad, tpad, dtype, stream, out_stats=None,
+                  out_groups=0, out_eps=1e-6) -> int:
+    """Raw-pointer call of conv3d_fwd_gn; returns the status code (no raise)."""
+    return _lib.conv3d_fwd_gn(x, stats, gamma, beta, groups, int(per_frame), int(apply_silu), w,
+                              bias, residual, y, N, Cin, D, H, W, Cout, _i3(*kernel),
+                              _i3(*stride), _i3(*pad), tpad, dtype, out_stats, int(out_groups),
+                              float(out_eps), stream)
+
+
+def conv3d_gn(x: torch.Tensor, stats, gamma, beta, w: torch.Tensor, bias=None,
+              residual=None, y: torch.Tensor | None = None, groups: int | None = None,
+              per_frame: bool = False, apply_silu: bool = True, stride=(1, 1, 1), pad=(0, 1, 1),
+              tpad=TPAD_CAUSAL_REPLICATE, out_groups: int = 0, out_eps: float = 1e-6,
+              stream=None):
+    """y = conv3d(silu(GroupNorm(x)), w) + bias + residual with the GroupNorm + SiLU
+    applied as the convolution reads x (``stats`` from groupnorm_stats over x, or
+    None for plain x).  With ``out_groups`` > 0 also returns the per-sample
+    GroupNorm statistics of y ([N, out_groups, 2] float64): (y, out_stats)."""
+    N, D, H, W, Cin = x.shape
+    Cout, kt, kh, kw, _ = w.shape
+    groups = (stats.shape[1] if stats is not None else 1) if groups is None else groups
+    if y is None:
+        out = output_shape(D, H, W, (kt, kh, kw), stride, pad, tpad)
+        y = torch.empty((N, *out, Cout), dtype=x.dtype, device=x.device)
+    for name, t in (("x", x), ("w", w), ("y", y)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype:
+            raise ValueError(f"{name} must be a contiguous CUDA tensor of x's dtype")
+    if stats is not None and (stats.dtype != torch.float64 or not stats.is_cuda):
+        raise ValueError("stats must be a float64 CUDA tensor")
+    out_stats = (torch.empty((N, out_groups, 2), dtype=torch.float64, device=x.device)
+                 if out_groups > 0 else None)
+    _check(conv3d_gn_ptr(x.data_ptr(), _ptr(stats), _ptr(gamma), _ptr(beta), groups,
+                         per_frame, apply_silu, w.data_ptr(), _ptr(bias), _ptr(residual),
+                         y.data_ptr(), N, Cin, D, H, W, Cout, (kt, kh, kw), stride, pad, tpad,
+                         _dtype_code(x.dtype), _stream_handle(stream), _ptr(out_stats), out_groups,
+                         out_eps))
+    return (y, out_stats) if out_stats is not None else y
 
 
 def poll_status(stream=None) -> int:

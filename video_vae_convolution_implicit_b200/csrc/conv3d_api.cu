@@ -21,6 +21,10 @@
 #include "conv3d_kernel.cuh"
 #include "wgrad_kernel.cuh"
 
+// GroupNorm finalize (groupnorm.cu): {sum, sum of squares} -> {mean, rstd}.
+cudaError_t conv3d_gn_finalize(double* stats, long long pairs, double count, double eps,
+                               cudaStream_t stream);
+
 namespace {
 
 using namespace conv3d;
@@ -84,6 +88,13 @@ struct Problem {
   bool out_f32;      // write y in fp32 (internal: the backward pass's padded-frame gradient)
   const void* prev;  // cached frames before the chunk (CONV3D_TPAD_CAUSAL_CACHED) or null
   bool fold;  // first-frame path: fold the temporal taps into a (hi, lo) pair
+  // GroupNorm + SiLU applied to x as it is read (conv3d_fwd_gn); gn_stats null otherwise
+  const double* gn_stats;
+  const void* gn_gamma;
+  const void* gn_beta;
+  int gn_groups, gn_per_frame, gn_silu;
+  double* gn_out;      // sums of y's GroupNorm statistics (per sample), or null
+  int gn_out_groups;
 };
 
 bool output_extents(int D, int H, int W, const int k[3], const int stride[3], const int pad[3],
@@ -214,6 +225,11 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
   // a single causal-replicate frame: every temporal tap of the one output
   // frame reads frame 0 (whatever the temporal stride)
   P.fold = (tpad == CONV3D_TPAD_CAUSAL_REPLICATE && D == 1 && kernel[0] > 1);
+  P.gn_stats = nullptr;
+  P.gn_gamma = P.gn_beta = nullptr;
+  P.gn_groups = P.gn_per_frame = P.gn_silu = 0;
+  P.gn_out = nullptr;
+  P.gn_out_groups = 0;
   return CONV3D_OK;
 }
 
@@ -356,7 +372,7 @@ struct DeviceState {
   };
   Scratch scratch[16] = {};
   int n_scratch = 0;
-  bool attr_set[8] = {};         // per kernel variant
+  bool attr_set[16] = {};        // per kernel variant
   int pair_clusters = 0;         // co-resident CTA pairs (occupancy query)
   int wg_pair_clusters = 0;      // the same for the weight-gradient kernel
   bool wg_attr_set[16] = {};     // per weight-gradient kernel variant
@@ -572,6 +588,8 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, b
   kp.Do = P.Do;
   kp.Ho = P.Ho;
   kp.Wo = P.Wo;
+  kp.H = P.H;
+  kp.W = P.W;
   kp.HoWo = P.Ho * P.Wo;
   kp.Cin = P.Cin;
   kp.Cout = P.Cout;
@@ -585,6 +603,14 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, b
   kp.ph = P.ph;
   kp.pw = P.pw;
   kp.tpad = P.fold ? 1 : static_cast<int>(P.tpad);
+  kp.gn_stats = P.gn_stats;
+  kp.gn_gamma = static_cast<const uint16_t*>(P.gn_gamma);
+  kp.gn_beta = static_cast<const uint16_t*>(P.gn_beta);
+  kp.gn_groups = P.gn_groups;
+  kp.gn_per_frame = P.gn_per_frame;
+  kp.gn_silu = P.gn_silu;
+  kp.gn_out = P.gn_out;
+  kp.gn_out_groups = P.gn_out_groups;
   kp.n_chunks = (P.Cin + BK - 1) / BK;
 
   // A tcgen05.mma step with N < 256 takes as long as one with N = 256, so
@@ -615,7 +641,8 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, b
     if (env[0] == '1') L.pair = true;
   }
   if (L.swap) L.pair = false;
-  if (P.out_f32) L.pair = false;   // the fp32 epilogue exists in the single and transposed variants
+  if (P.out_f32) L.pair = false;
+  if (P.gn_stats || P.gn_out) L.pair = false;   // both exist in the one-CTA variants   // the fp32 epilogue exists in the single and transposed variants
   const int ctas = L.pair ? 2 : 1;
   if (L.swap) {
     kp.co_tile = 128;
@@ -668,7 +695,7 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, b
   kp.out_f32 = P.out_f32 ? 1 : 0;
   const int reserve = 1024 /*alignment slack*/ + EPI_Y_BYTES * (kp.out_f32 ? 2 : 1) +
                       EPI_Y_BYTES * (kp.has_residual ? 1 : 0) +
-                      8 * (2 * MAX_STAGES + 5 + 2 * EPI_WARPS);
+                      8 * (3 * MAX_STAGES + 5 + 2 * EPI_WARPS);
   int stages = (S.max_smem_optin - reserve - 64 /*static smem*/) / stage_bytes;
   if (stages > MAX_STAGES) stages = MAX_STAGES;
   if (stages < 2) {
@@ -683,13 +710,14 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, b
   return CONV3D_OK;
 }
 
-template <bool kBF16, bool kPair, bool kSwap>
+template <bool kBF16, bool kPair, bool kSwap, bool kGN = false>
 conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtensorMap& map_a,
                               const CUtensorMap& map_b, const CUtensorMap& map_y,
                               const CUtensorMap& map_r, const CUtensorMap& map_p,
                               cudaStream_t stream) {
-  auto kern = conv3d_implicit_gemm_kernel<kBF16, kPair, kSwap>;
-  const int variant = (kBF16 ? 1 : 0) + (kPair ? 2 : 0) + (kSwap ? 4 : 0);
+  auto kern = conv3d_implicit_gemm_kernel<kBF16, kPair, kSwap, kGN>;
+  const int variant = (kBF16 ? 1 : 0) + (kPair ? 2 : 0) + (kSwap ? 4 : 0) + (kGN ? 8 : 0);
+  const int threads = kGN ? GN_THREADS : NUM_THREADS;
   cudaError_t e;
   int units = S.num_sms;  // co-resident CTAs (or CTA pairs)
   {
@@ -709,7 +737,7 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         cfg.gridDim = dim3(2 * (S.num_sms / 2), 1, 1);
-        cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+        cfg.blockDim = dim3(threads, 1, 1);
         cfg.dynamicSmemBytes = S.max_smem_optin - 64;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
@@ -729,17 +757,18 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3((kPair ? 2 : 1) * unit_count, 1, 1);
-  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = L.smem;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = kPair ? 1 : 0;
   if (plan_log())
     fprintf(stderr,
-            "libconv3d: implicit GEMM %s %s, %d tiles of %d pixels x %d channels, grid %d, "
+            "libconv3d: implicit GEMM %s%s %s, %d tiles of %d pixels x %d channels, grid %d, "
             "%d k-blocks x %d taps, %d stages, %zu B shared, %s output, last %d tiles in %d "
             "pieces\n",
-            kSwap ? "transposed" : kPair ? "CTA pair" : "single", kBF16 ? "bf16" : "fp16",
+            kSwap ? "transposed" : kPair ? "CTA pair" : "single",
+            kGN ? " with GroupNorm+SiLU of x" : "", kBF16 ? "bf16" : "fp16",
             L.kp.num_tiles, L.kp.pix_tile, L.kp.co_tile, static_cast<int>(cfg.gridDim.x),
             L.kp.n_chunks, L.kp.kt * L.kp.kh * L.kp.kw, L.kp.stages, L.smem,
             L.kp.out_f32 ? "fp32" : "16-bit", L.kp.num_tiles - L.kp.split_first, L.kp.split_s);
@@ -778,6 +807,13 @@ conv3d_status_t launch_planned(DeviceState& S, const Problem& P, LaunchPlan& L, 
     if (st != CONV3D_OK) return st;
   } else {
     map_p = map_a;  // never read: no tap reads before frame 0 in this mode
+  }
+  if (L.kp.gn_stats != nullptr) {   // GroupNorm + SiLU of x (never a CTA pair)
+    if (L.swap)
+      return bf16 ? launch_kernel<true, false, true, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream)
+                  : launch_kernel<false, false, true, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+    return bf16 ? launch_kernel<true, false, false, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream)
+                : launch_kernel<false, false, false, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
   }
   if (L.swap)
     return bf16 ? launch_kernel<true, false, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream)
@@ -1166,6 +1202,70 @@ conv3d_status_t conv3d_fwd_cached(const void* x, const void* prev, const void* w
                                 pad, CONV3D_TPAD_CAUSAL_CACHED, dtype, P, prev);
   if (st != CONV3D_OK) return st;
   return run(P, x, w, bias, residual, y, nullptr, 0, false, stream);
+}
+
+conv3d_status_t conv3d_fwd_gn(const void* x, const double* stats, const void* gamma,
+                              const void* beta, int groups, int per_frame, int apply_silu,
+                              const void* w, const void* bias, const void* residual, void* y,
+                              int N, int Cin, int D, int H, int W, int Cout, const int kernel[3],
+                              const int stride[3], const int pad[3], conv3d_tpad_t tpad,
+                              conv3d_dtype_t dtype, double* out_stats, int out_groups,
+                              float out_eps, struct CUstream_st* stream) {
+  if (tpad == CONV3D_TPAD_CAUSAL_CACHED) {
+    set_error("the GroupNorm-fused convolution does not take cached frames");
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  Problem P;
+  conv3d_status_t st = validate(x, w, bias, residual, y, N, Cin, D, H, W, Cout, kernel, stride,
+                                pad, tpad, dtype, P);
+  if (st != CONV3D_OK) return st;
+  if (stats && (groups < 1 || Cin % groups != 0 || (per_frame != 0 && per_frame != 1))) {
+    set_error("groups >= 1 must divide Cin and per_frame be 0 or 1");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if (out_stats && (out_groups < 1 || out_groups > 64 || Cout % out_groups != 0 ||
+                    !(out_eps >= 0.0f))) {
+    set_error("out_groups must divide Cout and be in [1, 64], out_eps >= 0");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if ((stats && (reinterpret_cast<uintptr_t>(stats) & 7u)) || (stats && gamma && !aligned16(gamma)) ||
+      (stats && beta && !aligned16(beta)) ||
+      (out_stats && (reinterpret_cast<uintptr_t>(out_stats) & 7u))) {
+    set_error("stats and out_stats must be 8-byte, gamma and beta 16-byte aligned");
+    return CONV3D_ERR_ALIGNMENT;
+  }
+  const size_t yb = static_cast<size_t>(N) * P.Do * P.Ho * P.Wo * Cout * 2;
+  const size_t sets = static_cast<size_t>(N) * (per_frame ? D : 1);
+  const size_t ob = static_cast<size_t>(N) * out_groups * 16;
+  if ((stats && (overlaps(y, yb, stats, sets * groups * 16) ||
+                 overlaps(y, yb, gamma, Cin * 2ull) || overlaps(y, yb, beta, Cin * 2ull))) ||
+      (out_stats && (overlaps(out_stats, ob, y, yb) || overlaps(out_stats, ob, x, 2ull * N * D * H * W * Cin) ||
+                     (stats && overlaps(out_stats, ob, stats, sets * groups * 16))))) {
+    set_error("y, stats and out_stats must not overlap each other or the inputs");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if (stats) {
+    P.gn_stats = stats;
+    P.gn_gamma = gamma;
+    P.gn_beta = beta;
+    P.gn_groups = groups;
+    P.gn_per_frame = per_frame;
+    P.gn_silu = apply_silu ? 1 : 0;
+  }
+  if (out_stats) {
+    cudaError_t e = cudaMemsetAsync(out_stats, 0, ob, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "statistics clear");
+    P.gn_out = out_stats;
+    P.gn_out_groups = out_groups;
+  }
+  if ((st = run(P, x, w, bias, residual, y, nullptr, 0, true, stream)) != CONV3D_OK) return st;
+  if (out_stats) {
+    const double count = static_cast<double>(P.Do) * P.Ho * P.Wo * (Cout / out_groups);
+    cudaError_t e = conv3d_gn_finalize(out_stats, static_cast<long long>(N) * out_groups, count,
+                                       static_cast<double>(out_eps), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "statistics finalize launch");
+  }
+  return CONV3D_OK;
 }
 
 size_t conv3d_bwd_data_workspace_bytes(int N, int Cin, int D, int H, int W, int Cout,

@@ -43,12 +43,14 @@ constexpr int BM = 128;             // output pixels per tile (TMEM lanes)
 constexpr int BK = 64;              // channels per k-block (128 bytes of fp16/bf16)
 constexpr int A_STAGE_BYTES = BM * BK * 2;
 constexpr int NUM_THREADS = 192;
+constexpr int GN_THREADS = 320;     // with the GroupNorm + SiLU operand transform (4 more warps)
 constexpr int MAX_STAGES = 8;
 
 constexpr int STATUS_TIMEOUT = 5;   // mirrors CONV3D_ERR_TIMEOUT
 
 struct KernelParams {
   int D, Do, Ho, Wo;                 // input frames; output extents
+  int H, W;                          // input extents
   int HoWo;
   int Cin, Cout;
   int kt, kh, kw;
@@ -83,6 +85,19 @@ struct KernelParams {
   unsigned long long timeout_ns;
   int test_stall;                    // failure-detection test: the producer skips the
                                      // copies of its first stage (armed from the host)
+  // GroupNorm + SiLU applied to x as the kernel reads it (GroupNorm variant):
+  // h = silu((x - mean) * rstd * gamma + beta) per statistic set and group
+  const double* gn_stats;            // [sets][groups][2] {mean, rstd}
+  const uint16_t* gn_gamma;          // [Cin] or null (1)
+  const uint16_t* gn_beta;           // [Cin] or null (0)
+  int gn_groups;
+  int gn_per_frame;                  // sets are frames of a sample (else whole samples)
+  int gn_silu;                       // apply the SiLU after the normalisation
+  // GroupNorm statistics of y (per sample) gathered by the epilogue from the
+  // rounded outputs: fp64 {sum, sum of squares} added into gn_out
+  // [N][gn_out_groups][2] (zeroed by the host), or null
+  double* gn_out;
+  int gn_out_groups;                 // at most 64; divides Cout
 };
 
 // Epilogue staging: each epilogue warp owns two 32-row x 32-channel buffers
@@ -340,6 +355,58 @@ __device__ __forceinline__ void sum_pieces(const KernelParams& p, int slot0, uin
   }
 }
 
+// silu(z) = z * sigmoid(z) = h + h * tanh(h) with h = z/2: one special-function
+// operation (the hardware tanh approximation, relative error about 2^-11,
+// below the 2^-9 of the rounding that follows).
+__device__ __forceinline__ float silu_fast(float z) {
+  const float h = 0.5f * z;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+  return fmaf(h, t, h);
+}
+
+// Output GroupNorm statistics of one epilogue warp: lane l keeps the fp64
+// {sum, sum of squares} of groups l and l + 32 of sample n.
+struct GnOut {
+  double s0, q0, s1, q1;
+  int n;   // sample being gathered, -1 for none yet
+};
+
+// Warp totals of each lane's (s, q) for group g, kept by the lane owning g.
+__device__ __forceinline__ void gn_out_add(GnOut& a, int g, float s, float q, uint32_t lane) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    s += __shfl_xor_sync(0xFFFFFFFFu, s, off);
+    q += __shfl_xor_sync(0xFFFFFFFFu, q, off);
+  }
+  if ((g & 31) == static_cast<int>(lane)) {
+    if (g < 32) {
+      a.s0 += s;
+      a.q0 += q;
+    } else {
+      a.s1 += s;
+      a.q1 += q;
+    }
+  }
+}
+
+// Adds the warp's sums of its current sample to the global statistics.
+__device__ __forceinline__ void gn_out_flush(double* gn_out, int groups, GnOut& a,
+                                             uint32_t lane) {
+  if (a.n >= 0) {
+    double* dst = gn_out + static_cast<size_t>(a.n) * groups * 2;
+    if (static_cast<int>(lane) < groups) {
+      atomicAdd(dst + 2 * lane, a.s0);
+      atomicAdd(dst + 2 * lane + 1, a.q0);
+    }
+    if (static_cast<int>(lane) + 32 < groups) {
+      atomicAdd(dst + 2 * (lane + 32), a.s1);
+      atomicAdd(dst + 2 * (lane + 32) + 1, a.q1);
+    }
+  }
+  a.s0 = a.q0 = a.s1 = a.q1 = 0.0;
+}
+
 template <bool kBF16>
 struct Cvt;
 
@@ -380,8 +447,14 @@ struct Cvt<false> {
 //   channels (the weight tile is the A operand), N = 256 output pixels (the
 //   im2col tile is the B operand).  TMEM lane = channel, column = pixel; the
 //   epilogue transposes through shared memory before the TMA store.
-template <bool kBF16, bool kPair, bool kSwap>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+// kGN (single-CTA and transposed variants): four more warps (6-9) apply
+//   GroupNorm + SiLU to the x operand in shared memory between its TMA load
+//   and the MMAs that read it, so that the normalised activation is never
+//   written to memory: rows that hold spatial padding stay zero (the padding
+//   belongs to the normalised tensor), and the tensor-core issuer waits for
+//   the transform of a stage instead of its load.
+template <bool kBF16, bool kPair, bool kSwap, bool kGN = false>
+__global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
     conv3d_implicit_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                                 const __grid_constant__ CUtensorMap map_b,
                                 const __grid_constant__ CUtensorMap map_y,
@@ -420,6 +493,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tempty_bar = tfull_bar + 16;             // [2]
   const uint32_t drain_bar = tempty_bar + 16;             // [1]
   const uint32_t rfull_bar = drain_bar + 8;               // [EPI_WARPS][2]
+  const uint32_t ready_bar = rfull_bar + 16 * EPI_WARPS;  // [stages] (GroupNorm variant)
 
   SharedCtl ctl{&s_abort, p.status, p.timeout_ns,
                 kPair ? mapa_shared(smem_addr(&s_abort), rank ^ 1u) : 0u};
@@ -439,6 +513,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(drain_bar, 1);
     mbar_init(peer_bar, 1);
     for (int e = 0; e < 2 * EPI_WARPS; ++e) mbar_init(rfull_bar + 8 * e, 1);
+    if constexpr (kGN)
+      for (int s = 0; s < p.stages; ++s) mbar_init(ready_bar + 8 * s, 4);
     fence_mbar_init();
     prefetch_tensormap(&map_a);
     prefetch_tensormap(&map_b);
@@ -551,7 +627,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * static_cast<uint32_t>(p.BN);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!wait_bounded(full_bar + 8 * stage, phase, ctl, true)) {
+          // the stage's copies have landed (and, GroupNorm variant, been transformed)
+          if (!wait_bounded((kGN ? ready_bar : full_bar) + 8 * stage, phase, ctl, true)) {
             ok = false;
             break;
           }
@@ -593,6 +670,110 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mma_commit(drain_bar);
       wait_bounded(drain_bar, 0, ctl, false);
     }
+  } else if (kGN && warp >= 2 + EPI_WARPS) {
+    // ------------------------------------------------------------ GroupNorm + SiLU of x
+    // The x operand of a stage is `rows` rows (output pixels) of 64 channels,
+    // 128 bytes each, 128-byte swizzled: 16-byte chunk c of row r sits at
+    // physical chunk c ^ (r & 7).  Thread t owns physical chunk t & 7 of the
+    // rows t/8 + 16j, whose low three bits are all those of t/8, so it always
+    // sees the same logical chunk: channels 8 * ((t & 7) ^ (t/8 & 7)) .. +7 of
+    // the k-block, whose scale and shift it keeps in registers.  Rows whose
+    // window position is spatial padding were zero-filled by the TMA and stay
+    // zero; the others become h = silu(x * scale + shift) rounded once.
+    using C = Cvt<kBF16>;
+    constexpr int kRows = kSwap ? 16 : 8;         // 256 or 128 rows per operand stage
+    const uint32_t t = threadIdx.x - 32u * (2 + EPI_WARPS);
+    const uint32_t pchunk = t & 7u;
+    const uint32_t r0 = t >> 3;
+    const uint32_t lchunk = pchunk ^ (r0 & 7u);
+    const uint32_t x_ring = kSwap ? b_ring : a_ring;
+    const uint32_t x_stage = kSwap ? b_stage_bytes : static_cast<uint32_t>(A_STAGE_BYTES);
+    const int cg = p.Cin / p.gn_groups;
+    uint32_t stage = 0, phase = 0;
+    bool ok = true;
+    for (int i = unit; ok && i < p.num_items; i += num_units) {
+      const Work wk = decode_work(p, i);
+      const Tile& tl = wk.tl;
+      // output pixel of each of this thread's rows (ho < 0: past the frame)
+      int rho[kRows], rwo[kRows];
+#pragma unroll
+      for (int j = 0; j < kRows; ++j) {
+        const int q = tl.p0 + static_cast<int>(r0) + 16 * j;
+        rho[j] = q < p.HoWo ? q / p.Wo : -0x100000;
+        rwo[j] = q < p.HoWo ? q - rho[j] * p.Wo : 0;
+      }
+      int kb = 0;
+      for (int it = 0; ok && kb < wk.kb_hi && it < p.kt; ++it) {
+        const int f = source_frame(p, tl.to, it);
+        if (f == kNoFrame) continue;
+        const int set = p.gn_per_frame ? tl.n * p.D + f : tl.n;
+        const double* st = p.gn_stats + static_cast<size_t>(set) * p.gn_groups * 2;
+        for (int ih = 0; ok && kb < wk.kb_hi && ih < p.kh; ++ih) {
+          for (int iw = 0; ok && kb < wk.kb_hi && iw < p.kw; ++iw) {
+            for (int cc = 0; cc < p.n_chunks && kb < wk.kb_hi; ++cc) {
+              if (kb++ < wk.kb_lo) continue;
+              if (!wait_bounded(full_bar + 8 * stage, phase, ctl, true)) {
+                ok = false;
+                break;
+              }
+              const int c0 = cc * BK + static_cast<int>(lchunk) * 8;
+              if (c0 < p.Cin) {          // channels past Cin meet zero weights
+                float sc[8], sh[8];
+                uint4 ga = make_uint4(0, 0, 0, 0), be = make_uint4(0, 0, 0, 0);
+                if (p.gn_gamma) ga = __ldg(reinterpret_cast<const uint4*>(p.gn_gamma + c0));
+                if (p.gn_beta) be = __ldg(reinterpret_cast<const uint4*>(p.gn_beta + c0));
+                const uint32_t gw[4] = {ga.x, ga.y, ga.z, ga.w};
+                const uint32_t bw[4] = {be.x, be.y, be.z, be.w};
+                int g_prev = -1;
+                float mean = 0.0f, rstd = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const int g = (c0 + e) / cg;
+                  if (g != g_prev) {
+                    mean = static_cast<float>(st[2 * g]);
+                    rstd = static_cast<float>(st[2 * g + 1]);
+                    g_prev = g;
+                  }
+                  const float gam = p.gn_gamma ? ((e & 1) ? C::hi(gw[e >> 1]) : C::lo(gw[e >> 1])) : 1.0f;
+                  const float bet = p.gn_beta ? ((e & 1) ? C::hi(bw[e >> 1]) : C::lo(bw[e >> 1])) : 0.0f;
+                  sc[e] = rstd * gam;
+                  sh[e] = fmaf(-mean, sc[e], bet);
+                }
+                const uint32_t base = x_ring + stage * x_stage + pchunk * 16u;
+#pragma unroll
+                for (int j = 0; j < kRows; ++j) {
+                  const int h = rho[j] * p.sh + ih - p.ph;
+                  const int w = rwo[j] * p.sw + iw - p.pw;
+                  if (h < 0 || h >= p.H || w < 0 || w >= p.W) continue;   // padding (or past the frame)
+                  const uint32_t addr = base + (r0 + 16u * j) * 128u;
+                  const uint4 q = ld_shared_v4(addr);
+                  const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+                  uint32_t o[4];
+#pragma unroll
+                  for (int e2 = 0; e2 < 4; ++e2) {
+                    float a = fmaf(C::lo(qw[e2]), sc[2 * e2], sh[2 * e2]);
+                    float b = fmaf(C::hi(qw[e2]), sc[2 * e2 + 1], sh[2 * e2 + 1]);
+                    if (p.gn_silu) {
+                      a = silu_fast(a);
+                      b = silu_fast(b);
+                    }
+                    o[e2] = C::pack(a, b);
+                  }
+                  st_shared_v4(addr, o[0], o[1], o[2], o[3]);
+                }
+              }
+              fence_proxy_async_shared();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(ready_bar + 8 * stage);
+              if (++stage == static_cast<uint32_t>(p.stages)) {
+                stage = 0;
+                phase ^= 1;
+              }
+            }
+          }
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     // Warp q drains TMEM lanes [32q, 32q+32) = 32 output pixels of the tile,
@@ -613,6 +794,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint4* bias4 = reinterpret_cast<const uint4*>(p.bias);
     const int chunks = p.BN / 32;
     bool ok = true;
+    GnOut gacc{0.0, 0.0, 0.0, 0.0, -1};
+    const int gn_cg = p.gn_out != nullptr ? p.Cout / p.gn_out_groups : 1;
     if constexpr (kSwap) {
       // Thread = one output channel (TMEM lane), 32 pixels (columns) per chunk.
       for (int i = unit; ok && i < p.num_items; i += num_units, ++local) {
@@ -621,6 +804,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const Work wk = decode_work(p, i);
         const Tile& tl = wk.tl;
         const bool piece = wk.slot >= 0;
+        if (p.gn_out != nullptr && tl.n != gacc.n) {
+          gn_out_flush(p.gn_out, p.gn_out_groups, gacc, lane);
+          gacc.n = tl.n;
+        }
         const int ch0 = tl.co0 + static_cast<int>(quarter) * 32;   // this warp's channels
         const bool warp_live = ch0 < p.Cout;
         int live_chunks = (p.HoWo - tl.p0 + 31) / 32;   // pixel chunks inside the frame
@@ -705,12 +892,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                              "f"(v[e])
                              : "memory");
             } else {
+              float gs = 0.0f, gq = 0.0f;   // this channel's rounded outputs, for the statistics
 #pragma unroll
               for (int e = 0; e < 32; ++e) {
                 const uint16_t q = static_cast<uint16_t>(C::pack(v[e], 0.0f) & 0xFFFFu);
                 asm volatile("st.shared.u16 [%0], %1;" ::"r"(yb + swz64(e, lane >> 3) + col_byte),
                              "h"(q)
                              : "memory");
+                if (p.gn_out != nullptr && tl.p0 + 32 * j + e < p.HoWo) {
+                  const float yv = C::lo(q);
+                  gs += yv;
+                  gq = fmaf(yv, yv, gq);
+                }
+              }
+              if (p.gn_out != nullptr) {
+                // lane = channel ch: add its sums to its group's warp total
+                const int my_g = ch < p.Cout ? ch / gn_cg : -1;
+                const int g_last = (ch0 + 31 < p.Cout ? ch0 + 31 : p.Cout - 1) / gn_cg;
+                for (int g = ch0 / gn_cg; g <= g_last; ++g)
+                  gn_out_add(gacc, g, my_g == g ? gs : 0.0f, my_g == g ? gq : 0.0f, lane);
               }
             }
             fence_proxy_async_shared();
@@ -745,6 +945,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const Work wk = decode_work(p, i);
       const Tile& tl = wk.tl;
       const bool piece = wk.slot >= 0;
+      if (p.gn_out != nullptr && tl.n != gacc.n) {
+        gn_out_flush(p.gn_out, p.gn_out_groups, gacc, lane);
+        gacc.n = tl.n;
+      }
       const int row_base = tl.p0 + static_cast<int>(rank) * BM + static_cast<int>(quarter) * 32;
       const bool rows_live = row_base < p.HoWo;   // some of this warp's rows are in the frame
       // channel chunks that hold at least one real output channel
@@ -829,11 +1033,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                            __float_as_uint(v[4 * c + 1]), __float_as_uint(v[4 * c + 2]),
                            __float_as_uint(v[4 * c + 3]));
           } else {
+            uint32_t pk[16];
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              st_shared_v4(ybuf + b * ybytes + swz64(lane, g),
-                           C::pack(v[8 * g + 0], v[8 * g + 1]), C::pack(v[8 * g + 2], v[8 * g + 3]),
-                           C::pack(v[8 * g + 4], v[8 * g + 5]), C::pack(v[8 * g + 6], v[8 * g + 7]));
+            for (int g = 0; g < 16; ++g) pk[g] = C::pack(v[2 * g], v[2 * g + 1]);
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              st_shared_v4(ybuf + b * ybytes + swz64(lane, g), pk[4 * g], pk[4 * g + 1],
+                           pk[4 * g + 2], pk[4 * g + 3]);
+            if (p.gn_out != nullptr) {
+              // this row's rounded outputs, per group of the chunk's channels
+              const bool row_in = row_base + static_cast<int>(lane) < p.HoWo;
+              const int c_end = p.Cout - cb < 32 ? p.Cout - cb : 32;
+              const int g_last = (cb + c_end - 1) / gn_cg;
+              for (int g = cb / gn_cg; g <= g_last; ++g) {
+                const int e_lo = g * gn_cg - cb, e_hi = (g + 1) * gn_cg - cb;
+                float gs = 0.0f, gq = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                  const float yv = (e & 1) ? C::hi(pk[e >> 1]) : C::lo(pk[e >> 1]);
+                  if (row_in && e >= e_lo && e < e_hi && e < c_end) {
+                    gs += yv;
+                    gq = fmaf(yv, yv, gq);
+                  }
+                }
+                gn_out_add(gacc, g, gs, gq, lane);
+              }
             }
           }
           fence_proxy_async_shared();
@@ -867,6 +1091,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mbar_arrive(tempty_bar + 8 * acc);
       }
     }
+    if (p.gn_out != nullptr) gn_out_flush(p.gn_out, p.gn_out_groups, gacc, lane);
     // y stores must be complete (and their shared-memory sources read) before exit
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();

@@ -173,6 +173,20 @@ __global__ void gn_finalize_kernel(double* stats, long long pairs, double count,
   }
 }
 
+}  // namespace conv3d_gn
+
+// {sum, sum of squares} -> {mean, 1/sqrt(var + eps)} in place, for `pairs`
+// statistic entries of `count` values each (used by the convolution that
+// gathers its output's statistics in its epilogue).
+cudaError_t conv3d_gn_finalize(double* stats, long long pairs, double count, double eps,
+                               cudaStream_t stream) {
+  conv3d_gn::gn_finalize_kernel<<<static_cast<unsigned>((pairs + 255) / 256), 256, 0, stream>>>(
+      stats, pairs, count, eps);
+  return cudaGetLastError();
+}
+
+namespace conv3d_gn {
+
 // y = silu((x - mean) * rstd * gamma + beta) (or without the silu).  The grid
 // stride is a multiple of C/8 vectors, so each thread keeps the same 8
 // channels: their gamma/beta are loaded once and the per-channel scale/shift
@@ -218,7 +232,8 @@ __global__ void __launch_bounds__(256, 3) gn_apply_kernel(const uint16_t* x,
         for (int j = 0; j < 8; ++j) {
           const double* st = stats + (set * groups + (c0 + j) / cg) * 2;
           scale[j] = static_cast<float>(st[1]) * (gamma ? to_f<kBF16>(ga[j]) : 1.0f);
-          shift[j] = (beta ? to_f<kBF16>(be[j]) : 0.0f) - static_cast<float>(st[0]) * scale[j];
+          // one fused multiply-add, as in the convolution's own operand transform
+          shift[j] = fmaf(-static_cast<float>(st[0]), scale[j], beta ? to_f<kBF16>(be[j]) : 0.0f);
         }
       }
       uint32_t e[8];
