@@ -72,6 +72,10 @@ def _load():
         lib.oracle_conv3d_backward_f64.argtypes = (
             [u16p, u16p, u16p, ctypes.c_int] + [ctypes.c_int] * 16
             + [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p])
+        lib.oracle_conv3d_backward_cached_f64.restype = ctypes.c_int
+        lib.oracle_conv3d_backward_cached_f64.argtypes = (
+            [u16p, u16p, u16p, u16p, ctypes.c_int] + [ctypes.c_int] * 14
+            + [ctypes.c_void_p] * 4)
         for fn in (lib.oracle_conv3d_dx_at_f64, lib.oracle_conv3d_dw_at_f64):
             fn.restype = ctypes.c_int
             fn.argtypes = ([u16p, u16p, ctypes.c_int] + [ctypes.c_int] * 16
@@ -194,6 +198,37 @@ def conv3d_backward(x_bits, w_bits, dy_bits, dtype, kernel, stride, pad, tpad):
     if rc != 0:
         raise ValueError("oracle rejected the problem")
     return dx, dw, db
+
+
+def conv3d_backward_cached(x_bits, prev_bits, w_bits, dy_bits, dtype, kernel, stride, pad):
+    """fp64 adjoints of :func:`conv3d` in the cached-frames mode (prev_bits the
+    previous chunk's last kt-1 frames [N, kt-1, H, W, Cin]): returns
+    (dx, dprev, dw, dbias)."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    w_bits = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    dy_bits = np.ascontiguousarray(dy_bits, dtype=np.uint16)
+    N, D, H, W, Cin = x_bits.shape
+    Cout = w_bits.shape[0]
+    kt = kernel[0]
+    if prev_bits is not None:
+        prev_bits = np.ascontiguousarray(prev_bits, dtype=np.uint16)
+        if prev_bits.shape != (N, kt - 1, H, W, Cin):
+            raise ValueError("prev shape")
+    Do, Ho, Wo = output_shape(D, H, W, kernel, stride, pad, TPAD_CAUSAL_CACHED)
+    if dy_bits.shape != (N, Do, Ho, Wo, Cout):
+        raise ValueError("dy shape")
+    dx = np.empty(x_bits.shape, dtype=np.float64)
+    dprev = np.zeros((N, kt - 1, H, W, Cin), dtype=np.float64)
+    dw = np.empty(w_bits.shape, dtype=np.float64)
+    db = np.empty((Cout,), dtype=np.float64)
+    rc = _load().oracle_conv3d_backward_cached_f64(
+        x_bits.ctypes.data, None if prev_bits is None else prev_bits.ctypes.data,
+        w_bits.ctypes.data, dy_bits.ctypes.data, dtype, N, Cin, D, H, W, Cout, *kernel, *stride,
+        pad[1], pad[2], dx.ctypes.data, dprev.ctypes.data if kt > 1 else None, dw.ctypes.data,
+        db.ctypes.data)
+    if rc != 0:
+        raise ValueError("oracle rejected the problem")
+    return dx, dprev, dw, db
 
 
 def conv3d_dx_at(w_bits, dy_bits, dtype, x_shape, kernel, stride, pad, tpad, pixels):

@@ -290,6 +290,65 @@ int oracle_conv3d_backward_f64(const uint16_t* x, const uint16_t* w, const uint1
 }
 
 /*
+ * The adjoints of the cached-frames chunk mode (mode 3; Qwen Image post,
+ * "Video VAE": the frames before a chunk are the previous chunk's last kt-1
+ * frames): the same reversed forward loop, in which a tap that reads frame
+ * f < 0 reads prev[n, kt-1+f], so its product sends dy * w to
+ * dprev[n, kt-1+f] and dy * prev[...] to dw.
+ *   dx [N,D,H,W,Cin], dprev [N,kt-1,H,W,Cin], dw [Cout,kt,kh,kw,Cin], dbias [Cout].
+ * Serial loops, fp64, unrounded; any output pointer may be NULL.
+ */
+int oracle_conv3d_backward_cached_f64(const uint16_t* x, const uint16_t* prev, const uint16_t* w,
+                                      const uint16_t* dy, int dtype, int N, int Cin, int D, int H,
+                                      int W, int Cout, int kt, int kh, int kw, int st, int sh,
+                                      int sw, int ph, int pw, double* dx, double* dprev,
+                                      double* dw, double* dbias) {
+  int od[3];
+  if (oracle_output_shape(D, H, W, kt, kh, kw, st, sh, sw, 0, ph, pw, 3, od) != 0) return -1;
+  if (kt > 1 && prev == NULL) return -1;
+  const int Do = od[0], Ho = od[1], Wo = od[2];
+  const int pf = kt - 1;
+  const int P = kt - 1; /* cached frames per sample */
+  if (dx) memset(dx, 0, sizeof(double) * (size_t)N * D * H * W * Cin);
+  if (dprev && P > 0) memset(dprev, 0, sizeof(double) * (size_t)N * P * H * W * Cin);
+  if (dw) memset(dw, 0, sizeof(double) * (size_t)Cout * kt * kh * kw * Cin);
+  if (dbias) memset(dbias, 0, sizeof(double) * (size_t)Cout);
+  for (int n = 0; n < N; ++n)
+    for (int to = 0; to < Do; ++to)
+      for (int ho = 0; ho < Ho; ++ho)
+        for (int wo = 0; wo < Wo; ++wo) {
+          const int64_t m = (((int64_t)n * Do + to) * Ho + ho) * Wo + wo;
+          for (int co = 0; co < Cout; ++co) {
+            const double g = oracle_decode(dy[m * Cout + co], dtype);
+            if (dbias) dbias[co] += g;
+            for (int it = 0; it < kt; ++it) {
+              const int f = to * st + it - pf;
+              if (f >= D) continue;
+              /* the frame read: x[n, f], or the cached prev[n, P + f] */
+              const uint16_t* src = f < 0 ? prev : x;
+              double* dsrc = f < 0 ? dprev : dx;
+              const int64_t frame = f < 0 ? (int64_t)n * P + (P + f) : (int64_t)n * D + f;
+              for (int ih = 0; ih < kh; ++ih) {
+                const int hi = ho * sh + ih - ph;
+                if (hi < 0 || hi >= H) continue;
+                for (int iw = 0; iw < kw; ++iw) {
+                  const int wi = wo * sw + iw - pw;
+                  if (wi < 0 || wi >= W) continue;
+                  const int64_t xo = ((frame * H + hi) * W + wi) * Cin;
+                  const int64_t wo_ = ((((int64_t)co * kt + it) * kh + ih) * kw + iw) * Cin;
+                  for (int ci = 0; ci < Cin; ++ci) {
+                    if (dsrc) dsrc[xo + ci] += g * oracle_decode(w[wo_ + ci], dtype);
+                    if (dw) dw[wo_ + ci] += g * oracle_decode(src[xo + ci], dtype);
+                  }
+                }
+              }
+            }
+          }
+        }
+  return 0;
+}
+
+/*
  * The same two adjoints, evaluated one element at a time for large problems
  * whose full backward the serial loop above cannot finish quickly.  Each
  * element is the plain sum that defines it, over every forward product it

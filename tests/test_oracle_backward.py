@@ -162,3 +162,73 @@ def test_elementwise_adjoints_reject_bad_indices():
                             [1 * 3 * 4 * 4])
     with pytest.raises(ValueError):
         oracle.conv3d_dw_at(xb, gb, BF16, 2, (3, 3, 3), (1, 1, 1), (1, 1, 1), ZERO, [-1])
+
+
+# ---------------------------------------------------------------- cached-frames chunk mode
+
+CACHED = oracle.TPAD_CAUSAL_CACHED
+
+CACHED_CASES = [
+    ((2, 3, 4, 5, 6, 4), (3, 3, 3), (1, 1, 1), (0, 1, 1)),
+    ((1, 4, 3, 4, 4, 3), (3, 3, 3), (2, 2, 2), (0, 1, 1)),
+    ((1, 3, 5, 6, 5, 2), (2, 3, 1), (1, 2, 1), (0, 0, 2)),
+    ((1, 2, 1, 4, 4, 3), (3, 1, 3), (1, 1, 1), (0, 0, 1)),      # a one-frame chunk
+]
+
+
+def cached_problem(N, Cin, D, H, W, Cout, k, stride, pad, seed):
+    fan = Cin * k[0] * k[1] * k[2]
+    xb = si.bits(si.tensor((N, D, H, W, Cin), seed, 0))
+    pb = si.bits(si.tensor((N, k[0] - 1, H, W, Cin), seed, 4))
+    wb = si.bits(si.tensor((Cout, *k, Cin), seed, 1, fan ** -0.5))
+    out = oracle.output_shape(D, H, W, k, stride, pad, CACHED)
+    gb = si.bits(si.tensor((N, *out, Cout), seed, 5))
+    return xb, pb, wb, gb
+
+
+@pytest.mark.parametrize("case", CACHED_CASES)
+def test_cached_backward_is_the_backward_of_the_joined_clip(case):
+    """The chunk convolution is the plain convolution (zero padding, pt = 0) of
+    the clip [prev; x]; its adjoints are those of the joined clip, split at
+    frame kt-1 -- against the separately pinned backward, bit for bit (same
+    products, same order)."""
+    (N, Cin, D, H, W, Cout), k, stride, pad = case
+    xb, pb, wb, gb = cached_problem(N, Cin, D, H, W, Cout, k, stride, pad, seed=13)
+    joined = np.concatenate([pb, xb], axis=1)
+    assert oracle.output_shape(D + k[0] - 1, H, W, k, stride, pad, ZERO) == \
+        oracle.output_shape(D, H, W, k, stride, pad, CACHED)
+    dx, dprev, dw, db = oracle.conv3d_backward_cached(xb, pb, wb, gb, BF16, k, stride, pad)
+    jdx, jdw, jdb = oracle.conv3d_backward(joined, wb, gb, BF16, k, stride, pad, ZERO)
+    np.testing.assert_array_equal(dprev, jdx[:, :k[0] - 1])
+    np.testing.assert_array_equal(dx, jdx[:, k[0] - 1:])
+    np.testing.assert_array_equal(dw, jdw)
+    np.testing.assert_array_equal(db, jdb)
+
+
+@pytest.mark.parametrize("case", CACHED_CASES)
+def test_cached_backward_adjoint_identities(case):
+    (N, Cin, D, H, W, Cout), k, stride, pad = case
+    xb, pb, wb, gb = cached_problem(N, Cin, D, H, W, Cout, k, stride, pad, seed=17)
+    y = oracle.conv3d(xb, wb, None, None, BF16, k, stride, pad, CACHED, prev_bits=pb)
+    dx, dprev, dw, db = oracle.conv3d_backward_cached(xb, pb, wb, gb, BF16, k, stride, pad)
+    g = dec(gb)
+    lhs = float(np.sum(y * g))
+    assert np.isclose(lhs, float(np.sum(dec(xb) * dx) + np.sum(dec(pb) * dprev)),
+                      rtol=1e-12, atol=1e-12)
+    assert np.isclose(lhs, float(np.sum(dec(wb) * dw)), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(db, g.reshape(-1, Cout).sum(axis=0), rtol=1e-12, atol=1e-12)
+
+
+def test_cached_backward_matches_torch_autograd_float64():
+    (N, Cin, D, H, W, Cout), k, stride, pad = CACHED_CASES[0]
+    xb, pb, wb, gb = cached_problem(N, Cin, D, H, W, Cout, k, stride, pad, seed=19)
+    dx, dprev, dw, _ = oracle.conv3d_backward_cached(xb, pb, wb, gb, BF16, k, stride, pad)
+    x = torch.from_numpy(dec(xb)).permute(0, 4, 1, 2, 3).requires_grad_(True)
+    pv = torch.from_numpy(dec(pb)).permute(0, 4, 1, 2, 3).requires_grad_(True)
+    w = torch.from_numpy(dec(wb)).permute(0, 4, 1, 2, 3).requires_grad_(True)
+    y = F.conv3d(torch.cat([pv, x], dim=2), w, stride=stride, padding=(0, pad[1], pad[2]))
+    y.backward(torch.from_numpy(dec(gb)).permute(0, 4, 1, 2, 3))
+    np.testing.assert_allclose(dx, x.grad.permute(0, 2, 3, 4, 1).numpy(), rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(dprev, pv.grad.permute(0, 2, 3, 4, 1).numpy(), rtol=1e-10,
+                               atol=1e-10)
+    np.testing.assert_allclose(dw, w.grad.permute(0, 2, 3, 4, 1).numpy(), rtol=1e-10, atol=1e-10)
