@@ -264,7 +264,7 @@ CONV3D_API conv3d_status_t conv3d_fwd_gn(const void* x, const double* stats, con
  * rules.  workspace: device, 256-byte aligned, conv3d_bwd_data_workspace_bytes()
  * bytes, not overlapping the tensors.  dx must not overlap dy or w.
  * Errors: CONV3D_ERR_UNSUPPORTED for a stride other than 1, the cached-frames
- * rule or pads beyond kernel extent - 1; CONV3D_ERR_WORKSPACE for a missing or
+ * rule (conv3d_bwd_data_cached) or pads beyond kernel extent - 1; CONV3D_ERR_WORKSPACE for a missing or
  * short workspace; otherwise as conv3d_fwd.
  */
 CONV3D_API conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, int Cin,
@@ -292,7 +292,7 @@ CONV3D_API size_t conv3d_bwd_data_workspace_bytes(int N, int Cin, int D, int H, 
  * Strides up to 8, temporal rules zero, causal replicate and causal zero.
  * workspace: device, 256-byte aligned, conv3d_bwd_weight_workspace_bytes()
  * bytes (cleared by the call).  Errors: CONV3D_ERR_UNSUPPORTED for the
- * cached-frames rule, CONV3D_ERR_INVALID_ARG for a null dw or overlapping
+ * cached-frames rule (conv3d_bwd_weight_cached), CONV3D_ERR_INVALID_ARG for a null dw or overlapping
  * buffers, CONV3D_ERR_ALIGNMENT for a dbias not 16-byte aligned,
  * CONV3D_ERR_WORKSPACE for a missing or short workspace; otherwise as conv3d_fwd.
  */
@@ -315,6 +315,40 @@ CONV3D_API size_t conv3d_bwd_weight_workspace_bytes(int Cin, int Cout, const int
  * a native op enqueues into the host framework's command stream rather than
  * committing per call), so device-side errors must be collected separately.
  */
+
+/*
+ * The backward pass of the cached-frames chunk mode (conv3d_fwd_cached): a
+ * decoder trained chunk by chunk needs the gradient of each chunk's cached
+ * frames as well, to pass it back to the chunk before (Qwen Image post,
+ * "Video VAE": the frames before a chunk are the previous chunk's last kt-1
+ * frames; LoRA post: the conv layers are trained on device).  The chunk is the
+ * zero-padded (pt = 0) convolution of the joined clip [prev; x], and these are
+ * its adjoints split at the join.
+ *
+ * conv3d_bwd_data_cached: dx [N, D, H, W, Cin] and dprev [N, kt-1, H, W, Cin]
+ *   (dprev may be NULL: not computed) for dy [N, Do, Ho, Wo, Cout]; two runs of
+ *   the forward kernel over dy with the mirrored, channel-transposed weight.
+ *   Stride 1 and pads <= kernel extent - 1 only (else CONV3D_ERR_UNSUPPORTED).
+ *   workspace: conv3d_bwd_data_workspace_bytes(..., CONV3D_TPAD_CAUSAL_CACHED)
+ *   bytes, 256-byte aligned.  No buffer may overlap another.
+ * conv3d_bwd_weight_cached: dw (and dbias) as conv3d_bwd_weight, with the taps
+ *   that read frames before the chunk reading prev [N, kt-1, H, W, Cin]
+ *   (required when kt > 1).  Strides up to 8; workspace as conv3d_bwd_weight.
+ * Otherwise the rules and errors of conv3d_bwd_data / conv3d_bwd_weight.
+ */
+CONV3D_API conv3d_status_t conv3d_bwd_data_cached(const void* dy, const void* w, void* dx,
+                                                  void* dprev, int N, int Cin, int D, int H,
+                                                  int W, int Cout, const int kernel[3],
+                                                  const int stride[3], const int pad[3],
+                                                  conv3d_dtype_t dtype, void* workspace,
+                                                  size_t ws_bytes, struct CUstream_st* stream);
+CONV3D_API conv3d_status_t conv3d_bwd_weight_cached(const void* x, const void* prev,
+                                                    const void* dy, void* dw, void* dbias, int N,
+                                                    int Cin, int D, int H, int W, int Cout,
+                                                    const int kernel[3], const int stride[3],
+                                                    const int pad[3], conv3d_dtype_t dtype,
+                                                    void* workspace, size_t ws_bytes,
+                                                    struct CUstream_st* stream);
 
 /* Device scratch bytes conv3d_fwd_ws needs for this problem: the folded
  * first-frame weight for CONV3D_TPAD_CAUSAL_REPLICATE with D == 1 and kt > 1,

@@ -30,6 +30,7 @@ __all__ = [
     "groupnorm_stats", "groupnorm_silu", "groupnorm_stats_ptr", "groupnorm_silu_ptr",
     "conv3d_bwd_data", "conv3d_bwd_data_ptr", "bwd_data_workspace_bytes",
     "conv3d_bwd_weight", "conv3d_bwd_weight_ptr", "bwd_weight_workspace_bytes",
+    "conv3d_bwd_data_cached", "conv3d_bwd_weight_cached",
     "Conv3dFunction", "conv3d_autograd",
     "poll_status", "selftest_wait_timeout", "release", "test_arm_stall",
 ]
@@ -89,6 +90,12 @@ _lib.conv3d_bwd_data_workspace_bytes.argtypes = [_c] * 6 + [_i3, _i3, _c]
 _lib.conv3d_bwd_weight.restype = _c
 _lib.conv3d_bwd_weight.argtypes = [_vp] * 4 + [_c] * 6 + [_i3] * 3 + [_c, _c, _vp,
                                                                      ctypes.c_size_t, _vp]
+_lib.conv3d_bwd_data_cached.restype = _c
+_lib.conv3d_bwd_data_cached.argtypes = [_vp] * 4 + [_c] * 6 + [_i3] * 3 + [_c, _vp, ctypes.c_size_t,
+                                                                          _vp]
+_lib.conv3d_bwd_weight_cached.restype = _c
+_lib.conv3d_bwd_weight_cached.argtypes = [_vp] * 5 + [_c] * 6 + [_i3] * 3 + [_c, _vp,
+                                                                            ctypes.c_size_t, _vp]
 _lib.conv3d_bwd_weight_workspace_bytes.restype = ctypes.c_size_t
 _lib.conv3d_bwd_weight_workspace_bytes.argtypes = [_c, _c, _i3]
 _lib.conv3d_fwd_noalloc.restype = _c
@@ -431,6 +438,51 @@ def conv3d_bwd_weight(x: torch.Tensor, dy: torch.Tensor, kernel, stride=(1, 1, 1
                                  H, W, Cout, tuple(kernel), stride, pad, tpad,
                                  _dtype_code(x.dtype), workspace.data_ptr(), workspace.numel(),
                                  _stream_handle(stream)))
+    return dw, db
+
+
+def conv3d_bwd_data_cached(dy: torch.Tensor, w: torch.Tensor, x_shape, pad=(0, 1, 1),
+                           with_prev: bool = True, workspace: torch.Tensor | None = None,
+                           stream=None):
+    """(dx, dprev) for one chunk of the cached-frames mode (stride 1): dprev is
+    the gradient of the kt-1 cached frames (None when with_prev is false)."""
+    N, D, H, W, Cin = x_shape
+    Cout, kt, kh, kw, _ = w.shape
+    dx = torch.empty(tuple(x_shape), dtype=dy.dtype, device=dy.device)
+    dprev = (torch.empty((N, kt - 1, H, W, Cin), dtype=dy.dtype, device=dy.device)
+             if with_prev and kt > 1 else None)
+    need = bwd_data_workspace_bytes(N, Cin, D, H, W, Cout, (kt, kh, kw), pad, TPAD_CAUSAL_CACHED)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dy.device)
+    for name, t in (("dy", dy), ("w", w)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != dy.dtype:
+            raise ValueError(f"{name} must be a contiguous CUDA tensor of dy's dtype")
+    _check(_lib.conv3d_bwd_data_cached(dy.data_ptr(), w.data_ptr(), dx.data_ptr(), _ptr(dprev), N,
+                                       Cin, D, H, W, Cout, _i3(kt, kh, kw), _i3(1, 1, 1),
+                                       _i3(*pad), _dtype_code(dy.dtype), workspace.data_ptr(),
+                                       workspace.numel(), _stream_handle(stream)))
+    return dx, dprev
+
+
+def conv3d_bwd_weight_cached(x: torch.Tensor, prev: torch.Tensor | None, dy: torch.Tensor, kernel,
+                             stride=(1, 1, 1), pad=(0, 1, 1), with_bias: bool = True,
+                             workspace: torch.Tensor | None = None, stream=None):
+    """(dw, dbias) for one chunk of the cached-frames mode; prev: the cached frames."""
+    N, D, H, W, Cin = x.shape
+    Cout = dy.shape[-1]
+    dw = torch.empty((Cout, *kernel, Cin), dtype=x.dtype, device=x.device)
+    db = torch.empty((Cout,), dtype=x.dtype, device=x.device) if with_bias else None
+    need = bwd_weight_workspace_bytes(Cin, Cout, kernel)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    for name, t in (("x", x), ("dy", dy), ("prev", prev)):
+        if t is not None and (not t.is_cuda or not t.is_contiguous() or t.dtype != x.dtype):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor of x's dtype")
+    _check(_lib.conv3d_bwd_weight_cached(x.data_ptr(), _ptr(prev), dy.data_ptr(), dw.data_ptr(),
+                                         _ptr(db), N, Cin, D, H, W, Cout, _i3(*kernel),
+                                         _i3(*stride), _i3(*pad), _dtype_code(x.dtype),
+                                         workspace.data_ptr(), workspace.numel(),
+                                         _stream_handle(stream)))
     return dw, db
 
 

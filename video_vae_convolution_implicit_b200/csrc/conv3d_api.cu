@@ -990,7 +990,7 @@ conv3d_status_t plan_bwd_data(const void* dy, const void* w, const void* dx, int
                               const int pad[3], conv3d_tpad_t tpad, conv3d_dtype_t dtype,
                               BwdDataPlan& B) {
   if (tpad == CONV3D_TPAD_CAUSAL_CACHED) {
-    set_error("the backward pass of the cached-frames mode is not supported");
+    set_error("the cached-frames rule needs the cached frames: conv3d_bwd_data_cached");
     return CONV3D_ERR_UNSUPPORTED;
   }
   // validate as the forward problem x -> y (x = dx, y = dy)
@@ -1393,18 +1393,19 @@ size_t conv3d_bwd_weight_workspace_bytes(int Cin, int Cout, const int kernel[3])
   return ((dw + 255) & ~size_t(255)) + ((static_cast<size_t>(Cout) * 4 + 255) & ~size_t(255));
 }
 
-conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void* dbias, int N,
-                                  int Cin, int D, int H, int W, int Cout, const int kernel[3],
-                                  const int stride[3], const int pad[3], conv3d_tpad_t tpad,
-                                  conv3d_dtype_t dtype, void* workspace, size_t ws_bytes,
-                                  struct CUstream_st* stream) {
-  if (tpad == CONV3D_TPAD_CAUSAL_CACHED) {
-    set_error("the backward pass of the cached-frames mode is not supported");
-    return CONV3D_ERR_UNSUPPORTED;
-  }
+}  // extern "C"
+
+namespace {
+
+// dw (+ dbias) for every temporal rule; prev: the cached frames (cached mode).
+conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy, void* dw,
+                                void* dbias, int N, int Cin, int D, int H, int W, int Cout,
+                                const int kernel[3], const int stride[3], const int pad[3],
+                                conv3d_tpad_t tpad, conv3d_dtype_t dtype, void* workspace,
+                                size_t ws_bytes, cudaStream_t stream) {
   Problem F;
   conv3d_status_t st = validate(x, dw ? dw : workspace, nullptr, nullptr, dy, N, Cin, D, H, W,
-                                Cout, kernel, stride, pad, tpad, dtype, F);
+                                Cout, kernel, stride, pad, tpad, dtype, F, prev);
   if (st != CONV3D_OK) return st;
   if (!dw) {
     set_error("dw must be non-null");
@@ -1427,10 +1428,12 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   const size_t dw_elems = static_cast<size_t>(Cout) * taps * Cin;
   const size_t x_bytes = static_cast<size_t>(N) * D * H * W * Cin * 2;
   const size_t dy_bytes = static_cast<size_t>(N) * F.Do * F.Ho * F.Wo * Cout * 2;
+  const size_t p_bytes = prev ? static_cast<size_t>(N) * (kernel[0] - 1) * H * W * Cin * 2 : 0;
   if (overlaps(workspace, need, x, x_bytes) || overlaps(workspace, need, dy, dy_bytes) ||
       overlaps(workspace, need, dw, dw_elems * 2) || overlaps(dw, dw_elems * 2, x, x_bytes) ||
-      overlaps(dw, dw_elems * 2, dy, dy_bytes)) {
-    set_error("x, dy, dw and the workspace must not overlap");
+      overlaps(dw, dw_elems * 2, dy, dy_bytes) || overlaps(workspace, need, prev, p_bytes) ||
+      overlaps(dw, dw_elems * 2, prev, p_bytes)) {
+    set_error("x, prev, dy, dw and the workspace must not overlap");
     return CONV3D_ERR_INVALID_ARG;
   }
   if ((st = load_entry_points()) != CONV3D_OK) return st;
@@ -1559,10 +1562,18 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
   wp.test_stall = take_stall(wp.timeout_ns) ? 1 : 0;
   const size_t smem = static_cast<size_t>(stages) * stage_bytes + reserve;
 
-  // x through the forward im2col map (pix pixels per load); dy as [frames][pixels][Cout]
-  CUtensorMap map_x, map_dy;
+  // x through the forward im2col map (pix pixels per load), the cached frames
+  // through a second one; dy as [frames][pixels][Cout]
+  CUtensorMap map_x, map_dy, map_p;
   if ((st = encode_im2col(F, x, static_cast<long long>(N) * D, pix, map_x)) != CONV3D_OK)
     return st;
+  if (tpad == CONV3D_TPAD_CAUSAL_CACHED && kernel[0] > 1) {
+    if ((st = encode_im2col(F, prev, static_cast<long long>(N) * (kernel[0] - 1), pix, map_p)) !=
+        CONV3D_OK)
+      return st;
+  } else {
+    map_p = map_x;   // never read
+  }
   {
     const CUtensorMapDataType dt =
         bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -1604,7 +1615,7 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
               swap ? "transposed" : pair ? "CTA pair" : "plain", bf16 ? "bf16" : "fp16",
               wp.num_units, wp.splits, wp.total_chunks, pix, static_cast<int>(cfg.gridDim.x),
               wp.stages, smem);
-    e = cudaLaunchKernelEx(&cfg, kern, map_x, map_dy, wp);
+    e = cudaLaunchKernelEx(&cfg, kern, map_x, map_dy, map_p, wp);
     if (e != cudaSuccess) return cuda_fail(e, "wgrad kernel launch");
   }
   {
@@ -1647,6 +1658,118 @@ conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void*
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dbias conversion launch");
   }
   return CONV3D_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+conv3d_status_t conv3d_bwd_weight(const void* x, const void* dy, void* dw, void* dbias, int N,
+                                  int Cin, int D, int H, int W, int Cout, const int kernel[3],
+                                  const int stride[3], const int pad[3], conv3d_tpad_t tpad,
+                                  conv3d_dtype_t dtype, void* workspace, size_t ws_bytes,
+                                  struct CUstream_st* stream) {
+  if (tpad == CONV3D_TPAD_CAUSAL_CACHED) {
+    set_error("the cached-frames rule needs the cached frames: conv3d_bwd_weight_cached");
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  return bwd_weight_impl(x, nullptr, dy, dw, dbias, N, Cin, D, H, W, Cout, kernel, stride, pad,
+                         tpad, dtype, workspace, ws_bytes, stream);
+}
+
+conv3d_status_t conv3d_bwd_weight_cached(const void* x, const void* prev, const void* dy, void* dw,
+                                         void* dbias, int N, int Cin, int D, int H, int W,
+                                         int Cout, const int kernel[3], const int stride[3],
+                                         const int pad[3], conv3d_dtype_t dtype, void* workspace,
+                                         size_t ws_bytes, struct CUstream_st* stream) {
+  return bwd_weight_impl(x, prev, dy, dw, dbias, N, Cin, D, H, W, Cout, kernel, stride, pad,
+                         CONV3D_TPAD_CAUSAL_CACHED, dtype, workspace, ws_bytes, stream);
+}
+
+conv3d_status_t conv3d_bwd_data_cached(const void* dy, const void* w, void* dx, void* dprev, int N,
+                                       int Cin, int D, int H, int W, int Cout, const int kernel[3],
+                                       const int stride[3], const int pad[3], conv3d_dtype_t dtype,
+                                       void* workspace, size_t ws_bytes,
+                                       struct CUstream_st* stream) {
+  // validate as the forward chunk problem x -> y (x = dx, prev = dprev, y = dy)
+  Problem F;
+  conv3d_status_t st = validate(dx, w, nullptr, nullptr, dy, N, Cin, D, H, W, Cout, kernel, stride,
+                                pad, CONV3D_TPAD_CAUSAL_CACHED, dtype, F, dprev ? dprev : dx);
+  if (st != CONV3D_OK) return st;
+  if (stride[0] != 1 || stride[1] != 1 || stride[2] != 1) {
+    set_error("the backward data pass supports stride (1,1,1) only");
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  if (F.ph > F.kh - 1 || F.pw > F.kw - 1) {
+    set_error("the backward data pass needs pads <= kernel extent - 1");
+    return CONV3D_ERR_UNSUPPORTED;
+  }
+  const size_t need = (static_cast<size_t>(Cout) * F.kt * F.kh * F.kw * Cin * 2 + 255) & ~size_t(255);
+  if (workspace == nullptr || ws_bytes < need) {
+    set_error("workspace of %zu bytes required", need);
+    return CONV3D_ERR_WORKSPACE;
+  }
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) {
+    set_error("workspace must be 256-byte aligned");
+    return CONV3D_ERR_ALIGNMENT;
+  }
+  const size_t dx_bytes = static_cast<size_t>(N) * D * H * W * Cin * 2;
+  const size_t dp_bytes = static_cast<size_t>(N) * (F.kt - 1) * H * W * Cin * 2;
+  const size_t dy_bytes = static_cast<size_t>(N) * F.Do * F.Ho * F.Wo * Cout * 2;
+  const size_t w_bytes = static_cast<size_t>(Cout) * F.kt * F.kh * F.kw * Cin * 2;
+  if (overlaps(workspace, need, dx, dx_bytes) || overlaps(workspace, need, dy, dy_bytes) ||
+      overlaps(workspace, need, w, w_bytes) || overlaps(dx, dx_bytes, dy, dy_bytes) ||
+      overlaps(workspace, need, dprev, dp_bytes) || overlaps(dprev, dp_bytes, dy, dy_bytes) ||
+      overlaps(dprev, dp_bytes, dx, dx_bytes) || overlaps(dprev, dp_bytes, w, w_bytes)) {
+    set_error("dx, dprev, dy, w and the workspace must not overlap");
+    return CONV3D_ERR_INVALID_ARG;
+  }
+  if ((st = load_entry_points()) != CONV3D_OK) return st;
+  DeviceState* S = nullptr;
+  int dev = 0;
+  if ((st = device_state(S, dev)) != CONV3D_OK) return st;
+  uint16_t* wt = static_cast<uint16_t*>(workspace);
+  {
+    const int taps = kernel[0] * kernel[1] * kernel[2];
+    const dim3 grid((Cin + 31) / 32, (Cout + 31) / 32, taps);
+    flip_transpose_weight_kernel<<<grid, dim3(32, 8), 0, stream>>>(
+        static_cast<const uint16_t*>(w), wt, Cout, taps, Cin);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
+  }
+  // The chunk is the zero-padded (pt = 0) convolution of the joined clip
+  // [prev; x], whose data gradient is the transposed convolution of dy: joined
+  // frame e gathers dy[e + it - (kt-1)] through the mirrored weight.  Frames
+  // kt-1.. of the joined clip are dx (dy frames to .. to+kt-1, pf = 0), frames
+  // 0..kt-2 are dprev (pf = kt-1); one launch each, all samples at once.
+  Problem T{};
+  T.N = N;
+  T.Cin = Cout;
+  T.D = F.Do;
+  T.H = F.Ho;
+  T.W = F.Wo;
+  T.Cout = Cin;
+  T.kt = F.kt; T.kh = F.kh; T.kw = F.kw;
+  T.st = T.sh = T.sw = 1;
+  T.ph = F.kh - 1 - F.ph;
+  T.pw = F.kw - 1 - F.pw;
+  T.Ho = H;
+  T.Wo = W;
+  T.tpad = CONV3D_TPAD_ZERO;   // dy frames outside [0, Do) contribute nothing
+  T.dtype = dtype;
+  Problem Tx = T;
+  Tx.pf = 0;
+  Tx.pb = F.kt - 1;
+  Tx.Do = D;
+  st = launch_main(*S, Tx, dy, nullptr, wt, nullptr, nullptr, dx, stream);
+  if (st == CONV3D_OK && dprev && F.kt > 1) {
+    Problem Tp = T;
+    Tp.pf = F.kt - 1;
+    Tp.pb = 0;
+    Tp.Do = F.kt - 1;
+    st = launch_main(*S, Tp, dy, nullptr, wt, nullptr, nullptr, dprev, stream);
+  }
+  return st;
 }
 
 size_t conv3d_workspace_bytes(int Cin, int Cout, const int kernel[3], int D, conv3d_tpad_t tpad) {

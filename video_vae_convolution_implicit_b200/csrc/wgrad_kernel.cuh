@@ -50,7 +50,7 @@ struct WgradParams {
   int kt, kh, kw;
   int st, sh, sw;
   int pf, ph, pw;
-  int tpad;                 // 0 zero, 1 causal replicate, 2 causal zero
+  int tpad;                 // 0 zero, 1 causal replicate, 2 causal zero, 3 cached frames
   int taps;
   int cblocks;              // ceil(Cin / 128)                  (plain variant)
   int BN;                   // output channels per unit: multiple of 64, <= 256 (plain), 128 (swap)
@@ -89,10 +89,13 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t 
   return d;
 }
 
+// Frame read by temporal tap `it` of output frame `to`: a frame of x (>= 0), a
+// cached frame of the previous chunk (-(kt-1) .. -1, cached mode), or kNoFrame
+// when the tap reads zero padding.
 __device__ __forceinline__ int wg_source_frame(const WgradParams& p, int to, int it) {
   const int f = to * p.st + it - p.pf;
-  if (f < 0) return p.tpad == 1 ? 0 : -1;
-  return f < p.D ? f : -1;
+  if (f < 0) return p.tpad == 1 ? 0 : (p.tpad == 3 ? f : kNoFrame);
+  return f < p.D ? f : kNoFrame;
 }
 
 struct WgUnit {
@@ -194,7 +197,8 @@ __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c
 template <bool kBF16, bool kSwap, bool kPair, int kPix>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     conv3d_wgrad_kernel(const __grid_constant__ CUtensorMap map_x,
-                        const __grid_constant__ CUtensorMap map_dy, const WgradParams p) {
+                        const __grid_constant__ CUtensorMap map_dy,
+                        const __grid_constant__ CUtensorMap map_p, const WgradParams p) {
   static_assert(!(kSwap && kPair), "the pair variant is the plain operand assignment");
   static_assert(kPix % 16 == 0 && kPix <= 256, "pixels per stage");
   constexpr uint32_t kBox = kPix * 128;          // one 64-channel box
@@ -245,6 +249,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fence_mbar_init();
     prefetch_tensormap(&map_x);
     prefetch_tensormap(&map_dy);
+    if (p.tpad == 3) prefetch_tensormap(&map_p);
   }
   if (warp == 1) {
     if constexpr (kPair) {
@@ -310,8 +315,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         FrameWalk fw(p, wu);
         while (ok && fw.next(p)) {
           const int f = wg_source_frame(p, fw.to, wu.it);
-          if (f < 0) continue;                  // this tap reads zero padding here
-          const int img = fw.n * p.D + f;
+          if (f == kNoFrame) continue;          // this tap reads zero padding here
+          // frames before the chunk come from the cached-frames tensor
+          const CUtensorMap* xmap = f < 0 ? &map_p : &map_x;
+          const int img = f < 0 ? fw.n * (p.kt - 1) + (p.kt - 1) + f : fw.n * p.D + f;
           int p0 = fw.pc * kPix;
           int ho0 = p0 / p.Wo;
           int wo0 = p0 - ho0 * p.Wo;
@@ -333,7 +340,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const uint32_t fb0 = mapa_shared(fb, 0);
 #pragma unroll
               for (int q = 0; q < 2; ++q)
-                tma_load_im2col_4d_pair(x_dst + q * kBox, &map_x, fb0, bc[q], wx, hx,
+                tma_load_im2col_4d_pair(x_dst + q * kBox, xmap, fb0, bc[q], wx, hx,
                                         img, static_cast<uint16_t>(bw[q]),
                                         static_cast<uint16_t>(bh[q]));
               for (int q = 0; q < ndy; ++q) {
@@ -346,7 +353,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int q = 0; q < 4; ++q)
                 if (q < nx)
-                  tma_load_im2col_4d(x_dst + q * kBox, &map_x, fb, bc[q], wx, hx, img,
+                  tma_load_im2col_4d(x_dst + q * kBox, xmap, fb, bc[q], wx, hx, img,
                                      static_cast<uint16_t>(bw[q]), static_cast<uint16_t>(bh[q]));
               for (int q = 0; q < ndy; ++q) {
                 const int dc = dy_c0 + 64 * q < p.Cout ? dy_c0 + 64 * q : wu.co0;
@@ -395,7 +402,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t accumulate = 0;
         FrameWalk fw(p, wu);
         while (ok && fw.next(p)) {
-          if (wg_source_frame(p, fw.to, wu.it) < 0) continue;
+          if (wg_source_frame(p, fw.to, wu.it) == kNoFrame) continue;
           for (int j = 0; j < fw.count; ++j) {
             if (!wait_bounded(full_bar + 8 * stage, phase, ctl, true)) {
               ok = false;
@@ -459,7 +466,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // a unit whose chunks all read zero padding issued no MMA: nothing to add
       bool any = false;
       FrameWalk fw(p, wu);
-      while (!any && fw.next(p)) any = wg_source_frame(p, fw.to, wu.it) >= 0;
+      while (!any && fw.next(p)) any = wg_source_frame(p, fw.to, wu.it) != kNoFrame;
       const uint32_t t_row =
           tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.acc_cols);
       if (kSwap) {
