@@ -547,6 +547,14 @@ conv3d_status_t encode_out_map(const Problem& P, const void* base, CUtensorMap& 
 
 // ------------------------------------------------------------------ launch
 
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* env = getenv("CONV3D_PDL");
+    return env == nullptr || env[0] != '0';
+  }();
+  return on;
+}
+
 uint32_t pow2_at_least(uint32_t v) {
   uint32_t p = 32;
   while (p < v) p <<= 1;
@@ -751,17 +759,29 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
   }
   const int unit_count = L.kp.num_items < units ? L.kp.num_items : units;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kPair ? 2 : 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  int n_attr = 0;
+  if (kPair) {
+    attr[n_attr].id = cudaLaunchAttributeClusterDimension;
+    attr[n_attr].val.clusterDim.x = 2;
+    attr[n_attr].val.clusterDim.y = 1;
+    attr[n_attr].val.clusterDim.z = 1;
+    ++n_attr;
+  }
+  // A programmatic dependent of the previous kernel on the stream: the
+  // kernel's set-up overlaps that kernel's end (it waits for it before
+  // touching global memory).  CONV3D_PDL=0 turns this off.
+  if (pdl_enabled()) {
+    attr[n_attr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n_attr].val.programmaticStreamSerializationAllowed = 1;
+    ++n_attr;
+  }
   cfg.gridDim = dim3((kPair ? 2 : 1) * unit_count, 1, 1);
   cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = L.smem;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = kPair ? 1 : 0;
+  cfg.numAttrs = n_attr;
   if (plan_log())
     fprintf(stderr,
             "libconv3d: implicit GEMM %s%s %s, %d tiles of %d pixels x %d channels, grid %d, "

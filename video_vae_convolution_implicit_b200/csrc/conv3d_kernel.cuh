@@ -536,6 +536,10 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
   if constexpr (kPair) cluster_sync();   // the peer's barriers are initialised
   tc_fence_after();
   const uint32_t tmem_base = s_tmem_base;
+  // Launched as a programmatic dependent of the previous kernel on the stream
+  // (which may still be running): everything above touched only this CTA's
+  // own resources; no global memory is read or written before this point.
+  griddep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -1124,6 +1128,8 @@ template <bool kBF16>
 __global__ void fold_temporal_taps_kernel(const uint16_t* __restrict__ w, uint16_t* __restrict__ w2,
                                           int Cout, int kt, int spatial_cin) {
   using C = Cvt<kBF16>;
+  // the convolution that reads w2 waits for this whole grid before reading
+  griddep_launch_dependents();
   const long long total = static_cast<long long>(Cout) * spatial_cin;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
