@@ -31,7 +31,7 @@ static int failures = 0;
   } while (0)
 
 static int cpu_checks(void) {
-  const int k3[3] = {3, 3, 3}, s1[3] = {1, 1, 1}, s2[3] = {1, 2, 2};
+  const int k3[3] = {3, 3, 3}, s1[3] = {1, 1, 1}, s2[3] = {1, 2, 2}, st2[3] = {2, 2, 2};
   const int p_causal[3] = {0, 1, 1}, p_zero[3] = {1, 1, 1};
   int out[3];
   CHECK(conv3d_output_shape(9, 128, 128, k3, s1, p_causal, CONV3D_TPAD_CAUSAL_REPLICATE, out) ==
@@ -67,7 +67,7 @@ static int cpu_checks(void) {
         (size_t)64 * 27 * 64 * 4 + (size_t)64 * 4);
   CHECK(conv3d_bwd_data_workspace_bytes(1, 64, 4, 8, 8, 64, k3, p_zero, CONV3D_TPAD_ZERO) ==
         (size_t)64 * 27 * 64 * 2);
-  CHECK(conv3d_bwd_data(y, w, dx, 1, 64, 4, 8, 8, 64, k3, s2, p_causal,
+  CHECK(conv3d_bwd_data(y, w, dx, 1, 64, 4, 8, 8, 64, k3, st2, p_causal,
                         CONV3D_TPAD_CAUSAL_REPLICATE, CONV3D_BF16, ws, (size_t)1 << 30,
                         NULL) == CONV3D_ERR_UNSUPPORTED);          /* stride 2 */
   CHECK(conv3d_bwd_data(y, w, dx, 1, 64, 4, 8, 8, 64, k3, s1, p_causal,

@@ -252,9 +252,10 @@ def test_bwd_workspace_bytes():
 
 
 @pytest.mark.parametrize("kw,expect", [
-    (dict(stride=(1, 2, 2)), Status.UNSUPPORTED),
+    (dict(stride=(2, 1, 1)), Status.UNSUPPORTED),          # temporal stride
+    (dict(stride=(2, 2, 2)), Status.UNSUPPORTED),
     (dict(tpad=c3.TPAD_CAUSAL_CACHED), Status.UNSUPPORTED),
-    (dict(pad=(0, 3, 1)), Status.UNSUPPORTED),             # pad > kernel extent - 1
+    (dict(pad=(0, 3, 1)), Status.UNSUPPORTED),             # pad > kernel extent - 1 at stride 1
     (dict(workspace=None), Status.WORKSPACE),
     (dict(ws_bytes=64), Status.WORKSPACE),
     (dict(workspace=WS + 16), Status.ALIGNMENT),

@@ -61,10 +61,10 @@ def test_bwd_data_every_element(case, variant):
 
 def test_bwd_data_rejects_strides_and_cached_mode():
     x, w, dy, _ = grads_problem(1, 64, 4, 8, 8, 64, (3, 3, 3), (0, 1, 1), CREP, 1, "bf16",
-                                stride=(1, 2, 2))
+                                stride=(2, 2, 2))
     ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
     st = c3.conv3d_bwd_data_ptr(dy.data_ptr(), w.data_ptr(), x.data_ptr(), 1, 64, 4, 8, 8, 64,
-                                (3, 3, 3), (1, 2, 2), (0, 1, 1), CREP, c3.BF16, ws.data_ptr(),
+                                (3, 3, 3), (2, 2, 2), (0, 1, 1), CREP, c3.BF16, ws.data_ptr(),
                                 ws.numel(), 0)
     assert st == c3.Status.UNSUPPORTED
 
@@ -207,3 +207,48 @@ def test_autograd_function_matches_the_oracle(tpad):
     assert_close(leaves[1].grad.double().cpu().numpy(), rdw, "dw")
     assert_close(leaves[2].grad.double().cpu().numpy(), rdb, "dbias")
     assert torch.equal(leaves[3].grad, dy)
+
+
+STRIDED_DATA_CASES = [
+    # N, Cin, D, H, W, Cout, kernel, stride, pad, tpad, dtype
+    (1, 64, 3, 16, 16, 64, (3, 3, 3), (1, 2, 2), (0, 1, 1), CREP, "bf16"),   # the downsampling layer
+    (2, 64, 3, 15, 17, 128, (3, 3, 3), (1, 2, 2), (0, 1, 1), CZERO, "bf16"), # odd sizes, 2 samples
+    (1, 32, 4, 13, 11, 48, (3, 3, 3), (1, 3, 2), (1, 1, 0), ZERO, "f16"),
+    (1, 64, 2, 9, 10, 64, (1, 1, 1), (1, 2, 2), (0, 0, 0), ZERO, "bf16"),    # phases without taps
+    (1, 64, 1, 12, 12, 64, (3, 3, 3), (1, 2, 2), (0, 1, 1), CREP, "bf16"),   # single frame: fold
+    (3, 64, 3, 8, 10, 64, (3, 3, 3), (1, 2, 2), (0, 1, 1), CREP, "bf16"),    # body launch per sample
+    (1, 48, 3, 12, 14, 40, (2, 3, 3), (1, 2, 2), (0, 2, 2), CREP, "bf16"),   # pads > kernel - 1
+    (1, 64, 2, 10, 9, 64, (3, 3, 3), (1, 1, 2), (0, 1, 1), CZERO, "bf16"),   # one axis strided
+]
+
+
+@pytest.mark.parametrize("case", STRIDED_DATA_CASES, ids=lambda c: "x".join(map(str, c[:6])) + f"-s{''.join(map(str, c[7]))}-t{c[9]}-{c[10]}")
+def test_bwd_data_strided_every_element(case, variant):
+    N, Cin, D, H, W, Cout, k, stride, pad, tpad, dt = case
+    x, w, dy, od = grads_problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=700 + Cin, dt=dt,
+                                 stride=stride)
+    dx = torch.full(x.shape, float("nan"), dtype=x.dtype, device="cuda")
+    dx = c3.conv3d_bwd_data(dy, w, x.shape, pad, tpad, dx=dx, stride=stride)
+    assert c3.poll_status() == c3.Status.OK
+    ref, _, _ = oracle.conv3d_backward(si.bits(x), si.bits(w), si.bits(dy), od, k, stride, pad,
+                                       tpad)
+    assert_close(dx.double().cpu().numpy(), ref, str(case))
+
+
+def test_bwd_data_strided_downsampling_layer_sampled():
+    # the 256-channel downsampling workload: 9 frames 256x256 -> 128x128, stride (1, 2, 2)
+    from seeded_inputs.workloads import WORKLOADS
+    wl = WORKLOADS["cfg2s"]
+    x, w, dy, od = grads_problem(wl.N, wl.Cin, wl.D, wl.H, wl.W, wl.Cout, wl.kernel, wl.pad,
+                                 wl.tpad, seed=wl.seed, dt=wl.dtype, stride=wl.stride)
+    dx = c3.conv3d_bwd_data(dy, w, x.shape, wl.pad, wl.tpad, stride=wl.stride)
+    assert c3.poll_status() == c3.Status.OK
+    HW = wl.H * wl.W
+    pix = sorted({0, 1, wl.W - 1, wl.W, wl.W + 1, HW - 1, HW, 2 * HW + 257, (wl.D - 1) * HW,
+                  wl.D * HW - 1} | set(range(5 * HW, 5 * HW + 40)))
+    import numpy as np
+    pixels = np.array(pix, dtype=np.int64)
+    ref = oracle.conv3d_dx_at(si.bits(w), si.bits(dy), od, x.shape, wl.kernel, wl.stride, wl.pad,
+                              wl.tpad, pixels)
+    got = dx.view(-1, wl.Cin)[torch.from_numpy(pixels).cuda()].double().cpu().numpy()
+    assert_close(got, ref, "cfg2s dx sampled")

@@ -390,8 +390,10 @@ def bwd_data_workspace_bytes(N, Cin, D, H, W, Cout, kernel, pad, tpad) -> int:
 
 def conv3d_bwd_data(dy: torch.Tensor, w: torch.Tensor, x_shape, pad=(0, 1, 1),
                     tpad=TPAD_CAUSAL_REPLICATE, dx: torch.Tensor | None = None,
-                    workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """dx for the forward problem x [x_shape] -> y (dy has y's shape), stride 1."""
+                    workspace: torch.Tensor | None = None, stream=None,
+                    stride=(1, 1, 1)) -> torch.Tensor:
+    """dx for the forward problem x [x_shape] -> y (dy has y's shape); temporal
+    stride 1, spatial strides up to 8."""
     N, D, H, W, Cin = x_shape
     Cout, kt, kh, kw, _ = w.shape
     if dx is None:
@@ -403,7 +405,7 @@ def conv3d_bwd_data(dy: torch.Tensor, w: torch.Tensor, x_shape, pad=(0, 1, 1),
         if not t.is_cuda or not t.is_contiguous() or t.dtype != dy.dtype:
             raise ValueError(f"{name} must be a contiguous CUDA tensor of dy's dtype")
     _check(conv3d_bwd_data_ptr(dy.data_ptr(), w.data_ptr(), dx.data_ptr(), N, Cin, D, H, W, Cout,
-                               (kt, kh, kw), (1, 1, 1), pad, tpad, _dtype_code(dy.dtype),
+                               (kt, kh, kw), tuple(stride), pad, tpad, _dtype_code(dy.dtype),
                                workspace.data_ptr(), workspace.numel(), _stream_handle(stream)))
     return dx
 
@@ -488,7 +490,7 @@ def conv3d_bwd_weight_cached(x: torch.Tensor, prev: torch.Tensor | None, dy: tor
 
 class Conv3dFunction(torch.autograd.Function):
     """torch.autograd wrapper: forward through conv3d_fwd, backward through
-    conv3d_bwd_data (dx; stride 1 only) and conv3d_bwd_weight (dw, dbias).
+    conv3d_bwd_data (dx; temporal stride 1) and conv3d_bwd_weight (dw, dbias).
     The residual's gradient is dy itself.  Marshalling only: every product runs
     in the library's kernels, none in torch."""
 
@@ -506,9 +508,9 @@ class Conv3dFunction(torch.autograd.Function):
         dy = dy.contiguous()
         dx = dw = db = dres = None
         if ctx.needs_input_grad[0]:
-            if stride != (1, 1, 1):
-                raise NotImplementedError("the input gradient supports stride (1, 1, 1) only")
-            dx = conv3d_bwd_data(dy, w, x.shape, pad, tpad)
+            if stride[0] != 1:
+                raise NotImplementedError("the input gradient supports temporal stride 1 only")
+            dx = conv3d_bwd_data(dy, w, x.shape, pad, tpad, stride=stride)
         if ctx.needs_input_grad[1] or (has_bias and ctx.needs_input_grad[2]):
             dw, db = conv3d_bwd_weight(x, dy, tuple(w.shape[1:4]), stride, pad, tpad,
                                        with_bias=has_bias)

@@ -95,6 +95,12 @@ struct Problem {
   int gn_groups, gn_per_frame, gn_silu;
   double* gn_out;      // sums of y's GroupNorm statistics (per sample), or null
   int gn_out_groups;
+  // data-gradient phases of a strided convolution: the im2col window box is
+  // sized for exactly Ho x Wo outputs (front pads ph, pw; stride 1), and the
+  // outputs go to strided positions of y_scatter (see KernelParams)
+  bool exact_out;
+  uint16_t* y_scatter;
+  int sc_sh, sc_sw, sc_rh, sc_rw, sc_H, sc_W;
 };
 
 bool output_extents(int D, int H, int W, const int k[3], const int stride[3], const int pad[3],
@@ -230,6 +236,11 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
   P.gn_groups = P.gn_per_frame = P.gn_silu = 0;
   P.gn_out = nullptr;
   P.gn_out_groups = 0;
+  P.exact_out = false;
+  P.y_scatter = nullptr;
+  P.sc_sh = P.sc_sw = 1;
+  P.sc_rh = P.sc_rw = 0;
+  P.sc_H = P.sc_W = 0;
   return CONV3D_OK;
 }
 
@@ -467,9 +478,11 @@ conv3d_status_t encode_im2col(const Problem& P, const void* base, long long imag
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(P.Cin) * 2,
                                  static_cast<cuuint64_t>(P.W) * P.Cin * 2,
                                  static_cast<cuuint64_t>(P.H) * P.W * P.Cin * 2};
-  // Window-origin box: first origin at -pad, last at dim-1+pad-(k-1).
+  // Window-origin box: first origin at -pad, last at dim-1+pad-(k-1) (or, for
+  // a data-gradient phase, the origin of the last of exactly Wo, Ho outputs).
   const int lower[2] = {-P.pw, -P.ph};
-  const int upper[2] = {P.pw - (P.kw - 1), P.ph - (P.kh - 1)};
+  const int upper[2] = {P.exact_out ? P.Wo - P.W - P.pw : P.pw - (P.kw - 1),
+                        P.exact_out ? P.Ho - P.H - P.ph : P.ph - (P.kh - 1)};
   // traversal strides: consecutive output pixels' window origins are sw
   // columns (sh rows at a row wrap) apart
   const cuuint32_t estr[4] = {1, static_cast<cuuint32_t>(P.sw), static_cast<cuuint32_t>(P.sh), 1};
@@ -619,6 +632,13 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, b
   kp.gn_silu = P.gn_silu;
   kp.gn_out = P.gn_out;
   kp.gn_out_groups = P.gn_out_groups;
+  kp.y_scatter = P.y_scatter;
+  kp.sc_sh = P.sc_sh;
+  kp.sc_sw = P.sc_sw;
+  kp.sc_rh = P.sc_rh;
+  kp.sc_rw = P.sc_rw;
+  kp.sc_H = P.sc_H;
+  kp.sc_W = P.sc_W;
   kp.n_chunks = (P.Cin + BK - 1) / BK;
 
   // A tcgen05.mma step with N < 256 takes as long as one with N = 256, so
@@ -650,7 +670,7 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, b
   }
   if (L.swap) L.pair = false;
   if (P.out_f32) L.pair = false;
-  if (P.gn_stats || P.gn_out) L.pair = false;   // both exist in the one-CTA variants   // the fp32 epilogue exists in the single and transposed variants
+  if (P.gn_stats || P.gn_out || P.y_scatter) L.pair = false;   // one-CTA variants only   // the fp32 epilogue exists in the single and transposed variants
   const int ctas = L.pair ? 2 : 1;
   if (L.swap) {
     kp.co_tile = 128;
@@ -994,6 +1014,10 @@ conv3d_status_t noalloc_scratch(void*& out) {
 // A single frame (D = 1) needs neither: dx[n, 0] = sum over taps of the 2D
 // transposed convolution of dy[n, 0], i.e. the forward first-frame problem on
 // dy with the transformed weight, which folds the taps into a (hi, lo) pair.
+// Workspace slack for the single-frame data gradient of a strided convolution:
+// each phase's folded weight starts on a 256-byte boundary (at most 64 phases).
+constexpr size_t kPhaseSlack = 64 * 256;
+
 struct BwdDataPlan {
   Problem fwd;      // the forward problem being differentiated
   Problem tr;       // the whole transposed convolution (no replicate padding), or
@@ -1001,6 +1025,7 @@ struct BwdDataPlan {
   Problem front;    // replicate padding, D > 1: extended frames, fp32
   Problem body;     // replicate padding, D > 1: frames 1.., one sample
   bool rep;         // front + body + fold
+  bool phased;      // spatial stride: one transposed convolution per phase
   size_t wt_bytes;  // flipped weight
   size_t ext_bytes; // fp32 gradient of the front frames, or the folded weight (D = 1)
 };
@@ -1017,12 +1042,14 @@ conv3d_status_t plan_bwd_data(const void* dy, const void* w, const void* dx, int
   conv3d_status_t st = validate(dx, w, nullptr, nullptr, dy, N, Cin, D, H, W, Cout, kernel,
                                 stride, pad, tpad, dtype, B.fwd);
   if (st != CONV3D_OK) return st;
-  if (stride[0] != 1 || stride[1] != 1 || stride[2] != 1) {
-    set_error("the backward data pass supports stride (1,1,1) only");
+  if (stride[0] != 1) {
+    set_error("the backward data pass supports temporal stride 1 only");
     return CONV3D_ERR_UNSUPPORTED;
   }
   const Problem& F = B.fwd;
-  if (F.ph > F.kh - 1 || F.pw > F.kw - 1 || F.pf > F.kt - 1 || F.pb > F.kt - 1) {
+  B.phased = stride[1] != 1 || stride[2] != 1;
+  if (F.pf > F.kt - 1 || F.pb > F.kt - 1 ||
+      (!B.phased && (F.ph > F.kh - 1 || F.pw > F.kw - 1))) {
     set_error("the backward data pass needs pads <= kernel extent - 1");
     return CONV3D_ERR_UNSUPPORTED;
   }
@@ -1076,7 +1103,129 @@ conv3d_status_t plan_bwd_data(const void* dy, const void* w, const void* dx, int
   if (B.rep)
     B.ext_bytes = (static_cast<size_t>(N) * F.kt * H * W * Cin * 4 + 255) & ~size_t(255);
   else if (T.fold)
-    B.ext_bytes = (fold_bytes(Cout, Cin, kernel) + 255) & ~size_t(255);
+    B.ext_bytes = ((fold_bytes(Cout, Cin, kernel) + 255) & ~size_t(255)) + kPhaseSlack;
+  return CONV3D_OK;
+}
+
+// The data gradient of a convolution with spatial strides (sh, sw), temporal
+// stride 1.  dx splits into sh*sw phases (rh, rw): rows h = a*sh + rh receive
+// only the taps ih = qh + sh*j (qh = (rh + ph) mod sh, j < Jh), from dy rows
+// a + ch - j (ch = (rh + ph - qh) / sh), i.e. phase (rh, rw) of dx is the
+// stride-1 convolution of dy with the mirrored sub-kernel of those taps and
+// front pads Jh-1-ch, Jw-1-cw, giving Ah x Aw outputs that the kernel's
+// epilogue stores straight to their strided positions of dx.  The temporal
+// direction is the stride-1 data gradient's (front frames in fp32 and a fold
+// for causal replicate padding, the first-frame fold for a single frame).
+// Phases that no tap reaches (a stride larger than the kernel) are zero.
+conv3d_status_t bwd_data_phases(DeviceState& S, const BwdDataPlan& B, const void* dy,
+                                const void* w, void* dx, void* workspace, cudaStream_t stream) {
+  const Problem& F = B.fwd;
+  const int N = F.N, Cin = F.Cin, Cout = F.Cout, D = F.D, H = F.H, W = F.W;
+  const int kt = F.kt, kh = F.kh, kw = F.kw, sh = F.sh, sw = F.sw;
+  const bool bf16 = F.dtype == CONV3D_BF16;
+  char* wt_at = static_cast<char*>(workspace);
+  char* ext_at = static_cast<char*>(workspace) + B.wt_bytes;
+  conv3d_status_t st = CONV3D_OK;
+  for (int rh = 0; rh < sh && rh < H; ++rh) {
+    for (int rw = 0; rw < sw && rw < W; ++rw) {
+      const int qh = (rh + F.ph) % sh, qw = (rw + F.pw) % sw;
+      const int Jh = qh < kh ? (kh - 1 - qh) / sh + 1 : 0;
+      const int Jw = qw < kw ? (kw - 1 - qw) / sw + 1 : 0;
+      const int ch = (rh + F.ph - qh) / sh, cw = (rw + F.pw - qw) / sw;
+      const int Ah = (H - 1 - rh) / sh + 1, Aw = (W - 1 - rw) / sw + 1;
+      const FoldPhase fp{Aw, sh, sw, rh, rw, H, W, Cin};
+      if (Jh == 0 || Jw == 0) {
+        const long long total = static_cast<long long>(N) * D * Ah * Aw * (Cin / 8);
+        int blocks = static_cast<int>((total + 255) / 256);
+        if (blocks > 8 * S.num_sms) blocks = 8 * S.num_sms;
+        zero_phase_kernel<<<blocks, 256, 0, stream>>>(static_cast<uint16_t*>(dx),
+                                                      static_cast<long long>(N) * D, Ah, Aw, fp);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "zero phase launch");
+        continue;
+      }
+      const int taps = kt * Jh * Jw;
+      uint16_t* wt = reinterpret_cast<uint16_t*>(wt_at);
+      wt_at += static_cast<size_t>(Cin) * taps * Cout * 2;   // a multiple of 16 bytes
+      {
+        const dim3 grid((Cin + 31) / 32, (Cout + 31) / 32, taps);
+        flip_transpose_weight_kernel<<<grid, dim3(32, 8), 0, stream>>>(
+            static_cast<const uint16_t*>(w), wt, Cout, taps, Cin, kh, kw, Jh, Jw, qh, qw, sh, sw);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
+      }
+      Problem T = B.tr;            // temporal rule and sizes of the stride-1 transposed problem
+      T.kh = Jh;
+      T.kw = Jw;
+      T.ph = Jh - 1 - ch;
+      T.pw = Jw - 1 - cw;
+      T.Ho = Ah;
+      T.Wo = Aw;
+      T.exact_out = true;
+      T.y_scatter = static_cast<uint16_t*>(dx);
+      T.sc_sh = sh;
+      T.sc_sw = sw;
+      T.sc_rh = rh;
+      T.sc_rw = rw;
+      T.sc_H = H;
+      T.sc_W = W;
+      if (T.ph < -127 || T.ph > 127 || T.pw < -127 || T.pw > 127) {
+        set_error("stride and padding out of range for the data gradient");
+        return CONV3D_ERR_UNSUPPORTED;
+      }
+      if (T.fold) {                // one causal-replicate frame: the first-frame fold
+        const int kp[3] = {kt, Jh, Jw};
+        const size_t fb = fold_bytes(Cout, Cin, kp);
+        st = run(T, dy, wt, nullptr, nullptr, dx, ext_at, fb, false, stream);
+        ext_at += fb;              // 256-byte multiples; the workspace has the slack
+        if (st != CONV3D_OK) return st;
+        continue;
+      }
+      if (!B.rep) {
+        if ((st = launch_main(S, T, dy, nullptr, wt, nullptr, nullptr, dx, stream)) != CONV3D_OK)
+          return st;
+        continue;
+      }
+      // causal replicate, D > 1: the kt front frames in fp32 (dense, this phase's
+      // pixels), frames 1.. straight to dx, then the fold into frame 0
+      float* ext = reinterpret_cast<float*>(ext_at);
+      ext_at += static_cast<size_t>(N) * kt * Ah * Aw * Cin * 4;
+      Problem Fr = T;
+      Fr.pf = T.pf + kt - 1;
+      Fr.Do = kt;
+      Fr.out_f32 = true;
+      Fr.y_scatter = nullptr;
+      if ((st = launch_main(S, Fr, dy, nullptr, wt, nullptr, nullptr, ext, stream)) != CONV3D_OK)
+        return st;
+      if (D > 1) {
+        Problem Bo = T;
+        Bo.N = 1;
+        Bo.D = F.Do - 1;
+        Bo.Do = D - 1;
+        const long long dy_frame = static_cast<long long>(F.Ho) * F.Wo * Cout;
+        const long long dx_frame = static_cast<long long>(H) * W * Cin;
+        for (int n = 0; n < N; ++n) {
+          Bo.y_scatter = static_cast<uint16_t*>(dx) + (n * static_cast<long long>(D) + 1) * dx_frame;
+          const uint16_t* dy_n = static_cast<const uint16_t*>(dy) + (n * static_cast<long long>(F.Do) + 1) * dy_frame;
+          if ((st = launch_main(S, Bo, dy_n, nullptr, wt, nullptr, nullptr, Bo.y_scatter, stream)) !=
+              CONV3D_OK)
+            return st;
+        }
+      }
+      const long long frame_elems = static_cast<long long>(Ah) * Aw * Cin;
+      const long long total = static_cast<long long>(N) * (frame_elems / 8);
+      int blocks = static_cast<int>((total + 255) / 256);
+      if (blocks > 8 * S.num_sms) blocks = 8 * S.num_sms;
+      if (bf16)
+        fold_front_gradient_kernel<true><<<blocks, 256, 0, stream>>>(
+            ext, static_cast<uint16_t*>(dx), N, D, kt, frame_elems, fp, 1);
+      else
+        fold_front_gradient_kernel<false><<<blocks, 256, 0, stream>>>(
+            ext, static_cast<uint16_t*>(dx), N, D, kt, frame_elems, fp, 1);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "gradient fold launch");
+    }
+  }
   return CONV3D_OK;
 }
 
@@ -1298,7 +1447,7 @@ size_t conv3d_bwd_data_workspace_bytes(int N, int Cin, int D, int H, int W, int 
     if (D > 1)
       ext = (static_cast<size_t>(N) * kernel[0] * H * W * Cin * 4 + 255) & ~size_t(255);
     else
-      ext = (fold_bytes(Cout, Cin, kernel) + 255) & ~size_t(255);
+      ext = ((fold_bytes(Cout, Cin, kernel) + 255) & ~size_t(255)) + kPhaseSlack;
   }
   return wt + ext;
 }
@@ -1332,12 +1481,14 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
   DeviceState* S = nullptr;
   int dev = 0;
   if ((st = device_state(S, dev)) != CONV3D_OK) return st;
+  if (B.phased) return bwd_data_phases(*S, B, dy, w, dx, workspace, stream);
   uint16_t* wt = static_cast<uint16_t*>(workspace);
   {
     const int taps = kernel[0] * kernel[1] * kernel[2];
     const dim3 grid((Cin + 31) / 32, (Cout + 31) / 32, taps);
     flip_transpose_weight_kernel<<<grid, dim3(32, 8), 0, stream>>>(
-        static_cast<const uint16_t*>(w), wt, Cout, taps, Cin);
+        static_cast<const uint16_t*>(w), wt, Cout, taps, Cin, kernel[1], kernel[2], kernel[1],
+        kernel[2], 0, 0, 1, 1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
   }
@@ -1396,10 +1547,10 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
     if (blocks > 8 * S->num_sms) blocks = 8 * S->num_sms;
     if (dtype == CONV3D_BF16)
       fold_front_gradient_kernel<true><<<blocks, 256, 0, stream>>>(
-          ext, static_cast<uint16_t*>(dx), N, D, kernel[0], frame_elems);
+          ext, static_cast<uint16_t*>(dx), N, D, kernel[0], frame_elems, FoldPhase{}, 0);
     else
       fold_front_gradient_kernel<false><<<blocks, 256, 0, stream>>>(
-          ext, static_cast<uint16_t*>(dx), N, D, kernel[0], frame_elems);
+          ext, static_cast<uint16_t*>(dx), N, D, kernel[0], frame_elems, FoldPhase{}, 0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "gradient fold launch");
   }
@@ -1753,7 +1904,8 @@ conv3d_status_t conv3d_bwd_data_cached(const void* dy, const void* w, void* dx, 
     const int taps = kernel[0] * kernel[1] * kernel[2];
     const dim3 grid((Cin + 31) / 32, (Cout + 31) / 32, taps);
     flip_transpose_weight_kernel<<<grid, dim3(32, 8), 0, stream>>>(
-        static_cast<const uint16_t*>(w), wt, Cout, taps, Cin);
+        static_cast<const uint16_t*>(w), wt, Cout, taps, Cin, kernel[1], kernel[2], kernel[1],
+        kernel[2], 0, 0, 1, 1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
   }

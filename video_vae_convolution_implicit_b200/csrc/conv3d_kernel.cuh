@@ -98,6 +98,13 @@ struct KernelParams {
   // [N][gn_out_groups][2] (zeroed by the host), or null
   double* gn_out;
   int gn_out_groups;                 // at most 64; divides Cout
+  // Strided output (one phase of the data gradient of a strided convolution):
+  // output pixel (a, b) of output frame f is element
+  // [f][a*sc_sh + sc_rh][b*sc_sw + sc_rw] of y_scatter, frames sc_H x sc_W,
+  // written by plain stores from registers instead of the TMA store map
+  // (16-bit outputs, no residual); null otherwise.
+  uint16_t* y_scatter;
+  int sc_sh, sc_sw, sc_rh, sc_rw, sc_H, sc_W;
 };
 
 // Epilogue staging: each epilogue warp owns two 32-row x 32-channel buffers
@@ -895,6 +902,24 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
                 asm volatile("st.shared.f32 [%0], %1;" ::"r"(yb + swz128(e, lane >> 2) + word),
                              "f"(v[e])
                              : "memory");
+            } else if (p.y_scatter != nullptr) {
+              // strided output: lane = channel, so each pixel's 32 channels are
+              // one 64-byte store of the warp
+              int q = tl.p0 + 32 * j;
+              int a = q / p.Wo, bq = q - a * p.Wo;
+#pragma unroll 4
+              for (int e = 0; e < 32; ++e, ++q) {
+                if (q < p.HoWo && ch < p.Cout) {
+                  const size_t off =
+                      ((static_cast<size_t>(tl.frame_out) * p.sc_H + a * p.sc_sh + p.sc_rh) *
+                           p.sc_W + bq * p.sc_sw + p.sc_rw) * p.Cout + ch;
+                  p.y_scatter[off] = static_cast<uint16_t>(C::pack(v[e], 0.0f) & 0xFFFFu);
+                }
+                if (++bq == p.Wo) {
+                  bq = 0;
+                  ++a;
+                }
+              }
             } else {
               float gs = 0.0f, gq = 0.0f;   // this channel's rounded outputs, for the statistics
 #pragma unroll
@@ -922,8 +947,10 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
             const int pix0 = tl.p0 + 32 * j;
             const bool refill = use_res && j + 2 < live_chunks;
             if (lane == 0) {
-              tma_store_3d(&map_y, yb, ch0, pix0, tl.frame_out);
-              bulk_commit_group();
+              if (p.y_scatter == nullptr) {
+                tma_store_3d(&map_y, yb, ch0, pix0, tl.frame_out);
+                bulk_commit_group();
+              }
               if (refill) {
                 mbar_arrive_expect_tx(rbar + 8 * b, EPI_BUF_BYTES);
                 tma_load_3d(rbuf + b * EPI_BUF_BYTES, &map_r, rbar + 8 * b, ch0, pix0 + 64,
@@ -1040,10 +1067,26 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int g = 0; g < 16; ++g) pk[g] = C::pack(v[2 * g], v[2 * g + 1]);
+            if (p.y_scatter != nullptr) {
+              // strided output: this thread's pixel, 32 channels as four 16-byte stores
+              const int q = row_base + static_cast<int>(lane);
+              if (q < p.HoWo) {
+                const int a = q / p.Wo, bq = q - a * p.Wo;
+                uint4* dst = reinterpret_cast<uint4*>(
+                    p.y_scatter +
+                    ((static_cast<size_t>(tl.frame_out) * p.sc_H + a * p.sc_sh + p.sc_rh) *
+                         p.sc_W + bq * p.sc_sw + p.sc_rw) * p.Cout + cb);
 #pragma unroll
-            for (int g = 0; g < 4; ++g)
-              st_shared_v4(ybuf + b * ybytes + swz64(lane, g), pk[4 * g], pk[4 * g + 1],
-                           pk[4 * g + 2], pk[4 * g + 3]);
+                for (int g = 0; g < 4; ++g)
+                  if (cb + 8 * g < p.Cout)
+                    dst[g] = make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
+              }
+            } else {
+#pragma unroll
+              for (int g = 0; g < 4; ++g)
+                st_shared_v4(ybuf + b * ybytes + swz64(lane, g), pk[4 * g], pk[4 * g + 1],
+                             pk[4 * g + 2], pk[4 * g + 3]);
+            }
             if (p.gn_out != nullptr) {
               // this row's rounded outputs, per group of the chunk's channels
               const bool row_in = row_base + static_cast<int>(lane) < p.HoWo;
@@ -1069,8 +1112,10 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
           // every lane has read residual buffer b: refill it with chunk j+2
           const bool refill = use_res && j + 2 < live_chunks;
           if (lane == 0) {
-            tma_store_3d(&map_y, ybuf + b * ybytes, cb, row_base, tl.frame_out);
-            bulk_commit_group();
+            if (p.y_scatter == nullptr) {
+              tma_store_3d(&map_y, ybuf + b * ybytes, cb, row_base, tl.frame_out);
+              bulk_commit_group();
+            }
             if (refill) {
               mbar_arrive_expect_tx(rbar + 8 * b, EPI_BUF_BYTES);
               tma_load_3d(rbuf + b * EPI_BUF_BYTES, &map_r, rbar + 8 * b, cb + 64, row_base,
@@ -1154,17 +1199,28 @@ __global__ void fold_temporal_taps_kernel(const uint16_t* __restrict__ w, uint16
 // transpose: block = one tap and a 32 x 32 tile, staged in shared memory so
 // that both the reads and the writes run along contiguous channels.
 // Launch: grid (ceil(Cin/32), ceil(Cout/32), taps), block (32, 8).
+//
+// With a spatial stride the data gradient splits into phases (rh, rw): dx rows
+// a*sh + rh receive only the taps ih = qh + sh*j (qh = (rh + ph) mod sh), so a
+// phase is a convolution of dy with the sub-kernel of those taps, mirrored.
+// Then wt holds that sub-kernel: wt[ci, it', jh', jw', co] =
+// w[co, kt-1-it', qh + sh*(Jh-1-jh'), qw + sw*(Jw-1-jw'), ci], taps = kt*Jh*Jw
+// (sh = sw = 1, qh = qw = 0, Jh = kh, Jw = kw: the plain mirror above).
 __global__ void flip_transpose_weight_kernel(const uint16_t* __restrict__ w,
                                              uint16_t* __restrict__ wt, int Cout, int taps,
-                                             int Cin) {
+                                             int Cin, int kh, int kw, int Jh, int Jw, int qh,
+                                             int qw, int sh, int sw) {
   __shared__ uint16_t tile[32][33];
   const int ci0 = blockIdx.x * 32, co0 = blockIdx.y * 32;
-  const int tap = blockIdx.z;                  // tap of wt
-  const int tap_src = taps - 1 - tap;          // mirrored tap of w
+  const int tap = blockIdx.z;                  // tap of wt: (it', jh', jw')
+  const int jw_ = tap % Jw, jh_ = (tap / Jw) % Jh, it_ = tap / (Jw * Jh);
+  const int kt = taps / (Jh * Jw);
+  const int tap_src = ((kt - 1 - it_) * kh + qh + sh * (Jh - 1 - jh_)) * kw + qw + sw * (Jw - 1 - jw_);
+  const int taps_src = kt * kh * kw;
   for (int r = threadIdx.y; r < 32; r += 8) {
     const int co = co0 + r, ci = ci0 + threadIdx.x;
     if (co < Cout && ci < Cin)
-      tile[r][threadIdx.x] = w[(static_cast<long long>(co) * taps + tap_src) * Cin + ci];
+      tile[r][threadIdx.x] = w[(static_cast<long long>(co) * taps_src + tap_src) * Cin + ci];
   }
   __syncthreads();
   for (int r = threadIdx.y; r < 32; r += 8) {
@@ -1179,10 +1235,18 @@ __global__ void flip_transpose_weight_kernel(const uint16_t* __restrict__ w,
 // ext[n, 0 .. kt-1], ext holding the fp32 gradient of the kt frames
 // -(kt-1)..0 (frame 0's own taps in ext[n, kt-1]); one rounding.  Frames >= 1
 // are written by the convolution itself.  8 values per thread.
+//
+// Strided phases: ext holds a phase's A_h x A_w pixels per frame, and pixel
+// (a, b) of it belongs at row a*sh + rh, column b*sw + rw of dx's H x W frame
+// (phase = nullptr: ext's frames are dx's, pixel for pixel).
+struct FoldPhase {
+  int Aw, sh, sw, rh, rw, H, W, C;
+};
+
 template <bool kBF16>
 __global__ void fold_front_gradient_kernel(const float* __restrict__ ext,
                                            uint16_t* __restrict__ dx, int N, int D, int kt,
-                                           long long frame_elems) {
+                                           long long frame_elems, FoldPhase ph, int phased) {
   using C = Cvt<kBF16>;
   const long long vecs_per_frame = frame_elems / 8;
   const long long total = static_cast<long long>(N) * vecs_per_frame;
@@ -1203,7 +1267,36 @@ __global__ void fold_front_gradient_kernel(const float* __restrict__ ext,
     out.y = C::pack(acc[2], acc[3]);
     out.z = C::pack(acc[4], acc[5]);
     out.w = C::pack(acc[6], acc[7]);
-    reinterpret_cast<uint4*>(dx)[n * D * vecs_per_frame + v] = out;
+    if (!phased) {
+      reinterpret_cast<uint4*>(dx)[n * D * vecs_per_frame + v] = out;
+    } else {
+      const long long pix = (v * 8) / ph.C, c = (v * 8) - pix * ph.C;
+      const long long a = pix / ph.Aw, b = pix - a * ph.Aw;
+      const long long off =
+          ((n * D * static_cast<long long>(ph.H) + a * ph.sh + ph.rh) * ph.W + b * ph.sw + ph.rw) *
+              ph.C + c;
+      *reinterpret_cast<uint4*>(dx + off) = out;
+    }
+  }
+}
+
+// dx positions of a phase that no tap reaches (a stride larger than the
+// kernel): every frame's rows a*sh + rh, columns b*sw + rw, all channels,
+// set to zero.  8 channels (16 bytes) per thread.
+__global__ void zero_phase_kernel(uint16_t* __restrict__ dx, long long frames, int Ah, int Aw,
+                                  FoldPhase ph) {
+  const long long vecs_per_pix = ph.C / 8;
+  const long long total = frames * Ah * Aw * vecs_per_pix;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long c = (i % vecs_per_pix) * 8;
+    long long pix = i / vecs_per_pix;
+    const long long b = pix % Aw;
+    pix /= Aw;
+    const long long a = pix % Ah;
+    const long long f = pix / Ah;
+    const long long off = ((f * ph.H + a * ph.sh + ph.rh) * ph.W + b * ph.sw + ph.rw) * ph.C + c;
+    *reinterpret_cast<uint4*>(dx + off) = make_uint4(0, 0, 0, 0);
   }
 }
 
