@@ -50,3 +50,35 @@ def test_plan_log_is_silent_by_default():
     r = _run(False)
     assert r.returncode == 0, r.stderr[-2000:]
     assert "libconv3d: " not in r.stderr
+
+
+SPLIT_SCRIPT = """
+import torch
+import seeded_inputs as si
+import video_vae_convolution_implicit_b200 as c3
+# 3 frames of 80x80 in 128-pixel tiles, 64 channels: 150 tiles, i.e. one full
+# round of 148 and a last round of 2 tiles, which the default rule splits
+x = si.tensor((1, 3, 80, 80, 64), 7, 0, 1.0, torch.bfloat16, "cuda")
+w = si.tensor((64, 3, 3, 3, 64), 7, 1, (27 * 64) ** -0.5, torch.bfloat16, "cuda")
+y = c3.conv3d(x, w)
+assert c3.poll_status() == c3.Status.OK
+print(torch.cuda.get_device_properties(0).multi_processor_count)
+"""
+
+
+def test_plan_log_shows_the_tail_split():
+    env = dict(os.environ)
+    env["CONV3D_LOG"] = "1"
+    env.pop("CONV3D_SPLIT", None)
+    r = subprocess.run([sys.executable, "-c", SPLIT_SCRIPT], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    sms = int(r.stdout.split()[-1])
+    lines = [l for l in r.stderr.splitlines() if "implicit GEMM" in l]
+    assert len(lines) == 1, lines
+    tail = 150 % sms
+    if sms <= 150 and 0 < tail <= sms // 2:
+        # 27 k-blocks a tile: pieces of at least 8 k-blocks, so 3 of them
+        assert f"last {tail} tiles in 3 pieces" in lines[0], lines
+    else:
+        assert "in 1 pieces" in lines[0], lines
