@@ -69,6 +69,7 @@ print(torch.cuda.get_device_properties(0).multi_processor_count)
 def test_plan_log_shows_the_tail_split():
     env = dict(os.environ)
     env["CONV3D_LOG"] = "1"
+    env["CONV3D_SWAP"] = "0"     # the 128-pixel tiles (the transposed variant would make 75)
     env.pop("CONV3D_SPLIT", None)
     r = subprocess.run([sys.executable, "-c", SPLIT_SCRIPT], cwd=ROOT, env=env,
                        capture_output=True, text=True, timeout=600)

@@ -57,6 +57,7 @@ def test_default_rule_splits_a_short_last_round(monkeypatch):
     # 3 frames of 80x80 in 128-pixel tiles = 150 tiles: one full round of 148
     # and a last round of 2, which the default rule cuts into pieces
     monkeypatch.delenv("CONV3D_SPLIT", raising=False)
+    monkeypatch.setenv("CONV3D_SWAP", "0")      # 128-pixel tiles: 150 of them
     p = problem(1, 64, 3, 80, 80, 64, (3, 3, 3), (0, 1, 1), CREP, seed=47, residual=True)
     y = run(p)
     assert_close(y.double().cpu().numpy(), oracle_ref(p), "default split")
