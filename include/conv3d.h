@@ -259,12 +259,19 @@ CONV3D_API conv3d_status_t conv3d_fwd_gn(const void* x, const double* stats, con
  *
  * Arguments describe the FORWARD problem: dy is [N, Do, Ho, Wo, Cout] (y's
  * shape), w [Cout, kt, kh, kw, Cin], dx [N, D, H, W, Cin] (written).  Supported:
- * stride (1,1,1), pads <= kernel extent - 1, temporal rules zero, causal
- * replicate and causal zero, plus the forward call's channel and alignment
+ * temporal stride 1 and spatial strides up to 8, pads <= kernel extent - 1 at
+ * stride 1, temporal rules zero, causal replicate and causal zero, plus the
+ * forward call's channel and alignment
  * rules.  workspace: device, 256-byte aligned, conv3d_bwd_data_workspace_bytes()
- * bytes, not overlapping the tensors.  dx must not overlap dy or w.
- * Errors: CONV3D_ERR_UNSUPPORTED for a stride other than 1, the cached-frames
- * rule (conv3d_bwd_data_cached) or pads beyond kernel extent - 1; CONV3D_ERR_WORKSPACE for a missing or
+ * bytes, not overlapping the tensors (it includes about 21 MB in which a launch
+ * that is one partly filled wave of tiles -- the front frames, a single frame,
+ * a short clip -- splits its tiles along K across the idle SMs).  dx must not
+ * overlap dy or w.  Spatial strides: dx is computed phase by phase, each phase
+ * (rows h = a*sh + rh, columns a*sw + rw) a stride-1 convolution of dy with the
+ * mirrored taps that reach it, stored straight to its strided positions.
+ * Errors: CONV3D_ERR_UNSUPPORTED for a temporal stride other than 1, the
+ * cached-frames rule (conv3d_bwd_data_cached) or pads beyond kernel extent - 1
+ * at stride 1; CONV3D_ERR_WORKSPACE for a missing or
  * short workspace; otherwise as conv3d_fwd.
  */
 CONV3D_API conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, int Cin,

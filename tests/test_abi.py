@@ -243,10 +243,14 @@ def call_bwd_weight(**kw):
 def test_bwd_workspace_bytes():
     # flipped weight + (replicate padding) the fp32 gradient of frames -2..0
     wt = 64 * 27 * 64 * 2
+    split = 160 * (128 * 256 * 4 + 32)       # the tail-split region: 160 pieces and tickets
     assert c3.bwd_data_workspace_bytes(1, 64, 4, 16, 16, 64, (3, 3, 3), (0, 1, 1),
-                                       c3.TPAD_CAUSAL_REPLICATE) == wt + 3 * 16 * 16 * 64 * 4
+                                       c3.TPAD_CAUSAL_REPLICATE) == wt + 3 * 16 * 16 * 64 * 4 + split
     assert c3.bwd_data_workspace_bytes(2, 64, 4, 16, 16, 64, (3, 3, 3), (1, 1, 1),
-                                       c3.TPAD_ZERO) == wt
+                                       c3.TPAD_ZERO) == wt + split
+    # the cached-frames data gradient needs the flipped weight only
+    assert c3.bwd_data_workspace_bytes(2, 64, 4, 16, 16, 64, (3, 3, 3), (0, 1, 1),
+                                       c3.TPAD_CAUSAL_CACHED) == wt
     dw = 64 * 27 * 32 * 4
     assert c3.bwd_weight_workspace_bytes(32, 64, (3, 3, 3)) >= dw + 64 * 4
 

@@ -594,7 +594,8 @@ int split_override() {
   return v == 0 ? 0 : (v >= 2 && v <= 8 ? v : -1);
 }
 
-conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, bool allow_split,
+// split_room: bytes of scratch the tail split may use (0: no split).
+conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, size_t split_room,
                             LaunchPlan& L) {
   // The folded weight is a kt = 2 (hi, lo) kernel over the single frame; with
   // causal replicate padding both of its taps read frame 0.
@@ -688,15 +689,16 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, b
   // (S <= SMs / R, at most 8, at least 8 k-blocks a piece), the pieces run
   // side by side on S*R SMs, and the piece that completes a tile adds up the
   // S fp32 partials (in piece order) before the usual epilogue: the last
-  // round takes about 1/S of a tile's time.  Only with a library-owned
-  // workspace (conv3d_fwd), never for CTA pairs or fp32 outputs.
+  // round takes about 1/S of a tile's time.  Only with scratch for it (the
+  // library's own for conv3d_fwd, a region of the data gradient's workspace),
+  // never for CTA pairs or strided outputs.
   kp.num_items = kp.num_tiles;
   kp.split_first = kp.num_tiles;
   kp.split_s = 1;
   L.split_bytes = 0;
   L.split_part_bytes = 0;
   const int forced = split_override();
-  if (allow_split && forced != 0 && !L.pair && !P.out_f32) {
+  if (split_room > 0 && forced != 0 && !L.pair && !P.y_scatter) {
     const int U = S.num_sms;
     const int T = kp.num_tiles;
     int R = T % U;
@@ -708,6 +710,10 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, b
         if (sp > 8) sp = 8;
         while (sp > 1 && kb_nominal / sp < 8) --sp;
       }
+      // no more pieces than the scratch holds
+      const size_t slot = static_cast<size_t>(BM) * kp.BN * sizeof(float);
+      while (sp >= 2 && static_cast<size_t>(R) * sp * slot + static_cast<size_t>(R) * 32 > split_room)
+        --sp;
       if (sp >= 2) {
         kp.split_first = T - R;
         kp.split_s = sp;
@@ -865,13 +871,35 @@ conv3d_status_t launch_planned(DeviceState& S, const Problem& P, LaunchPlan& L, 
                 : launch_kernel<false, false, false>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
 }
 
-// The main kernel without a tail split (no scratch needed).
+// Scratch a launch may use for the tail split: `bytes` at `ptr` (256-byte
+// aligned).  The tickets are cleared on the stream before the launch, so the
+// region needs no state between calls.
+struct SplitRegion {
+  void* ptr;
+  size_t bytes;
+};
+
+// Points the plan's split at `base` (partials, then tickets) with generation `gen`.
+void assign_split(LaunchPlan& L, void* base, unsigned int gen) {
+  char* b = static_cast<char*>(base);
+  L.kp.part = reinterpret_cast<float*>(b);
+  L.kp.ticket = reinterpret_cast<unsigned long long*>(b + L.split_part_bytes);
+  L.kp.gen = gen;
+}
+
+// The main kernel, with a tail split only where `split` offers scratch for it.
 conv3d_status_t launch_main(DeviceState& S, const Problem& P, const void* x, const void* prev,
                             const void* wmat, const void* bias, const void* residual, void* y,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, const SplitRegion* split = nullptr) {
   LaunchPlan L;
-  conv3d_status_t st = plan_launch(S, P, P.dtype == CONV3D_BF16, false, L);
+  conv3d_status_t st = plan_launch(S, P, P.dtype == CONV3D_BF16, split ? split->bytes : 0, L);
   if (st != CONV3D_OK) return st;
+  if (L.split_bytes > 0) {
+    cudaError_t e = cudaMemsetAsync(static_cast<char*>(split->ptr) + L.split_part_bytes, 0,
+                                    L.split_bytes - L.split_part_bytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "split tickets clear");
+    assign_split(L, split->ptr, 1u);
+  }
   return launch_planned(S, P, L, x, prev, wmat, bias, residual, y, stream);
 }
 
@@ -911,7 +939,7 @@ conv3d_status_t cached_scratch(DeviceState& S, cudaStream_t stream, size_t need,
 
 conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* bias,
                     const void* residual, void* y, void* ws, size_t ws_bytes, bool cached_ws,
-                    cudaStream_t stream) {
+                    cudaStream_t stream, const SplitRegion* split = nullptr) {
   conv3d_status_t st = load_entry_points();
   if (st != CONV3D_OK) return st;
   DeviceState* S = nullptr;
@@ -920,7 +948,8 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
   const bool bf16 = P.dtype == CONV3D_BF16;
   const void* wmat = w;
   LaunchPlan L;
-  if ((st = plan_launch(*S, P, bf16, cached_ws, L)) != CONV3D_OK) return st;
+  const size_t room = cached_ws ? ~size_t(0) : (split ? split->bytes : 0);
+  if ((st = plan_launch(*S, P, bf16, room, L)) != CONV3D_OK) return st;
   const int kfold[3] = {P.kt, P.kh, P.kw};
   const size_t fold_need = P.fold ? fold_bytes(P.Cin, P.Cout, kfold) : 0;   // 256-byte multiple
   if (cached_ws && fold_need + L.split_bytes > 0) {
@@ -928,12 +957,12 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
     if ((st = cached_scratch(*S, stream, fold_need + L.split_bytes, ws, gen)) != CONV3D_OK)
       return st;
     ws_bytes = fold_need + L.split_bytes;
-    if (L.split_bytes > 0) {
-      char* base = static_cast<char*>(ws) + fold_need;
-      L.kp.part = reinterpret_cast<float*>(base);
-      L.kp.ticket = reinterpret_cast<unsigned long long*>(base + L.split_part_bytes);
-      L.kp.gen = gen;
-    }
+    if (L.split_bytes > 0) assign_split(L, static_cast<char*>(ws) + fold_need, gen);
+  } else if (L.split_bytes > 0) {   // a caller's split region (the data gradient)
+    cudaError_t e = cudaMemsetAsync(static_cast<char*>(split->ptr) + L.split_part_bytes, 0,
+                                    L.split_bytes - L.split_part_bytes, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "split tickets clear");
+    assign_split(L, split->ptr, 1u);
   }
   if (P.fold) {
     const size_t need = fold_need;
@@ -1018,6 +1047,12 @@ conv3d_status_t noalloc_scratch(void*& out) {
 // each phase's folded weight starts on a 256-byte boundary (at most 64 phases).
 constexpr size_t kPhaseSlack = 64 * 256;
 
+// The data gradient's tail-split region: the partials of up to 160 pieces of a
+// 128 x 256 fp32 accumulator and their tickets (160 >= the SMs of a B200, and
+// the split never runs more pieces than SMs).
+constexpr size_t kSplitRegionBytes =
+    ((160 * (static_cast<size_t>(BM) * 256 * sizeof(float) + 32)) + 255) & ~size_t(255);
+
 struct BwdDataPlan {
   Problem fwd;      // the forward problem being differentiated
   Problem tr;       // the whole transposed convolution (no replicate padding), or
@@ -1026,6 +1061,7 @@ struct BwdDataPlan {
   Problem body;     // replicate padding, D > 1: frames 1.., one sample
   bool rep;         // front + body + fold
   bool phased;      // spatial stride: one transposed convolution per phase
+  size_t split_bytes;  // the tail-split region, after the flipped weight and ext
   size_t wt_bytes;  // flipped weight
   size_t ext_bytes; // fp32 gradient of the front frames, or the folded weight (D = 1)
 };
@@ -1104,6 +1140,7 @@ conv3d_status_t plan_bwd_data(const void* dy, const void* w, const void* dx, int
     B.ext_bytes = (static_cast<size_t>(N) * F.kt * H * W * Cin * 4 + 255) & ~size_t(255);
   else if (T.fold)
     B.ext_bytes = ((fold_bytes(Cout, Cin, kernel) + 255) & ~size_t(255)) + kPhaseSlack;
+  B.split_bytes = kSplitRegionBytes;
   return CONV3D_OK;
 }
 
@@ -1118,7 +1155,8 @@ conv3d_status_t plan_bwd_data(const void* dy, const void* w, const void* dx, int
 // for causal replicate padding, the first-frame fold for a single frame).
 // Phases that no tap reaches (a stride larger than the kernel) are zero.
 conv3d_status_t bwd_data_phases(DeviceState& S, const BwdDataPlan& B, const void* dy,
-                                const void* w, void* dx, void* workspace, cudaStream_t stream) {
+                                const void* w, void* dx, void* workspace, cudaStream_t stream,
+                                const SplitRegion* split) {
   const Problem& F = B.fwd;
   const int N = F.N, Cin = F.Cin, Cout = F.Cout, D = F.D, H = F.H, W = F.W;
   const int kt = F.kt, kh = F.kh, kw = F.kw, sh = F.sh, sw = F.sw;
@@ -1195,7 +1233,8 @@ conv3d_status_t bwd_data_phases(DeviceState& S, const BwdDataPlan& B, const void
       Fr.Do = kt;
       Fr.out_f32 = true;
       Fr.y_scatter = nullptr;
-      if ((st = launch_main(S, Fr, dy, nullptr, wt, nullptr, nullptr, ext, stream)) != CONV3D_OK)
+      if ((st = launch_main(S, Fr, dy, nullptr, wt, nullptr, nullptr, ext, stream, split)) !=
+          CONV3D_OK)
         return st;
       if (D > 1) {
         Problem Bo = T;
@@ -1449,7 +1488,8 @@ size_t conv3d_bwd_data_workspace_bytes(int N, int Cin, int D, int H, int W, int 
     else
       ext = ((fold_bytes(Cout, Cin, kernel) + 255) & ~size_t(255)) + kPhaseSlack;
   }
-  return wt + ext;
+  if (tpad == CONV3D_TPAD_CAUSAL_CACHED) return wt;
+  return wt + ext + kSplitRegionBytes;
 }
 
 conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, int Cin, int D,
@@ -1460,11 +1500,13 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
   conv3d_status_t st = plan_bwd_data(dy, w, dx, N, Cin, D, H, W, Cout, kernel, stride, pad, tpad,
                                      dtype, B);
   if (st != CONV3D_OK) return st;
-  const size_t need = B.wt_bytes + B.ext_bytes;
+  const size_t need = B.wt_bytes + B.ext_bytes + B.split_bytes;
   if (workspace == nullptr || ws_bytes < need) {
     set_error("workspace of %zu bytes required", need);
     return CONV3D_ERR_WORKSPACE;
   }
+  // the launches that run as one partial wave of tiles split them along K here
+  const SplitRegion split{static_cast<char*>(workspace) + B.wt_bytes + B.ext_bytes, B.split_bytes};
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) {
     set_error("workspace must be 256-byte aligned");
     return CONV3D_ERR_ALIGNMENT;
@@ -1481,7 +1523,7 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
   DeviceState* S = nullptr;
   int dev = 0;
   if ((st = device_state(S, dev)) != CONV3D_OK) return st;
-  if (B.phased) return bwd_data_phases(*S, B, dy, w, dx, workspace, stream);
+  if (B.phased) return bwd_data_phases(*S, B, dy, w, dx, workspace, stream, &split);
   uint16_t* wt = static_cast<uint16_t*>(workspace);
   {
     const int taps = kernel[0] * kernel[1] * kernel[2];
@@ -1494,9 +1536,9 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
   }
   if (B.tr.fold)
     return run(B.tr, dy, wt, nullptr, nullptr, dx, static_cast<char*>(workspace) + B.wt_bytes,
-               B.ext_bytes, false, stream);
+               B.ext_bytes, false, stream, &split);
   if (!B.rep)
-    return launch_main(*S, B.tr, dy, nullptr, wt, nullptr, nullptr, dx, stream);
+    return launch_main(*S, B.tr, dy, nullptr, wt, nullptr, nullptr, dx, stream, &split);
 
   float* ext = reinterpret_cast<float*>(static_cast<char*>(workspace) + B.wt_bytes);
   const long long frame_elems = static_cast<long long>(H) * W * Cin;
@@ -1523,7 +1565,7 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
     if (e != cudaSuccess) return cuda_fail(e, "aux stream fork");
     front_stream = S->aux;
   }
-  st = launch_main(*S, B.front, dy, nullptr, wt, nullptr, nullptr, ext, front_stream);
+  st = launch_main(*S, B.front, dy, nullptr, wt, nullptr, nullptr, ext, front_stream, &split);
   if (st == CONV3D_OK && B.body.Do > 0) {
     const long long dy_frame = static_cast<long long>(B.fwd.Ho) * B.fwd.Wo * Cout;
     for (int n = 0; n < N && st == CONV3D_OK; ++n) {
