@@ -179,11 +179,14 @@ def test_workload_sampled(name, monkeypatch):
 
 
 @pytest.mark.parametrize("first", [CREP, CZERO])
-def test_chunked_decoding_equals_whole_clip(first, cta_mode):
+def test_chunked_decoding_equals_whole_clip(first, cta_mode, monkeypatch):
     """A clip convolved in one call equals the same clip convolved chunk by
     chunk (first chunk: the causal rule; later chunks: conv3d_fwd_cached with
     the previous chunk's last kt-1 input frames), bit for bit: every tile sums
-    the same products in the same order."""
+    the same products in the same order.  Without the tail split, which cuts
+    different tiles of the whole clip and of a chunk along K (the results then
+    differ only by the fp32 summation order of those tiles)."""
+    monkeypatch.setenv("CONV3D_SPLIT", "0")
     N, Cin, D, H, W, Cout = 1, 64, 9, 16, 20, 128
     p = problem(N, Cin, D, H, W, Cout, (3, 3, 3), (0, 1, 1), first, seed=51, residual=True)
     whole = run(p)

@@ -684,8 +684,8 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   kp.tiles_per_frame = (kp.HoWo + kp.pix_tile - 1) / kp.pix_tile;
   kp.num_tiles = P.N * P.Do * kp.tiles_per_frame * kp.n_tiles_n;
   // Tail split.  The persistent grid runs the tiles in rounds of one per SM;
-  // when the last round is at most half full (R tiles), the other SMs would
-  // idle through it.  Each of those R tiles is then cut into S pieces along K
+  // when the last round (or the only one) is at most half full (R tiles), the
+  // other SMs would idle through it.  Each of those R tiles is then cut into S pieces along K
   // (S <= SMs / R, at most 8, at least 8 k-blocks a piece), the pieces run
   // side by side on S*R SMs, and the piece that completes a tile adds up the
   // S fp32 partials (in piece order) before the usual epilogue: the last
@@ -701,10 +701,10 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   if (split_room > 0 && forced != 0 && !L.pair && !P.y_scatter) {
     const int U = S.num_sms;
     const int T = kp.num_tiles;
-    int R = T % U;
+    int R = T % U;                 // the last round (all of them for a single round)
     const int kb_nominal = kt_eff * P.kh * P.kw * kp.n_chunks;
-    if (forced > 0 && R == 0) R = T < U ? T : U;
-    if (forced > 0 || (T >= U && R > 0 && 2 * R <= U)) {
+    if (R == 0 && (forced > 0 || T < U)) R = T < U ? T : U;
+    if (forced > 0 || (R > 0 && 2 * R <= U)) {
       int sp = forced > 0 ? forced : U / R;
       if (forced < 0) {
         if (sp > 8) sp = 8;

@@ -294,17 +294,23 @@ __device__ void producer_finish(bool aborted, long long issued, bool skip_first,
 }
 
 // Ticket of one lane quarter of a split tail tile: counts, for this launch's
-// generation, the pieces whose partial is stored (an older generation counts
-// as none, so the tickets never need clearing).  True for the piece that
-// completes the quarter.  Each retry means another piece got in first, so at
-// most split_s attempts.
+// generation, the pieces whose partial is stored (a count of another
+// generation -- left by a launch that aborted -- counts as none).  True for
+// the piece that completes the quarter, which also resets the ticket to 0: no
+// other piece of the launch touches it afterwards, so a launch that runs again
+// with the same parameters (a CUDA graph replay) starts from zero.  Each
+// retry means another piece got in first, so at most split_s attempts.
 __device__ __forceinline__ bool take_ticket(unsigned long long* t, unsigned int gen, int pieces) {
   unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(t);
   for (;;) {
     const unsigned long long done = (cur >> 32) == gen ? (cur & 0xFFFFFFFFull) : 0ull;
     const unsigned long long next = (static_cast<unsigned long long>(gen) << 32) | (done + 1);
     const unsigned long long seen = atomicCAS(t, cur, next);
-    if (seen == cur) return done + 1 == static_cast<unsigned long long>(pieces);
+    if (seen == cur) {
+      const bool last = done + 1 == static_cast<unsigned long long>(pieces);
+      if (last) atomicExch(t, 0ull);
+      return last;
+    }
     cur = seen;
   }
 }
