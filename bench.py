@@ -952,13 +952,16 @@ def run_norm(args, wl, rank, world, local_rank):
 
 def run_gnblock(args, wl, rank, world, local_rank):
     """One decoder block (GroupNorm(32) + SiLU, then the workload's convolution)
-    timed three ways on the same inputs: `separate` = statistics pass, apply
-    pass (writes h) and conv3d_fwd(h); `fused` = statistics pass and
-    conv3d_fwd_gn (h never written); `chained` = conv3d_fwd_gn that also
-    gathers the GroupNorm statistics of its own output (what the next block
-    needs), with this block's statistics taken as given.  value = the chained
-    form's TFLOP/s; every form is parity-gated on sampled rows against the
-    oracle composition (GroupNorm + SiLU in fp64, one rounding, fp64 conv)."""
+    timed four ways on the same inputs: `separate` = statistics pass, apply
+    pass (writes h) and conv3d_fwd(h); `apply_conv_stats` = apply pass and a
+    convolution that gathers the GroupNorm statistics of its own output (what
+    the next block needs), this block's statistics coming from the previous
+    block's; `fused` = statistics pass and conv3d_fwd_gn with the transform in
+    the operand path (h never written); `chained` = the operand-path form that
+    also gathers its output's statistics.  value = the fastest form's TFLOP/s
+    (conv FLOPs over the block's time); every form is parity-gated on sampled
+    rows against the oracle composition (GroupNorm + SiLU in fp64, one
+    rounding, fp64 conv)."""
     import oracle
     import video_vae_convolution_implicit_b200 as c3
     dev = torch.device("cuda", local_rank)
@@ -994,7 +997,16 @@ def run_gnblock(args, wl, rank, world, local_rank):
         c3.conv3d_gn(x, stats, gamma, beta, p["w"], p["bias"], p["residual"], y, G,
                      out_groups=G, **kw)
 
-    forms = {"separate": (separate, 3), "fused": (fused, 2), "chained": (chained, 3)}
+    def apply_conv_stats():
+        # this block's statistics come from the previous block's epilogue; the
+        # convolution gathers the next block's in its own
+        c3.groupnorm_silu(x, stats, gamma, beta, h, G, False, True, stream)
+        c3.conv3d_gn(h, None, None, None, p["w"], p["bias"], p["residual"], y, out_groups=G,
+                     **kw)
+
+    # launches per step (stats clear and finalize included)
+    forms = {"separate": (separate, 3), "apply_conv_stats": (apply_conv_stats, 4),
+             "fused": (fused, 2), "chained": (chained, 4)}
     flops = algorithmic_flops(wl)
     res = {}
     if rank == 0:
@@ -1038,18 +1050,19 @@ def run_gnblock(args, wl, rank, world, local_rank):
                            "ok": bool(np.isfinite(got).all() and mr <= 1e-2 and rl <= 2e-3)}
         res[name] = r
     peaks, peak_kind = load_peaks()
-    conv_roof = roofline_for(flops, algorithmic_bytes(wl), res["chained"]["ms_per_step"], peaks,
+    best = min(res, key=lambda k: res[k]["ms_per_step"])
+    conv_roof = roofline_for(flops, algorithmic_bytes(wl), res[best]["ms_per_step"], peaks,
                              peak_kind)
     line = {
         "metric": "decoder block (GroupNorm+SiLU -> conv3d) TFLOPS, conv FLOPs over the block's time",
-        "value": res["chained"]["tflops"], "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["chained"]["ms_per_step"],
+        "value": res[best]["tflops"], "unit": "TFLOP/s", "n_gpus": world, "best_form": best,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res[best]["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
         "data": "synthetic (seeded SplitMix64 normals)",
         "config": dict(describe(wl, world), groupnorm_groups=G, l2="flushed between steps"),
-        "roofline": dict(conv_roof, kernel=KERNEL_NAME + " (GroupNorm variant)"),
+        "roofline": dict(conv_roof, kernel=KERNEL_NAME, timed="the whole block (every launch)"),
         "forms": res,
-        "gpu_launches": res["chained"]["gpu_launches"],
+        "gpu_launches": res[best]["gpu_launches"],
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -38,7 +38,7 @@ CASES = [
     # N, Cin, D, H, W, Cout, kernel, pad, dtype
     (1, 64, 4, 10, 12, 64, (3, 3, 3), (0, 1, 1), "bf16"),
     (2, 64, 3, 9, 13, 128, (3, 3, 3), (0, 1, 1), "bf16"),
-    (1, 32, 5, 8, 8, 48, (3, 3, 3), (1, 1, 1), "f16"),
+    (1, 32, 5, 8, 8, 48, (3, 3, 3), (0, 1, 1), "f16"),
     (1, 48, 3, 11, 10, 40, (2, 3, 3), (0, 0, 1), "bf16"),
     (1, 64, 1, 12, 12, 64, (3, 3, 3), (0, 1, 1), "bf16"),        # a one-frame chunk
     (1, 128, 2, 16, 16, 64, (1, 1, 1), (0, 0, 0), "bf16"),       # no cached frames

@@ -281,19 +281,23 @@ conv3d_status_t load_entry_points() {
 
 // A tensor map is a pure function of its encode arguments (address, sizes,
 // strides, box, traversal, swizzle), so a call that repeats an earlier call's
-// pointers and shape reuses the maps encoded then instead of asking the driver
-// again (3-5 encodes per launch).  Keyed by the raw argument bytes; at most
+// pointers and shape could reuse the maps encoded then instead of asking the
+// driver again (3-5 encodes per launch).  Measured on B200, host time per
+// conv3d_fwd call with / without this cache: 4.79 / 4.53 us (the small fp16
+// layer), 3.34 / 3.17 us (the 256-channel layer) -- the driver's encode is
+// cheaper than building and hashing the key -- so it is off unless
+// CONV3D_MAP_CACHE=1.  Keyed by the raw argument bytes; at most
 // kMapCacheEntries maps are kept (the cache is emptied when full) and
 // conv3d_release empties it.
 constexpr size_t kMapCacheEntries = 1024;
 std::mutex g_map_mu;
 std::unordered_map<std::string, CUtensorMap> g_map_cache;
 
-// CONV3D_MAP_CACHE=0 encodes every map afresh (for measuring the cache).
+// CONV3D_MAP_CACHE=1 turns the cache on.
 bool map_cache_on() {
   static const bool on = [] {
     const char* env = getenv("CONV3D_MAP_CACHE");
-    return env == nullptr || env[0] != '0';
+    return env != nullptr && env[0] == '1';
   }();
   return on;
 }
