@@ -387,7 +387,7 @@ struct DeviceState {
   };
   Scratch scratch[16] = {};
   int n_scratch = 0;
-  bool attr_set[16] = {};        // per kernel variant
+  bool attr_set[128] = {};       // per kernel instance (variant and features)
   int pair_clusters = 0;         // co-resident CTA pairs (occupancy query)
   int wg_pair_clusters = 0;      // the same for the weight-gradient kernel
   bool wg_attr_set[16] = {};     // per weight-gradient kernel variant
@@ -702,7 +702,7 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   L.split_bytes = 0;
   L.split_part_bytes = 0;
   const int forced = split_override();
-  if (split_room > 0 && forced != 0 && !L.pair && !P.y_scatter) {
+  if (split_room > 0 && forced != 0 && !L.pair && !P.y_scatter && !P.gn_stats && !P.gn_out) {
     const int U = S.num_sms;
     const int T = kp.num_tiles;
     int R = T % U;                 // the last round (all of them for a single round)
@@ -748,13 +748,14 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   return CONV3D_OK;
 }
 
-template <bool kBF16, bool kPair, bool kSwap, bool kGN = false>
+template <bool kBF16, bool kPair, bool kSwap, int kFeat = 0>
 conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtensorMap& map_a,
                               const CUtensorMap& map_b, const CUtensorMap& map_y,
                               const CUtensorMap& map_r, const CUtensorMap& map_p,
                               cudaStream_t stream) {
-  auto kern = conv3d_implicit_gemm_kernel<kBF16, kPair, kSwap, kGN>;
-  const int variant = (kBF16 ? 1 : 0) + (kPair ? 2 : 0) + (kSwap ? 4 : 0) + (kGN ? 8 : 0);
+  constexpr bool kGN = (kFeat & FEAT_GN) != 0;
+  auto kern = conv3d_implicit_gemm_kernel<kBF16, kPair, kSwap, kFeat>;
+  const int variant = (kBF16 ? 1 : 0) + (kPair ? 2 : 0) + (kSwap ? 4 : 0) + 8 * kFeat;
   const int threads = kGN ? GN_THREADS : NUM_THREADS;
   cudaError_t e;
   int units = S.num_sms;  // co-resident CTAs (or CTA pairs)
@@ -831,6 +832,30 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
   return CONV3D_OK;
 }
 
+// The one-CTA instances with optional parts: the tail split, the output
+// statistics, the strided output, the GroupNorm operand transform (with or
+// without the statistics).  The plan never combines the split with the others.
+template <bool kBF16, bool kSwap>
+conv3d_status_t launch_features(DeviceState& S, const LaunchPlan& L, int feat,
+                                const CUtensorMap& map_a, const CUtensorMap& map_b,
+                                const CUtensorMap& map_y, const CUtensorMap& map_r,
+                                const CUtensorMap& map_p, cudaStream_t stream) {
+  switch (feat) {
+    case FEAT_SPLIT:
+      return launch_kernel<kBF16, false, kSwap, FEAT_SPLIT>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+    case FEAT_STATS:
+      return launch_kernel<kBF16, false, kSwap, FEAT_STATS>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+    case FEAT_SCATTER:
+      return launch_kernel<kBF16, false, kSwap, FEAT_SCATTER>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+    case FEAT_GN:
+      return launch_kernel<kBF16, false, kSwap, FEAT_GN>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+    case FEAT_GN | FEAT_STATS:
+      return launch_kernel<kBF16, false, kSwap, FEAT_GN | FEAT_STATS>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+  }
+  set_error("internal: no kernel instance for feature set %d", feat);
+  return CONV3D_ERR_UNSUPPORTED;
+}
+
 // Launches the main kernel with a plan from plan_launch (whose split scratch,
 // if any, the caller has filled in).
 conv3d_status_t launch_planned(DeviceState& S, const Problem& P, LaunchPlan& L, const void* x,
@@ -858,12 +883,18 @@ conv3d_status_t launch_planned(DeviceState& S, const Problem& P, LaunchPlan& L, 
   } else {
     map_p = map_a;  // never read: no tap reads before frame 0 in this mode
   }
-  if (L.kp.gn_stats != nullptr) {   // GroupNorm + SiLU of x (never a CTA pair)
+  // the optional parts this launch needs (each combination is its own instance)
+  int feat = 0;
+  if (L.kp.split_s > 1) feat |= FEAT_SPLIT;
+  if (P.gn_out) feat |= FEAT_STATS;
+  if (P.y_scatter) feat |= FEAT_SCATTER;
+  if (P.gn_stats) feat |= FEAT_GN;
+  if (feat != 0) {   // never a CTA pair
     if (L.swap)
-      return bf16 ? launch_kernel<true, false, true, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream)
-                  : launch_kernel<false, false, true, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
-    return bf16 ? launch_kernel<true, false, false, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream)
-                : launch_kernel<false, false, false, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+      return bf16 ? launch_features<true, true>(S, L, feat, map_a, map_b, map_y, map_r, map_p, stream)
+                  : launch_features<false, true>(S, L, feat, map_a, map_b, map_y, map_r, map_p, stream);
+    return bf16 ? launch_features<true, false>(S, L, feat, map_a, map_b, map_y, map_r, map_p, stream)
+                : launch_features<false, false>(S, L, feat, map_a, map_b, map_y, map_r, map_p, stream);
   }
   if (L.swap)
     return bf16 ? launch_kernel<true, false, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream)

@@ -43,6 +43,15 @@ constexpr int BM = 128;             // output pixels per tile (TMEM lanes)
 constexpr int BK = 64;              // channels per k-block (128 bytes of fp16/bf16)
 constexpr int A_STAGE_BYTES = BM * BK * 2;
 constexpr int NUM_THREADS = 192;
+
+// Optional parts of the forward kernel, compiled into the instances that use
+// them only, so the plain convolution keeps a compact epilogue (measured: with
+// these paths behind run-time flags in one instance the 1x1x1 layer, whose
+// epilogue runs every 8 k-blocks, slowed from 159 to 260 us).
+constexpr int FEAT_SPLIT = 1;      // tail split: K pieces, partials, tickets
+constexpr int FEAT_STATS = 2;      // GroupNorm statistics of the output
+constexpr int FEAT_SCATTER = 4;    // strided output (data-gradient phases)
+constexpr int FEAT_GN = 8;         // GroupNorm + SiLU of the x operand (4 more warps)
 constexpr int GN_THREADS = 320;     // with the GroupNorm + SiLU operand transform (4 more warps)
 constexpr int MAX_STAGES = 8;
 
@@ -153,10 +162,11 @@ struct Work {
 
 __device__ __forceinline__ int kblocks_of_tile(const KernelParams& p, int to);
 
+template <bool kSplit>
 __device__ __forceinline__ Work decode_work(const KernelParams& p, int i) {
   Work w;
   int t = i, piece = -1;
-  if (i >= p.split_first) {
+  if (kSplit && i >= p.split_first) {
     const int j = i - p.split_first;
     const int q = j / p.split_s;
     t = p.split_first + q;
@@ -315,6 +325,14 @@ __device__ __forceinline__ bool take_ticket(unsigned long long* t, unsigned int 
   }
 }
 
+// A slot holds a 128-lane x BN-column fp32 accumulator as float4 groups
+// [column chunk j][group q of 4 columns][lane]: lane l's columns 32j + 4q ..
+// +3 are float4 number (j*8 + q)*128 + l, so each warp access covers 32
+// consecutive float4 (512 contiguous bytes).
+__device__ __forceinline__ float4* slot_at(const KernelParams& p, int slot) {
+  return reinterpret_cast<float4*>(p.part) + static_cast<size_t>(slot) * (BM / 4) * p.BN;
+}
+
 // Tail piece, for the calling warp's 32 TMEM lanes (lane row = quarter*32 +
 // lane): store the raw fp32 accumulator (BN columns per lane) in the piece's
 // slot, then take the quarter's ticket.  Returns true in every lane of the
@@ -323,18 +341,17 @@ __device__ __forceinline__ bool take_ticket(unsigned long long* t, unsigned int 
 // waited for), so an abort in another warp cannot hold this one.
 __device__ __forceinline__ bool store_piece(const KernelParams& p, int slot, uint32_t t_row,
                                             bool has_acc, uint32_t quarter, uint32_t lane) {
-  float4* dst = reinterpret_cast<float4*>(
-      p.part + (static_cast<size_t>(slot) * BM + quarter * 32u + lane) * p.BN);
+  float4* dst = slot_at(p, slot) + quarter * 32u + lane;
   for (int j = 0; j < p.BN / 32; ++j) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(t_row + j * 32, r);
     tmem_ld_wait();
 #pragma unroll
     for (int q = 0; q < 8; ++q)
-      dst[j * 8 + q] = has_acc ? make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                             __uint_as_float(r[4 * q + 2]),
-                                             __uint_as_float(r[4 * q + 3]))
-                               : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      dst[(j * 8 + q) * BM] =
+          has_acc ? make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]))
+                  : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   }
   __threadfence();
   __syncwarp();
@@ -355,11 +372,10 @@ __device__ __forceinline__ void sum_pieces(const KernelParams& p, int slot0, uin
 #pragma unroll
   for (int e = 0; e < 32; ++e) v[e] = 0.0f;
   for (int sp = 0; sp < p.split_s; ++sp) {
-    const float4* src = reinterpret_cast<const float4*>(
-        p.part + (static_cast<size_t>(slot0 + sp) * BM + lane_row) * p.BN + j * 32);
+    const float4* src = slot_at(p, slot0 + sp) + j * 8 * BM + lane_row;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const float4 a = __ldcg(src + q);
+      const float4 a = __ldcg(src + q * BM);
       v[4 * q] += a.x;
       v[4 * q + 1] += a.y;
       v[4 * q + 2] += a.z;
@@ -466,8 +482,8 @@ struct Cvt<false> {
 //   written to memory: rows that hold spatial padding stay zero (the padding
 //   belongs to the normalised tensor), and the tensor-core issuer waits for
 //   the transform of a stage instead of its load.
-template <bool kBF16, bool kPair, bool kSwap, bool kGN = false>
-__global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
+template <bool kBF16, bool kPair, bool kSwap, int kFeat = 0>
+__global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 1)
     conv3d_implicit_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                                 const __grid_constant__ CUtensorMap map_b,
                                 const __grid_constant__ CUtensorMap map_y,
@@ -480,6 +496,10 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
   __shared__ __align__(8) uint64_t s_peer_bar;      // pairs: the odd CTA's end-of-run report
   __shared__ unsigned long long s_peer_count;
 
+  constexpr bool kSplit = (kFeat & FEAT_SPLIT) != 0;
+  constexpr bool kStats = (kFeat & FEAT_STATS) != 0;
+  constexpr bool kScatter = (kFeat & FEAT_SCATTER) != 0;
+  constexpr bool kGN = (kFeat & FEAT_GN) != 0;
   constexpr int kCtas = kPair ? 2 : 1;
   const uint32_t warp = threadIdx.x / 32;
   const uint32_t lane = threadIdx.x % 32;
@@ -563,7 +583,7 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
       long long issued = 0;
       bool ok = true;
       for (int i = unit; ok && i < p.num_items; i += num_units) {
-        const Work wk = decode_work(p, i);
+        const Work wk = decode_work<kSplit>(p, i);
         const Tile& tl = wk.tl;
         int kb = 0;          // k-block index within the tile; the item issues [kb_lo, kb_hi)
         // first output pixel of this CTA's rows; rows past the frame are
@@ -636,7 +656,7 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
       bool ok = true;
       int local = 0;
       for (int i = unit; ok && i < p.num_items; i += num_units, ++local) {
-        const Work wk = decode_work(p, i);
+        const Work wk = decode_work<kSplit>(p, i);
         const int nkb = wk.kb_hi - wk.kb_lo;
         const uint32_t acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
@@ -709,7 +729,7 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
     uint32_t stage = 0, phase = 0;
     bool ok = true;
     for (int i = unit; ok && i < p.num_items; i += num_units) {
-      const Work wk = decode_work(p, i);
+      const Work wk = decode_work<kSplit>(p, i);
       const Tile& tl = wk.tl;
       // output pixel of each of this thread's rows (ho < 0: past the frame)
       int rho[kRows], rwo[kRows];
@@ -812,16 +832,16 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
     const int chunks = p.BN / 32;
     bool ok = true;
     GnOut gacc{0.0, 0.0, 0.0, 0.0, -1};
-    const int gn_cg = p.gn_out != nullptr ? p.Cout / p.gn_out_groups : 1;
+    const int gn_cg = kStats ? p.Cout / p.gn_out_groups : 1;
     if constexpr (kSwap) {
       // Thread = one output channel (TMEM lane), 32 pixels (columns) per chunk.
       for (int i = unit; ok && i < p.num_items; i += num_units, ++local) {
         const uint32_t acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
-        const Work wk = decode_work(p, i);
+        const Work wk = decode_work<kSplit>(p, i);
         const Tile& tl = wk.tl;
-        const bool piece = wk.slot >= 0;
-        if (p.gn_out != nullptr && tl.n != gacc.n) {
+        const bool piece = kSplit && wk.slot >= 0;
+        if (kStats && tl.n != gacc.n) {
           gn_out_flush(p.gn_out, p.gn_out_groups, gacc, lane);
           gacc.n = tl.n;
         }
@@ -857,17 +877,19 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
           const uint32_t t_row =
               tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.BN);
           bool from_parts = false;
-          if (piece) {
-            write_out = store_piece(p, wk.slot, t_row, has_acc, quarter, lane);
-            from_parts = write_out;
-            if (write_out && use_res) prefetch_residual();
+          if constexpr (kSplit) {
+            if (piece) {
+              write_out = store_piece(p, wk.slot, t_row, has_acc, quarter, lane);
+              from_parts = write_out;
+              if (write_out && use_res) prefetch_residual();
+            }
           }
           // byte offset of (pixel e, this thread's channel) in a 32 x 32 buffer
           const uint32_t col_byte = (lane & 7u) * 2u;
           for (int j = 0; write_out && j < live_chunks; ++j) {
             const uint32_t b = j & 1;
             float v[32];
-            if (from_parts) {
+            if (kSplit && from_parts) {
               sum_pieces(p, wk.slot - wk.slot % p.split_s, quarter * 32u + lane, j, v);
             } else {
               uint32_t r[32];
@@ -908,7 +930,7 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
                 asm volatile("st.shared.f32 [%0], %1;" ::"r"(yb + swz128(e, lane >> 2) + word),
                              "f"(v[e])
                              : "memory");
-            } else if (p.y_scatter != nullptr) {
+            } else if (kScatter) {
               // strided output: lane = channel, so each pixel's 32 channels are
               // one 64-byte store of the warp
               int q = tl.p0 + 32 * j;
@@ -934,13 +956,13 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
                 asm volatile("st.shared.u16 [%0], %1;" ::"r"(yb + swz64(e, lane >> 3) + col_byte),
                              "h"(q)
                              : "memory");
-                if (p.gn_out != nullptr && tl.p0 + 32 * j + e < p.HoWo) {
+                if (kStats && tl.p0 + 32 * j + e < p.HoWo) {
                   const float yv = C::lo(q);
                   gs += yv;
                   gq = fmaf(yv, yv, gq);
                 }
               }
-              if (p.gn_out != nullptr) {
+              if constexpr (kStats) {
                 // lane = channel ch: add its sums to its group's warp total
                 const int my_g = ch < p.Cout ? ch / gn_cg : -1;
                 const int g_last = (ch0 + 31 < p.Cout ? ch0 + 31 : p.Cout - 1) / gn_cg;
@@ -953,7 +975,7 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
             const int pix0 = tl.p0 + 32 * j;
             const bool refill = use_res && j + 2 < live_chunks;
             if (lane == 0) {
-              if (p.y_scatter == nullptr) {
+              if (!kScatter) {
                 tma_store_3d(&map_y, yb, ch0, pix0, tl.frame_out);
                 bulk_commit_group();
               }
@@ -979,10 +1001,10 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
     for (int i = unit; ok && i < p.num_items; i += num_units, ++local) {
       const uint32_t acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
-      const Work wk = decode_work(p, i);
+      const Work wk = decode_work<kSplit>(p, i);
       const Tile& tl = wk.tl;
-      const bool piece = wk.slot >= 0;
-      if (p.gn_out != nullptr && tl.n != gacc.n) {
+      const bool piece = kSplit && wk.slot >= 0;
+      if (kStats && tl.n != gacc.n) {
         gn_out_flush(p.gn_out, p.gn_out_groups, gacc, lane);
         gacc.n = tl.n;
       }
@@ -1014,15 +1036,17 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
         const uint32_t t_row =
             tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.BN);
         bool from_parts = false;
-        if (piece) {
-          write_out = store_piece(p, wk.slot, t_row, has_acc, quarter, lane);
-          from_parts = write_out;
-          if (write_out && use_res) prefetch_residual();
+        if constexpr (kSplit) {
+          if (piece) {
+            write_out = store_piece(p, wk.slot, t_row, has_acc, quarter, lane);
+            from_parts = write_out;
+            if (write_out && use_res) prefetch_residual();
+          }
         }
         for (int j = 0; write_out && rows_live && j < live_chunks; ++j) {
           const uint32_t b = j & 1;
           float v[32];
-          if (from_parts) {
+          if (kSplit && from_parts) {
             sum_pieces(p, wk.slot - wk.slot % p.split_s, quarter * 32u + lane, j, v);
           } else {
             uint32_t r[32];
@@ -1073,7 +1097,7 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int g = 0; g < 16; ++g) pk[g] = C::pack(v[2 * g], v[2 * g + 1]);
-            if (p.y_scatter != nullptr) {
+            if constexpr (kScatter) {
               // strided output: this thread's pixel, 32 channels as four 16-byte stores
               const int q = row_base + static_cast<int>(lane);
               if (q < p.HoWo) {
@@ -1093,7 +1117,7 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
                 st_shared_v4(ybuf + b * ybytes + swz64(lane, g), pk[4 * g], pk[4 * g + 1],
                              pk[4 * g + 2], pk[4 * g + 3]);
             }
-            if (p.gn_out != nullptr) {
+            if constexpr (kStats) {
               // this row's rounded outputs, per group of the chunk's channels
               const bool row_in = row_base + static_cast<int>(lane) < p.HoWo;
               const int c_end = p.Cout - cb < 32 ? p.Cout - cb : 32;
@@ -1118,7 +1142,7 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
           // every lane has read residual buffer b: refill it with chunk j+2
           const bool refill = use_res && j + 2 < live_chunks;
           if (lane == 0) {
-            if (p.y_scatter == nullptr) {
+            if (!kScatter) {
               tma_store_3d(&map_y, ybuf + b * ybytes, cb, row_base, tl.frame_out);
               bulk_commit_group();
             }
@@ -1146,7 +1170,7 @@ __global__ void __launch_bounds__(kGN ? GN_THREADS : NUM_THREADS, 1)
           mbar_arrive(tempty_bar + 8 * acc);
       }
     }
-    if (p.gn_out != nullptr) gn_out_flush(p.gn_out, p.gn_out_groups, gacc, lane);
+    if constexpr (kStats) gn_out_flush(p.gn_out, p.gn_out_groups, gacc, lane);
     // y stores must be complete (and their shared-memory sources read) before exit
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
