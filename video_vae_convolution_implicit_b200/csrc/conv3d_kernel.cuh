@@ -394,46 +394,53 @@ __device__ __forceinline__ float silu_fast(float z) {
   return fmaf(h, t, h);
 }
 
-// Output GroupNorm statistics of one epilogue warp: lane l keeps the fp64
-// {sum, sum of squares} of groups l and l + 32 of sample n.
-struct GnOut {
-  double s0, q0, s1, q1;
-  int n;   // sample being gathered, -1 for none yet
+// Output GroupNorm statistics, gathered by each epilogue warp for the
+// channels it meets: lane l keeps fp64 {sum, sum of squares} of channel
+// base + 32k + l for every 32-channel window k of the current tiles (the
+// single variant: a tile's BN channels, one window per 32-channel chunk; the
+// transposed variant: the warp's own 32 channels, one window).  A chunk adds
+// its fp32 partial (at most 32 values); the windows are reduced to their
+// groups and added to the global sums only when the sample or the channel
+// base changes, and at the end.
+struct GnAcc {
+  double s[8], q[8];
+  int n, co0;   // sample and channel base being gathered (n < 0: none)
 };
 
-// Warp totals of each lane's (s, q) for group g, kept by the lane owning g.
-__device__ __forceinline__ void gn_out_add(GnOut& a, int g, float s, float q, uint32_t lane) {
+// Adds the warp's sums of window k (channels c0 + lane) to the global sums of
+// their groups, then clears them.
+__device__ __forceinline__ void gn_flush_window(double* dst, int Cout, int cg, int c0, double& s,
+                                                double& q, uint32_t lane) {
+  const int c = c0 + static_cast<int>(lane);
+  const int my_g = c < Cout ? c / cg : -1;
+  const int g_last = (c0 + 31 < Cout ? c0 + 31 : Cout - 1) / cg;
+  for (int g = c0 / cg; g <= g_last; ++g) {
+    double ts = my_g == g ? s : 0.0, tq = my_g == g ? q : 0.0;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    s += __shfl_xor_sync(0xFFFFFFFFu, s, off);
-    q += __shfl_xor_sync(0xFFFFFFFFu, q, off);
-  }
-  if ((g & 31) == static_cast<int>(lane)) {
-    if (g < 32) {
-      a.s0 += s;
-      a.q0 += q;
-    } else {
-      a.s1 += s;
-      a.q1 += q;
+    for (int off = 16; off > 0; off >>= 1) {
+      ts += __shfl_xor_sync(0xFFFFFFFFu, ts, off);
+      tq += __shfl_xor_sync(0xFFFFFFFFu, tq, off);
+    }
+    if (lane == 0) {
+      atomicAdd(dst + 2 * g, ts);
+      atomicAdd(dst + 2 * g + 1, tq);
     }
   }
+  s = q = 0.0;
 }
 
-// Adds the warp's sums of its current sample to the global statistics.
-__device__ __forceinline__ void gn_out_flush(double* gn_out, int groups, GnOut& a,
-                                             uint32_t lane) {
+// Flushes every window of the accumulator (windows of 32 channels from a.co0,
+// or from a.co0 + base_off for the transposed variant's one window).
+__device__ __forceinline__ void gn_flush(double* gn_out, int groups, int Cout, GnAcc& a,
+                                         int windows, int base_off, uint32_t lane) {
   if (a.n >= 0) {
     double* dst = gn_out + static_cast<size_t>(a.n) * groups * 2;
-    if (static_cast<int>(lane) < groups) {
-      atomicAdd(dst + 2 * lane, a.s0);
-      atomicAdd(dst + 2 * lane + 1, a.q0);
-    }
-    if (static_cast<int>(lane) + 32 < groups) {
-      atomicAdd(dst + 2 * (lane + 32), a.s1);
-      atomicAdd(dst + 2 * (lane + 32) + 1, a.q1);
+    const int cg = Cout / groups;
+    for (int k = 0; k < windows; ++k) {
+      const int c0 = a.co0 + base_off + 32 * k;
+      if (c0 < Cout) gn_flush_window(dst, Cout, cg, c0, a.s[k], a.q[k], lane);
     }
   }
-  a.s0 = a.q0 = a.s1 = a.q1 = 0.0;
 }
 
 template <bool kBF16>
@@ -586,6 +593,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
         const Work wk = decode_work<kSplit>(p, i);
         const Tile& tl = wk.tl;
         int kb = 0;          // k-block index within the tile; the item issues [kb_lo, kb_hi)
+        const int kb_hi = kSplit ? wk.kb_hi : 0x7FFFFFFF;   // whole tiles: no bound to test
         // first output pixel of this CTA's rows; rows past the frame are
         // computed from any valid window origin and masked by the epilogue
         int row0 = tl.p0 + static_cast<int>(rank) * BM;
@@ -595,17 +603,17 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
         const int w_org = wo0 * p.sw - p.pw;   // window origin of the first pixel
         const int h_org = ho0 * p.sh - p.ph;
         const int co_b = tl.co0 + static_cast<int>(rank * b_rows);
-        for (int it = 0; ok && kb < wk.kb_hi && it < p.kt; ++it) {
+        for (int it = 0; ok && kb < kb_hi && it < p.kt; ++it) {
           const int f = source_frame(p, tl.to, it);
           if (f == kNoFrame) continue;
           // frames before the chunk come from the cached-frames tensor
           const CUtensorMap* xmap = f < 0 ? &map_p : &map_a;
           const int img = f < 0 ? tl.n * (p.kt - 1) + (p.kt - 1) + f : tl.n * p.D + f;
-          for (int ih = 0; ok && kb < wk.kb_hi && ih < p.kh; ++ih) {
-            for (int iw = 0; ok && kb < wk.kb_hi && iw < p.kw; ++iw) {
+          for (int ih = 0; ok && kb < kb_hi && ih < p.kh; ++ih) {
+            for (int iw = 0; ok && kb < kb_hi && iw < p.kw; ++iw) {
               const int tap = (it * p.kh + ih) * p.kw + iw;
-              for (int cc = 0; cc < p.n_chunks && kb < wk.kb_hi; ++cc) {
-                if (kb++ < wk.kb_lo) continue;   // an earlier piece's k-block
+              for (int cc = 0; cc < p.n_chunks && kb < kb_hi; ++cc) {
+                if (kSplit && kb++ < wk.kb_lo) continue;   // an earlier piece's k-block
                 if (!wait_bounded(empty_bar + 8 * stage, phase ^ 1, ctl, true)) {
                   ok = false;
                   break;
@@ -831,8 +839,16 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
     const uint4* bias4 = reinterpret_cast<const uint4*>(p.bias);
     const int chunks = p.BN / 32;
     bool ok = true;
-    GnOut gacc{0.0, 0.0, 0.0, 0.0, -1};
-    const int gn_cg = kStats ? p.Cout / p.gn_out_groups : 1;
+    GnAcc gacc;
+    if constexpr (kStats) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) gacc.s[k] = gacc.q[k] = 0.0;
+      gacc.n = -1;
+      gacc.co0 = 0;
+    }
+    // windows of the accumulator and their offset from the tile's channel base
+    const int gn_windows = kSwap ? 1 : p.BN / 32;
+    const int gn_off = kSwap ? static_cast<int>(quarter) * 32 : 0;
     if constexpr (kSwap) {
       // Thread = one output channel (TMEM lane), 32 pixels (columns) per chunk.
       for (int i = unit; ok && i < p.num_items; i += num_units, ++local) {
@@ -841,9 +857,10 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
         const Work wk = decode_work<kSplit>(p, i);
         const Tile& tl = wk.tl;
         const bool piece = kSplit && wk.slot >= 0;
-        if (kStats && tl.n != gacc.n) {
-          gn_out_flush(p.gn_out, p.gn_out_groups, gacc, lane);
+        if (kStats && (tl.n != gacc.n || tl.co0 != gacc.co0)) {
+          gn_flush(p.gn_out, p.gn_out_groups, p.Cout, gacc, gn_windows, gn_off, lane);
           gacc.n = tl.n;
+          gacc.co0 = tl.co0;
         }
         const int ch0 = tl.co0 + static_cast<int>(quarter) * 32;   // this warp's channels
         const bool warp_live = ch0 < p.Cout;
@@ -963,11 +980,9 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
                 }
               }
               if constexpr (kStats) {
-                // lane = channel ch: add its sums to its group's warp total
-                const int my_g = ch < p.Cout ? ch / gn_cg : -1;
-                const int g_last = (ch0 + 31 < p.Cout ? ch0 + 31 : p.Cout - 1) / gn_cg;
-                for (int g = ch0 / gn_cg; g <= g_last; ++g)
-                  gn_out_add(gacc, g, my_g == g ? gs : 0.0f, my_g == g ? gq : 0.0f, lane);
+                // lane = channel ch: its pixels' sums go to its own accumulator
+                gacc.s[0] += gs;
+                gacc.q[0] += gq;
               }
             }
             fence_proxy_async_shared();
@@ -1004,9 +1019,10 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
       const Work wk = decode_work<kSplit>(p, i);
       const Tile& tl = wk.tl;
       const bool piece = kSplit && wk.slot >= 0;
-      if (kStats && tl.n != gacc.n) {
-        gn_out_flush(p.gn_out, p.gn_out_groups, gacc, lane);
+      if (kStats && (tl.n != gacc.n || tl.co0 != gacc.co0)) {
+        gn_flush(p.gn_out, p.gn_out_groups, p.Cout, gacc, gn_windows, gn_off, lane);
         gacc.n = tl.n;
+        gacc.co0 = tl.co0;
       }
       const int row_base = tl.p0 + static_cast<int>(rank) * BM + static_cast<int>(quarter) * 32;
       const bool rows_live = row_base < p.HoWo;   // some of this warp's rows are in the frame
@@ -1118,23 +1134,25 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
                              pk[4 * g + 2], pk[4 * g + 3]);
             }
             if constexpr (kStats) {
-              // this row's rounded outputs, per group of the chunk's channels
-              const bool row_in = row_base + static_cast<int>(lane) < p.HoWo;
-              const int c_end = p.Cout - cb < 32 ? p.Cout - cb : 32;
-              const int g_last = (cb + c_end - 1) / gn_cg;
-              for (int g = cb / gn_cg; g <= g_last; ++g) {
-                const int e_lo = g * gn_cg - cb, e_hi = (g + 1) * gn_cg - cb;
-                float gs = 0.0f, gq = 0.0f;
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                  const float yv = (e & 1) ? C::hi(pk[e >> 1]) : C::lo(pk[e >> 1]);
-                  if (row_in && e >= e_lo && e < e_hi && e < c_end) {
-                    gs += yv;
-                    gq = fmaf(yv, yv, gq);
-                  }
-                }
-                gn_out_add(gacc, g, gs, gq, lane);
+              // lane = channel cb + lane: its column of the staged 32 x 32
+              // block (the rows inside the frame), read back from shared memory
+              __syncwarp();
+              int rows_in = p.HoWo - row_base;
+              if (rows_in > 32) rows_in = 32;
+              const uint32_t col = ybuf + b * ybytes + (lane & 7u) * 2u;
+              float gs = 0.0f, gq = 0.0f;
+              for (int e = 0; e < rows_in; ++e) {
+                uint16_t qv;
+                asm volatile("ld.shared.u16 %0, [%1];"
+                             : "=h"(qv)
+                             : "r"(col + swz64(static_cast<uint32_t>(e), lane >> 3))
+                             : "memory");
+                const float yv = C::lo(qv);
+                gs += yv;
+                gq = fmaf(yv, yv, gq);
               }
+              gacc.s[j] += gs;
+              gacc.q[j] += gq;
             }
           }
           fence_proxy_async_shared();
@@ -1170,7 +1188,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
           mbar_arrive(tempty_bar + 8 * acc);
       }
     }
-    if constexpr (kStats) gn_out_flush(p.gn_out, p.gn_out_groups, gacc, lane);
+    if constexpr (kStats) gn_flush(p.gn_out, p.gn_out_groups, p.Cout, gacc, gn_windows, gn_off, lane);
     // y stores must be complete (and their shared-memory sources read) before exit
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
