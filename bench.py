@@ -1004,9 +1004,26 @@ def run_gnblock(args, wl, rank, world, local_rank):
         c3.conv3d_gn(h, None, None, None, p["w"], p["bias"], p["residual"], y, out_groups=G,
                      **kw)
 
+    # the parts on their own, to decompose the forms
+    def stats_only():
+        c3.groupnorm_stats(x, G, 1e-6, False, stats, stream)
+
+    def apply_only():
+        c3.groupnorm_silu(x, stats, gamma, beta, h, G, False, True, stream)
+
+    def conv_only():
+        c3.conv3d_fwd(h, p["w"], p["bias"], p["residual"], y, wl.stride, wl.pad, wl.tpad,
+                      stream=stream)
+
+    def conv_stats_only():
+        c3.conv3d_gn(h, None, None, None, p["w"], p["bias"], p["residual"], y, out_groups=G,
+                     **kw)
+
     # launches per step (stats clear and finalize included)
     forms = {"separate": (separate, 3), "apply_conv_stats": (apply_conv_stats, 4),
              "fused": (fused, 2), "chained": (chained, 4)}
+    parts = {"stats": stats_only, "apply": apply_only, "conv": conv_only,
+             "conv_with_stats": conv_stats_only}
     flops = algorithmic_flops(wl)
     res = {}
     if rank == 0:
@@ -1049,6 +1066,20 @@ def run_gnblock(args, wl, rank, world, local_rank):
             r["parity"] = {"rows": int(rows.size), "max_err_over_max_ref": mr, "rel_l1": rl,
                            "ok": bool(np.isfinite(got).all() and mr <= 1e-2 and rl <= 2e-3)}
         res[name] = r
+    part_ms = {}
+    for name, fn in parts.items():
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        part_ms[name] = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev) / args.steps
     peaks, peak_kind = load_peaks()
     best = min(res, key=lambda k: res[k]["ms_per_step"])
     conv_roof = roofline_for(flops, algorithmic_bytes(wl), res[best]["ms_per_step"], peaks,
@@ -1062,6 +1093,7 @@ def run_gnblock(args, wl, rank, world, local_rank):
         "config": dict(describe(wl, world), groupnorm_groups=G, l2="flushed between steps"),
         "roofline": dict(conv_roof, kernel=KERNEL_NAME, timed="the whole block (every launch)"),
         "forms": res,
+        "parts_ms": part_ms,
         "gpu_launches": res[best]["gpu_launches"],
     }
     if rank == 0:
