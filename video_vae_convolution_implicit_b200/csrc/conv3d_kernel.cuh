@@ -74,9 +74,11 @@ struct KernelParams {
   int tiles_per_frame;               // ceil(HoWo / pix_tile)
   int num_tiles;
   // Tail split: tiles [split_first, num_tiles) are each cut into split_s
-  // pieces along K, so that the last, partly filled round of tiles spreads
-  // over the otherwise idle SMs.  Work items: tiles 0 .. split_first-1 whole,
-  // then split_s consecutive pieces per tail tile (num_items in all).
+  // pieces along K, so that the work of the last, partly filled round of
+  // tiles spreads over every SM.  Work items: split_s consecutive pieces per
+  // split tile first, then tiles 0 .. split_first-1 whole (num_items in all).
+  // The pieces run in the first round, so the epilogue that adds up their
+  // partials overlaps the whole tiles' main loops instead of ending the launch.
   int num_items;
   int split_first;
   int split_s;                       // 1: no tail split
@@ -166,11 +168,15 @@ template <bool kSplit>
 __device__ __forceinline__ Work decode_work(const KernelParams& p, int i) {
   Work w;
   int t = i, piece = -1;
-  if (kSplit && i >= p.split_first) {
-    const int j = i - p.split_first;
-    const int q = j / p.split_s;
-    t = p.split_first + q;
-    piece = j - q * p.split_s;
+  if (kSplit) {
+    const int pieces = (p.num_tiles - p.split_first) * p.split_s;
+    if (i < pieces) {
+      const int q = i / p.split_s;
+      t = p.split_first + q;
+      piece = i - q * p.split_s;
+    } else {
+      t = i - pieces;
+    }
   }
   w.tl = decode_tile(p, t);
   const int nkb = kblocks_of_tile(p, w.tl.to);
