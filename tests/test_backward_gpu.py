@@ -110,6 +110,27 @@ def test_bwd_weight_every_element(case, wgrad_variant):
     assert_close(db.double().cpu().numpy(), ref_db, "dbias " + str(case))
 
 
+@pytest.mark.parametrize("side", ["beside", "after"])
+@pytest.mark.parametrize("case", [WEIGHT_CASES[i] for i in (0, 1, 2, 4, 6, 8, 9)],
+                         ids=lambda c: "x".join(map(str, c[:6])) + f"-t{c[9]}-{c[10]}")
+def test_bwd_weight_bias_gradient_beside_and_after(case, side, monkeypatch):
+    # The bias-gradient pass runs on the aux stream beside the weight-gradient
+    # kernel (the default) or after it on the caller's stream
+    # (CONV3D_WGRAD_DBIAS_SIDE=0); either way dbias is the oracle's sum over
+    # every output pixel, and dw is unchanged.
+    monkeypatch.setenv("CONV3D_WGRAD_DBIAS_SIDE", "1" if side == "beside" else "0")
+    N, Cin, D, H, W, Cout, k, stride, pad, tpad, dt = case
+    x, w, dy, od = grads_problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=450 + Cout, dt=dt,
+                                 stride=stride)
+    dw, db = c3.conv3d_bwd_weight(x, dy, k, stride, pad, tpad)
+    assert c3.poll_status() == c3.Status.OK
+    ref_db = oracle.decode16(si.bits(dy), od).reshape(-1, Cout).sum(axis=0)
+    assert_close(db.double().cpu().numpy(), ref_db, f"dbias {case} {side}")
+    _, ref_dw, _ = oracle.conv3d_backward(si.bits(x), si.bits(w), si.bits(dy), od, k, stride,
+                                          pad, tpad)
+    assert_close(dw.double().cpu().numpy(), ref_dw, f"dw {case} {side}")
+
+
 # ------------------------------------------------------ full-size workloads, sampled
 
 from seeded_inputs.workloads import WORKLOADS  # noqa: E402

@@ -1015,7 +1015,7 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
       }
     }
     const int spatial_cin = P.kh * P.kw * P.Cin;
-    const long long total = static_cast<long long>(P.Cout) * spatial_cin;
+    const long long total = static_cast<long long>(P.Cout) * (spatial_cin / 8);   // 16-byte vectors
     int blocks = static_cast<int>((total + 255) / 256);
     if (blocks > 4 * S->num_sms) blocks = 4 * S->num_sms;
     if (bf16)
@@ -1224,7 +1224,7 @@ conv3d_status_t bwd_data_phases(DeviceState& S, const BwdDataPlan& B, const void
       uint16_t* wt = reinterpret_cast<uint16_t*>(wt_at);
       wt_at += static_cast<size_t>(Cin) * taps * Cout * 2;   // a multiple of 16 bytes
       {
-        const dim3 grid((Cin + 31) / 32, (Cout + 31) / 32, taps);
+        const dim3 grid((Cin + 63) / 64, (Cout + 63) / 64, taps);
         flip_transpose_weight_kernel<<<grid, dim3(32, 8), 0, stream>>>(
             static_cast<const uint16_t*>(w), wt, Cout, taps, Cin, kh, kw, Jh, Jw, qh, qw, sh, sw);
         cudaError_t e = cudaGetLastError();
@@ -1565,7 +1565,7 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
   uint16_t* wt = static_cast<uint16_t*>(workspace);
   {
     const int taps = kernel[0] * kernel[1] * kernel[2];
-    const dim3 grid((Cin + 31) / 32, (Cout + 31) / 32, taps);
+    const dim3 grid((Cin + 63) / 64, (Cout + 63) / 64, taps);
     flip_transpose_weight_kernel<<<grid, dim3(32, 8), 0, stream>>>(
         static_cast<const uint16_t*>(w), wt, Cout, taps, Cin, kernel[1], kernel[2], kernel[1],
         kernel[2], 0, 0, 1, 1);
@@ -1845,6 +1845,22 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
   }
   cudaError_t e = cudaMemsetAsync(workspace, 0, need, stream);
   if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
+  // The bias gradient reads dy once more.  Its kernel uses no shared memory,
+  // so its blocks fit beside the weight-gradient CTAs, and it runs on the aux
+  // stream at the same time (forked after the clear, joined before the
+  // rounding); CONV3D_WGRAD_DBIAS_SIDE=0 runs it after the kernel instead.
+  bool side = false;
+  if (dbias) {
+    const char* env = getenv("CONV3D_WGRAD_DBIAS_SIDE");
+    side = (env == nullptr || env[0] != '0') && aux_stream(*S, stream);
+  }
+  std::unique_lock<std::mutex> aux_lock;
+  if (side) {
+    aux_lock = std::unique_lock<std::mutex>(g_aux_mu);
+    e = cudaEventRecord(S->aux_fork, stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(S->aux, S->aux_fork, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "aux stream fork");
+  }
   {
     const int grid_units = wp.num_units < lanes ? wp.num_units : lanes;
     cudaLaunchConfig_t cfg = {};
@@ -1885,23 +1901,33 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dw conversion launch");
   }
   if (dbias) {
-    // channel groups of up to 2048 along y; about four blocks per SM in all,
-    // the pixels split evenly between the blocks of a group
+    // 256-channel groups along y; about three blocks per SM in all (as many
+    // as fit beside a weight-gradient CTA), the pixels split evenly between
+    // the blocks of a group
     const long long pixels = static_cast<long long>(N) * F.Do * F.Ho * F.Wo;
     const int groups = (Cout + BIAS_CHANNELS - 1) / BIAS_CHANNELS;
-    long long blocks = (4LL * S->num_sms + groups - 1) / groups;
+    long long blocks = (3LL * S->num_sms + groups - 1) / groups;
     long long per = (pixels + blocks - 1) / blocks;
     if (per < 64) per = 64;
     blocks = (pixels + per - 1) / per;
     const dim3 grid(static_cast<unsigned>(blocks), static_cast<unsigned>(groups));
-    const size_t part_bytes = BIAS_THREADS * 8 * sizeof(float);
+    cudaStream_t bs = side ? S->aux : stream;
     if (bf16)
-      bias_grad_kernel<true><<<grid, BIAS_THREADS, part_bytes, stream>>>(
-          static_cast<const uint16_t*>(dy), db32, pixels, Cout, per);
+      bias_grad_kernel<true><<<grid, BIAS_THREADS, 0, bs>>>(static_cast<const uint16_t*>(dy),
+                                                              db32, pixels, Cout, per);
     else
-      bias_grad_kernel<false><<<grid, BIAS_THREADS, part_bytes, stream>>>(
-          static_cast<const uint16_t*>(dy), db32, pixels, Cout, per);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dbias launch");
+      bias_grad_kernel<false><<<grid, BIAS_THREADS, 0, bs>>>(static_cast<const uint16_t*>(dy),
+                                                               db32, pixels, Cout, per);
+    cudaError_t le = cudaGetLastError();
+    if (side) {
+      // join even after a failed launch, so the caller's stream never runs
+      // ahead of work left on the aux stream
+      e = cudaEventRecord(S->aux_join, S->aux);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, S->aux_join, 0);
+      aux_lock.unlock();
+      if (e != cudaSuccess) return cuda_fail(e, "aux stream join");
+    }
+    if (le != cudaSuccess) return cuda_fail(le, "dbias launch");
     if (bf16)
       f32_to_16_kernel<true><<<1, 256, 0, stream>>>(db32, static_cast<uint16_t*>(dbias), Cout);
     else
@@ -1982,7 +2008,7 @@ conv3d_status_t conv3d_bwd_data_cached(const void* dy, const void* w, void* dx, 
   uint16_t* wt = static_cast<uint16_t*>(workspace);
   {
     const int taps = kernel[0] * kernel[1] * kernel[2];
-    const dim3 grid((Cin + 31) / 32, (Cout + 31) / 32, taps);
+    const dim3 grid((Cin + 63) / 64, (Cout + 63) / 64, taps);
     flip_transpose_weight_kernel<<<grid, dim3(32, 8), 0, stream>>>(
         static_cast<const uint16_t*>(w), wt, Cout, taps, Cin, kernel[1], kernel[2], kernel[1],
         kernel[2], 0, 0, 1, 1);

@@ -1229,20 +1229,29 @@ __global__ void fold_temporal_taps_kernel(const uint16_t* __restrict__ w, uint16
   using C = Cvt<kBF16>;
   // the convolution that reads w2 waits for this whole grid before reading
   griddep_launch_dependents();
-  const long long total = static_cast<long long>(Cout) * spatial_cin;
+  // thread = 8 consecutive entries (16 bytes) of one output channel's row:
+  // spatial_cin is a multiple of 8 and both weights are 16-byte aligned
+  const int vecs = spatial_cin / 8;
+  const long long total = static_cast<long long>(Cout) * vecs;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long co = i / spatial_cin;
-    const long long rest = i - co * spatial_cin;
-    float s = 0.0f;
+    const long long co = i / vecs;
+    const long long rest = (i - co * vecs) * 8;
+    float s[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     for (int it = 0; it < kt; ++it) {
-      const uint32_t v = w[(co * kt + it) * spatial_cin + rest];
-      s += C::lo(v);
+      const uint4 v = *reinterpret_cast<const uint4*>(w + (co * kt + it) * spatial_cin + rest);
+      s[0] += C::lo(v.x); s[1] += C::hi(v.x); s[2] += C::lo(v.y); s[3] += C::hi(v.y);
+      s[4] += C::lo(v.z); s[5] += C::hi(v.z); s[6] += C::lo(v.w); s[7] += C::hi(v.w);
     }
-    const uint32_t hi = C::pack(s, 0.0f) & 0xFFFFu;
-    const uint32_t lo = C::pack(s - C::lo(hi), 0.0f) & 0xFFFFu;
-    w2[co * 2 * spatial_cin + rest] = static_cast<uint16_t>(hi);
-    w2[co * 2 * spatial_cin + spatial_cin + rest] = static_cast<uint16_t>(lo);
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      hi[q] = C::pack(s[2 * q], s[2 * q + 1]);
+      lo[q] = C::pack(s[2 * q] - C::lo(hi[q]), s[2 * q + 1] - C::hi(hi[q]));
+    }
+    *reinterpret_cast<uint4*>(w2 + co * 2 * spatial_cin + rest) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(w2 + co * 2 * spatial_cin + spatial_cin + rest) =
+        make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
 }
 
@@ -1250,9 +1259,9 @@ __global__ void fold_temporal_taps_kernel(const uint16_t* __restrict__ w, uint16
 // wt[ci, it, ih, iw, co] = w[co, kt-1-it, kh-1-ih, kw-1-iw, ci] (every tap
 // mirrored, the channel roles exchanged).  Mirroring all three tap indices
 // reverses the linear tap order, so each tap is a [Cout x Cin] -> [Cin x Cout]
-// transpose: block = one tap and a 32 x 32 tile, staged in shared memory so
+// transpose: block = one tap and a 64 x 64 tile, staged in shared memory so
 // that both the reads and the writes run along contiguous channels.
-// Launch: grid (ceil(Cin/32), ceil(Cout/32), taps), block (32, 8).
+// Launch: grid (ceil(Cin/64), ceil(Cout/64), taps), block (32, 8).
 //
 // With a spatial stride the data gradient splits into phases (rh, rw): dx rows
 // a*sh + rh receive only the taps ih = qh + sh*j (qh = (rh + ph) mod sh), so a
@@ -1264,23 +1273,28 @@ __global__ void flip_transpose_weight_kernel(const uint16_t* __restrict__ w,
                                              uint16_t* __restrict__ wt, int Cout, int taps,
                                              int Cin, int kh, int kw, int Jh, int Jw, int qh,
                                              int qw, int sh, int sw) {
-  __shared__ uint16_t tile[32][33];
-  const int ci0 = blockIdx.x * 32, co0 = blockIdx.y * 32;
+  // 64 x 64 tile, two 16-bit values (4 bytes) per thread access: Cin and Cout
+  // are even, so a pair never straddles the end of a row
+  __shared__ __align__(4) uint16_t tile[64][66];    // [co][ci], 33-word rows
+  const int ci0 = blockIdx.x * 64, co0 = blockIdx.y * 64;
   const int tap = blockIdx.z;                  // tap of wt: (it', jh', jw')
   const int jw_ = tap % Jw, jh_ = (tap / Jw) % Jh, it_ = tap / (Jw * Jh);
   const int kt = taps / (Jh * Jw);
   const int tap_src = ((kt - 1 - it_) * kh + qh + sh * (Jh - 1 - jh_)) * kw + qw + sw * (Jw - 1 - jw_);
   const int taps_src = kt * kh * kw;
-  for (int r = threadIdx.y; r < 32; r += 8) {
-    const int co = co0 + r, ci = ci0 + threadIdx.x;
+  const int x2 = 2 * static_cast<int>(threadIdx.x);
+  for (int r = threadIdx.y; r < 64; r += 8) {
+    const int co = co0 + r, ci = ci0 + x2;
     if (co < Cout && ci < Cin)
-      tile[r][threadIdx.x] = w[(static_cast<long long>(co) * taps_src + tap_src) * Cin + ci];
+      *reinterpret_cast<uint32_t*>(&tile[r][x2]) = *reinterpret_cast<const uint32_t*>(
+          w + (static_cast<long long>(co) * taps_src + tap_src) * Cin + ci);
   }
   __syncthreads();
-  for (int r = threadIdx.y; r < 32; r += 8) {
-    const int ci = ci0 + r, co = co0 + threadIdx.x;
+  for (int r = threadIdx.y; r < 64; r += 8) {
+    const int ci = ci0 + r, co = co0 + x2;
     if (co < Cout && ci < Cin)
-      wt[(static_cast<long long>(ci) * taps + tap) * Cout + co] = tile[threadIdx.x][r];
+      *reinterpret_cast<uint32_t*>(wt + (static_cast<long long>(ci) * taps + tap) * Cout + co) =
+          static_cast<uint32_t>(tile[x2][r]) | (static_cast<uint32_t>(tile[x2 + 1][r]) << 16);
   }
 }
 

@@ -556,59 +556,62 @@ __global__ void f32_to_16_bcast_kernel(const float* __restrict__ src, uint16_t* 
   }
 }
 
-// dbias[co] += sum over pixels of dy[m, co].  Block = a slab of pixels and
-// up to 2048 channels (blockIdx.y picks the group); thread = 8 channels (one
-// 16-byte load) of every rows-th pixel of the slab, four loads in flight.  The
-// block's rows are then reduced in shared memory and each channel takes one
-// atomic per block.  256 threads, 8 KB of dynamic shared memory.
+// dbias[co] += sum over pixels of dy[m, co], with no shared memory, so that its
+// blocks fit beside a weight-gradient CTA on every SM and the two run at once.
+// Block = 8 warps over a slab of pixels and up to 256 channels (blockIdx.y
+// picks the group); lane = 8 v + r of warp w covers the 16-byte vector
+// (8 channels) 4w + v of pixel rows r, r + 8, ... of the slab, eight loads in
+// flight (a warp reads 64 contiguous bytes of each of eight rows).  The eight
+// row lanes are added with shuffles, then lanes r = 0 add their 8 sums to db
+// with two 16-byte reductions.
 constexpr int BIAS_THREADS = 256;
-constexpr int BIAS_CHANNELS = 2048;
+constexpr int BIAS_CHANNELS = 256;
 
 template <bool kBF16>
 __global__ void __launch_bounds__(BIAS_THREADS) bias_grad_kernel(
     const uint16_t* __restrict__ dy, float* __restrict__ db, long long pixels, int Cout,
     long long pixels_per_block) {
   using C = Cvt<kBF16>;
-  extern __shared__ float s_part[];                 // [rows][channels of the group]
-  const int c0 = blockIdx.y * BIAS_CHANNELS;
-  const int cb = Cout - c0 < BIAS_CHANNELS ? Cout - c0 : BIAS_CHANNELS;
-  const int vecs = cb / 8;
-  const int rows = BIAS_THREADS / vecs;
-  const int v = threadIdx.x % vecs;
-  const int r = threadIdx.x / vecs;
+  const int lane = threadIdx.x & 31;
+  const int vec = 4 * (threadIdx.x >> 5) + (lane >> 3);    // 16-byte vector of the group
+  const int r = lane & 7;
+  const int c = blockIdx.y * BIAS_CHANNELS + 8 * vec;      // first channel of the vector
+  const bool live = c < Cout;
   const long long p_begin = blockIdx.x * pixels_per_block;
   long long p_end = p_begin + pixels_per_block;
   if (p_end > pixels) p_end = pixels;
-  if (r < rows) {
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    const long long stride = Cout / 8;              // 16-byte vectors per pixel
-    const uint4* src = reinterpret_cast<const uint4*>(dy) + c0 / 8 + v;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (live) {
+    const long long stride = Cout / 8;                     // 16-byte vectors per pixel
+    const uint4* src = reinterpret_cast<const uint4*>(dy) + c / 8;
     long long p = p_begin + r;
-    for (; p + 3 * rows < p_end; p += 4 * rows) {
-      uint4 q[4];
+    for (; p + 56 < p_end; p += 64) {
+      uint4 q[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) q[u] = __ldg(src + (p + u * rows) * stride);
+      for (int u = 0; u < 8; ++u) q[u] = __ldg(src + (p + 8 * u) * stride);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         acc[0] += C::lo(q[u].x); acc[1] += C::hi(q[u].x);
         acc[2] += C::lo(q[u].y); acc[3] += C::hi(q[u].y);
         acc[4] += C::lo(q[u].z); acc[5] += C::hi(q[u].z);
         acc[6] += C::lo(q[u].w); acc[7] += C::hi(q[u].w);
       }
     }
-    for (; p < p_end; p += rows) {
+    for (; p < p_end; p += 8) {
       const uint4 q = __ldg(src + p * stride);
       acc[0] += C::lo(q.x); acc[1] += C::hi(q.x); acc[2] += C::lo(q.y); acc[3] += C::hi(q.y);
       acc[4] += C::lo(q.z); acc[5] += C::hi(q.z); acc[6] += C::lo(q.w); acc[7] += C::hi(q.w);
     }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) s_part[r * cb + 8 * v + j] = acc[j];
   }
-  __syncthreads();
-  for (int c = threadIdx.x; c < cb; c += BIAS_THREADS) {
-    float t = 0.0f;
-    for (int q = 0; q < rows; ++q) t += s_part[q * cb + c];
-    atomicAdd(db + c0 + c, t);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    acc[e] += __shfl_xor_sync(0xFFFFFFFFu, acc[e], 1);
+    acc[e] += __shfl_xor_sync(0xFFFFFFFFu, acc[e], 2);
+    acc[e] += __shfl_xor_sync(0xFFFFFFFFu, acc[e], 4);
+  }
+  if (live && r == 0) {
+    red_add_v4(db + c, acc[0], acc[1], acc[2], acc[3]);
+    red_add_v4(db + c + 4, acc[4], acc[5], acc[6], acc[7]);
   }
 }
 
