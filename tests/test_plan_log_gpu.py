@@ -38,10 +38,12 @@ def test_plan_log_reports_each_launch():
     r = _run(True)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stderr.splitlines() if l.startswith("libconv3d: ")]
-    # forward, then the data gradient (its plan line, front and body launches),
-    # then the weight gradient
+    # forward, then the data gradient (its plan line and its one launch), then
+    # the weight gradient
     assert any("implicit GEMM" in l and "16-bit output" in l for l in lines), lines
-    assert any("implicit GEMM" in l and "fp32 output" in l for l in lines), lines
+    # the data gradient's launch: the fp32 parts of frame 0 beside the 16-bit frames
+    assert any("implicit GEMM" in l and "fp32 (front frames) and 16-bit output" in l
+               for l in lines), lines
     assert any(l.startswith("libconv3d: data gradient: 3 front frames") for l in lines), lines
     assert any(l.startswith("libconv3d: weight gradient") for l in lines), lines
 

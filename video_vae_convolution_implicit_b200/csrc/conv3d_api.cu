@@ -86,6 +86,13 @@ struct Problem {
   conv3d_dtype_t dtype;
   bool has_residual;
   bool out_f32;      // write y in fp32 (internal: the backward pass's padded-frame gradient)
+  // mixed output (internal: the data gradient under causal replicate padding):
+  // output frames 0 .. f32_frames-1 of each sample, the fp32 parts of dx
+  // frame 0, go to f32_out ([N][f32_frames][Ho][Wo][Cout]); frame to >=
+  // f32_frames is frame to - f32_frames + 1 of y ([N][y_frames][Ho][Wo][Cout])
+  int f32_frames;
+  int y_frames;
+  void* f32_out;
   const void* prev;  // cached frames before the chunk (CONV3D_TPAD_CAUSAL_CACHED) or null
   bool fold;  // first-frame path: fold the temporal taps into a (hi, lo) pair
   // GroupNorm + SiLU applied to x as it is read (conv3d_fwd_gn); gn_stats null otherwise
@@ -238,6 +245,9 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
   P.gn_out_groups = 0;
   P.exact_out = false;
   P.y_scatter = nullptr;
+  P.f32_frames = 0;
+  P.y_frames = 0;
+  P.f32_out = nullptr;
   P.sc_sh = P.sc_sw = 1;
   P.sc_rh = P.sc_rw = 0;
   P.sc_H = P.sc_W = 0;
@@ -538,15 +548,16 @@ conv3d_status_t encode_maps(const Problem& P, const void* x, const void* wmat, i
 // channels x 32 pixels of one frame, 64-byte swizzled.  Stores clip pixels
 // past the frame and channels past Cout; loads read them as zero.
 conv3d_status_t encode_out_map(const Problem& P, const void* base, CUtensorMap& map,
-                               bool f32 = false) {
+                               bool f32 = false, long long frames = -1) {
   const CUtensorMapDataType dt =
       f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
           : (P.dtype == CONV3D_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
   const cuuint64_t esize = f32 ? 4 : 2;
   const cuuint64_t howo = static_cast<cuuint64_t>(P.Ho) * P.Wo;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(P.Cout), howo,
-                              static_cast<cuuint64_t>(P.N) * static_cast<cuuint64_t>(P.Do)};
+  const cuuint64_t nframes = frames >= 0 ? static_cast<cuuint64_t>(frames)
+                                          : static_cast<cuuint64_t>(P.N) * static_cast<cuuint64_t>(P.Do);
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(P.Cout), howo, nframes};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(P.Cout) * esize, howo * P.Cout * esize};
   const cuuint32_t box[3] = {32, 32, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
@@ -629,6 +640,8 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   kp.ph = P.ph;
   kp.pw = P.pw;
   kp.tpad = P.fold ? 1 : static_cast<int>(P.tpad);
+  kp.f32_frames = P.f32_frames;
+  kp.y_frames = P.y_frames;
   kp.gn_stats = P.gn_stats;
   kp.gn_gamma = static_cast<const uint16_t*>(P.gn_gamma);
   kp.gn_beta = static_cast<const uint16_t*>(P.gn_beta);
@@ -674,7 +687,7 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
     if (env[0] == '1') L.pair = true;
   }
   if (L.swap) L.pair = false;
-  if (P.out_f32) L.pair = false;
+  if (P.out_f32 || P.f32_frames > 0) L.pair = false;
   if (P.gn_stats || P.gn_out || P.y_scatter) L.pair = false;   // one-CTA variants only   // the fp32 epilogue exists in the single and transposed variants
   const int ctas = L.pair ? 2 : 1;
   if (L.swap) {
@@ -734,7 +747,7 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   const int stage_bytes = A_STAGE_BYTES + b_stage;
   kp.has_residual = P.has_residual ? 1 : 0;
   kp.out_f32 = P.out_f32 ? 1 : 0;
-  const int reserve = 1024 /*alignment slack*/ + EPI_Y_BYTES * (kp.out_f32 ? 2 : 1) +
+  const int reserve = 1024 /*alignment slack*/ + EPI_Y_BYTES * (kp.out_f32 || kp.f32_frames ? 2 : 1) +
                       EPI_Y_BYTES * (kp.has_residual ? 1 : 0) +
                       8 * (3 * MAX_STAGES + 5 + 2 * EPI_WARPS);
   int stages = (S.max_smem_optin - reserve - 64 /*static smem*/) / stage_bytes;
@@ -755,7 +768,7 @@ template <bool kBF16, bool kPair, bool kSwap, int kFeat = 0>
 conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtensorMap& map_a,
                               const CUtensorMap& map_b, const CUtensorMap& map_y,
                               const CUtensorMap& map_r, const CUtensorMap& map_p,
-                              cudaStream_t stream) {
+                              const CUtensorMap& map_f, cudaStream_t stream) {
   constexpr bool kGN = (kFeat & FEAT_GN) != 0;
   auto kern = conv3d_implicit_gemm_kernel<kBF16, kPair, kSwap, kFeat>;
   const int variant = (kBF16 ? 1 : 0) + (kPair ? 2 : 0) + (kSwap ? 4 : 0) + 8 * kFeat;
@@ -825,10 +838,11 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
             kGN ? " with GroupNorm+SiLU of x" : "", kBF16 ? "bf16" : "fp16",
             L.kp.num_tiles, L.kp.pix_tile, L.kp.co_tile, static_cast<int>(cfg.gridDim.x),
             L.kp.n_chunks, L.kp.kt * L.kp.kh * L.kp.kw, L.kp.stages, L.smem,
-            L.kp.out_f32 ? "fp32" : "16-bit", L.kp.num_tiles - L.kp.split_first, L.kp.split_s);
+            L.kp.out_f32 ? "fp32" : L.kp.f32_frames ? "fp32 (front frames) and 16-bit" : "16-bit",
+            L.kp.num_tiles - L.kp.split_first, L.kp.split_s);
   KernelParams kp = L.kp;
   kp.test_stall = take_stall(kp.timeout_ns) ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, kern, map_a, map_b, map_y, map_r, map_p, kp);
+  e = cudaLaunchKernelEx(&cfg, kern, map_a, map_b, map_y, map_r, map_p, map_f, kp);
   if (e != cudaSuccess) return cuda_fail(e, "conv3d kernel launch");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "conv3d kernel launch");
@@ -842,18 +856,19 @@ template <bool kBF16, bool kSwap>
 conv3d_status_t launch_features(DeviceState& S, const LaunchPlan& L, int feat,
                                 const CUtensorMap& map_a, const CUtensorMap& map_b,
                                 const CUtensorMap& map_y, const CUtensorMap& map_r,
-                                const CUtensorMap& map_p, cudaStream_t stream) {
+                                const CUtensorMap& map_p, const CUtensorMap& map_f,
+                                cudaStream_t stream) {
   switch (feat) {
     case FEAT_SPLIT:
-      return launch_kernel<kBF16, false, kSwap, FEAT_SPLIT>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+      return launch_kernel<kBF16, false, kSwap, FEAT_SPLIT>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_STATS:
-      return launch_kernel<kBF16, false, kSwap, FEAT_STATS>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+      return launch_kernel<kBF16, false, kSwap, FEAT_STATS>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_SCATTER:
-      return launch_kernel<kBF16, false, kSwap, FEAT_SCATTER>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+      return launch_kernel<kBF16, false, kSwap, FEAT_SCATTER>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_GN:
-      return launch_kernel<kBF16, false, kSwap, FEAT_GN>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+      return launch_kernel<kBF16, false, kSwap, FEAT_GN>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_GN | FEAT_STATS:
-      return launch_kernel<kBF16, false, kSwap, FEAT_GN | FEAT_STATS>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+      return launch_kernel<kBF16, false, kSwap, FEAT_GN | FEAT_STATS>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
   }
   set_error("internal: no kernel instance for feature set %d", feat);
   return CONV3D_ERR_UNSUPPORTED;
@@ -868,11 +883,20 @@ conv3d_status_t launch_planned(DeviceState& S, const Problem& P, LaunchPlan& L, 
   conv3d_status_t st = CONV3D_OK;
   L.kp.bias = bias;
   L.kp.status = S.status;
-  CUtensorMap map_a, map_b, map_y, map_r, map_p;
+  CUtensorMap map_a, map_b, map_y, map_r, map_p, map_f;
   st = L.swap ? encode_maps(P, x, wmat, L.kp.kt, L.kp.co_tile, L.kp.pix_tile, map_a, map_b)
               : encode_maps(P, x, wmat, L.kp.kt, L.kp.BN / (L.pair ? 2 : 1), BM, map_a, map_b);
   if (st != CONV3D_OK) return st;
-  if ((st = encode_out_map(P, y, map_y, P.out_f32)) != CONV3D_OK) return st;
+  if (P.f32_frames > 0) {
+    // mixed output: the fp32 front frames and the 16-bit frames after them
+    const long long n = P.N;
+    if ((st = encode_out_map(P, y, map_y, false, n * P.y_frames)) != CONV3D_OK) return st;
+    if ((st = encode_out_map(P, P.f32_out, map_f, true, n * P.f32_frames)) != CONV3D_OK)
+      return st;
+  } else {
+    if ((st = encode_out_map(P, y, map_y, P.out_f32)) != CONV3D_OK) return st;
+    map_f = map_y;  // never written: f32_frames == 0
+  }
   if (residual) {
     if ((st = encode_out_map(P, residual, map_r)) != CONV3D_OK) return st;
   } else {
@@ -894,19 +918,19 @@ conv3d_status_t launch_planned(DeviceState& S, const Problem& P, LaunchPlan& L, 
   if (P.gn_stats) feat |= FEAT_GN;
   if (feat != 0) {   // never a CTA pair
     if (L.swap)
-      return bf16 ? launch_features<true, true>(S, L, feat, map_a, map_b, map_y, map_r, map_p, stream)
-                  : launch_features<false, true>(S, L, feat, map_a, map_b, map_y, map_r, map_p, stream);
-    return bf16 ? launch_features<true, false>(S, L, feat, map_a, map_b, map_y, map_r, map_p, stream)
-                : launch_features<false, false>(S, L, feat, map_a, map_b, map_y, map_r, map_p, stream);
+      return bf16 ? launch_features<true, true>(S, L, feat, map_a, map_b, map_y, map_r, map_p, map_f, stream)
+                  : launch_features<false, true>(S, L, feat, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+    return bf16 ? launch_features<true, false>(S, L, feat, map_a, map_b, map_y, map_r, map_p, map_f, stream)
+                : launch_features<false, false>(S, L, feat, map_a, map_b, map_y, map_r, map_p, map_f, stream);
   }
   if (L.swap)
-    return bf16 ? launch_kernel<true, false, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream)
-                : launch_kernel<false, false, true>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+    return bf16 ? launch_kernel<true, false, true>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream)
+                : launch_kernel<false, false, true>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
   if (bf16)
-    return L.pair ? launch_kernel<true, true, false>(S, L, map_a, map_b, map_y, map_r, map_p, stream)
-                  : launch_kernel<true, false, false>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
-  return L.pair ? launch_kernel<false, true, false>(S, L, map_a, map_b, map_y, map_r, map_p, stream)
-                : launch_kernel<false, false, false>(S, L, map_a, map_b, map_y, map_r, map_p, stream);
+    return L.pair ? launch_kernel<true, true, false>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream)
+                  : launch_kernel<true, false, false>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+  return L.pair ? launch_kernel<false, true, false>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream)
+                : launch_kernel<false, false, false>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
 }
 
 // Scratch a launch may use for the tail split: `bytes` at `ptr` (256-byte
@@ -1095,9 +1119,9 @@ struct BwdDataPlan {
   Problem fwd;      // the forward problem being differentiated
   Problem tr;       // the whole transposed convolution (no replicate padding), or
                     // the first-frame problem (replicate padding, D = 1)
-  Problem front;    // replicate padding, D > 1: extended frames, fp32
-  Problem body;     // replicate padding, D > 1: frames 1.., one sample
-  bool rep;         // front + body + fold
+  Problem whole;    // replicate padding, D > 1: the extended frames in fp32 and frames
+                    // 1.. in 16 bits, one launch (mixed output)
+  bool rep;         // whole + fold
   bool phased;      // spatial stride: one transposed convolution per phase
   size_t split_bytes;  // the tail-split region, after the flipped weight and ext
   size_t wt_bytes;  // flipped weight
@@ -1160,17 +1184,16 @@ conv3d_status_t plan_bwd_data(const void* dy, const void* w, const void* dx, int
     T.fold = true;
   }
   if (B.rep) {
-    // causal: pf = kt-1, so T.pf = 0 and output frame f reads dy[f .. f+kt-1]
-    Problem& Fr = B.front;
-    Fr = T;
-    Fr.pf = T.pf + F.kt - 1;    // output frames -(kt-1)..0
-    Fr.Do = F.kt;
-    Fr.out_f32 = true;
-    Problem& Bo = B.body;
-    Bo = T;
-    Bo.N = 1;
-    Bo.D = F.Do - 1;            // dy[n, 1:]
-    Bo.Do = D - 1;              // dx[n, 1:]
+    // causal: pf = kt-1, so T.pf = 0 and output frame f reads dy[f .. f+kt-1].
+    // One launch over output frames -(kt-1) .. D-1: frames -(kt-1)..0 are the
+    // kt fp32 parts of dx frame 0 (frame 0's own taps in the last), frames
+    // 1..D-1 go to dx in 16 bits.
+    Problem& Wh = B.whole;
+    Wh = T;
+    Wh.pf = T.pf + F.kt - 1;
+    Wh.Do = D + F.kt - 1;
+    Wh.f32_frames = F.kt;
+    Wh.y_frames = D;
   }
   B.wt_bytes = (static_cast<size_t>(Cout) * F.kt * F.kh * F.kw * Cin * 2 + 255) & ~size_t(255);
   B.ext_bytes = 0;
@@ -1179,6 +1202,24 @@ conv3d_status_t plan_bwd_data(const void* dy, const void* w, const void* dx, int
   else if (T.fold)
     B.ext_bytes = ((fold_bytes(Cout, Cin, kernel) + 255) & ~size_t(255)) + kPhaseSlack;
   B.split_bytes = kSplitRegionBytes;
+  return CONV3D_OK;
+}
+
+// dx[n, 0] = the rounded sum of the kt fp32 parts in ext (causal replicate padding).
+conv3d_status_t fold_front(const float* ext, void* dx, int N, int D, int kt,
+                           long long frame_elems, conv3d_dtype_t dtype, int sms,
+                           cudaStream_t stream) {
+  const long long total = static_cast<long long>(N) * (frame_elems / 8);
+  int blocks = static_cast<int>((total + 255) / 256);
+  if (blocks > 8 * sms) blocks = 8 * sms;
+  if (dtype == CONV3D_BF16)
+    fold_front_gradient_kernel<true><<<blocks, 256, 0, stream>>>(
+        ext, static_cast<uint16_t*>(dx), N, D, kt, frame_elems, FoldPhase{}, 0);
+  else
+    fold_front_gradient_kernel<false><<<blocks, 256, 0, stream>>>(
+        ext, static_cast<uint16_t*>(dx), N, D, kt, frame_elems, FoldPhase{}, 0);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "gradient fold launch");
   return CONV3D_OK;
 }
 
@@ -1580,61 +1621,18 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
 
   float* ext = reinterpret_cast<float*>(static_cast<char*>(workspace) + B.wt_bytes);
   const long long frame_elems = static_cast<long long>(H) * W * Cin;
-  // The front (kt frames, their tiles 1/kt .. 1 of the full reduction) and the
-  // body write disjoint buffers, so they may run at once: the front goes first
-  // on the high-priority aux stream, the body fills the remaining SMs, and the
-  // fold waits for both.  The overlap can save at most the front's time, kt
-  // frames against the body's D - 1, so it is used where the front is at least
-  // a quarter of the body.  Measured on B200 (sequential -> concurrent,
-  // TFLOP/s): 9-frame layers 708 -> 735, 1340 -> 1383, 1234 -> 1256; 17 and 33
-  // frames 1419 -> 1404 and 1447 -> 1403.
-  bool concurrent = B.body.Do > 0 && D - 1 <= 4 * kernel[0];
-  if (const char* env = getenv("CONV3D_DGRAD_CONCURRENT")) concurrent = concurrent && env[0] != '0';
-  if (concurrent) concurrent = aux_stream(*S, stream);
+  // One launch computes every frame: the kt fp32 parts of frame 0 and the
+  // 16-bit frames 1.., as one persistent grid whose last round the tail split
+  // balances.  (Measured on B200 against a front launch beside a body launch
+  // per sample: 128->512 9x64x64 176 -> 130 us, no change on the larger layers.)
+  Problem Wh = B.whole;
+  Wh.f32_out = ext;
   if (plan_log())
-    fprintf(stderr, "libconv3d: data gradient: %d front frames %s %d body frames x %d samples\n",
-            kernel[0], concurrent ? "beside" : "before", B.body.Do, N);
-  std::unique_lock<std::mutex> aux_lock;
-  cudaStream_t front_stream = stream;
-  if (concurrent) {
-    aux_lock = std::unique_lock<std::mutex>(g_aux_mu);
-    cudaError_t e = cudaEventRecord(S->aux_fork, stream);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(S->aux, S->aux_fork, 0);
-    if (e != cudaSuccess) return cuda_fail(e, "aux stream fork");
-    front_stream = S->aux;
-  }
-  st = launch_main(*S, B.front, dy, nullptr, wt, nullptr, nullptr, ext, front_stream, &split);
-  if (st == CONV3D_OK && B.body.Do > 0) {
-    const long long dy_frame = static_cast<long long>(B.fwd.Ho) * B.fwd.Wo * Cout;
-    for (int n = 0; n < N && st == CONV3D_OK; ++n) {
-      const uint16_t* dy_n = static_cast<const uint16_t*>(dy) + (n * static_cast<long long>(B.fwd.Do) + 1) * dy_frame;
-      uint16_t* dx_n = static_cast<uint16_t*>(dx) + (n * static_cast<long long>(D) + 1) * frame_elems;
-      st = launch_main(*S, B.body, dy_n, nullptr, wt, nullptr, nullptr, dx_n, stream);
-    }
-  }
-  if (concurrent) {
-    // join even after a failed launch, so the caller's stream never runs
-    // ahead of work left on the aux stream
-    cudaError_t e = cudaEventRecord(S->aux_join, S->aux);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, S->aux_join, 0);
-    aux_lock.unlock();
-    if (e != cudaSuccess && st == CONV3D_OK) return cuda_fail(e, "aux stream join");
-  }
+    fprintf(stderr, "libconv3d: data gradient: %d front frames and %d body frames x %d samples "
+            "in one launch\n", kernel[0], D - 1, N);
+  st = launch_main(*S, Wh, dy, nullptr, wt, nullptr, nullptr, dx, stream, &split);
   if (st != CONV3D_OK) return st;
-  {
-    const long long total = static_cast<long long>(N) * (frame_elems / 8);
-    int blocks = static_cast<int>((total + 255) / 256);
-    if (blocks > 8 * S->num_sms) blocks = 8 * S->num_sms;
-    if (dtype == CONV3D_BF16)
-      fold_front_gradient_kernel<true><<<blocks, 256, 0, stream>>>(
-          ext, static_cast<uint16_t*>(dx), N, D, kernel[0], frame_elems, FoldPhase{}, 0);
-    else
-      fold_front_gradient_kernel<false><<<blocks, 256, 0, stream>>>(
-          ext, static_cast<uint16_t*>(dx), N, D, kernel[0], frame_elems, FoldPhase{}, 0);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "gradient fold launch");
-  }
-  return CONV3D_OK;
+  return fold_front(ext, dx, N, D, kernel[0], frame_elems, dtype, S->num_sms, stream);
 }
 
 

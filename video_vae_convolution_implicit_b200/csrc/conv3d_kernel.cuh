@@ -91,7 +91,14 @@ struct KernelParams {
   uint32_t idesc;
   const void* bias;                  // [Cout] or null
   int has_residual;                  // residual is read through map_r
-  int out_f32;                       // y is fp32 (single-CTA, non-transposed variant only)
+  int out_f32;                       // y is fp32 (one-CTA variants)
+  // Mixed output (the data gradient under causal replicate padding): the
+  // first f32_frames output frames of each sample are the fp32 parts of dx
+  // frame 0 and go through map_f (N * f32_frames frames); output frame
+  // to >= f32_frames is dx frame to - f32_frames + 1, 16-bit, through map_y
+  // (N * y_frames frames).  0: every frame through map_y.
+  int f32_frames;
+  int y_frames;
   int* status;                       // device status word
   unsigned long long timeout_ns;
   int test_stall;                    // failure-detection test: the producer skips the
@@ -502,6 +509,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
                                 const __grid_constant__ CUtensorMap map_y,
                                 const __grid_constant__ CUtensorMap map_r,
                                 const __grid_constant__ CUtensorMap map_p,
+                                const __grid_constant__ CUtensorMap map_f,
                                 const KernelParams p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
@@ -529,7 +537,8 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
   const uint32_t b_stage_bytes = b_rows * BK * 2;
   const uint32_t a_ring = base;
   const uint32_t b_ring = a_ring + p.stages * A_STAGE_BYTES;
-  const uint32_t ybytes = p.out_f32 ? 2 * EPI_BUF_BYTES : EPI_BUF_BYTES;   // one y buffer
+  const uint32_t ybytes =
+      (p.out_f32 || p.f32_frames > 0) ? 2 * EPI_BUF_BYTES : EPI_BUF_BYTES;   // one y buffer
   const uint32_t y_stage = b_ring + p.stages * b_stage_bytes;        // [EPI_WARPS][2] buffers
   const uint32_t r_stage = y_stage + EPI_WARPS * 2 * ybytes;          // same, with a residual
   const uint32_t bars = r_stage + (p.has_residual ? EPI_Y_BYTES : 0);
@@ -567,6 +576,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
     prefetch_tensormap(&map_y);
     if (p.has_residual) prefetch_tensormap(&map_r);
     if (p.tpad == 3) prefetch_tensormap(&map_p);
+    if (p.f32_frames > 0) prefetch_tensormap(&map_f);
   }
   if (warp == 1) {
     if constexpr (kPair) {
@@ -863,6 +873,14 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
         const Work wk = decode_work<kSplit>(p, i);
         const Tile& tl = wk.tl;
         const bool piece = kSplit && wk.slot >= 0;
+        // where this tile's output goes: with mixed output, the fp32 parts of
+        // frame 0 through map_f, the other frames 16-bit through map_y
+        const bool front_tile = tl.to < p.f32_frames;
+        const bool f32_tile = p.out_f32 != 0 || front_tile;
+        const CUtensorMap* ymap = front_tile ? &map_f : &map_y;
+        const int yframe = p.f32_frames == 0 ? tl.frame_out
+                           : front_tile      ? tl.n * p.f32_frames + tl.to
+                                             : tl.n * p.y_frames + tl.to - p.f32_frames + 1;
         if (kStats && (tl.n != gacc.n || tl.co0 != gacc.co0)) {
           gn_flush(p.gn_out, p.gn_out_groups, p.Cout, gacc, gn_windows, gn_off, lane);
           gacc.n = tl.n;
@@ -944,7 +962,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
             if (lane == 0) bulk_wait_group_read<1>();
             __syncwarp();
             const uint32_t yb = ybuf + b * ybytes;
-            if (p.out_f32) {
+            if (f32_tile) {
               // fp32 rows of 32 channels (128 bytes, 128-byte swizzle): this
               // thread's channel is 4-byte word (lane & 3) of 16-byte chunk lane >> 2
               const uint32_t word = (lane & 3u) * 4u;
@@ -997,7 +1015,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
             const bool refill = use_res && j + 2 < live_chunks;
             if (lane == 0) {
               if (!kScatter) {
-                tma_store_3d(&map_y, yb, ch0, pix0, tl.frame_out);
+                tma_store_3d(ymap, yb, ch0, pix0, yframe);
                 bulk_commit_group();
               }
               if (refill) {
@@ -1025,6 +1043,14 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
       const Work wk = decode_work<kSplit>(p, i);
       const Tile& tl = wk.tl;
       const bool piece = kSplit && wk.slot >= 0;
+      // where this tile's output goes: with mixed output, the fp32 parts of
+      // frame 0 through map_f, the other frames 16-bit through map_y
+      const bool front_tile = tl.to < p.f32_frames;
+      const bool f32_tile = p.out_f32 != 0 || front_tile;
+      const CUtensorMap* ymap = front_tile ? &map_f : &map_y;
+      const int yframe = p.f32_frames == 0 ? tl.frame_out
+                         : front_tile      ? tl.n * p.f32_frames + tl.to
+                                           : tl.n * p.y_frames + tl.to - p.f32_frames + 1;
       if (kStats && (tl.n != gacc.n || tl.co0 != gacc.co0)) {
         gn_flush(p.gn_out, p.gn_out_groups, p.Cout, gacc, gn_windows, gn_off, lane);
         gacc.n = tl.n;
@@ -1109,7 +1135,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
           // the store issued from this buffer two chunks ago must have read it
           if (lane == 0) bulk_wait_group_read<1>();
           __syncwarp();
-          if (p.out_f32) {
+          if (f32_tile) {
 #pragma unroll
             for (int c = 0; c < 8; ++c)
               st_shared_v4(ybuf + b * ybytes + swz128(lane, c), __float_as_uint(v[4 * c + 0]),
@@ -1167,7 +1193,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
           const bool refill = use_res && j + 2 < live_chunks;
           if (lane == 0) {
             if (!kScatter) {
-              tma_store_3d(&map_y, ybuf + b * ybytes, cb, row_base, tl.frame_out);
+              tma_store_3d(ymap, ybuf + b * ybytes, cb, row_base, yframe);
               bulk_commit_group();
             }
             if (refill) {
