@@ -8,7 +8,8 @@ folded first-frame weight) is a fixed 16 MiB array inside the library.
 
 These tests call it through the C ABI on first-frame problems, which use that
 scratch.  It runs the same fold kernel and main kernel on the same bits as
-conv3d_fwd (with conv3d_fwd's tail split off, which noalloc never uses), so the
+conv3d_fwd (with conv3d_fwd's tail split and 8-bit lo product off, which
+noalloc never uses), so the
 two must agree bit for bit, on two calls in a row, with the
 larger problem first so that the second call runs over leftover scratch
 beyond its own size; one output is also checked against the fp64 oracle, and
@@ -43,8 +44,11 @@ def _out(p, fill=float("nan")):
 
 def test_noalloc_equals_conv3d_fwd_bit_for_bit_on_two_calls_in_a_row(monkeypatch):
     # conv3d_fwd_noalloc never splits its tiles along K (that needs scratch
-    # beyond the fold), so it is compared with conv3d_fwd with the split off
+    # beyond the fold) and keeps the lo part of the folded weight in 16 bits
+    # (an 8-bit copy of x would need scratch too), so it is compared with
+    # conv3d_fwd with the split off and the 16-bit lo part (the default)
     monkeypatch.setenv("CONV3D_SPLIT", "0")
+    monkeypatch.setenv("CONV3D_LO8", "0")
     # the larger fold first (2 * 192*9*160 16-bit values), then a smaller one
     # (2 * 64*9*64) that runs over the larger one's leftover scratch
     big = problem(1, 160, 1, 20, 28, 192, (3, 3, 3), (0, 1, 1), CREP, seed=24, residual=True)

@@ -95,6 +95,11 @@ struct Problem {
   void* f32_out;
   const void* prev;  // cached frames before the chunk (CONV3D_TPAD_CAUSAL_CACHED) or null
   bool fold;  // first-frame path: fold the temporal taps into a (hi, lo) pair
+  // first frame with the lo part in e5m2: lo weights w8 ([Cout][kh*kw][Cin],
+  // scaled by 2^8) and x8 (x scaled by 2^-8), both one byte a value
+  bool lo8;
+  const void* x8;
+  const void* w8;
   // GroupNorm + SiLU applied to x as it is read (conv3d_fwd_gn); gn_stats null otherwise
   const double* gn_stats;
   const void* gn_gamma;
@@ -248,6 +253,9 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
   P.f32_frames = 0;
   P.y_frames = 0;
   P.f32_out = nullptr;
+  P.lo8 = false;
+  P.x8 = nullptr;
+  P.w8 = nullptr;
   P.sc_sh = P.sc_sw = 1;
   P.sc_rh = P.sc_rw = 0;
   P.sc_H = P.sc_W = 0;
@@ -258,6 +266,31 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
 size_t fold_bytes(int Cin, int Cout, const int k[3]) {
   const size_t b = 2 * static_cast<size_t>(Cout) * k[1] * k[2] * Cin * 2;
   return (b + 255) & ~static_cast<size_t>(255);
+}
+
+size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+// Scratch of the first frame with the lo part in e5m2: the 16-bit hi weight,
+// the 8-bit lo weight, then the 8-bit copy of x (N frames).
+size_t lo8_hi_bytes(const Problem& P) {
+  return align256(static_cast<size_t>(P.Cout) * P.kh * P.kw * P.Cin * 2);
+}
+size_t lo8_w8_bytes(const Problem& P) {
+  return align256(static_cast<size_t>(P.Cout) * P.kh * P.kw * P.Cin);
+}
+size_t lo8_bytes(const Problem& P) {
+  return lo8_hi_bytes(P) + lo8_w8_bytes(P) +
+         align256(static_cast<size_t>(P.N) * P.H * P.W * P.Cin);
+}
+
+// CONV3D_LO8=1: the first frame's lo product in e5m2 (conv3d_fwd only).
+// Off by default: measured on B200 on a 256->256 256x256 first frame, the
+// main kernel went from 119 to 108 us, but converting x to e5m2 takes 8.5 us
+// more and the call was slower (127 against 114 us): the 8-bit k-blocks move
+// as many bytes as 16-bit ones and ran at 1.2x, not 2x, their rate.
+bool lo8_enabled() {
+  const char* env = getenv("CONV3D_LO8");
+  return env != nullptr && env[0] == '1';
 }
 
 // ------------------------------------------------------------------ driver entry points
@@ -397,7 +430,7 @@ struct DeviceState {
   };
   Scratch scratch[16] = {};
   int n_scratch = 0;
-  bool attr_set[128] = {};       // per kernel instance (variant and features)
+  bool attr_set[256] = {};       // per kernel instance: variant + 8 * features (< 32)
   int pair_clusters = 0;         // co-resident CTA pairs (occupancy query)
   int wg_pair_clusters = 0;      // the same for the weight-gradient kernel
   bool wg_attr_set[16] = {};     // per weight-gradient kernel variant
@@ -484,14 +517,18 @@ bool aux_stream(DeviceState& s, cudaStream_t caller) {
 // channels; each load gathers `pixels_per_load` output pixels' windows shifted
 // by one tap (the tap is the load's im2col offset).
 conv3d_status_t encode_im2col(const Problem& P, const void* base, long long images,
-                              int pixels_per_load, CUtensorMap& map) {
+                              int pixels_per_load, CUtensorMap& map, bool bytes8 = false) {
+  // 8-bit (the e5m2 copy of x): one byte a value, 128-channel boxes
   const CUtensorMapDataType dt =
-      P.dtype == CONV3D_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+      bytes8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+             : (P.dtype == CONV3D_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  const cuuint64_t es = bytes8 ? 1 : 2;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(P.Cin), static_cast<cuuint64_t>(P.W),
                               static_cast<cuuint64_t>(P.H), static_cast<cuuint64_t>(images)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(P.Cin) * 2,
-                                 static_cast<cuuint64_t>(P.W) * P.Cin * 2,
-                                 static_cast<cuuint64_t>(P.H) * P.W * P.Cin * 2};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(P.Cin) * es,
+                                 static_cast<cuuint64_t>(P.W) * P.Cin * es,
+                                 static_cast<cuuint64_t>(P.H) * P.W * P.Cin * es};
   // Window-origin box: first origin at -pad, last at dim-1+pad-(k-1) (or, for
   // a data-gradient phase, the origin of the last of exactly Wo, Ho outputs).
   const int lower[2] = {-P.pw, -P.ph};
@@ -501,7 +538,7 @@ conv3d_status_t encode_im2col(const Problem& P, const void* base, long long imag
   // columns (sh rows at a row wrap) apart
   const cuuint32_t estr[4] = {1, static_cast<cuuint32_t>(P.sw), static_cast<cuuint32_t>(P.sh), 1};
   CUresult r = encode_im2col_cached(&map, dt, 4, const_cast<void*>(base), dims, strides, lower, upper,
-                               BK, static_cast<cuuint32_t>(pixels_per_load), estr,
+                               bytes8 ? BK8 : BK, static_cast<cuuint32_t>(pixels_per_load), estr,
                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -540,6 +577,28 @@ conv3d_status_t encode_maps(const Problem& P, const void* x, const void* wmat, i
       set_error("cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
       return CONV3D_ERR_CUDA;
     }
+  }
+  return CONV3D_OK;
+}
+
+// The e5m2 lo weight viewed as [Cout][kh*kw][Cin] bytes; a box is 128
+// channels of one spatial tap for b_box_rows output channels (128-byte rows,
+// like a 64-channel box of the 16-bit weight).
+conv3d_status_t encode_w8_map(const Problem& P, const void* w8, int b_box_rows, CUtensorMap& map) {
+  const int taps = P.kh * P.kw;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(P.Cin), static_cast<cuuint64_t>(taps),
+                              static_cast<cuuint64_t>(P.Cout)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(P.Cin),
+                                 static_cast<cuuint64_t>(taps) * P.Cin};
+  const cuuint32_t box[3] = {BK8, 1, static_cast<cuuint32_t>(b_box_rows)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode_tiled_cached(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(w8),
+                                   dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled (8-bit lo weight) failed (%d)", static_cast<int>(r));
+    return CONV3D_ERR_CUDA;
   }
   return CONV3D_OK;
 }
@@ -658,6 +717,7 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   kp.sc_H = P.sc_H;
   kp.sc_W = P.sc_W;
   kp.n_chunks = (P.Cin + BK - 1) / BK;
+  kp.n_chunks8 = P.lo8 ? (P.Cin + BK8 - 1) / BK8 : 0;
 
   // A tcgen05.mma step with N < 256 takes as long as one with N = 256, so
   // layers whose channel count leaves the N side short run transposed
@@ -688,7 +748,10 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   }
   if (L.swap) L.pair = false;
   if (P.out_f32 || P.f32_frames > 0) L.pair = false;
-  if (P.gn_stats || P.gn_out || P.y_scatter) L.pair = false;   // one-CTA variants only   // the fp32 epilogue exists in the single and transposed variants
+  // one-CTA variants only (the fp32 epilogue exists in the single and the
+  // transposed variant)
+  if (P.gn_stats || P.gn_out || P.y_scatter) L.pair = false;
+  if (P.lo8) L.swap = L.pair = false;   // the e5m2 lo product: one CTA, M = pixels
   const int ctas = L.pair ? 2 : 1;
   if (L.swap) {
     kp.co_tile = 128;
@@ -722,7 +785,8 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
     const int U = S.num_sms;
     const int T = kp.num_tiles;
     int R = T % U;                 // the last round (all of them for a single round)
-    const int kb_nominal = kt_eff * P.kh * P.kw * kp.n_chunks;
+    const int kb_nominal = P.lo8 ? P.kh * P.kw * (kp.n_chunks + kp.n_chunks8)
+                                 : kt_eff * P.kh * P.kw * kp.n_chunks;
     if (R == 0 && (forced > 0 || T < U)) R = T < U ? T : U;
     if (forced > 0 || (R > 0 && 2 * R <= U)) {
       int sp = forced > 0 ? forced : U / R;
@@ -759,6 +823,7 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   kp.stages = stages;
   kp.tmem_cols = pow2_at_least(2u * kp.BN);
   kp.idesc = idesc_f16(bf16, ctas * BM, kp.BN);  // swapped: M = 128 channels, N = 256 pixels
+  kp.idesc8 = idesc_f8_e5m2(BM, kp.BN);
   kp.timeout_ns = kDefaultTimeoutNs;
   L.smem = static_cast<size_t>(stages) * stage_bytes + reserve;
   return CONV3D_OK;
@@ -869,6 +934,14 @@ conv3d_status_t launch_features(DeviceState& S, const LaunchPlan& L, int feat,
       return launch_kernel<kBF16, false, kSwap, FEAT_GN>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_GN | FEAT_STATS:
       return launch_kernel<kBF16, false, kSwap, FEAT_GN | FEAT_STATS>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+    case FEAT_LO8:
+      if constexpr (!kSwap)
+        return launch_kernel<kBF16, false, false, FEAT_LO8>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+      break;
+    case FEAT_LO8 | FEAT_SPLIT:
+      if constexpr (!kSwap)
+        return launch_kernel<kBF16, false, false, FEAT_LO8 | FEAT_SPLIT>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+      break;
   }
   set_error("internal: no kernel instance for feature set %d", feat);
   return CONV3D_ERR_UNSUPPORTED;
@@ -884,8 +957,10 @@ conv3d_status_t launch_planned(DeviceState& S, const Problem& P, LaunchPlan& L, 
   L.kp.bias = bias;
   L.kp.status = S.status;
   CUtensorMap map_a, map_b, map_y, map_r, map_p, map_f;
-  st = L.swap ? encode_maps(P, x, wmat, L.kp.kt, L.kp.co_tile, L.kp.pix_tile, map_a, map_b)
-              : encode_maps(P, x, wmat, L.kp.kt, L.kp.BN / (L.pair ? 2 : 1), BM, map_a, map_b);
+  // with the lo part in e5m2 the 16-bit weight holds the hi taps only
+  const int kt_w = P.lo8 ? 1 : L.kp.kt;
+  st = L.swap ? encode_maps(P, x, wmat, kt_w, L.kp.co_tile, L.kp.pix_tile, map_a, map_b)
+              : encode_maps(P, x, wmat, kt_w, L.kp.BN / (L.pair ? 2 : 1), BM, map_a, map_b);
   if (st != CONV3D_OK) return st;
   if (P.f32_frames > 0) {
     // mixed output: the fp32 front frames and the 16-bit frames after them
@@ -910,8 +985,17 @@ conv3d_status_t launch_planned(DeviceState& S, const Problem& P, LaunchPlan& L, 
   } else {
     map_p = map_a;  // never read: no tap reads before frame 0 in this mode
   }
+  if (P.lo8) {
+    // the e5m2 operands of the lo product take the cached-frames and the
+    // fp32-output slots, which a first frame does not use
+    if ((st = encode_im2col(P, P.x8, static_cast<long long>(P.N) * P.D, BM, map_p, true)) !=
+        CONV3D_OK)
+      return st;
+    if ((st = encode_w8_map(P, P.w8, L.kp.BN, map_f)) != CONV3D_OK) return st;
+  }
   // the optional parts this launch needs (each combination is its own instance)
   int feat = 0;
+  if (P.lo8) feat |= FEAT_LO8;
   if (L.kp.split_s > 1) feat |= FEAT_SPLIT;
   if (P.gn_out) feat |= FEAT_STATS;
   if (P.y_scatter) feat |= FEAT_SCATTER;
@@ -1009,11 +1093,17 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
   if ((st = device_state(S, dev)) != CONV3D_OK) return st;
   const bool bf16 = P.dtype == CONV3D_BF16;
   const void* wmat = w;
+  // conv3d_fwd's own scratch can also hold the e5m2 copy of x, so there the
+  // first frame's lo product may run in 8 bits (CONV3D_LO8=1; Cin a multiple
+  // of 16: the 8-bit tensor maps need 16-byte rows)
+  Problem Q = P;
+  Q.lo8 = cached_ws && P.fold && P.Cin % 16 == 0 && lo8_enabled();
   LaunchPlan L;
   const size_t room = cached_ws ? ~size_t(0) : (split ? split->bytes : 0);
-  if ((st = plan_launch(*S, P, bf16, room, L)) != CONV3D_OK) return st;
+  if ((st = plan_launch(*S, Q, bf16, room, L)) != CONV3D_OK) return st;
   const int kfold[3] = {P.kt, P.kh, P.kw};
-  const size_t fold_need = P.fold ? fold_bytes(P.Cin, P.Cout, kfold) : 0;   // 256-byte multiple
+  const size_t fold_need =
+      !P.fold ? 0 : (Q.lo8 ? lo8_bytes(Q) : fold_bytes(P.Cin, P.Cout, kfold));   // 256-byte multiple
   if (cached_ws && fold_need + L.split_bytes > 0) {
     unsigned int gen = 0;
     if ((st = cached_scratch(*S, stream, fold_need + L.split_bytes, ws, gen)) != CONV3D_OK)
@@ -1042,6 +1132,30 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
     const long long total = static_cast<long long>(P.Cout) * (spatial_cin / 8);   // 16-byte vectors
     int blocks = static_cast<int>((total + 255) / 256);
     if (blocks > 4 * S->num_sms) blocks = 4 * S->num_sms;
+    if (Q.lo8) {
+      char* base = static_cast<char*>(ws);
+      uint8_t* w8 = reinterpret_cast<uint8_t*>(base + lo8_hi_bytes(Q));
+      uint8_t* x8 = reinterpret_cast<uint8_t*>(base + lo8_hi_bytes(Q) + lo8_w8_bytes(Q));
+      const long long xn = static_cast<long long>(P.N) * P.H * P.W * P.Cin;   // one frame a sample
+      long long xb = (xn / 8 + 255) / 256;
+      if (xb > 8LL * S->num_sms) xb = 8LL * S->num_sms;
+      if (bf16) {
+        fold_taps_lo8_kernel<true><<<blocks, 256, 0, stream>>>(
+            static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), w8, P.Cout, P.kt, spatial_cin);
+        x_to_e5m2_kernel<true><<<static_cast<int>(xb), 256, 0, stream>>>(
+            static_cast<const uint16_t*>(x), x8, xn);
+      } else {
+        fold_taps_lo8_kernel<false><<<blocks, 256, 0, stream>>>(
+            static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), w8, P.Cout, P.kt, spatial_cin);
+        x_to_e5m2_kernel<false><<<static_cast<int>(xb), 256, 0, stream>>>(
+            static_cast<const uint16_t*>(x), x8, xn);
+      }
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "8-bit fold launch");
+      Q.w8 = w8;
+      Q.x8 = x8;
+      return launch_planned(*S, Q, L, x, P.prev, ws, bias, residual, y, stream);
+    }
     if (bf16)
       fold_temporal_taps_kernel<true><<<blocks, 256, 0, stream>>>(
           static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), P.Cout, P.kt, spatial_cin);

@@ -34,6 +34,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "ptx.cuh"
 
@@ -52,6 +53,8 @@ constexpr int FEAT_SPLIT = 1;      // tail split: K pieces, partials, tickets
 constexpr int FEAT_STATS = 2;      // GroupNorm statistics of the output
 constexpr int FEAT_SCATTER = 4;    // strided output (data-gradient phases)
 constexpr int FEAT_GN = 8;         // GroupNorm + SiLU of the x operand (4 more warps)
+constexpr int FEAT_LO8 = 16;       // first frame: the lo weight product in e5m2 (kind::f8f6f4)
+constexpr int BK8 = 128;           // 8-bit channels per k-block (128-byte rows, like BK 16-bit ones)
 constexpr int GN_THREADS = 320;     // with the GroupNorm + SiLU operand transform (4 more warps)
 constexpr int MAX_STAGES = 8;
 
@@ -67,6 +70,15 @@ struct KernelParams {
   int st, sh, sw;                    // strides
   int tpad;                          // 0 zero, 1 causal replicate, 2 causal zero, 3 cached
   int n_chunks;                      // ceil(Cin / BK)
+  // First frame with the lo product in 8 bits (FEAT_LO8): temporal tap 1 of
+  // the folded (hi, lo) pair runs n_chunks8 = ceil(Cin / BK8) k-blocks per
+  // spatial tap of e5m2 operands -- x * 2^-8 through map_p (im2col, 128
+  // channels a box) and lo * 2^8 through map_f ([Cout][kh*kw][Cin]) -- with
+  // tcgen05.mma kind::f8f6f4 and instruction descriptor idesc8; the scales
+  // cancel in the product, which adds into the same fp32 accumulator.
+  // n_chunks8 = 0 otherwise.
+  int n_chunks8;
+  uint32_t idesc8;
   int BN;                            // MMA N: channels per tile, or 256 pixels (swapped)
   int co_tile;                       // output channels per tile
   int pix_tile;                      // output pixels per tile (128, or 256 for a CTA pair / swapped)
@@ -217,6 +229,7 @@ __device__ __forceinline__ int source_frame(const KernelParams& p, int to, int i
 __device__ __forceinline__ int kblocks_of_tile(const KernelParams& p, int to) {
   int valid = 0;
   for (int it = 0; it < p.kt; ++it) valid += source_frame(p, to, it) != kNoFrame;
+  if (p.n_chunks8 > 0) return p.kh * p.kw * (p.n_chunks + p.n_chunks8);   // folded hi + e5m2 lo
   return valid * p.kh * p.kw * p.n_chunks;
 }
 
@@ -483,6 +496,12 @@ struct Cvt<false> {
   }
 };
 
+// Two floats to two e5m2 bytes (first in the low byte), round to nearest,
+// saturating to the largest finite value.
+__device__ __forceinline__ uint32_t e5m2x2(float a, float b) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E5M2));
+}
+
 // kPair = false: one CTA per tile of 128 pixels x BN channels (cta_group::1).
 // kPair = true:  a cluster of two CTAs per tile of 256 pixels x BN channels
 //   (cta_group::2, M = 256): CTA r loads the A rows [128r, 128r+128) of the
@@ -521,6 +540,8 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
   constexpr bool kStats = (kFeat & FEAT_STATS) != 0;
   constexpr bool kScatter = (kFeat & FEAT_SCATTER) != 0;
   constexpr bool kGN = (kFeat & FEAT_GN) != 0;
+  constexpr bool kLo8 = (kFeat & FEAT_LO8) != 0;
+  static_assert(!(kLo8 && (kPair || kSwap)), "the e5m2 lo product: one CTA, M = pixels");
   constexpr int kCtas = kPair ? 2 : 1;
   const uint32_t warp = threadIdx.x / 32;
   const uint32_t lane = threadIdx.x % 32;
@@ -628,7 +649,9 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
           for (int ih = 0; ok && kb < kb_hi && ih < p.kh; ++ih) {
             for (int iw = 0; ok && kb < kb_hi && iw < p.kw; ++iw) {
               const int tap = (it * p.kh + ih) * p.kw + iw;
-              for (int cc = 0; cc < p.n_chunks && kb < kb_hi; ++cc) {
+              const bool lo8 = kLo8 && it == 1;   // the e5m2 lo product
+              const int nch = lo8 ? p.n_chunks8 : p.n_chunks;
+              for (int cc = 0; cc < nch && kb < kb_hi; ++cc) {
                 if (kSplit && kb++ < wk.kb_lo) continue;   // an earlier piece's k-block
                 if (!wait_bounded(empty_bar + 8 * stage, phase ^ 1, ctl, true)) {
                   ok = false;
@@ -653,6 +676,14 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
                                           static_cast<uint16_t>(ih));
                   tma_load_3d_pair(b_ring + stage * b_stage_bytes, &map_b, fb_leader, cc * BK,
                                    tap, co_b);
+                } else if (lo8) {
+                  // same bytes as a 16-bit k-block: 128-byte rows of 128 channels
+                  mbar_arrive_expect_tx(fb, tx_bytes);
+                  tma_load_im2col_4d(a_ring + stage * A_STAGE_BYTES, &map_p, fb, cc * BK8, w_org,
+                                     h_org, img, static_cast<uint16_t>(iw),
+                                     static_cast<uint16_t>(ih));
+                  tma_load_3d(b_ring + stage * b_stage_bytes, &map_f, fb, cc * BK8,
+                              ih * p.kw + iw, co_b);
                 } else {
                   mbar_arrive_expect_tx(fb, tx_bytes);
                   tma_load_im2col_4d(a_ring + stage * A_STAGE_BYTES, xmap, fb, cc * BK, w_org,
@@ -696,12 +727,16 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
           tc_fence_after();
           const uint64_t da = smem_desc_k_sw128(a_ring + stage * A_STAGE_BYTES);
           const uint64_t db = smem_desc_k_sw128(b_ring + stage * b_stage_bytes);
+          // the e5m2 lo k-blocks follow the kh*kw*n_chunks hi ones in a tile
+          const bool lo8 = kLo8 && wk.kb_lo + kb >= p.kh * p.kw * p.n_chunks;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             // +32 bytes along K inside the swizzled 128-byte row = +2 in the
-            // descriptor's address field.
+            // descriptor's address field (16 16-bit or 32 8-bit values).
             if constexpr (kPair)
               mma_f16_ss_pair(d_tmem, da + 2 * k, db + 2 * k, p.idesc, (kb | k) != 0);
+            else if (lo8)
+              mma_f8_ss(d_tmem, da + 2 * k, db + 2 * k, p.idesc8, (kb | k) != 0);
             else
               mma_f16_ss(d_tmem, da + 2 * k, db + 2 * k, p.idesc, (kb | k) != 0);
           }
@@ -1278,6 +1313,64 @@ __global__ void fold_temporal_taps_kernel(const uint16_t* __restrict__ w, uint16
     *reinterpret_cast<uint4*>(w2 + co * 2 * spatial_cin + rest) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     *reinterpret_cast<uint4*>(w2 + co * 2 * spatial_cin + spatial_cin + rest) =
         make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
+// The same fold with the lo part in 8 bits: hi = round16(s) into w2
+// ([Cout][kh*kw*Cin], 16-bit) and lo8 = e5m2((s - hi) * 2^8) into w8 (same
+// layout, one byte each).  The x operand of the lo product is e5m2(x * 2^-8)
+// (x_to_e5m2_kernel), so the scales cancel in the product.  e5m2 keeps 3
+// significant bits: the lo product's error is about 2^-3 of a term that is
+// itself at most 2^-8 of the weight, below the output's 16-bit rounding; the
+// scales keep both operands in e5m2's normal range (2^-14 .. 57344) for
+// weights above 2^-14 and activations up to 1.4e7.
+template <bool kBF16>
+__global__ void fold_taps_lo8_kernel(const uint16_t* __restrict__ w, uint16_t* __restrict__ w2,
+                                     uint8_t* __restrict__ w8, int Cout, int kt, int spatial_cin) {
+  using C = Cvt<kBF16>;
+  griddep_launch_dependents();
+  const int vecs = spatial_cin / 8;
+  const long long total = static_cast<long long>(Cout) * vecs;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long co = i / vecs;
+    const long long rest = (i - co * vecs) * 8;
+    float s[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int it = 0; it < kt; ++it) {
+      const uint4 v = *reinterpret_cast<const uint4*>(w + (co * kt + it) * spatial_cin + rest);
+      s[0] += C::lo(v.x); s[1] += C::hi(v.x); s[2] += C::lo(v.y); s[3] += C::hi(v.y);
+      s[4] += C::lo(v.z); s[5] += C::hi(v.z); s[6] += C::lo(v.w); s[7] += C::hi(v.w);
+    }
+    uint32_t hi[4], lo[2];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) hi[q] = C::pack(s[2 * q], s[2 * q + 1]);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const uint32_t a = e5m2x2(256.0f * (s[4 * q] - C::lo(hi[2 * q])),
+                                256.0f * (s[4 * q + 1] - C::hi(hi[2 * q])));
+      const uint32_t b = e5m2x2(256.0f * (s[4 * q + 2] - C::lo(hi[2 * q + 1])),
+                                256.0f * (s[4 * q + 3] - C::hi(hi[2 * q + 1])));
+      lo[q] = a | (b << 16);
+    }
+    *reinterpret_cast<uint4*>(w2 + co * spatial_cin + rest) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint2*>(w8 + co * spatial_cin + rest) = make_uint2(lo[0], lo[1]);
+  }
+}
+
+// x8 = e5m2(x * 2^-8), 8 values per thread (n a multiple of 8).
+template <bool kBF16>
+__global__ void x_to_e5m2_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ x8,
+                                 long long n) {
+  using C = Cvt<kBF16>;
+  // the convolution that reads x8 waits for this whole grid before reading
+  griddep_launch_dependents();
+  const float sc = 1.0f / 256.0f;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n / 8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint4 v = reinterpret_cast<const uint4*>(x)[i];
+    const uint32_t a = e5m2x2(sc * C::lo(v.x), sc * C::hi(v.x)) | (e5m2x2(sc * C::lo(v.y), sc * C::hi(v.y)) << 16);
+    const uint32_t b = e5m2x2(sc * C::lo(v.z), sc * C::hi(v.z)) | (e5m2x2(sc * C::lo(v.w), sc * C::hi(v.w)) << 16);
+    reinterpret_cast<uint2*>(x8)[i] = make_uint2(a, b);
   }
 }
 
