@@ -1083,9 +1083,11 @@ conv3d_status_t cached_scratch(DeviceState& S, cudaStream_t stream, size_t need,
   return CONV3D_OK;
 }
 
+// folded: (first frame) ws already holds the folded (hi, lo) weight.
 conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* bias,
                     const void* residual, void* y, void* ws, size_t ws_bytes, bool cached_ws,
-                    cudaStream_t stream, const SplitRegion* split = nullptr) {
+                    cudaStream_t stream, const SplitRegion* split = nullptr,
+                    bool folded = false) {
   conv3d_status_t st = load_entry_points();
   if (st != CONV3D_OK) return st;
   DeviceState* S = nullptr;
@@ -1097,7 +1099,7 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
   // first frame's lo product may run in 8 bits (CONV3D_LO8=1; Cin a multiple
   // of 16: the 8-bit tensor maps need 16-byte rows)
   Problem Q = P;
-  Q.lo8 = cached_ws && P.fold && P.Cin % 16 == 0 && lo8_enabled();
+  Q.lo8 = cached_ws && P.fold && !folded && P.Cin % 16 == 0 && lo8_enabled();
   LaunchPlan L;
   const size_t room = cached_ws ? ~size_t(0) : (split ? split->bytes : 0);
   if ((st = plan_launch(*S, Q, bf16, room, L)) != CONV3D_OK) return st;
@@ -1156,14 +1158,16 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
       Q.x8 = x8;
       return launch_planned(*S, Q, L, x, P.prev, ws, bias, residual, y, stream);
     }
-    if (bf16)
-      fold_temporal_taps_kernel<true><<<blocks, 256, 0, stream>>>(
-          static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), P.Cout, P.kt, spatial_cin);
-    else
-      fold_temporal_taps_kernel<false><<<blocks, 256, 0, stream>>>(
-          static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), P.Cout, P.kt, spatial_cin);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "fold kernel launch");
+    if (!folded) {   // (else the caller's kernel wrote it)
+      if (bf16)
+        fold_temporal_taps_kernel<true><<<blocks, 256, 0, stream>>>(
+            static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), P.Cout, P.kt, spatial_cin);
+      else
+        fold_temporal_taps_kernel<false><<<blocks, 256, 0, stream>>>(
+            static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), P.Cout, P.kt, spatial_cin);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e, "fold kernel launch");
+    }
     wmat = ws;
   }
   (void)dev;
@@ -1417,33 +1421,21 @@ conv3d_status_t bwd_data_phases(DeviceState& S, const BwdDataPlan& B, const void
           return st;
         continue;
       }
-      // causal replicate, D > 1: the kt front frames in fp32 (dense, this phase's
-      // pixels), frames 1.. straight to dx, then the fold into frame 0
+      // causal replicate, D > 1: one launch over output frames -(kt-1)..D-1 of
+      // every sample -- the kt front frames in fp32 (dense, this phase's
+      // pixels), frames 1.. straight to their strided places in dx -- then the
+      // fold into frame 0
       float* ext = reinterpret_cast<float*>(ext_at);
       ext_at += static_cast<size_t>(N) * kt * Ah * Aw * Cin * 4;
-      Problem Fr = T;
-      Fr.pf = T.pf + kt - 1;
-      Fr.Do = kt;
-      Fr.out_f32 = true;
-      Fr.y_scatter = nullptr;
-      if ((st = launch_main(S, Fr, dy, nullptr, wt, nullptr, nullptr, ext, stream, split)) !=
+      Problem Wh = T;
+      Wh.pf = T.pf + kt - 1;
+      Wh.Do = D + kt - 1;
+      Wh.f32_frames = kt;
+      Wh.y_frames = D;
+      Wh.f32_out = ext;
+      if ((st = launch_main(S, Wh, dy, nullptr, wt, nullptr, nullptr, dx, stream, split)) !=
           CONV3D_OK)
         return st;
-      if (D > 1) {
-        Problem Bo = T;
-        Bo.N = 1;
-        Bo.D = F.Do - 1;
-        Bo.Do = D - 1;
-        const long long dy_frame = static_cast<long long>(F.Ho) * F.Wo * Cout;
-        const long long dx_frame = static_cast<long long>(H) * W * Cin;
-        for (int n = 0; n < N; ++n) {
-          Bo.y_scatter = static_cast<uint16_t*>(dx) + (n * static_cast<long long>(D) + 1) * dx_frame;
-          const uint16_t* dy_n = static_cast<const uint16_t*>(dy) + (n * static_cast<long long>(F.Do) + 1) * dy_frame;
-          if ((st = launch_main(S, Bo, dy_n, nullptr, wt, nullptr, nullptr, Bo.y_scatter, stream)) !=
-              CONV3D_OK)
-            return st;
-        }
-      }
       const long long frame_elems = static_cast<long long>(Ah) * Aw * Cin;
       const long long total = static_cast<long long>(N) * (frame_elems / 8);
       int blocks = static_cast<int>((total + 255) / 256);
@@ -1717,6 +1709,24 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
   int dev = 0;
   if ((st = device_state(S, dev)) != CONV3D_OK) return st;
   if (B.phased) return bwd_data_phases(*S, B, dy, w, dx, workspace, stream, &split);
+  if (B.tr.fold) {
+    // a single frame: mirror, transpose and fold the weight in one pass
+    // straight into the first-frame path's folded-weight scratch
+    void* ws = static_cast<char*>(workspace) + B.wt_bytes;
+    const dim3 grid((Cin + 63) / 64, (Cout + 63) / 64, kernel[1] * kernel[2]);
+    if (dtype == CONV3D_BF16)
+      flip_fold_weight_kernel<true><<<grid, dim3(32, 8), 0, stream>>>(
+          static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), Cout, kernel[0], kernel[1],
+          kernel[2], Cin);
+    else
+      flip_fold_weight_kernel<false><<<grid, dim3(32, 8), 0, stream>>>(
+          static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), Cout, kernel[0], kernel[1],
+          kernel[2], Cin);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
+    return run(B.tr, dy, nullptr, nullptr, nullptr, dx, ws, B.ext_bytes, false, stream, &split,
+               true);
+  }
   uint16_t* wt = static_cast<uint16_t*>(workspace);
   {
     const int taps = kernel[0] * kernel[1] * kernel[2];
@@ -1727,9 +1737,6 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
   }
-  if (B.tr.fold)
-    return run(B.tr, dy, wt, nullptr, nullptr, dx, static_cast<char*>(workspace) + B.wt_bytes,
-               B.ext_bytes, false, stream, &split);
   if (!B.rep)
     return launch_main(*S, B.tr, dy, nullptr, wt, nullptr, nullptr, dx, stream, &split);
 

@@ -1015,7 +1015,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
               for (int e = 0; e < 32; ++e, ++q) {
                 if (q < p.HoWo && ch < p.Cout) {
                   const size_t off =
-                      ((static_cast<size_t>(tl.frame_out) * p.sc_H + a * p.sc_sh + p.sc_rh) *
+                      ((static_cast<size_t>(yframe) * p.sc_H + a * p.sc_sh + p.sc_rh) *
                            p.sc_W + bq * p.sc_sw + p.sc_rw) * p.Cout + ch;
                   p.y_scatter[off] = static_cast<uint16_t>(C::pack(v[e], 0.0f) & 0xFFFFu);
                 }
@@ -1049,7 +1049,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
             const int pix0 = tl.p0 + 32 * j;
             const bool refill = use_res && j + 2 < live_chunks;
             if (lane == 0) {
-              if (!kScatter) {
+              if (!kScatter || f32_tile) {   // strided 16-bit frames were stored above
                 tma_store_3d(ymap, yb, ch0, pix0, yframe);
                 bulk_commit_group();
               }
@@ -1187,7 +1187,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
                 const int a = q / p.Wo, bq = q - a * p.Wo;
                 uint4* dst = reinterpret_cast<uint4*>(
                     p.y_scatter +
-                    ((static_cast<size_t>(tl.frame_out) * p.sc_H + a * p.sc_sh + p.sc_rh) *
+                    ((static_cast<size_t>(yframe) * p.sc_H + a * p.sc_sh + p.sc_rh) *
                          p.sc_W + bq * p.sc_sw + p.sc_rw) * p.Cout + cb);
 #pragma unroll
                 for (int g = 0; g < 4; ++g)
@@ -1227,7 +1227,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
           // every lane has read residual buffer b: refill it with chunk j+2
           const bool refill = use_res && j + 2 < live_chunks;
           if (lane == 0) {
-            if (!kScatter) {
+            if (!kScatter || f32_tile) {   // strided 16-bit frames were stored above
               tma_store_3d(ymap, ybuf + b * ybytes, cb, row_base, yframe);
               bulk_commit_group();
             }
@@ -1414,6 +1414,54 @@ __global__ void flip_transpose_weight_kernel(const uint16_t* __restrict__ w,
     if (co < Cout && ci < Cin)
       *reinterpret_cast<uint32_t*>(wt + (static_cast<long long>(ci) * taps + tap) * Cout + co) =
           static_cast<uint32_t>(tile[x2][r]) | (static_cast<uint32_t>(tile[x2 + 1][r]) << 16);
+  }
+}
+
+// The single-frame data gradient's weight in one pass: the transposed
+// convolution's weight (every tap mirrored, Cin and Cout exchanged) with its kt
+// temporal taps summed and split into hi and lo 16-bit parts, as the first-frame
+// fold does -- w2[ci][0][jh][jw][co] = hi(s), w2[ci][1][jh][jw][co] = lo(s) with
+// s = sum over it of w[co][it][kh-1-jh][kw-1-jw][ci], summed in fp32.  Block =
+// one spatial tap and a 64 x 64 (co, ci) tile; the sums are staged in shared
+// memory so that reads and writes both run along contiguous channels.
+// Launch: grid (ceil(Cin/64), ceil(Cout/64), kh*kw), block (32, 8).
+template <bool kBF16>
+__global__ void flip_fold_weight_kernel(const uint16_t* __restrict__ w,
+                                        uint16_t* __restrict__ w2, int Cout, int kt, int kh,
+                                        int kw, int Cin) {
+  using C = Cvt<kBF16>;
+  griddep_launch_dependents();
+  __shared__ float tile[64][65];                  // [co][ci] sums
+  const int ci0 = blockIdx.x * 64, co0 = blockIdx.y * 64;
+  const int tap = blockIdx.z;                     // (jh, jw) of w2
+  const int taps2 = kh * kw;
+  const int src_sp = taps2 - 1 - tap;             // mirrored spatial tap of w
+  const int x2 = 2 * static_cast<int>(threadIdx.x);
+  for (int r = threadIdx.y; r < 64; r += 8) {
+    const int co = co0 + r, ci = ci0 + x2;
+    if (co < Cout && ci < Cin) {
+      float a = 0.0f, b = 0.0f;
+      for (int it = 0; it < kt; ++it) {
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(
+            w + ((static_cast<long long>(co) * kt + it) * taps2 + src_sp) * Cin + ci);
+        a += C::lo(v);
+        b += C::hi(v);
+      }
+      tile[r][x2] = a;
+      tile[r][x2 + 1] = b;
+    }
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 64; r += 8) {
+    const int ci = ci0 + r, co = co0 + x2;
+    if (co < Cout && ci < Cin) {
+      const float a = tile[x2][r], b = tile[x2 + 1][r];
+      const uint32_t hi = C::pack(a, b);
+      const uint32_t lo = C::pack(a - C::lo(hi), b - C::hi(hi));
+      const long long row = static_cast<long long>(ci) * 2 * taps2;
+      *reinterpret_cast<uint32_t*>(w2 + (row + tap) * Cout + co) = hi;
+      *reinterpret_cast<uint32_t*>(w2 + (row + taps2 + tap) * Cout + co) = lo;
+    }
   }
 }
 
