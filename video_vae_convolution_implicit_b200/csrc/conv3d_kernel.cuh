@@ -1437,19 +1437,31 @@ __global__ void flip_fold_weight_kernel(const uint16_t* __restrict__ w,
   const int taps2 = kh * kw;
   const int src_sp = taps2 - 1 - tap;             // mirrored spatial tap of w
   const int x2 = 2 * static_cast<int>(threadIdx.x);
-  for (int r = threadIdx.y; r < 64; r += 8) {
-    const int co = co0 + r, ci = ci0 + x2;
-    if (co < Cout && ci < Cin) {
-      float a = 0.0f, b = 0.0f;
-      for (int it = 0; it < kt; ++it) {
-        const uint32_t v = *reinterpret_cast<const uint32_t*>(
-            w + ((static_cast<long long>(co) * kt + it) * taps2 + src_sp) * Cin + ci);
-        a += C::lo(v);
-        b += C::hi(v);
-      }
-      tile[r][x2] = a;
-      tile[r][x2 + 1] = b;
+  // rows ty, ty + 8, ..., ty + 56: eight loads in flight per temporal tap
+  float a[8], b[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = b[k] = 0.0f;
+  const int ci = ci0 + x2;
+  for (int it = 0; it < kt; ++it) {
+    uint32_t v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int co = co0 + static_cast<int>(threadIdx.y) + 8 * k;
+      v[k] = (co < Cout && ci < Cin)
+                 ? *reinterpret_cast<const uint32_t*>(
+                       w + ((static_cast<long long>(co) * kt + it) * taps2 + src_sp) * Cin + ci)
+                 : 0u;
     }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      a[k] += C::lo(v[k]);
+      b[k] += C::hi(v[k]);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    tile[threadIdx.y + 8 * k][x2] = a[k];
+    tile[threadIdx.y + 8 * k][x2 + 1] = b[k];
   }
   __syncthreads();
   for (int r = threadIdx.y; r < 64; r += 8) {
