@@ -430,7 +430,7 @@ struct DeviceState {
   };
   Scratch scratch[16] = {};
   int n_scratch = 0;
-  bool attr_set[256] = {};       // per kernel instance: variant + 8 * features (< 32)
+  bool attr_set[512] = {};       // per kernel instance: variant + 8 * features (< 64)
   int pair_clusters = 0;         // co-resident CTA pairs (occupancy query)
   int wg_pair_clusters = 0;      // the same for the weight-gradient kernel
   bool wg_attr_set[16] = {};     // per weight-gradient kernel variant
@@ -916,7 +916,10 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
 
 // The one-CTA instances with optional parts: the tail split, the output
 // statistics, the strided output, the GroupNorm operand transform (with or
-// without the statistics).  The plan never combines the split with the others.
+// without the statistics), the mixed fp32/16-bit output of the data gradient
+// (alone, split, or strided) and the first frame's 8-bit lo product (alone or
+// split).  The plan never combines the split with the statistics, the strided
+// output or the GroupNorm transform.
 template <bool kBF16, bool kSwap>
 conv3d_status_t launch_features(DeviceState& S, const LaunchPlan& L, int feat,
                                 const CUtensorMap& map_a, const CUtensorMap& map_b,
@@ -934,6 +937,12 @@ conv3d_status_t launch_features(DeviceState& S, const LaunchPlan& L, int feat,
       return launch_kernel<kBF16, false, kSwap, FEAT_GN>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_GN | FEAT_STATS:
       return launch_kernel<kBF16, false, kSwap, FEAT_GN | FEAT_STATS>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+    case FEAT_MIXED:
+      return launch_kernel<kBF16, false, kSwap, FEAT_MIXED>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+    case FEAT_MIXED | FEAT_SPLIT:
+      return launch_kernel<kBF16, false, kSwap, FEAT_MIXED | FEAT_SPLIT>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+    case FEAT_MIXED | FEAT_SCATTER:
+      return launch_kernel<kBF16, false, kSwap, FEAT_MIXED | FEAT_SCATTER>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_LO8:
       if constexpr (!kSwap)
         return launch_kernel<kBF16, false, false, FEAT_LO8>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
@@ -996,6 +1005,7 @@ conv3d_status_t launch_planned(DeviceState& S, const Problem& P, LaunchPlan& L, 
   // the optional parts this launch needs (each combination is its own instance)
   int feat = 0;
   if (P.lo8) feat |= FEAT_LO8;
+  if (P.f32_frames > 0) feat |= FEAT_MIXED;
   if (L.kp.split_s > 1) feat |= FEAT_SPLIT;
   if (P.gn_out) feat |= FEAT_STATS;
   if (P.y_scatter) feat |= FEAT_SCATTER;
@@ -1834,7 +1844,16 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
   wp.co_tiles = (Cout + wp.BN - 1) / wp.BN;
   wp.c64s = Cin / 64;
   wp.ents = F.kh * F.kw * wp.c64s;
-  wp.eblocks = (wp.ents + 3) / 4;
+  // Entry blocks of the swapped variant: four 64-channel entries (N = 256) by
+  // default; CONV3D_WGRAD_ENTRIES=3 takes three (N = 192), which leaves no
+  // half-filled last block when a temporal tap has 18 entries.  Measured on
+  // B200, 128->128 layers: 9x256x256 406 -> 454 us, 121x256x256 5528 -> 5900 us
+  // with three: six N = 192 blocks cost more than four N = 256 and one N = 128,
+  // and every block reloads the dy tile.
+  wp.ent_per_block = 4;
+  if (const char* env = getenv("CONV3D_WGRAD_ENTRIES"))
+    if (env[0] == '3') wp.ent_per_block = 3;
+  wp.eblocks = (wp.ents + wp.ent_per_block - 1) / wp.ent_per_block;
   // The swapped variant needs whole 64-channel input boxes; it wins when it
   // issues fewer MMA steps (an N = 128 step costs about as much as N = 256).
   bool swap = false;

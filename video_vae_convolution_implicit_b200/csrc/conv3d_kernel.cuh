@@ -54,6 +54,7 @@ constexpr int FEAT_STATS = 2;      // GroupNorm statistics of the output
 constexpr int FEAT_SCATTER = 4;    // strided output (data-gradient phases)
 constexpr int FEAT_GN = 8;         // GroupNorm + SiLU of the x operand (4 more warps)
 constexpr int FEAT_LO8 = 16;       // first frame: the lo weight product in e5m2 (kind::f8f6f4)
+constexpr int FEAT_MIXED = 32;     // fp32 front frames and 16-bit frames in one launch (data gradient)
 constexpr int BK8 = 128;           // 8-bit channels per k-block (128-byte rows, like BK 16-bit ones)
 constexpr int GN_THREADS = 320;     // with the GroupNorm + SiLU operand transform (4 more warps)
 constexpr int MAX_STAGES = 8;
@@ -541,6 +542,8 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
   constexpr bool kScatter = (kFeat & FEAT_SCATTER) != 0;
   constexpr bool kGN = (kFeat & FEAT_GN) != 0;
   constexpr bool kLo8 = (kFeat & FEAT_LO8) != 0;
+  constexpr bool kMixed = (kFeat & FEAT_MIXED) != 0;
+  constexpr int kYBufs = 2;   // output staging buffers per epilogue warp
   static_assert(!(kLo8 && (kPair || kSwap)), "the e5m2 lo product: one CTA, M = pixels");
   constexpr int kCtas = kPair ? 2 : 1;
   const uint32_t warp = threadIdx.x / 32;
@@ -561,7 +564,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
   const uint32_t ybytes =
       (p.out_f32 || p.f32_frames > 0) ? 2 * EPI_BUF_BYTES : EPI_BUF_BYTES;   // one y buffer
   const uint32_t y_stage = b_ring + p.stages * b_stage_bytes;        // [EPI_WARPS][2] buffers
-  const uint32_t r_stage = y_stage + EPI_WARPS * 2 * ybytes;          // same, with a residual
+  const uint32_t r_stage = y_stage + EPI_WARPS * kYBufs * ybytes;     // 2 per warp, with a residual
   const uint32_t bars = r_stage + (p.has_residual ? EPI_Y_BYTES : 0);
   const uint32_t full_bar = bars;                         // [stages]
   const uint32_t empty_bar = bars + 8 * p.stages;         // [stages]
@@ -881,7 +884,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
     using C = Cvt<kBF16>;
     const uint32_t quarter = warp & 3;            // TMEM lanes [32q, 32q+32)
     const uint32_t ew = warp - 2;                 // epilogue warp index, 0..3
-    const uint32_t ybuf = y_stage + ew * 2 * ybytes;
+    const uint32_t ybuf = y_stage + ew * kYBufs * ybytes;
     const uint32_t rbuf = r_stage + ew * 2 * EPI_BUF_BYTES;
     const uint32_t rbar = rfull_bar + ew * 16;
     uint32_t rphase[2] = {0, 0};
@@ -910,10 +913,10 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
         const bool piece = kSplit && wk.slot >= 0;
         // where this tile's output goes: with mixed output, the fp32 parts of
         // frame 0 through map_f, the other frames 16-bit through map_y
-        const bool front_tile = tl.to < p.f32_frames;
+        const bool front_tile = kMixed && tl.to < p.f32_frames;
         const bool f32_tile = p.out_f32 != 0 || front_tile;
         const CUtensorMap* ymap = front_tile ? &map_f : &map_y;
-        const int yframe = p.f32_frames == 0 ? tl.frame_out
+        const int yframe = !kMixed ? tl.frame_out
                            : front_tile      ? tl.n * p.f32_frames + tl.to
                                              : tl.n * p.y_frames + tl.to - p.f32_frames + 1;
         if (kStats && (tl.n != gacc.n || tl.co0 != gacc.co0)) {
@@ -994,9 +997,9 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
                 v[e] += C::lo(q);
               }
             }
-            if (lane == 0) bulk_wait_group_read<1>();
+            if (lane == 0) bulk_wait_group_read<kYBufs - 1>();
             __syncwarp();
-            const uint32_t yb = ybuf + b * ybytes;
+            const uint32_t yb = ybuf + (j & (kYBufs - 1)) * ybytes;
             if (f32_tile) {
               // fp32 rows of 32 channels (128 bytes, 128-byte swizzle): this
               // thread's channel is 4-byte word (lane & 3) of 16-byte chunk lane >> 2
@@ -1080,10 +1083,10 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
       const bool piece = kSplit && wk.slot >= 0;
       // where this tile's output goes: with mixed output, the fp32 parts of
       // frame 0 through map_f, the other frames 16-bit through map_y
-      const bool front_tile = tl.to < p.f32_frames;
+      const bool front_tile = kMixed && tl.to < p.f32_frames;
       const bool f32_tile = p.out_f32 != 0 || front_tile;
       const CUtensorMap* ymap = front_tile ? &map_f : &map_y;
-      const int yframe = p.f32_frames == 0 ? tl.frame_out
+      const int yframe = !kMixed ? tl.frame_out
                          : front_tile      ? tl.n * p.f32_frames + tl.to
                                            : tl.n * p.y_frames + tl.to - p.f32_frames + 1;
       if (kStats && (tl.n != gacc.n || tl.co0 != gacc.co0)) {
@@ -1168,12 +1171,13 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
             }
           }
           // the store issued from this buffer two chunks ago must have read it
-          if (lane == 0) bulk_wait_group_read<1>();
+          if (lane == 0) bulk_wait_group_read<kYBufs - 1>();
           __syncwarp();
+          const uint32_t yb = ybuf + (j & (kYBufs - 1)) * ybytes;
           if (f32_tile) {
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-              st_shared_v4(ybuf + b * ybytes + swz128(lane, c), __float_as_uint(v[4 * c + 0]),
+              st_shared_v4(yb + swz128(lane, c), __float_as_uint(v[4 * c + 0]),
                            __float_as_uint(v[4 * c + 1]), __float_as_uint(v[4 * c + 2]),
                            __float_as_uint(v[4 * c + 3]));
           } else {
@@ -1197,7 +1201,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
             } else {
 #pragma unroll
               for (int g = 0; g < 4; ++g)
-                st_shared_v4(ybuf + b * ybytes + swz64(lane, g), pk[4 * g], pk[4 * g + 1],
+                st_shared_v4(yb + swz64(lane, g), pk[4 * g], pk[4 * g + 1],
                              pk[4 * g + 2], pk[4 * g + 3]);
             }
             if constexpr (kStats) {
@@ -1206,7 +1210,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
               __syncwarp();
               int rows_in = p.HoWo - row_base;
               if (rows_in > 32) rows_in = 32;
-              const uint32_t col = ybuf + b * ybytes + (lane & 7u) * 2u;
+              const uint32_t col = yb + (lane & 7u) * 2u;
               float gs = 0.0f, gq = 0.0f;
               for (int e = 0; e < rows_in; ++e) {
                 uint16_t qv;
@@ -1228,7 +1232,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
           const bool refill = use_res && j + 2 < live_chunks;
           if (lane == 0) {
             if (!kScatter || f32_tile) {   // strided 16-bit frames were stored above
-              tma_store_3d(ymap, ybuf + b * ybytes, cb, row_base, yframe);
+              tma_store_3d(ymap, yb, cb, row_base, yframe);
               bulk_commit_group();
             }
             if (refill) {

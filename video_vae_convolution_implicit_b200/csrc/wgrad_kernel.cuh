@@ -57,7 +57,8 @@ struct WgradParams {
   int co_tiles;             // ceil(Cout / BN)
   int c64s;                 // Cin / 64                          (swap variant)
   int ents;                 // kh * kw * Cin / 64 entries per temporal tap (swap)
-  int eblocks;              // ceil(ents / 4)                    (swap)
+  int eblocks;              // ceil(ents / ent_per_block)        (swap)
+  int ent_per_block;        // entries per block: 4 (N = 256) or 3 (N = 192)  (swap)
   int pairs_per_it;         // ceil(kh * kw * cblocks / 2)       (pair)
   int chunks_per_frame;     // ceil(HoWo / 64)
   long long total_chunks;   // N * Do * chunks_per_frame
@@ -101,7 +102,7 @@ __device__ __forceinline__ int wg_source_frame(const WgradParams& p, int to, int
 struct WgUnit {
   int it;            // temporal tap
   int tap, cb;       // plain / pair: tap and 128-channel block of this CTA
-  int e0, nent;      // swap: first entry of the block and entries in it (1..4)
+  int e0, nent;      // swap: first entry of the block and entries in it (1..ent_per_block)
   bool dup;          // pair: this CTA's block repeats its peer's (odd count): not written
   int co0;
   long long c_begin, c_end;
@@ -133,8 +134,8 @@ __device__ __forceinline__ WgUnit wg_decode(const WgradParams& p, int u, uint32_
     r.e0 = r.nent = 0;
   } else if (kSwap) {
     r.it = mb / p.eblocks;
-    r.e0 = (mb - r.it * p.eblocks) * 4;
-    r.nent = p.ents - r.e0 < 4 ? p.ents - r.e0 : 4;
+    r.e0 = (mb - r.it * p.eblocks) * p.ent_per_block;
+    r.nent = p.ents - r.e0 < p.ent_per_block ? p.ents - r.e0 : p.ent_per_block;
     r.tap = r.cb = 0;
   } else {
     r.tap = mb / p.cblocks;
