@@ -131,6 +131,33 @@ def test_bwd_weight_bias_gradient_beside_and_after(case, side, monkeypatch):
     assert_close(dw.double().cpu().numpy(), ref_dw, f"dw {case} {side}")
 
 
+@pytest.mark.parametrize("block", ["1", "0"])
+@pytest.mark.parametrize("case", [
+    # N, Cin, D, H, W, Cout, kernel, stride, pad, tpad, dtype
+    (1, 256, 2, 16, 16, 320, (1, 1, 1), (1, 1, 1), (0, 0, 0), ZERO, "bf16"),   # 2 output tiles, 64 live
+    (2, 128, 3, 9, 11, 64, (1, 1, 1), (1, 1, 1), (0, 0, 0), CREP, "f16"),      # ragged frames
+    (1, 512, 2, 12, 12, 256, (1, 1, 1), (1, 2, 2), (0, 0, 0), ZERO, "bf16"),   # strided
+    (1, 64, 3, 8, 8, 64, (1, 1, 1), (1, 1, 1), (1, 0, 0), ZERO, "bf16"),       # padded end frames
+], ids=lambda c: "x".join(map(str, c[:6])) + f"-s{''.join(map(str, c[7]))}-p{c[8][0]}-{c[10]}")
+def test_bwd_weight_single_tap_bias_block(case, block, monkeypatch):
+    """A single-tap weight gradient sums dy for dbias in one more block of the
+    kernel whose A operand is a tile of ones (CONV3D_WGRAD_DBIAS_BLOCK=0: the
+    separate pass instead).  With temporal zero padding that leaves output
+    frames reading only padding, no tap covers every frame and the separate
+    pass runs either way.  dw and dbias against the oracle."""
+    monkeypatch.setenv("CONV3D_WGRAD_DBIAS_BLOCK", block)
+    N, Cin, D, H, W, Cout, k, stride, pad, tpad, dt = case
+    x, w, dy, od = grads_problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=470 + Cin, dt=dt,
+                                 stride=stride)
+    dw, db = c3.conv3d_bwd_weight(x, dy, k, stride, pad, tpad)
+    assert c3.poll_status() == c3.Status.OK
+    ref_db = oracle.decode16(si.bits(dy), od).reshape(-1, Cout).sum(axis=0)
+    assert_close(db.double().cpu().numpy(), ref_db, f"dbias {case} block={block}")
+    _, ref_dw, _ = oracle.conv3d_backward(si.bits(x), si.bits(w), si.bits(dy), od, k, stride,
+                                          pad, tpad)
+    assert_close(dw.double().cpu().numpy(), ref_dw, f"dw {case} block={block}")
+
+
 # ------------------------------------------------------ full-size workloads, sampled
 
 from seeded_inputs.workloads import WORKLOADS  # noqa: E402

@@ -433,7 +433,7 @@ struct DeviceState {
   bool attr_set[512] = {};       // per kernel instance: variant + 8 * features (< 64)
   int pair_clusters = 0;         // co-resident CTA pairs (occupancy query)
   int wg_pair_clusters = 0;      // the same for the weight-gradient kernel
-  bool wg_attr_set[16] = {};     // per weight-gradient kernel variant
+  bool wg_attr_set[16] = {};     // per weight-gradient kernel variant (4 kinds x pix x dtype)
   // Second stream (highest priority) on which the data gradient's front frames
   // run beside its body; created on first use, never if creation fails.
   cudaStream_t aux = nullptr;
@@ -1486,7 +1486,10 @@ using WgradKernel = decltype(&conv3d_wgrad_kernel<true, false, false, WG_PIX>);
 // two stages (see the launch code).  CTA pairs always fit three 128-pixel
 // stages (96-pixel ones measured no faster), so they have one instance.
 template <bool kBF16>
-WgradKernel wgrad_kernel_of(bool swap, bool pair, int pix) {
+WgradKernel wgrad_kernel_of(bool swap, bool pair, int pix, bool bias) {
+  if (bias)
+    return pix == 96 ? conv3d_wgrad_kernel<kBF16, false, false, 96, true>
+                     : conv3d_wgrad_kernel<kBF16, false, false, 128, true>;
   if (pair) return conv3d_wgrad_kernel<kBF16, false, true, 128>;
   if (swap)
     return pix == 96 ? conv3d_wgrad_kernel<kBF16, true, false, 96>
@@ -1495,8 +1498,9 @@ WgradKernel wgrad_kernel_of(bool swap, bool pair, int pix) {
                    : conv3d_wgrad_kernel<kBF16, false, false, 128>;
 }
 
-WgradKernel wgrad_kernel_for(bool bf16, bool swap, bool pair, int pix) {
-  return bf16 ? wgrad_kernel_of<true>(swap, pair, pix) : wgrad_kernel_of<false>(swap, pair, pix);
+WgradKernel wgrad_kernel_for(bool bf16, bool swap, bool pair, int pix, bool bias) {
+  return bf16 ? wgrad_kernel_of<true>(swap, pair, pix, bias)
+              : wgrad_kernel_of<false>(swap, pair, pix, bias);
 }
 
 // Number of pixel ranges each (tap block, output-channel tile) is split into.
@@ -1876,6 +1880,28 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
   wp.pairs_per_it = (F.kh * F.kw * wp.cblocks + 1) / 2;
   const int kCtas = pair ? 2 : 1;
   int lanes = S->num_sms;   // co-resident CTAs, or CTA pairs
+  // A single tap (1x1x1 and the like) is HBM-bound: its bias gradient comes
+  // from one more block per output-channel tile whose A operand is a tile of
+  // ones (kBias), which reads only the dy tiles that the other blocks bring
+  // into L2 at the same time, instead of a second pass over dy.  It needs a
+  // temporal tap whose source frame exists for every output frame, so that its
+  // units walk every dy pixel; CONV3D_WGRAD_DBIAS_BLOCK=0 turns it off.
+  wp.db = nullptr;
+  wp.db_it = -1;
+  bool bias_block = false;
+  if (dbias && !swap && !pair && taps_run == 1) {
+    const char* env = getenv("CONV3D_WGRAD_DBIAS_BLOCK");
+    if (env == nullptr || env[0] != '0') {
+      for (int it = 0; it < kt_run && wp.db_it < 0; ++it) {
+        const long long f_lo = static_cast<long long>(it) - wp.pf;
+        const long long f_hi = static_cast<long long>(F.Do - 1) * wp.st + it - wp.pf;
+        const bool lo_ok = f_lo >= 0 || wp.tpad == 1 || wp.tpad == 3;   // replicate / cached frames
+        if (lo_ok && f_hi < wp.D) wp.db_it = it;
+      }
+      bias_block = wp.db_it >= 0;
+    }
+  }
+  if (bias_block) wp.db = db32;
   // Pixels per stage.  A stage holds two 64-channel x boxes and the dy boxes
   // (plain, pair) or two dy boxes and four x boxes (swapped), 128 bytes per
   // pixel each.  Three stages in flight keep the tensor cores fed; where
@@ -1884,17 +1910,18 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
   // B200: swapped 128-channel workloads 2 x 128 px 921-1113, 4 x 64 px
   // 987-1016, 3 x 96 px 1156-1260 TFLOP/s; 1x1x1 512->256 648 -> 677.
   const int boxes = swap ? 6 : 2 + wp.BN / kCtas / 64;
-  const int reserve = 1024 + 8 * (2 * MAX_STAGES + 5);
+  // (+ 4 KB of ones, 1024-byte aligned, for the bias block)
+  const int reserve = 1024 + 8 * (2 * MAX_STAGES + 5) + (bias_block ? 4096 + 1024 : 0);
   const int smem_room = S->max_smem_optin - reserve - 64;
   int pix = smem_room / (boxes * WG_PIX * 128) >= 3 ? WG_PIX : 96;
   if (const char* env = getenv("CONV3D_WGRAD_PIX")) {
     const int v = atoi(env);
     if (!pair && (v == 96 || v == 128)) pix = v;
   }
-  auto kern = wgrad_kernel_for(bf16, swap, pair, pix);
+  auto kern = wgrad_kernel_for(bf16, swap, pair, pix, bias_block);
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    const int kind = swap ? 2 : pair ? 1 : 0;
+    const int kind = bias_block ? 3 : swap ? 2 : pair ? 1 : 0;
     const int wg_variant = 4 * kind + 2 * (pix == 96 ? 1 : 0) + (bf16 ? 1 : 0);
     cudaError_t e = cudaSuccess;
     if (!S->wg_attr_set[wg_variant]) {
@@ -1929,7 +1956,7 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
   const long long base_units =
       swap   ? static_cast<long long>(kt_run) * wp.eblocks * wp.co_tiles
       : pair ? static_cast<long long>(kt_run) * wp.pairs_per_it * wp.co_tiles
-             : static_cast<long long>(wp.taps) * wp.cblocks * wp.co_tiles;
+             : (static_cast<long long>(wp.taps) * wp.cblocks + (bias_block ? 1 : 0)) * wp.co_tiles;
   const long long splits = choose_wgrad_splits(base_units, wp.total_chunks, lanes, pix);
   if (base_units * splits > 0x7FFFFFFFLL) {
     set_error("problem too large");
@@ -1988,7 +2015,7 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
   // stream at the same time (forked after the clear, joined before the
   // rounding); CONV3D_WGRAD_DBIAS_SIDE=0 runs it after the kernel instead.
   bool side = false;
-  if (dbias) {
+  if (dbias && !bias_block) {
     const char* env = getenv("CONV3D_WGRAD_DBIAS_SIDE");
     side = (env == nullptr || env[0] != '0') && aux_stream(*S, stream);
   }
@@ -2016,10 +2043,11 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
     if (plan_log())
       fprintf(stderr,
               "libconv3d: weight gradient %s %s, %d units (%d splits of %lld chunks of %d pixels), "
-              "grid %d, %d stages, %zu B shared\n",
+              "grid %d, %d stages, %zu B shared, bias gradient %s\n",
               swap ? "transposed" : pair ? "CTA pair" : "plain", bf16 ? "bf16" : "fp16",
               wp.num_units, wp.splits, wp.total_chunks, pix, static_cast<int>(cfg.gridDim.x),
-              wp.stages, smem);
+              wp.stages, smem,
+              bias_block ? "in the kernel (block of ones)" : dbias ? "in a pass beside it" : "none");
     e = cudaLaunchKernelEx(&cfg, kern, map_x, map_dy, map_p, wp);
     if (e != cudaSuccess) return cuda_fail(e, "wgrad kernel launch");
   }
@@ -2038,7 +2066,7 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
       f32_to_16_kernel<false><<<blocks, 256, 0, stream>>>(dw32, d16, static_cast<long long>(dw_elems));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dw conversion launch");
   }
-  if (dbias) {
+  if (dbias && !bias_block) {
     // 256-channel groups along y; about three blocks per SM in all (as many
     // as fit beside a weight-gradient CTA), the pixels split evenly between
     // the blocks of a group
@@ -2066,6 +2094,8 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
       if (e != cudaSuccess) return cuda_fail(e, "aux stream join");
     }
     if (le != cudaSuccess) return cuda_fail(le, "dbias launch");
+  }
+  if (dbias) {
     if (bf16)
       f32_to_16_kernel<true><<<1, 256, 0, stream>>>(db32, static_cast<uint16_t*>(dbias), Cout);
     else

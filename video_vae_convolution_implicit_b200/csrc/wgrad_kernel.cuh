@@ -69,6 +69,8 @@ struct WgradParams {
   uint32_t acc_cols;        // TMEM columns per accumulator (BN plain, 256 swapped)
   uint32_t idesc;
   float* dw;                // [Cout][taps][Cin] fp32, accumulated
+  float* db;                // [Cout] fp32 bias gradient, accumulated (bias block instances)
+  int db_it;                // temporal tap whose frame walk the bias block follows
   int* status;
   unsigned long long timeout_ns;
   int test_stall;           // failure-detection test: the producer skips its first stage's copies
@@ -104,14 +106,16 @@ struct WgUnit {
   int tap, cb;       // plain / pair: tap and 128-channel block of this CTA
   int e0, nent;      // swap: first entry of the block and entries in it (1..ent_per_block)
   bool dup;          // pair: this CTA's block repeats its peer's (odd count): not written
+  bool bias;         // the bias block: A = ones, so every row of the product is sum(dy)
   int co0;
   long long c_begin, c_end;
 };
 
-template <bool kSwap, bool kPair>
+template <bool kSwap, bool kPair, bool kBias = false>
 __device__ __forceinline__ WgUnit wg_decode(const WgradParams& p, int u, uint32_t rank = 0) {
   WgUnit r;
   r.dup = false;
+  r.bias = false;
   // split-major: the units that run at the same time share a pixel range, so
   // x and dy come from DRAM about once and serve every tap block from L2
   const int per_split = p.num_units / p.splits;
@@ -137,6 +141,12 @@ __device__ __forceinline__ WgUnit wg_decode(const WgradParams& p, int u, uint32_
     r.e0 = (mb - r.it * p.eblocks) * p.ent_per_block;
     r.nent = p.ents - r.e0 < p.ent_per_block ? p.ents - r.e0 : p.ent_per_block;
     r.tap = r.cb = 0;
+  } else if (kBias && mb == p.taps * p.cblocks) {
+    // one more block per output-channel tile: the bias gradient
+    r.bias = true;
+    r.tap = r.cb = 0;
+    r.it = p.db_it;
+    r.e0 = r.nent = 0;
   } else {
     r.tap = mb / p.cblocks;
     r.cb = mb - r.tap * p.cblocks;
@@ -195,12 +205,18 @@ __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c
 
 // kPix = pixels (K) per stage, a multiple of 16: every operand box is kPix
 // rows of 128 bytes (64 channels), and the A stage holds two of them.
-template <bool kBF16, bool kSwap, bool kPair, int kPix>
+// kBias: the plain variant with one more block per output-channel tile whose
+// A operand is a constant tile of ones in shared memory, so that its product
+// is the bias gradient (every row: the sum of dy over the unit's pixels); the
+// block loads only dy, which the other blocks of the same pixel range bring
+// into L2 at the same time, and its epilogue adds one row to db.
+template <bool kBF16, bool kSwap, bool kPair, int kPix, bool kBias = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     conv3d_wgrad_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_dy,
                         const __grid_constant__ CUtensorMap map_p, const WgradParams p) {
   static_assert(!(kSwap && kPair), "the pair variant is the plain operand assignment");
+  static_assert(!(kBias && (kSwap || kPair)), "the bias block: plain variant only");
   static_assert(kPix % 16 == 0 && kPix <= 256, "pixels per stage");
   constexpr uint32_t kBox = kPix * 128;          // one 64-channel box
   constexpr uint32_t kABytes = 2 * kBox;
@@ -230,6 +246,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tfull_bar = bars + 16 * p.stages;
   const uint32_t tempty_bar = tfull_bar + 16;
   const uint32_t drain_bar = tempty_bar + 16;
+  // bias block: 4 KB of ones, two 64-row blocks (2 KB apart) of 16 pixel rows
+  // in the 128-byte-swizzled MN-major layout -- one K = 16 step, reused for
+  // every step, as all its values are 1
+  const uint32_t ones = (drain_bar + 8 + 1023u) & ~1023u;
   SharedCtl ctl{&s_abort, p.status, p.timeout_ns,
                 kPair ? mapa_shared(smem_addr(&s_abort), rank ^ 1u) : 0u};
   const uint32_t peer_bar = smem_addr(&s_peer_bar);
@@ -261,6 +281,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_relinquish();
     }
   }
+  if constexpr (kBias) {
+    if (warp >= 2) {   // the epilogue warps fill the ones, then make them visible to the MMAs
+      const uint32_t one2 = kBF16 ? 0x3F803F80u : 0x3C003C00u;
+      for (uint32_t i = threadIdx.x - 64u; i < 1024u; i += NUM_THREADS - 64u)
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(ones + 4u * i), "r"(one2) : "memory");
+      fence_proxy_async_shared();
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if constexpr (kPair) cluster_sync();   // the peer's barriers are initialised
@@ -277,7 +305,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // one CTA's share of a stage (the same for every unit of a pair)
       const uint32_t half_bytes = static_cast<uint32_t>(2 + p.BN / 64 / kCtas) * kBox;
       for (int u = first_unit; ok && u < p.num_units; u += unit_step) {
-        const WgUnit wu = wg_decode<kSwap, kPair>(p, u, rank);
+        const WgUnit wu = wg_decode<kSwap, kPair, kBias>(p, u, rank);
         // The im2col boxes of the unit: (kw offset, kh offset, first channel).
         // A box whose channels all lie past Cin (or past Cout for dy) is loaded
         // from the unit's first box instead: those rows/columns of the product
@@ -295,7 +323,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             bw[j] = sp - bh[j] * p.kw;
           }
         } else {
-          nx = 2;
+          nx = (kBias && wu.bias) ? 0 : 2;   // the bias block loads dy only
           const int sp = wu.tap - wu.it * p.kh * p.kw;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -389,8 +417,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // (bits 0-13, in 16-byte units) only
       const uint64_t da0 = smem_desc_mn_sw128(a_ring, kBox);
       const uint64_t db0 = smem_desc_mn_sw128(b_ring, kBox);
+      const uint64_t d_ones = smem_desc_mn_sw128(ones, 2048);   // bias block: the same K step each time
       for (int u = first_unit; ok && u < p.num_units; u += unit_step, ++local) {
-        const WgUnit wu = wg_decode<kSwap, kPair>(p, u);
+        const WgUnit wu = wg_decode<kSwap, kPair, kBias>(p, u);
         // swapped: N = 64 per entry of the block
         const uint32_t idesc =
             kSwap ? (p.idesc & ~(0x3Fu << 17)) | (static_cast<uint32_t>(wu.nent * 64 >> 3) << 17)
@@ -412,6 +441,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tc_fence_after();
             const uint64_t da = da0 + ((stage * kABytes) >> 4);
             const uint64_t db = db0 + ((stage * b_stage_bytes) >> 4);
+            const bool ones_a = kBias && wu.bias;
 #pragma unroll
             for (int k = 0; k < kPix / 16; ++k) {
               // 16 pixels = two 8-row groups (2 KB) further along K
@@ -419,7 +449,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 mma_f16_ss_pair(d_tmem, da + k * (2048 >> 4), db + k * (2048 >> 4), idesc,
                                 accumulate);
               else
-                mma_f16_ss(d_tmem, da + k * (2048 >> 4), db + k * (2048 >> 4), idesc, accumulate);
+                mma_f16_ss(d_tmem, ones_a ? d_ones : da + k * (2048 >> 4), db + k * (2048 >> 4),
+                           idesc, accumulate);
               accumulate = 1;
             }
             if constexpr (kPair) {
@@ -463,7 +494,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!wait_bounded(tfull_bar + 8 * acc, acc_phase, ctl, true)) break;
       tc_fence_after();
-      const WgUnit wu = wg_decode<kSwap, kPair>(p, u, rank);
+      const WgUnit wu = wg_decode<kSwap, kPair, kBias>(p, u, rank);
       // a unit whose chunks all read zero padding issued no MMA: nothing to add
       bool any = false;
       FrameWalk fw(p, wu);
@@ -488,6 +519,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int q = 0; q < 8; ++q)
               red_add_v4(dst + 4 * q, __uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
                          __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+          }
+        }
+      } else if (kBias && wu.bias) {
+        // every row of the bias block holds sum(dy): row 0 (lane 0 of the
+        // first quarter) is added to db, 16 bytes at a time
+        if (quarter == 0) {
+          for (int j = 0; j < p.BN / 32; ++j) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + j * 32, r);
+            tmem_ld_wait();
+            const int c0 = wu.co0 + j * 32;
+            if (any && lane == 0) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                if (c0 + 4 * q < p.Cout)
+                  red_add_v4(p.db + c0 + 4 * q, __uint_as_float(r[4 * q]),
+                             __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                             __uint_as_float(r[4 * q + 3]));
+            }
           }
         }
       } else {
