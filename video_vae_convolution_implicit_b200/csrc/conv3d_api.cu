@@ -2060,10 +2060,14 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
       f32_to_16_bcast_kernel<true><<<blocks, 256, 0, stream>>>(dw32, d16, Cout, F.kt, run_per_co);
     else if (frame0)
       f32_to_16_bcast_kernel<false><<<blocks, 256, 0, stream>>>(dw32, d16, Cout, F.kt, run_per_co);
-    else if (bf16)
-      f32_to_16_kernel<true><<<blocks, 256, 0, stream>>>(dw32, d16, static_cast<long long>(dw_elems));
+    else if (bf16)   // with the bias block, db is final here too: one launch for both
+      f32_to_16_kernel<true><<<blocks, 256, 0, stream>>>(
+          dw32, d16, static_cast<long long>(dw_elems), db32, static_cast<uint16_t*>(dbias),
+          dbias && bias_block ? Cout : 0);
     else
-      f32_to_16_kernel<false><<<blocks, 256, 0, stream>>>(dw32, d16, static_cast<long long>(dw_elems));
+      f32_to_16_kernel<false><<<blocks, 256, 0, stream>>>(
+          dw32, d16, static_cast<long long>(dw_elems), db32, static_cast<uint16_t*>(dbias),
+          dbias && bias_block ? Cout : 0);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dw conversion launch");
   }
   if (dbias && !bias_block) {
@@ -2095,7 +2099,7 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
     }
     if (le != cudaSuccess) return cuda_fail(le, "dbias launch");
   }
-  if (dbias) {
+  if (dbias && (!bias_block || frame0)) {   // (else rounded with dw above)
     if (bf16)
       f32_to_16_kernel<true><<<1, 256, 0, stream>>>(db32, static_cast<uint16_t*>(dbias), Cout);
     else

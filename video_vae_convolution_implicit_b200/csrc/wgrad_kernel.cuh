@@ -582,14 +582,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-// fp32 accumulation -> the 16-bit weight gradient (one rounding).
+// fp32 accumulation -> the 16-bit weight gradient (one rounding); the n2
+// values of a second array (the bias gradient) in the same launch.
 template <bool kBF16>
 __global__ void f32_to_16_kernel(const float* __restrict__ src, uint16_t* __restrict__ dst,
-                                 long long n) {
+                                 long long n, const float* __restrict__ src2 = nullptr,
+                                 uint16_t* __restrict__ dst2 = nullptr, long long n2 = 0) {
   using C = Cvt<kBF16>;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x)
-    dst[i] = static_cast<uint16_t>(C::pack(src[i], 0.0f) & 0xFFFFu);
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n + n2;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    if (i < n)
+      dst[i] = static_cast<uint16_t>(C::pack(src[i], 0.0f) & 0xFFFFu);
+    else
+      dst2[i - n] = static_cast<uint16_t>(C::pack(src2[i - n], 0.0f) & 0xFFFFu);
+  }
 }
 
 // The same rounding, written to each of kt equal temporal taps:
