@@ -248,14 +248,12 @@ CONV3D_API conv3d_status_t conv3d_fwd_gn(const void* x, const double* stats, con
  * padding (kh-1-ph, kw-1-pw spatially; kt-1-pf in front temporally); with
  * causal replicate padding the gradient of the kt-1 virtual frames in front
  * is added to frame 0.  Runs the forward kernel on dy, after a weight
- * transform into the workspace; with causal replicate padding it runs twice
- * (frames 1.. straight into dx, one launch per sample; the kt frames
- * -(kt-1)..0 in fp32 into the workspace, summed into frame 0 with one
- * rounding).  For short clips (D - 1 <= 4 kt) the front frames run on a
- * library-owned high-priority stream, forked from and joined back into
- * `stream` with events (so the call still orders after and before the
- * caller's work on `stream`, and can be captured in a CUDA graph), beside the
- * body on `stream`.
+ * transform into the workspace; with causal replicate padding one launch
+ * covers the output frames -(kt-1)..D-1 of every sample: frames 1.. go
+ * straight into dx, the kt frames -(kt-1)..0 in fp32 into the workspace, and
+ * a last kernel sums them into frame 0 with one rounding.  A single frame
+ * (D = 1) takes the forward pass's first-frame fold, its weight mirrored and
+ * folded by one kernel.  Everything runs on `stream`.
  *
  * Arguments describe the FORWARD problem: dy is [N, Do, Ho, Wo, Cout] (y's
  * shape), w [Cout, kt, kh, kw, Cin], dx [N, D, H, W, Cin] (written).  Supported:
@@ -292,7 +290,12 @@ CONV3D_API size_t conv3d_bwd_data_workspace_bytes(int N, int Cin, int D, int H, 
  * dy[.., co] * Xpad[.., tap-shifted, ci] (the same implicit im2col matrix the
  * forward pass reads, with the same padding rules), dbias[co] = sum of dy.
  * Accumulated in fp32 in the workspace (split over pixel ranges, fp32
- * atomics: the summation order varies from run to run), rounded once.
+ * atomics: the summation order varies from run to run), rounded once.  dbias:
+ * for a single tap (1x1x1) a block of the kernel itself sums dy; otherwise a
+ * pass over dy runs beside the kernel on the library's auxiliary stream,
+ * forked from and joined back into `stream` with events (the call still
+ * orders after and before the caller's work on `stream`, and can be captured
+ * in a CUDA graph).
  *
  * Arguments describe the FORWARD problem: x [N, D, H, W, Cin], dy [N, Do, Ho,
  * Wo, Cout], dw [Cout, kt, kh, kw, Cin] (written), dbias [Cout] or NULL.
@@ -381,8 +384,8 @@ CONV3D_API const char* conv3d_status_string(conv3d_status_t status);
 CONV3D_API const char* conv3d_last_error(void);
 
 /* Frees the cached per-device workspace, the cached tensor maps and the
- * backward pass's auxiliary stream.  Not to be called while work that uses
- * them is being enqueued. */
+ * auxiliary stream (which the weight gradient's bias pass runs on).  Not to be
+ * called while work that uses them is being enqueued. */
 CONV3D_API void conv3d_release(void);
 
 /* Failure-detection self test: launches one CTA that waits, with the same
