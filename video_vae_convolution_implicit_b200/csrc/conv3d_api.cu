@@ -2052,7 +2052,7 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
     if (e != cudaSuccess) return cuda_fail(e, "wgrad kernel launch");
   }
   {
-    int blocks = static_cast<int>((dw_elems + 255) / 256);
+    int blocks = static_cast<int>((dw_elems / 8 + 255) / 256);   // 8 values a thread
     if (blocks > 8 * S->num_sms) blocks = 8 * S->num_sms;
     uint16_t* d16 = static_cast<uint16_t*>(dw);
     const long long run_per_co = taps_run * Cin;

@@ -582,34 +582,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// 8 fp32 values -> 8 rounded 16-bit ones (16 bytes).
+template <bool kBF16>
+__device__ __forceinline__ uint4 round8(const float* __restrict__ src) {
+  using C = Cvt<kBF16>;
+  const float4 a = *reinterpret_cast<const float4*>(src);
+  const float4 b = *reinterpret_cast<const float4*>(src + 4);
+  return make_uint4(C::pack(a.x, a.y), C::pack(a.z, a.w), C::pack(b.x, b.y), C::pack(b.z, b.w));
+}
+
 // fp32 accumulation -> the 16-bit weight gradient (one rounding); the n2
-// values of a second array (the bias gradient) in the same launch.
+// values of a second array (the bias gradient) in the same launch.  8 values
+// per thread: n and n2 are multiples of 8 and every pointer 16-byte aligned.
 template <bool kBF16>
 __global__ void f32_to_16_kernel(const float* __restrict__ src, uint16_t* __restrict__ dst,
                                  long long n, const float* __restrict__ src2 = nullptr,
                                  uint16_t* __restrict__ dst2 = nullptr, long long n2 = 0) {
-  using C = Cvt<kBF16>;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n + n2;
+  const long long v1 = n / 8, v = v1 + n2 / 8;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < v;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    if (i < n)
-      dst[i] = static_cast<uint16_t>(C::pack(src[i], 0.0f) & 0xFFFFu);
+    if (i < v1)
+      reinterpret_cast<uint4*>(dst)[i] = round8<kBF16>(src + 8 * i);
     else
-      dst2[i - n] = static_cast<uint16_t>(C::pack(src2[i - n], 0.0f) & 0xFFFFu);
+      reinterpret_cast<uint4*>(dst2)[i - v1] = round8<kBF16>(src2 + 8 * (i - v1));
   }
 }
 
 // The same rounding, written to each of kt equal temporal taps:
-// dst[co][it][s] = src[co][s] for s < per_co (kh * kw * Cin entries).
+// dst[co][it][s] = src[co][s] for s < per_co (kh * kw * Cin entries, a
+// multiple of 8), 8 values per thread.
 template <bool kBF16>
 __global__ void f32_to_16_bcast_kernel(const float* __restrict__ src, uint16_t* __restrict__ dst,
                                        int Cout, int kt, long long per_co) {
-  using C = Cvt<kBF16>;
-  const long long n = static_cast<long long>(Cout) * kt * per_co;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+  const long long v = static_cast<long long>(Cout) * kt * per_co / 8;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < v;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long co = i / (kt * per_co);
-    const long long s = i % per_co;
-    dst[i] = static_cast<uint16_t>(C::pack(src[co * per_co + s], 0.0f) & 0xFFFFu);
+    const long long e = 8 * i;
+    const long long co = e / (kt * per_co);
+    const long long s = e % per_co;
+    reinterpret_cast<uint4*>(dst)[i] = round8<kBF16>(src + co * per_co + s);
   }
 }
 
