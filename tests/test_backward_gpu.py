@@ -158,6 +158,30 @@ def test_bwd_weight_single_tap_bias_block(case, block, monkeypatch):
     assert_close(dw.double().cpu().numpy(), ref_dw, f"dw {case} block={block}")
 
 
+@pytest.mark.parametrize("mix", ["1", "0"])
+@pytest.mark.parametrize("case", [WEIGHT_CASES[i] for i in (0, 2, 6, 7, 11)],
+                         ids=lambda c: "x".join(map(str, c[:6])) + f"-p{c[8][0]}-t{c[9]}-{c[10]}")
+def test_bwd_weight_swapped_entry_blocks_across_taps(case, mix, monkeypatch):
+    """The swapped weight gradient numbers its 64-channel entries across the
+    temporal taps (CONV3D_WGRAD_MIX=1, the default where a tap's entries do not
+    fill whole blocks): a block may hold entries of two taps, and a tap that
+    reads zero padding for a frame loads zeros.  Against the oracle either way,
+    including a temporal pad wider than the kernel reaches."""
+    monkeypatch.setenv("CONV3D_WGRAD_SWAP", "1")
+    monkeypatch.setenv("CONV3D_WGRAD_MIX", mix)
+    N, Cin, D, H, W, Cout, k, stride, pad, tpad, dt = case
+    if Cin % 64:
+        pytest.skip("the swapped weight gradient needs Cin % 64 == 0")
+    x, w, dy, od = grads_problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=490 + Cin, dt=dt,
+                                 stride=stride)
+    dw, db = c3.conv3d_bwd_weight(x, dy, k, stride, pad, tpad)
+    assert c3.poll_status() == c3.Status.OK
+    _, ref_dw, ref_db = oracle.conv3d_backward(si.bits(x), si.bits(w), si.bits(dy), od, k, stride,
+                                               pad, tpad)
+    assert_close(dw.double().cpu().numpy(), ref_dw, f"dw {case} mix={mix}")
+    assert_close(db.double().cpu().numpy(), ref_db, f"dbias {case} mix={mix}")
+
+
 # ------------------------------------------------------ full-size workloads, sampled
 
 from seeded_inputs.workloads import WORKLOADS  # noqa: E402

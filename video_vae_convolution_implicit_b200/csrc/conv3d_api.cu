@@ -433,7 +433,7 @@ struct DeviceState {
   bool attr_set[512] = {};       // per kernel instance: variant + 8 * features (< 64)
   int pair_clusters = 0;         // co-resident CTA pairs (occupancy query)
   int wg_pair_clusters = 0;      // the same for the weight-gradient kernel
-  bool wg_attr_set[16] = {};     // per weight-gradient kernel variant (4 kinds x pix x dtype)
+  bool wg_attr_set[32] = {};     // per weight-gradient kernel variant (5 kinds x pix x dtype)
   // Second stream (highest priority) on which the data gradient's front frames
   // run beside its body; created on first use, never if creation fails.
   cudaStream_t aux = nullptr;
@@ -1486,7 +1486,10 @@ using WgradKernel = decltype(&conv3d_wgrad_kernel<true, false, false, WG_PIX>);
 // two stages (see the launch code).  CTA pairs always fit three 128-pixel
 // stages (96-pixel ones measured no faster), so they have one instance.
 template <bool kBF16>
-WgradKernel wgrad_kernel_of(bool swap, bool pair, int pix, bool bias) {
+WgradKernel wgrad_kernel_of(bool swap, bool pair, int pix, bool bias, bool mix) {
+  if (mix)
+    return pix == 96 ? conv3d_wgrad_kernel<kBF16, true, false, 96, false, true>
+                     : conv3d_wgrad_kernel<kBF16, true, false, 128, false, true>;
   if (bias)
     return pix == 96 ? conv3d_wgrad_kernel<kBF16, false, false, 96, true>
                      : conv3d_wgrad_kernel<kBF16, false, false, 128, true>;
@@ -1498,9 +1501,9 @@ WgradKernel wgrad_kernel_of(bool swap, bool pair, int pix, bool bias) {
                    : conv3d_wgrad_kernel<kBF16, false, false, 128>;
 }
 
-WgradKernel wgrad_kernel_for(bool bf16, bool swap, bool pair, int pix, bool bias) {
-  return bf16 ? wgrad_kernel_of<true>(swap, pair, pix, bias)
-              : wgrad_kernel_of<false>(swap, pair, pix, bias);
+WgradKernel wgrad_kernel_for(bool bf16, bool swap, bool pair, int pix, bool bias, bool mix) {
+  return bf16 ? wgrad_kernel_of<true>(swap, pair, pix, bias, mix)
+              : wgrad_kernel_of<false>(swap, pair, pix, bias, mix);
 }
 
 // Number of pixel ranges each (tap block, output-channel tile) is split into.
@@ -1918,10 +1921,17 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
     const int v = atoi(env);
     if (!pair && (v == 96 || v == 128)) pix = v;
   }
-  auto kern = wgrad_kernel_for(bf16, swap, pair, pix, bias_block);
+  // Swapped entry blocks numbered across the temporal taps, so that only the
+  // last block of all is partly filled (with 18 entries a tap, 14 blocks of
+  // four instead of 15 with three half-filled); a tap that reads zero padding
+  // for a frame then loads zeros instead of skipping the chunk.
+  // CONV3D_WGRAD_MIX=0 keeps the blocks within one temporal tap.
+  bool mix = swap && kt_run > 1 && wp.ents % wp.ent_per_block != 0;
+  if (const char* env = getenv("CONV3D_WGRAD_MIX")) mix = mix && env[0] != '0';
+  auto kern = wgrad_kernel_for(bf16, swap, pair, pix, bias_block, mix);
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    const int kind = bias_block ? 3 : swap ? 2 : pair ? 1 : 0;
+    const int kind = mix ? 4 : bias_block ? 3 : swap ? 2 : pair ? 1 : 0;
     const int wg_variant = 4 * kind + 2 * (pix == 96 ? 1 : 0) + (bf16 ? 1 : 0);
     cudaError_t e = cudaSuccess;
     if (!S->wg_attr_set[wg_variant]) {
@@ -1954,7 +1964,8 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
   wp.chunks_per_frame = (wp.HoWo + pix - 1) / pix;
   wp.total_chunks = static_cast<long long>(N) * F.Do * wp.chunks_per_frame;
   const long long base_units =
-      swap   ? static_cast<long long>(kt_run) * wp.eblocks * wp.co_tiles
+      swap   ? (mix ? (static_cast<long long>(kt_run) * wp.ents + wp.ent_per_block - 1) / wp.ent_per_block
+                    : static_cast<long long>(kt_run) * wp.eblocks) * wp.co_tiles
       : pair ? static_cast<long long>(kt_run) * wp.pairs_per_it * wp.co_tiles
              : (static_cast<long long>(wp.taps) * wp.cblocks + (bias_block ? 1 : 0)) * wp.co_tiles;
   const long long splits = choose_wgrad_splits(base_units, wp.total_chunks, lanes, pix);
@@ -2044,7 +2055,9 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
       fprintf(stderr,
               "libconv3d: weight gradient %s %s, %d units (%d splits of %lld chunks of %d pixels), "
               "grid %d, %d stages, %zu B shared, bias gradient %s\n",
-              swap ? "transposed" : pair ? "CTA pair" : "plain", bf16 ? "bf16" : "fp16",
+              swap ? (mix ? "transposed (entry blocks across taps)" : "transposed")
+                   : pair ? "CTA pair" : "plain",
+              bf16 ? "bf16" : "fp16",
               wp.num_units, wp.splits, wp.total_chunks, pix, static_cast<int>(cfg.gridDim.x),
               wp.stages, smem,
               bias_block ? "in the kernel (block of ones)" : dbias ? "in a pass beside it" : "none");

@@ -111,7 +111,7 @@ struct WgUnit {
   long long c_begin, c_end;
 };
 
-template <bool kSwap, bool kPair, bool kBias = false>
+template <bool kSwap, bool kPair, bool kBias = false, bool kMix = false>
 __device__ __forceinline__ WgUnit wg_decode(const WgradParams& p, int u, uint32_t rank = 0) {
   WgUnit r;
   r.dup = false;
@@ -136,6 +136,14 @@ __device__ __forceinline__ WgUnit wg_decode(const WgradParams& p, int u, uint32_
     r.cb = e - sp * p.cblocks;
     r.tap = r.it * p.kh * p.kw + sp;
     r.e0 = r.nent = 0;
+  } else if (kSwap && kMix) {
+    // entries numbered across the temporal taps (entry e: tap e / ents), so
+    // that only the last block of all may be partly filled
+    r.it = 0;
+    r.e0 = mb * p.ent_per_block;
+    const int all = p.kt * p.ents;
+    r.nent = all - r.e0 < p.ent_per_block ? all - r.e0 : p.ent_per_block;
+    r.tap = r.cb = 0;
   } else if (kSwap) {
     r.it = mb / p.eblocks;
     r.e0 = (mb - r.it * p.eblocks) * p.ent_per_block;
@@ -210,13 +218,14 @@ __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c
 // is the bias gradient (every row: the sum of dy over the unit's pixels); the
 // block loads only dy, which the other blocks of the same pixel range bring
 // into L2 at the same time, and its epilogue adds one row to db.
-template <bool kBF16, bool kSwap, bool kPair, int kPix, bool kBias = false>
+template <bool kBF16, bool kSwap, bool kPair, int kPix, bool kBias = false, bool kMix = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     conv3d_wgrad_kernel(const __grid_constant__ CUtensorMap map_x,
                         const __grid_constant__ CUtensorMap map_dy,
                         const __grid_constant__ CUtensorMap map_p, const WgradParams p) {
   static_assert(!(kSwap && kPair), "the pair variant is the plain operand assignment");
   static_assert(!(kBias && (kSwap || kPair)), "the bias block: plain variant only");
+  static_assert(!kMix || kSwap, "entry blocks across temporal taps: swapped variant only");
   static_assert(kPix % 16 == 0 && kPix <= 256, "pixels per stage");
   constexpr uint32_t kBox = kPix * 128;          // one 64-channel box
   constexpr uint32_t kABytes = 2 * kBox;
@@ -305,18 +314,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // one CTA's share of a stage (the same for every unit of a pair)
       const uint32_t half_bytes = static_cast<uint32_t>(2 + p.BN / 64 / kCtas) * kBox;
       for (int u = first_unit; ok && u < p.num_units; u += unit_step) {
-        const WgUnit wu = wg_decode<kSwap, kPair, kBias>(p, u, rank);
+        const WgUnit wu = wg_decode<kSwap, kPair, kBias, kMix>(p, u, rank);
         // The im2col boxes of the unit: (kw offset, kh offset, first channel).
         // A box whose channels all lie past Cin (or past Cout for dy) is loaded
         // from the unit's first box instead: those rows/columns of the product
         // are never written out, and every copy starts in bounds.
-        int bw[4], bh[4], bc[4];
+        int bw[4], bh[4], bc[4], bt[4];   // bt: temporal tap of the box (kMix)
         int nx;
         if (kSwap) {
           nx = wu.nent;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int e = wu.e0 + (j < nx ? j : 0);
+            int e = wu.e0 + (j < nx ? j : 0);
+            bt[j] = kMix ? e / p.ents : wu.it;
+            if (kMix) e -= bt[j] * p.ents;
             const int sp = e / p.c64s;
             bc[j] = (e - sp * p.c64s) * 64;
             bh[j] = sp / p.kw;
@@ -344,10 +355,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         FrameWalk fw(p, wu);
         while (ok && fw.next(p)) {
           const int f = wg_source_frame(p, fw.to, wu.it);
-          if (f == kNoFrame) continue;          // this tap reads zero padding here
+          if (!kMix && f == kNoFrame) continue;   // this tap reads zero padding here
           // frames before the chunk come from the cached-frames tensor
           const CUtensorMap* xmap = f < 0 ? &map_p : &map_x;
           const int img = f < 0 ? fw.n * (p.kt - 1) + (p.kt - 1) + f : fw.n * p.D + f;
+          // kMix: each box's own frame; a tap that reads zero padding loads an
+          // image index past the tensor, which the copy fills with zeros
+          const CUtensorMap* bmap[4];
+          int bimg[4];
+          if constexpr (kMix) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int fq = wg_source_frame(p, fw.to, bt[q]);
+              bmap[q] = fq != kNoFrame && fq < 0 ? &map_p : &map_x;
+              bimg[q] = fq == kNoFrame ? -1
+                        : fq < 0       ? fw.n * (p.kt - 1) + (p.kt - 1) + fq
+                                       : fw.n * p.D + fq;
+            }
+          }
           int p0 = fw.pc * kPix;
           int ho0 = p0 / p.Wo;
           int wo0 = p0 - ho0 * p.Wo;
@@ -382,8 +407,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int q = 0; q < 4; ++q)
                 if (q < nx)
-                  tma_load_im2col_4d(x_dst + q * kBox, xmap, fb, bc[q], wx, hx, img,
-                                     static_cast<uint16_t>(bw[q]), static_cast<uint16_t>(bh[q]));
+                  tma_load_im2col_4d(x_dst + q * kBox, kMix ? bmap[q] : xmap, fb, bc[q], wx, hx,
+                                     kMix ? bimg[q] : img, static_cast<uint16_t>(bw[q]),
+                                     static_cast<uint16_t>(bh[q]));
               for (int q = 0; q < ndy; ++q) {
                 const int dc = dy_c0 + 64 * q < p.Cout ? dy_c0 + 64 * q : wu.co0;
                 tma_load_3d(dy_dst + q * kBox, &map_dy, fb, dc, p0,
@@ -419,7 +445,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t db0 = smem_desc_mn_sw128(b_ring, kBox);
       const uint64_t d_ones = smem_desc_mn_sw128(ones, 2048);   // bias block: the same K step each time
       for (int u = first_unit; ok && u < p.num_units; u += unit_step, ++local) {
-        const WgUnit wu = wg_decode<kSwap, kPair, kBias>(p, u);
+        const WgUnit wu = wg_decode<kSwap, kPair, kBias, kMix>(p, u);
         // swapped: N = 64 per entry of the block
         const uint32_t idesc =
             kSwap ? (p.idesc & ~(0x3Fu << 17)) | (static_cast<uint32_t>(wu.nent * 64 >> 3) << 17)
@@ -432,7 +458,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t accumulate = 0;
         FrameWalk fw(p, wu);
         while (ok && fw.next(p)) {
-          if (wg_source_frame(p, fw.to, wu.it) == kNoFrame) continue;
+          if (!kMix && wg_source_frame(p, fw.to, wu.it) == kNoFrame) continue;
           for (int j = 0; j < fw.count; ++j) {
             if (!wait_bounded(full_bar + 8 * stage, phase, ctl, true)) {
               ok = false;
@@ -494,11 +520,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t acc_phase = (local >> 1) & 1;
       if (!wait_bounded(tfull_bar + 8 * acc, acc_phase, ctl, true)) break;
       tc_fence_after();
-      const WgUnit wu = wg_decode<kSwap, kPair, kBias>(p, u, rank);
+      const WgUnit wu = wg_decode<kSwap, kPair, kBias, kMix>(p, u, rank);
       // a unit whose chunks all read zero padding issued no MMA: nothing to add
       bool any = false;
       FrameWalk fw(p, wu);
-      while (!any && fw.next(p)) any = wg_source_frame(p, fw.to, wu.it) != kNoFrame;
+      while (!any && fw.next(p)) any = kMix || wg_source_frame(p, fw.to, wu.it) != kNoFrame;
       const uint32_t t_row =
           tmem_base + ((quarter * 32u) << 16) + acc * static_cast<uint32_t>(p.acc_cols);
       if (kSwap) {
@@ -509,9 +535,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_ld_32x32b_x32(t_row + j * 32, r);
           tmem_ld_wait();
           if (row_ok) {
-            const int e = wu.e0 + j / 2;
+            int e = wu.e0 + j / 2;
+            const int it = kMix ? e / p.ents : wu.it;
+            if (kMix) e -= it * p.ents;
             const int sp = e / p.c64s;
-            const int tap = wu.it * p.kh * p.kw + sp;
+            const int tap = it * p.kh * p.kw + sp;
             const int ci0 = (e - sp * p.c64s) * 64 + (j & 1) * 32;
             float* dst = p.dw + static_cast<long long>(co) * K +
                          static_cast<long long>(tap) * p.Cin + ci0;
