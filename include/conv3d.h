@@ -249,9 +249,12 @@ CONV3D_API conv3d_status_t conv3d_fwd_gn(const void* x, const double* stats, con
  * causal replicate padding the gradient of the kt-1 virtual frames in front
  * is added to frame 0.  Runs the forward kernel on dy, after a weight
  * transform into the workspace; with causal replicate padding one launch
- * covers the output frames -(kt-1)..D-1 of every sample: frames 1.. go
- * straight into dx, the kt frames -(kt-1)..0 in fp32 into the workspace, and
- * a last kernel sums them into frame 0 with one rounding.  A single frame
+ * covers every frame: when it has at least 4 rounds of tiles (one tile per
+ * SM a round) the tiles of frame 0 also run the taps of the kt-1 virtual
+ * frames, into the same fp32 accumulator (one rounding); with fewer, the
+ * launch writes the kt parts of frame 0 (frames -(kt-1)..0) in fp32 into the
+ * workspace beside frames 1.. in dx, and a last kernel sums them into frame 0
+ * with one rounding.  A single frame
  * (D = 1) takes the forward pass's first-frame fold, its weight mirrored and
  * folded by one kernel.  Everything runs on `stream`.
  *

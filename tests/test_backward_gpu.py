@@ -207,6 +207,7 @@ def test_bwd_data_full_size_sampled(name):
     rng = np.random.default_rng(5)
     pix = {0, wl.W - 1, HW - 1, HW // 2 + wl.W // 2, total - 1, (wl.D - 1) * HW}
     pix |= {int(v) for v in rng.integers(0, total, 40)}
+    pix |= {int(v) for v in rng.integers(0, HW, 16)}    # frame 0: the replicated copies' sum
     pix = np.array(sorted(pix), dtype=np.int64)
     ref = oracle.conv3d_dx_at(si.bits(w), si.bits(dy), od, x.shape, wl.kernel, wl.stride, wl.pad,
                               wl.tpad, pix)
@@ -242,12 +243,16 @@ def test_bwd_data_deterministic_bitwise():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+@pytest.mark.parametrize("combine", ["1", "0"])
 @pytest.mark.parametrize("D", [2, 4, 20])
-def test_bwd_data_causal_one_launch_on_a_side_stream(D):
-    """Under causal replicate padding one launch writes the kt fp32 parts of
-    frame 0 and the 16-bit frames 1.. of every sample (mixed output), then the
-    fold rounds frame 0: every element against the oracle, on a stream other
-    than the default one, whose later work sees the finished dx."""
+def test_bwd_data_causal_one_launch_on_a_side_stream(D, combine, monkeypatch):
+    """Under causal replicate padding one launch computes every frame: with
+    CONV3D_DGRAD_COMBINE=1 frame 0's tiles also run the taps of its kt-1
+    replicated copies into the same accumulator; with 0 the launch writes the
+    kt fp32 parts of frame 0 beside the 16-bit frames 1.. (mixed output) and a
+    fold rounds frame 0.  Every element against the oracle, on a stream
+    other than the default one, whose later work sees the finished dx."""
+    monkeypatch.setenv("CONV3D_DGRAD_COMBINE", combine)
     x, w, dy, od = grads_problem(2, 64, D, 8, 10, 64, (3, 3, 3), (0, 1, 1), CREP, 23, "bf16")
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -297,6 +302,24 @@ STRIDED_DATA_CASES = [
 
 @pytest.mark.parametrize("case", STRIDED_DATA_CASES, ids=lambda c: "x".join(map(str, c[:6])) + f"-s{''.join(map(str, c[7]))}-t{c[9]}-{c[10]}")
 def test_bwd_data_strided_every_element(case, variant):
+    N, Cin, D, H, W, Cout, k, stride, pad, tpad, dt = case
+    x, w, dy, od = grads_problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=700 + Cin, dt=dt,
+                                 stride=stride)
+    dx = torch.full(x.shape, float("nan"), dtype=x.dtype, device="cuda")
+    dx = c3.conv3d_bwd_data(dy, w, x.shape, pad, tpad, dx=dx, stride=stride)
+    assert c3.poll_status() == c3.Status.OK
+    ref, _, _ = oracle.conv3d_backward(si.bits(x), si.bits(w), si.bits(dy), od, k, stride, pad,
+                                       tpad)
+    assert_close(dx.double().cpu().numpy(), ref, str(case))
+
+
+@pytest.mark.parametrize("case", [c for c in STRIDED_DATA_CASES if c[9] == CREP and c[2] > 1],
+                         ids=lambda c: "x".join(map(str, c[:6])) + f"-s{''.join(map(str, c[7]))}")
+def test_bwd_data_strided_combined_front(case, monkeypatch):
+    """CONV3D_DGRAD_COMBINE=1 on the strided causal cases (whose few tiles would
+    otherwise take the fp32 front frames and the fold): each phase's frame-0
+    tiles also run the taps of the replicated copies, straight into dx."""
+    monkeypatch.setenv("CONV3D_DGRAD_COMBINE", "1")
     N, Cin, D, H, W, Cout, k, stride, pad, tpad, dt = case
     x, w, dy, od = grads_problem(N, Cin, D, H, W, Cout, k, pad, tpad, seed=700 + Cin, dt=dt,
                                  stride=stride)

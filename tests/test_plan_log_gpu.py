@@ -28,6 +28,7 @@ assert c3.poll_status() == c3.Status.OK
 def _run(log):
     env = dict(os.environ)
     env.pop("CONV3D_LOG", None)
+    env["CONV3D_DGRAD_COMBINE"] = "1"   # this small case would take the fp32 front frames
     if log:
         env["CONV3D_LOG"] = "1"
     return subprocess.run([sys.executable, "-c", SCRIPT], cwd=ROOT, env=env,
@@ -41,10 +42,10 @@ def test_plan_log_reports_each_launch():
     # forward, then the data gradient (its plan line and its one launch), then
     # the weight gradient
     assert any("implicit GEMM" in l and "16-bit output" in l for l in lines), lines
-    # the data gradient's launch: the fp32 parts of frame 0 beside the 16-bit frames
-    assert any("implicit GEMM" in l and "fp32 (front frames) and 16-bit output" in l
-               for l in lines), lines
-    assert any(l.startswith("libconv3d: data gradient: 3 front frames") for l in lines), lines
+    # the data gradient: one launch whose frame-0 tiles also sum the 2 replicated copies
+    assert any(l.startswith("libconv3d: data gradient: 3 frames x 1 samples in one launch, "
+                            "frame 0 with its 2 replicated copies") for l in lines), lines
+    assert sum("implicit GEMM" in l for l in lines) == 2, lines
     assert any(l.startswith("libconv3d: weight gradient") for l in lines), lines
 
 
@@ -85,3 +86,18 @@ def test_plan_log_shows_the_tail_split():
         assert f"last {tail} tiles in 3 pieces" in lines[0], lines
     else:
         assert "in 1 pieces" in lines[0], lines
+
+
+def test_plan_log_data_gradient_with_fp32_front_frames():
+    """CONV3D_DGRAD_COMBINE=0: the data gradient writes the kt parts of frame 0
+    in fp32 beside the 16-bit frames, then folds them."""
+    env = dict(os.environ)
+    env["CONV3D_LOG"] = "1"
+    env["CONV3D_DGRAD_COMBINE"] = "0"
+    r = subprocess.run([sys.executable, "-c", SCRIPT], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stderr.splitlines() if l.startswith("libconv3d: ")]
+    assert any("implicit GEMM" in l and "fp32 (front frames) and 16-bit output" in l
+               for l in lines), lines
+    assert any(l.startswith("libconv3d: data gradient: 3 front frames") for l in lines), lines

@@ -93,6 +93,10 @@ struct Problem {
   int f32_frames;
   int y_frames;
   void* f32_out;
+  // combined front (internal: the data gradient under causal replicate
+  // padding): output frame 0 also sums the taps of the combine-1 virtual
+  // frames before it (0: off)
+  int combine;
   const void* prev;  // cached frames before the chunk (CONV3D_TPAD_CAUSAL_CACHED) or null
   bool fold;  // first-frame path: fold the temporal taps into a (hi, lo) pair
   // first frame with the lo part in e5m2: lo weights w8 ([Cout][kh*kw][Cin],
@@ -253,6 +257,7 @@ conv3d_status_t validate(const void* x, const void* w, const void* bias, const v
   P.f32_frames = 0;
   P.y_frames = 0;
   P.f32_out = nullptr;
+  P.combine = 0;
   P.lo8 = false;
   P.x8 = nullptr;
   P.w8 = nullptr;
@@ -430,7 +435,7 @@ struct DeviceState {
   };
   Scratch scratch[16] = {};
   int n_scratch = 0;
-  bool attr_set[512] = {};       // per kernel instance: variant + 8 * features (< 64)
+  bool attr_set[1024] = {};      // per kernel instance: variant + 8 * features (< 128)
   int pair_clusters = 0;         // co-resident CTA pairs (occupancy query)
   int wg_pair_clusters = 0;      // the same for the weight-gradient kernel
   bool wg_attr_set[32] = {};     // per weight-gradient kernel variant (5 kinds x pix x dtype)
@@ -701,6 +706,7 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   kp.tpad = P.fold ? 1 : static_cast<int>(P.tpad);
   kp.f32_frames = P.f32_frames;
   kp.y_frames = P.y_frames;
+  kp.combine = P.combine;
   kp.gn_stats = P.gn_stats;
   kp.gn_gamma = static_cast<const uint16_t*>(P.gn_gamma);
   kp.gn_beta = static_cast<const uint16_t*>(P.gn_beta);
@@ -752,6 +758,7 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   // transposed variant)
   if (P.gn_stats || P.gn_out || P.y_scatter) L.pair = false;
   if (P.lo8) L.swap = L.pair = false;   // the e5m2 lo product: one CTA, M = pixels
+  if (P.combine) L.pair = false;
   const int ctas = L.pair ? 2 : 1;
   if (L.swap) {
     kp.co_tile = 128;
@@ -774,7 +781,10 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   // pieces last, their adding-up ended the launch: measured on B200, a
   // 512-tile first frame took 129 us split in two against 124 unsplit.)  Only
   // with scratch for it (the library's own for conv3d_fwd, a region of the
-  // data gradient's workspace), never for CTA pairs or strided outputs.
+  // data gradient's workspace), never for CTA pairs or strided outputs, and
+  // only below 16 rounds: beyond that it saves under 1/16 of the launch, and
+  // data gradients of 57 and 209 rounds (256->512 33x128x128, 128->128
+  // 121x256x256) measured 3% slower with it than without.
   kp.num_items = kp.num_tiles;
   kp.split_first = kp.num_tiles;
   kp.split_s = 1;
@@ -788,7 +798,7 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
     const int kb_nominal = P.lo8 ? P.kh * P.kw * (kp.n_chunks + kp.n_chunks8)
                                  : kt_eff * P.kh * P.kw * kp.n_chunks;
     if (R == 0 && (forced > 0 || T < U)) R = T < U ? T : U;
-    if (forced > 0 || (R > 0 && 2 * R <= U)) {
+    if (forced > 0 || (R > 0 && 2 * R <= U && T < 16 * U)) {
       int sp = forced > 0 ? forced : U / R;
       if (forced < 0) {
         if (sp > 8) sp = 8;
@@ -937,6 +947,12 @@ conv3d_status_t launch_features(DeviceState& S, const LaunchPlan& L, int feat,
       return launch_kernel<kBF16, false, kSwap, FEAT_GN>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_GN | FEAT_STATS:
       return launch_kernel<kBF16, false, kSwap, FEAT_GN | FEAT_STATS>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+    case FEAT_COMBINE:
+      return launch_kernel<kBF16, false, kSwap, FEAT_COMBINE>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+    case FEAT_COMBINE | FEAT_SPLIT:
+      return launch_kernel<kBF16, false, kSwap, FEAT_COMBINE | FEAT_SPLIT>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+    case FEAT_COMBINE | FEAT_SCATTER:
+      return launch_kernel<kBF16, false, kSwap, FEAT_COMBINE | FEAT_SCATTER>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_MIXED:
       return launch_kernel<kBF16, false, kSwap, FEAT_MIXED>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_MIXED | FEAT_SPLIT:
@@ -1006,6 +1022,7 @@ conv3d_status_t launch_planned(DeviceState& S, const Problem& P, LaunchPlan& L, 
   int feat = 0;
   if (P.lo8) feat |= FEAT_LO8;
   if (P.f32_frames > 0) feat |= FEAT_MIXED;
+  if (P.combine) feat |= FEAT_COMBINE;
   if (L.kp.split_s > 1) feat |= FEAT_SPLIT;
   if (P.gn_out) feat |= FEAT_STATS;
   if (P.y_scatter) feat |= FEAT_SCATTER;
@@ -1333,6 +1350,28 @@ conv3d_status_t plan_bwd_data(const void* dy, const void* w, const void* dx, int
   return CONV3D_OK;
 }
 
+// The data gradient under causal replicate padding has two ways to give frame 0
+// the gradient of its kt-1 replicated copies: its tiles run the copies' taps
+// too, into the same accumulator (combined: no fp32 frames, no fold), or one
+// launch writes the kt parts of frame 0 in fp32 beside the 16-bit frames and a
+// fold kernel adds them (mixed).  A combined frame-0 tile carries kt(kt+1)/2
+// taps against kt for the others, and the persistent grid deals tiles out in
+// rounds of one per SM, so with few rounds those tiles set the launch time:
+// measured on B200, 512->128 9x64x64 (144 tiles, one round) took 173 us
+// combined against 131 us mixed, while with 8 or more rounds combined won
+// (128->128 9x256x256: 388 against 439 us; 256->256 9x128x128: 366 against
+// 376).  Combined from 4 rounds of tiles up; CONV3D_DGRAD_COMBINE=0/1 forces
+// the choice.
+bool combine_front(const DeviceState& S, const Problem& T) {
+  const char* e = getenv("CONV3D_DGRAD_COMBINE");
+  if (e != nullptr && (e[0] == '0' || e[0] == '1')) return e[0] == '1';
+  Problem Cb = T;
+  Cb.combine = T.kt;
+  LaunchPlan L;
+  if (plan_launch(S, Cb, T.dtype == CONV3D_BF16, 0, L) != CONV3D_OK) return false;
+  return L.kp.num_tiles >= 4 * S.num_sms;
+}
+
 // dx[n, 0] = the rounded sum of the kt fp32 parts in ext (causal replicate padding).
 conv3d_status_t fold_front(const float* ext, void* dx, int N, int D, int kt,
                            long long frame_elems, conv3d_dtype_t dtype, int sms,
@@ -1431,10 +1470,19 @@ conv3d_status_t bwd_data_phases(DeviceState& S, const BwdDataPlan& B, const void
           return st;
         continue;
       }
-      // causal replicate, D > 1: one launch over output frames -(kt-1)..D-1 of
-      // every sample -- the kt front frames in fp32 (dense, this phase's
-      // pixels), frames 1.. straight to their strided places in dx -- then the
-      // fold into frame 0
+      // causal replicate, D > 1: one launch, frame 0's tiles with the taps of
+      // the kt-1 replicated copies before it
+      if (combine_front(S, T)) {
+        Problem Cb = T;
+        Cb.combine = kt;
+        if ((st = launch_main(S, Cb, dy, nullptr, wt, nullptr, nullptr, dx, stream, split)) !=
+            CONV3D_OK)
+          return st;
+        continue;
+      }
+      // or over output frames -(kt-1)..D-1 of every sample -- the kt front
+      // frames in fp32 (dense, this phase's pixels), frames 1.. straight to
+      // their strided places in dx -- then the fold into frame 0
       float* ext = reinterpret_cast<float*>(ext_at);
       ext_at += static_cast<size_t>(N) * kt * Ah * Aw * Cin * 4;
       Problem Wh = T;
@@ -1759,10 +1807,18 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
 
   float* ext = reinterpret_cast<float*>(static_cast<char*>(workspace) + B.wt_bytes);
   const long long frame_elems = static_cast<long long>(H) * W * Cin;
-  // One launch computes every frame: the kt fp32 parts of frame 0 and the
-  // 16-bit frames 1.., as one persistent grid whose last round the tail split
-  // balances.  (Measured on B200 against a front launch beside a body launch
-  // per sample: 128->512 9x64x64 176 -> 130 us, no change on the larger layers.)
+  // One launch computes every frame: frame 0's tiles also run the taps of the
+  // kt-1 virtual frames before it (the replicated copies), so frame 0 gets
+  // its whole gradient in one accumulator and one rounding -- or, with few
+  // rounds of tiles, frame 0's kt parts go out in fp32 and a fold adds them.
+  if (combine_front(*S, B.tr)) {
+    Problem Cb = B.tr;
+    Cb.combine = kernel[0];
+    if (plan_log())
+      fprintf(stderr, "libconv3d: data gradient: %d frames x %d samples in one launch, frame 0 "
+              "with its %d replicated copies\n", D, N, kernel[0] - 1);
+    return launch_main(*S, Cb, dy, nullptr, wt, nullptr, nullptr, dx, stream, &split);
+  }
   Problem Wh = B.whole;
   Wh.f32_out = ext;
   if (plan_log())

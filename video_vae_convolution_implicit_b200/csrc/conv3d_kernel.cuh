@@ -55,6 +55,7 @@ constexpr int FEAT_SCATTER = 4;    // strided output (data-gradient phases)
 constexpr int FEAT_GN = 8;         // GroupNorm + SiLU of the x operand (4 more warps)
 constexpr int FEAT_LO8 = 16;       // first frame: the lo weight product in e5m2 (kind::f8f6f4)
 constexpr int FEAT_MIXED = 32;     // fp32 front frames and 16-bit frames in one launch (data gradient)
+constexpr int FEAT_COMBINE = 64;   // output frame 0 also sums the kt-1 virtual frames before it
 constexpr int BK8 = 128;           // 8-bit channels per k-block (128-byte rows, like BK 16-bit ones)
 constexpr int GN_THREADS = 320;     // with the GroupNorm + SiLU operand transform (4 more warps)
 constexpr int MAX_STAGES = 8;
@@ -112,6 +113,12 @@ struct KernelParams {
   // (N * y_frames frames).  0: every frame through map_y.
   int f32_frames;
   int y_frames;
+  // Combined front (the data gradient under causal replicate padding,
+  // FEAT_COMBINE): the tiles of output frame 0 also run the taps of the kt-1
+  // virtual frames -1 .. -(kt-1) before it, all into one accumulator, so that
+  // frame 0 gets the gradient of its replicated copies with one rounding.
+  // 0: off (kt when on).
+  int combine;
   int* status;                       // device status word
   unsigned long long timeout_ns;
   int test_stall;                    // failure-detection test: the producer skips the
@@ -229,7 +236,9 @@ __device__ __forceinline__ int source_frame(const KernelParams& p, int to, int i
 
 __device__ __forceinline__ int kblocks_of_tile(const KernelParams& p, int to) {
   int valid = 0;
-  for (int it = 0; it < p.kt; ++it) valid += source_frame(p, to, it) != kNoFrame;
+  const int nv = p.combine > 0 && to == 0 ? p.combine : 1;   // frame 0 and the frames before it
+  for (int v = 0; v < nv; ++v)
+    for (int it = 0; it < p.kt; ++it) valid += source_frame(p, to - v, it) != kNoFrame;
   if (p.n_chunks8 > 0) return p.kh * p.kw * (p.n_chunks + p.n_chunks8);   // folded hi + e5m2 lo
   return valid * p.kh * p.kw * p.n_chunks;
 }
@@ -543,6 +552,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
   constexpr bool kGN = (kFeat & FEAT_GN) != 0;
   constexpr bool kLo8 = (kFeat & FEAT_LO8) != 0;
   constexpr bool kMixed = (kFeat & FEAT_MIXED) != 0;
+  constexpr bool kComb = (kFeat & FEAT_COMBINE) != 0;
   constexpr int kYBufs = 2;   // output staging buffers per epilogue warp
   static_assert(!(kLo8 && (kPair || kSwap)), "the e5m2 lo product: one CTA, M = pixels");
   constexpr int kCtas = kPair ? 2 : 1;
@@ -643,8 +653,11 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
         const int w_org = wo0 * p.sw - p.pw;   // window origin of the first pixel
         const int h_org = ho0 * p.sh - p.ph;
         const int co_b = tl.co0 + static_cast<int>(rank * b_rows);
-        for (int it = 0; ok && kb < kb_hi && it < p.kt; ++it) {
-          const int f = source_frame(p, tl.to, it);
+        // kComb: frame 0's tiles also take the taps of the virtual frames before it
+        const int nvt = (kComb && tl.to == 0 ? p.combine : 1) * p.kt;
+        for (int vt = 0; ok && kb < kb_hi && vt < nvt; ++vt) {
+          const int it = kComb ? vt % p.kt : vt;
+          const int f = source_frame(p, kComb ? tl.to - vt / p.kt : tl.to, it);
           if (f == kNoFrame) continue;
           // frames before the chunk come from the cached-frames tensor
           const CUtensorMap* xmap = f < 0 ? &map_p : &map_a;
