@@ -66,7 +66,7 @@ static int cpu_checks(void) {
   CHECK(conv3d_bwd_weight_workspace_bytes(64, 64, k3) >=
         (size_t)64 * 27 * 64 * 4 + (size_t)64 * 4);
   CHECK(conv3d_bwd_data_workspace_bytes(1, 64, 4, 8, 8, 64, k3, p_zero, CONV3D_TPAD_ZERO) ==
-        (size_t)64 * 27 * 64 * 2 + (size_t)160 * (128 * 256 * 4 + 32));
+        (size_t)64 * 27 * 64 * 2 + (size_t)160 * (128 * 256 * 4 + 64));
   CHECK(conv3d_bwd_data(y, w, dx, 1, 64, 4, 8, 8, 64, k3, st2, p_causal,
                         CONV3D_TPAD_CAUSAL_REPLICATE, CONV3D_BF16, ws, (size_t)1 << 30,
                         NULL) == CONV3D_ERR_UNSUPPORTED);          /* stride 2 */

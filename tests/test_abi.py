@@ -243,7 +243,7 @@ def call_bwd_weight(**kw):
 def test_bwd_workspace_bytes():
     # flipped weight + (replicate padding) the fp32 gradient of frames -2..0
     wt = 64 * 27 * 64 * 2
-    split = 160 * (128 * 256 * 4 + 32)       # the tail-split region: 160 pieces and tickets
+    split = 160 * (128 * 256 * 4 + 64)       # the tail-split region: 160 pieces, 8 tickets each
     assert c3.bwd_data_workspace_bytes(1, 64, 4, 16, 16, 64, (3, 3, 3), (0, 1, 1),
                                        c3.TPAD_CAUSAL_REPLICATE) == wt + 3 * 16 * 16 * 64 * 4 + split
     assert c3.bwd_data_workspace_bytes(2, 64, 4, 16, 16, 64, (3, 3, 3), (1, 1, 1),

@@ -435,7 +435,7 @@ struct DeviceState {
   };
   Scratch scratch[16] = {};
   int n_scratch = 0;
-  bool attr_set[1024] = {};      // per kernel instance: variant + 8 * features (< 128)
+  bool attr_set[2048] = {};      // per kernel instance: variant + 8 * features (< 256)
   int pair_clusters = 0;         // co-resident CTA pairs (occupancy query)
   int wg_pair_clusters = 0;      // the same for the weight-gradient kernel
   bool wg_attr_set[32] = {};     // per weight-gradient kernel variant (5 kinds x pix x dtype)
@@ -659,6 +659,7 @@ struct LaunchPlan {
   bool swap;          // transposed product: M = 128 channels, N = 256 pixels
   KernelParams kp;
   size_t smem;
+  bool epi8;          // 8 epilogue warps
   size_t split_bytes; // scratch of the tail split (partials, then tickets); 0 if none
   size_t split_part_bytes;
 };
@@ -806,24 +807,42 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
       }
       // no more pieces than the scratch holds
       const size_t slot = static_cast<size_t>(BM) * kp.BN * sizeof(float);
-      while (sp >= 2 && static_cast<size_t>(R) * sp * slot + static_cast<size_t>(R) * 32 > split_room)
+      while (sp >= 2 && static_cast<size_t>(R) * sp * slot + static_cast<size_t>(R) * 64 > split_room)
         --sp;
       if (sp >= 2) {
         kp.split_first = T - R;
         kp.split_s = sp;
         kp.num_items = T - R + R * sp;
         L.split_part_bytes = static_cast<size_t>(R) * sp * BM * kp.BN * sizeof(float);
-        L.split_bytes = L.split_part_bytes + static_cast<size_t>(R) * 4 * sizeof(unsigned long long);
+        L.split_bytes = L.split_part_bytes + static_cast<size_t>(R) * 8 * sizeof(unsigned long long);
       }
     }
   }
+  // Eight epilogue warps (two per TMEM lane quarter, each draining every
+  // other 32-column chunk) where a tile has at most 8 k-blocks: there the
+  // MMAs of a tile take less time than draining its 128 x 256 accumulator
+  // through four warps, so the epilogue sets the pace.  Plain and split
+  // launches of one CTA; CONV3D_EPI8=0/1 forces the choice where it applies.
+  {
+    const int kb_tile = P.lo8 ? P.kh * P.kw * (kp.n_chunks + kp.n_chunks8)
+                              : kt_eff * P.kh * P.kw * kp.n_chunks;
+    const bool allowed = !L.pair && !P.gn_stats && !P.gn_out && !P.y_scatter &&
+                         P.f32_frames == 0 && !P.lo8 && P.combine == 0;
+    L.epi8 = allowed && kb_tile <= 8;
+    if (const char* env = getenv("CONV3D_EPI8")) {
+      if (env[0] == '0') L.epi8 = false;
+      if (env[0] == '1') L.epi8 = allowed;
+    }
+  }
+  const int epi_mul = L.epi8 ? 2 : 1;
   const int b_stage = kp.BN / ctas * BK * 2;
   const int stage_bytes = A_STAGE_BYTES + b_stage;
   kp.has_residual = P.has_residual ? 1 : 0;
   kp.out_f32 = P.out_f32 ? 1 : 0;
-  const int reserve = 1024 /*alignment slack*/ + EPI_Y_BYTES * (kp.out_f32 || kp.f32_frames ? 2 : 1) +
-                      EPI_Y_BYTES * (kp.has_residual ? 1 : 0) +
-                      8 * (3 * MAX_STAGES + 5 + 2 * EPI_WARPS);
+  const int reserve = 1024 /*alignment slack*/ +
+                      epi_mul * EPI_Y_BYTES * (kp.out_f32 || kp.f32_frames ? 2 : 1) +
+                      epi_mul * EPI_Y_BYTES * (kp.has_residual ? 1 : 0) +
+                      8 * (3 * MAX_STAGES + 5 + 2 * 2 * EPI_WARPS);
   int stages = (S.max_smem_optin - reserve - 64 /*static smem*/) / stage_bytes;
   if (stages > MAX_STAGES) stages = MAX_STAGES;
   if (stages < 2) {
@@ -847,7 +866,7 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
   constexpr bool kGN = (kFeat & FEAT_GN) != 0;
   auto kern = conv3d_implicit_gemm_kernel<kBF16, kPair, kSwap, kFeat>;
   const int variant = (kBF16 ? 1 : 0) + (kPair ? 2 : 0) + (kSwap ? 4 : 0) + 8 * kFeat;
-  const int threads = kGN ? GN_THREADS : NUM_THREADS;
+  const int threads = kGN ? GN_THREADS : (kFeat & FEAT_EPI8) ? EPI8_THREADS : NUM_THREADS;
   cudaError_t e;
   int units = S.num_sms;  // co-resident CTAs (or CTA pairs)
   {
@@ -910,7 +929,8 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
             "%d k-blocks x %d taps, %d stages, %zu B shared, %s output, last %d tiles in %d "
             "pieces\n",
             kSwap ? "transposed" : kPair ? "CTA pair" : "single",
-            kGN ? " with GroupNorm+SiLU of x" : "", kBF16 ? "bf16" : "fp16",
+            kGN ? " with GroupNorm+SiLU of x" : (kFeat & FEAT_EPI8) ? " with 8 epilogue warps" : "",
+            kBF16 ? "bf16" : "fp16",
             L.kp.num_tiles, L.kp.pix_tile, L.kp.co_tile, static_cast<int>(cfg.gridDim.x),
             L.kp.n_chunks, L.kp.kt * L.kp.kh * L.kp.kw, L.kp.stages, L.smem,
             L.kp.out_f32 ? "fp32" : L.kp.f32_frames ? "fp32 (front frames) and 16-bit" : "16-bit",
@@ -926,10 +946,11 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
 
 // The one-CTA instances with optional parts: the tail split, the output
 // statistics, the strided output, the GroupNorm operand transform (with or
-// without the statistics), the mixed fp32/16-bit output of the data gradient
-// (alone, split, or strided) and the first frame's 8-bit lo product (alone or
-// split).  The plan never combines the split with the statistics, the strided
-// output or the GroupNorm transform.
+// without the statistics), the data gradient's combined front frame and its
+// mixed fp32/16-bit output (each alone, split, or strided), the first frame's
+// 8-bit lo product (alone or split) and the 8 epilogue warps of short-K
+// launches (alone or split).  The plan never combines the split with the
+// statistics, the strided output or the GroupNorm transform.
 template <bool kBF16, bool kSwap>
 conv3d_status_t launch_features(DeviceState& S, const LaunchPlan& L, int feat,
                                 const CUtensorMap& map_a, const CUtensorMap& map_b,
@@ -947,6 +968,10 @@ conv3d_status_t launch_features(DeviceState& S, const LaunchPlan& L, int feat,
       return launch_kernel<kBF16, false, kSwap, FEAT_GN>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_GN | FEAT_STATS:
       return launch_kernel<kBF16, false, kSwap, FEAT_GN | FEAT_STATS>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+    case FEAT_EPI8:
+      return launch_kernel<kBF16, false, kSwap, FEAT_EPI8>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
+    case FEAT_EPI8 | FEAT_SPLIT:
+      return launch_kernel<kBF16, false, kSwap, FEAT_EPI8 | FEAT_SPLIT>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_COMBINE:
       return launch_kernel<kBF16, false, kSwap, FEAT_COMBINE>(S, L, map_a, map_b, map_y, map_r, map_p, map_f, stream);
     case FEAT_COMBINE | FEAT_SPLIT:
@@ -1027,6 +1052,7 @@ conv3d_status_t launch_planned(DeviceState& S, const Problem& P, LaunchPlan& L, 
   if (P.gn_out) feat |= FEAT_STATS;
   if (P.y_scatter) feat |= FEAT_SCATTER;
   if (P.gn_stats) feat |= FEAT_GN;
+  if (L.epi8) feat |= FEAT_EPI8;
   if (feat != 0) {   // never a CTA pair
     if (L.swap)
       return bf16 ? launch_features<true, true>(S, L, feat, map_a, map_b, map_y, map_r, map_p, map_f, stream)
@@ -1258,7 +1284,7 @@ constexpr size_t kPhaseSlack = 64 * 256;
 // 128 x 256 fp32 accumulator and their tickets (160 >= the SMs of a B200, and
 // the split never runs more pieces than SMs).
 constexpr size_t kSplitRegionBytes =
-    ((160 * (static_cast<size_t>(BM) * 256 * sizeof(float) + 32)) + 255) & ~size_t(255);
+    ((160 * (static_cast<size_t>(BM) * 256 * sizeof(float) + 64)) + 255) & ~size_t(255);
 
 struct BwdDataPlan {
   Problem fwd;      // the forward problem being differentiated

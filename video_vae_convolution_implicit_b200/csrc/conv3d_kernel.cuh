@@ -56,8 +56,10 @@ constexpr int FEAT_GN = 8;         // GroupNorm + SiLU of the x operand (4 more 
 constexpr int FEAT_LO8 = 16;       // first frame: the lo weight product in e5m2 (kind::f8f6f4)
 constexpr int FEAT_MIXED = 32;     // fp32 front frames and 16-bit frames in one launch (data gradient)
 constexpr int FEAT_COMBINE = 64;   // output frame 0 also sums the kt-1 virtual frames before it
+constexpr int FEAT_EPI8 = 128;     // 8 epilogue warps, two per TMEM lane quarter (short-K launches)
 constexpr int BK8 = 128;           // 8-bit channels per k-block (128-byte rows, like BK 16-bit ones)
 constexpr int GN_THREADS = 320;     // with the GroupNorm + SiLU operand transform (4 more warps)
+constexpr int EPI8_THREADS = 320;   // with 8 epilogue warps
 constexpr int MAX_STAGES = 8;
 
 constexpr int STATUS_TIMEOUT = 5;   // mirrors CONV3D_ERR_TIMEOUT
@@ -370,15 +372,17 @@ __device__ __forceinline__ float4* slot_at(const KernelParams& p, int slot) {
 }
 
 // Tail piece, for the calling warp's 32 TMEM lanes (lane row = quarter*32 +
-// lane): store the raw fp32 accumulator (BN columns per lane) in the piece's
-// slot, then take the quarter's ticket.  Returns true in every lane of the
-// warp whose piece completed the quarter; every piece's partial of these
-// lanes is then visible to the warp.  Warp-level only (no other warp is
+// lane) and its 32-column chunks j0, j0 + jstep, ...: store the raw fp32
+// accumulator in the piece's slot, then take the ticket of epilogue warp ew
+// (8 per tail tile).  Returns true in every lane of the warp whose piece
+// completed these lanes and chunks; every piece's partial of them is then
+// visible to the warp.  Warp-level only (no other warp is
 // waited for), so an abort in another warp cannot hold this one.
 __device__ __forceinline__ bool store_piece(const KernelParams& p, int slot, uint32_t t_row,
-                                            bool has_acc, uint32_t quarter, uint32_t lane) {
+                                            bool has_acc, uint32_t quarter, uint32_t lane,
+                                            int j0, int jstep, uint32_t ew) {
   float4* dst = slot_at(p, slot) + quarter * 32u + lane;
-  for (int j = 0; j < p.BN / 32; ++j) {
+  for (int j = j0; j < p.BN / 32; j += jstep) {
     uint32_t r[32];
     tmem_ld_32x32b_x32(t_row + j * 32, r);
     tmem_ld_wait();
@@ -393,7 +397,7 @@ __device__ __forceinline__ bool store_piece(const KernelParams& p, int slot, uin
   __syncwarp();
   int last = 0;
   if (lane == 0)
-    last = take_ticket(p.ticket + (slot / p.split_s) * 4 + quarter, p.gen, p.split_s) ? 1 : 0;
+    last = take_ticket(p.ticket + (slot / p.split_s) * 8 + ew, p.gen, p.split_s) ? 1 : 0;
   last = __shfl_sync(0xFFFFFFFFu, last, 0);
   if (last) __threadfence();
   return last != 0;
@@ -532,7 +536,10 @@ __device__ __forceinline__ uint32_t e5m2x2(float a, float b) {
 //   belongs to the normalised tensor), and the tensor-core issuer waits for
 //   the transform of a stage instead of its load.
 template <bool kBF16, bool kPair, bool kSwap, int kFeat = 0>
-__global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 1)
+__global__ void __launch_bounds__((kFeat & FEAT_GN)     ? GN_THREADS
+                                  : (kFeat & FEAT_EPI8) ? EPI8_THREADS
+                                                        : NUM_THREADS,
+                                  1)
     conv3d_implicit_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                                 const __grid_constant__ CUtensorMap map_b,
                                 const __grid_constant__ CUtensorMap map_y,
@@ -553,7 +560,14 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
   constexpr bool kLo8 = (kFeat & FEAT_LO8) != 0;
   constexpr bool kMixed = (kFeat & FEAT_MIXED) != 0;
   constexpr bool kComb = (kFeat & FEAT_COMBINE) != 0;
+  constexpr bool kEpi8 = (kFeat & FEAT_EPI8) != 0;
   constexpr int kYBufs = 2;   // output staging buffers per epilogue warp
+  // With 8 epilogue warps, warps q and q+4 of the epilogue share TMEM lane
+  // quarter q and take its even and odd 32-column chunks.
+  constexpr int kEpiWarps = kEpi8 ? 2 * EPI_WARPS : EPI_WARPS;
+  constexpr int kJStep = kEpi8 ? 2 : 1;
+  static_assert(!(kEpi8 && (kPair || kGN || kStats || kScatter || kLo8 || kMixed || kComb)),
+                "8 epilogue warps: one CTA, plain output (optionally split)");
   static_assert(!(kLo8 && (kPair || kSwap)), "the e5m2 lo product: one CTA, M = pixels");
   constexpr int kCtas = kPair ? 2 : 1;
   const uint32_t warp = threadIdx.x / 32;
@@ -573,16 +587,16 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
   const uint32_t b_ring = a_ring + p.stages * A_STAGE_BYTES;
   const uint32_t ybytes =
       (p.out_f32 || p.f32_frames > 0) ? 2 * EPI_BUF_BYTES : EPI_BUF_BYTES;   // one y buffer
-  const uint32_t y_stage = b_ring + p.stages * b_stage_bytes;        // [EPI_WARPS][2] buffers
-  const uint32_t r_stage = y_stage + EPI_WARPS * kYBufs * ybytes;     // 2 per warp, with a residual
-  const uint32_t bars = r_stage + (p.has_residual ? EPI_Y_BYTES : 0);
+  const uint32_t y_stage = b_ring + p.stages * b_stage_bytes;        // [kEpiWarps][2] buffers
+  const uint32_t r_stage = y_stage + kEpiWarps * kYBufs * ybytes;     // 2 per warp, with a residual
+  const uint32_t bars = r_stage + (p.has_residual ? kEpiWarps * 2 * EPI_BUF_BYTES : 0);
   const uint32_t full_bar = bars;                         // [stages]
   const uint32_t empty_bar = bars + 8 * p.stages;         // [stages]
   const uint32_t tfull_bar = bars + 16 * p.stages;        // [2]
   const uint32_t tempty_bar = tfull_bar + 16;             // [2]
   const uint32_t drain_bar = tempty_bar + 16;             // [1]
-  const uint32_t rfull_bar = drain_bar + 8;               // [EPI_WARPS][2]
-  const uint32_t ready_bar = rfull_bar + 16 * EPI_WARPS;  // [stages] (GroupNorm variant)
+  const uint32_t rfull_bar = drain_bar + 8;               // [kEpiWarps][2]
+  const uint32_t ready_bar = rfull_bar + 16 * kEpiWarps;  // [stages] (GroupNorm variant)
 
   SharedCtl ctl{&s_abort, p.status, p.timeout_ns,
                 kPair ? mapa_shared(smem_addr(&s_abort), rank ^ 1u) : 0u};
@@ -597,11 +611,11 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar + 8 * a, 1);
-      mbar_init(tempty_bar + 8 * a, 4 * kCtas);
+      mbar_init(tempty_bar + 8 * a, kEpiWarps * kCtas);
     }
     mbar_init(drain_bar, 1);
     mbar_init(peer_bar, 1);
-    for (int e = 0; e < 2 * EPI_WARPS; ++e) mbar_init(rfull_bar + 8 * e, 1);
+    for (int e = 0; e < 2 * kEpiWarps; ++e) mbar_init(rfull_bar + 8 * e, 1);
     if constexpr (kGN)
       for (int s = 0; s < p.stages; ++s) mbar_init(ready_bar + 8 * s, 4);
     fence_mbar_init();
@@ -893,10 +907,12 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
     // rounding -> swizzled shared-memory buffer -> TMA store into y viewed as
     // [frames][Ho*Wo][Cout], which clips rows past the frame and channels past
     // Cout.  The residual chunk is fetched by TMA two chunks ahead (the first
-    // two before the accumulator is ready).
+    // two before the accumulator is ready).  With 8 epilogue warps two warps
+    // share each lane quarter, one taking the even chunks and one the odd.
     using C = Cvt<kBF16>;
     const uint32_t quarter = warp & 3;            // TMEM lanes [32q, 32q+32)
-    const uint32_t ew = warp - 2;                 // epilogue warp index, 0..3
+    const uint32_t ew = warp - 2;                 // epilogue warp index, 0..kEpiWarps-1
+    const int j0 = kEpi8 ? static_cast<int>(ew) / EPI_WARPS : 0;   // this warp's first chunk
     const uint32_t ybuf = y_stage + ew * kYBufs * ybytes;
     const uint32_t rbuf = r_stage + ew * 2 * EPI_BUF_BYTES;
     const uint32_t rbar = rfull_bar + ew * 16;
@@ -950,13 +966,13 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
         // the first two residual chunks, fetched ahead of the accumulator (for a
         // tail piece only once it is known to complete the tile)
         auto prefetch_residual = [&]() {
-          for (int j = 0; j < 2 && j < live_chunks; ++j) {
+          for (int m = 0; m < 2 && j0 + m * kJStep < live_chunks; ++m) {
             if (lane == 0) {
-              mbar_arrive_expect_tx(rbar + 8 * j, EPI_BUF_BYTES);
-              tma_load_3d(rbuf + j * EPI_BUF_BYTES, &map_r, rbar + 8 * j, ch0, tl.p0 + 32 * j,
-                          tl.frame_out);
+              mbar_arrive_expect_tx(rbar + 8 * m, EPI_BUF_BYTES);
+              tma_load_3d(rbuf + m * EPI_BUF_BYTES, &map_r, rbar + 8 * m, ch0,
+                          tl.p0 + 32 * (j0 + m * kJStep), tl.frame_out);
             }
-            rpending[j] = true;
+            rpending[m] = true;
           }
         };
         if (use_res && !piece) prefetch_residual();
@@ -971,15 +987,15 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
           bool from_parts = false;
           if constexpr (kSplit) {
             if (piece) {
-              write_out = store_piece(p, wk.slot, t_row, has_acc, quarter, lane);
+              write_out = store_piece(p, wk.slot, t_row, has_acc, quarter, lane, j0, kJStep, ew);
               from_parts = write_out;
               if (write_out && use_res) prefetch_residual();
             }
           }
           // byte offset of (pixel e, this thread's channel) in a 32 x 32 buffer
           const uint32_t col_byte = (lane & 7u) * 2u;
-          for (int j = 0; write_out && j < live_chunks; ++j) {
-            const uint32_t b = j & 1;
+          for (int j = j0, m = 0; write_out && j < live_chunks; j += kJStep, ++m) {
+            const uint32_t b = m & 1;
             float v[32];
             if (kSplit && from_parts) {
               sum_pieces(p, wk.slot - wk.slot % p.split_s, quarter * 32u + lane, j, v);
@@ -1012,7 +1028,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
             }
             if (lane == 0) bulk_wait_group_read<kYBufs - 1>();
             __syncwarp();
-            const uint32_t yb = ybuf + (j & (kYBufs - 1)) * ybytes;
+            const uint32_t yb = ybuf + (m & (kYBufs - 1)) * ybytes;
             if (f32_tile) {
               // fp32 rows of 32 channels (128 bytes, 128-byte swizzle): this
               // thread's channel is 4-byte word (lane & 3) of 16-byte chunk lane >> 2
@@ -1063,7 +1079,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
             fence_proxy_async_shared();
             __syncwarp();
             const int pix0 = tl.p0 + 32 * j;
-            const bool refill = use_res && j + 2 < live_chunks;
+            const bool refill = use_res && j + 2 * kJStep < live_chunks;
             if (lane == 0) {
               if (!kScatter || f32_tile) {   // strided 16-bit frames were stored above
                 tma_store_3d(ymap, yb, ch0, pix0, yframe);
@@ -1071,8 +1087,8 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
               }
               if (refill) {
                 mbar_arrive_expect_tx(rbar + 8 * b, EPI_BUF_BYTES);
-                tma_load_3d(rbuf + b * EPI_BUF_BYTES, &map_r, rbar + 8 * b, ch0, pix0 + 64,
-                            tl.frame_out);
+                tma_load_3d(rbuf + b * EPI_BUF_BYTES, &map_r, rbar + 8 * b, ch0,
+                            pix0 + 64 * kJStep, tl.frame_out);
               }
             }
             if (refill) rpending[b] = true;
@@ -1116,13 +1132,13 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
       // the first two residual chunks, fetched ahead of the accumulator (for a
       // tail piece only once it is known to complete the tile)
       auto prefetch_residual = [&]() {
-        for (int j = 0; j < 2 && j < live_chunks; ++j) {
+        for (int m = 0; m < 2 && j0 + m * kJStep < live_chunks; ++m) {
           if (lane == 0) {
-            mbar_arrive_expect_tx(rbar + 8 * j, EPI_BUF_BYTES);
-            tma_load_3d(rbuf + j * EPI_BUF_BYTES, &map_r, rbar + 8 * j, tl.co0 + 32 * j,
-                        row_base, tl.frame_out);
+            mbar_arrive_expect_tx(rbar + 8 * m, EPI_BUF_BYTES);
+            tma_load_3d(rbuf + m * EPI_BUF_BYTES, &map_r, rbar + 8 * m,
+                        tl.co0 + 32 * (j0 + m * kJStep), row_base, tl.frame_out);
           }
-          rpending[j] = true;
+          rpending[m] = true;
         }
       };
       if (use_res && !piece) prefetch_residual();
@@ -1137,13 +1153,13 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
         bool from_parts = false;
         if constexpr (kSplit) {
           if (piece) {
-            write_out = store_piece(p, wk.slot, t_row, has_acc, quarter, lane);
+            write_out = store_piece(p, wk.slot, t_row, has_acc, quarter, lane, j0, kJStep, ew);
             from_parts = write_out;
             if (write_out && use_res) prefetch_residual();
           }
         }
-        for (int j = 0; write_out && rows_live && j < live_chunks; ++j) {
-          const uint32_t b = j & 1;
+        for (int j = j0, m = 0; write_out && rows_live && j < live_chunks; j += kJStep, ++m) {
+          const uint32_t b = m & 1;
           float v[32];
           if (kSplit && from_parts) {
             sum_pieces(p, wk.slot - wk.slot % p.split_s, quarter * 32u + lane, j, v);
@@ -1186,7 +1202,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
           // the store issued from this buffer two chunks ago must have read it
           if (lane == 0) bulk_wait_group_read<kYBufs - 1>();
           __syncwarp();
-          const uint32_t yb = ybuf + (j & (kYBufs - 1)) * ybytes;
+          const uint32_t yb = ybuf + (m & (kYBufs - 1)) * ybytes;
           if (f32_tile) {
 #pragma unroll
             for (int c = 0; c < 8; ++c)
@@ -1242,7 +1258,7 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
           fence_proxy_async_shared();
           __syncwarp();
           // every lane has read residual buffer b: refill it with chunk j+2
-          const bool refill = use_res && j + 2 < live_chunks;
+          const bool refill = use_res && j + 2 * kJStep < live_chunks;
           if (lane == 0) {
             if (!kScatter || f32_tile) {   // strided 16-bit frames were stored above
               tma_store_3d(ymap, yb, cb, row_base, yframe);
@@ -1250,8 +1266,8 @@ __global__ void __launch_bounds__((kFeat & FEAT_GN) ? GN_THREADS : NUM_THREADS, 
             }
             if (refill) {
               mbar_arrive_expect_tx(rbar + 8 * b, EPI_BUF_BYTES);
-              tma_load_3d(rbuf + b * EPI_BUF_BYTES, &map_r, rbar + 8 * b, cb + 64, row_base,
-                          tl.frame_out);
+              tma_load_3d(rbuf + b * EPI_BUF_BYTES, &map_r, rbar + 8 * b, cb + 64 * kJStep,
+                          row_base, tl.frame_out);
             }
           }
           if (refill) rpending[b] = true;
