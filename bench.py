@@ -362,6 +362,15 @@ def max_over_ranks(value, device):
     return float(t.item())
 
 
+def sum_over_ranks(count, device):
+    """A count summed over the ranks (SUM all-reduce; every rank takes part)."""
+    if not torch.distributed.is_initialized() or torch.distributed.get_world_size() == 1:
+        return int(count)
+    t = torch.tensor([int(count)], dtype=torch.int64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return int(t.item())
+
+
 def whole_job_tflops(flops_per_rank_step, world, steps, max_ms):
     """Units processed by all ranks divided by the slowest rank's time."""
     return flops_per_rank_step * world * steps / (max_ms * 1e-3) / 1e12
@@ -434,6 +443,7 @@ def measure_forward(args, wl, rank, world, local_rank, c3, keep=False):
     with ClockSampler(local_rank) as clocks:
         region0 = torch.cuda.Event(enable_timing=True)
         region1 = torch.cuda.Event(enable_timing=True)
+        launches0 = c3.kernel_launches()
         region0.record(stream)
         for i in range(args.steps):
             flush.zero_()                       # L2 flushed between timed steps
@@ -441,6 +451,7 @@ def measure_forward(args, wl, rank, world, local_rank, c3, keep=False):
             step()
             ends[i].record(stream)
         region1.record(stream)
+        launches1 = c3.kernel_launches()
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
@@ -464,7 +475,7 @@ def measure_forward(args, wl, rank, world, local_rank, c3, keep=False):
         "roofline": roof,
         "nominal_tflops": whole_job_tflops(nominal_flops(wl), world, args.steps, max_ms),
         "algorithmic_gbs": abytes * world * args.steps / (max_ms * 1e-3) / 1e9,
-        "gpu_launches": forward_launches(wl) * args.steps,
+        "gpu_launches": sum_over_ranks(launches1 - launches0, dev),
         "clocks": clocks.summary(),
         "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms),
                     "p90": sorted(step_ms)[int(0.9 * (len(step_ms) - 1))], "max": max(step_ms),
@@ -697,11 +708,13 @@ def run_backward(args, wl, rank, world, local_rank):
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local_rank) as clocks:
+        launches0 = c3.kernel_launches()
         for i in range(args.steps):
             flush.zero_()
             starts[i].record(stream)
             step()
             ends[i].record(stream)
+        launches = c3.kernel_launches() - launches0
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
@@ -727,20 +740,9 @@ def run_backward(args, wl, rank, world, local_rank):
         roof = {"bound": "hbm", "achieved": abytes / (call_ms * 1e-3) / 1e9,
                 "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                 "peak_source": f"{peak_kind} hbm_gbs"}
-    rep = wl.tpad == 1 and wl.kernel[0] > 1
     if args.pass_ == "dgrad":
-        # weight transform + the GEMM; with replicate padding and D > 1 the front
-        # GEMM, one body GEMM per sample and the front-frame fold; a single
-        # replicate frame folds the weight taps (one more launch) instead
-        if rep and wl.D > 1:
-            launches = 1 + 1 + wl.N + 1
-        elif rep:
-            launches = 3
-        else:
-            launches = 2
         kernel = "conv3d_implicit_gemm_kernel (dgrad: transposed convolution of dy)"
     else:
-        launches = 4          # GEMM, dw rounding, bias column sums, dbias rounding
         kernel = "conv3d_wgrad_kernel"
     line = {
         "metric": f"conv3d backward {args.pass_} TFLOPS (forward-equivalent FLOPs)",
@@ -757,7 +759,7 @@ def run_backward(args, wl, rank, world, local_rank):
                          algorithmic_flops_per_launch=flops, algorithmic_bytes_per_launch=abytes,
                          flop_per_byte=flops / abytes, ridge_flop_per_byte=ridge),
         "nominal_tflops": whole_job_tflops(nominal_flops(wl), world, args.steps, max_ms),
-        "gpu_launches": launches * args.steps,
+        "gpu_launches": sum_over_ranks(launches, dev),
         "clocks": clocks.summary(),
         "step_ms": {"min": min(step_ms), "median": statistics.median(step_ms),
                     "p90": sorted(step_ms)[int(0.9 * (len(step_ms) - 1))], "max": max(step_ms)},
@@ -893,9 +895,11 @@ def run_norm(args, wl, rank, world, local_rank):
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local_rank) as clocks:
+        launches0 = c3.kernel_launches()
         for i in range(args.steps):
             flush.zero_()
             step(evs[i])
+        launches = c3.kernel_launches() - launches0
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
@@ -923,7 +927,7 @@ def run_norm(args, wl, rank, world, local_rank):
                      "peak_source": f"{peak_kind} hbm_gbs", "kernel": "gn_apply_kernel",
                      "algorithmic_bytes_per_launch": 2 * tensor_bytes,
                      "stats_kernel_gbs": stats_gbs, "stats_kernel_frac": stats_gbs / peak},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": sum_over_ranks(launches, dev),
         "clocks": clocks.summary(),
     }
     if rank == 0:
@@ -1019,9 +1023,8 @@ def run_gnblock(args, wl, rank, world, local_rank):
         c3.conv3d_gn(h, None, None, None, p["w"], p["bias"], p["residual"], y, out_groups=G,
                      **kw)
 
-    # launches per step (stats clear and finalize included)
-    forms = {"separate": (separate, 3), "apply_conv_stats": (apply_conv_stats, 4),
-             "fused": (fused, 2), "chained": (chained, 4)}
+    forms = {"separate": separate, "apply_conv_stats": apply_conv_stats, "fused": fused,
+             "chained": chained}
     parts = {"stats": stats_only, "apply": apply_only, "conv": conv_only,
              "conv_with_stats": conv_stats_only}
     flops = algorithmic_flops(wl)
@@ -1033,7 +1036,7 @@ def run_gnblock(args, wl, rank, world, local_rank):
             oracle.BF16 if wl.dtype == "bf16" else oracle.F16, G, eps=1e-6)).to(td))
         hb = dict(host_bits(p), x=hbits)
         rows = _rows_for_parity(wl)
-    for name, (fn, launches) in forms.items():
+    for name, fn in forms.items():
         for _ in range(max(3, args.warmup)):
             flush.zero_()
             fn()
@@ -1043,18 +1046,20 @@ def run_gnblock(args, wl, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
         with ClockSampler(local_rank) as clocks:
+            launches0 = c3.kernel_launches()
             for a, b in ev:
                 flush.zero_()
                 a.record(stream)
                 fn()
                 b.record(stream)
+            launches = c3.kernel_launches() - launches0
             torch.cuda.synchronize(dev)
         ms = [a.elapsed_time(b) for a, b in ev]
         max_ms = max_over_ranks(sum(ms), dev)
         st = c3.poll_status(stream)
         r = {"ms_per_step": max_ms / args.steps,
              "tflops": whole_job_tflops(flops, world, args.steps, max_ms),
-             "gpu_launches": launches * args.steps, "device_status": c3.status_string(st),
+             "gpu_launches": sum_over_ranks(launches, dev), "device_status": c3.status_string(st),
              "clocks": clocks.summary()}
         if r["clocks"]:
             r["clocks"].pop("sm_mhz_series", None)

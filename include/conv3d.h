@@ -386,6 +386,14 @@ CONV3D_API const char* conv3d_status_string(conv3d_status_t status);
 /* Text of the last CONV3D_ERR_CUDA / CONV3D_ERR_UNSUPPORTED detail on this thread. */
 CONV3D_API const char* conv3d_last_error(void);
 
+/* Number of GPU kernels this library has launched in the process, on every
+ * device and stream, counted when each launch is enqueued (the convolution,
+ * weight-gradient and GroupNorm kernels and their small companions: weight
+ * transforms, folds, roundings).  Workspace clears done with cudaMemsetAsync
+ * are not kernels of the library and are not counted.  Needs no GPU (0 until
+ * the first launch); never fails. */
+CONV3D_API unsigned long long conv3d_kernel_launches(void);
+
 /* Frees the cached per-device workspace, the cached tensor maps and the
  * auxiliary stream (which the weight gradient's bias pass runs on).  Not to be
  * called while work that uses them is being enqueued. */

@@ -59,6 +59,7 @@ static int cpu_checks(void) {
   CHECK(conv3d_fwd_cached(x, NULL, w, NULL, NULL, y, 1, 64, 4, 8, 8, 64, k3, s1, p_causal,
                           CONV3D_BF16, NULL) == CONV3D_ERR_INVALID_ARG);
   CHECK(strlen(conv3d_last_error()) > 0);
+  CHECK(conv3d_kernel_launches() == 0);   /* rejected calls launch nothing */
 
   /* backward entry points: workspace sizes and argument errors */
   void* ws = (void*)0x400000000ull;

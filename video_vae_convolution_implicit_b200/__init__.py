@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "TPAD_ZERO", "TPAD_CAUSAL_REPLICATE", "TPAD_CAUSAL_ZERO", "TPAD_CAUSAL_CACHED", "F16", "BF16",
-    "Status", "Conv3dError", "lib_path", "status_string", "last_error",
+    "Status", "Conv3dError", "lib_path", "status_string", "last_error", "kernel_launches",
     "conv3d", "conv3d_fwd", "conv3d_fwd_ptr", "conv3d_fwd_ws_ptr", "conv3d_fwd_noalloc_ptr",
     "conv3d_fwd_cached_ptr", "conv3d_gn", "conv3d_gn_ptr", "output_shape", "workspace_bytes",
     "groupnorm_stats", "groupnorm_silu", "groupnorm_stats_ptr", "groupnorm_silu_ptr",
@@ -110,6 +110,8 @@ _lib.conv3d_status_string.restype = ctypes.c_char_p
 _lib.conv3d_status_string.argtypes = [_c]
 _lib.conv3d_last_error.restype = ctypes.c_char_p
 _lib.conv3d_last_error.argtypes = []
+_lib.conv3d_kernel_launches.restype = ctypes.c_ulonglong
+_lib.conv3d_kernel_launches.argtypes = []
 _lib.conv3d_release.restype = None
 _lib.conv3d_release.argtypes = []
 _lib.conv3d_selftest_wait_timeout.restype = _c
@@ -132,6 +134,11 @@ def status_string(status: int) -> str:
 
 def last_error() -> str:
     return _lib.conv3d_last_error().decode()
+
+
+def kernel_launches() -> int:
+    """GPU kernels the library has launched in this process (counted at enqueue)."""
+    return int(_lib.conv3d_kernel_launches())
 
 
 def _check(status: int) -> None:

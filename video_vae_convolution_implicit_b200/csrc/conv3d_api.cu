@@ -25,9 +25,23 @@
 cudaError_t conv3d_gn_finalize(double* stats, long long pairs, double count, double eps,
                                cudaStream_t stream);
 
+// Kernel launches this library has issued in the process (every device and
+// stream), counted at enqueue; conv3d_kernel_launches() reads it.
+std::atomic<unsigned long long> g_kernel_launches{0};
+
+// The status of `n` launches just enqueued by the GroupNorm kernels'
+// translation unit, which it also counts.
+cudaError_t conv3d_count_launches(int n) {
+  g_kernel_launches.fetch_add(static_cast<unsigned long long>(n), std::memory_order_relaxed);
+  return cudaGetLastError();
+}
+
 namespace {
 
 using namespace conv3d;
+
+// The status of the `n` launches just enqueued, which it also counts.
+cudaError_t launched(int n = 1) { return conv3d_count_launches(n); }
 
 constexpr int kMaxDevices = 64;
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
@@ -939,7 +953,7 @@ conv3d_status_t launch_kernel(DeviceState& S, const LaunchPlan& L, const CUtenso
   kp.test_stall = take_stall(kp.timeout_ns) ? 1 : 0;
   e = cudaLaunchKernelEx(&cfg, kern, map_a, map_b, map_y, map_r, map_p, map_f, kp);
   if (e != cudaSuccess) return cuda_fail(e, "conv3d kernel launch");
-  e = cudaGetLastError();
+  e = launched();
   if (e != cudaSuccess) return cuda_fail(e, "conv3d kernel launch");
   return CONV3D_OK;
 }
@@ -1205,7 +1219,7 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
         x_to_e5m2_kernel<false><<<static_cast<int>(xb), 256, 0, stream>>>(
             static_cast<const uint16_t*>(x), x8, xn);
       }
-      cudaError_t e = cudaGetLastError();
+      cudaError_t e = launched(2);
       if (e != cudaSuccess) return cuda_fail(e, "8-bit fold launch");
       Q.w8 = w8;
       Q.x8 = x8;
@@ -1218,7 +1232,7 @@ conv3d_status_t run(const Problem& P, const void* x, const void* w, const void* 
       else
         fold_temporal_taps_kernel<false><<<blocks, 256, 0, stream>>>(
             static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), P.Cout, P.kt, spatial_cin);
-      cudaError_t e = cudaGetLastError();
+      cudaError_t e = launched();
       if (e != cudaSuccess) return cuda_fail(e, "fold kernel launch");
     }
     wmat = ws;
@@ -1411,7 +1425,7 @@ conv3d_status_t fold_front(const float* ext, void* dx, int N, int D, int kt,
   else
     fold_front_gradient_kernel<false><<<blocks, 256, 0, stream>>>(
         ext, static_cast<uint16_t*>(dx), N, D, kt, frame_elems, FoldPhase{}, 0);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launched();
   if (e != cudaSuccess) return cuda_fail(e, "gradient fold launch");
   return CONV3D_OK;
 }
@@ -1450,7 +1464,7 @@ conv3d_status_t bwd_data_phases(DeviceState& S, const BwdDataPlan& B, const void
         if (blocks > 8 * S.num_sms) blocks = 8 * S.num_sms;
         zero_phase_kernel<<<blocks, 256, 0, stream>>>(static_cast<uint16_t*>(dx),
                                                       static_cast<long long>(N) * D, Ah, Aw, fp);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launched();
         if (e != cudaSuccess) return cuda_fail(e, "zero phase launch");
         continue;
       }
@@ -1461,7 +1475,7 @@ conv3d_status_t bwd_data_phases(DeviceState& S, const BwdDataPlan& B, const void
         const dim3 grid((Cin + 63) / 64, (Cout + 63) / 64, taps);
         flip_transpose_weight_kernel<<<grid, dim3(32, 8), 0, stream>>>(
             static_cast<const uint16_t*>(w), wt, Cout, taps, Cin, kh, kw, Jh, Jw, qh, qw, sh, sw);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launched();
         if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
       }
       Problem T = B.tr;            // temporal rule and sizes of the stride-1 transposed problem
@@ -1530,7 +1544,7 @@ conv3d_status_t bwd_data_phases(DeviceState& S, const BwdDataPlan& B, const void
       else
         fold_front_gradient_kernel<false><<<blocks, 256, 0, stream>>>(
             ext, static_cast<uint16_t*>(dx), N, D, kt, frame_elems, fp, 1);
-      cudaError_t e = cudaGetLastError();
+      cudaError_t e = launched();
       if (e != cudaSuccess) return cuda_fail(e, "gradient fold launch");
     }
   }
@@ -1813,7 +1827,7 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
       flip_fold_weight_kernel<false><<<grid, dim3(32, 8), 0, stream>>>(
           static_cast<const uint16_t*>(w), static_cast<uint16_t*>(ws), Cout, kernel[0], kernel[1],
           kernel[2], Cin);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launched();
     if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
     return run(B.tr, dy, nullptr, nullptr, nullptr, dx, ws, B.ext_bytes, false, stream, &split,
                true);
@@ -1825,7 +1839,7 @@ conv3d_status_t conv3d_bwd_data(const void* dy, const void* w, void* dx, int N, 
     flip_transpose_weight_kernel<<<grid, dim3(32, 8), 0, stream>>>(
         static_cast<const uint16_t*>(w), wt, Cout, taps, Cin, kernel[1], kernel[2], kernel[1],
         kernel[2], 0, 0, 1, 1);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launched();
     if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
   }
   if (!B.rep)
@@ -2145,6 +2159,7 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
               bias_block ? "in the kernel (block of ones)" : dbias ? "in a pass beside it" : "none");
     e = cudaLaunchKernelEx(&cfg, kern, map_x, map_dy, map_p, wp);
     if (e != cudaSuccess) return cuda_fail(e, "wgrad kernel launch");
+    launched();
   }
   {
     int blocks = static_cast<int>((dw_elems / 8 + 255) / 256);   // 8 values a thread
@@ -2163,7 +2178,7 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
       f32_to_16_kernel<false><<<blocks, 256, 0, stream>>>(
           dw32, d16, static_cast<long long>(dw_elems), db32, static_cast<uint16_t*>(dbias),
           dbias && bias_block ? Cout : 0);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dw conversion launch");
+    if ((e = launched()) != cudaSuccess) return cuda_fail(e, "dw conversion launch");
   }
   if (dbias && !bias_block) {
     // 256-channel groups along y; about three blocks per SM in all (as many
@@ -2183,7 +2198,7 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
     else
       bias_grad_kernel<false><<<grid, BIAS_THREADS, 0, bs>>>(static_cast<const uint16_t*>(dy),
                                                                db32, pixels, Cout, per);
-    cudaError_t le = cudaGetLastError();
+    cudaError_t le = launched();
     if (side) {
       // join even after a failed launch, so the caller's stream never runs
       // ahead of work left on the aux stream
@@ -2199,7 +2214,7 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
       f32_to_16_kernel<true><<<1, 256, 0, stream>>>(db32, static_cast<uint16_t*>(dbias), Cout);
     else
       f32_to_16_kernel<false><<<1, 256, 0, stream>>>(db32, static_cast<uint16_t*>(dbias), Cout);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "dbias conversion launch");
+    if ((e = launched()) != cudaSuccess) return cuda_fail(e, "dbias conversion launch");
   }
   return CONV3D_OK;
 }
@@ -2279,7 +2294,7 @@ conv3d_status_t conv3d_bwd_data_cached(const void* dy, const void* w, void* dx, 
     flip_transpose_weight_kernel<<<grid, dim3(32, 8), 0, stream>>>(
         static_cast<const uint16_t*>(w), wt, Cout, taps, Cin, kernel[1], kernel[2], kernel[1],
         kernel[2], 0, 0, 1, 1);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launched();
     if (e != cudaSuccess) return cuda_fail(e, "weight transform launch");
   }
   // The chunk is the zero-padded (pt = 0) convolution of the joined clip
@@ -2383,6 +2398,10 @@ const char* conv3d_status_string(conv3d_status_t s) {
 
 const char* conv3d_last_error(void) { return g_last_error; }
 
+unsigned long long conv3d_kernel_launches(void) {
+  return g_kernel_launches.load(std::memory_order_relaxed);
+}
+
 void conv3d_release(void) {
   {
     std::lock_guard<std::mutex> map_lock(g_map_mu);
@@ -2433,7 +2452,7 @@ conv3d_status_t conv3d_selftest_wait_timeout(int timeout_ms) {
   cudaError_t e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreate");
   selftest_wait_kernel<<<1, 32, 0, s>>>(S->status, static_cast<unsigned long long>(timeout_ms) * 1000000ull);
-  e = cudaGetLastError();
+  e = launched();
   if (e != cudaSuccess) {
     cudaStreamDestroy(s);
     return cuda_fail(e, "self-test launch");

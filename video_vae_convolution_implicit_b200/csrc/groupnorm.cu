@@ -22,6 +22,10 @@
 
 #include "conv3d.h"
 
+// Defined beside the convolution kernels: counts `n` launches just enqueued
+// (conv3d_kernel_launches) and returns their status.
+cudaError_t conv3d_count_launches(int n);
+
 namespace conv3d_gn {
 
 template <bool kBF16>
@@ -182,7 +186,7 @@ cudaError_t conv3d_gn_finalize(double* stats, long long pairs, double count, dou
                                cudaStream_t stream) {
   conv3d_gn::gn_finalize_kernel<<<static_cast<unsigned>((pairs + 255) / 256), 256, 0, stream>>>(
       stats, pairs, count, eps);
-  return cudaGetLastError();
+  return conv3d_count_launches(1);
 }
 
 namespace conv3d_gn {
@@ -322,11 +326,11 @@ conv3d_status_t conv3d_groupnorm_stats(const void* x, int N, int D, int H, int W
     gn_stats_kernel<false><<<static_cast<unsigned>(blocks), threads, smem, stream>>>(
         static_cast<const uint16_t*>(x), stats, C, groups, set_pixels,
         static_cast<int>(chunk_pixels), static_cast<int>(chunks));
-  if (cudaGetLastError() != cudaSuccess) return CONV3D_ERR_CUDA;
+  if (conv3d_count_launches(1) != cudaSuccess) return CONV3D_ERR_CUDA;
   const long long pairs = sets * groups;
   gn_finalize_kernel<<<static_cast<unsigned>((pairs + 255) / 256), 256, 0, stream>>>(
       stats, pairs, static_cast<double>(set_pixels) * (C / groups), static_cast<double>(eps));
-  return cudaGetLastError() == cudaSuccess ? CONV3D_OK : CONV3D_ERR_CUDA;
+  return conv3d_count_launches(1) == cudaSuccess ? CONV3D_OK : CONV3D_ERR_CUDA;
 }
 
 conv3d_status_t conv3d_groupnorm_silu(const void* x, const double* stats, const void* gamma,
@@ -370,7 +374,7 @@ conv3d_status_t conv3d_groupnorm_silu(const void* x, const double* stats, const 
         static_cast<const uint16_t*>(x), stats, static_cast<const uint16_t*>(gamma),
         static_cast<const uint16_t*>(beta), static_cast<uint16_t*>(y), pixels, C, groups,
         set_pixels, apply_silu);
-  return cudaGetLastError() == cudaSuccess ? CONV3D_OK : CONV3D_ERR_CUDA;
+  return conv3d_count_launches(1) == cudaSuccess ? CONV3D_OK : CONV3D_ERR_CUDA;
 }
 
 }  // extern "C"
