@@ -265,8 +265,9 @@ CONV3D_API conv3d_status_t conv3d_fwd_gn(const void* x, const double* stats, con
  * forward call's channel and alignment
  * rules.  workspace: device, 256-byte aligned, conv3d_bwd_data_workspace_bytes()
  * bytes, not overlapping the tensors (it includes about 21 MB in which a launch
- * that is one partly filled wave of tiles -- the front frames, a single frame,
- * a short clip -- splits its tiles along K across the idle SMs).  dx must not
+ * of under 16 rounds of tiles whose last round is at most half full -- a
+ * single frame, a short clip -- splits that round's tiles along K across the
+ * idle SMs).  dx must not
  * overlap dy or w.  Spatial strides: dx is computed phase by phase, each phase
  * (rows h = a*sh + rh, columns a*sw + rw) a stride-1 convolution of dy with the
  * mirrored taps that reach it, stored straight to its strided positions.

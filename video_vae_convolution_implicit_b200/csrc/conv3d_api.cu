@@ -1304,9 +1304,9 @@ struct BwdDataPlan {
   Problem fwd;      // the forward problem being differentiated
   Problem tr;       // the whole transposed convolution (no replicate padding), or
                     // the first-frame problem (replicate padding, D = 1)
-  Problem whole;    // replicate padding, D > 1: the extended frames in fp32 and frames
-                    // 1.. in 16 bits, one launch (mixed output)
-  bool rep;         // whole + fold
+  Problem whole;    // replicate padding, D > 1, few tiles: the extended frames in fp32
+                    // and frames 1.. in 16 bits, one launch (mixed output)
+  bool rep;         // replicate padding, D > 1: tr with frame 0 combined, or whole + fold
   bool phased;      // spatial stride: one transposed convolution per phase
   size_t split_bytes;  // the tail-split region, after the flipped weight and ext
   size_t wt_bytes;  // flipped weight
@@ -1437,8 +1437,9 @@ conv3d_status_t fold_front(const float* ext, void* dx, int N, int D, int kt,
 // stride-1 convolution of dy with the mirrored sub-kernel of those taps and
 // front pads Jh-1-ch, Jw-1-cw, giving Ah x Aw outputs that the kernel's
 // epilogue stores straight to their strided positions of dx.  The temporal
-// direction is the stride-1 data gradient's (front frames in fp32 and a fold
-// for causal replicate padding, the first-frame fold for a single frame).
+// direction is the stride-1 data gradient's (frame 0 combined with its
+// replicated copies, or for few tiles the front frames in fp32 and a fold,
+// for causal replicate padding; the first-frame fold for a single frame).
 // Phases that no tap reaches (a stride larger than the kernel) are zero.
 conv3d_status_t bwd_data_phases(DeviceState& S, const BwdDataPlan& B, const void* dy,
                                 const void* w, void* dx, void* workspace, cudaStream_t stream,
