@@ -148,8 +148,7 @@ struct KernelParams {
 };
 
 // Epilogue staging: each epilogue warp owns two 32-row x 32-channel buffers
-// (64-byte rows, 64-byte swizzle) for y and, with a residual, two more
-// (sizes below for four epilogue warps; the eight-warp instances take twice).
+// (64-byte rows, 64-byte swizzle) for y and, with a residual, two more.
 constexpr int EPI_WARPS = 4;
 constexpr int EPI_BUF_BYTES = 32 * 32 * 2;
 constexpr int EPI_Y_BYTES = EPI_WARPS * 2 * EPI_BUF_BYTES;
