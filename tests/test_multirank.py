@@ -1,8 +1,9 @@
 """Host-side multi-rank logic of bench.py on CPU with gloo, world size 2.
 
 The convolution shards as independent replicas (each rank its own batch
-sample), so the only cross-rank steps are the timing barrier and the MAX
-reduction of per-rank times; these run here without a GPU.
+sample), so the only cross-rank steps are the timing barrier, the MAX
+reduction of per-rank times and the SUM of the ranks' kernel-launch counts;
+these run here without a GPU.
 """
 import os
 import socket
@@ -28,10 +29,11 @@ def _worker(rank, world, port, out):
         wl = WORKLOADS["cfg2"]
         my_ms = 10.0 + 5.0 * rank                      # rank 1 is the slow one
         mx = bench.max_over_ranks(my_ms, torch.device("cpu"))
+        launches = bench.sum_over_ranks(20 + rank, torch.device("cpu"))   # per-rank kernel counts
         seeds = [None] * world
         dist.all_gather_object(seeds, bench.rank_seed(wl, rank))
         dist.barrier()
-        out.put((rank, mx, seeds))
+        out.put((rank, mx, launches, seeds))
     finally:
         dist.destroy_process_group()
 
@@ -47,8 +49,9 @@ def test_two_rank_timing_and_sharding():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, mx, seeds in res:
+    for rank, mx, launches, seeds in res:
         assert mx == 15.0                              # max over ranks, on every rank
+        assert launches == 41                          # the job's launches: summed over ranks
         assert len(set(seeds)) == 2                    # distinct samples per rank
 
 
