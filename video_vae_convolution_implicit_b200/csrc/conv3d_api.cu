@@ -661,6 +661,28 @@ bool pdl_enabled() {
   return on;
 }
 
+// Launches `kern` (256 threads a block, no shared memory) as a programmatic
+// dependent of the kernel before it on the stream, when that is enabled: its
+// blocks may be scheduled before that kernel ends and wait for it in
+// griddepcontrol.wait.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), int blocks, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  if (pdl_enabled()) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 uint32_t pow2_at_least(uint32_t v) {
   uint32_t p = 32;
   while (p < v) p <<= 1;
@@ -2116,8 +2138,20 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
       return CONV3D_ERR_CUDA;
     }
   }
-  cudaError_t e = cudaMemsetAsync(workspace, 0, need, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "workspace clear");
+  // Clear the fp32 sums with a kernel that lets the weight-gradient kernel
+  // start at once: only that kernel's epilogue waits for the clear, so the
+  // clear overlaps its first MMAs, and the rounding kernel after it is
+  // launched the same way.
+  cudaError_t e = cudaSuccess;
+  {
+    const long long n4 = static_cast<long long>(need / 16);   // a multiple of 256 bytes
+    // one block per SM at most, so that a weight-gradient CTA fits beside it
+    long long blocks = (n4 + 255) / 256;
+    if (blocks > S->num_sms) blocks = S->num_sms;
+    zero_f32x4_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<float4*>(workspace), n4);
+    if ((e = launched()) != cudaSuccess) return cuda_fail(e, "workspace clear launch");
+  }
   // The bias gradient reads dy once more.  Its kernel uses no shared memory,
   // so its blocks fit beside the weight-gradient CTAs, and it runs on the aux
   // stream at the same time (forked after the clear, joined before the
@@ -2137,17 +2171,26 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
   {
     const int grid_units = wp.num_units < lanes ? wp.num_units : lanes;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kCtas;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    unsigned n_attr = 0;
+    if (pair) {
+      attr[n_attr].id = cudaLaunchAttributeClusterDimension;
+      attr[n_attr].val.clusterDim.x = kCtas;
+      attr[n_attr].val.clusterDim.y = 1;
+      attr[n_attr].val.clusterDim.z = 1;
+      ++n_attr;
+    }
+    if (pdl_enabled()) {   // a programmatic dependent of the clear (CONV3D_PDL=0: off)
+      attr[n_attr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[n_attr].val.programmaticStreamSerializationAllowed = 1;
+      ++n_attr;
+    }
     cfg.gridDim = dim3(static_cast<unsigned>(kCtas * grid_units), 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cfg.attrs = attr;
-    cfg.numAttrs = pair ? 1 : 0;
+    cfg.numAttrs = n_attr;
     if (plan_log())
       fprintf(stderr,
               "libconv3d: weight gradient %s %s, %d units (%d splits of %lld chunks of %d pixels), "
@@ -2167,18 +2210,23 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
     if (blocks > 8 * S->num_sms) blocks = 8 * S->num_sms;
     uint16_t* d16 = static_cast<uint16_t*>(dw);
     const long long run_per_co = taps_run * Cin;
+    const float* cdw = dw32;
+    const float* cdb = db32;
+    uint16_t* d16b = static_cast<uint16_t*>(dbias);
+    const long long n_dw = static_cast<long long>(dw_elems);
+    const long long n_db = dbias && bias_block ? Cout : 0;
+    // a programmatic dependent of the weight-gradient kernel (it waits for it)
     if (frame0 && bf16)
-      f32_to_16_bcast_kernel<true><<<blocks, 256, 0, stream>>>(dw32, d16, Cout, F.kt, run_per_co);
+      e = launch_dependent(f32_to_16_bcast_kernel<true>, blocks, stream, cdw, d16, Cout, F.kt,
+                           run_per_co);
     else if (frame0)
-      f32_to_16_bcast_kernel<false><<<blocks, 256, 0, stream>>>(dw32, d16, Cout, F.kt, run_per_co);
+      e = launch_dependent(f32_to_16_bcast_kernel<false>, blocks, stream, cdw, d16, Cout, F.kt,
+                           run_per_co);
     else if (bf16)   // with the bias block, db is final here too: one launch for both
-      f32_to_16_kernel<true><<<blocks, 256, 0, stream>>>(
-          dw32, d16, static_cast<long long>(dw_elems), db32, static_cast<uint16_t*>(dbias),
-          dbias && bias_block ? Cout : 0);
+      e = launch_dependent(f32_to_16_kernel<true>, blocks, stream, cdw, d16, n_dw, cdb, d16b, n_db);
     else
-      f32_to_16_kernel<false><<<blocks, 256, 0, stream>>>(
-          dw32, d16, static_cast<long long>(dw_elems), db32, static_cast<uint16_t*>(dbias),
-          dbias && bias_block ? Cout : 0);
+      e = launch_dependent(f32_to_16_kernel<false>, blocks, stream, cdw, d16, n_dw, cdb, d16b, n_db);
+    if (e != cudaSuccess) return cuda_fail(e, "dw conversion launch");
     if ((e = launched()) != cudaSuccess) return cuda_fail(e, "dw conversion launch");
   }
   if (dbias && !bias_block) {

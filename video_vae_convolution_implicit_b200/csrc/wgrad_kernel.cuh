@@ -512,6 +512,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // warp-wide instruction covering 32 consecutive ci of one co (128 bytes).
     // Swapped: thread = one output channel, 32 consecutive ci of one entry per
     // TMEM load, added with eight 16-byte reductions.
+    // Launched as a programmatic dependent of the kernel that clears the fp32
+    // accumulators: only these warps touch them, so only they wait for it
+    // (long before their first unit's MMAs are done); the producer streams x
+    // and dy, which the work before the clear wrote, from the start.
+    griddep_wait();
     const uint32_t quarter = warp & 3;
     int local = 0;
     const long long K = static_cast<long long>(p.taps) * p.Cin;
@@ -619,6 +624,16 @@ __device__ __forceinline__ uint4 round8(const float* __restrict__ src) {
   return make_uint4(C::pack(a.x, a.y), C::pack(a.z, a.w), C::pack(b.x, b.y), C::pack(b.z, b.w));
 }
 
+// Clears n4 16-byte words at p.  The weight-gradient kernel that follows it
+// on the stream may start at once (programmatic launch): only its epilogue
+// waits for this grid.
+__global__ void zero_f32x4_kernel(float4* __restrict__ p, long long n4) {
+  griddep_launch_dependents();
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    p[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+}
+
 // fp32 accumulation -> the 16-bit weight gradient (one rounding); the n2
 // values of a second array (the bias gradient) in the same launch.  8 values
 // per thread: n and n2 are multiples of 8 and every pointer 16-byte aligned.
@@ -626,6 +641,7 @@ template <bool kBF16>
 __global__ void f32_to_16_kernel(const float* __restrict__ src, uint16_t* __restrict__ dst,
                                  long long n, const float* __restrict__ src2 = nullptr,
                                  uint16_t* __restrict__ dst2 = nullptr, long long n2 = 0) {
+  griddep_wait();   // (a programmatic dependent of the weight-gradient kernel)
   const long long v1 = n / 8, v = v1 + n2 / 8;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < v;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -642,6 +658,7 @@ __global__ void f32_to_16_kernel(const float* __restrict__ src, uint16_t* __rest
 template <bool kBF16>
 __global__ void f32_to_16_bcast_kernel(const float* __restrict__ src, uint16_t* __restrict__ dst,
                                        int Cout, int kt, long long per_co) {
+  griddep_wait();   // (a programmatic dependent of the weight-gradient kernel)
   const long long v = static_cast<long long>(Cout) * kt * per_co / 8;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < v;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
