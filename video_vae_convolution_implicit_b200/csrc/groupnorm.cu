@@ -65,20 +65,42 @@ __device__ __forceinline__ void unpack8(const uint4 q, uint32_t (&e)[8]) {
   e[4] = q.z & 0xFFFFu; e[5] = q.z >> 16; e[6] = q.w & 0xFFFFu; e[7] = q.w >> 16;
 }
 
+// Asynchronous 16-byte copy global -> shared (no registers held while it is
+// in flight) and its group bookkeeping.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
+}
+
+// Pixel rows each thread of the statistics pass keeps in flight.
+constexpr int GN_DEPTH = 8;
+
 // Block (v, r): thread (v + vecs * r) owns the 8 channels [8v, 8v+8) of the
-// pixels r, r + rows, r + 2 rows, ... of its chunk.  Per channel it sums
-// (x - K) and (x - K)^2 in fp32 with K = x at the set's first pixel (shifting
-// by a sample of the data keeps the fp32 partial sums small).  The block folds
-// the rows together, expands to {sum x, sum x^2} in fp64 per channel, adds the
-// channels of each group in shared memory and issues one pair of fp64 atomics
-// per group.
+// pixels r, r + rows, r + 2 rows, ... of its chunk.  Its 16-byte vectors
+// stream through its own GN_DEPTH slots of a shared-memory ring by cp.async,
+// GN_DEPTH rows ahead of the one it adds (a thread reads only the slots it
+// filled, so no barrier is needed; measured on B200: with four loads held in
+// registers instead, the single-set 75 MB tensor streamed at 2.0 TB/s).  Per
+// channel it sums (x - K) and (x - K)^2 in fp32 with K = x at the set's first
+// pixel (shifting by a sample of the data keeps the fp32 partial sums small).
+// The block folds the rows together, expands to {sum x, sum x^2} in fp64 per
+// channel, adds the channels of each group in shared memory and issues one
+// pair of fp64 atomics per group.
 template <bool kBF16>
 __global__ void __launch_bounds__(256, 4)
     gn_stats_kernel(const uint16_t* __restrict__ x,
                                                        double* __restrict__ stats, int C,
                                                        int groups, long long set_pixels,
                                                        int chunk_pixels, int chunks_per_set) {
-  extern __shared__ float red[];                 // [rows][C][2] floats, then [C][2] doubles
+  // the ring [GN_DEPTH][threads] of 16-byte slots while streaming; afterwards
+  // [rows][C][2] floats, then [C][2] doubles
+  extern __shared__ __align__(16) float red[];
   const int vecs = C / 8;
   const int rows = blockDim.x / vecs;
   const int v = threadIdx.x % vecs;
@@ -102,29 +124,41 @@ __global__ void __launch_bounds__(256, 4)
       s2[j] = 0.0f;
     }
   }
-  // four rows' loads in flight per thread; with four 8-warp blocks per SM that
-  // keeps ~64 KB of reads outstanding on every SM
-  constexpr int U = 4;
-  for (long long p = p_begin + r; p < p_end; p += U * rows) {
-    uint4 q[U];
+  // GN_DEPTH rows in flight per thread: with four 8-warp blocks per SM that
+  // keeps 128 KB of reads outstanding on every SM
+  const long long first = p_begin + r;
+  const long long nrow = first < p_end ? (p_end - first + rows - 1) / rows : 0;   // rows of this thread
+  const uint32_t ring = static_cast<uint32_t>(__cvta_generic_to_shared(red)) + threadIdx.x * 16u;
+  const uint32_t ring_step = blockDim.x * 16u;
+  const uint16_t* src = xs + first * C + 8 * v;
+  const long long src_step = static_cast<long long>(rows) * C;
 #pragma unroll
-    for (int u = 0; u < U; ++u)
-      if (p + u * rows < p_end)
-        q[u] = __ldg(reinterpret_cast<const uint4*>(xs + (p + u * rows) * C + 8 * v));
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (p + u * rows < p_end) {
-        uint32_t e[8];
-        unpack8(q[u], e);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float d = to_f<kBF16>(e[j]) - K[j];
-          s1[j] += d;
-          s2[j] = fmaf(d, d, s2[j]);
-        }
-      }
-    }
+  for (int k = 0; k < GN_DEPTH; ++k) {
+    if (k < nrow) cp_async16(ring + k * ring_step, src + k * src_step);
+    cp_async_commit();   // one group per row, empty ones included, so the count stays fixed
   }
+  for (long long k = 0; k < nrow; ++k) {
+    cp_async_wait<GN_DEPTH - 1>();   // row k has landed
+    const uint32_t slot = ring + static_cast<uint32_t>(k % GN_DEPTH) * ring_step;
+    uint4 q;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w)
+                 : "r"(slot)
+                 : "memory");
+    uint32_t e[8];
+    unpack8(q, e);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float d = to_f<kBF16>(e[j]) - K[j];
+      s1[j] += d;
+      s2[j] = fmaf(d, d, s2[j]);
+    }
+    // the slot was read into registers above: refill it with row k + GN_DEPTH
+    if (k + GN_DEPTH < nrow) cp_async16(slot, src + (k + GN_DEPTH) * src_step);
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+  __syncthreads();   // every thread's ring slots are drained before red reuses them
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     red[(r * C + 8 * v + j) * 2 + 0] = s1[j];
@@ -314,7 +348,10 @@ conv3d_status_t conv3d_groupnorm_stats(const void* x, int N, int D, int H, int W
 
   const long long blocks = sets * chunks;
   if (blocks > 0x7FFFFFFFLL) return CONV3D_ERR_UNSUPPORTED;
-  const size_t smem = static_cast<size_t>(rows) * C * 2 * sizeof(float) + 2 * C * sizeof(double);
+  const size_t red_bytes =
+      static_cast<size_t>(rows) * C * 2 * sizeof(float) + 2 * C * sizeof(double);
+  const size_t ring_bytes = static_cast<size_t>(GN_DEPTH) * threads * 16;
+  const size_t smem = red_bytes > ring_bytes ? red_bytes : ring_bytes;
   if (smem > 48 * 1024) return CONV3D_ERR_UNSUPPORTED;
   cudaError_t e = cudaMemsetAsync(stats, 0, sets * groups * 2 * sizeof(double), stream);
   if (e != cudaSuccess) return CONV3D_ERR_CUDA;
