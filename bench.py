@@ -157,7 +157,10 @@ class ClockSampler:
         0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index):
+    def __init__(self, device_index, label=None):
+        # the timed region is also an NVTX range (`label`), so that profilers
+        # can select it (ncu --nvtx --nvtx-include "<label>/")
+        self.label = label
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
         self._ok = False
@@ -194,6 +197,8 @@ class ClockSampler:
             pass
 
     def __enter__(self):
+        if self.label and torch.cuda.is_available():
+            torch.cuda.nvtx.range_push(self.label)
         if self._ok:
             self._sample()
             self._t.start()
@@ -204,6 +209,8 @@ class ClockSampler:
             self._stop.set()
             self._t.join()
             self._sample()
+        if self.label and torch.cuda.is_available():
+            torch.cuda.nvtx.range_pop()
 
     def summary(self):
         if not self._ok or not self.samples:
@@ -440,7 +447,7 @@ def measure_forward(args, wl, rank, world, local_rank, c3, keep=False):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(local_rank) as clocks:
+    with ClockSampler(local_rank, f"timed {wl.name} fwd") as clocks:
         region0 = torch.cuda.Event(enable_timing=True)
         region1 = torch.cuda.Event(enable_timing=True)
         launches0 = c3.kernel_launches()
@@ -707,7 +714,7 @@ def run_backward(args, wl, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(local_rank) as clocks:
+    with ClockSampler(local_rank, f"timed {wl.name} {args.pass_}") as clocks:
         launches0 = c3.kernel_launches()
         for i in range(args.steps):
             flush.zero_()
@@ -894,7 +901,7 @@ def run_norm(args, wl, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(local_rank) as clocks:
+    with ClockSampler(local_rank, f"timed {wl.name} groupnorm") as clocks:
         launches0 = c3.kernel_launches()
         for i in range(args.steps):
             flush.zero_()
@@ -1045,7 +1052,7 @@ def run_gnblock(args, wl, rank, world, local_rank):
               for _ in range(args.steps)]
         if world > 1:
             torch.distributed.barrier()
-        with ClockSampler(local_rank) as clocks:
+        with ClockSampler(local_rank, f"timed {wl.name} block {name}") as clocks:
             launches0 = c3.kernel_launches()
             for a, b in ev:
                 flush.zero_()
