@@ -101,3 +101,81 @@ def test_plan_log_data_gradient_with_fp32_front_frames():
     assert any("implicit GEMM" in l and "fp32 (front frames) and 16-bit output" in l
                for l in lines), lines
     assert any(l.startswith("libconv3d: data gradient: 3 front frames") for l in lines), lines
+
+
+ROUNDS_SCRIPT = """
+import sys
+import torch
+import seeded_inputs as si
+import video_vae_convolution_implicit_b200 as c3
+sms = torch.cuda.get_device_properties(0).multi_processor_count
+rounds, extra = int(sys.argv[1]), int(sys.argv[2])
+# 2 frames of H x 128 pixels in 128-pixel tiles, 64 channels (one channel tile):
+# rounds * sms + extra tiles in all
+tiles = rounds * sms + extra
+H = tiles // 2
+x = si.tensor((1, 2, H, 128, 64), 9, 0, 1.0, torch.bfloat16, "cuda")
+w = si.tensor((64, 3, 3, 3, 64), 9, 1, (27 * 64) ** -0.5, torch.bfloat16, "cuda")
+y = c3.conv3d(x, w)
+assert c3.poll_status() == c3.Status.OK
+print(tiles)
+"""
+
+
+@pytest.mark.parametrize("rounds,split", [(15, True), (16, False)])
+def test_tail_split_only_below_sixteen_rounds(rounds, split):
+    """A short last round (10 tiles) is split along K when the launch has fewer
+    than 16 rounds of tiles, and left whole from 16 rounds up."""
+    env = dict(os.environ)
+    env["CONV3D_LOG"] = "1"
+    env["CONV3D_SWAP"] = "0"
+    env.pop("CONV3D_SPLIT", None)
+    r = subprocess.run([sys.executable, "-c", ROUNDS_SCRIPT, str(rounds), "10"], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    tiles = int(r.stdout.split()[-1])
+    lines = [l for l in r.stderr.splitlines() if "implicit GEMM" in l]
+    assert len(lines) == 1 and f"{tiles} tiles" in lines[0], lines
+    if split:
+        assert "last 10 tiles in 3 pieces" in lines[0], lines   # 27 k-blocks: pieces of >= 8
+    else:
+        assert "in 1 pieces" in lines[0], lines
+
+
+COMBINE_SCRIPT = """
+import sys
+import torch
+import seeded_inputs as si
+import video_vae_convolution_implicit_b200 as c3
+H = int(sys.argv[1])
+shape = (1, 4, H, 128, 64)
+w = si.tensor((64, 3, 3, 3, 64), 9, 1, (27 * 64) ** -0.5, torch.bfloat16, "cuda")
+dy = si.tensor(shape, 9, 2, 1.0, torch.bfloat16, "cuda")
+dx = c3.conv3d_bwd_data(dy, w, shape, (0, 1, 1), c3.TPAD_CAUSAL_REPLICATE)
+assert c3.poll_status() == c3.Status.OK
+print(torch.cuda.get_device_properties(0).multi_processor_count)
+"""
+
+
+@pytest.mark.parametrize("many", [True, False])
+def test_data_gradient_front_rule(many):
+    """By default the data gradient combines frame 0 with its replicated
+    copies from 4 rounds of tiles up, and takes the fp32 front frames and the
+    fold below that."""
+    env = dict(os.environ)
+    env["CONV3D_LOG"] = "1"
+    env.pop("CONV3D_DGRAD_COMBINE", None)
+    env.pop("CONV3D_SWAP", None)
+    # 4 frames of H x 128 pixels, 64 channels: the transposed variant's
+    # 256-pixel tiles give 4 * H / 2 tiles (H = 296: 592 = 4 rounds of 148)
+    H = 296 if many else 8
+    r = subprocess.run([sys.executable, "-c", COMBINE_SCRIPT, str(H)], cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    sms = int(r.stdout.split()[-1])
+    lines = [l for l in r.stderr.splitlines() if l.startswith("libconv3d: data gradient")]
+    assert len(lines) == 1, r.stderr[-2000:]
+    if many and sms <= 148:
+        assert "frame 0 with its 2 replicated copies" in lines[0], lines
+    elif not many:
+        assert "front frames and" in lines[0], lines
