@@ -2087,7 +2087,11 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
                     : static_cast<long long>(kt_run) * wp.eblocks) * wp.co_tiles
       : pair ? static_cast<long long>(kt_run) * wp.pairs_per_it * wp.co_tiles
              : (static_cast<long long>(wp.taps) * wp.cblocks + (bias_block ? 1 : 0)) * wp.co_tiles;
-  const long long splits = choose_wgrad_splits(base_units, wp.total_chunks, lanes, pix);
+  long long splits = choose_wgrad_splits(base_units, wp.total_chunks, lanes, pix);
+  if (const char* env = getenv("CONV3D_WGRAD_SPLITS")) {   // tuning: pixel ranges per unit block
+    const long long v = atoll(env);
+    if (v >= 1 && v <= wp.total_chunks) splits = v;
+  }
   if (base_units * splits > 0x7FFFFFFFLL) {
     set_error("problem too large");
     return CONV3D_ERR_UNSUPPORTED;
