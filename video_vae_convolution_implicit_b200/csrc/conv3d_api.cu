@@ -768,14 +768,17 @@ conv3d_status_t plan_launch(const DeviceState& S, const Problem& P, bool bf16, s
   // still gives every SM pair a tile.  A single-tap (1x1x1) layer is bound by
   // streaming x from HBM: transposed, x fills the larger operand slot (32 KB
   // of each stage instead of 16 KB), so more of it is in flight per SM; with
-  // at least 8 k-blocks per tile it runs transposed whenever that needs no
-  // more steps (measured on B200: 512->256 33x128x128, 5.06 -> 5.27 TB/s; with
-  // 4 k-blocks, 256->512, the transposing epilogue dominates and it lost 9%).
-  // CONV3D_SWAP=0/1 forces the choice.
+  // more than 8 k-blocks per tile (four epilogue warps) it runs transposed
+  // whenever that needs no more steps (measured on B200 with four epilogue
+  // warps: 512->256 33x128x128, 5.06 -> 5.27 TB/s; with 4 k-blocks, 256->512,
+  // the transposing epilogue dominates and it lost 9%).  With at most 8
+  // k-blocks the tile gets eight epilogue warps, and then the untransposed
+  // variant measured as fast or faster (512->256: 159.6-159.7 against
+  // 160.8-161.7 us).  CONV3D_SWAP=0/1 forces the choice.
   const long long frames_out = static_cast<long long>(P.N) * P.Do;
   const long long normal_steps = frames_out * ((kp.HoWo + BM - 1) / BM) * kp.n_tiles_n;
   const long long swap_tiles = frames_out * ((kp.HoWo + 255) / 256) * ((P.Cout + 127) / 128);
-  const bool single_tap = kt_eff * P.kh * P.kw == 1 && kp.n_chunks >= 8;
+  const bool single_tap = kt_eff * P.kh * P.kw == 1 && kp.n_chunks > 8;
   L.swap = (swap_tiles < normal_steps || (single_tap && swap_tiles <= normal_steps)) &&
            swap_tiles >= S.num_sms / 2;
   if (const char* env = getenv("CONV3D_SWAP")) {
