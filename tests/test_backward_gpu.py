@@ -267,6 +267,27 @@ def test_bwd_data_causal_one_launch_on_a_side_stream(D, combine, monkeypatch):
     assert torch.equal(a_copy.view(torch.int16), a.view(torch.int16))
 
 
+@pytest.mark.parametrize("combine", ["1", "0"])
+@pytest.mark.parametrize("case", [
+    # N, Cin, D, H, W, Cout, kernel, pad, dtype
+    (2, 64, 3, 9, 11, 48, (3, 3, 3), (0, 1, 1), "f16"),
+    (1, 32, 5, 12, 7, 64, (2, 3, 3), (0, 1, 1), "f16"),      # kt = 2: one replicated copy
+    (1, 48, 4, 10, 10, 40, (3, 1, 1), (0, 0, 0), "bf16"),    # temporal taps only
+], ids=lambda c: "x".join(map(str, c[:6])) + f"-k{''.join(map(str, c[6]))}-{c[8]}")
+def test_bwd_data_causal_front_variants(case, combine, monkeypatch):
+    """Both forms of frame 0's gradient under causal replicate padding on fp16,
+    kt = 2 and a temporal-only kernel: every element against the oracle."""
+    monkeypatch.setenv("CONV3D_DGRAD_COMBINE", combine)
+    N, Cin, D, H, W, Cout, k, pad, dt = case
+    x, w, dy, od = grads_problem(N, Cin, D, H, W, Cout, k, pad, CREP, 41 + Cin, dt)
+    dx = torch.full(x.shape, float("nan"), dtype=x.dtype, device="cuda")
+    dx = c3.conv3d_bwd_data(dy, w, x.shape, pad, CREP, dx=dx)
+    assert c3.poll_status() == c3.Status.OK
+    ref, _, _ = oracle.conv3d_backward(si.bits(x), si.bits(w), si.bits(dy), od, k, (1, 1, 1), pad,
+                                       CREP)
+    assert_close(dx.double().cpu().numpy(), ref, f"dx {case} combine={combine}")
+
+
 @pytest.mark.parametrize("tpad", [CREP, CZERO])
 def test_autograd_function_matches_the_oracle(tpad):
     """Conv3dFunction: one backward through the library gives the oracle's adjoints
