@@ -294,7 +294,10 @@ CONV3D_API size_t conv3d_bwd_data_workspace_bytes(int N, int Cin, int D, int H, 
  * dy[.., co] * Xpad[.., tap-shifted, ci] (the same implicit im2col matrix the
  * forward pass reads, with the same padding rules), dbias[co] = sum of dy.
  * Accumulated in fp32 in the workspace (split over pixel ranges, fp32
- * atomics: the summation order varies from run to run), rounded once.  dbias:
+ * atomics: the summation order varies from run to run), rounded once: a clear
+ * kernel, the weight-gradient kernel and a rounding kernel on `stream`, the
+ * last two launched as programmatic dependents of the one before (each waits
+ * for it on the device before touching its results).  dbias:
  * for a single tap (1x1x1) a block of the kernel itself sums dy; otherwise a
  * pass over dy runs beside the kernel on the library's auxiliary stream,
  * forked from and joined back into `stream` with events (the call still
