@@ -2149,8 +2149,13 @@ conv3d_status_t bwd_weight_impl(const void* x, const void* prev, const void* dy,
   // start at once: only that kernel's epilogue waits for the clear, so the
   // clear overlaps its first MMAs, and the rounding kernel after it is
   // launched the same way.
+  // (Without programmatic launches, CONV3D_PDL=0, the clear has nothing to
+  // overlap and is a plain memset.)
   cudaError_t e = cudaSuccess;
-  {
+  if (!pdl_enabled()) {
+    if ((e = cudaMemsetAsync(workspace, 0, need, stream)) != cudaSuccess)
+      return cuda_fail(e, "workspace clear");
+  } else {
     const long long n4 = static_cast<long long>(need / 16);   // a multiple of 256 bytes
     // one block per SM at most, so that a weight-gradient CTA fits beside it
     long long blocks = (n4 + 255) / 256;
